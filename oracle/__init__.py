@@ -1,0 +1,241 @@
+"""CPU oracle for the quantized KV-cache hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package.  The CUDA library never routes through
+it; it shares no code with ``quantized_kv_cache_20_b200``.
+
+The arithmetic lives in ``kvq_oracle.c`` (plain C, IEEE binary32 for the
+quantizers exactly as the formulas are written, fp64 for attention).  This
+module builds it on demand with gcc and wraps it with ctypes over numpy arrays.
+bf16 tensors travel as their raw ``uint16`` bit patterns.
+
+Sources (page title, section) are cited in ``kvq_oracle.c``; each wrapper below
+names the one it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkvq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MODE_INT8_AFFINE = 0
+MODE_FP8_E4M3 = 1
+MODE_MXFP8 = 2
+MODE_MXFP4 = 3
+
+_CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kvq_oracle.c`` into ``libkvq_oracle.so`` if stale; return its path."""
+    stale = force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+        lib.kvqo_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.kvqo_e4m3_value.restype = ctypes.c_double
+        lib.kvqo_e4m3_encode.argtypes = [f32]
+        lib.kvqo_e4m3_encode.restype = ctypes.c_uint8
+        lib.kvqo_e2m1_value.argtypes = [ctypes.c_uint8]
+        lib.kvqo_e2m1_value.restype = ctypes.c_double
+        lib.kvqo_e2m1_encode.argtypes = [f32]
+        lib.kvqo_e2m1_encode.restype = ctypes.c_uint8
+        lib.kvqo_e8m0_value.argtypes = [ctypes.c_uint8]
+        lib.kvqo_e8m0_value.restype = ctypes.c_double
+        lib.kvqo_e8m0_ceil.argtypes = [f32]
+        lib.kvqo_e8m0_ceil.restype = ctypes.c_uint8
+        lib.kvqo_affine_int8_row.argtypes = [P, i32, P, P, P]
+        lib.kvqo_affine_int8_row.restype = None
+        lib.kvqo_block_row.argtypes = [i32, P, i32, P, P, P]
+        lib.kvqo_block_row.restype = None
+        lib.kvqo_write.argtypes = [i32, P, i32, i32, i32, i32, P, P, i64, P, P, P, P]
+        lib.kvqo_write.restype = None
+        lib.kvqo_sink_plan.argtypes = [i32, i32, i32, i32, i64, P, P, P]
+        lib.kvqo_sink_plan.restype = None
+        lib.kvqo_sink_mask.argtypes = [i32, i32, P, i64, P]
+        lib.kvqo_sink_mask.restype = None
+        sdpa_args = [P, i32, i32, i32, i32, P, P, P, P, P, P, i32, i64, i32, P, i32, f32]
+        lib.kvqo_sdpa_row.argtypes = sdpa_args + [i32, i32, i32, P]
+        lib.kvqo_sdpa_row.restype = None
+        lib.kvqo_sdpa.argtypes = sdpa_args + [P]
+        lib.kvqo_sdpa.restype = None
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _u16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    assert x.dtype in (np.uint16, np.int16), "bf16 data travels as uint16 bit patterns"
+    return x.view(np.uint16)
+
+
+# --- number formats (OCP FP8 E4M3 "fn", OCP MX E2M1 / E8M0) ----------------
+
+def e4m3_value(code: int) -> float:
+    return _load().kvqo_e4m3_value(int(code))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(_load().kvqo_e4m3_encode(float(v)))
+
+
+def e2m1_value(code: int) -> float:
+    return _load().kvqo_e2m1_value(int(code))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(_load().kvqo_e2m1_encode(float(v)))
+
+
+def e8m0_value(code: int) -> float:
+    return _load().kvqo_e8m0_value(int(code))
+
+
+def e8m0_ceil(s: float) -> int:
+    return int(_load().kvqo_e8m0_ceil(float(s)))
+
+
+# --- quantizers --------------------------------------------------------------
+
+def affine_int8_row(x_bits: np.ndarray):
+    """ExecuTorch PR 24473, Summary: per-token-and-head affine int8 of one row.
+
+    Returns (codes int8 [D], scale float32, zero_point int8)."""
+    x = _u16(x_bits)
+    D = x.shape[-1]
+    q = np.zeros(D, np.int8)
+    scale = np.zeros(1, np.float32)
+    zp = np.zeros(1, np.int8)
+    _load().kvqo_affine_int8_row(_ptr(x), D, _ptr(q), _ptr(scale), _ptr(zp))
+    return q, scale[0], zp[0]
+
+
+def block_row(mode: int, x_bits: np.ndarray):
+    """IndexerQuantCache, 计算公式: per-32 block quantization of one row.
+
+    Returns (codes uint8 [d or d/2], scales float32 [d/32] or uint8 E8M0 [d/32])."""
+    x = _u16(x_bits)
+    d = x.shape[-1]
+    codes = np.zeros(d // 2 if mode == MODE_MXFP4 else d, np.uint8)
+    sf = np.zeros(d // 32, np.float32)
+    se = np.zeros(d // 32, np.uint8)
+    _load().kvqo_block_row(mode, _ptr(x), d, _ptr(codes), _ptr(sf), _ptr(se))
+    return codes, (sf if mode == MODE_FP8_E4M3 else se)
+
+
+def write(mode: int, x_bits: np.ndarray, slot_mapping: np.ndarray, num_slots: int,
+          codes: np.ndarray, scales: np.ndarray, zero_points: np.ndarray | None = None) -> int:
+    """The cache write (quantize + scatter by slot_mapping, -1 = skip), in place.
+
+    x_bits: uint16 [B, H, T, D] (any strides are flattened to contiguous here).
+    Returns the error word (bit 0 = a slot outside [0, num_slots) was skipped)."""
+    x = _u16(x_bits)
+    B, H, T, D = x.shape
+    xs = np.array([H * T * D, T * D, D, 1], np.int64)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
+    assert sm.size == B * T
+    err = np.zeros(1, np.int32)
+    _load().kvqo_write(mode, _ptr(x), B, H, T, D, _ptr(xs), _ptr(sm), int(num_slots), _ptr(codes),
+                       _ptr(scales), _ptr(zero_points), _ptr(err))
+    return int(err[0])
+
+
+# --- sink / ring layout --------------------------------------------------------
+
+def sink_plan(input_pos: int, B: int, T: int, sink: int, S: int, slot_pos: np.ndarray):
+    """ExecuTorch PR 24473, Summary (CachePositionsManagerWithSink): slots for
+    positions input_pos .. input_pos+T-1; updates slot_pos in place.
+
+    Returns (slot_mapping int32 [B*T], kv_len)."""
+    assert slot_pos.dtype == np.int32 and slot_pos.size == S
+    sm = np.zeros(B * T, np.int32)
+    kv = np.zeros(1, np.int32)
+    _load().kvqo_sink_plan(int(input_pos), B, T, int(sink), int(S), _ptr(sm), _ptr(slot_pos), _ptr(kv))
+    return sm, int(kv[0])
+
+
+def sink_mask(input_pos: int, Lq: int, slot_pos: np.ndarray) -> np.ndarray:
+    """ExecuTorch PR 24473, Summary (_create_causal_mask_for_attention_sink):
+    additive float mask [Lq, S]."""
+    S = slot_pos.size
+    mask = np.zeros((Lq, S), np.float32)
+    _load().kvqo_sink_mask(int(input_pos), Lq, _ptr(np.ascontiguousarray(slot_pos, np.int32)), S,
+                           _ptr(mask))
+    return mask
+
+
+# --- attention -------------------------------------------------------------------
+
+def _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask):
+    q = _u16(q_bits)
+    arrs = [np.ascontiguousarray(a) for a in (k, ks, kz, v, vs, vz)]
+    assert arrs[0].dtype == np.int8 and arrs[3].dtype == np.int8
+    assert arrs[1].dtype == np.float32 and arrs[4].dtype == np.float32
+    assert arrs[2].dtype == np.int8 and arrs[5].dtype == np.int8
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.float32)
+    return q, arrs, m
+
+
+def sdpa(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, mask=None,
+         is_causal: bool = False) -> np.ndarray:
+    """fp64 attention over the dequantized int8 cache (abaddon KvCache::forward_attention
+    shapes; ExecuTorch PR 20351 kv_len bound and causal rule; PR 24473 additive mask).
+
+    q_bits uint16 [B, Hq, Lq, D]; k/v int8 [B, Hkv, S, D]; ks/vs f32 and kz/vz int8
+    [B, Hkv, S].  Returns float64 [B, Hq, Lq, D]."""
+    q, (k, ks, kz, v, vs, vz), m = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    out = np.zeros((B, Hq, Lq, D), np.float64)
+    _load().kvqo_sdpa(_ptr(q), B, Hq, Lq, D, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs), _ptr(vz),
+                      Hkv, S, int(kv_len), _ptr(m), int(bool(is_causal)), float(sm_scale), _ptr(out))
+    return out
+
+
+def sdpa_rows(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, rows, mask=None,
+              is_causal: bool = False) -> np.ndarray:
+    """Same as ``sdpa`` for selected (b, h, i) rows only; returns float64 [len(rows), D]."""
+    q, (k, ks, kz, v, vs, vz), m = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    out = np.zeros((len(rows), D), np.float64)
+    lib = _load()
+    for n, (b, h, i) in enumerate(rows):
+        lib.kvqo_sdpa_row(_ptr(q), B, Hq, Lq, D, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs),
+                          _ptr(vz), Hkv, S, int(kv_len), _ptr(m), int(bool(is_causal)), float(sm_scale),
+                          int(b), int(h), int(i), out[n].ctypes.data)
+    return out
+
+
+def dequant_int8(codes: np.ndarray, scale: np.ndarray, zp: np.ndarray) -> np.ndarray:
+    """(q - zp) * scale in fp64 (the dequantization of the affine int8 reading)."""
+    return (codes.astype(np.float64) - zp.astype(np.float64)[..., None]) * scale.astype(np.float64)[..., None]

@@ -1,0 +1,187 @@
+"""Pins for the oracle's quantizers (CPU only).
+
+int8 affine per token and head: ExecuTorch PR 24473, Summary (affine
+asymmetric, float32 scale, int8 zero point) -- the formula is a reading, pinned
+by hand-derived rows and by the dequantization error bound.
+Per-32 block modes: IndexerQuantCache page, 计算公式 (scale_g = max|x_g| / Q_MAX,
+q_i = round(x_i / scale_g)) and the quant_mode list -- pinned by hand-derived
+groups, the scale identity and the format error bounds.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_kv_cache_20_b200 import workloads as wl
+
+FLT_EPS = float(np.finfo(np.float32).eps)
+
+
+def _bits(values):
+    t = torch.tensor([float(v) for v in values], dtype=torch.float32).to(torch.bfloat16)
+    assert torch.equal(t.float(), torch.tensor([float(v) for v in values], dtype=torch.float32)), \
+        "golden inputs must be exact in bf16"
+    return wl.u16(t)
+
+
+def _blocks(path):
+    blocks, cur = [], {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line.startswith("#"):
+                continue
+            if not line:
+                if cur:
+                    blocks.append(cur)
+                cur = {}
+                continue
+            k, v = line.split(":", 1)
+            cur[k.strip()] = v.split()
+    if cur:
+        blocks.append(cur)
+    return blocks
+
+
+def test_affine_golden_rows(golden_dir):
+    blocks = _blocks(os.path.join(golden_dir, "affine_int8_rows.txt"))
+    assert len(blocks) == 5
+    for b in blocks:
+        q, scale, zp = oracle.affine_int8_row(_bits(b["x"]))
+        assert q.tolist() == [int(v) for v in b["q"]], b
+        assert float(scale) == float(np.float32(b["scale"][0]))
+        assert int(zp) == int(b["zp"][0])
+
+
+def _rows():
+    g = wl.generator(21)
+    rows = [wl.bf16_normal((64,), g) for _ in range(200)]
+    rows += [wl.bf16_normal((128,), g, outlier_p=0.05, outlier_scale=30.0) for _ in range(100)]
+    rows += [wl.bf16_normal((128,), g).abs() for _ in range(50)]          # all >= 0
+    rows += [-wl.bf16_normal((256,), g).abs() for _ in range(50)]         # all <= 0
+    rows += [wl.bf16_normal((64,), g) * 1e-6 for _ in range(20)]          # below the epsilon floor
+    rows += [torch.full((64,), 3.0, dtype=torch.bfloat16), torch.zeros(64, dtype=torch.bfloat16)]
+    return rows
+
+
+def test_affine_dequant_error_bound():
+    # |(q - zp) * scale - x| <= scale * (1/2 + 2^-13): half a step, plus the
+    # binary32 rounding of x / scale (<= 2^-16 of a step for |x/scale| <= 256)
+    # and of scale itself at the clamped top code (< 5e-5 of a step).
+    for row in _rows():
+        q, scale, zp = oracle.affine_int8_row(wl.u16(row))
+        x = row.double().numpy()
+        deq = (q.astype(np.float64) - float(zp)) * float(scale)
+        assert np.all(np.abs(deq - x) <= float(scale) * (0.5 + 2.0 ** -13)), row
+
+
+def test_affine_range_is_used():
+    for row in _rows():
+        q, scale, zp = oracle.affine_int8_row(wl.u16(row))
+        x = row.float().numpy()
+        mn, mx = min(0.0, x.min()), max(0.0, x.max())
+        if mn < 0:
+            assert q[np.argmin(x)] == -128           # the minimum lands on the lowest code
+        else:
+            assert int(zp) == -128                    # zero is the lowest value
+        if mx > 0 and float(scale) > FLT_EPS:
+            assert q[np.argmax(x)] >= 126             # the maximum lands at the top
+        assert float(scale) >= FLT_EPS
+
+
+def test_affine_zero_maps_to_zero_point():
+    # an exact 0 dequantizes to exactly 0 (0 is always inside [mn, mx])
+    row = torch.tensor([0.0, -1.5, 2.25, 0.0, 0.5, -0.75, 0.0, 1.0], dtype=torch.bfloat16)
+    q, scale, zp = oracle.affine_int8_row(wl.u16(row))
+    assert q[0] == zp and q[3] == zp and q[6] == zp
+
+
+def test_block_golden_groups(golden_dir):
+    for b in _blocks(os.path.join(golden_dir, "block_groups.txt")):
+        mode = int(b["mode"][0])
+        xs = [float(v) for v in b["x"]]
+        xs += [float(b["fill"][0])] * (32 - len(xs))
+        codes, scales = oracle.block_row(mode, _bits(xs))
+        want = [int(c, 16) for c in b["codes"]]
+        nbytes = 16 if mode == 3 else 32
+        want += [int(b["codefill"][0], 16)] * (nbytes - len(want))
+        assert codes.tolist() == want, (mode, [hex(c) for c in codes], b)
+        if mode == 1:
+            assert float(scales[0]) == float(np.float32(b["scale"][0]))
+        else:
+            assert int(scales[0]) == int(b["scale"][0])
+
+
+def _block_input(rows, d, seed):
+    g = wl.generator(seed)
+    x = wl.bf16_normal((rows, d), g, outlier_p=0.01, outlier_scale=10.0)
+    x[0, :32] = 0                                   # an all-zero group
+    x[1, 32:64] = torch.linspace(-1e-30, 1e-30, 32).to(torch.bfloat16)  # tiny group
+    return x
+
+
+def _decode_e4m3(codes):
+    table = np.array([oracle.e4m3_value(c) for c in range(256)])
+    return table[codes]
+
+
+def _decode_e2m1(packed):
+    table = np.array([oracle.e2m1_value(c) for c in range(16)])
+    lo, hi = packed & 0xF, packed >> 4
+    return np.stack([table[lo], table[hi]], axis=-1).reshape(*packed.shape[:-1], -1)
+
+
+@pytest.mark.parametrize("mode", [1, 2, 3])
+def test_block_scale_and_error_bounds(mode):
+    x = _block_input(64, 512, 31 + mode)
+    for r in range(x.shape[0]):
+        row = x[r]
+        codes, scales = oracle.block_row(mode, wl.u16(row))
+        xv = row.double().numpy().reshape(-1, 32)
+        amax = np.abs(xv).max(axis=1)
+        if mode == 1:
+            scale = scales.astype(np.float64)
+            # scale_g = max|x_g| / 448 in binary32: within half an ulp of the real quotient
+            assert np.all(np.abs(scale - amax / 448) <= np.spacing(scales).astype(np.float64) / 2 + 1e-300)
+            deq = _decode_e4m3(codes).reshape(-1, 32) * scale[:, None]
+        else:
+            scale = np.exp2(scales.astype(np.float64) - 127)
+            qmax = 448.0 if mode == 2 else 6.0
+            nz = amax > 0
+            # the E8M0 scale is the smallest power of two with amax/scale <= Q_MAX
+            # (up to the binary32 rounding of amax / Q_MAX)
+            r_ = amax[nz] / scale[nz]
+            assert np.all(r_ <= qmax * (1 + 2.0 ** -23)) and np.all(r_ > qmax / 2 * (1 - 2.0 ** -23))
+            assert np.all(scales[~nz] == 0)
+            if mode == 2:
+                deq = _decode_e4m3(codes).reshape(-1, 32) * scale[:, None]
+            else:
+                deq = _decode_e2m1(codes).reshape(-1, 32) * scale[:, None]
+        err = np.abs(deq - xv)
+        if mode in (1, 2):
+            # E4M3: half an ulp is 2^-4 relative for normals; 2^-10 absolute
+            # (units of scale) in the subnormal range; + binary32 rounding of x/scale
+            bound = 2.0 ** -4 * np.abs(xv) + 2.0 ** -10 * scale[:, None] + 1e-6 * np.abs(xv)
+        else:
+            bound = 1.0 * scale[:, None] * (1 + 1e-6)   # widest E2M1 gap (4 -> 6) is 2
+        assert np.all(err <= bound), (mode, r, err.max())
+        # all-zero groups write zero codes
+        zero_groups = np.where(amax == 0)[0]
+        for gi in zero_groups:
+            nb = 16 if mode == 3 else 32
+            assert np.all(codes[gi * nb:(gi + 1) * nb] == 0)
+
+
+def test_block_amax_element_hits_the_top_code():
+    x = _block_input(16, 256, 77)
+    for r in range(x.shape[0]):
+        row = x[r]
+        codes, _ = oracle.block_row(1, wl.u16(row))
+        xv = row.float().numpy().reshape(-1, 32)
+        for gi in range(xv.shape[0]):
+            if np.abs(xv[gi]).max() == 0:
+                continue
+            j = np.argmax(np.abs(xv[gi]))
+            assert codes[gi * 32 + j] & 0x7F == 0x7E    # |x| = amax -> 448

@@ -1,0 +1,129 @@
+"""Pins for the oracle's fp64 attention over the int8 cache (CPU only).
+
+abaddon src/attention_cache/mod.rs, trait KvCache (forward_attention shapes,
+GQA through repeat_kv, scale typically 1/sqrt(head_dim)); ExecuTorch PR 20351
+commit notes (kv_len bounds the loop; causal row i sees kv_len - Lq + i; at
+Lq = 1 the causal bound is the whole kv_len); ExecuTorch PR 24473, Summary
+(additive float mask).  Checked against torch's scaled_dot_product_attention
+in float64 (an independent library routine), closed forms and invariances.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from quantized_kv_cache_20_b200 import workloads as wl
+
+
+def _case(seed, B=2, Hq=4, Hkv=2, Lq=3, D=16, S=24):
+    g = wl.generator(seed)
+    q = wl.bf16_normal((B, Hq, Lq, D), g)
+    k, ks, kz = wl.int8_cache_like(B, Hkv, S, D, g)
+    v, vs, vz = wl.int8_cache_like(B, Hkv, S, D, g)
+    return q, (k, ks, kz), (v, vs, vz)
+
+
+def _np(c):
+    return [t.numpy() for t in c]
+
+
+def _torch_ref(q, K, V, kv_len, sm_scale, mask=None, is_causal=False):
+    k, ks, kz = K
+    v, vs, vz = V
+    kd = (k.double() - kz.double()[..., None]) * ks.double()[..., None]
+    vd = (v.double() - vz.double()[..., None]) * vs.double()[..., None]
+    kd, vd = kd[:, :, :kv_len], vd[:, :, :kv_len]
+    G = q.shape[1] // k.shape[1]
+    kd = kd.repeat_interleave(G, dim=1)      # contiguous GQA groups (repeat_kv)
+    vd = vd.repeat_interleave(G, dim=1)
+    Lq = q.shape[2]
+    bias = torch.zeros(Lq, kv_len, dtype=torch.float64)
+    if mask is not None:
+        bias = bias + torch.from_numpy(mask[:, :kv_len]).double()
+    if is_causal:
+        i = torch.arange(Lq)[:, None]
+        j = torch.arange(kv_len)[None, :]
+        bias = bias.masked_fill(j > kv_len - Lq + i, -math.inf)
+    # the oracle takes sm_scale as binary32, as the C ABI does
+    sm_scale = float(np.float32(sm_scale))
+    return F.scaled_dot_product_attention(q.double(), kd, vd, attn_mask=bias, scale=sm_scale).numpy()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (4, 4), (8, 1)])
+@pytest.mark.parametrize("is_causal", [False, True])
+def test_matches_torch_sdpa_fp64(Hq, Hkv, is_causal):
+    q, K, V = _case(1, Hq=Hq, Hkv=Hkv)
+    kv_len, sm = 19, 1 / math.sqrt(16)
+    ours = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=sm, is_causal=is_causal)
+    ref = _torch_ref(q, K, V, kv_len, sm, is_causal=is_causal)
+    np.testing.assert_allclose(ours, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_matches_torch_with_additive_mask():
+    q, K, V = _case(2, Lq=2)
+    rng = np.random.default_rng(3)
+    mask = np.where(rng.random((2, 24)) < 0.3, -np.inf, rng.normal(size=(2, 24))).astype(np.float32)
+    mask[:, 0] = 0.0
+    ours = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=24, sm_scale=0.3, mask=mask)
+    ref = _torch_ref(q, K, V, 24, 0.3, mask=mask)
+    np.testing.assert_allclose(ours, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_uniform_keys_give_mean_of_values():
+    q, K, V = _case(3, B=1, Lq=1)
+    k, ks, kz = K
+    k[:] = k[:, :, :1]
+    ks[:] = ks[:, :, :1]
+    kz[:] = kz[:, :, :1]
+    kv_len = 11
+    out = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=0.25)
+    vd = oracle.dequant_int8(*_np(V))[:, :, :kv_len].mean(axis=2)     # [B, Hkv, D]
+    G = q.shape[1] // k.shape[1]
+    for h in range(q.shape[1]):
+        np.testing.assert_allclose(out[0, h, 0], vd[0, h // G], rtol=1e-12, atol=1e-12)
+
+
+def test_single_visible_slot_returns_its_value():
+    q, K, V = _case(4, B=1, Lq=1)
+    mask = np.full((1, 24), -np.inf, np.float32)
+    mask[0, 7] = 0.0
+    out = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=20, sm_scale=0.25, mask=mask)
+    vd = oracle.dequant_int8(*_np(V))
+    for h in range(4):
+        np.testing.assert_allclose(out[0, h, 0], vd[0, h // 2, 7], rtol=0, atol=1e-12)
+
+
+def test_causal_at_lq1_equals_unbounded_and_kv_len_truncates():
+    q, K, V = _case(5, Lq=1)
+    a = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=17, sm_scale=0.2, is_causal=True)
+    b = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=17, sm_scale=0.2)
+    assert np.array_equal(a, b)
+    # kv_len = n over a cache equals attention over a cache that only has n slots
+    K17 = [t[:, :, :17].contiguous() for t in K]
+    V17 = [t[:, :, :17].contiguous() for t in V]
+    c = oracle.sdpa(wl.u16(q), *_np(K17), *_np(V17), kv_len=17, sm_scale=0.2)
+    assert np.array_equal(b, c)
+
+
+def test_constant_mask_shift_changes_nothing_and_empty_row_is_zero():
+    q, K, V = _case(6, Lq=2)
+    m0 = np.zeros((2, 24), np.float32)
+    a = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=24, sm_scale=0.2, mask=m0)
+    b = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=24, sm_scale=0.2, mask=m0 + 3.5)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    m1 = np.full((2, 24), -np.inf, np.float32)
+    z = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=24, sm_scale=0.2, mask=m1)
+    assert np.all(z == 0)
+
+
+def test_rows_helper_matches_full():
+    q, K, V = _case(7, Lq=3)
+    full = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=21, sm_scale=0.2, is_causal=True)
+    rows = [(0, 0, 0), (1, 3, 2), (0, 2, 1)]
+    part = oracle.sdpa_rows(wl.u16(q), *_np(K), *_np(V), kv_len=21, sm_scale=0.2, rows=rows,
+                            is_causal=True)
+    for n, (b, h, i) in enumerate(rows):
+        assert np.array_equal(part[n], full[b, h, i])

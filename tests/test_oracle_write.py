@@ -1,0 +1,117 @@
+"""Pins for the oracle's cache write = quantize + scatter (CPU only).
+
+IndexerQuantCache page, 功能说明 / 约束说明: results are scattered by slot_mapping,
+-1 skips the token, valid slots lie in [0, num_slots); the cache is updated in
+place.  coreai_opt KVCacheQuantConfig, "Precondition on the cache op": the
+cache op is pure data movement, so it commutes with quantize/dequantize.
+ExecuTorch PR 24473, Summary: a write outside the slot count is rejected; an
+already-quantized cache is left alone, so a second identical pass is a no-op.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_kv_cache_20_b200 import workloads as wl
+
+
+def _setup(mode, seed, B=2, H=3, T=12, D=64, S=40):
+    g = wl.generator(seed)
+    x = wl.bf16_normal((B, H, T, D), g, outlier_p=0.02, outlier_scale=8.0)
+    sm = torch.stack([wl.slot_mapping_random(T, S, 3, g) for _ in range(B)]).reshape(-1)
+    if mode == 0:
+        codes, scales, zps = wl.int8_cache_random(B, H, S, D, g)
+        cache = [codes.numpy().copy(), scales.numpy().copy(), zps.numpy().copy()]
+    else:
+        codes, scales = wl.block_cache_random(B, H, S, D, mode, g)
+        cache = [codes.numpy().copy(), scales.numpy().copy(), None]
+    return x, sm.numpy(), cache
+
+
+def _write(mode, x, sm, S, cache):
+    return oracle.write(mode, wl.u16(x), sm, S, cache[0], cache[1], cache[2])
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_skipped_and_unwritten_slots_are_untouched(mode):
+    S = 40
+    x, sm, cache = _setup(mode, 100 + mode, S=S)
+    before = [None if c is None else c.copy() for c in cache]
+    assert _write(mode, x, sm, S, cache) == 0
+    B, H, T, _ = x.shape
+    written = np.zeros((B, S), bool)
+    for b in range(B):
+        for t in range(T):
+            s = sm[b * T + t]
+            if s >= 0:
+                written[b, s] = True
+    for c, c0 in zip(cache, before):
+        if c is None:
+            continue
+        for b in range(B):
+            for s in range(S):
+                if not written[b, s]:
+                    assert np.array_equal(c[b, :, s], c0[b, :, s])
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_written_row_equals_the_row_quantized_alone(mode):
+    # commuting: slot placement does not change the row's codes
+    S = 40
+    x, sm, cache = _setup(mode, 200 + mode, S=S)
+    _write(mode, x, sm, S, cache)
+    B, H, T, D = x.shape
+    for b in range(B):
+        for t in range(T):
+            s = sm[b * T + t]
+            if s < 0:
+                continue
+            for h in range(H):
+                row = wl.u16(x[b, h, t])
+                if mode == 0:
+                    q, sc, zp = oracle.affine_int8_row(row)
+                    assert np.array_equal(cache[0][b, h, s], q)
+                    assert cache[1][b, h, s] == sc and cache[2][b, h, s] == zp
+                else:
+                    q, sc = oracle.block_row(mode, row)
+                    assert np.array_equal(cache[0][b, h, s], q)
+                    assert np.array_equal(cache[1][b, h, s], sc)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_second_identical_write_is_a_no_op(mode):
+    S = 40
+    x, sm, cache = _setup(mode, 300 + mode, S=S)
+    _write(mode, x, sm, S, cache)
+    once = [None if c is None else c.copy() for c in cache]
+    _write(mode, x, sm, S, cache)
+    for c, c1 in zip(cache, once):
+        if c is not None:
+            assert np.array_equal(c, c1)
+
+
+@pytest.mark.parametrize("mode", [0, 3])
+def test_permuting_tokens_with_their_slots(mode):
+    S = 40
+    x, sm, cache = _setup(mode, 400 + mode, B=1, S=S)
+    cache2 = [None if c is None else c.copy() for c in cache]
+    _write(mode, x, sm, S, cache)
+    perm = torch.randperm(x.shape[2], generator=wl.generator(9))
+    _write(mode, x[:, :, perm].contiguous(), sm[perm.numpy()], S, cache2)
+    for a, b in zip(cache, cache2):
+        if a is not None:
+            assert np.array_equal(a, b)
+
+
+def test_out_of_range_slot_is_skipped_and_reported():
+    S = 40
+    x, sm, cache = _setup(0, 500, B=1, S=S)
+    sm = sm.copy()
+    sm[0], sm[1] = S, -7
+    before = [c.copy() for c in cache]
+    err = _write(0, x, sm, S, cache)
+    assert err & 1
+    # the bad tokens wrote nothing: every changed slot belongs to a valid token
+    valid = set(int(s) for s in sm if 0 <= s < S)
+    changed = {s for s in range(S) if not np.array_equal(cache[0][0, :, s], before[0][0, :, s])}
+    assert changed <= valid
