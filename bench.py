@@ -1,0 +1,522 @@
+"""Benchmark of the quantized KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+A step is one decode step of the `decode` workload on one GPU: write one new
+token's K and V (int8 affine per token and head) for batch 8 x 8 kv heads into
+slot 4095, then run decode attention for 32 q heads at kv_len 4096 (read from
+device memory) over the 8192-slot cache.  Eight independent layer caches are
+rotated step by step, so each step reads a cache that is not in L2 (8 x 66.6
+MiB > 126 MB).  Steps are replayed from CUDA graphs.  With N > 1 (torchrun),
+every rank runs its own replica (weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+Printed (rank 0): one JSON line with the headline metric (tokens/s), the
+roofline of the dominant kernel (decode attention, HBM-bound), the end-to-end
+number through the Python binding with host buffers, the CPU oracle baseline,
+clocks sampled during the timed region, and per-kernel detail lines for the
+bulk fill write, the block-quantized writes and the long-context decode.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KV-write GB/s + int8-KV decode attn tokens/s, % of B200 HBM roofline"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--no-detail", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of this GPU's SM clock and throttle reasons."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- dist
+class Dist:
+    def __init__(self, n_req: int):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if n_req != self.world and self.world != 1:
+            raise SystemExit(f"--gpus {n_req} but WORLD_SIZE={self.world}")
+        self.torch = torch
+        self.device = None
+        self.pg = False
+
+    def setup_cuda(self):
+        torch = self.torch
+        self.device = torch.device("cuda", self.local)
+        torch.cuda.set_device(self.device)
+        if self.world > 1:
+            import torch.distributed as td
+            td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=self.device)
+            self.pg = True
+
+    def setup_cpu(self):
+        if self.world > 1:
+            import torch.distributed as td
+            td.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as td
+            if self.device is not None:
+                td.barrier(device_ids=[self.local])
+            else:
+                td.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch.distributed as td
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.device or "cpu")
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as td
+            td.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | None = None):
+    """Time the CPU oracle on the decode workload: each step writes one token's K
+    and V (64 rows each) and computes all 256 (b, h) attention rows at kv_len 4096."""
+    import numpy as np
+    import oracle
+    from quantized_kv_cache_20_b200 import workloads as wl
+
+    w = wl.DECODE
+    g = wl.generator(w.seed)
+    S = w.kv_len  # only the first kv_len slots take part in a step
+    K = [t.numpy().copy() for t in wl.int8_cache_like(w.B, w.Hkv, S, w.D, g)]
+    V = [t.numpy().copy() for t in wl.int8_cache_like(w.B, w.Hkv, S, w.D, g)]
+    k = wl.u16(wl.bf16_normal((w.B, w.Hkv, 1, w.D), g))
+    v = wl.u16(wl.bf16_normal((w.B, w.Hkv, 1, w.D), g))
+    q = wl.u16(wl.bf16_normal((w.B, w.Hq, 1, w.D), g))
+    sm = np.full(w.B, S - 1, np.int32)
+    oracle.build()
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.write(0, k, sm, S, *K)
+        oracle.write(0, v, sm, S, *V)
+        oracle.sdpa(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D))
+        steps += 1
+        el = time.perf_counter() - t0
+        if (steps >= min_steps and el >= seconds) or (max_steps is not None and steps >= max_steps):
+            break
+    return steps, el
+
+
+def run_reference(args, dist: Dist):
+    dist.setup_cpu()
+    if dist.rank != 0:
+        dist.close()
+        return
+    from quantized_kv_cache_20_b200 import workloads as wl
+    w = wl.DECODE
+    _oracle_decode_steps(0.0, min_steps=args.warmup, max_steps=args.warmup)
+    steps, el = _oracle_decode_steps(0.0, min_steps=args.steps, max_steps=args.steps)
+    value = w.B * steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * el / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{steps} full decode steps (write 1 token K/V for 8x8 rows + 256 attention "
+                                   f"rows at kv_len 4096), single-threaded C oracle"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def _config(args):
+    return {
+        "workload": "decode step: batch 8, 32 q / 8 kv heads (GQA 4:1), D=128, int8 per-token-head KV cache of "
+                    "8192 slots with 4096 filled; write 1 token K/V then decode attention at kv_len 4096 "
+                    "read on device",
+        "global_batch": 8 * args.gpus,
+        "seq_len": 4096,
+        "l2": f"{args.layers} independent layer caches rotated per step ({args.layers} x 66.6 MiB read > 126 MB L2)",
+        "graphs": "each step replayed from a CUDA graph",
+        "parallelism": f"replicas x{args.gpus} (weak scaling, no collective on the data path)",
+    }
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def run_kvq(args, dist: Dist):
+    import torch
+    from quantized_kv_cache_20_b200 import build as kbuild
+    from quantized_kv_cache_20_b200 import kvq
+    from quantized_kv_cache_20_b200 import workloads as wl
+
+    dist.setup_cuda()
+    if dist.local == 0:
+        kbuild.build()
+    dist.barrier()
+    kvq.load()
+    dev = dist.device
+    w = wl.DECODE
+    B, Hq, Hkv, D, S, KV = w.B, w.Hq, w.Hkv, w.D, w.S, w.kv_len
+    NL = args.layers
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + dist.rank)
+
+    # ---- caches, filled by the write kernel (positions 0..4094, slot = position)
+    Tf = KV - 1
+    xk = torch.randn((B, Hkv, Tf, D), generator=gen, device=dev).to(torch.bfloat16)
+    xv = torch.randn((B, Hkv, Tf, D), generator=gen, device=dev).to(torch.bfloat16)
+    sm_fill = torch.arange(Tf, dtype=torch.int32, device=dev).repeat(B)
+    layers = []
+    for _ in range(NL):
+        K = (torch.empty((B, Hkv, S, D), dtype=torch.int8, device=dev),
+             torch.empty((B, Hkv, S), dtype=torch.float32, device=dev),
+             torch.empty((B, Hkv, S), dtype=torch.int8, device=dev))
+        V = (torch.empty_like(K[0]), torch.empty_like(K[1]), torch.empty_like(K[2]))
+        kvq.write(0, xk, sm_fill, *K)
+        kvq.write(0, xv, sm_fill, *V)
+        layers.append((K, V))
+    q = torch.randn((B, Hq, 1, D), generator=gen, device=dev).to(torch.bfloat16)
+    kn = torch.randn((B, Hkv, 1, D), generator=gen, device=dev).to(torch.bfloat16)
+    vn = torch.randn((B, Hkv, 1, D), generator=gen, device=dev).to(torch.bfloat16)
+    sm_step = torch.full((B,), KV - 1, dtype=torch.int32, device=dev)
+    kv_len = torch.tensor([KV], dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=dev)
+    ws = kvq.decode_workspace(B, Hq, Hkv, D, S, dev)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(l):
+        K, V = layers[l]
+        kvq.write(0, kn, sm_step, *K)
+        kvq.write(0, vn, sm_step, *V)
+        kvq.decode_attn(q, *K, *V, kv_len, out=out, workspace=ws)
+
+    def decode_only(l):
+        K, V = layers[l]
+        kvq.decode_attn(q, *K, *V, kv_len, out=out, workspace=ws)
+
+    # warm the launch path once outside capture, then capture one graph per layer
+    with torch.cuda.stream(stream):
+        for l in range(NL):
+            step(l)
+    torch.cuda.synchronize()
+    step_graphs, dec_graphs = [], []
+    for l in range(NL):
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=stream):
+            step(l)
+        step_graphs.append(gph)
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            decode_only(l)
+        dec_graphs.append(gd)
+    torch.cuda.synchronize()
+
+    # ---- headline: K steps
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step_graphs[i % NL].replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            step_graphs[i % NL].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = dist.max(ms_local)
+    value = dist.world * B / (ms / 1000.0)
+
+    # ---- dominant kernel: decode attention alone, same rotation, events on its stream
+    reps = max(1, args.steps // NL)
+    with torch.cuda.stream(stream):
+        for l in range(NL):
+            dec_graphs[l].replay()
+        e0.record(stream)
+        for r in range(reps):
+            for l in range(NL):
+                dec_graphs[l].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = e0.elapsed_time(e1) / (reps * NL)
+    dec_bytes = 2 * B * Hkv * KV * (D + 4 + 1) + 2 * (B * Hq * D * 2)
+    peak, peak_kind = _peaks()
+    achieved = dec_bytes / (dec_ms / 1000.0) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
+                "kernel": "decode_kernel (split-K int8 decode attention)", "bytes_per_launch": dec_bytes,
+                "launch_us": dec_ms * 1000.0, "traffic": None}
+
+    # ---- end to end through the binding with host buffers
+    e2e = _e2e(args, dist, kvq, layers, ws, kv_len, sm_step)
+
+    detail = {}
+    if not args.no_detail:
+        detail = _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk, "detail": detail,
+    }
+    if dist.rank == 0 and dist.world == 1:
+        steps_c, el_c = _oracle_decode_steps(args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": B * steps_c / el_c, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{steps_c} full decode steps of the same workload (write 1 token K/V for 8x8 rows + "
+                      f"256 attention rows at kv_len 4096), single-threaded C oracle, {el_c:.1f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    for gph in step_graphs + dec_graphs:
+        del gph
+    dist.close()
+
+
+def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
+    import torch
+    from quantized_kv_cache_20_b200 import workloads as wl
+    w = wl.DECODE
+    B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
+    dev = dist.device
+    NL = len(layers)
+    steps = max(NL, min(args.steps, 200))
+    g = torch.Generator().manual_seed(7)
+    hq = torch.randn((B, Hq, 1, D), generator=g).to(torch.bfloat16).pin_memory()
+    hk = torch.randn((B, Hkv, 1, D), generator=g).to(torch.bfloat16).pin_memory()
+    hv = torch.randn((B, Hkv, 1, D), generator=g).to(torch.bfloat16).pin_memory()
+    hout = torch.empty((steps, B, Hq, 1, D), dtype=torch.bfloat16).pin_memory()
+    dq = torch.empty_like(hq, device=dev)
+    dk = torch.empty_like(hk, device=dev)
+    dv = torch.empty_like(hv, device=dev)
+    dout = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=dev)
+
+    def one(i):
+        K, V = layers[i % NL]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        kvq.write(0, dk, sm_step, *K)
+        kvq.write(0, dv, sm_step, *V)
+        kvq.decode_attn(dq, *K, *V, kv_len, out=dout, workspace=ws)
+        hout[i].copy_(dout, non_blocking=True)
+
+    for i in range(min(NL, steps)):
+        one(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        one(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.max(e0.elapsed_time(e1) / steps)
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    return {"value": dist.world * B / (ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": dout.numel() * 2, "ms_per_step": ms, "steps": steps,
+            "path": "pinned host -> device copies, kvq.write x2 + kvq.decode_attn via the Python binding "
+                    "(no graph), device -> pinned host copy of the output"}
+
+
+def _time_graph(stream, fn, reps):
+    """Capture fn() into a graph, replay reps times; return mean ms per replay."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=stream):
+        fn()
+    with torch.cuda.stream(stream):
+        gph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            gph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del gph
+    return ms
+
+
+def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
+    import torch
+    dev = dist.device
+    res = {}
+    # bulk fill write (decode workload): positions 0..4094 of K and V, rotated over the layers
+    w = wl.DECODE
+    NL = len(layers)
+    Tf = xk.shape[2]
+
+    def fill():
+        for K, V in layers:
+            kvq.write(0, xk, sm_fill, *K)
+            kvq.write(0, xv, sm_fill, *V)
+    ms = _time_graph(stream, fill, 3) / (2 * NL)
+    rows = w.B * w.Hkv * Tf
+    fbytes = rows * w.D * 2 + rows * w.D + rows * 5 + w.B * Tf * 4
+    res["int8_fill_write"] = {"what": "kvq_write int8, 8x8 heads x 4095 tokens, D=128", "us": ms * 1000,
+                              "GB/s": fbytes / (ms / 1000) / 1e9, "frac": fbytes / (ms / 1000) / 1e9 / peak,
+                              "bytes": fbytes}
+    # block writes: x [16384, 512], 65536 slots, 10% skipped; 6 rotated input/cache sets (> L2)
+    bw = wl.BLOCK
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    NB = 6
+    sets = []
+    for i in range(NB):
+        x = torch.randn((1, 1, bw.tokens, bw.d), generator=g, device=dev)
+        hit = torch.rand(x.shape, generator=g, device=dev) < bw.outlier_p
+        x = torch.where(hit, x * bw.outlier_scale, x).to(torch.bfloat16)
+        sm = torch.randperm(bw.num_slots, generator=g, device=dev)[: bw.tokens].to(torch.int32)
+        sm[torch.randperm(bw.tokens, generator=g, device=dev)[: int(bw.tokens * bw.skip_frac)]] = -1
+        sets.append((x, sm))
+    valid = bw.tokens - int(bw.tokens * bw.skip_frac)
+    for mode, name in ((1, "fp8_e4m3"), (2, "mxfp8"), (3, "mxfp4")):
+        code_row = bw.d // 2 if mode == 3 else bw.d
+        caches = []
+        for i in range(NB):
+            c = torch.zeros((1, 1, bw.num_slots, code_row), dtype=torch.uint8, device=dev)
+            s = torch.zeros((1, 1, bw.num_slots, bw.d // 32), dtype=torch.float32 if mode == 1 else torch.uint8,
+                            device=dev)
+            caches.append((c, s))
+
+        def blk():
+            for (x, sm), (c, s) in zip(sets, caches):
+                kvq.write(mode, x, sm, c, s)
+        ms = _time_graph(stream, blk, 10) / NB
+        sbytes = (bw.d // 32) * (4 if mode == 1 else 1)
+        byts = valid * (bw.d * 2 + code_row + sbytes) + bw.tokens * 4
+        res[f"block_write_{name}"] = {"what": f"kvq_write mode {mode}, x [16384, 512], 10% skipped",
+                                      "us": ms * 1000, "GB/s": byts / (ms / 1000) / 1e9,
+                                      "frac": byts / (ms / 1000) / 1e9 / peak, "bytes": byts}
+        del caches
+    del sets
+    torch.cuda.empty_cache()
+    # long-context decode: batch 1, 32 q / 16 kv heads, D=256, kv_len 131072 (1 GiB of codes > L2)
+    lw = wl.LONG
+    K = (torch.randint(-128, 128, (1, lw.Hkv, lw.S, lw.D), dtype=torch.int8, device=dev),
+         torch.rand((1, lw.Hkv, lw.S), device=dev) * 0.012 + 0.018,
+         torch.randint(-6, 7, (1, lw.Hkv, lw.S), dtype=torch.int8, device=dev))
+    V = (torch.randint(-128, 128, (1, lw.Hkv, lw.S, lw.D), dtype=torch.int8, device=dev),
+         torch.rand((1, lw.Hkv, lw.S), device=dev) * 0.012 + 0.018,
+         torch.randint(-6, 7, (1, lw.Hkv, lw.S), dtype=torch.int8, device=dev))
+    ql = torch.randn((1, lw.Hq, 1, lw.D), device=dev).to(torch.bfloat16)
+    ol = torch.empty_like(ql)
+    kvl = torch.tensor([lw.kv_len], dtype=torch.int32, device=dev)
+    wsl = kvq.decode_workspace(1, lw.Hq, lw.Hkv, lw.D, lw.S, dev)
+
+    def ldec():
+        kvq.decode_attn(ql, *K, *V, kvl, out=ol, workspace=wsl)
+    ms = _time_graph(stream, ldec, 20)
+    lbytes = 2 * lw.Hkv * lw.kv_len * (lw.D + 5) + 2 * lw.Hq * lw.D * 2
+    res["long_decode"] = {"what": "kvq_decode_attn, batch 1, 32 q / 16 kv heads, D=256, kv_len 131072",
+                          "us": ms * 1000, "tokens/s": 1 / (ms / 1000), "GB/s": lbytes / (ms / 1000) / 1e9,
+                          "frac": lbytes / (ms / 1000) / 1e9 / peak, "bytes": lbytes}
+    return res
+
+
+def main():
+    args = _args()
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, dist)
+    else:
+        run_kvq(args, dist)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * kvq.h -- C ABI of libkvq.so, the B200 (sm_100a) quantized KV-cache library.
+ *
+ * Two halves of one hot path:
+ *   1. kvq_write: quantize bf16 K/V rows and scatter them into a preallocated
+ *      cache by slot (int8 affine per token+head, or per-32 FP8 E4M3 /
+ *      MX-FP8 / MX-FP4 blocks); kvq_sink_plan / kvq_sink_mask assign the slots
+ *      and build the additive mask of an attention-sink / ring cache.
+ *   2. kvq_decode_attn / kvq_prefill_attn: scaled dot-product attention that
+ *      reads the int8 cache and dequantizes it in registers, with GQA, a
+ *      kv_len bound read on the device, a per-tile causal bound and an
+ *      additive mask.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers (CUDA global memory of the current device)
+ *     unless a parameter says "host".  The caller owns every buffer; the
+ *     library never allocates, frees, or synchronizes the host.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it; no call reads
+ *     device memory on the host, so every call can be captured in a CUDA graph.
+ *   - bf16 means IEEE binary16-brain (torch.bfloat16) bit patterns.
+ *   - Return value: KVQ_OK (0) or a negative host status (below).  A non-zero
+ *     status means nothing was enqueued, except KVQ_ECUDA from a failed launch.
+ *   - Conditions only visible on the device never trap: the offending item is
+ *     skipped (or clamped) and a KVQ_ERR_* bit is OR-ed into *err_word
+ *     (nullable, int32 device word, never cleared by the library).
+ *   - Calls that share output buffers must be ordered on streams by the caller.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host status codes. */
+#define KVQ_OK 0
+#define KVQ_EINVAL (-1)       /* null pointer, bad size, misaligned pointer, bad stride */
+#define KVQ_EUNSUPPORTED (-2) /* a valid request this build does not implement */
+#define KVQ_ECUDA (-3)        /* the CUDA launch itself failed */
+
+/* Device error-word bits (OR-ed into *err_word). */
+#define KVQ_ERR_SLOT_RANGE 1   /* a slot outside [0, num_slots) other than -1 was skipped */
+#define KVQ_ERR_KV_LEN_RANGE 2 /* *kv_len outside [0, S] (or [Lq, S] for prefill) was clamped */
+#define KVQ_ERR_INPUT_POS 4    /* *input_pos < 0: the plan wrote -1 slots and kv_len 0 */
+#define KVQ_ERR_TIMEOUT 8      /* a bounded wait inside a kernel gave up; its output is invalid */
+
+/* Cache-write modes. */
+#define KVQ_MODE_INT8_AFFINE 0 /* int8 codes, f32 scale + int8 zero point per (token, head) */
+#define KVQ_MODE_FP8_E4M3 1    /* E4M3 codes, f32 scale per 32 elements ("Normal") */
+#define KVQ_MODE_MXFP8 2       /* E4M3 codes, E8M0 scale per 32 elements */
+#define KVQ_MODE_MXFP4 3       /* E2M1 codes two per byte, E8M0 scale per 32 elements */
+
+/*
+ * kvq_write -- quantize x and scatter it into the cache, in place.
+ *
+ * Defines: ExecuTorch PR 24473, Summary (int8 entries quantized per token and
+ * head, affine asymmetric, float32 scale, int8 zero point, written through
+ * update_cache_with_indices); IndexerQuantCache page, 功能说明 / 计算公式 /
+ * 参数说明 / 约束说明 (per-block dynamic quantization scale_g = max|x_g| / Q_MAX,
+ * q_i = round(x_i / scale_g); results and scales scattered to slot_mapping,
+ * -1 skips the token; cache and scale updated in place; d % 32 == 0, d <= 8192);
+ * ExecuTorch PR 20351 commit notes (a static scatter along the position dim,
+ * capturable in a CUDA graph).
+ *
+ * x            bf16, element (b, h, t, i) at x[b*xs[0] + h*xs[1] + t*xs[2] + i];
+ *              x_strides (host, 4 entries, in elements) with xs[3] implied 1.
+ *              The row start of every (b, h, t) must be 16-byte aligned.
+ * B, H, T, D   batch, heads, tokens per batch row, row length.
+ * slot_mapping int32 [B*T]: cache slot of token (b, t) = slot_mapping[b*T + t];
+ *              -1 skips it; any other value outside [0, num_slots) is skipped
+ *              and sets KVQ_ERR_SLOT_RANGE.  Duplicate slots: undefined result.
+ * num_slots    S, slots per (b, h) in the cache.
+ * Cache layouts (row-major, contiguous, 16-byte aligned):
+ *   mode 0: codes int8 [B, H, S, D]; scales float [B, H, S]; zero_points int8 [B, H, S]
+ *   mode 1: codes u8   [B, H, S, D]; scales float [B, H, S, D/32]; zero_points NULL
+ *   mode 2: codes u8   [B, H, S, D]; scales u8 (E8M0) [B, H, S, D/32]
+ *   mode 3: codes u8   [B, H, S, D/2] (element 2i in the low nibble); scales u8 (E8M0)
+ *   With B = H = 1 the block modes are the IndexerQuantCache [num_slots, d] layout.
+ * round_scale  mode 2 only: must be 1 (scale rounded up to a power of two);
+ *              0 returns KVQ_EUNSUPPORTED.  Ignored by the other modes.
+ * Sizes: mode 0 needs D in {64, 128, 256}; modes 1-3 need D % 32 == 0 and
+ * D <= 8192 (KVQ_EUNSUPPORTED otherwise).  B, H, T >= 0 (0 enqueues nothing).
+ * The arithmetic is binary32 with one round-to-nearest-even per operation, in
+ * a fixed order, so codes, scales and zero points are reproducible bit for bit.
+ */
+int kvq_write(int mode, int round_scale, const void *x, int B, int H, int T, int D,
+              const int64_t *x_strides, const int32_t *slot_mapping, int64_t num_slots, void *codes,
+              void *scales, int8_t *zero_points, int32_t *err_word, void *stream);
+
+/*
+ * kvq_sink_plan -- slots of an attention-sink / ring cache for T new tokens.
+ *
+ * Defines: ExecuTorch PR 24473, Summary (CachePositionsManagerWithSink: a
+ * pinned sink prefix plus a ring; the ring cache is the case sink_size = 0).
+ * Position p = *input_pos + t goes to slot p if p < sink_size, else to
+ * sink_size + (p - sink_size) mod (S - sink_size).
+ *
+ * input_pos    int32 device scalar, first position of the T tokens.
+ * B, T         batch rows (all at the same positions) and tokens.
+ * sink_size    pinned prefix length, 0 <= sink_size < S.
+ * S            cache slots; T must be <= S - sink_size (else KVQ_EUNSUPPORTED).
+ * slot_mapping int32 [B*T] out: the slot of token (b, t), ready for kvq_write.
+ * slot_pos     int32 [S] in/out: the position each slot holds, -1 = empty.
+ *              Initialise it to -1 once per sequence.
+ * kv_len       int32 device scalar out: min(*input_pos + T, S), the attention bound.
+ * *input_pos < 0 writes -1 slots and kv_len 0 and sets KVQ_ERR_INPUT_POS.
+ */
+int kvq_sink_plan(const int32_t *input_pos, int B, int T, int sink_size, int64_t S,
+                  int32_t *slot_mapping, int32_t *slot_pos, int32_t *kv_len, int32_t *err_word,
+                  void *stream);
+
+/*
+ * kvq_sink_mask -- additive float mask of an attention-sink / ring cache.
+ *
+ * Defines: ExecuTorch PR 24473, Summary (_create_causal_mask_for_attention_sink;
+ * ring and sink caches use an additive float mask).  Query row r sits at
+ * position *input_pos + r and sees slot s iff 0 <= slot_pos[s] <= *input_pos + r:
+ * mask[r*S + s] = 0.0f if visible, -INFINITY otherwise.  Call it after the
+ * kvq_sink_plan of the same tokens.
+ *
+ * input_pos  int32 device scalar.   Lq  query rows (>= 1).
+ * slot_pos   int32 [S] from kvq_sink_plan.   mask  float [Lq, S] out.
+ */
+int kvq_sink_mask(const int32_t *input_pos, int Lq, const int32_t *slot_pos, int64_t S, float *mask,
+                  void *stream);
+
+/*
+ * kvq_decode_workspace_bytes -- size of the kvq_decode_attn workspace.
+ *
+ * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S), or 0 for
+ * arguments kvq_decode_attn would reject.  The workspace must be zero-filled
+ * once before its first use; every completed call leaves its counters at zero
+ * again, so it can be reused by later calls in stream order (not by two calls
+ * running at the same time).
+ */
+size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
+
+/*
+ * kvq_decode_attn -- one-query attention over the int8 cache (split-K).
+ *
+ * Defines: abaddon 0.2.0-rc.1 src/attention_cache/mod.rs, trait KvCache
+ * (forward_attention: q [batch, num_heads, q_len, head_dim], GQA over
+ * num_kv_heads, scale typically 1/sqrt(head_dim); a fused kernel that does not
+ * materialise K/V); ExecuTorch PR 20351 commit notes (kv_len is an int32 GPU
+ * scalar read on the device, no host sync, bounding the loop to the filled
+ * length); ExecuTorch PR 24473, Summary (ring / sink caches add a float mask).
+ *
+ *   out[b, h, :] = softmax_j(sm_scale * q[b,h,:] . K[b,hk,j,:] + mask[j]) V[b,hk,j,:]
+ *   over j in [0, *kv_len), hk = h / (Hq / Hkv),
+ *   K[b,hk,j,d] = (k[b,hk,j,d] - k_zp[b,hk,j]) * k_scale[b,hk,j] (same for V).
+ *
+ * q            bf16 [B, Hq, 1, D] contiguous.   out  bf16 [B, Hq, 1, D] contiguous.
+ * k, v         int8 [B, Hkv, S, D];  k_scale, v_scale float [B, Hkv, S];
+ *              k_zp, v_zp int8 [B, Hkv, S] (the kvq_write mode-0 layout).
+ * kv_len       int32 device scalar; values outside [0, S] are clamped and set
+ *              KVQ_ERR_KV_LEN_RANGE.  kv_len 0 gives zeros.
+ * mask         nullable float [S] (row 0 of an [Lq, S] mask), added to the
+ *              scaled scores; -INFINITY hides a slot.  A row that sees no slot
+ *              outputs zeros.
+ * workspace    device buffer of workspace_bytes >= kvq_decode_workspace_bytes().
+ * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; every pointer
+ * 16-byte aligned.
+ */
+int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
+                    const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
+                    int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
+                    void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
+
+/*
+ * kvq_prefill_attn -- Lq-query (chunked prefill) attention over the int8 cache.
+ *
+ * Defines: as kvq_decode_attn, plus ExecuTorch PR 20351 commit notes (the
+ * chunk's rows sit at positions kv_len - Lq + i; with a causal mask row i sees
+ * j <= kv_len - Lq + i; mask_is_causal enables the per-tile causal upper bound
+ * loop_end = min(kv_len, (kv_len - Lq) + max(seq_pos in tile) + 1), which skips
+ * KV tiles that are fully masked, so the output is bit-identical either way).
+ *
+ * q, out        bf16 [B, Hq, Lq, D] contiguous.  Cache arguments as for decode.
+ * kv_len        int32 device scalar, clamped to [Lq, S] (KVQ_ERR_KV_LEN_RANGE).
+ * mask          nullable float [Lq, S] additive (row stride S).
+ * is_causal     1: apply the causal rule above (full-context cache).
+ * mask_is_causal 1: the caller asserts the combined mask is causal in slot
+ *               order (is_causal, or a mask that hides j > kv_len - Lq + i),
+ *               which enables the per-tile bound.
+ * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; 1 <= Lq <= S.
+ */
+int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
+                     const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
+                     const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
+                     int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
+                     void *stream);
+
+/* A static, human-readable name for a host status code. */
+const char *kvq_strerror(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

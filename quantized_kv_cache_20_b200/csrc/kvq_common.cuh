@@ -1,0 +1,155 @@
+// kvq_common.cuh -- device helpers shared by the kvq kernels (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "kvq is built for sm_100a only"
+#endif
+
+#define KVQ_DEVINL __device__ __forceinline__
+
+namespace kvq {
+
+// ---------------------------------------------------------------------------
+// Host-side helpers
+// ---------------------------------------------------------------------------
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA; }
+
+inline int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ---------------------------------------------------------------------------
+// Global memory access
+// ---------------------------------------------------------------------------
+// 16-byte streaming load that bypasses L1 (data read exactly once).
+KVQ_DEVINL uint4 ld_stream_v4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+KVQ_DEVINL void st_v2(void *p, uint32_t a, uint32_t b) {
+  asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+
+KVQ_DEVINL void st_u32(void *p, uint32_t a) {
+  asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
+}
+
+KVQ_DEVINL void report(int32_t *err_word, int32_t bits) {
+  if (err_word) atomicOr(err_word, bits);
+}
+
+// bf16 pair (packed in a u32, element 0 in the low half) -> two floats, exact.
+KVQ_DEVINL float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+KVQ_DEVINL float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+KVQ_DEVINL uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk async copy (TMA, untiled) helpers
+// ---------------------------------------------------------------------------
+KVQ_DEVINL uint32_t smem_u32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+KVQ_DEVINL void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+KVQ_DEVINL void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+KVQ_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+KVQ_DEVINL void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+KVQ_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Every wait in this library is bounded: after ~kWaitLimitNs without the
+// phase completing the wait gives up and the caller reports KVQ_ERR_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+KVQ_DEVINL bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// 1-D bulk copy global -> shared, completion signalled on `bar` (tx bytes).
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+KVQ_DEVINL void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+KVQ_DEVINL void bulk_g2s_hint(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar,
+                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, "
+      "[%3], %4;" ::"r"(smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+KVQ_DEVINL uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// int8 -> float, exact, without I2F: the byte (biased by 128) is placed in the
+// low mantissa bits of 2^23, giving 2^23 + (c + 128); subtracting the per-row
+// constant 2^23 + 128 + zp leaves exactly c - zp.
+// ---------------------------------------------------------------------------
+KVQ_DEVINL float magic_byte(uint32_t w_biased, uint32_t sel) {
+  return __uint_as_float(__byte_perm(w_biased, 0x4B000000u, sel));
+}
+// The float -(2^23 + 128 + zp) for a zero point zp in [-128, 127].
+KVQ_DEVINL float neg_magic_zp(int zp) { return __uint_as_float(0xCB000080u + static_cast<uint32_t>(zp)); }
+
+// Four int8 codes in w -> two float2 holding (c - zp) exactly; mzp2 holds
+// neg_magic_zp(zp) in both lanes.
+KVQ_DEVINL void codes4_to_f2(uint32_t w, float2 mzp2, float2 &a, float2 &b) {
+  const uint32_t wb = w ^ 0x80808080u;
+  float2 t0 = make_float2(magic_byte(wb, 0x7540u), magic_byte(wb, 0x7541u));
+  float2 t1 = make_float2(magic_byte(wb, 0x7542u), magic_byte(wb, 0x7543u));
+  a = __fadd2_rn(t0, mzp2);
+  b = __fadd2_rn(t1, mzp2);
+}
+
+}  // namespace kvq

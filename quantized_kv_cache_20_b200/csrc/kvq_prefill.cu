@@ -1,0 +1,49 @@
+// kvq_prefill.cu -- chunked-prefill attention entry point.
+#include "kvq_common.cuh"
+#include "kvq_prefill_simt.cuh"
+
+extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
+                                const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
+                                const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
+                                int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
+                                void *stream) {
+  using namespace kvq;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S > INT32_MAX || Lq <= 0 || Lq > S)
+    return KVQ_EINVAL;
+  if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
+  if (S % 16 != 0) return KVQ_EUNSUPPORTED;
+  if (B == 0) return KVQ_OK;
+  if (!q || !k || !k_scale || !k_zp || !v || !v_scale || !v_zp || !kv_len || !out) return KVQ_EINVAL;
+  const void *ptrs[] = {q, k, k_scale, k_zp, v, v_scale, v_zp, out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return KVQ_EINVAL;
+  if (mask && !aligned16(mask)) return KVQ_EINVAL;
+  if (!(sm_scale == sm_scale)) return KVQ_EINVAL;
+  if (Hq > 65535 || B > 65535) return KVQ_EUNSUPPORTED;
+  simt::PrefillArgs a;
+  a.q = static_cast<const uint16_t *>(q);
+  a.k = k;
+  a.ks = k_scale;
+  a.kz = k_zp;
+  a.v = v;
+  a.vs = v_scale;
+  a.vz = v_zp;
+  a.mask = mask;
+  a.kv_len = kv_len;
+  a.out = static_cast<uint16_t *>(out);
+  a.err = err_word;
+  a.S = S;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Lq = Lq;
+  a.is_causal = is_causal ? 1 : 0;
+  a.mask_is_causal = mask_is_causal ? 1 : 0;
+  a.qscale = sm_scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 64: return simt::launch_prefill_simt<64>(a, s);
+    case 128: return simt::launch_prefill_simt<128>(a, s);
+    default: return simt::launch_prefill_simt<256>(a, s);
+  }
+}

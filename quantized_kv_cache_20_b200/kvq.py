@@ -1,0 +1,217 @@
+"""Thin ctypes binding of libkvq.so (the C ABI in include/kvq.h).
+
+Argument marshalling only: shapes, dtypes and devices are read from torch
+tensors, pointers and sizes are passed to the library, and every kernel runs
+on torch's current CUDA stream.  There is no fallback: if libkvq.so is missing
+or a call fails, a RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+KVQ_OK = 0
+KVQ_EINVAL = -1
+KVQ_EUNSUPPORTED = -2
+KVQ_ECUDA = -3
+
+KVQ_ERR_SLOT_RANGE = 1
+KVQ_ERR_KV_LEN_RANGE = 2
+KVQ_ERR_INPUT_POS = 4
+KVQ_ERR_TIMEOUT = 8
+
+MODE_INT8_AFFINE = 0
+MODE_FP8_E4M3 = 1
+MODE_MXFP8 = 2
+MODE_MXFP4 = 3
+
+EXPORTS = (
+    "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
+    "kvq_decode_attn", "kvq_prefill_attn", "kvq_strerror", "kvq_version",
+)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libkvq.so (once) and declare its signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libkvq.so not found at {p}; build it with "
+                               "`python -m quantized_kv_cache_20_b200.build`")
+        lib = ctypes.CDLL(p)
+        P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        lib.kvq_write.argtypes = [I, I, P, I, I, I, I, P, P, I64, P, P, P, P, P]
+        lib.kvq_write.restype = I
+        lib.kvq_sink_plan.argtypes = [P, I, I, I, I64, P, P, P, P, P]
+        lib.kvq_sink_plan.restype = I
+        lib.kvq_sink_mask.argtypes = [P, I, P, I64, P, P]
+        lib.kvq_sink_mask.restype = I
+        lib.kvq_decode_workspace_bytes.argtypes = [I, I, I, I, I64]
+        lib.kvq_decode_workspace_bytes.restype = SZ
+        lib.kvq_decode_attn.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
+        lib.kvq_decode_attn.restype = I
+        lib.kvq_prefill_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I, I, F, P, P, P]
+        lib.kvq_prefill_attn.restype = I
+        lib.kvq_strerror.argtypes = [I]
+        lib.kvq_strerror.restype = ctypes.c_char_p
+        lib.kvq_version.argtypes = []
+        lib.kvq_version.restype = I
+        _lib = lib
+        return lib
+
+
+def strerror(status: int) -> str:
+    return load().kvq_strerror(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != KVQ_OK:
+        raise KvqError(fn, status, strerror(status))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _cuda(name, t, dtype=None, contiguous=True):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def write(mode: int, x: torch.Tensor, slot_mapping: torch.Tensor, codes: torch.Tensor,
+          scales: torch.Tensor, zero_points: torch.Tensor | None = None, *, round_scale: bool = True,
+          err_word: torch.Tensor | None = None) -> None:
+    """kvq_write: quantize x [B, H, T, D] (bf16, any strides with unit last stride)
+    and scatter into the cache in place.  num_slots is codes.shape[2]."""
+    _cuda("x", x, torch.bfloat16, contiguous=False)
+    if x.dim() != 4 or x.stride(3) != 1:
+        raise ValueError("x must be [B, H, T, D] with a unit last stride")
+    _cuda("slot_mapping", slot_mapping, torch.int32)
+    _cuda("codes", codes)
+    _cuda("scales", scales)
+    _cuda("zero_points", zero_points)
+    _cuda("err_word", err_word, torch.int32)
+    B, H, T, D = x.shape
+    strides = (ctypes.c_int64 * 4)(*x.stride())
+    st = load().kvq_write(int(mode), int(bool(round_scale)), _ptr(x), B, H, T, D, strides,
+                          _ptr(slot_mapping), int(codes.shape[2]), _ptr(codes), _ptr(scales),
+                          _ptr(zero_points), _ptr(err_word), _stream(x.device))
+    _check("kvq_write", st)
+
+
+def sink_plan(input_pos: torch.Tensor, B: int, T: int, sink_size: int, slot_pos: torch.Tensor,
+              slot_mapping: torch.Tensor, kv_len: torch.Tensor,
+              err_word: torch.Tensor | None = None) -> None:
+    """kvq_sink_plan: slot_mapping [B*T] and kv_len (device scalar) for T tokens
+    starting at the device scalar input_pos; updates slot_pos [S] in place."""
+    for n, t in (("input_pos", input_pos), ("slot_pos", slot_pos), ("slot_mapping", slot_mapping),
+                 ("kv_len", kv_len), ("err_word", err_word)):
+        _cuda(n, t, torch.int32)
+    st = load().kvq_sink_plan(_ptr(input_pos), B, T, sink_size, slot_pos.numel(), _ptr(slot_mapping),
+                              _ptr(slot_pos), _ptr(kv_len), _ptr(err_word), _stream(slot_pos.device))
+    _check("kvq_sink_plan", st)
+
+
+def sink_mask(input_pos: torch.Tensor, Lq: int, slot_pos: torch.Tensor, mask: torch.Tensor) -> None:
+    """kvq_sink_mask: additive mask [Lq, S] (float32) from slot_pos."""
+    _cuda("input_pos", input_pos, torch.int32)
+    _cuda("slot_pos", slot_pos, torch.int32)
+    _cuda("mask", mask, torch.float32)
+    st = load().kvq_sink_mask(_ptr(input_pos), Lq, _ptr(slot_pos), slot_pos.numel(), _ptr(mask),
+                              _stream(mask.device))
+    _check("kvq_sink_mask", st)
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, S: int) -> int:
+    return int(load().kvq_decode_workspace_bytes(B, Hq, Hkv, D, S))
+
+
+def decode_workspace(B: int, Hq: int, Hkv: int, D: int, S: int, device) -> torch.Tensor:
+    """A zero-filled workspace of the size kvq_decode_attn needs."""
+    n = decode_workspace_bytes(B, Hq, Hkv, D, S)
+    if n == 0:
+        raise ValueError("unsupported decode configuration")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word):
+    _cuda("q", q, torch.bfloat16)
+    for n, t in (("k", k), ("k_zp", k_zp), ("v", v), ("v_zp", v_zp)):
+        _cuda(n, t, torch.int8)
+    _cuda("k_scale", k_scale, torch.float32)
+    _cuda("v_scale", v_scale, torch.float32)
+    _cuda("kv_len", kv_len, torch.int32)
+    _cuda("mask", mask, torch.float32)
+    _cuda("out", out, torch.bfloat16)
+    _cuda("err_word", err_word, torch.int32)
+    if k.dim() != 4 or q.dim() != 4:
+        raise ValueError("q must be [B, Hq, Lq, D] and k/v [B, Hkv, S, D]")
+
+
+def decode_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,
+                workspace=None, err_word=None) -> torch.Tensor:
+    """kvq_decode_attn: q [B, Hq, 1, D] bf16 over the int8 cache [B, Hkv, S, D]."""
+    if out is None:
+        out = torch.empty_like(q)
+    _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if Lq != 1:
+        raise ValueError("decode takes one query row (use prefill_attn)")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, D, S, q.device)
+    st = load().kvq_decode_attn(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
+                                _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
+                                _stream(q.device))
+    _check("kvq_decode_attn", st)
+    return out
+
+
+def prefill_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, is_causal=False,
+                 mask_is_causal=False, sm_scale=None, err_word=None) -> torch.Tensor:
+    """kvq_prefill_attn: q [B, Hq, Lq, D] bf16 (rows at positions kv_len - Lq + i)."""
+    if out is None:
+        out = torch.empty_like(q)
+    _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    st = load().kvq_prefill_attn(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                 _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), int(bool(is_causal)),
+                                 int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
+                                 _stream(q.device))
+    _check("kvq_prefill_attn", st)
+    return out

@@ -1,0 +1,71 @@
+"""The C-ABI library loads and exports every entry point include/kvq.h declares
+(CPU only: no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_kv_cache_20_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = kbuild.build()
+    import torch  # noqa: F401  (loads the shared CUDA runtime first, as the binding does)
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("kvq_write", "kvq_decode_attn", "kvq_prefill_attn", "kvq_sink_plan", "kvq_sink_mask",
+              "kvq_decode_workspace_bytes", "kvq_strerror", "kvq_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_declares_the_same_symbols():
+    from quantized_kv_cache_20_b200 import kvq
+    assert sorted(kvq.EXPORTS) == _declared()
+
+
+def test_host_only_calls(lib):
+    lib.kvq_strerror.restype = ctypes.c_char_p
+    assert lib.kvq_strerror(0) == b"ok"
+    assert b"invalid" in lib.kvq_strerror(-1)
+    assert lib.kvq_version() >= 100
+
+
+def test_argument_checks_reject_before_any_launch(lib):
+    P = ctypes.c_void_p
+    lib.kvq_write.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_int, P, P, ctypes.c_int64, P, P, P, P, P]
+    strides = (ctypes.c_int64 * 4)(8, 8, 8, 1)
+    fake = P(16)
+    # unknown mode
+    assert lib.kvq_write(9, 1, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
+    # int8 mode needs D in {64, 128, 256}
+    assert lib.kvq_write(0, 1, fake, 1, 1, 1, 96, strides, fake, 8, fake, fake, fake, None, None) == -2
+    # block modes need d % 32 == 0 and d <= 8192
+    assert lib.kvq_write(1, 1, fake, 1, 1, 1, 48, strides, fake, 8, fake, fake, None, None, None) == -2
+    assert lib.kvq_write(1, 1, fake, 1, 1, 1, 8224, strides, fake, 8, fake, fake, None, None, None) == -2
+    # MX-FP8 without round_scale is not built
+    assert lib.kvq_write(2, 0, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, None, None, None) == -2
+    # null x
+    assert lib.kvq_write(0, 1, None, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
+    # misaligned x
+    assert lib.kvq_write(0, 1, P(18), 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
+    # empty work is a no-op
+    assert lib.kvq_write(0, 1, fake, 0, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == 0

@@ -1,0 +1,293 @@
+"""GPU parity of kvq_decode_attn / kvq_prefill_attn against the fp64 oracle:
+|gpu - oracle| <= 2e-3 + 1e-2 |oracle| element by element, plus the
+bit-identities the pages fix (per-tile causal skip on/off, kv_len = S)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_kv_cache_20_b200 import kvq
+from quantized_kv_cache_20_b200 import workloads as wl
+from tests.helpers import DEV, assert_attn_close, bf16_to_f64, err_word, int32_scalar
+
+pytestmark = pytest.mark.gpu
+
+
+def _cache(B, Hkv, S, D, g):
+    K = wl.int8_cache_like(B, Hkv, S, D, g)
+    V = wl.int8_cache_like(B, Hkv, S, D, g)
+    return K, V
+
+
+def _np(c):
+    return [t.numpy() for t in c]
+
+
+def _decode_gpu(q, K, V, kv_len, mask=None, sm=None, err=None):
+    Kd = [t.to(DEV) for t in K]
+    Vd = [t.to(DEV) for t in V]
+    out = kvq.decode_attn(q.to(DEV), *Kd, *Vd, int32_scalar(kv_len) if isinstance(kv_len, int) else kv_len,
+                          mask=None if mask is None else mask.to(DEV), sm_scale=sm, err_word=err)
+    torch.cuda.synchronize()
+    return out
+
+
+# ---------------------------------------------------------------------------- decode
+
+def test_tiny_write_then_decode():
+    """16 tokens x 2 kv heads, D=64, written at random slots of a 64-slot cache;
+    4 q heads (GQA 2:1) attend at kv_len 40.  The oracle writes its own cache."""
+    w = wl.TINY
+    g = wl.generator(w.seed)
+    k = wl.bf16_normal((w.B, w.Hkv, w.T, w.D), g)
+    v = wl.bf16_normal((w.B, w.Hkv, w.T, w.D), g)
+    sm = wl.slot_mapping_random(w.T, w.S, 3, g)
+    K0 = wl.int8_cache_like(w.B, w.Hkv, w.S, w.D, g)
+    V0 = wl.int8_cache_like(w.B, w.Hkv, w.S, w.D, g)
+    q = wl.bf16_normal((w.B, w.Hq, 1, w.D), g)
+    Kd = [t.to(DEV) for t in K0]
+    Vd = [t.to(DEV) for t in V0]
+    kvq.write(0, k.to(DEV), sm.to(DEV), *Kd)
+    kvq.write(0, v.to(DEV), sm.to(DEV), *Vd)
+    out = kvq.decode_attn(q.to(DEV), *Kd, *Vd, int32_scalar(w.kv_len))
+    Ko = [t.numpy().copy() for t in K0]
+    Vo = [t.numpy().copy() for t in V0]
+    oracle.write(0, wl.u16(k), sm.numpy(), w.S, *Ko)
+    oracle.write(0, wl.u16(v), sm.numpy(), w.S, *Vo)
+    ref = oracle.sdpa(wl.u16(q), *Ko, *Vo, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D))
+    assert_attn_close(bf16_to_f64(out), ref, "tiny")
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (6, 2), (8, 2), (16, 2), (10, 2)])
+@pytest.mark.parametrize("kv_len", [1, 37, 200, 512])
+def test_decode_shapes(D, Hq, Hkv, kv_len):
+    g = wl.generator(D * 7 + Hq * 3 + kv_len)
+    B, S = 2, 512
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    out = _decode_gpu(q, K, V, kv_len)
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=1 / math.sqrt(D))
+    assert_attn_close(bf16_to_f64(out), ref, f"D={D} Hq={Hq} Hkv={Hkv} kv={kv_len}")
+
+
+def test_decode_with_additive_mask():
+    g = wl.generator(77)
+    B, Hq, Hkv, D, S = 1, 8, 2, 128, 256
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    rng = np.random.default_rng(1)
+    m = np.where(rng.random(S) < 0.4, -np.inf, rng.normal(size=S) * 2).astype(np.float32)
+    m[5] = 0.0
+    mask = torch.from_numpy(m).reshape(1, S)
+    out = _decode_gpu(q, K, V, 230, mask=mask)
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=230, sm_scale=1 / math.sqrt(D), mask=m.reshape(1, S))
+    assert_attn_close(bf16_to_f64(out), ref, "mask")
+
+
+def test_decode_config_full_size():
+    """batch 8, 32 q / 8 kv heads, D=128, 8192 slots, kv_len 4096 read on device."""
+    w = wl.DECODE
+    g = wl.generator(w.seed)
+    K, V = _cache(w.B, w.Hkv, w.S, w.D, g)
+    q = wl.bf16_normal((w.B, w.Hq, 1, w.D), g)
+    out = _decode_gpu(q, K, V, w.kv_len)
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D))
+    assert_attn_close(bf16_to_f64(out), ref, "decode config")
+
+
+def test_long_config_decode_full_size():
+    """batch 1, 32 q / 16 kv heads, D=256, kv_len = 131072 (the whole cache)."""
+    w = wl.LONG
+    g = wl.generator(w.seed + 100)
+    K, V = _cache(w.B, w.Hkv, w.S, w.D, g)
+    q = wl.bf16_normal((w.B, w.Hq, 1, w.D), g)
+    out = _decode_gpu(q, K, V, w.kv_len)
+    rows = [(0, h, 0) for h in range(w.Hq)]
+    ref = oracle.sdpa_rows(wl.u16(q), *_np(K), *_np(V), kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D), rows=rows)
+    assert_attn_close(bf16_to_f64(out)[0, :, 0], ref, "long decode")
+
+
+def test_sink_config_decode_steps():
+    """4 sink + 2044 ring slots: plan -> write K/V -> mask -> decode, checked at
+    positions around the wrap; the oracle keeps its own cache and plan."""
+    w = wl.SINK
+    g = wl.generator(w.seed)
+    S, D = w.S, w.D
+    K0 = wl.int8_cache_random(1, w.Hkv, S, D, g)
+    V0 = wl.int8_cache_random(1, w.Hkv, S, D, g)
+    Kd = [t.to(DEV) for t in K0]
+    Vd = [t.to(DEV) for t in V0]
+    Ko = [t.numpy().copy() for t in K0]
+    Vo = [t.numpy().copy() for t in V0]
+    sp_d = torch.full((S,), -1, dtype=torch.int32, device=DEV)
+    sp_o = np.full(S, -1, np.int32)
+    ip = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sm_d = torch.empty(1, dtype=torch.int32, device=DEV)
+    kv_d = torch.empty(1, dtype=torch.int32, device=DEV)
+    mask_d = torch.empty((1, S), dtype=torch.float32, device=DEV)
+    ws = kvq.decode_workspace(1, w.Hq, w.Hkv, D, S, DEV)
+    checks = {0, 3, 4, 5, 2047, 2048, 2049, 2300, 4095, 4096}
+    last = max(checks)
+    gen = wl.generator(w.seed + 1)
+    for p in range(last + 1):
+        k = wl.bf16_normal((1, w.Hkv, 1, D), gen)
+        v = wl.bf16_normal((1, w.Hkv, 1, D), gen)
+        ip.fill_(p)
+        kvq.sink_plan(ip, 1, 1, w.sink, sp_d, sm_d, kv_d)
+        kvq.write(0, k.to(DEV), sm_d, *Kd)
+        kvq.write(0, v.to(DEV), sm_d, *Vd)
+        sm_o, kv_o = oracle.sink_plan(p, 1, 1, w.sink, S, sp_o)
+        oracle.write(0, wl.u16(k), sm_o, S, *Ko)
+        oracle.write(0, wl.u16(v), sm_o, S, *Vo)
+        if p in checks:
+            q = wl.bf16_normal((1, w.Hq, 1, D), gen)
+            kvq.sink_mask(ip, 1, sp_d, mask_d)
+            out = kvq.decode_attn(q.to(DEV), *Kd, *Vd, kv_d, mask=mask_d, workspace=ws)
+            mask_o = oracle.sink_mask(p, 1, sp_o)
+            ref = oracle.sdpa(wl.u16(q), *Ko, *Vo, kv_len=kv_o, sm_scale=1 / math.sqrt(D), mask=mask_o)
+            assert_attn_close(bf16_to_f64(out), ref, f"sink decode p={p}")
+
+
+def test_kv_len_is_read_on_device_each_call():
+    g = wl.generator(91)
+    B, Hq, Hkv, D, S = 1, 4, 1, 128, 1024
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g).to(DEV)
+    Kd = [t.to(DEV) for t in K]
+    Vd = [t.to(DEV) for t in V]
+    kv = int32_scalar(1)
+    ws = kvq.decode_workspace(B, Hq, Hkv, D, S, DEV)
+    for n in (1, 100, 1024, 513):
+        kv.fill_(n)  # only device memory changes; the launch arguments do not
+        out = kvq.decode_attn(q, *Kd, *Vd, kv, workspace=ws)
+        ref = oracle.sdpa(wl.u16(q.cpu()), *_np(K), *_np(V), kv_len=n, sm_scale=1 / math.sqrt(D))
+        assert_attn_close(bf16_to_f64(out), ref, f"kv_len {n}")
+    # the split counters are back at zero after every call
+    nc = B * Hkv
+    assert torch.all(ws[: nc * 4].view(torch.int32) == 0)
+
+
+def test_kv_len_full_equals_bound_at_s_and_out_of_range_is_clamped():
+    g = wl.generator(92)
+    B, Hq, Hkv, D, S = 2, 8, 2, 64, 256
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    a = _decode_gpu(q, K, V, S)
+    err = err_word()
+    b = _decode_gpu(q, K, V, S + 50, err=err)
+    assert torch.equal(a, b)
+    assert err.item() & kvq.KVQ_ERR_KV_LEN_RANGE
+    err2 = err_word()
+    z = _decode_gpu(q, K, V, -5, err=err2)
+    assert err2.item() & kvq.KVQ_ERR_KV_LEN_RANGE
+    assert torch.all(z == 0)
+
+
+def test_decode_is_deterministic():
+    g = wl.generator(93)
+    B, Hq, Hkv, D, S = 4, 16, 4, 128, 2048
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    a = _decode_gpu(q, K, V, 2000)
+    b = _decode_gpu(q, K, V, 2000)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------- prefill
+
+def _prefill_gpu(q, K, V, kv_len, **kw):
+    Kd = [t.to(DEV) for t in K]
+    Vd = [t.to(DEV) for t in V]
+    if "mask" in kw and kw["mask"] is not None:
+        kw["mask"] = kw["mask"].to(DEV)
+    out = kvq.prefill_attn(q.to(DEV), *Kd, *Vd, int32_scalar(kv_len), **kw)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (4, 4), (6, 3)])
+@pytest.mark.parametrize("Lq,kv_len", [(1, 50), (5, 50), (33, 160), (128, 128), (70, 300)])
+def test_prefill_causal_shapes(D, Hq, Hkv, Lq, kv_len):
+    g = wl.generator(D + Hq * 11 + Lq * 13 + kv_len)
+    B, S = 2, 320
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, Lq, D), g)
+    out = _prefill_gpu(q, K, V, kv_len, is_causal=True, mask_is_causal=True)
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=1 / math.sqrt(D), is_causal=True)
+    assert_attn_close(bf16_to_f64(out), ref, f"prefill D={D} G={Hq // Hkv} Lq={Lq} kv={kv_len}")
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_prefill_tile_skip_is_bit_identical(D):
+    g = wl.generator(500 + D)
+    B, Hq, Hkv, S, Lq, kv_len = 1, 8, 2, 640, 200, 600
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, Lq, D), g)
+    a = _prefill_gpu(q, K, V, kv_len, is_causal=True, mask_is_causal=False)
+    b = _prefill_gpu(q, K, V, kv_len, is_causal=True, mask_is_causal=True)
+    assert torch.equal(a, b)
+    # and at Lq = 1 the bound is the whole kv_len: prefill equals decode bit for bit
+    q1 = wl.bf16_normal((B, Hq, 1, D), g)
+    c = _prefill_gpu(q1, K, V, kv_len, is_causal=True, mask_is_causal=True)
+    d = _prefill_gpu(q1, K, V, kv_len, is_causal=False, mask_is_causal=False)
+    assert torch.equal(c, d)
+
+
+def test_sink_config_prefill_chunks():
+    """128-token chunks through the 4 + 2044 ring, checked on chunks that span
+    positions 2048 and 4096 (masked attention, no causal flag)."""
+    w = wl.SINK
+    g = wl.generator(w.seed + 7)
+    S, D, Lq = w.S, w.D, w.Lq
+    K0 = wl.int8_cache_random(1, w.Hkv, S, D, g)
+    V0 = wl.int8_cache_random(1, w.Hkv, S, D, g)
+    Kd = [t.to(DEV) for t in K0]
+    Vd = [t.to(DEV) for t in V0]
+    Ko = [t.numpy().copy() for t in K0]
+    Vo = [t.numpy().copy() for t in V0]
+    sp_d = torch.full((S,), -1, dtype=torch.int32, device=DEV)
+    sp_o = np.full(S, -1, np.int32)
+    ip = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sm_d = torch.empty(Lq, dtype=torch.int32, device=DEV)
+    kv_d = torch.empty(1, dtype=torch.int32, device=DEV)
+    mask_d = torch.empty((Lq, S), dtype=torch.float32, device=DEV)
+    for c in range(33):
+        p = c * Lq
+        k = wl.bf16_normal((1, w.Hkv, Lq, D), g)
+        v = wl.bf16_normal((1, w.Hkv, Lq, D), g)
+        ip.fill_(p)
+        kvq.sink_plan(ip, 1, Lq, w.sink, sp_d, sm_d, kv_d)
+        kvq.write(0, k.to(DEV), sm_d, *Kd)
+        kvq.write(0, v.to(DEV), sm_d, *Vd)
+        sm_o, kv_o = oracle.sink_plan(p, 1, Lq, w.sink, S, sp_o)
+        oracle.write(0, wl.u16(k), sm_o, S, *Ko)
+        oracle.write(0, wl.u16(v), sm_o, S, *Vo)
+        if p <= 2048 < p + Lq or p <= 4096 < p + Lq or c == 3:
+            q = wl.bf16_normal((1, w.Hq, Lq, D), g)
+            kvq.sink_mask(ip, Lq, sp_d, mask_d)
+            out = kvq.prefill_attn(q.to(DEV), *Kd, *Vd, kv_d, mask=mask_d)
+            mask_o = oracle.sink_mask(p, Lq, sp_o)
+            rows = [(0, h, i) for h in (0, 5, 31) for i in range(0, Lq, 9)] + [(0, 17, Lq - 1)]
+            ref = oracle.sdpa_rows(wl.u16(q), *Ko, *Vo, kv_len=kv_o, sm_scale=1 / math.sqrt(D), rows=rows,
+                                   mask=mask_o)
+            got = bf16_to_f64(out)
+            assert_attn_close(np.stack([got[b, h, i] for b, h, i in rows]), ref, f"sink prefill p={p}")
+
+
+def test_long_config_prefill_sampled_rows():
+    """Lq = 2048 causal chunk at kv_len 131072 (32 q / 16 kv heads, D=256),
+    checked on sampled rows: the first and last row of several 128-row tiles."""
+    w = wl.LONG
+    g = wl.generator(w.seed + 200)
+    K, V = _cache(w.B, w.Hkv, w.S, w.D, g)
+    q = wl.bf16_normal((w.B, w.Hq, w.Lq, w.D), g)
+    out = _prefill_gpu(q, K, V, w.kv_len, is_causal=True, mask_is_causal=True)
+    rows = [(0, 0, 0), (0, 1, 127), (0, 7, 128), (0, 16, 1023), (0, 30, 1920), (0, 31, 2047)]
+    ref = oracle.sdpa_rows(wl.u16(q), *_np(K), *_np(V), kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D),
+                           rows=rows, is_causal=True)
+    got = bf16_to_f64(out)
+    assert_attn_close(np.stack([got[b, h, i] for b, h, i in rows]), ref, "long prefill")
