@@ -41,12 +41,14 @@ FALLBACK_HBM_GBS = 6650.0
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=65536)
+    ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--kernel", choices=["decode", "fill", "block1", "block2", "block3", "long_decode"],
+                    help="profiling aid: launch only this kernel on its workload --steps times, print nothing")
     return ap.parse_args()
 
 
@@ -277,27 +279,34 @@ def run_kvq(args, dist: Dist):
         K, V = layers[l]
         kvq.decode_attn(q, *K, *V, kv_len, out=out, workspace=ws)
 
-    # warm the launch path once outside capture, then capture one graph per layer
+    # warm the launch path once outside capture, then capture one graph per rotation
+    # (NL steps, one per layer) and one of decode launches alone
     with torch.cuda.stream(stream):
         for l in range(NL):
             step(l)
     torch.cuda.synchronize()
-    step_graphs, dec_graphs = [], []
+    rot_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(rot_graph, stream=stream):
+        for l in range(NL):
+            step(l)
+    dec_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(dec_graph, stream=stream):
+        for l in range(NL):
+            decode_only(l)
+    step_graphs = []
     for l in range(NL):
         gph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gph, stream=stream):
             step(l)
         step_graphs.append(gph)
-        gd = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gd, stream=stream):
-            decode_only(l)
-        dec_graphs.append(gd)
     torch.cuda.synchronize()
 
-    # ---- headline: K steps
+    # ---- headline: exactly K steps (whole rotations, then single steps)
+    reps, rem = divmod(args.steps, NL)
+    nsteps = args.steps
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step_graphs[i % NL].replay()
+        for i in range(max(1, (args.warmup + NL - 1) // NL)):
+            rot_graph.replay()
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
@@ -306,28 +315,28 @@ def run_kvq(args, dist: Dist):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(args.steps):
-            step_graphs[i % NL].replay()
+        for i in range(reps):
+            rot_graph.replay()
+        for l in range(rem):
+            step_graphs[l].replay()
         e1.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
     clk = clocks.stop()
-    ms_local = e0.elapsed_time(e1) / args.steps
+    ms_local = e0.elapsed_time(e1) / nsteps
     ms = dist.max(ms_local)
     value = dist.world * B / (ms / 1000.0)
 
     # ---- dominant kernel: decode attention alone, same rotation, events on its stream
-    reps = max(1, args.steps // NL)
+    dreps = max(4, reps // 4)
     with torch.cuda.stream(stream):
-        for l in range(NL):
-            dec_graphs[l].replay()
+        dec_graph.replay()
         e0.record(stream)
-        for r in range(reps):
-            for l in range(NL):
-                dec_graphs[l].replay()
+        for r in range(dreps):
+            dec_graph.replay()
         e1.record(stream)
     torch.cuda.synchronize()
-    dec_ms = e0.elapsed_time(e1) / (reps * NL)
+    dec_ms = e0.elapsed_time(e1) / (dreps * NL)
     dec_bytes = 2 * B * Hkv * KV * (D + 4 + 1) + 2 * (B * Hq * D * 2)
     peak, peak_kind = _peaks()
     achieved = dec_bytes / (dec_ms / 1000.0) / 1e9
@@ -347,7 +356,7 @@ def run_kvq(args, dist: Dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk, "detail": detail,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * nsteps, "clocks": clk, "detail": detail,
     }
     if dist.rank == 0 and dist.world == 1:
         steps_c, el_c = _oracle_decode_steps(args.cpu_seconds)
@@ -357,8 +366,7 @@ def run_kvq(args, dist: Dist):
                       f"256 attention rows at kv_len 4096), single-threaded C oracle, {el_c:.1f} s"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
-    for gph in step_graphs + dec_graphs:
-        del gph
+    del rot_graph, dec_graph, step_graphs
     dist.close()
 
 
@@ -369,7 +377,7 @@ def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
     B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
     dev = dist.device
     NL = len(layers)
-    steps = max(NL, min(args.steps, 200))
+    steps = max(NL, min(args.steps, 2000))
     g = torch.Generator().manual_seed(7)
     hq = torch.randn((B, Hq, 1, D), generator=g).to(torch.bfloat16).pin_memory()
     hk = torch.randn((B, Hkv, 1, D), generator=g).to(torch.bfloat16).pin_memory()
@@ -509,8 +517,56 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
     return res
 
 
+def run_kernel(args):
+    """Launch one kernel on its workload --steps times (for ncu); no timing, no output."""
+    import torch
+    from quantized_kv_cache_20_b200 import build as kbuild
+    from quantized_kv_cache_20_b200 import kvq
+    from quantized_kv_cache_20_b200 import workloads as wl
+    kbuild.build()
+    kvq.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    if args.kernel in ("decode", "fill", "long_decode"):
+        w = wl.LONG if args.kernel == "long_decode" else wl.DECODE
+        B, Hq, Hkv, D, S, KV = w.B, w.Hq, w.Hkv, w.D, w.S, w.kv_len
+        K = (torch.randint(-128, 128, (B, Hkv, S, D), dtype=torch.int8, device=dev),
+             torch.rand((B, Hkv, S), device=dev) * 0.012 + 0.018,
+             torch.randint(-6, 7, (B, Hkv, S), dtype=torch.int8, device=dev))
+        V = tuple(t.clone() for t in K)
+        if args.kernel == "fill":
+            x = torch.randn((B, Hkv, KV - 1, D), generator=g, device=dev).to(torch.bfloat16)
+            sm = torch.arange(KV - 1, dtype=torch.int32, device=dev).repeat(B)
+            for _ in range(args.steps):
+                kvq.write(0, x, sm, *K)
+        else:
+            q = torch.randn((B, Hq, 1, D), generator=g, device=dev).to(torch.bfloat16)
+            kv = torch.tensor([KV], dtype=torch.int32, device=dev)
+            ws = kvq.decode_workspace(B, Hq, Hkv, D, S, dev)
+            out = torch.empty_like(q)
+            for _ in range(args.steps):
+                kvq.decode_attn(q, *K, *V, kv, out=out, workspace=ws)
+    else:
+        mode = int(args.kernel[-1])
+        bw = wl.BLOCK
+        x = torch.randn((1, 1, bw.tokens, bw.d), generator=g, device=dev).to(torch.bfloat16)
+        sm = torch.randperm(bw.num_slots, generator=g, device=dev)[: bw.tokens].to(torch.int32)
+        sm[torch.randperm(bw.tokens, generator=g, device=dev)[: int(bw.tokens * bw.skip_frac)]] = -1
+        c = torch.zeros((1, 1, bw.num_slots, bw.d // 2 if mode == 3 else bw.d), dtype=torch.uint8, device=dev)
+        s = torch.zeros((1, 1, bw.num_slots, bw.d // 32), dtype=torch.float32 if mode == 1 else torch.uint8,
+                        device=dev)
+        for _ in range(args.steps):
+            kvq.write(mode, x, sm, c, s)
+    torch.cuda.synchronize()
+
+
 def main():
     args = _args()
+    if args.kernel:
+        run_kernel(args)
+        return
     dist = Dist(args.gpus)
     if args.impl == "reference":
         run_reference(args, dist)

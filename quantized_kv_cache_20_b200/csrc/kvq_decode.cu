@@ -6,26 +6,39 @@
 //   out[b,h] = softmax_j(sm_scale * q[b,h] . K[b,hk,j] + mask[j]) . V[b,hk,j],
 //   j in [0, kv_len), hk = h / G, K = (k - k_zp) * k_scale, V likewise.
 //
-// Design (HBM-bound; B200 sm_100a):
-//  - Grid (split * head_chunks, Hkv, B).  Each CTA streams a contiguous slot
-//    range of one (b, kv head) and serves HC query heads of its GQA group, so
-//    every K/V byte is read once for all of them.  The split length is derived
-//    on the device from *kv_len (no host sync, graph-replayable).
-//  - One producer warp issues 1-D bulk async copies (TMA, cp.async.bulk) of
-//    K/V code tiles, scales, zero points and mask into an NST-stage ring of
-//    shared memory, synchronised by mbarriers (full: tx bytes; empty: one
-//    arrival per consumer warp).  Every wait is bounded.
-//  - NW consumer warps each own 32 slots of a tile.  A lane owns 16 dims
-//    (16 code bytes = one 128-bit shared load) of L = D/16 slots in turn; the
-//    codes become exact floats (c - zp) through a byte-permute into the
-//    mantissa of 2^23 and one packed subtract, and q.k runs on packed fp32 FMA
-//    (fma.rn.f32x2).  A butterfly reduce-scatter across the L lanes leaves each
-//    lane with the full dot products of one slot, so the online-softmax state
-//    is per lane-group and PV reuses the same lane/dim ownership.
-//  - The CTA combines its groups in a fixed order; split partials go to the
-//    workspace and the last CTA of a (b, kv head, head chunk) to finish (an
-//    atomic counter it then resets) merges them in split order.  No atomics
-//    touch the output, so results are deterministic.
+// Design (B200, sm_100a).  Decode is HBM-bound in bytes but, with GQA, heavy in
+// CUDA-core instructions per byte, so the kernel is built to keep the issue
+// slots busy:
+//  - Persistent grid: one CTA per SM.  The work -- units (b, kv head, head
+//    chunk) x tiles of TS slots, with the tile count derived on the device from
+//    *kv_len -- is flattened and cut into equal contiguous ranges, one per CTA,
+//    so every SM streams the same number of bytes whatever B, Hkv and kv_len
+//    are.  A CTA closes a segment whenever its range moves to the next unit.
+//  - One producer warp issues 1-D bulk async copies (TMA) of the K/V code
+//    tiles, scales, zero points, mask and (on a unit's first tile) the q rows
+//    into an NST-stage shared-memory ring (mbarrier tx counts; one arrival per
+//    consumer warp frees a stage).  Every wait is bounded.
+//  - NW consumer warps each take 32 slots of a tile.  A lane owns 16 dims of
+//    L = D/16 slots in turn.
+//      q.k: q is rounded once per segment onto a 16-bit fixed-point grid
+//      (n = rne(q * sm_scale * log2e / 2^E), |n| <= 32767, a power-of-two
+//      step per head), so the dot product with the int8 codes is exact integer
+//      arithmetic on dp4a (high and low bytes of n); the zero point enters as
+//      - zp * sum(n).  The only rounding is q's: |error| <= 2^(E-1) per element,
+//      i.e. below 2^-15 of max|q| -- far below bf16's own resolution of q.
+//      A butterfly reduce-scatter across the L lanes leaves each lane with the
+//      full dot products of one slot.
+//      softmax: online, per lane group, in the log2 domain, with the running
+//      maximum only raised when a new score exceeds it by more than 8 (the
+//      accumulators then hold values up to 2^8 times larger, harmless in fp32).
+//      p.v: the V codes become exact floats (c - zp) through a byte permute into
+//      the mantissa of 2^23 and one packed subtract; p*v_scale is broadcast per
+//      slot through shared memory and accumulated with packed fp32 FMA.
+//  - Segment close: groups merge by shuffles, warps through shared memory, in
+//    a fixed order.  A unit that a CTA covers alone is written directly; a
+//    unit split across CTAs leaves one partial per CTA in the workspace and the
+//    last CTA to finish it (atomic counter, reset afterwards) merges them in
+//    CTA order.  No atomics touch the output: results are deterministic.
 #include <cuda_bf16.h>
 
 #include "kvq_common.cuh"
@@ -34,6 +47,7 @@ namespace kvq {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p kept without rescaling
 
 struct DecodeArgs {
   const uint16_t *q;
@@ -46,22 +60,22 @@ struct DecodeArgs {
   const float *mask;
   const int32_t *kv_len;
   uint16_t *out;
-  float *ws_ml;  // [B, Hkv, nsplit, G, 2]
-  float *ws_o;   // [B, Hkv, nsplit, G, D]
-  int32_t *counters;  // [B, Hkv, nhc]
+  float *ws_ml;       // [C * smax][HC][2]
+  float *ws_o;        // [C * smax][HC][D]
+  int32_t *counters;  // [U]
   int32_t *err;
   int64_t S;
-  int B, Hq, Hkv, G, nsplit, nhc;
+  int B, Hq, Hkv, G, nhc, smax;
   float qscale;  // sm_scale * log2(e)
 };
 
 template <int D_, int HC_, int NW_, int NST_>
 struct Cfg {
   static constexpr int D = D_, HC = HC_, NW = NW_, NST = NST_;
-  static constexpr int DPL = 16;       // dims per lane
-  static constexpr int L = D / DPL;    // lanes per slot group
+  static constexpr int L = D / 16;     // lanes per slot group (16 dims per lane)
   static constexpr int NG = 32 / L;    // slot groups per warp
   static constexpr int TS = 32 * NW;   // slots per tile
+  // one ring stage
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = TS * D;
   static constexpr int KS_OFF = 2 * TS * D;
@@ -69,29 +83,68 @@ struct Cfg {
   static constexpr int M_OFF = VS_OFF + 4 * TS;
   static constexpr int KZ_OFF = M_OFF + 4 * TS;
   static constexpr int VZ_OFF = KZ_OFF + TS;
-  static constexpr int STAGE = VZ_OFF + TS;
-  static constexpr int RING = NST * STAGE;
-  // combine scratch (reuses the ring once it is drained)
-  static constexpr int OBUF = NW * NG * HC * D * 4;
-  static constexpr int MLBUF = NW * NG * HC * 2 * 4;
-  static_assert(OBUF + MLBUF <= RING, "combine scratch must fit in the ring");
-  static constexpr int BAR_OFF = RING;
-  static constexpr int SMEM = RING + 2 * NST * 8 + 16;
+  static constexpr int Q_OFF = VZ_OFF + TS;
+  static constexpr int STAGE = Q_OFF + 2 * HC * D;
+  static_assert(STAGE % 16 == 0, "stage alignment");
+  // after the ring
+  static constexpr int WBUF_OFF = NST * STAGE;                 // [NW][32][4] float
+  static constexpr int OSCR_OFF = WBUF_OFF + NW * 32 * 16;     // [NW][HC][D] float
+  static constexpr int MLSCR_OFF = OSCR_OFF + NW * HC * D * 4; // [NW][HC][2] float
+  static constexpr int BAR_OFF = MLSCR_OFF + NW * HC * 8;
+  static constexpr int SH_OFF = BAR_OFF + 2 * NST * 8;
+  static constexpr int SMEM = SH_OFF + 16;
+  static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr int THREADS = (NW + 1) * 32;
 };
 
+KVQ_DEVINL int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+KVQ_DEVINL int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+KVQ_DEVINL float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+KVQ_DEVINL void consumer_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
+
+// Work split: CTA c owns flattened tiles [c*W/C, (c+1)*W/C).
+KVQ_DEVINL int64_t range_start(int64_t c, int64_t W, int64_t C) { return c * W / C; }
+KVQ_DEVINL int64_t cta_of(int64_t idx, int64_t W, int64_t C) { return ((idx + 1) * C - 1) / W; }
+// The CTA after c that owns a tile of [.., last], or -1: CTAs with empty ranges
+// (more CTAs than tiles) are skipped.
+KVQ_DEVINL int64_t next_owner(int64_t c, int64_t last, int64_t W, int64_t C) {
+  const int64_t e = range_start(c + 1, W, C);
+  return e > last ? -1 : cta_of(e, W, C);
+}
+
+KVQ_DEVINL bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
 template <class C>
-__global__ void __launch_bounds__(C::THREADS) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, HC = C::HC, NW = C::NW, NST = C::NST, L = C::L, NG = C::NG, TS = C::TS;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint64_t *empty = full + NST;
-  int32_t *sh = reinterpret_cast<int32_t *>(empty + NST);  // [0] kv_len, [1] abort, [2] last
+  volatile int32_t *sh = reinterpret_cast<volatile int32_t *>(smem + C::SH_OFF);  // kv, abort, last
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hc = blockIdx.x % a.nhc, split = blockIdx.x / a.nhc;
-  const int hk = blockIdx.y, b = blockIdx.z;
-
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
@@ -100,41 +153,62 @@ __global__ void __launch_bounds__(C::THREADS) decode_kernel(const DecodeArgs a) 
     fence_mbar_init();
     int kv = *a.kv_len;
     if (kv < 0 || kv > a.S) {
-      if (blockIdx.x == 0 && hk == 0 && b == 0) report(a.err, KVQ_ERR_KV_LEN_RANGE);
+      if (blockIdx.x == 0) report(a.err, KVQ_ERR_KV_LEN_RANGE);
       kv = kv < 0 ? 0 : static_cast<int>(a.S);
     }
     sh[0] = kv;
     sh[1] = 0;
+    sh[2] = 0;
   }
   __syncthreads();
 
   const int kv = sh[0];
-  int chunk = (kv + a.nsplit - 1) / a.nsplit;
-  chunk = (chunk + TS - 1) / TS * TS;
-  const int start = split * chunk;
-  const int end = min(kv, start + chunk);
-  const int ntiles = start < end ? (end - start + TS - 1) / TS : 0;
-  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+  const int ntiles = (kv + TS - 1) / TS;
+  const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
+  const int64_t CT = gridDim.x, cta = blockIdx.x;
 
-  // ---------------------------------------------------------------- producer
+  if (ntiles == 0) {  // nothing to attend to: every row is zero
+    for (int64_t u = cta; u < U; u += CT) {
+      const int hc = static_cast<int>(u % a.nhc);
+      const int64_t bhk = u / a.nhc;
+      const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+      for (int e = tid; e < HC * D; e += C::THREADS) {
+        const int hq = hk * a.G + hc * HC + e / D;
+        a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + e % D] = 0;
+      }
+    }
+    return;
+  }
+  const int64_t W = U * ntiles;
+  const int64_t t_begin = range_start(cta, W, CT), t_end = range_start(cta + 1, W, CT);
+
+  // ------------------------------------------------------------------ producer
   if (warp == NW) {
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % NST;
-        if (i >= NST && !mbar_wait_bounded(&empty[st], ((i / NST) - 1) & 1)) {
+      int64_t issued = 0;
+      int64_t u = t_begin / ntiles;
+      int t = static_cast<int>(t_begin - u * ntiles);
+      int st = 0;
+      uint32_t ephase = 0;  // parity of the empty-barrier phase to wait for at stage st
+      for (int64_t idx = t_begin; idx < t_end; ++idx) {
+        const int64_t i = idx - t_begin;
+        if (i >= NST && !wait_or_abort(&empty[st], ephase, sh + 1)) {
           report(a.err, KVQ_ERR_TIMEOUT);
           sh[1] = 1;
           break;
         }
-        const int s0 = start + i * TS;
-        const int n = min(TS, end - s0);
-        const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the (b, hk) slab
+        const int hc = static_cast<int>(u % a.nhc);
+        const int64_t bhk = u / a.nhc;  // = b * Hkv + hk
+        const int s0 = t * TS;
+        const int n = min(TS, kv - s0);
+        const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
+        const bool first = (t == 0) || (idx == t_begin);
         uint8_t *stage = smem + st * C::STAGE;
-        const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * D + 10) + (a.mask ? 4u * n16 : 0u);
+        const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * D + 10) + (a.mask ? 4u * n16 : 0u) +
+                               (first ? 2u * HC * D : 0u);
         mbar_arrive_expect_tx(&full[st], bytes);
-        const int64_t row = bh * a.S + s0;
+        const int64_t row = bhk * a.S + s0;
         bulk_g2s_hint(stage + C::K_OFF, a.k + row * D, n16 * D, &full[st], pol);
         bulk_g2s_hint(stage + C::V_OFF, a.v + row * D, n16 * D, &full[st], pol);
         bulk_g2s(stage + C::KS_OFF, a.ks + row, n16 * 4, &full[st]);
@@ -142,216 +216,334 @@ __global__ void __launch_bounds__(C::THREADS) decode_kernel(const DecodeArgs a) 
         bulk_g2s(stage + C::KZ_OFF, a.kz + row, n16, &full[st]);
         bulk_g2s(stage + C::VZ_OFF, a.vz + row, n16, &full[st]);
         if (a.mask) bulk_g2s(stage + C::M_OFF, a.mask + s0, n16 * 4, &full[st]);
+        if (first) {
+          const int64_t hk = bhk % a.Hkv, b = bhk / a.Hkv;
+          const int64_t q0 = (b * a.Hq + hk * a.G + static_cast<int64_t>(hc) * HC) * D;
+          bulk_g2s(stage + C::Q_OFF, a.q + q0, 2 * HC * D, &full[st]);
+        }
         issued = i + 1;
+        if (++t == ntiles) {
+          t = 0;
+          ++u;
+        }
+        if (++st == NST) {  // entering round r = (i+1)/NST waits for empty phase (r-1) & 1
+          st = 0;
+          if (i + 1 >= 2 * NST) ephase ^= 1u;
+        }
       }
-      // Drain: the last copy issued into each stage must have landed before
-      // shared memory is reused or the CTA exits.
-      for (int i = max(0, issued - NST); i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % NST], (i / NST) & 1)) report(a.err, KVQ_ERR_TIMEOUT);
+      // the last copy issued into each stage must land before the CTA exits
+      for (int64_t i = issued > NST ? issued - NST : 0; i < issued; ++i)
+        if (!mbar_wait_bounded(&full[i % NST], static_cast<uint32_t>(i / NST) & 1u)) report(a.err, KVQ_ERR_TIMEOUT);
     }
+    return;
   }
 
-  // ---------------------------------------------------------------- consumers
+  // ------------------------------------------------------------------ consumers
+  const int g = lane / L, sub = lane % L;
+  const int own = g + NG * sub;  // this lane's slot within the warp's 32 after the reduce-scatter
+  float *wbuf = reinterpret_cast<float *>(smem + C::WBUF_OFF) + warp * 32 * 4;
+
+  uint32_t qhi[HC][4], qlo[HC][4];
+  int nsum[HC];
+  float escale[HC];
   float m[HC], lsum[HC];
   float2 o2[HC][8];
-  const int g = lane / L, sub = lane % L;
-  if (warp < NW) {
-    float2 q2[HC][8];
+  int64_t cur_u = -1;
+  int seg = -1;
+
+  auto close_segment = [&](int64_t u, int sg) {
+    // (1) denominators over the lane group, then merge the NG groups of the warp
 #pragma unroll
     for (int h = 0; h < HC; ++h) {
-      const int hq = hk * a.G + hc * HC + h;
-      const uint16_t *qp = a.q + (static_cast<int64_t>(b) * a.Hq + hq) * D + sub * 16;
-      const uint4 c0 = *reinterpret_cast<const uint4 *>(qp);
-      const uint4 c1 = *reinterpret_cast<const uint4 *>(qp + 8);
-      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        q2[h][k] = make_float2(bf16lo(w[k]) * a.qscale, bf16hi(w[k]) * a.qscale);
-      m[h] = -INFINITY;
-      lsum[h] = 0.0f;
+      for (int o = L / 2; o >= 1; o >>= 1) lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o2[h][k] = make_float2(0.0f, 0.0f);
+      for (int o = L; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m[h], o);
+        const float lo = __shfl_xor_sync(0xffffffffu, lsum[h], o);
+        const float M = fmaxf(m[h], mo);
+        const float fs = m[h] == -INFINITY ? 0.0f : ex2(m[h] - M);
+        const float fo = mo == -INFINITY ? 0.0f : ex2(mo - M);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float2 oo = make_float2(__shfl_xor_sync(0xffffffffu, o2[h][k].x, o),
+                                        __shfl_xor_sync(0xffffffffu, o2[h][k].y, o));
+          o2[h][k] = __ffma2_rn(o2[h][k], make_float2(fs, fs), __fmul2_rn(oo, make_float2(fo, fo)));
+        }
+        lsum[h] = lsum[h] * fs + lo * fo;
+        m[h] = M;
+      }
+    }
+    // (2) group 0 of each warp publishes the warp's state
+    float *oscr = reinterpret_cast<float *>(smem + C::OSCR_OFF);
+    float *mlscr = reinterpret_cast<float *>(smem + C::MLSCR_OFF);
+    if (g == 0) {
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        float4 *dst = reinterpret_cast<float4 *>(oscr + (warp * HC + h) * D + sub * 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          dst[k] = make_float4(o2[h][2 * k].x, o2[h][2 * k].y, o2[h][2 * k + 1].x, o2[h][2 * k + 1].y);
+        if (sub == 0) {
+          mlscr[(warp * HC + h) * 2] = m[h];
+          mlscr[(warp * HC + h) * 2 + 1] = lsum[h];
+        }
+      }
+    }
+    consumer_sync(NW * 32);
+    // (3) merge the warps in order; write the output or this CTA's partial
+    const int64_t ntl = ntiles;
+    const int64_t c_first = cta_of(u * ntl, W, CT), c_last = cta_of(u * ntl + ntl - 1, W, CT);
+    const bool alone = c_first == c_last;
+    const int hc = static_cast<int>(u % a.nhc);
+    const int64_t bhk = u / a.nhc;
+    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    const int64_t rec = cta * a.smax + sg;
+    for (int e = tid; e < HC * D; e += NW * 32) {
+      const int h = e / D, d = e - h * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, mlscr[(w * HC + h) * 2]);
+      float Lt = 0.0f, O = 0.0f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float mw = mlscr[(w * HC + h) * 2];
+          const float f = mw == -INFINITY ? 0.0f : ex2(mw - M);
+          Lt = fmaf(f, mlscr[(w * HC + h) * 2 + 1], Lt);
+          O = fmaf(f, oscr[(w * HC + h) * D + d], O);
+        }
+      }
+      if (alone) {
+        const int hq = hk * a.G + hc * HC + h;
+        const float r = Lt > 0.0f ? O / Lt : 0.0f;
+        a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+      } else {
+        a.ws_o[(rec * HC + h) * D + d] = O;
+        if (d == 0) {
+          a.ws_ml[(rec * HC + h) * 2] = M;
+          a.ws_ml[(rec * HC + h) * 2 + 1] = Lt;
+        }
+      }
+    }
+    if (!alone) {
+      __threadfence();
+      consumer_sync(NW * 32);
+      const int64_t last_tile = u * ntl + ntl - 1;
+      if (tid == 0) {
+        int owners = 0;
+        for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) ++owners;
+        sh[2] = atomicAdd(a.counters + u, 1) == owners - 1;
+      }
+      consumer_sync(NW * 32);
+      if (sh[2]) {
+        __threadfence();
+        for (int e = tid; e < HC * D; e += NW * 32) {
+          const int h = e / D, d = e - h * D;
+          float M = -INFINITY;
+          for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
+            const int64_t r = c * a.smax + (u - range_start(c, W, CT) / ntl);
+            M = fmaxf(M, __ldcg(a.ws_ml + (r * HC + h) * 2));
+          }
+          float Lt = 0.0f, O = 0.0f;
+          if (M != -INFINITY) {
+            for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
+              const int64_t r = c * a.smax + (u - range_start(c, W, CT) / ntl);
+              const float mc = __ldcg(a.ws_ml + (r * HC + h) * 2);
+              if (mc == -INFINITY) continue;
+              const float f = ex2(mc - M);
+              Lt = fmaf(f, __ldcg(a.ws_ml + (r * HC + h) * 2 + 1), Lt);
+              O = fmaf(f, __ldcg(a.ws_o + (r * HC + h) * D + d), O);
+            }
+          }
+          const int hq = hk * a.G + hc * HC + h;
+          const float r = Lt > 0.0f ? O / Lt : 0.0f;
+          a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+        }
+        if (tid == 0) a.counters[u] = 0;  // ready for the next call
+      }
+    }
+    consumer_sync(NW * 32);  // scratch free for the next segment
+  };
+
+  int64_t u = t_begin / ntiles;
+  int t = static_cast<int>(t_begin - u * ntiles);
+  int st = 0;
+  uint32_t fphase = 0;
+  for (int64_t idx = t_begin; idx < t_end; ++idx) {
+    const bool ok = wait_or_abort(&full[st], fphase, sh + 1);
+    if (!ok && lane == 0) {
+      report(a.err, KVQ_ERR_TIMEOUT);
+      sh[1] = 1;
+    }
+    const uint8_t *stage = smem + st * C::STAGE;
+    if (u != cur_u) {
+      if (cur_u >= 0) close_segment(cur_u, seg);
+      cur_u = u;
+      ++seg;
+      // new unit: q (from this stage) onto the fixed-point grid, fresh softmax state
+      const uint16_t *qs = reinterpret_cast<const uint16_t *>(stage + C::Q_OFF);
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(qs + h * D + sub * 16);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(qs + h * D + sub * 16 + 8);
+        const uint32_t wq[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        float x[16];
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          x[2 * k] = bf16lo(wq[k]) * a.qscale;
+          x[2 * k + 1] = bf16hi(wq[k]) * a.qscale;
+          amax = fmaxf(amax, fmaxf(fabsf(x[2 * k]), fabsf(x[2 * k + 1])));
+        }
+#pragma unroll
+        for (int o = L / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        // step 2^E with amax / 2^E < 2^15: E = floor(log2 amax) + 1 - 15
+        int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1 - 15;
+        E = E < -126 ? -126 : E;
+        const float inv = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);  // 2^-E (E in [-126, 113])
+        escale[h] = __uint_as_float(static_cast<uint32_t>(127 + E) << 23);       // 2^E
+        int s = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t hw = 0, lw = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            int n = __float2int_rn(x[4 * k + j] * inv);
+            n = n > 32767 ? 32767 : (n < -32767 ? -32767 : n);
+            s += n;
+            hw |= (static_cast<uint32_t>(n >> 8) & 0xFFu) << (8 * j);
+            lw |= (static_cast<uint32_t>(n) & 0xFFu) << (8 * j);
+          }
+          qhi[h][k] = hw;
+          qlo[h][k] = lw;
+        }
+#pragma unroll
+        for (int o = L / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        nsum[h] = s;
+        m[h] = -INFINITY;
+        lsum[h] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o2[h][k] = make_float2(0.0f, 0.0f);
+      }
     }
 
-    for (int i = 0; i < ntiles; ++i) {
-      const int st = i % NST;
-      if (!mbar_wait_bounded(&full[st], (i / NST) & 1)) {
-        if (lane == 0) report(a.err, KVQ_ERR_TIMEOUT);
-        break;
-      }
-      const int s0 = start + i * TS;
-      const uint8_t *stage = smem + st * C::STAGE;
-      const int wbase = warp * 32;
-      if (s0 + wbase < end) {
-        // ---- q . k for the L slots of this lane group (slot = wbase + g + NG*jj)
-        float part[L][HC];
+    const int s0 = t * TS;
+    const int wbase = warp * 32;
+    if (ok && s0 + wbase < kv) {
+      // ---- q . k on dp4a for the L slots of this lane group (slot = wbase + g + NG*jj)
+      int part[L][HC];
 #pragma unroll
-        for (int jj = 0; jj < L; ++jj) {
-          const int sl = wbase + g + NG * jj;
-          const int zp = static_cast<int8_t>(stage[C::KZ_OFF + sl]);
-          const float mz = neg_magic_zp(zp);
-          const float2 mz2 = make_float2(mz, mz);
-          const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
-          float2 kv2[8];
-          codes4_to_f2(c.x, mz2, kv2[0], kv2[1]);
-          codes4_to_f2(c.y, mz2, kv2[2], kv2[3]);
-          codes4_to_f2(c.z, mz2, kv2[4], kv2[5]);
-          codes4_to_f2(c.w, mz2, kv2[6], kv2[7]);
-#pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            float2 acc = __fmul2_rn(q2[h][0], kv2[0]);
-#pragma unroll
-            for (int k = 1; k < 8; ++k) acc = __ffma2_rn(q2[h][k], kv2[k], acc);
-            part[jj][h] = acc.x + acc.y;
-          }
-        }
-        // ---- butterfly reduce-scatter: lane `sub` ends with slot jj = sub
-#pragma unroll
-        for (int o = L / 2; o >= 1; o >>= 1) {
-          const bool upper = (sub & o) != 0;
-#pragma unroll
-          for (int j = 0; j < o; ++j)
-#pragma unroll
-            for (int h = 0; h < HC; ++h) {
-              const float keep = upper ? part[j + o][h] : part[j][h];
-              const float send = upper ? part[j][h] : part[j + o][h];
-              part[j][h] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
-        }
-        // ---- scores (log2 domain) and online softmax per lane group
-        const int own = wbase + g + NG * sub;
-        const bool valid = s0 + own < end;
-        const float ksc = reinterpret_cast<const float *>(stage + C::KS_OFF)[own];
-        const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[own];
-        const float madd = a.mask ? reinterpret_cast<const float *>(stage + C::M_OFF)[own] * kLog2e : 0.0f;
-        float w[HC];
+      for (int jj = 0; jj < L; ++jj) {
+        const int sl = wbase + g + NG * jj;
+        const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
 #pragma unroll
         for (int h = 0; h < HC; ++h) {
-          const float s = valid ? fmaf(part[0][h], ksc, madd) : -INFINITY;
-          float mt = s;
-#pragma unroll
-          for (int o = L / 2; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-          const float mnew = fmaxf(m[h], mt);
-          const float muse = mnew == -INFINITY ? 0.0f : mnew;
-          const float alpha = exp2f(m[h] - muse);
-          const float p = exp2f(s - muse);
-          lsum[h] = fmaf(lsum[h], alpha, p);
-          m[h] = mnew;
-          const float2 al2 = make_float2(alpha, alpha);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) o2[h][k] = __fmul2_rn(o2[h][k], al2);
-          w[h] = p > 0.0f ? p * vsc : 0.0f;
+          int acc = dp4a_ss(qhi[h][0], c.x, 0);
+          acc = dp4a_ss(qhi[h][1], c.y, acc);
+          acc = dp4a_ss(qhi[h][2], c.z, acc);
+          acc = dp4a_ss(qhi[h][3], c.w, acc);
+          acc *= 256;
+          acc = dp4a_us(qlo[h][0], c.x, acc);
+          acc = dp4a_us(qlo[h][1], c.y, acc);
+          acc = dp4a_us(qlo[h][2], c.z, acc);
+          acc = dp4a_us(qlo[h][3], c.w, acc);
+          part[jj][h] = acc;
         }
-        // ---- p . v over the same L slots
+      }
+      // ---- butterfly reduce-scatter: lane `sub` ends with slot jj = sub
 #pragma unroll
-        for (int jj = 0; jj < L; ++jj) {
-          const int sl = wbase + g + NG * jj;
-          const int zp = static_cast<int8_t>(stage[C::VZ_OFF + sl]);
-          const float mz = neg_magic_zp(zp);
-          const float2 mz2 = make_float2(mz, mz);
-          const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + sl * D + sub * 16);
-          float2 vv2[8];
-          codes4_to_f2(c.x, mz2, vv2[0], vv2[1]);
-          codes4_to_f2(c.y, mz2, vv2[2], vv2[3]);
-          codes4_to_f2(c.z, mz2, vv2[4], vv2[5]);
-          codes4_to_f2(c.w, mz2, vv2[6], vv2[7]);
+      for (int o = L / 2; o >= 1; o >>= 1) {
+        const bool upper = (sub & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j)
 #pragma unroll
           for (int h = 0; h < HC; ++h) {
-            const float wj = __shfl_sync(0xffffffffu, w[h], g * L + jj);
-            const float2 w2 = make_float2(wj, wj);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) o2[h][k] = __ffma2_rn(w2, vv2[k], o2[h][k]);
+            const int keep = upper ? part[j + o][h] : part[j][h];
+            const int send = upper ? part[j][h] : part[j + o][h];
+            part[j][h] = keep + __shfl_xor_sync(0xffffffffu, send, o);
           }
+      }
+      // ---- scores (log2 domain) for this lane's slot
+      const int sl_own = wbase + own;
+      const bool valid = s0 + sl_own < kv;
+      const int kzp = static_cast<int8_t>(stage[C::KZ_OFF + sl_own]);
+      const float ksc = reinterpret_cast<const float *>(stage + C::KS_OFF)[sl_own];
+      const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[sl_own];
+      const float madd = a.mask ? reinterpret_cast<const float *>(stage + C::M_OFF)[sl_own] * kLog2e : 0.0f;
+      float sc[HC], mt[HC];
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        // exact: |sum n (c - zp)| < 2^31 for D <= 256 (computed modulo 2^32)
+        const int dz = static_cast<int>(static_cast<uint32_t>(part[0][h]) -
+                                        static_cast<uint32_t>(kzp) * static_cast<uint32_t>(nsum[h]));
+        sc[h] = valid ? fmaf(static_cast<float>(dz), escale[h] * ksc, madd) : -INFINITY;
+        mt[h] = sc[h];
+#pragma unroll
+        for (int o = L / 2; o >= 1; o >>= 1) mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
+        need |= mt[h] > m[h] + kRescaleThreshold;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          const float mnew = fmaxf(m[h], mt[h]);
+          if (mnew > m[h]) {
+            const float alpha = m[h] == -INFINITY ? 0.0f : ex2(m[h] - mnew);
+            lsum[h] *= alpha;
+            const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o2[h][k] = __fmul2_rn(o2[h][k], al2);
+            m[h] = mnew;
+          }
+        }
+      }
+      float wv[4];
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        const float p = sc[h] == -INFINITY ? 0.0f : ex2(sc[h] - m[h]);
+        lsum[h] += p;
+        wv[h] = p > 0.0f ? p * vsc : 0.0f;
+      }
+#pragma unroll
+      for (int h = HC; h < 4; ++h) wv[h] = 0.0f;
+      *reinterpret_cast<float4 *>(wbuf + own * 4) = make_float4(wv[0], wv[1], wv[2], wv[3]);
+      __syncwarp();
+      // ---- p . v over the same L slots
+#pragma unroll
+      for (int jj = 0; jj < L; ++jj) {
+        const int sl = g + NG * jj;
+        const float4 w4 = *reinterpret_cast<const float4 *>(wbuf + sl * 4);
+        const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
+        const int zp = static_cast<int8_t>(stage[C::VZ_OFF + wbase + sl]);
+        const float mz = neg_magic_zp(zp);
+        const float2 mz2 = make_float2(mz, mz);
+        const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + (wbase + sl) * D + sub * 16);
+        float2 vv2[8];
+        codes4_to_f2(c.x, mz2, vv2[0], vv2[1]);
+        codes4_to_f2(c.y, mz2, vv2[2], vv2[3]);
+        codes4_to_f2(c.z, mz2, vv2[4], vv2[5]);
+        codes4_to_f2(c.w, mz2, vv2[6], vv2[7]);
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          const float2 w2 = make_float2(wj[h], wj[h]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) o2[h][k] = __ffma2_rn(w2, vv2[k], o2[h][k]);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
     }
-    // per-group denominator
-#pragma unroll
-    for (int h = 0; h < HC; ++h)
-#pragma unroll
-      for (int o = L / 2; o >= 1; o >>= 1) lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
-  }
-  __syncthreads();  // ring drained (producer waited on every outstanding copy)
-
-  // ---------------------------------------------------------------- CTA combine
-  float *obuf = reinterpret_cast<float *>(smem);                     // [NW*NG][HC][D]
-  float *mlbuf = reinterpret_cast<float *>(smem + C::OBUF);          // [NW*NG][HC][2]
-  if (warp < NW) {
-    const int gid = warp * NG + g;
-#pragma unroll
-    for (int h = 0; h < HC; ++h) {
-      float4 *dst = reinterpret_cast<float4 *>(obuf + (gid * HC + h) * D + sub * 16);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) dst[k] = make_float4(o2[h][2 * k].x, o2[h][2 * k].y, o2[h][2 * k + 1].x, o2[h][2 * k + 1].y);
-      if (sub == 0) {
-        mlbuf[(gid * HC + h) * 2 + 0] = m[h];
-        mlbuf[(gid * HC + h) * 2 + 1] = lsum[h];
-      }
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (++t == ntiles) {
+      t = 0;
+      ++u;
+    }
+    if (++st == NST) {
+      st = 0;
+      fphase ^= 1u;
     }
   }
-  __syncthreads();
-
-  const bool single = a.nsplit == 1;
-  const int64_t part_idx = (bh * a.nsplit + split) * a.G + hc * HC;  // first head row of this CTA
-  for (int e = tid; e < HC * D; e += C::THREADS) {
-    const int h = e / D, d = e - h * D;
-    float M = -INFINITY;
-    for (int gi = 0; gi < NW * NG; ++gi) M = fmaxf(M, mlbuf[(gi * HC + h) * 2]);
-    float Ltot = 0.0f, O = 0.0f;
-    if (M != -INFINITY) {
-      for (int gi = 0; gi < NW * NG; ++gi) {
-        const float mg = mlbuf[(gi * HC + h) * 2];
-        if (mg == -INFINITY) continue;
-        const float f = exp2f(mg - M);
-        Ltot = fmaf(f, mlbuf[(gi * HC + h) * 2 + 1], Ltot);
-        O = fmaf(f, obuf[(gi * HC + h) * D + d], O);
-      }
-    }
-    if (single) {
-      const int hq = hk * a.G + hc * HC + h;
-      const float r = Ltot > 0.0f ? O / Ltot : 0.0f;
-      a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-    } else {
-      a.ws_o[(part_idx + h) * D + d] = O;
-      if (d == 0) {
-        a.ws_ml[(part_idx + h) * 2 + 0] = M;
-        a.ws_ml[(part_idx + h) * 2 + 1] = Ltot;
-      }
-    }
-  }
-  if (single) return;
-
-  // ---------------------------------------------------------------- split merge
-  __threadfence();
-  __syncthreads();
-  int32_t *counter = a.counters + bh * a.nhc + hc;
-  if (tid == 0) sh[2] = (atomicAdd(counter, 1) == a.nsplit - 1);
-  __syncthreads();
-  if (!sh[2]) return;
-  __threadfence();
-  for (int e = tid; e < HC * D; e += C::THREADS) {
-    const int h = e / D, d = e - h * D;
-    float M = -INFINITY;
-    for (int sp = 0; sp < a.nsplit; ++sp)
-      M = fmaxf(M, __ldcg(a.ws_ml + ((bh * a.nsplit + sp) * a.G + hc * HC + h) * 2));
-    float Ltot = 0.0f, O = 0.0f;
-    if (M != -INFINITY) {
-      for (int sp = 0; sp < a.nsplit; ++sp) {
-        const int64_t pi = (bh * a.nsplit + sp) * a.G + hc * HC + h;
-        const float ms = __ldcg(a.ws_ml + pi * 2);
-        if (ms == -INFINITY) continue;
-        const float f = exp2f(ms - M);
-        Ltot = fmaf(f, __ldcg(a.ws_ml + pi * 2 + 1), Ltot);
-        O = fmaf(f, __ldcg(a.ws_o + pi * D + d), O);
-      }
-    }
-    const int hq = hk * a.G + hc * HC + h;
-    const float r = Ltot > 0.0f ? O / Ltot : 0.0f;
-    a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-  }
-  if (tid == 0) *counter = 0;  // leave the workspace ready for the next call
+  if (cur_u >= 0) close_segment(cur_u, seg);
 }
 
 // ----------------------------------------------------------------------------
@@ -359,48 +551,36 @@ __global__ void __launch_bounds__(C::THREADS) decode_kernel(const DecodeArgs a) 
 // ----------------------------------------------------------------------------
 int head_chunk(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1)); }
 
+// Tile geometry per head dim: (consumer warps, ring stages).
 template <int D>
-struct DCfgFor;
+struct DTune;
 template <>
-struct DCfgFor<64> { static constexpr int NW = 8, NST = 3; };
+struct DTune<64> { static constexpr int NW = 7, NST = 4; };
 template <>
-struct DCfgFor<128> { static constexpr int NW = 4, NST = 3; };
+struct DTune<128> { static constexpr int NW = 7, NST = 3; };
 template <>
-struct DCfgFor<256> { static constexpr int NW = 2, NST = 3; };
-
-int tile_slots(int D) { return 32 * (D == 64 ? DCfgFor<64>::NW : D == 128 ? DCfgFor<128>::NW : DCfgFor<256>::NW); }
-
-// Split count: enough CTAs for ~4 per SM (two resident rounds of two), never
-// more than one tile per split at full S.
-int choose_nsplit(int B, int Hkv, int nhc, int D, int64_t S) {
-  const int64_t units = static_cast<int64_t>(B) * Hkv * nhc;
-  const int64_t target = static_cast<int64_t>(sm_count()) * 4;
-  int64_t ns = (target + units - 1) / units;
-  const int64_t max_split = (S + tile_slots(D) - 1) / tile_slots(D);
-  if (ns > max_split) ns = max_split;
-  if (ns < 1) ns = 1;
-  if (ns > 1024) ns = 1024;
-  return static_cast<int>(ns);
-}
+struct DTune<256> { static constexpr int NW = 4, NST = 3; };
 
 struct WsLayout {
   size_t counters, ml, o, total;
+  int smax;
 };
 
-WsLayout ws_layout(int B, int Hq, int Hkv, int D, int nsplit, int nhc) {
+WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
   WsLayout w;
-  const size_t nc = static_cast<size_t>(B) * Hkv * nhc;
+  const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
+  w.smax = static_cast<int>((U + ctas - 1) / ctas + 2);
+  const size_t recs = static_cast<size_t>(ctas) * w.smax;
   w.counters = 0;
-  w.ml = (nc * 4 + 255) / 256 * 256;
-  const size_t rows = static_cast<size_t>(B) * Hkv * nsplit * (Hq / Hkv);
-  w.o = w.ml + (rows * 2 * 4 + 255) / 256 * 256;
-  w.total = nsplit > 1 ? w.o + rows * D * 4 : 0;
+  w.ml = (static_cast<size_t>(U) * 4 + 255) / 256 * 256;
+  w.o = w.ml + (recs * HC * 2 * 4 + 255) / 256 * 256;
+  w.total = w.o + recs * HC * D * 4;
   return w;
 }
 
 template <int D, int HC>
-int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
-  using C = Cfg<D, HC, DCfgFor<D>::NW, DCfgFor<D>::NST>;
+int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
+  using C = Cfg<D, HC, DTune<D>::NW, DTune<D>::NST>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
@@ -408,18 +588,17 @@ int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
       return KVQ_ECUDA;
     configured = true;
   }
-  dim3 grid(a.nsplit * a.nhc, a.Hkv, a.B);
-  decode_kernel<C><<<grid, C::THREADS, C::SMEM, stream>>>(a);
+  decode_kernel<C><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
   return launch_status();
 }
 
 template <int D>
-int dispatch_hc(const DecodeArgs &a, int hc, cudaStream_t s) {
+int dispatch_hc(const DecodeArgs &a, int hc, int ctas, cudaStream_t s) {
   switch (hc) {
-    case 1: return launch_decode<D, 1>(a, s);
-    case 2: return launch_decode<D, 2>(a, s);
-    case 3: return launch_decode<D, 3>(a, s);
-    default: return launch_decode<D, 4>(a, s);
+    case 1: return launch_decode<D, 1>(a, ctas, s);
+    case 2: return launch_decode<D, 2>(a, ctas, s);
+    case 3: return launch_decode<D, 3>(a, ctas, s);
+    default: return launch_decode<D, 4>(a, ctas, s);
   }
 }
 
@@ -430,10 +609,8 @@ extern "C" size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int6
   using namespace kvq;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S % 16 != 0) return 0;
   if (D != 64 && D != 128 && D != 256) return 0;
-  const int nhc = (Hq / Hkv) / head_chunk(Hq / Hkv);
-  const int ns = choose_nsplit(B, Hkv, nhc, D, S);
-  const WsLayout w = ws_layout(B, Hq, Hkv, D, ns, nhc);
-  return w.total > 0 ? w.total : 256;
+  const int G = Hq / Hkv, hc = head_chunk(G);
+  return ws_layout(B, Hkv, D, G / hc, hc, sm_count()).total;
 }
 
 extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
@@ -454,12 +631,9 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   const int G = Hq / Hkv;
   const int hc = head_chunk(G);
   const int nhc = G / hc;
-  if (static_cast<int64_t>(B) * Hkv > 65535 * 65535LL || Hkv > 65535 || B > 65535) return KVQ_EUNSUPPORTED;
-  const int ns = choose_nsplit(B, Hkv, nhc, D, S);
-  const WsLayout w = ws_layout(B, Hq, Hkv, D, ns, nhc);
-  if (ns > 1) {
-    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KVQ_EINVAL;
-  }
+  const int ctas = sm_count();
+  const WsLayout w = ws_layout(B, Hkv, D, nhc, hc, ctas);
+  if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KVQ_EINVAL;
   DecodeArgs a;
   a.q = static_cast<const uint16_t *>(q);
   a.k = k;
@@ -472,22 +646,22 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   a.kv_len = kv_len;
   a.out = static_cast<uint16_t *>(out);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  a.counters = ns > 1 ? reinterpret_cast<int32_t *>(ws + w.counters) : nullptr;
-  a.ws_ml = ns > 1 ? reinterpret_cast<float *>(ws + w.ml) : nullptr;
-  a.ws_o = ns > 1 ? reinterpret_cast<float *>(ws + w.o) : nullptr;
+  a.counters = reinterpret_cast<int32_t *>(ws + w.counters);
+  a.ws_ml = reinterpret_cast<float *>(ws + w.ml);
+  a.ws_o = reinterpret_cast<float *>(ws + w.o);
   a.err = err_word;
   a.S = S;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.G = G;
-  a.nsplit = ns;
   a.nhc = nhc;
+  a.smax = w.smax;
   a.qscale = sm_scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 64: return dispatch_hc<64>(a, hc, s);
-    case 128: return dispatch_hc<128>(a, hc, s);
-    default: return dispatch_hc<256>(a, hc, s);
+    case 64: return dispatch_hc<64>(a, hc, ctas, s);
+    case 128: return dispatch_hc<128>(a, hc, ctas, s);
+    default: return dispatch_hc<256>(a, hc, ctas, s);
   }
 }

@@ -96,6 +96,31 @@ KVQ_DEVINL float e8m0_inverse(int e) {
   return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(1u << 22);
 }
 
+// rne(x / scale) as an int, bit-identical to __float2int_rn(__fdiv_rn(x, scale)):
+// y = x * rcp (rcp = correctly rounded 1/scale) is within 3 ulp of the
+// correctly rounded quotient q, so whenever y is more than 2^-12 away from a
+// half-integer (|y| <= 512 here), y and q round to the same integer.  Otherwise
+// (about 1 element in 4000) the exact division decides.
+KVQ_DEVINL int div_rint(float x, float scale, float rcp) {
+  const float y = __fmul_rn(x, rcp);
+  const float r = rintf(y);
+  if (fabsf(__fsub_rn(y, r)) < 0.5f - 0x1p-12f && fabsf(y) <= 512.0f) return static_cast<int>(r);
+  return __float2int_rn(__fdiv_rn(x, scale));
+}
+
+// E4M3 codes of (lo / scale, hi / scale), bit-identical to converting the
+// correctly rounded quotients: y = x * rcp is within 3 ulp of the quotient, so
+// if the codes of y - d and y + d (d = 2^-20 |y|) agree, no E4M3 rounding
+// boundary lies between y and the quotient.  Otherwise divide exactly.
+KVQ_DEVINL uint32_t e4m3x2(float lo, float hi);
+KVQ_DEVINL uint32_t e4m3x2_div(float x0, float x1, float scale, float rcp) {
+  const float y0 = __fmul_rn(x0, rcp), y1 = __fmul_rn(x1, rcp);
+  const float d0 = fabsf(y0) * 0x1p-20f, d1 = fabsf(y1) * 0x1p-20f;
+  const uint32_t c = e4m3x2(y0, y1);
+  if (e4m3x2(y0 - d0, y1 - d1) == c && e4m3x2(y0 + d0, y1 + d1) == c) return c;
+  return e4m3x2(__fdiv_rn(x0, scale), __fdiv_rn(x1, scale));
+}
+
 KVQ_DEVINL void unpack8(const uint4 &c, float (&v)[8]) {
   v[0] = bf16lo(c.x); v[1] = bf16hi(c.x);
   v[2] = bf16lo(c.y); v[3] = bf16hi(c.y);
@@ -187,10 +212,11 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         if (scale < FLT_EPSILON) scale = FLT_EPSILON;
         int zp = -128 - __float2int_rn(__fdiv_rn(mn, scale));
         zp = zp < -128 ? -128 : (zp > 127 ? 127 : zp);
+        const float rcp = __frcp_rn(scale);
         uint32_t w[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          int q = __float2int_rn(__fdiv_rn(v[i], scale)) + zp;
+          int q = div_rint(v[i], scale, rcp) + zp;
           q = q < -128 ? -128 : (q > 127 ? 127 : q);
           w[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
         }
@@ -214,11 +240,9 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
           const float scale = __fdiv_rn(amax, 448.0f);
           uint32_t w0 = 0u, w1 = 0u;
           if (amax != 0.0f) {
-            float q[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[i], scale);
-            w0 = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
-            w1 = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
+            const float rcp = __frcp_rn(scale);
+            w0 = e4m3x2_div(v[0], v[1], scale, rcp) | (e4m3x2_div(v[2], v[3], scale, rcp) << 16);
+            w1 = e4m3x2_div(v[4], v[5], scale, rcp) | (e4m3x2_div(v[6], v[7], scale, rcp) << 16);
           }
           if (slot[k] >= 0) {
             uint8_t *crow = static_cast<uint8_t *>(a.codes) + r * a.D;
