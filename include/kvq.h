@@ -131,11 +131,11 @@ int kvq_sink_mask(const int32_t *input_pos, int Lq, const int32_t *slot_pos, int
 /*
  * kvq_decode_workspace_bytes -- size of the kvq_decode_attn workspace.
  *
- * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S), or 0 for
- * arguments kvq_decode_attn would reject.  The workspace must be zero-filled
- * once before its first use; every completed call leaves its counters at zero
- * again, so it can be reused by later calls in stream order (not by two calls
- * running at the same time).
+ * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S) on the
+ * current device (the size depends on its SM count), or 0 for arguments
+ * kvq_decode_attn would reject.  The workspace holds per-CTA partial results
+ * only: it needs no initialisation and can be reused by later calls in stream
+ * order (not by two calls running at the same time).
  */
 size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
 
@@ -162,6 +162,8 @@ size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
  *              scaled scores; -INFINITY hides a slot.  A row that sees no slot
  *              outputs zeros.
  * workspace    device buffer of workspace_bytes >= kvq_decode_workspace_bytes().
+ * Launches two kernels on `stream`: the split decode and, behind it, the merge
+ * of split partials (programmatic dependent launch).
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; every pointer
  * 16-byte aligned.
  */

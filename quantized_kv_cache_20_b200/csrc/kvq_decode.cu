@@ -36,9 +36,10 @@
 //      slot through shared memory and accumulated with packed fp32 FMA.
 //  - Segment close: groups merge by shuffles, warps through shared memory, in
 //    a fixed order.  A unit that a CTA covers alone is written directly; a
-//    unit split across CTAs leaves one partial per CTA in the workspace and the
-//    last CTA to finish it (atomic counter, reset afterwards) merges them in
-//    CTA order.  No atomics touch the output: results are deterministic.
+//    unit split across CTAs leaves one partial per CTA in the workspace, and a
+//    small merge kernel, launched behind the decode kernel with programmatic
+//    dependent launch, combines them in CTA order.  No atomics, no counters:
+//    results are deterministic and the workspace needs no initialisation.
 #include <cuda_bf16.h>
 
 #include "kvq_common.cuh"
@@ -62,7 +63,7 @@ struct DecodeArgs {
   uint16_t *out;
   float *ws_ml;       // [C * smax][HC][2]
   float *ws_o;        // [C * smax][HC][D]
-  int32_t *counters;  // [U]
+  int merge_ctas;     // grid of the merge kernel
   int32_t *err;
   int64_t S;
   int B, Hq, Hkv, G, nhc, smax;
@@ -127,12 +128,10 @@ KVQ_DEVINL int64_t next_owner(int64_t c, int64_t last, int64_t W, int64_t C) {
 KVQ_DEVINL bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    }
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
@@ -161,6 +160,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     sh[2] = 0;
   }
   __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;");
 
   const int kv = sh[0];
   const int ntiles = (kv + TS - 1) / TS;
@@ -324,43 +324,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
           a.ws_ml[(rec * HC + h) * 2] = M;
           a.ws_ml[(rec * HC + h) * 2 + 1] = Lt;
         }
-      }
-    }
-    if (!alone) {
-      __threadfence();
-      consumer_sync(NW * 32);
-      const int64_t last_tile = u * ntl + ntl - 1;
-      if (tid == 0) {
-        int owners = 0;
-        for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) ++owners;
-        sh[2] = atomicAdd(a.counters + u, 1) == owners - 1;
-      }
-      consumer_sync(NW * 32);
-      if (sh[2]) {
-        __threadfence();
-        for (int e = tid; e < HC * D; e += NW * 32) {
-          const int h = e / D, d = e - h * D;
-          float M = -INFINITY;
-          for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
-            const int64_t r = c * a.smax + (u - range_start(c, W, CT) / ntl);
-            M = fmaxf(M, __ldcg(a.ws_ml + (r * HC + h) * 2));
-          }
-          float Lt = 0.0f, O = 0.0f;
-          if (M != -INFINITY) {
-            for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
-              const int64_t r = c * a.smax + (u - range_start(c, W, CT) / ntl);
-              const float mc = __ldcg(a.ws_ml + (r * HC + h) * 2);
-              if (mc == -INFINITY) continue;
-              const float f = ex2(mc - M);
-              Lt = fmaf(f, __ldcg(a.ws_ml + (r * HC + h) * 2 + 1), Lt);
-              O = fmaf(f, __ldcg(a.ws_o + (r * HC + h) * D + d), O);
-            }
-          }
-          const int hq = hk * a.G + hc * HC + h;
-          const float r = Lt > 0.0f ? O / Lt : 0.0f;
-          a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-        }
-        if (tid == 0) a.counters[u] = 0;  // ready for the next call
       }
     }
     consumer_sync(NW * 32);  // scratch free for the next segment
@@ -547,6 +510,78 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 }
 
 // ----------------------------------------------------------------------------
+// Merge of split units: one CTA per unit.  Launched right after the decode
+// kernel (programmatic dependent launch: it may start while the decode grid
+// drains and waits for its completion, so all partials are visible); a unit
+// whose tiles one CTA owned alone was written by the decode kernel already.
+// Partials are combined in owner (CTA) order.
+// ----------------------------------------------------------------------------
+template <class C>
+__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int decode_ctas) {
+  constexpr int D = C::D, HC = C::HC, TS = C::TS;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int32_t recs[1024];
+  __shared__ float mls[1024 * 2];
+  int kv = *a.kv_len;
+  kv = kv < 0 ? 0 : (kv > a.S ? static_cast<int>(a.S) : kv);
+  const int64_t ntl = (kv + TS - 1) / TS;
+  if (ntl == 0) return;
+  const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
+  const int64_t W = U * ntl, CT = decode_ctas;
+  for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
+    const int64_t last_tile = u * ntl + ntl - 1;
+    const int64_t c_first = cta_of(u * ntl, W, CT);
+    const int64_t c_last = cta_of(last_tile, W, CT);
+    if (c_first == c_last) continue;
+    __syncthreads();  // recs / mls reuse across units
+    int owners;
+    if (W >= CT) {  // no CTA has an empty range: the owners are c_first..c_last
+      owners = static_cast<int>(c_last - c_first + 1);
+      for (int i = threadIdx.x; i < owners; i += blockDim.x) {
+        const int64_t c = c_first + i;
+        recs[i] = static_cast<int32_t>(c * a.smax + (u - range_start(c, W, CT) / ntl));
+      }
+    } else {
+      owners = 0;
+      for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
+        if (threadIdx.x == 0) recs[owners] = static_cast<int32_t>(c * a.smax + (u - range_start(c, W, CT) / ntl));
+        ++owners;
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < owners * HC; i += blockDim.x) {
+      const int o = i / HC, h = i - o * HC;
+      const int64_t r = static_cast<int64_t>(recs[o]) * HC + h;
+      mls[i * 2] = a.ws_ml[r * 2];
+      mls[i * 2 + 1] = a.ws_ml[r * 2 + 1];
+    }
+    __syncthreads();
+    const int hc = static_cast<int>(u % a.nhc);
+    const int64_t bhk = u / a.nhc;
+    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    for (int e = threadIdx.x; e < HC * D; e += blockDim.x) {
+      const int h = e / D, d = e - h * D;
+      float M = -INFINITY;
+      for (int o = 0; o < owners; ++o) M = fmaxf(M, mls[(o * HC + h) * 2]);
+      float Lt = 0.0f, O = 0.0f;
+      if (M != -INFINITY) {
+#pragma unroll 4
+        for (int o = 0; o < owners; ++o) {
+          const float oc = a.ws_o[(static_cast<int64_t>(recs[o]) * HC + h) * D + d];
+          const float mc = mls[(o * HC + h) * 2];
+          const float f = mc == -INFINITY ? 0.0f : ex2(mc - M);
+          Lt = fmaf(f, mls[(o * HC + h) * 2 + 1], Lt);
+          O = fmaf(f, oc, O);
+        }
+      }
+      const int hq = hk * a.G + hc * HC + h;
+      const float r = Lt > 0.0f ? O / Lt : 0.0f;
+      a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Host side
 // ----------------------------------------------------------------------------
 int head_chunk(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1)); }
@@ -555,25 +590,26 @@ int head_chunk(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 
 template <int D>
 struct DTune;
 template <>
-struct DTune<64> { static constexpr int NW = 7, NST = 4; };
+struct DTune<64> { static constexpr int NW = 11, NST = 3; };
 template <>
-struct DTune<128> { static constexpr int NW = 7, NST = 3; };
+struct DTune<128> { static constexpr int NW = 11, NST = 2; };
 template <>
 struct DTune<256> { static constexpr int NW = 4, NST = 3; };
 
 struct WsLayout {
-  size_t counters, ml, o, total;
+  size_t ml, o, total;
   int smax;
 };
 
+// Partials of split units: one record per (CTA, segment) slot; a CTA touches
+// at most ceil(U / ctas) + 2 units.
 WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
   WsLayout w;
   const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
   w.smax = static_cast<int>((U + ctas - 1) / ctas + 2);
   const size_t recs = static_cast<size_t>(ctas) * w.smax;
-  w.counters = 0;
-  w.ml = (static_cast<size_t>(U) * 4 + 255) / 256 * 256;
-  w.o = w.ml + (recs * HC * 2 * 4 + 255) / 256 * 256;
+  w.ml = 0;
+  w.o = (recs * HC * 2 * 4 + 255) / 256 * 256;
   w.total = w.o + recs * HC * D * 4;
   return w;
 }
@@ -589,6 +625,18 @@ int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
     configured = true;
   }
   decode_kernel<C><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.merge_ctas));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, merge_kernel<C>, a, ctas) != cudaSuccess) return KVQ_ECUDA;
   return launch_status();
 }
 
@@ -633,6 +681,7 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   const int nhc = G / hc;
   const int ctas = sm_count();
   const WsLayout w = ws_layout(B, Hkv, D, nhc, hc, ctas);
+  if (ctas > 256) return KVQ_EUNSUPPORTED;  // merge staging holds 256 owners x 4 heads
   if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KVQ_EINVAL;
   DecodeArgs a;
   a.q = static_cast<const uint16_t *>(q);
@@ -646,7 +695,6 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   a.kv_len = kv_len;
   a.out = static_cast<uint16_t *>(out);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  a.counters = reinterpret_cast<int32_t *>(ws + w.counters);
   a.ws_ml = reinterpret_cast<float *>(ws + w.ml);
   a.ws_o = reinterpret_cast<float *>(ws + w.o);
   a.err = err_word;
@@ -657,6 +705,10 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   a.G = G;
   a.nhc = nhc;
   a.smax = w.smax;
+  {
+    const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
+    a.merge_ctas = static_cast<int>(U < 4 * ctas ? U : 4 * ctas);
+  }
   a.qscale = sm_scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {

@@ -1,19 +1,22 @@
 // kvq_write.cu -- the quantized KV-cache write (quantize + scatter by slot).
 //
-// One streaming kernel per mode.  Work is split into units: a (token, head)
-// row for the int8 affine mode (ExecuTorch PR 24473, Summary: per token and
-// head), a 32-element group for the block modes (IndexerQuantCache page,
-// 计算公式: scale_g = max|x_g| / Q_MAX, q_i = round(x_i / scale_g)).  Each unit
-// is covered by LANES consecutive lanes, each owning one 16-byte chunk of 8
-// bf16 values, so a warp reads 512 contiguous bytes per load instruction and
-// reduces with xor-shuffles inside the unit.  UNROLL units per lane are loaded
-// before any arithmetic, to keep enough bytes in flight to cover HBM latency.
-// Tokens whose slot is -1 are skipped before their x is read (IndexerQuantCache
-// page, 约束说明), so skipped rows cost no input bandwidth.
+// Work is cut into 32-element groups along the last dim; one lane owns one
+// group (64 bytes of bf16 x: four 16-byte loads) and writes its codes.
+//   - block modes (IndexerQuantCache page, 计算公式: scale_g = max|x_g| / Q_MAX,
+//     q_i = round(x_i / scale_g)) need nothing outside the group;
+//   - the int8 affine mode (ExecuTorch PR 24473, Summary: per token and head)
+//     reduces min/max over the D/32 lanes of a row with xor-shuffles.
+// A warp covers 32 consecutive groups, i.e. 2 KB of contiguous input for
+// contiguous K/V.  Tokens whose slot is -1 are skipped before their x is read
+// (IndexerQuantCache page, 约束说明), so skipped rows cost no input bandwidth.
 //
-// The arithmetic is binary32 with explicit round-to-nearest-even intrinsics
-// (__fdiv_rn, __fsub_rn, __float2int_rn) in the order the definitions state,
-// so results are bit-reproducible and independent of contraction.
+// The arithmetic is binary32, one round-to-nearest-even per operation, in the
+// order the definitions state, so codes, scales and zero points are
+// reproducible bit for bit.  A division by the per-row/per-group scale is done
+// as y = x * rcp(scale) (rcp correctly rounded): y lies within 3 ulp of the
+// correctly rounded quotient, so whenever y is provably clear of every rounding
+// boundary of the final code, the code is the same; a group with any element
+// next to a boundary is redone with exact IEEE division (__fdiv_rn).
 #include <float.h>
 
 #include "kvq_common.cuh"
@@ -38,20 +41,21 @@ struct FastDiv {
 struct WriteArgs {
   const uint16_t *x;
   int64_t xs0, xs1, xs2;  // element strides of b, h, t
-  int B, H, T, D;
-  FastDiv div_T, div_H, div_G;  // by T, by H, by groups per row
+  int B, H, T, D, GPR;    // GPR: 32-element groups per row
+  FastDiv div_T, div_H, div_G;
   const int32_t *slot_mapping;
   int64_t S;
   void *codes;
   void *scales;
   int8_t *zps;
   int32_t *err;
-  int64_t units;  // total units
+  uint32_t groups;  // total groups
 };
 
 constexpr int kThreads = 256;
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: v + kMagic holds rne(v) in its low mantissa bits
 
-// --- E4M3 / E2M1 conversion on the hardware cvt (round-to-nearest-even,
+// E4M3 / E2M1 conversion on the hardware cvt (round-to-nearest-even,
 // saturating to the largest finite value).  PTX puts the FIRST source in the
 // UPPER half, so the element that must land low is passed second.
 KVQ_DEVINL uint32_t e4m3x2(float lo, float hi) {
@@ -60,8 +64,7 @@ KVQ_DEVINL uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-// 8 floats -> 4 bytes of E2M1 pairs (element 2i in the low nibble of byte i).
-KVQ_DEVINL uint32_t e2m1x8(const float (&v)[8]) {
+KVQ_DEVINL uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6, float v7) {
   uint32_t r;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -70,7 +73,7 @@ KVQ_DEVINL uint32_t e2m1x8(const float (&v)[8]) {
       "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(r)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
   return r;
 }
 
@@ -96,48 +99,10 @@ KVQ_DEVINL float e8m0_inverse(int e) {
   return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(1u << 22);
 }
 
-// rne(x / scale) as an int, bit-identical to __float2int_rn(__fdiv_rn(x, scale)):
-// y = x * rcp (rcp = correctly rounded 1/scale) is within 3 ulp of the
-// correctly rounded quotient q, so whenever y is more than 2^-12 away from a
-// half-integer (|y| <= 512 here), y and q round to the same integer.  Otherwise
-// (about 1 element in 4000) the exact division decides.
-KVQ_DEVINL int div_rint(float x, float scale, float rcp) {
-  const float y = __fmul_rn(x, rcp);
-  const float r = rintf(y);
-  if (fabsf(__fsub_rn(y, r)) < 0.5f - 0x1p-12f && fabsf(y) <= 512.0f) return static_cast<int>(r);
-  return __float2int_rn(__fdiv_rn(x, scale));
-}
-
-// E4M3 codes of (lo / scale, hi / scale), bit-identical to converting the
-// correctly rounded quotients: y = x * rcp is within 3 ulp of the quotient, so
-// if the codes of y - d and y + d (d = 2^-20 |y|) agree, no E4M3 rounding
-// boundary lies between y and the quotient.  Otherwise divide exactly.
-KVQ_DEVINL uint32_t e4m3x2(float lo, float hi);
-KVQ_DEVINL uint32_t e4m3x2_div(float x0, float x1, float scale, float rcp) {
-  const float y0 = __fmul_rn(x0, rcp), y1 = __fmul_rn(x1, rcp);
-  const float d0 = fabsf(y0) * 0x1p-20f, d1 = fabsf(y1) * 0x1p-20f;
-  const uint32_t c = e4m3x2(y0, y1);
-  if (e4m3x2(y0 - d0, y1 - d1) == c && e4m3x2(y0 + d0, y1 + d1) == c) return c;
-  return e4m3x2(__fdiv_rn(x0, scale), __fdiv_rn(x1, scale));
-}
-
-KVQ_DEVINL void unpack8(const uint4 &c, float (&v)[8]) {
-  v[0] = bf16lo(c.x); v[1] = bf16hi(c.x);
-  v[2] = bf16lo(c.y); v[3] = bf16hi(c.y);
-  v[4] = bf16lo(c.z); v[5] = bf16hi(c.z);
-  v[6] = bf16lo(c.w); v[7] = bf16hi(c.w);
-}
-
-// Locate unit u: for the affine mode a unit is a row (b, h, t) with t fastest;
-// for block modes it is group `gi` of that row.
-template <int MODE>
-KVQ_DEVINL void unit_coords(const WriteArgs &a, uint32_t u, int &b, int &h, int &t, int &gi) {
-  uint32_t row = u;
-  gi = 0;
-  if (MODE != KVQ_MODE_INT8_AFFINE) {
-    row = a.div_G.div(u);
-    gi = static_cast<int>(u - row * a.div_G.d);
-  }
+// Locate group g: row (b, h, t) with t fastest, and the group index in the row.
+KVQ_DEVINL void group_coords(const WriteArgs &a, uint32_t g, int &b, int &h, int &t, int &gi) {
+  const uint32_t row = a.div_G.div(g);
+  gi = static_cast<int>(g - row * a.div_G.d);
   const uint32_t bh = a.div_T.div(row);
   t = static_cast<int>(row - bh * a.div_T.d);
   const uint32_t bq = a.div_H.div(bh);
@@ -145,149 +110,189 @@ KVQ_DEVINL void unit_coords(const WriteArgs &a, uint32_t u, int &b, int &h, int 
   b = static_cast<int>(bq);
 }
 
-// LANES lanes per unit; UNROLL units per lane per pass.
-template <int MODE, int LANES, int UNROLL>
-__global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
-  constexpr int UPW = 32 / LANES;  // units per warp per unroll step
-  const int lane = threadIdx.x & 31;
-  const int sub = lane % LANES;
-  const int uw = lane / LANES;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+// Low bytes of four floats that hold integers in their low mantissa bits.
+KVQ_DEVINL uint32_t pack_low_bytes(float a, float b, float c, float d) {
+  const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040u);
+  const uint32_t cd = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040u);
+  return __byte_perm(ab, cd, 0x5410u);
+}
 
-  for (int64_t base = warp * (UPW * UNROLL); base < a.units; base += nwarps * (UPW * UNROLL)) {
-    int64_t unit[UNROLL];
-    int slot[UNROLL];
-    int bb[UNROLL], hh[UNROLL], gg[UNROLL];
-    uint4 raw[UNROLL];
-    // Phase 1: slots (one per unit; the same address across the unit's lanes).
-#pragma unroll
-    for (int k = 0; k < UNROLL; ++k) {
-      unit[k] = base + k * UPW + uw;
-      slot[k] = -1;
-      bb[k] = hh[k] = gg[k] = 0;
-      if (unit[k] < a.units) {
-        int t;
-        unit_coords<MODE>(a, static_cast<uint32_t>(unit[k]), bb[k], hh[k], t, gg[k]);
-        const int s = __ldg(a.slot_mapping + static_cast<int64_t>(bb[k]) * a.T + t);
-        if (s != -1 && (s < 0 || s >= a.S)) {
-          if (sub == 0) report(a.err, KVQ_ERR_SLOT_RANGE);
-          slot[k] = -1;
-        } else {
-          slot[k] = s;
-        }
-        if (slot[k] >= 0) {
-          const uint16_t *row = a.x + bb[k] * a.xs0 + hh[k] * a.xs1 + static_cast<int64_t>(t) * a.xs2;
-          raw[k] = ld_stream_v4(row + gg[k] * 32 + sub * 8);
-        }
+template <int MODE>
+__global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
+  const uint32_t stride = gridDim.x * kThreads;
+  // Every lane of a warp runs the loop the same number of times (the bound is
+  // rounded up to whole warps), so the int8 mode's row shuffles see the whole warp.
+  const uint32_t total = (a.groups + 31u) & ~31u;
+  for (uint32_t g = blockIdx.x * kThreads + threadIdx.x; g < total; g += stride) {
+    int b = 0, h = 0, t = 0, gi = 0, slot = -1;
+    if (g < a.groups) {
+      group_coords(a, g, b, h, t, gi);
+      const int s = __ldg(a.slot_mapping + static_cast<int64_t>(b) * a.T + t);
+      if (s != -1 && (s < 0 || s >= a.S)) {
+        if (gi == 0) report(a.err, KVQ_ERR_SLOT_RANGE);
+      } else {
+        slot = s;
       }
     }
-    // Phase 2: quantize and store.
+    float v[32];
+    if (slot >= 0) {
+      const uint16_t *p = a.x + b * a.xs0 + h * a.xs1 + static_cast<int64_t>(t) * a.xs2 + gi * 32;
+      uint4 c[4];
 #pragma unroll
-    for (int k = 0; k < UNROLL; ++k) {
-      float v[8];
-      if (slot[k] >= 0)
-        unpack8(raw[k], v);
-      else
+      for (int k = 0; k < 4; ++k) c[k] = __ldg(reinterpret_cast<const uint4 *>(p) + k);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      const int64_t r = (static_cast<int64_t>(bb[k]) * a.H + hh[k]) * a.S + (slot[k] < 0 ? 0 : slot[k]);
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t w[4] = {c[k].x, c[k].y, c[k].z, c[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * k + 2 * j] = bf16lo(w[j]);
+          v[8 * k + 2 * j + 1] = bf16hi(w[j]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    }
+    const int64_t r = (static_cast<int64_t>(b) * a.H + h) * a.S + (slot < 0 ? 0 : slot);
 
-      if constexpr (MODE == KVQ_MODE_INT8_AFFINE) {
-        // mn = min(0, min x), mx = max(0, max x): exact, order-free.
-        float mn = 0.0f, mx = 0.0f;
+    if constexpr (MODE == KVQ_MODE_INT8_AFFINE) {
+      // mn = min(0, min x), mx = max(0, max x) over the row: exact, order-free
+      float mn = 0.0f, mx = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          mn = v[i] < mn ? v[i] : mn;
-          mx = v[i] > mx ? v[i] : mx;
-        }
+      for (int i = 0; i < 32; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+      }
+      for (int o = a.GPR >> 1; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (slot < 0) continue;
+      float scale = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+      if (scale < FLT_EPSILON) scale = FLT_EPSILON;
+      int zp = -128 - __float2int_rn(__fdiv_rn(mn, scale));
+      zp = zp < -128 ? -128 : (zp > 127 ? 127 : zp);
+      const float rcp = __frcp_rn(scale);
+      const float zpf = static_cast<float>(zp);
+      // q = clamp(rne(x/scale) + zp) = rne(clamp(y + zp)) for y = x*rcp, taken
+      // with the kMagic add.  y is within 1.5 * 2^-23 |y| of the correctly
+      // rounded quotient and forming y + zp moves it by at most 2^-18 without
+      // crossing a half-integer, so a distance to the nearest half-integer
+      // above 2^-22 |y| + 2^-17 settles the code.
+      float t2[32];
+      float worst = 0.0f;
 #pragma unroll
-        for (int o = LANES / 2; o > 0; o >>= 1) {
-          const float omn = __shfl_xor_sync(0xffffffffu, mn, o);
-          const float omx = __shfl_xor_sync(0xffffffffu, mx, o);
-          mn = omn < mn ? omn : mn;
-          mx = omx > mx ? omx : mx;
-        }
-        float scale = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
-        if (scale < FLT_EPSILON) scale = FLT_EPSILON;
-        int zp = -128 - __float2int_rn(__fdiv_rn(mn, scale));
-        zp = zp < -128 ? -128 : (zp > 127 ? 127 : zp);
-        const float rcp = __frcp_rn(scale);
-        uint32_t w[2] = {0u, 0u};
+      for (int i = 0; i < 32; i += 2) {
+        const float2 y = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(rcp, rcp));
+        float2 yz = __fadd2_rn(y, make_float2(zpf, zpf));
+        yz.x = fminf(fmaxf(yz.x, -128.0f), 127.0f);
+        yz.y = fminf(fmaxf(yz.y, -128.0f), 127.0f);
+        const float2 tt = __fadd2_rn(yz, make_float2(kMagic, kMagic));
+        const float2 rr = __fadd2_rn(tt, make_float2(-kMagic, -kMagic));
+        const float2 dd = __ffma2_rn(rr, make_float2(-1.0f, -1.0f), yz);  // yz - rne(yz)
+        worst = fmaxf(worst, fmaf(fabsf(y.x), 0x1p-22f, fabsf(dd.x)));
+        worst = fmaxf(worst, fmaf(fabsf(y.y), 0x1p-22f, fabsf(dd.y)));
+        t2[i] = tt.x;
+        t2[i + 1] = tt.y;
+      }
+      if (worst >= 0.5f - 0x1p-17f) {  // rare: settle the group with exact division
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          int q = div_rint(v[i], scale, rcp) + zp;
+        for (int i = 0; i < 32; ++i) {
+          int q = __float2int_rn(__fdiv_rn(v[i], scale)) + zp;
           q = q < -128 ? -128 : (q > 127 ? 127 : q);
-          w[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
+          t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
         }
-        if (slot[k] >= 0) {
-          int8_t *crow = static_cast<int8_t *>(a.codes) + r * a.D;
-          st_v2(crow + sub * 8, w[0], w[1]);
-          if (sub == 0) {
-            static_cast<float *>(a.scales)[r] = scale;
-            a.zps[r] = static_cast<int8_t>(zp);
+      }
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<int8_t *>(a.codes) + r * a.D + gi * 32);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      if (gi == 0) {
+        static_cast<float *>(a.scales)[r] = scale;
+        a.zps[r] = static_cast<int8_t>(zp);
+      }
+    } else {
+      if (slot < 0) continue;
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      const int64_t sidx = r * a.GPR + gi;  // scale index
+      if constexpr (MODE == KVQ_MODE_FP8_E4M3) {
+        const float scale = __fdiv_rn(amax, 448.0f);
+        uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (amax != 0.0f) {
+          const float rcp = __frcp_rn(scale);
+          // cvt is monotone: if y(1 - 2^-20) and y(1 + 2^-20) -- which bracket
+          // the correctly rounded quotient -- get the same code, so does it.
+          uint32_t diff = 0u;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float2 y0 = __fmul2_rn(make_float2(v[4 * k], v[4 * k + 1]), make_float2(rcp, rcp));
+            const float2 y1 = __fmul2_rn(make_float2(v[4 * k + 2], v[4 * k + 3]), make_float2(rcp, rcp));
+            const float2 l0 = __fmul2_rn(y0, make_float2(1.0f - 0x1p-20f, 1.0f - 0x1p-20f));
+            const float2 h0 = __fmul2_rn(y0, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
+            const float2 l1 = __fmul2_rn(y1, make_float2(1.0f - 0x1p-20f, 1.0f - 0x1p-20f));
+            const float2 h1 = __fmul2_rn(y1, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
+            const uint32_t c = e4m3x2(y0.x, y0.y) | (e4m3x2(y1.x, y1.y) << 16);
+            const uint32_t cl = e4m3x2(l0.x, l0.y) | (e4m3x2(l1.x, l1.y) << 16);
+            const uint32_t ch = e4m3x2(h0.x, h0.y) | (e4m3x2(h1.x, h1.y) << 16);
+            diff |= (c ^ cl) | (c ^ ch);
+            w[k] = c;
+          }
+          if (diff) {  // rare: exact division for the whole group
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              w[k] = e4m3x2(__fdiv_rn(v[4 * k], scale), __fdiv_rn(v[4 * k + 1], scale)) |
+                     (e4m3x2(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
           }
         }
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        static_cast<float *>(a.scales)[sidx] = scale;
       } else {
-        float amax = 0.0f;
+        constexpr float kQmax = (MODE == KVQ_MODE_MXFP8) ? 448.0f : 6.0f;
+        const int e = e8m0_ceil(__fdiv_rn(amax, kQmax));
+        const float inv = e8m0_inverse(e);  // x / 2^(e-127) == x * 2^(127-e), exactly rounded
+        float y[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const int ngroups = a.D >> 5;
-        const int64_t gidx = r * ngroups + gg[k];  // scale index
-        if constexpr (MODE == KVQ_MODE_FP8_E4M3) {
-          const float scale = __fdiv_rn(amax, 448.0f);
-          uint32_t w0 = 0u, w1 = 0u;
-          if (amax != 0.0f) {
-            const float rcp = __frcp_rn(scale);
-            w0 = e4m3x2_div(v[0], v[1], scale, rcp) | (e4m3x2_div(v[2], v[3], scale, rcp) << 16);
-            w1 = e4m3x2_div(v[4], v[5], scale, rcp) | (e4m3x2_div(v[6], v[7], scale, rcp) << 16);
-          }
-          if (slot[k] >= 0) {
-            uint8_t *crow = static_cast<uint8_t *>(a.codes) + r * a.D;
-            st_v2(crow + gg[k] * 32 + sub * 8, w0, w1);
-            if (sub == 0) static_cast<float *>(a.scales)[gidx] = scale;
-          }
-        } else {
-          constexpr float kQmax = (MODE == KVQ_MODE_MXFP8) ? 448.0f : 6.0f;
-          const int e = e8m0_ceil(__fdiv_rn(amax, kQmax));
-          const float inv = e8m0_inverse(e);  // x / 2^(e-127) == x * 2^(127-e), exactly rounded
-          float q[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
-          if constexpr (MODE == KVQ_MODE_MXFP8) {
-            uint32_t w0 = 0u, w1 = 0u;
-            if (amax != 0.0f) {
-              w0 = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
-              w1 = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
-            }
-            if (slot[k] >= 0) {
-              uint8_t *crow = static_cast<uint8_t *>(a.codes) + r * a.D;
-              st_v2(crow + gg[k] * 32 + sub * 8, w0, w1);
-            }
-          } else {
-            const uint32_t w = (amax != 0.0f) ? e2m1x8(q) : 0u;
-            if (slot[k] >= 0) {
-              uint8_t *crow = static_cast<uint8_t *>(a.codes) + r * (a.D >> 1);
-              st_u32(crow + gg[k] * 16 + sub * 4, w);
-            }
-          }
-          if (slot[k] >= 0 && sub == 0) static_cast<uint8_t *>(a.scales)[gidx] = static_cast<uint8_t>(e);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 yy = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(inv, inv));
+          y[i] = yy.x;
+          y[i + 1] = yy.y;
         }
+        if constexpr (MODE == KVQ_MODE_MXFP8) {
+          uint32_t w[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            w[k] = amax != 0.0f ? (e4m3x2(y[4 * k], y[4 * k + 1]) | (e4m3x2(y[4 * k + 2], y[4 * k + 3]) << 16)) : 0u;
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w[k] = amax != 0.0f ? e2m1x8(y[8 * k], y[8 * k + 1], y[8 * k + 2], y[8 * k + 3], y[8 * k + 4],
+                                         y[8 * k + 5], y[8 * k + 6], y[8 * k + 7])
+                                : 0u;
+          *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * (a.D >> 1) + gi * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        static_cast<uint8_t *>(a.scales)[sidx] = static_cast<uint8_t>(e);
       }
     }
   }
 }
 
-template <int MODE, int LANES, int UNROLL>
+template <int MODE>
 int launch_write(const WriteArgs &a, cudaStream_t stream) {
-  constexpr int UPW = 32 / LANES;
-  const int64_t warps_needed = (a.units + UPW * UNROLL - 1) / (UPW * UNROLL);
-  const int64_t blocks_needed = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads = full SM
+  const int64_t blocks_needed = (static_cast<int64_t>(a.groups) + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads = a full SM
   const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-  write_kernel<MODE, LANES, UNROLL><<<grid, kThreads, 0, stream>>>(a);
+  write_kernel<MODE><<<grid, kThreads, 0, stream>>>(a);
   return launch_status();
 }
 
@@ -316,9 +321,9 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   // float scales (modes 0 and 1) must be 4-byte aligned; E8M0 scales are bytes
   if ((mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_FP8_E4M3) && (reinterpret_cast<uintptr_t>(scales) & 3u))
     return KVQ_EINVAL;
-  // unit indices use 32-bit arithmetic
-  if (static_cast<int64_t>(B) * H * T * (mode == KVQ_MODE_INT8_AFFINE ? 1 : D / 32) >= (int64_t(1) << 31))
-    return KVQ_EUNSUPPORTED;
+  // group indices use 32-bit arithmetic
+  const int64_t groups = static_cast<int64_t>(B) * H * T * (D / 32);
+  if (groups >= (int64_t(1) << 31)) return KVQ_EUNSUPPORTED;
 
   WriteArgs a;
   a.x = static_cast<const uint16_t *>(x);
@@ -329,31 +334,22 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   a.H = H;
   a.T = T;
   a.D = D;
+  a.GPR = D / 32;
   a.div_T = FastDiv(static_cast<uint32_t>(T));
   a.div_H = FastDiv(static_cast<uint32_t>(H));
-  a.div_G = FastDiv(static_cast<uint32_t>(mode == KVQ_MODE_INT8_AFFINE ? 1 : D / 32));
+  a.div_G = FastDiv(static_cast<uint32_t>(D / 32));
   a.slot_mapping = slot_mapping;
   a.S = num_slots;
   a.codes = codes;
   a.scales = scales;
   a.zps = zero_points;
   a.err = err_word;
-  const int64_t rows = static_cast<int64_t>(B) * H * T;
+  a.groups = static_cast<uint32_t>(groups);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (mode) {
-    case KVQ_MODE_INT8_AFFINE:
-      a.units = rows;
-      if (D == 64) return launch_write<KVQ_MODE_INT8_AFFINE, 8, 4>(a, s);
-      if (D == 128) return launch_write<KVQ_MODE_INT8_AFFINE, 16, 4>(a, s);
-      return launch_write<KVQ_MODE_INT8_AFFINE, 32, 4>(a, s);
-    case KVQ_MODE_FP8_E4M3:
-      a.units = rows * (D / 32);
-      return launch_write<KVQ_MODE_FP8_E4M3, 4, 4>(a, s);
-    case KVQ_MODE_MXFP8:
-      a.units = rows * (D / 32);
-      return launch_write<KVQ_MODE_MXFP8, 4, 4>(a, s);
-    default:
-      a.units = rows * (D / 32);
-      return launch_write<KVQ_MODE_MXFP4, 4, 4>(a, s);
+    case KVQ_MODE_INT8_AFFINE: return launch_write<KVQ_MODE_INT8_AFFINE>(a, s);
+    case KVQ_MODE_FP8_E4M3: return launch_write<KVQ_MODE_FP8_E4M3>(a, s);
+    case KVQ_MODE_MXFP8: return launch_write<KVQ_MODE_MXFP8>(a, s);
+    default: return launch_write<KVQ_MODE_MXFP4>(a, s);
   }
 }

@@ -156,11 +156,12 @@ def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, S: int) -> int:
 
 
 def decode_workspace(B: int, Hq: int, Hkv: int, D: int, S: int, device) -> torch.Tensor:
-    """A zero-filled workspace of the size kvq_decode_attn needs."""
-    n = decode_workspace_bytes(B, Hq, Hkv, D, S)
+    """A workspace of the size kvq_decode_attn needs (no initialisation required)."""
+    with torch.cuda.device(device):
+        n = decode_workspace_bytes(B, Hq, Hkv, D, S)
     if n == 0:
         raise ValueError("unsupported decode configuration")
-    return torch.zeros(n, dtype=torch.uint8, device=device)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word):

@@ -165,9 +165,6 @@ def test_kv_len_is_read_on_device_each_call():
         out = kvq.decode_attn(q, *Kd, *Vd, kv, workspace=ws)
         ref = oracle.sdpa(wl.u16(q.cpu()), *_np(K), *_np(V), kv_len=n, sm_scale=1 / math.sqrt(D))
         assert_attn_close(bf16_to_f64(out), ref, f"kv_len {n}")
-    # the split counters are back at zero after every call
-    nc = B * Hkv
-    assert torch.all(ws[: nc * 4].view(torch.int32) == 0)
 
 
 def test_kv_len_full_equals_bound_at_s_and_out_of_range_is_clamped():
