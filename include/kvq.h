@@ -41,6 +41,7 @@ extern "C" {
 #define KVQ_EINVAL (-1)       /* null pointer, bad size, misaligned pointer, bad stride */
 #define KVQ_EUNSUPPORTED (-2) /* a valid request this build does not implement */
 #define KVQ_ECUDA (-3)        /* the CUDA launch itself failed */
+#define KVQ_ESCRATCH (-4)     /* kvq_decode_attn_static: the problem needs more than the static scratch */
 
 /* Device error-word bits (OR-ed into *err_word). */
 #define KVQ_ERR_SLOT_RANGE 1   /* a slot outside [0, num_slots) other than -1 was skipped */
@@ -195,6 +196,36 @@ int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const
                      const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
                      int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
                      void *stream);
+
+/*
+ * kvq_decode_attn_static -- kvq_decode_attn without a caller-supplied workspace.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory when they run attention: runtimes that
+ * plan and own every byte of device memory up front, plain C hosts that have
+ * no device allocator, and callers that must not let an allocation (and the
+ * synchronisation cudaMalloc can imply) into their decode loop.  Instead of
+ * the workspace it uses a buffer of KVQ_STATIC_SCRATCH_BYTES that lives in
+ * the library itself (a file-scope __device__ array: every GPU that loads the
+ * library holds it until the process exits).  It allocates nothing and frees
+ * nothing.
+ *
+ * Arguments, layouts and results are those of kvq_decode_attn.  A problem
+ * whose partial results would not fit the buffer (kvq_decode_workspace_bytes
+ * above KVQ_STATIC_SCRATCH_BYTES) returns KVQ_ESCRATCH and enqueues nothing.
+ * The first call on a device looks up the buffer's device address (with that
+ * device current); make that first call before capturing a stream into a CUDA
+ * graph.  All calls on a device share the one buffer, which keeps whatever the
+ * last call left in it: nothing in it has to start at zero, but two calls
+ * whose kernels overlap on the GPU (different streams without ordering) race
+ * on it and produce wrong results.
+ */
+#define KVQ_STATIC_SCRATCH_BYTES (8u << 20) /* 8 MiB per device */
+int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
+                           const float *k_scale, const int8_t *k_zp, const int8_t *v,
+                           const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_len,
+                           const float *mask, float sm_scale, void *out, int32_t *err_word,
+                           void *stream);
 
 /* A static, human-readable name for a host status code. */
 const char *kvq_strerror(int status);

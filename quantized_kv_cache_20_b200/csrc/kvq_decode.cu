@@ -42,6 +42,8 @@
 //    results are deterministic and the workspace needs no initialisation.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "kvq_common.cuh"
 
 namespace kvq {
@@ -716,4 +718,48 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
     case 128: return dispatch_hc<128>(a, hc, ctas, s);
     default: return dispatch_hc<256>(a, hc, ctas, s);
   }
+}
+
+// ----------------------------------------------------------------------------
+// Decode without a caller-supplied workspace (for callers that cannot
+// allocate device memory): the partials go to a buffer that is part of the
+// library image.  In host code the symbol is only a handle; its device address
+// is looked up once per device, with that device current.
+// ----------------------------------------------------------------------------
+namespace kvq {
+namespace {
+static __device__ __align__(256) uint8_t g_static_scratch[KVQ_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void *g_static_scratch_addr[kMaxDevices] = {};
+
+int static_scratch_address(void **addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return KVQ_ECUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *addr = g_static_scratch_addr[dev];
+  return KVQ_OK;
+}
+}  // namespace
+}  // namespace kvq
+
+extern "C" int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
+                                      const float *k_scale, const int8_t *k_zp, const int8_t *v,
+                                      const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_len,
+                                      const float *mask, float sm_scale, void *out, int32_t *err_word,
+                                      void *stream) {
+  const size_t need = kvq_decode_workspace_bytes(B > 0 ? B : 1, Hq, Hkv, D, S);
+  if (need > KVQ_STATIC_SCRATCH_BYTES) return KVQ_ESCRATCH;
+  void *scratch = nullptr;
+  const int st = kvq::static_scratch_address(&scratch);
+  if (st != KVQ_OK) return st;
+  return kvq_decode_attn(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, mask, sm_scale, out,
+                         scratch, KVQ_STATIC_SCRATCH_BYTES, err_word, stream);
 }

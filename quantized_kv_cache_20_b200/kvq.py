@@ -21,6 +21,8 @@ KVQ_OK = 0
 KVQ_EINVAL = -1
 KVQ_EUNSUPPORTED = -2
 KVQ_ECUDA = -3
+KVQ_ESCRATCH = -4
+STATIC_SCRATCH_BYTES = 8 << 20
 
 KVQ_ERR_SLOT_RANGE = 1
 KVQ_ERR_KV_LEN_RANGE = 2
@@ -34,7 +36,7 @@ MODE_MXFP4 = 3
 
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
-    "kvq_decode_attn", "kvq_prefill_attn", "kvq_strerror", "kvq_version",
+    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_prefill_attn", "kvq_strerror", "kvq_version",
 )
 
 _lib = None
@@ -69,6 +71,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_workspace_bytes.restype = SZ
         lib.kvq_decode_attn.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
         lib.kvq_decode_attn.restype = I
+        lib.kvq_decode_attn_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, P]
+        lib.kvq_decode_attn_static.restype = I
         lib.kvq_prefill_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I, I, F, P, P, P]
         lib.kvq_prefill_attn.restype = I
         lib.kvq_strerror.argtypes = [I]
@@ -197,6 +201,26 @@ def decode_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask
                                 _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
                                 _stream(q.device))
     _check("kvq_decode_attn", st)
+    return out
+
+
+def decode_attn_static(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,
+                       err_word=None) -> torch.Tensor:
+    """kvq_decode_attn_static: decode attention that allocates nothing; its scratch
+    is the library's own per-device buffer (for callers that cannot allocate)."""
+    if out is None:
+        out = torch.empty_like(q)
+    _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if Lq != 1:
+        raise ValueError("decode takes one query row (use prefill_attn)")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    st = load().kvq_decode_attn_static(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                       _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask),
+                                       float(sm_scale), _ptr(out), _ptr(err_word), _stream(q.device))
+    _check("kvq_decode_attn_static", st)
     return out
 
 
