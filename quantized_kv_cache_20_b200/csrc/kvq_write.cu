@@ -17,6 +17,7 @@
 // correctly rounded quotient, so whenever y is provably clear of every rounding
 // boundary of the final code, the code is the same; a group with any element
 // next to a boundary is redone with exact IEEE division (__fdiv_rn).
+#include <cuda_bf16.h>
 #include <float.h>
 
 #include "kvq_common.cuh"
@@ -134,35 +135,36 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         slot = s;
       }
     }
-    float v[32];
+    uint32_t wx[16];  // 32 bf16 values, element 2j in the low half of wx[j]
     if (slot >= 0) {
-      const uint16_t *p = a.x + b * a.xs0 + h * a.xs1 + static_cast<int64_t>(t) * a.xs2 + gi * 32;
-      uint4 c[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) c[k] = __ldg(reinterpret_cast<const uint4 *>(p) + k);
+      const uint4 *p =
+          reinterpret_cast<const uint4 *>(a.x + b * a.xs0 + h * a.xs1 + static_cast<int64_t>(t) * a.xs2 + gi * 32);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint32_t w[4] = {c[k].x, c[k].y, c[k].z, c[k].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[8 * k + 2 * j] = bf16lo(w[j]);
-          v[8 * k + 2 * j + 1] = bf16hi(w[j]);
-        }
+        const uint4 c = __ldg(p + k);
+        wx[4 * k] = c.x;
+        wx[4 * k + 1] = c.y;
+        wx[4 * k + 2] = c.z;
+        wx[4 * k + 3] = c.w;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+      for (int j = 0; j < 16; ++j) wx[j] = 0u;
     }
     const int64_t r = (static_cast<int64_t>(b) * a.H + h) * a.S + (slot < 0 ? 0 : slot);
 
     if constexpr (MODE == KVQ_MODE_INT8_AFFINE) {
-      // mn = min(0, min x), mx = max(0, max x) over the row: exact, order-free
-      float mn = 0.0f, mx = 0.0f;
+      // mn = min(0, min x), mx = max(0, max x) over the row: exact, order-free,
+      // taken two bf16 at a time
+      __nv_bfloat162 mn2 = __float2bfloat162_rn(0.0f), mx2 = mn2;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mn = fminf(mn, v[i]);
-        mx = fmaxf(mx, v[i]);
+      for (int j = 0; j < 16; ++j) {
+        const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162 *>(&wx[j]);
+        mn2 = __hmin2(mn2, x2);
+        mx2 = __hmax2(mx2, x2);
       }
+      float mn = fminf(__low2float(mn2), __high2float(mn2));
+      float mx = fmaxf(__low2float(mx2), __high2float(mx2));
       for (int o = a.GPR >> 1; o > 0; o >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -182,23 +184,20 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
       float t2[32];
       float worst = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float2 y = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(rcp, rcp));
-        float2 yz = __fadd2_rn(y, make_float2(zpf, zpf));
-        yz.x = fminf(fmaxf(yz.x, -128.0f), 127.0f);
-        yz.y = fminf(fmaxf(yz.y, -128.0f), 127.0f);
-        const float2 tt = __fadd2_rn(yz, make_float2(kMagic, kMagic));
-        const float2 rr = __fadd2_rn(tt, make_float2(-kMagic, -kMagic));
-        const float2 dd = __ffma2_rn(rr, make_float2(-1.0f, -1.0f), yz);  // yz - rne(yz)
-        worst = fmaxf(worst, fmaf(fabsf(y.x), 0x1p-22f, fabsf(dd.x)));
-        worst = fmaxf(worst, fmaf(fabsf(y.y), 0x1p-22f, fabsf(dd.y)));
-        t2[i] = tt.x;
-        t2[i + 1] = tt.y;
+      for (int i = 0; i < 32; ++i) {
+        const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
+        const float y = __fmul_rn(x, rcp);
+        const float yz = fminf(fmaxf(__fadd_rn(y, zpf), -128.0f), 127.0f);
+        const float tt = __fadd_rn(yz, kMagic);
+        const float dd = __fsub_rn(yz, __fsub_rn(tt, kMagic));  // yz - rne(yz)
+        worst = fmaxf(worst, fmaf(fabsf(y), 0x1p-22f, fabsf(dd)));
+        t2[i] = tt;
       }
       if (worst >= 0.5f - 0x1p-17f) {  // rare: settle the group with exact division
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          int q = __float2int_rn(__fdiv_rn(v[i], scale)) + zp;
+          const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
+          int q = __float2int_rn(__fdiv_rn(x, scale)) + zp;
           q = q < -128 ? -128 : (q > 127 ? 127 : q);
           t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
         }
@@ -215,9 +214,16 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
       }
     } else {
       if (slot < 0) continue;
-      float amax = 0.0f;
+      __nv_bfloat162 am2 = __float2bfloat162_rn(0.0f);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      for (int j = 0; j < 16; ++j) am2 = __hmax2(am2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&wx[j])));
+      const float amax = fmaxf(__low2float(am2), __high2float(am2));
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[2 * j] = bf16lo(wx[j]);
+        v[2 * j + 1] = bf16hi(wx[j]);
+      }
       const int64_t sidx = r * a.GPR + gi;  // scale index
       if constexpr (MODE == KVQ_MODE_FP8_E4M3) {
         const float scale = __fdiv_rn(amax, 448.0f);
