@@ -190,6 +190,11 @@ int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *
  *               order (is_causal, or a mask that hides j > kv_len - Lq + i),
  *               which enables the per-tile bound.
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; 1 <= Lq <= S.
+ * Launches one kernel on `stream`: 128 query rows per CTA on the tcgen05
+ * tensor cores, S = Q K^T and O += P V in bf16 with fp32 accumulation in
+ * tensor memory.  K/V codes enter as the exact bf16 values (c - zp); the scales
+ * are applied in fp32 (k_scale to the scores, v_scale folded into P, which
+ * enters as the sum of two bf16 terms so that it keeps ~16 significant bits).
  */
 int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
                      const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,

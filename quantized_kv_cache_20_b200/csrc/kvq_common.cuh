@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kvq.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -20,6 +22,21 @@ namespace kvq {
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int launch_status() { return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ECUDA; }
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// is per device context).  `Tag` names the kernel instantiation.
+template <class Tag, class Kernel>
+inline int ensure_smem(Kernel kernel, int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ECUDA;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return KVQ_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return KVQ_ECUDA;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return KVQ_OK;
+}
 
 inline int sm_count() {
   int dev = 0, n = 148;

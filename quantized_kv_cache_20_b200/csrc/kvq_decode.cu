@@ -619,13 +619,7 @@ WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
 template <int D, int HC>
 int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
   using C = Cfg<D, HC, DTune<D>::NW, DTune<D>::NST>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-        cudaSuccess)
-      return KVQ_ECUDA;
-    configured = true;
-  }
+  if (const int st = ensure_smem<C>(decode_kernel<C>, C::SMEM)) return st;
   decode_kernel<C><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
   cudaLaunchConfig_t cfg = {};

@@ -1,6 +1,6 @@
 // kvq_prefill.cu -- chunked-prefill attention entry point.
 #include "kvq_common.cuh"
-#include "kvq_prefill_simt.cuh"
+#include "kvq_prefill_tc.cuh"
 
 extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
                                 const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
@@ -20,7 +20,7 @@ extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, i
   if (mask && !aligned16(mask)) return KVQ_EINVAL;
   if (!(sm_scale == sm_scale)) return KVQ_EINVAL;
   if (Hq > 65535 || B > 65535) return KVQ_EUNSUPPORTED;
-  simt::PrefillArgs a;
+  tc::PrefillArgs a;
   a.q = static_cast<const uint16_t *>(q);
   a.k = k;
   a.ks = k_scale;
@@ -36,14 +36,16 @@ extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, i
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
+  a.G = Hq / Hkv;
   a.Lq = Lq;
+  a.nhc = 1;
   a.is_causal = is_causal ? 1 : 0;
   a.mask_is_causal = mask_is_causal ? 1 : 0;
   a.qscale = sm_scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 64: return simt::launch_prefill_simt<64>(a, s);
-    case 128: return simt::launch_prefill_simt<128>(a, s);
-    default: return simt::launch_prefill_simt<256>(a, s);
+    case 64: return tc::dispatch_prefill_tc<64>(a, s);
+    case 128: return tc::dispatch_prefill_tc<128>(a, s);
+    default: return tc::dispatch_prefill_tc<256>(a, s);
   }
 }

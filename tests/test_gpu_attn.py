@@ -227,7 +227,7 @@ def test_prefill_tile_skip_is_bit_identical(D):
     a = _prefill_gpu(q, K, V, kv_len, is_causal=True, mask_is_causal=False)
     b = _prefill_gpu(q, K, V, kv_len, is_causal=True, mask_is_causal=True)
     assert torch.equal(a, b)
-    # and at Lq = 1 the bound is the whole kv_len: prefill equals decode bit for bit
+    # at Lq = 1 the bound is the whole kv_len: the causal and plain settings agree bit for bit
     q1 = wl.bf16_normal((B, Hq, 1, D), g)
     c = _prefill_gpu(q1, K, V, kv_len, is_causal=True, mask_is_causal=True)
     d = _prefill_gpu(q1, K, V, kv_len, is_causal=False, mask_is_causal=False)
