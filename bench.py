@@ -15,7 +15,8 @@ Printed (rank 0): one JSON line with the headline metric (tokens/s), the
 roofline of the dominant kernel (decode attention, HBM-bound), the end-to-end
 number through the Python binding with host buffers, the CPU oracle baseline,
 clocks sampled during the timed region, and per-kernel detail lines for the
-bulk fill write, the block-quantized writes and the long-context decode.
+bulk fill write, the block-quantized writes, the long-context decode, and the
+two chunked prefills (long causal chunk, sink/ring chunk) on the tensor cores.
 """
 from __future__ import annotations
 
@@ -36,6 +37,7 @@ if ROOT not in sys.path:
 METRIC = "KV-write GB/s + int8-KV decode attn tokens/s, % of B200 HBM roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def _args():
@@ -47,8 +49,11 @@ def _args():
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--kernel", choices=["decode", "fill", "block1", "block2", "block3", "long_decode"],
+    ap.add_argument("--kernel", choices=["decode", "fill", "block1", "block2", "block3", "long_decode",
+                                         "long_prefill", "sink_prefill"],
                     help="profiling aid: launch only this kernel on its workload --steps times, print nothing")
+    ap.add_argument("--kv-len", type=int, default=0,
+                    help="with --kernel long_prefill: cache length and kv_len (default: the full 131072)")
     return ap.parse_args()
 
 
@@ -60,6 +65,23 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def _tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (kernels here are timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def causal_prefill_flops(Hq, D, Lq, kv_len):
+    """Algorithmic FLOPs of a causal chunk: 2 D (q.k) + 2 D (p.v) per visible (row, key) pair;
+    row i sees kv_len - Lq + i + 1 keys."""
+    pairs = Lq * (kv_len - Lq) + Lq * (Lq + 1) // 2
+    return 4 * D * Hq * pairs
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -159,9 +181,13 @@ class Dist:
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | None = None):
-    """Time the CPU oracle on the decode workload: each step writes one token's K
-    and V (64 rows each) and computes all 256 (b, h) attention rows at kv_len 4096."""
+def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | None = None,
+                         rows_per_step: int | None = None):
+    """Time the CPU oracle on the decode workload.  A step writes one token's K
+    and V (64 rows each) and computes `rows_per_step` of the 256 (b, h)
+    attention rows at kv_len 4096 (all of them by default; a sample cycles
+    through the rows).  Returns (steps, seconds, full_step_seconds): the last
+    is the time a step with all 256 rows takes, estimated from the sample."""
     import numpy as np
     import oracle
     from quantized_kv_cache_20_b200 import workloads as wl
@@ -175,41 +201,63 @@ def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | No
     v = wl.u16(wl.bf16_normal((w.B, w.Hkv, 1, w.D), g))
     q = wl.u16(wl.bf16_normal((w.B, w.Hq, 1, w.D), g))
     sm = np.full(w.B, S - 1, np.int32)
+    rows = [(b, h, 0) for b in range(w.B) for h in range(w.Hq)]
+    r = len(rows) if rows_per_step is None else max(1, min(len(rows), rows_per_step))
     oracle.build()
-    steps, t0 = 0, time.perf_counter()
+    steps, t_write, t_attn = 0, 0.0, 0.0
+    t0 = time.perf_counter()
     while True:
+        ta = time.perf_counter()
         oracle.write(0, k, sm, S, *K)
         oracle.write(0, v, sm, S, *V)
-        oracle.sdpa(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D))
+        tb = time.perf_counter()
+        if r == len(rows):
+            oracle.sdpa(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D))
+        else:
+            sel = [rows[(steps * r + j) % len(rows)] for j in range(r)]
+            oracle.sdpa_rows(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D), rows=sel)
+        tc = time.perf_counter()
+        t_write += tb - ta
+        t_attn += tc - tb
         steps += 1
-        el = time.perf_counter() - t0
+        el = tc - t0
         if (steps >= min_steps and el >= seconds) or (max_steps is not None and steps >= max_steps):
             break
-    return steps, el
+    full = (t_write + t_attn * len(rows) / r) / steps
+    return steps, el, full
+
+
+REFERENCE_BUDGET_S = 120.0  # the timed part of --impl reference stays near this
 
 
 def run_reference(args, dist: Dist):
-    dist.setup_cpu()
+    """The oracle arm: rank 0 alone times the C oracle on the host cores (other
+    ranks exit at once).  Each step attends a bounded sample of the 256 rows,
+    sized so that --steps K stays within about REFERENCE_BUDGET_S seconds; the
+    metric is scaled to full steps."""
     if dist.rank != 0:
-        dist.close()
         return
     from quantized_kv_cache_20_b200 import workloads as wl
     w = wl.DECODE
-    _oracle_decode_steps(0.0, min_steps=args.warmup, max_steps=args.warmup)
-    steps, el = _oracle_decode_steps(0.0, min_steps=args.steps, max_steps=args.steps)
-    value = w.B * steps / el
+    _, _, full = _oracle_decode_steps(0.0, min_steps=1, max_steps=1)  # calibration (and build)
+    rows_total = w.B * w.Hq
+    per_row = full / rows_total
+    r = int(max(1, min(rows_total, REFERENCE_BUDGET_S / max(1, args.steps) / per_row)))
+    _oracle_decode_steps(0.0, min_steps=args.warmup, max_steps=args.warmup, rows_per_step=r)
+    steps, el, full = _oracle_decode_steps(0.0, min_steps=args.steps, max_steps=args.steps, rows_per_step=r)
+    value = w.B / full
+    sample = (f"{steps} decode steps, each writing 1 token K/V for 8x8 rows and computing {r} of the 256 "
+              f"attention rows at kv_len 4096 (rows cycle); tokens/s scaled to full 256-row steps; "
+              f"single-threaded C oracle, {el:.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * el / steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": _config(args),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{steps} full decode steps (write 1 token K/V for 8x8 rows + 256 attention "
-                                   f"rows at kv_len 4096), single-threaded C oracle"},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * full,
+        "measured_ms_per_sampled_step": 1000 * el / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-    dist.close()
 
 
 def _config(args):
@@ -356,10 +404,10 @@ def run_kvq(args, dist: Dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * nsteps, "clocks": clk, "detail": detail,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 4 * nsteps, "clocks": clk, "detail": detail,
     }
     if dist.rank == 0 and dist.world == 1:
-        steps_c, el_c = _oracle_decode_steps(args.cpu_seconds)
+        steps_c, el_c, _ = _oracle_decode_steps(args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": B * steps_c / el_c, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{steps_c} full decode steps of the same workload (write 1 token K/V for 8x8 rows + "
@@ -514,6 +562,55 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
     res["long_decode"] = {"what": "kvq_decode_attn, batch 1, 32 q / 16 kv heads, D=256, kv_len 131072",
                           "us": ms * 1000, "tokens/s": 1 / (ms / 1000), "GB/s": lbytes / (ms / 1000) / 1e9,
                           "frac": lbytes / (ms / 1000) / 1e9 / peak, "bytes": lbytes}
+    # long-context chunked prefill: the last 2048-row causal chunk at kv_len 131072 (tensor cores)
+    tpeak, tkind = _tensor_peak()
+    qp = torch.randn((1, lw.Hq, lw.Lq, lw.D), device=dev).to(torch.bfloat16)
+    op = torch.empty_like(qp)
+
+    def lpre():
+        kvq.prefill_attn(qp, *K, *V, kvl, out=op, is_causal=True, mask_is_causal=True)
+    ms = _time_graph(stream, lpre, 5)
+    fl = causal_prefill_flops(lw.Hq, lw.D, lw.Lq, lw.kv_len)
+    res["long_prefill"] = {"what": "kvq_prefill_attn, causal chunk Lq 2048 at kv_len 131072, 32 q / 16 kv heads, "
+                                   "D=256, per-tile causal bound", "us": ms * 1000,
+                           "tokens/s": lw.Lq / (ms / 1000), "TFLOP/s": fl / (ms / 1000) / 1e12,
+                           "frac": fl / (ms / 1000) / 1e12 / tpeak, "peak_TFLOP/s": tpeak, "peak_kind": tkind,
+                           "flops": fl}
+    del K, V, qp, op, wsl
+    torch.cuda.empty_cache()
+    # attention-sink ring: one 128-row chunk over the full 2048-slot ring with the additive mask
+    sw = wl.SINK
+    NS = 16  # rotated caches (16 x 4.5 MiB K/V codes) so the chunk reads cold-ish data
+    rings = []
+    for i in range(NS):
+        Kr = (torch.randint(-128, 128, (1, sw.Hkv, sw.S, sw.D), dtype=torch.int8, device=dev),
+              torch.rand((1, sw.Hkv, sw.S), device=dev) * 0.012 + 0.018,
+              torch.randint(-6, 7, (1, sw.Hkv, sw.S), dtype=torch.int8, device=dev))
+        Vr = tuple(t.clone() for t in Kr)
+        rings.append((Kr, Vr))
+    ip = torch.tensor([10000 - sw.Lq], dtype=torch.int32, device=dev)
+    spos = torch.full((sw.S,), -1, dtype=torch.int32, device=dev)
+    smp = torch.empty(sw.Lq, dtype=torch.int32, device=dev)
+    kvs = torch.empty(1, dtype=torch.int32, device=dev)
+    mask = torch.empty((sw.Lq, sw.S), dtype=torch.float32, device=dev)
+    ipp = torch.zeros(1, dtype=torch.int32, device=dev)
+    for p in range(0, 10000 - sw.Lq, sw.Lq):  # step the ring so slot positions wrap as in the workload
+        ipp.fill_(p)
+        kvq.sink_plan(ipp, 1, sw.Lq, sw.sink, spos, smp, kvs)
+    kvq.sink_plan(ip, 1, sw.Lq, sw.sink, spos, smp, kvs)
+    kvq.sink_mask(ip, sw.Lq, spos, mask)
+    qs = torch.randn((1, sw.Hq, sw.Lq, sw.D), device=dev).to(torch.bfloat16)
+    os_ = torch.empty_like(qs)
+
+    def spre():
+        for Kr, Vr in rings:
+            kvq.prefill_attn(qs, *Kr, *Vr, kvs, out=os_, mask=mask)
+    ms = _time_graph(stream, spre, 20) / NS
+    fl = 4 * sw.D * sw.Hq * sw.Lq * sw.S
+    res["sink_prefill_chunk"] = {"what": "kvq_prefill_attn, 128-row chunk at position 9872 over the 4 + 2044 ring, "
+                                         "32 q / 8 kv heads, D=128, additive mask", "us": ms * 1000,
+                                 "tokens/s": sw.Lq / (ms / 1000), "TFLOP/s": fl / (ms / 1000) / 1e12,
+                                 "frac": fl / (ms / 1000) / 1e12 / tpeak, "flops": fl}
     return res
 
 
@@ -529,9 +626,11 @@ def run_kernel(args):
     torch.cuda.set_device(dev)
     g = torch.Generator(device=dev)
     g.manual_seed(5)
-    if args.kernel in ("decode", "fill", "long_decode"):
-        w = wl.LONG if args.kernel == "long_decode" else wl.DECODE
-        B, Hq, Hkv, D, S, KV = w.B, w.Hq, w.Hkv, w.D, w.S, w.kv_len
+    if args.kernel in ("decode", "fill", "long_decode", "long_prefill", "sink_prefill"):
+        w = {"decode": wl.DECODE, "fill": wl.DECODE, "sink_prefill": wl.SINK}.get(args.kernel, wl.LONG)
+        B, Hq, Hkv, D, S, KV = w.B, w.Hq, w.Hkv, w.D, w.S, (w.kv_len or w.S)
+        if args.kernel == "long_prefill" and args.kv_len:
+            S = KV = args.kv_len
         K = (torch.randint(-128, 128, (B, Hkv, S, D), dtype=torch.int8, device=dev),
              torch.rand((B, Hkv, S), device=dev) * 0.012 + 0.018,
              torch.randint(-6, 7, (B, Hkv, S), dtype=torch.int8, device=dev))
@@ -541,6 +640,14 @@ def run_kernel(args):
             sm = torch.arange(KV - 1, dtype=torch.int32, device=dev).repeat(B)
             for _ in range(args.steps):
                 kvq.write(0, x, sm, *K)
+        elif args.kernel.endswith("prefill"):
+            q = torch.randn((B, Hq, w.Lq, D), generator=g, device=dev).to(torch.bfloat16)
+            kv = torch.tensor([KV], dtype=torch.int32, device=dev)
+            out = torch.empty_like(q)
+            causal = args.kernel == "long_prefill"
+            mask = None if causal else torch.zeros((w.Lq, S), dtype=torch.float32, device=dev)
+            for _ in range(args.steps):
+                kvq.prefill_attn(q, *K, *V, kv, out=out, mask=mask, is_causal=causal, mask_is_causal=causal)
         else:
             q = torch.randn((B, Hq, 1, D), generator=g, device=dev).to(torch.bfloat16)
             kv = torch.tensor([KV], dtype=torch.int32, device=dev)

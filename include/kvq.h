@@ -16,8 +16,9 @@
  *     unless a parameter says "host".  The caller owns every buffer; the
  *     library never allocates, frees, or synchronizes the host.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
- *     stream).  All work is enqueued asynchronously on it; no call reads
- *     device memory on the host, so every call can be captured in a CUDA graph.
+ *     stream).  All work is enqueued asynchronously on it and no call reads
+ *     device memory on the host: kvq_write, kvq_sink_plan, kvq_sink_mask,
+ *     kvq_decode_attn and kvq_prefill_attn can be captured in a CUDA graph.
  *   - bf16 means IEEE binary16-brain (torch.bfloat16) bit patterns.
  *   - Return value: KVQ_OK (0) or a negative host status (below).  A non-zero
  *     status means nothing was enqueued, except KVQ_ECUDA from a failed launch.

@@ -8,32 +8,48 @@
 // V = (v - v_zp) * v_scale, for the chunk's Lq query rows at positions
 // kv_len - Lq + i.
 //
-// Design:
-//  - One CTA = one warpgroup (128 threads) = 128 query rows.  With GQA the rows
-//    are HPT heads x RPH positions of the same kv head, so every K/V tile is
-//    dequantized once for all of them.  Thread t owns row t: TMEM lane t.
-//  - K/V tiles of 64 slots: int8 codes are turned into the exact bf16 values
-//    (c - zp) (|c - zp| <= 255, exact in bf16) and written into 128-byte
-//    swizzled shared memory, the layout the tensor core reads; the per-slot
-//    scales are applied outside the MMAs: k_scale to the score columns, v_scale
-//    folded into P.
-//  - S = Q K^T: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128, N=64, into
-//    TMEM; the softmax warpgroup reads S with tcgen05.ld, keeps an online
-//    softmax in the log2 domain (running max raised only when a score exceeds
-//    it by more than 8), and writes P = p * v_scale to swizzled shared memory as
-//    two bf16 terms, P_hi = bf16(P) and P_lo = bf16(P - P_hi), so the product
-//    keeps about 16 significant bits (a single bf16 P would cost up to 2^-9 of
-//    max|V| in the output); then O += P_hi V + P_lo V: tcgen05.mma M=128, N=D
-//    into TMEM.  V = (c - zp) is exact in bf16.  O is rescaled in TMEM only when
-//    the running max moves.
-//  - Per-tile causal bound: with mask_is_causal the tile loop stops at
-//    min(kv_len, kv_len - Lq + (last row of the CTA) + 1); later tiles would be
-//    fully masked, so the output is bit-identical with or without the skip.
-//  - Two or more CTAs per SM (D <= 128) overlap one CTA's CUDA-core phases with
-//    another's tensor-core phases.
+// Design.  One CTA holds 128 query rows of one kv head (HPT q heads x RPH
+// positions with GQA, so every K/V tile is dequantized once for all of them)
+// and runs three roles, connected by mbarriers:
+//   - softmax warpgroup (warps 0-3): thread t owns query row t, i.e. TMEM lane t;
+//   - converter warpgroup (warps 4-7): turns the int8 codes of 128-slot K and
+//     V tiles into fp16 in the 128-byte-swizzled shared-memory layout the
+//     tensor core reads;
+//   - MMA warp (warp 8): one thread issues every tcgen05.mma.
+// Tensor-core work per tile j:  S_j = Q K_j^T (M 128, N 128) into one of two
+// TMEM buffers; the softmax writes P_j back over the columns of S_j it came
+// from, and O += P_j V_j takes P from TMEM (A operand in tensor memory) and V
+// from shared memory.  Issue order QK_0, QK_1, PV_0, QK_2, PV_1, ...: the
+// softmax of tile j overlaps QK_{j+1}; the converters rebuild K_{j+1} as soon
+// as QK_j has read K_j and V_j as soon as PV_{j-1} has read V_{j-1}, so one
+// shared-memory buffer of each suffices.
+//
+// Numerics: fp16 operands, fp32 accumulation.
+//   - K/V codes become the exact fp16 values (c - zp), |c - zp| <= 255, through
+//     a byte permute into the mantissa of 1024 and one packed subtract.
+//   - Q is multiplied per row by the power of two that brings max|q| into
+//     [2^14, 2^15), then rounded to fp16: exact for every element above 2^-14
+//     in that scale (bf16 carries 8 significant bits, fp16 11); the power of
+//     two is folded back into the row's score scale.
+//   - k_scale multiplies the fp32 scores; v_scale is folded into
+//     P = p * v_scale * 2^-E, where E is a per-CTA exponent kept between 2 and
+//     10 binades above the tile's largest v_scale, so P < 2^7 and P is rounded
+//     to fp16 once (relative error <= 2^-11).  When E moves, O is rescaled in
+//     TMEM by the exact power of two.
+//   - Online softmax in the log2 domain; the running max is raised only when
+//     a score exceeds it by more than 8 (O and l then hold values up to 2^8
+//     larger, harmless in fp32).
+// Per-tile causal bound: with mask_is_causal the tile loop stops at
+// min(kv_len, kv_len - Lq + (last row of the CTA) + 1); later tiles would be
+// fully masked, so the output is bit-identical with or without the skip.
+//
+// Every wait is bounded.  A wait that gives up raises a CTA-wide abort flag;
+// every role leaves its loop at its next wait, the MMA thread waits (bounded)
+// for what it issued, TMEM is freed and KVQ_ERR_TIMEOUT is reported.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kvq_common.cuh"
 
@@ -41,8 +57,14 @@ namespace kvq {
 namespace tc {
 
 constexpr int kRows = 128;  // query rows per CTA (tcgen05 M)
-constexpr int kTile = 64;   // slots per K/V tile (tcgen05 N of S, K of P.V)
-constexpr int kThreads = 128;
+constexpr int kTile = 128;  // slots per K/V tile (N of Q K^T, K of P V)
+constexpr int kSoftmaxThreads = 128;
+constexpr int kConvThreads = 128;
+constexpr int kThreads = kSoftmaxThreads + kConvThreads + 32;
+constexpr int kMmaWarp = 8;
+constexpr int kScaleBufs = 3;  // k_scale / v_scale tile buffers
+// registers per thread: 9 warps, one SM sub-partition holds three of them
+constexpr int kRegsLaunch = 168;
 
 struct PrefillArgs {
   const uint16_t *q;
@@ -62,23 +84,47 @@ struct PrefillArgs {
   float qscale;  // sm_scale * log2(e)
 };
 
-template <int D_, int HPT_>
+// mbarriers.  A parity wait is only meaningful when the barrier has already
+// completed every phase before the awaited one and not the one after it; each
+// wait below is placed where both hold (the epilogue has its own barrier for
+// that reason: O may still be a PV or two behind the softmax).
+enum : int {
+  kBarQ = 0,   // Q tile written (softmax warpgroup, 128 arrivals)
+  kBarKFull,   // K tile written (converters, 128 arrivals)
+  kBarKEmpty,  // QK done with the K tile (commit)
+  kBarVFull,   // V tile written (converters, 128 arrivals)
+  kBarVEmpty,  // PV done with the V tile (commit)
+  kBarSFull0,  // S buffer 0 / 1 computed (commit)
+  kBarSFull1,
+  kBarPFull0,  // P in S buffer 0 / 1 written (softmax, 128 arrivals)
+  kBarPFull1,
+  kBarODone,   // a PV finished (commit)
+  kBarOFinal,  // the last PV finished (commit, once)
+  kBarDrain,   // abort path: everything issued has finished (commit)
+  kNumBars
+};
+
+template <int D_, int HPT_, bool MASK_>
 struct Cfg {
   static constexpr int D = D_, HPT = HPT_, RPH = kRows / HPT;
-  static constexpr int KB = D / 64;  // 64-element (128-byte) blocks along D
-  // shared memory (operand regions 1024-byte aligned for the 128-byte swizzle)
-  static constexpr int Q_OFF = 0;                        // KB x [128 rows x 128 B]
-  static constexpr int K_OFF = Q_OFF + KB * kRows * 128;  // KB x [64 slots x 128 B]
-  static constexpr int V_OFF = K_OFF + KB * kTile * 128;  // KB x [64 slots x 128 B]
-  static constexpr int P_OFF = V_OFF + KB * kTile * 128;  // 2 x [128 rows x 128 B]: P_hi, P_lo
-  static constexpr int KS_OFF = P_OFF + 2 * kRows * 128;  // float[64]
-  static constexpr int VS_OFF = KS_OFF + kTile * 4;       // float[64]
-  static constexpr int BAR_OFF = VS_OFF + kTile * 4;      // 2 mbarriers
-  static constexpr int TM_OFF = BAR_OFF + 16;             // TMEM base address
-  static constexpr int SMEM = TM_OFF + 16 + 1024;         // + slack to align the base to 1024
-  static constexpr int S_COL = 0, O_COL = kTile;
-  static constexpr int TMEM_COLS = (kTile + D) <= 128 ? 128 : ((kTile + D) <= 256 ? 256 : 512);
-  static_assert(kTile + D <= TMEM_COLS, "TMEM budget");
+  static constexpr bool MASK = MASK_;
+  static constexpr int PPR = D / 16;                    // 16-code parts per slot row
+  static constexpr int NSG = kConvThreads / PPR;        // groups of consecutive slots
+  static constexpr int NCH = kTile / NSG;               // slots per group = chunks per converter thread
+  static constexpr int Q_OFF = 0;                       // D/64 x [128 rows  x 128 B]
+  static constexpr int K_OFF = Q_OFF + kRows * 2 * D;   // D/64 x [128 slots x 128 B]
+  static constexpr int V_OFF = K_OFF + kTile * 2 * D;   // D/64 x [128 slots x 128 B]
+  static constexpr int KS_OFF = V_OFF + kTile * 2 * D;  // float [kScaleBufs][128]
+  static constexpr int VS_OFF = KS_OFF + kScaleBufs * kTile * 4;
+  static constexpr int VMX_OFF = VS_OFF + kScaleBufs * kTile * 4;  // float [kScaleBufs][4]
+  static constexpr int BAR_OFF = VMX_OFF + kScaleBufs * 16;
+  static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;        // + slack to align the base to 1024
+  static constexpr int S_COL0 = 0, S_COL1 = kTile, O_COL = 2 * kTile;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(NCH * NSG == kTile && NSG * PPR == kConvThreads && NCH % 4 == 0, "converter mapping");
 };
 
 // ---- descriptors -------------------------------------------------------------
@@ -89,20 +135,30 @@ KVQ_DEVINL uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// Instruction descriptor, kind::f16: f32 accumulator (bits 4-5 = 1), bf16 A and
-// B (bits 7-9, 10-12 = 1), A/B major in bits 15/16 (0 = K-major), N >> 3 in
-// bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn_major) << 16) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// Instruction descriptor, kind::f16: f32 accumulator (bits 4-5 = 1), f16 A and
+// B (bits 7-9, 10-12 = 0), A/B major in bits 15/16 (0 = K-major, 1 = MN-major),
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn_major) {
+  return (1u << 4) | (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-KVQ_DEVINL void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+// D (TMEM) (+)= A (shared) x B (shared)
+KVQ_DEVINL void mma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D (TMEM) (+)= A (TMEM) x B (shared)
+KVQ_DEVINL void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 KVQ_DEVINL void mma_commit(uint64_t *bar) {
@@ -113,9 +169,8 @@ KVQ_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_s
 KVQ_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 KVQ_DEVINL void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-KVQ_DEVINL void tmem_ld32(uint32_t taddr, float (&r)[32]) {
-  uint32_t u[32];
+// 32 consecutive 32-bit columns of this thread's TMEM lane (completes at tmem_ld_wait).
+KVQ_DEVINL void tmem_ld32(uint32_t taddr, uint32_t (&u)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -124,34 +179,51 @@ KVQ_DEVINL void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
         "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
-KVQ_DEVINL void tmem_st32(uint32_t taddr, const float (&r)[32]) {
+KVQ_DEVINL void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+KVQ_DEVINL void tmem_st32(uint32_t taddr, const uint32_t (&u)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(r[0])), "r"(__float_as_uint(r[1])), "r"(__float_as_uint(r[2])), "r"(__float_as_uint(r[3])),
-      "r"(__float_as_uint(r[4])), "r"(__float_as_uint(r[5])), "r"(__float_as_uint(r[6])), "r"(__float_as_uint(r[7])),
-      "r"(__float_as_uint(r[8])), "r"(__float_as_uint(r[9])), "r"(__float_as_uint(r[10])),
-      "r"(__float_as_uint(r[11])), "r"(__float_as_uint(r[12])), "r"(__float_as_uint(r[13])),
-      "r"(__float_as_uint(r[14])), "r"(__float_as_uint(r[15])), "r"(__float_as_uint(r[16])),
-      "r"(__float_as_uint(r[17])), "r"(__float_as_uint(r[18])), "r"(__float_as_uint(r[19])),
-      "r"(__float_as_uint(r[20])), "r"(__float_as_uint(r[21])), "r"(__float_as_uint(r[22])),
-      "r"(__float_as_uint(r[23])), "r"(__float_as_uint(r[24])), "r"(__float_as_uint(r[25])),
-      "r"(__float_as_uint(r[26])), "r"(__float_as_uint(r[27])), "r"(__float_as_uint(r[28])),
-      "r"(__float_as_uint(r[29])), "r"(__float_as_uint(r[30])), "r"(__float_as_uint(r[31]))
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]), "r"(u[9]),
+      "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15]), "r"(u[16]), "r"(u[17]), "r"(u[18]),
+      "r"(u[19]), "r"(u[20]), "r"(u[21]), "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]),
+      "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
       : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+KVQ_DEVINL void tmem_st16(uint32_t taddr, const uint32_t *u) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]), "r"(u[9]),
+      "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+      : "memory");
+}
+KVQ_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// MMA completion arrives within microseconds; give up after 100 ms.
-KVQ_DEVINL bool wait_mma(uint64_t *bar, uint32_t parity) {
+// One probe of a phase, suspending up to 20 us while it is incomplete.
+KVQ_DEVINL bool try_wait_short(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait that also gives up once another role has raised the abort flag.
+KVQ_DEVINL bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  if (try_wait_short(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > 100000000ull) return false;
+    if (try_wait_short(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      return false;
+    }
   }
 }
 
@@ -160,58 +232,101 @@ KVQ_DEVINL float ex2f(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^e for e in [-126, 127]
+KVQ_DEVINL float exp2i(int e) { return __uint_as_float(static_cast<uint32_t>(e + 127) << 23); }
+// ceil(log2 v) for v > 0 (v below the normal range counts as 2^-126)
+KVQ_DEVINL int ceil_log2(float v) {
+  const uint32_t bits = __float_as_uint(v);
+  const int e = static_cast<int>(bits >> 23) - 127;
+  if (e < -126) return -126;
+  return e + ((bits & 0x7FFFFFu) != 0u ? 1 : 0);
+}
 
-// Byte offset of the 16-byte chunk `c` (8 bf16) of row `r` inside a 128-byte
+// Byte offset of the 16-byte chunk `c` (8 halves) of row `r` inside a 128-byte
 // swizzled region (rows of 128 B, chunks XOR-permuted by r % 8).
 KVQ_DEVINL uint32_t swz(int r, int c) { return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// 16 int8 codes -> 16 bf16 values (c - zp), exact, as two 16-byte chunks.
-KVQ_DEVINL void codes16_to_bf16(const uint4 &w, int zp, uint4 &lo, uint4 &hi) {
-  const float mz = neg_magic_zp(zp);
-  const float2 mz2 = make_float2(mz, mz);
-  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-  uint32_t outw[8];
+// 16 int8 codes -> 16 fp16 values (c - zp), exact: (c + 128) goes into the low
+// mantissa bits of 1024 (fp16 0x6400 | byte is 1024 + byte exactly), and one
+// packed subtract of (1152 + zp) leaves c - zp.
+KVQ_DEVINL void codes16_to_f16(const uint4 &w, uint32_t zc2, uint4 &lo, uint4 &hi) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o[8];
+  const __half2 z = *reinterpret_cast<const __half2 *>(&zc2);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float2 a, b;
-    codes4_to_f2(words[k], mz2, a, b);
-    const __nv_bfloat162 ba = __float22bfloat162_rn(a);
-    const __nv_bfloat162 bb = __float22bfloat162_rn(b);
-    outw[2 * k] = *reinterpret_cast<const uint32_t *>(&ba);
-    outw[2 * k + 1] = *reinterpret_cast<const uint32_t *>(&bb);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t u = in[i] ^ 0x80808080u;
+    const uint32_t h0 = __byte_perm(u, 0x64646464u, 0x4140);
+    const uint32_t h1 = __byte_perm(u, 0x64646464u, 0x4342);
+    const __half2 r0 = __hsub2(*reinterpret_cast<const __half2 *>(&h0), z);
+    const __half2 r1 = __hsub2(*reinterpret_cast<const __half2 *>(&h1), z);
+    o[2 * i] = *reinterpret_cast<const uint32_t *>(&r0);
+    o[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&r1);
   }
-  lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-  hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+// Global loads that stay in program order with the mbarrier operations (the
+// compiler may not hoist them above a wait or an arrive, which would keep two
+// tiles of codes in registers).
+KVQ_DEVINL uint4 ld_codes(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+KVQ_DEVINL uint32_t ld_u32(const void *p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+KVQ_DEVINL float ld_f32(const float *p) {
+  float r;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r) : "l"(p));
+  return r;
+}
+// fp16 pair of (1152 + zp): bits 0x6400 | (128 + zp)
+KVQ_DEVINL uint32_t zp_const2(int zp) {
+  const uint32_t h = 0x6400u | static_cast<uint32_t>((zp + 128) & 0xFF);
+  return h | (h << 16);
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads, 2) prefill_tc_kernel(const PrefillArgs a) {
+__global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const PrefillArgs a) {
   constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
-  constexpr int CH = D / 16;  // 16-code chunks per slot row
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (the 128-byte swizzle is a function of address bits 4-9)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-  uint64_t *bar_o = bar_s + 1;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::TM_OFF);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
   float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
   float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
+  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int xrow = blockIdx.x;  // row block
-  const int hkc = blockIdx.y;   // kv head x head chunk
-  const int b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
   const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
   const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
 
-  // ---- set-up: barriers, TMEM, kv_len
+  // ---- set-up
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    mbar_init(&bars[kBarQ], kSoftmaxThreads);
+    mbar_init(&bars[kBarKFull], kConvThreads);
+    mbar_init(&bars[kBarKEmpty], 1);
+    mbar_init(&bars[kBarVFull], kConvThreads);
+    mbar_init(&bars[kBarVEmpty], 1);
+    mbar_init(&bars[kBarSFull0], 1);
+    mbar_init(&bars[kBarSFull1], 1);
+    mbar_init(&bars[kBarPFull0], kSoftmaxThreads);
+    mbar_init(&bars[kBarPFull1], kSoftmaxThreads);
+    mbar_init(&bars[kBarODone], 1);
+    mbar_init(&bars[kBarOFinal], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    *abort_flag = 0;
     fence_mbar_init();
   }
   __syncwarp();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
                  "r"(C::TMEM_COLS)
                  : "memory");
@@ -226,203 +341,354 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_tc_kernel(const PrefillAr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tm_s = tmem + C::S_COL, tm_o = tmem + C::O_COL;
 
-  // ---- this thread's query row
-  const int g = tid / RPH;
-  const int pos = xrow * RPH + (tid - g * RPH);  // row index in the chunk
-  const int hq = hk * a.G + hc * HPT + g;
-  const bool row_ok = pos < a.Lq;
-  const int row_limit = kv - a.Lq + pos;  // last visible slot under the causal rule
-
-  // ---- Q tile -> swizzled smem (bf16 as given; scales are applied in fp32 later)
-  {
-    const uint4 *qp = reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + pos) * D);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 w = row_ok ? __ldg(qp + c) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4 *>(smem + C::Q_OFF + (c >> 3) * (kRows * 128) + swz(tid, c & 7)) = w;
-    }
-  }
-
-  // ---- tile loop bound (per-tile causal upper bound)
+  // per-tile causal bound (the same in every role)
   const int last_pos = min(xrow * RPH + RPH, a.Lq) - 1;
   const int loop_end = a.mask_is_causal ? min(kv, kv - a.Lq + last_pos + 1) : kv;
   const int ntiles = (loop_end + kTile - 1) / kTile;
 
-  constexpr uint32_t ID_QK = idesc_bf16(kRows, kTile, 0);
-  constexpr uint32_t ID_PV = idesc_bf16(kRows, D, 1);
-  const uint32_t q_base = smem_u32(smem + C::Q_OFF), k_base = smem_u32(smem + C::K_OFF);
-  const uint32_t v_base = smem_u32(smem + C::V_OFF), p_base = smem_u32(smem + C::P_OFF);
+  if (warp < 4) {
+    // ======================= softmax warpgroup: query row t
+    const int t = tid;
+    const int g = t / RPH;
+    const int pos = xrow * RPH + (t - g * RPH);
+    const int hq = hk * a.G + hc * HPT + g;
+    const bool row_ok = pos < a.Lq;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // last visible slot of this row (the loop bound and the causal rule), -1 if none
+    int vis_last = loop_end - 1;
+    if (a.is_causal) vis_last = min(vis_last, kv - a.Lq + pos);
+    if (!row_ok) vis_last = -1;
 
-  float m = -INFINITY, l = 0.0f;
-  uint32_t phase = 0;
-  // `good`: this thread's last MMA wait completed.  The decision to stop is
-  // taken at the CTA barriers, so every thread leaves the loop at the same point.
-  bool good = true, failed = false;
-
-  for (int it = 0; it < ntiles; ++it) {
-    const int t0 = it * kTile;
-    const int n = min(kTile, loop_end - t0);
-    // ---- K / V tile: int8 -> exact bf16 (c - zp) in swizzled smem; zero rows past n
-#pragma unroll 2
-    for (int c = tid; c < kTile * CH; c += kThreads) {
-      const int s = c / CH, part = c - s * CH;
-      uint4 klo = make_uint4(0u, 0u, 0u, 0u), khi = klo, vlo = klo, vhi = klo;
-      if (s < n) {
-        const int64_t row = bh * a.S + t0 + s;
-        const uint4 kw = __ldg(reinterpret_cast<const uint4 *>(a.k + row * D) + part);
-        const uint4 vw = __ldg(reinterpret_cast<const uint4 *>(a.v + row * D) + part);
-        codes16_to_bf16(kw, __ldg(a.kz + row), klo, khi);
-        codes16_to_bf16(vw, __ldg(a.vz + row), vlo, vhi);
+    // Q row -> fp16 x 2^-sh, swizzled into shared memory
+    float qs = a.qscale;  // qscale * 2^sh
+    {
+      const uint4 *qp =
+          reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D);
+      uint32_t mx = 0;
+      if (row_ok) {
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 w = __ldg(qp + c);
+          mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                     __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+        }
       }
-      const int e0 = part * 16;  // first element of the 16 codes
-      const uint32_t reg = static_cast<uint32_t>(e0 >> 6) * (kTile * 128);
-      const int ch = (e0 & 63) >> 3;
-      *reinterpret_cast<uint4 *>(smem + C::K_OFF + reg + swz(s, ch)) = klo;
-      *reinterpret_cast<uint4 *>(smem + C::K_OFF + reg + swz(s, ch + 1)) = khi;
-      *reinterpret_cast<uint4 *>(smem + C::V_OFF + reg + swz(s, ch)) = vlo;
-      *reinterpret_cast<uint4 *>(smem + C::V_OFF + reg + swz(s, ch + 1)) = vhi;
-    }
-    if (tid < kTile) {
-      const bool in = tid < n;
-      ks_s[tid] = in ? __ldg(a.ks + bh * a.S + t0 + tid) : 0.0f;
-      vs_s[tid] = in ? __ldg(a.vs + bh * a.S + t0 + tid) : 0.0f;
+      const uint32_t mb = max(mx & 0xFFFFu, mx >> 16);  // largest |q| as bf16 bits
+      int sh = 0;
+      if (mb != 0u) sh = max(-100, min(100, static_cast<int>((mb >> 7) & 0xFFu) - 127 - 14));
+      const float f = exp2i(-sh);
+      qs = a.qscale * exp2i(sh);
+#pragma unroll 2
+      for (int c = 0; c < D / 8; ++c) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (row_ok) w = __ldg(qp + c);
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half2 h = __floats2half2_rn(bf16lo(in[i]) * f, bf16hi(in[i]) * f);
+          o[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(smem + C::Q_OFF + (c >> 3) * (kRows * 128) + swz(t, c & 7)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
     proxy_fence();
-    tc_fence_before();
-    if (__syncthreads_or(!good)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
+    mbar_arrive(&bars[kBarQ]);
 
-    // ---- S = Q K^T
-    if (tid == 0) {
+    float m = -INFINITY, l = 0.0f;
+    int E = 0;
+    bool have_e = false, ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int buf = j & 1;
+      const int t0 = j * kTile;
+      const int sb = j % kScaleBufs;
+      const uint32_t s_addr = tmem + (buf ? C::S_COL1 : C::S_COL0) + lane_base;
+      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // pass 1, per 32 columns: scores (without qs unless masked), the tile max,
+      // and the scores written back over S
+      const float4 *ks4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
+      const bool full = t0 + kTile - 1 <= vis_last;
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(s_addr + c * 32, u);
+        tmem_ld_wait();
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t aoff = static_cast<uint32_t>(k >> 2) * (kRows * 128) + (k & 3) * 32;
-        const uint32_t boff = static_cast<uint32_t>(k >> 2) * (kTile * 128) + (k & 3) * 32;
-        mma_bf16(tm_s, sdesc(q_base + aoff, 16, 1024), sdesc(k_base + boff, 16, 1024), ID_QK, k > 0);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 kk = ks4[c * 8 + q4];
+          const float kf[4] = {kk.x, kk.y, kk.z, kk.w};
+          float mk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (C::MASK && row_ok && t0 + c * 32 + q4 * 4 < loop_end) {  // in bounds: loop_end <= S, S % 4 == 0
+            const float4 mv = *reinterpret_cast<const float4 *>(a.mask + static_cast<int64_t>(pos) * a.S + t0 +
+                                                                c * 32 + q4 * 4);
+            mk[0] = mv.x;
+            mk[1] = mv.y;
+            mk[2] = mv.z;
+            mk[3] = mv.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int jj = c * 32 + q4 * 4 + e;
+            float sc = __uint_as_float(u[q4 * 4 + e]) * kf[e];
+            if (C::MASK) sc = fmaf(sc, qs, mk[e] * 1.4426950408889634f);
+            if (!full && t0 + jj > vis_last) sc = -INFINITY;
+            u[q4 * 4 + e] = __float_as_uint(sc);
+            mt = fmaxf(mt, sc);
+          }
+        }
+        tmem_st32(s_addr + c * 32, u);
       }
-      mma_commit(bar_s);
-    }
-    good = wait_mma(bar_s, phase);
-    if (!good && tid == 0) wait_mma(bar_s, phase);  // the issuer lets its MMAs finish (bounded)
-    tc_fence_after();
-
-    // ---- online softmax on this row's 64 scores
-    float sc[kTile];
-    {
-      float r32[32];
-      tmem_ld32(tm_s + lane_base, r32);
+      tmem_st_wait();
+      // running max (raised only by more than 8) and the P exponent E
+      const float mt_l = C::MASK ? mt : mt * qs;  // tile max in log2 units
+      const bool raise = mt_l > m + 8.0f;
+      const float mnew = raise ? mt_l : m;
+      const float am = (raise && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+      const float4 vm4 = *reinterpret_cast<const float4 *>(vmx_s + sb * 4);
+      const float vmx = fmaxf(fmaxf(vm4.x, vm4.y), fmaxf(vm4.z, vm4.w));
+      int Enew = E;
+      if (vmx > 0.0f) {
+        const int et = ceil_log2(vmx);  // every v_scale of the tile is <= 2^et
+        if (!have_e || et > E - 2 || et < E - 10) Enew = max(-100, min(100, et + 2));
+      }
+      const float ae = have_e ? exp2i(E - Enew) : 1.0f;
+      have_e = have_e || vmx > 0.0f;
+      const float ao = am * ae;
+      if (j > 0 && __any_sync(0xffffffffu, ao != 1.0f)) {
+        // O must hold everything up to PV_{j-1} before it is rescaled
+        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) sc[j] = r32[j];
-      tmem_ld32(tm_s + lane_base + 32, r32);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * ao);
+          tmem_st32(tmem + C::O_COL + lane_base + c * 32, o);
+        }
+        tmem_st_wait();
+      }
+      l *= am;
+      m = mnew;
+      E = Enew;
+      const float fe = exp2i(-E);
+      const float mm = m == -INFINITY ? 0.0f : m;  // a row that has seen nothing yet: every p is 0
+      // P = p * v_scale * 2^-E as fp16 pairs, written over the first 64 columns of S
+      const float4 *vs4 = reinterpret_cast<const float4 *>(vs_s + sb * kTile);
+      // pass 2: P = p * v_scale * 2^-E as fp16 pairs; slots 32c..32c+31 become the
+      // packed columns 16c..16c+15, below every column not yet read back
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(s_addr + c * 32, u);
+        tmem_ld_wait();
+        uint32_t pw[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) sc[32 + j] = r32[j];
-    }
-    float mt = -INFINITY;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 vv = vs4[c * 8 + q4];
+          const float vf[4] = {vv.x * fe, vv.y * fe, vv.z * fe, vv.w * fe};
+          float p[4];
 #pragma unroll
-    for (int j = 0; j < kTile; ++j) {
-      const int slot = t0 + j;
-      bool vis = row_ok && j < n;
-      if (a.is_causal && slot > row_limit) vis = false;
-      float s = sc[j] * (a.qscale * ks_s[j]);
-      if (a.mask && vis) s += a.mask[static_cast<int64_t>(pos) * a.S + slot] * 1.4426950408889634f;
-      sc[j] = vis ? s : -INFINITY;
-      mt = fmaxf(mt, sc[j]);
+          for (int e = 0; e < 4; ++e) {
+            const float sc = __uint_as_float(u[q4 * 4 + e]);
+            p[e] = ex2f(C::MASK ? sc - mm : fmaf(sc, qs, -mm));  // -inf -> 0
+            l += p[e];
+            p[e] *= vf[e];
+          }
+          const __half2 h0 = __floats2half2_rn(p[0], p[1]);
+          const __half2 h1 = __floats2half2_rn(p[2], p[3]);
+          pw[q4 * 2] = *reinterpret_cast<const uint32_t *>(&h0);
+          pw[q4 * 2 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+        }
+        tmem_st16(s_addr + c * 16, pw);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[kBarPFull0 + buf]);
     }
-    // raise the running max only when a score exceeds it by more than 8
-    const bool raise = mt > m + 8.0f;
-    const float mnew = raise ? mt : m;
-    const float alpha = (raise && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
-    if (it > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {  // rescale O (warp-collective TMEM access)
+    // ---- epilogue: O * 2^E / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
+    if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
+      const float inv = l > 0.0f ? exp2i(E) / l : 0.0f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(tm_o + lane_base + c * 32, o);
+        uint32_t o[32];
+        tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
+        tmem_ld_wait();
+        if (row_ok) {
+          uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] *= alpha;
-        tmem_st32(tm_o + lane_base + c * 32, o);
-      }
-    }
-    l *= alpha;
-    m = mnew;
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 v2 =
+                __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            w[i] = *reinterpret_cast<const uint32_t *>(&v2);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
 #pragma unroll
-    for (int c = 0; c < kTile / 8; ++c) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = c * 8 + 2 * u;
-        const float p0 = sc[j] == -INFINITY ? 0.0f : ex2f(sc[j] - m);
-        const float p1 = sc[j + 1] == -INFINITY ? 0.0f : ex2f(sc[j + 1] - m);
-        l += p0 + p1;
-        const float x0 = p0 * vs_s[j], x1 = p1 * vs_s[j + 1];
-        const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-        const float2 hf = __bfloat1622float2(hb);
-        const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-        hw[u] = *reinterpret_cast<const uint32_t *>(&hb);
-        lw[u] = *reinterpret_cast<const uint32_t *>(&lb);
-      }
-      *reinterpret_cast<uint4 *>(smem + C::P_OFF + swz(tid, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4 *>(smem + C::P_OFF + kRows * 128 + swz(tid, c)) =
-          make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-    proxy_fence();
-    tc_fence_before();
-    if (__syncthreads_or(!good)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-
-    // ---- O += P V
-    if (tid == 0) {
-#pragma unroll
-      for (int k = 0; k < kTile / 16; ++k) {
-        const uint64_t vd = sdesc(v_base + k * 2048, kTile * 128, 1024);
-        mma_bf16(tm_o, sdesc(p_base + k * 32, 16, 1024), vd, ID_PV, (it > 0 || k > 0) ? 1u : 0u);
-        mma_bf16(tm_o, sdesc(p_base + kRows * 128 + k * 32, 16, 1024), vd, ID_PV, 1u);
-      }
-      mma_commit(bar_o);
-    }
-    good = wait_mma(bar_o, phase);
-    if (!good && tid == 0) wait_mma(bar_o, phase);
-    tc_fence_after();
-    phase ^= 1u;
-  }
-  // every thread reaches this barrier (a break above is taken by all of them)
-  failed = __syncthreads_or(failed || !good) != 0;
-  if (failed) {
-    if (tid == 0) report(a.err, KVQ_ERR_TIMEOUT);
-  } else
-  // ---- epilogue: O / l -> bf16.  The TMEM loads are warp-collective, so every
-  // lane runs them; only rows inside the chunk store.
-  {
-    uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
-    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      tmem_ld32(tm_o + lane_base + c * 32, o);
-      if (row_ok) {
-        uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 v2 = __floats2bfloat162_rn(o[2 * j] * inv, o[2 * j + 1] * inv);
-          w[j] = *reinterpret_cast<const uint32_t *>(&v2);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
     }
+  } else if (warp < 8) {
+    // ======================= converter warpgroup
+    const int c = tid - kSoftmaxThreads;  // 0..127
+    const int part = c % C::PPR;          // which 16 codes of a slot row
+    const int sg = c / C::PPR;            // this thread's slots: sg*NCH .. sg*NCH + NCH-1
+    // placement: 64-element block and 16-byte chunk of the two halves; lanes
+    // with bit 2 set store their halves in the other order, which puts the 8
+    // lanes of every quarter-warp on 8 different 16-byte bank groups
+    const int blk = part >> 2;
+    const int ch = (part & 3) * 2;
+    const bool swap = (c & 4) != 0;
+    const int8_t *kbase = a.k + bh * a.S * D + part * 16;
+    const int8_t *vbase = a.v + bh * a.S * D + part * 16;
+    const int8_t *kzb = a.kz + bh * a.S + sg * C::NCH;
+    const int8_t *vzb = a.vz + bh * a.S + sg * C::NCH;
+
+    uint4 w[C::NCH];
+    uint32_t zw[C::NCH / 4];  // the group's zero points, 4 per word
+    auto load_tile = [&](const int8_t *base, const int8_t *zb, int t0, int n) {
+      const bool any = sg * C::NCH < n;  // the group starts inside the tile (and inside the cache)
+#pragma unroll
+      for (int i = 0; i < C::NCH / 4; ++i) zw[i] = any ? ld_u32(zb + t0 + 4 * i) : 0u;
+#pragma unroll
+      for (int r = 0; r < C::NCH; ++r) {
+        const int s = sg * C::NCH + r;
+        w[r] = s < n ? ld_codes(base + static_cast<int64_t>(t0 + s) * D)
+                     : make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+      }
+      // past the tile's end: code -128 with zero point -128 gives exactly 0
+#pragma unroll
+      for (int r = 0; r < C::NCH; ++r)
+        if (sg * C::NCH + r >= n) zw[r >> 2] = (zw[r >> 2] & ~(0xFFu << (8 * (r & 3)))) | (0x80u << (8 * (r & 3)));
+    };
+    auto store_tile = [&](int off) {
+#pragma unroll
+      for (int r = 0; r < C::NCH; ++r) {
+        const int s = sg * C::NCH + r;
+        const int zp = static_cast<int8_t>((zw[r >> 2] >> (8 * (r & 3))) & 0xFFu);
+        uint4 lo, hi;
+        codes16_to_f16(w[r], zp_const2(zp), lo, hi);
+        const uint32_t base = static_cast<uint32_t>(off + blk * (kTile * 128));
+        const uint32_t a_lo = base + swz(s, ch), a_hi = base + swz(s, ch + 1);
+        *reinterpret_cast<uint4 *>(smem + (swap ? a_hi : a_lo)) = swap ? hi : lo;
+        *reinterpret_cast<uint4 *>(smem + (swap ? a_lo : a_hi)) = swap ? lo : hi;
+      }
+    };
+    auto store_scales = [&](int sb, float ksv, float vsv) {
+      ks_s[sb * kTile + c] = ksv;
+      vs_s[sb * kTile + c] = vsv;
+      float vm = vsv;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+      if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
+    };
+    bool ok = true;
+    {  // K_0
+      const int n0 = min(kTile, loop_end);
+      load_tile(kbase, kzb, 0, n0);
+      const float ksv = c < n0 ? ld_f32(a.ks + bh * a.S + c) : 0.0f;
+      const float vsv = c < n0 ? ld_f32(a.vs + bh * a.S + c) : 0.0f;
+      store_tile(C::K_OFF);
+      store_scales(0, ksv, vsv);
+      proxy_fence();
+      mbar_arrive(&bars[kBarKFull]);
+    }
+    for (int j = 0; j < ntiles; ++j) {
+      if (j + 1 < ntiles) {  // K_{j+1}: the buffer is free once QK_j has run
+        const int t1 = (j + 1) * kTile;
+        const int n1 = min(kTile, loop_end - t1);
+        load_tile(kbase, kzb, t1, n1);
+        const float ksv = c < n1 ? ld_f32(a.ks + bh * a.S + t1 + c) : 0.0f;
+        const float vsv = c < n1 ? ld_f32(a.vs + bh * a.S + t1 + c) : 0.0f;
+        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarKEmpty], j & 1, abort_flag));
+        if (!ok) break;
+        store_tile(C::K_OFF);
+        store_scales((j + 1) % kScaleBufs, ksv, vsv);
+        proxy_fence();
+        mbar_arrive(&bars[kBarKFull]);
+      }
+      {  // V_j: the buffer is free once PV_{j-1} has run
+        const int t0 = j * kTile;
+        load_tile(vbase, vzb, t0, min(kTile, loop_end - t0));
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        store_tile(C::V_OFF);
+        proxy_fence();
+        mbar_arrive(&bars[kBarVFull]);
+      }
+    }
+  } else {
+    // ======================= MMA warp: lane 0 issues
+    if (lane == 0) {
+      constexpr uint32_t ID_QK = idesc_f16(kRows, kTile, 0);
+      constexpr uint32_t ID_PV = idesc_f16(kRows, D, 1);
+      const uint32_t q_base = smem_u32(smem + C::Q_OFF), k_base = smem_u32(smem + C::K_OFF);
+      const uint32_t v_base = smem_u32(smem + C::V_OFF);
+      // Q and K regions share the [128 rows x 128 B] block shape (kRows == kTile)
+      static_assert(kRows == kTile, "Q and K block strides");
+      auto issue_qk = [&](int j) {
+        const uint32_t d = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = static_cast<uint32_t>(k >> 2) * (kRows * 128) + (k & 3) * 32;
+          mma_ss(d, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), ID_QK, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[kBarSFull0 + (j & 1)]);
+        mma_commit(&bars[kBarKEmpty]);
+      };
+      bool ok = wait_phase(&bars[kBarQ], 0, abort_flag);
+      if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+      }
+      for (int j = 0; j < ntiles && ok; ++j) {
+        if (j + 1 < ntiles) {
+          ok = wait_phase(&bars[kBarKFull], (j + 1) & 1, abort_flag);
+          // S buffer (j+1)&1 holds P_{j-1} until PV_{j-1} has run
+          if (ok && j >= 1) ok = wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(j + 1);
+        }
+        ok = wait_phase(&bars[kBarVFull], j & 1, abort_flag);
+        if (ok) ok = wait_phase(&bars[kBarPFull0 + (j & 1)], (j >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k)  // 16 slots = 8 packed TMEM columns of P
+          mma_ts(tmem + C::O_COL, p_tmem + k * 8, sdesc(v_base + k * 2048, kTile * 128, 1024), ID_PV,
+                 (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&bars[kBarODone]);
+        mma_commit(&bars[kBarVEmpty]);
+        if (j + 1 == ntiles) mma_commit(&bars[kBarOFinal]);
+      }
+      if (!ok) {  // everything issued finishes before TMEM is released
+        mma_commit(&bars[kBarDrain]);
+        mbar_wait_bounded(&bars[kBarDrain], 0);
+      }
+    }
+    __syncwarp();
   }
+
+  // ---- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (tid == 0 && *abort_flag) report(a.err, KVQ_ERR_TIMEOUT);
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                  : "memory");
@@ -431,9 +697,9 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_tc_kernel(const PrefillAr
 
 inline int hpt_for(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
 
-template <int D, int HPT>
+template <int D, int HPT, bool MASK>
 int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
-  using C = Cfg<D, HPT>;
+  using C = Cfg<D, HPT, MASK>;
   if (const int st = ensure_smem<C>(prefill_tc_kernel<C>, C::SMEM)) return st;
   a.nhc = a.G / HPT;
   dim3 grid((a.Lq + C::RPH - 1) / C::RPH, a.Hkv * a.nhc, a.B);
@@ -441,13 +707,18 @@ int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   return launch_status();
 }
 
+template <int D, bool MASK>
+int dispatch_hpt(const PrefillArgs &a, cudaStream_t s) {
+  switch (hpt_for(a.G)) {
+    case 4: return launch_prefill_tc<D, 4, MASK>(a, s);
+    case 2: return launch_prefill_tc<D, 2, MASK>(a, s);
+    default: return launch_prefill_tc<D, 1, MASK>(a, s);
+  }
+}
+
 template <int D>
 int dispatch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
-  switch (hpt_for(a.G)) {
-    case 4: return launch_prefill_tc<D, 4>(a, s);
-    case 2: return launch_prefill_tc<D, 2>(a, s);
-    default: return launch_prefill_tc<D, 1>(a, s);
-  }
+  return a.mask ? dispatch_hpt<D, true>(a, s) : dispatch_hpt<D, false>(a, s);
 }
 
 }  // namespace tc
