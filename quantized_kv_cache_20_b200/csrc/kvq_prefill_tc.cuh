@@ -10,12 +10,14 @@
 //
 // Design.  One CTA holds 128 query rows of one kv head (HPT q heads x RPH
 // positions with GQA, so every K/V tile is dequantized once for all of them)
-// and runs three roles, connected by mbarriers:
+// and runs four roles, connected by mbarriers:
 //   - softmax warpgroup (warps 0-3): thread t owns query row t, i.e. TMEM lane t;
-//   - converter warpgroup (warps 4-7): turns the int8 codes of 128-slot K and
-//     V tiles into fp16 in the 128-byte-swizzled shared-memory layout the
-//     tensor core reads;
-//   - MMA warp (warp 8): one thread issues every tcgen05.mma.
+//   - K and V converter warpgroups (warps 4-7, 8-11): turn the int8 codes of
+//     128-slot K and V tiles into fp16 in the 128-byte-swizzled shared-memory
+//     layout the tensor core reads; each issues the loads of its next tile as
+//     soon as it has stored the current one, so the memory latency overlaps
+//     the wait for the tensor core to release the buffer;
+//   - MMA warp (warp 12): one thread issues every tcgen05.mma.
 // Tensor-core work per tile j:  S_j = Q K_j^T (M 128, N 128) into one of two
 // TMEM buffers; the softmax writes P_j back over the columns of S_j it came
 // from, and O += P_j V_j takes P from TMEM (A operand in tensor memory) and V
@@ -59,12 +61,12 @@ namespace tc {
 constexpr int kRows = 128;  // query rows per CTA (tcgen05 M)
 constexpr int kTile = 128;  // slots per K/V tile (N of Q K^T, K of P V)
 constexpr int kSoftmaxThreads = 128;
-constexpr int kConvThreads = 128;
-constexpr int kThreads = kSoftmaxThreads + kConvThreads + 32;
-constexpr int kMmaWarp = 8;
+constexpr int kConvThreads = 128;  // per converter warpgroup (one for K, one for V)
+constexpr int kThreads = kSoftmaxThreads + 2 * kConvThreads + 32;
+constexpr int kMmaWarp = 12;
 constexpr int kScaleBufs = 3;  // k_scale / v_scale tile buffers
-// registers per thread: 9 warps, one SM sub-partition holds three of them
-constexpr int kRegsLaunch = 168;
+// registers per thread: 13 warps, one SM sub-partition holds four of them
+constexpr int kRegsLaunch = 128;
 
 struct PrefillArgs {
   const uint16_t *q;
@@ -90,9 +92,9 @@ struct PrefillArgs {
 // that reason: O may still be a PV or two behind the softmax).
 enum : int {
   kBarQ = 0,   // Q tile written (softmax warpgroup, 128 arrivals)
-  kBarKFull,   // K tile written (converters, 128 arrivals)
+  kBarKFull,   // K tile written (K converters, 128 arrivals)
   kBarKEmpty,  // QK done with the K tile (commit)
-  kBarVFull,   // V tile written (converters, 128 arrivals)
+  kBarVFull,   // V tile written (V converters, 128 arrivals)
   kBarVEmpty,  // PV done with the V tile (commit)
   kBarSFull0,  // S buffer 0 / 1 computed (commit)
   kBarSFull1,
@@ -118,8 +120,8 @@ struct Cfg {
   static constexpr int VS_OFF = KS_OFF + kScaleBufs * kTile * 4;
   static constexpr int VMX_OFF = VS_OFF + kScaleBufs * kTile * 4;  // float [kScaleBufs][4]
   static constexpr int BAR_OFF = VMX_OFF + kScaleBufs * 16;
-  static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag
-  static constexpr int SMEM = MISC_OFF + 16 + 1024;        // + slack to align the base to 1024
+  static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag, qs, 4 x max|q|
+  static constexpr int SMEM = MISC_OFF + 32 + 1024;        // + slack to align the base to 1024
   static constexpr int S_COL0 = 0, S_COL1 = kTile, O_COL = 2 * kTile;
   static constexpr int TMEM_COLS = 512;
   static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
@@ -290,8 +292,498 @@ KVQ_DEVINL uint32_t zp_const2(int zp) {
   return h | (h << 16);
 }
 
+// State shared by the roles (each role runs in its own function, so that the
+// register allocation of one does not constrain the others).
+struct Ctx {
+  uint8_t *smem;  // 1024-byte aligned dynamic shared memory
+  uint32_t tmem;  // TMEM base address
+  int kv, loop_end, ntiles;
+};
+
+// softmax warpgroup: query row t = threadIdx.x, TMEM lane t
 template <class C>
-__global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const PrefillArgs a) {
+__device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
+  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
+  (void)HPT;
+  (void)RPH;
+  uint8_t *smem = x.smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
+  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
+  float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
+  float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
+  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
+  (void)qs_s;
+  (void)qmax_s;
+  (void)ks_s;
+  (void)vs_s;
+  (void)vmx_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)lane;
+  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
+  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
+  (void)xrow;
+  (void)hc;
+  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+  (void)bh;
+  const uint32_t tmem = x.tmem;
+  (void)tmem;
+  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
+  (void)kv;
+  // ======================= softmax warpgroup: query row t
+  const int t = tid;
+  const int g = t / RPH;
+  const int pos = xrow * RPH + (t - g * RPH);
+  const int hq = hk * a.G + hc * HPT + g;
+  const bool row_ok = pos < a.Lq;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  // last visible slot of this row (the loop bound and the causal rule), -1 if none
+  int vis_last = loop_end - 1;
+  if (a.is_causal) vis_last = min(vis_last, kv - a.Lq + pos);
+  if (!row_ok) vis_last = -1;
+
+  // Q -> fp16 x 2^-sh, swizzled into shared memory; sh is one power of two for
+  // the CTA, chosen so that the largest |q| lands in [2^14, 2^15)
+  const uint4 *qp =
+      reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D);
+  {
+    uint32_t mx = 0;
+    if (row_ok) {
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 w = __ldg(qp + c);
+        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                   __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+      }
+    }
+    const uint32_t mw = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    if (lane == 0) qmax_s[warp] = mw;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+  const uint32_t mb = max(max(qmax_s[0], qmax_s[1]), max(qmax_s[2], qmax_s[3]));  // largest |q| (bf16 bits)
+  int sh = 0;
+  if (mb != 0u) sh = max(-100, min(100, static_cast<int>((mb >> 7) & 0xFFu) - 127 - 14));
+  const float qs = a.qscale * exp2i(sh);
+  {
+    const float f = exp2i(-sh);
+#pragma unroll 2
+    for (int c = 0; c < D / 8; ++c) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok) w = __ldg(qp + c);
+      const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 h = __floats2half2_rn(bf16lo(in[i]) * f, bf16hi(in[i]) * f);
+        o[i] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      *reinterpret_cast<uint4 *>(smem + C::Q_OFF + (c >> 3) * (kRows * 128) + swz(t, c & 7)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (t == 0) *qs_s = qs;
+  proxy_fence();
+  mbar_arrive(&bars[kBarQ]);
+
+  // Scores in the log2 domain: x = S_raw * kq (kq = k_scale * qs per slot,
+  // prepared by the converters) [+ mask * log2e].  With the running max m and
+  // the P exponent E, p' = 2^(x - m - E) = p * 2^-E; P = p' * v_scale, and
+  // l and O are both kept in units of 2^-E, so out = O / l.
+  float m = -INFINITY, l = 0.0f;
+  int E = 0;
+  bool have_e = false, ok = true;
+  for (int j = 0; j < ntiles; ++j) {
+    const int buf = j & 1;
+    const int t0 = j * kTile;
+    const int sb = j % kScaleBufs;
+    const uint32_t s_addr = tmem + (buf ? C::S_COL1 : C::S_COL0) + lane_base;
+    const float4 *kq4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
+    const float4 *vs4 = reinterpret_cast<const float4 *>(vs_s + sb * kTile);
+    const bool full = t0 + kTile - 1 <= vis_last;  // every slot of the tile visible to this row
+    ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag));
+    if (!ok) break;
+    tc_fence_after();
+    // pass 1, per 32 columns: the tile max (masked scores are written back over S)
+    float mt = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      tmem_ld32(s_addr + c * 32, u);
+      tmem_ld_wait();
+      if constexpr (C::MASK) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int j0 = t0 + c * 32 + q4 * 4;
+          const float4 kk = kq4[c * 8 + q4];
+          float4 mv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (row_ok && j0 < loop_end)  // in bounds: loop_end <= S, S % 4 == 0
+            mv = *reinterpret_cast<const float4 *>(a.mask + static_cast<int64_t>(pos) * a.S + j0);
+          const float kf[4] = {kk.x, kk.y, kk.z, kk.w}, mf[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float x = fmaf(__uint_as_float(u[q4 * 4 + e]), kf[e], mf[e] * 1.4426950408889634f);
+            if (!full && j0 + e > vis_last) x = -INFINITY;
+            u[q4 * 4 + e] = __float_as_uint(x);
+            mt = fmaxf(mt, x);
+          }
+        }
+        tmem_st32(s_addr + c * 32, u);
+      } else if (full) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent chains
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 kk = kq4[c * 8 + q4];
+          m4[0] = fmaxf(m4[0], __uint_as_float(u[q4 * 4]) * kk.x);
+          m4[1] = fmaxf(m4[1], __uint_as_float(u[q4 * 4 + 1]) * kk.y);
+          m4[2] = fmaxf(m4[2], __uint_as_float(u[q4 * 4 + 2]) * kk.z);
+          m4[3] = fmaxf(m4[3], __uint_as_float(u[q4 * 4 + 3]) * kk.w);
+        }
+        mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+      } else {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int j0 = t0 + c * 32 + q4 * 4;
+          const float4 kk = kq4[c * 8 + q4];
+          const float kf[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (j0 + e <= vis_last) mt = fmaxf(mt, __uint_as_float(u[q4 * 4 + e]) * kf[e]);
+        }
+      }
+    }
+    if constexpr (C::MASK) tmem_st_wait();
+    // running max (raised only by more than 8) and the P exponent E
+    const bool raise = mt > m + 8.0f;
+    const float mnew = raise ? mt : m;
+    const float am = (raise && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+    const float4 vm4 = *reinterpret_cast<const float4 *>(vmx_s + sb * 4);
+    const float vmx = fmaxf(fmaxf(vm4.x, vm4.y), fmaxf(vm4.z, vm4.w));
+    int Enew = E;
+    if (vmx > 0.0f) {
+      const int et = ceil_log2(vmx);  // every v_scale of the tile is <= 2^et
+      if (!have_e || et > E - 2 || et < E - 10) Enew = max(-100, min(100, et + 2));
+    }
+    const float ae = have_e ? exp2i(E - Enew) : 1.0f;
+    have_e = have_e || vmx > 0.0f;
+    const float ao = am * ae;
+    if (j > 0 && __any_sync(0xffffffffu, ao != 1.0f)) {
+      // O must hold everything up to PV_{j-1} before it is rescaled
+      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * ao);
+        tmem_st32(tmem + C::O_COL + lane_base + c * 32, o);
+      }
+      tmem_st_wait();
+    }
+    l *= ao;
+    m = mnew;
+    E = Enew;
+    // a row that has seen nothing yet has m = -inf: every p' is then 0
+    const float me = (m == -INFINITY ? 0.0f : m) + static_cast<float>(E);
+    // pass 2: P = p' * v_scale as fp16 pairs; slots 32c..32c+31 become the
+    // packed columns 16c..16c+15, below every column not yet read back
+    float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent chains for the row sum
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      tmem_ld32(s_addr + c * 32, u);
+      tmem_ld_wait();
+      uint32_t pw[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const int j0 = t0 + c * 32 + q4 * 4;
+        const float4 kk = kq4[c * 8 + q4];
+        const float4 vv = vs4[c * 8 + q4];
+        const float kf[4] = {kk.x, kk.y, kk.z, kk.w}, vf[4] = {vv.x, vv.y, vv.z, vv.w};
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float r = __uint_as_float(u[q4 * 4 + e]);
+          float x = C::MASK ? r - me : fmaf(r, kf[e], -me);
+          if (!C::MASK && !full && j0 + e > vis_last) x = -INFINITY;
+          p[e] = ex2f(x);  // -inf -> 0
+          l4[e] += p[e];
+          p[e] *= vf[e];
+        }
+        const __half2 h0 = __floats2half2_rn(p[0], p[1]);
+        const __half2 h1 = __floats2half2_rn(p[2], p[3]);
+        pw[q4 * 2] = *reinterpret_cast<const uint32_t *>(&h0);
+        pw[q4 * 2 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+      }
+      tmem_st16(s_addr + c * 16, pw);
+    }
+    l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(&bars[kBarPFull0 + buf]);
+  }
+  // ---- epilogue: O / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
+  if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag));
+  if (ok) {
+    tc_fence_after();
+    uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
+    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
+      tmem_ld_wait();
+      if (row_ok) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat162 v2 =
+              __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          w[i] = *reinterpret_cast<const uint32_t *>(&v2);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+  }
+}
+
+// converter warpgroups: K (warps 4-7), V (warps 8-11)
+template <class C>
+__device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
+  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
+  (void)HPT;
+  (void)RPH;
+  uint8_t *smem = x.smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
+  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
+  float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
+  float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
+  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
+  (void)qs_s;
+  (void)qmax_s;
+  (void)ks_s;
+  (void)vs_s;
+  (void)vmx_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)lane;
+  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
+  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
+  (void)xrow;
+  (void)hc;
+  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+  (void)bh;
+  const uint32_t tmem = x.tmem;
+  (void)tmem;
+  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
+  (void)kv;
+  // ======================= converter warpgroups: K (warps 4-7), V (warps 8-11)
+  const bool is_k = warp < 8;
+  const int c = tid - kSoftmaxThreads - (is_k ? 0 : kConvThreads);  // 0..127
+  const int part = c % C::PPR;  // which 16 codes of a slot row
+  const int sg = c / C::PPR;    // this thread's slots: sg*NCH .. sg*NCH + NCH-1
+  // placement: 64-element block and 16-byte chunk of the two halves; lanes
+  // with bit 2 set store their halves in the other order, which puts the 8
+  // lanes of every quarter-warp on 8 different 16-byte bank groups
+  const int blk = part >> 2;
+  const int ch = (part & 3) * 2;
+  const bool swap = (c & 4) != 0;
+  const int8_t *base = (is_k ? a.k : a.v) + bh * a.S * D + part * 16;
+  const int8_t *zb = (is_k ? a.kz : a.vz) + bh * a.S + sg * C::NCH;
+  const int off = is_k ? C::K_OFF : C::V_OFF;
+
+  // Each thread streams its chunks through a window of W registers: right
+  // after chunk r of tile j is converted and stored, the load of the chunk W
+  // places later (in this tile or the next) is issued into the same
+  // registers, so loads are in flight while earlier chunks are converted and
+  // while the tensor core still holds the buffer.
+  constexpr int W = C::NCH < 8 ? C::NCH : 8;
+  static_assert(C::NCH % W == 0, "window");
+  uint4 w[W];
+  uint32_t zw[C::NCH / 4], zn[C::NCH / 4];  // zero points of this / the next tile, 4 per word
+  auto load_chunk = [&](int r, int t0, int n) {
+    const int s = sg * C::NCH + r;
+    w[r % W] = s < n ? ld_codes(base + static_cast<int64_t>(t0 + s) * D)
+                     : make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+  };
+  auto load_zp = [&](uint32_t (&z)[C::NCH / 4], int t0, int n) {
+    const bool any = sg * C::NCH < n;  // the group starts inside the tile (and inside the cache)
+#pragma unroll
+    for (int i = 0; i < C::NCH / 4; ++i) z[i] = any ? ld_u32(zb + t0 + 4 * i) : 0u;
+    // past the tile's end: code -128 with zero point -128 gives exactly 0
+#pragma unroll
+    for (int r = 0; r < C::NCH; ++r)
+      if (sg * C::NCH + r >= n) z[r >> 2] = (z[r >> 2] & ~(0xFFu << (8 * (r & 3)))) | (0x80u << (8 * (r & 3)));
+  };
+  auto tile_n = [&](int j) { return min(kTile, loop_end - j * kTile); };
+  // convert + store this tile's chunks, loading W chunks ahead behind them
+  auto convert_tile = [&](int j) {
+    const bool next = j + 1 < ntiles;
+    const int t0 = j * kTile, n0 = tile_n(j);
+    const int t1 = (j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
+#pragma unroll
+    for (int r = 0; r < C::NCH; ++r) {
+      const int s = sg * C::NCH + r;
+      const int zp = static_cast<int8_t>((zw[r >> 2] >> (8 * (r & 3))) & 0xFFu);
+      uint4 lo, hi;
+      codes16_to_f16(w[r % W], zp_const2(zp), lo, hi);
+      const uint32_t o = static_cast<uint32_t>(off + blk * (kTile * 128));
+      const uint32_t a_lo = o + swz(s, ch), a_hi = o + swz(s, ch + 1);
+      *reinterpret_cast<uint4 *>(smem + (swap ? a_hi : a_lo)) = swap ? hi : lo;
+      *reinterpret_cast<uint4 *>(smem + (swap ? a_lo : a_hi)) = swap ? lo : hi;
+      if (r + W < C::NCH)
+        load_chunk(r + W, t0, n0);
+      else if (next)
+        load_chunk(r + W - C::NCH, t1, n1);
+    }
+#pragma unroll
+    for (int i = 0; i < C::NCH / 4; ++i) zw[i] = zn[i];
+  };
+  bool ok = true;
+  {
+    const int n0 = tile_n(0);
+#pragma unroll
+    for (int r = 0; r < W; ++r) load_chunk(r, 0, n0);
+    load_zp(zw, 0, n0);
+  }
+  if (is_k) {
+    // K tiles, and with each the per-slot k_scale * qs, v_scale and max v_scale
+    float qs = 0.0f;
+    float ksv = c < tile_n(0) ? ld_f32(a.ks + bh * a.S + c) : 0.0f;
+    float vsv = c < tile_n(0) ? ld_f32(a.vs + bh * a.S + c) : 0.0f;
+    for (int j = 0; j < ntiles; ++j) {
+      float ksn = 0.0f, vsn = 0.0f;
+      if (j + 1 < ntiles) {
+        const int t1 = (j + 1) * kTile, n1 = tile_n(j + 1);
+        load_zp(zn, t1, n1);
+        ksn = c < n1 ? ld_f32(a.ks + bh * a.S + t1 + c) : 0.0f;
+        vsn = c < n1 ? ld_f32(a.vs + bh * a.S + t1 + c) : 0.0f;
+      }
+      // the buffer is free once QK_{j-1} has run; qs is published with Q
+      ok = __all_sync(0xffffffffu, j == 0 ? wait_phase(&bars[kBarQ], 0, abort_flag)
+                                          : wait_phase(&bars[kBarKEmpty], (j - 1) & 1, abort_flag));
+      if (!ok) break;
+      if (j == 0) qs = *qs_s;
+      convert_tile(j);
+      const int sb = j % kScaleBufs;
+      ks_s[sb * kTile + c] = ksv * qs;
+      vs_s[sb * kTile + c] = vsv;
+      float vm = vsv;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+      if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
+      proxy_fence();
+      mbar_arrive(&bars[kBarKFull]);
+      ksv = ksn;
+      vsv = vsn;
+    }
+  } else {
+    for (int j = 0; j < ntiles; ++j) {
+      if (j + 1 < ntiles) load_zp(zn, (j + 1) * kTile, tile_n(j + 1));
+      if (j > 0) {  // the buffer is free once PV_{j-1} has run
+        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      convert_tile(j);
+      proxy_fence();
+      mbar_arrive(&bars[kBarVFull]);
+    }
+  }
+}
+
+// MMA warp: lane 0 issues
+template <class C>
+__device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
+  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
+  (void)HPT;
+  (void)RPH;
+  uint8_t *smem = x.smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
+  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
+  float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
+  float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
+  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
+  (void)qs_s;
+  (void)qmax_s;
+  (void)ks_s;
+  (void)vs_s;
+  (void)vmx_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)lane;
+  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
+  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
+  (void)xrow;
+  (void)hc;
+  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+  (void)bh;
+  const uint32_t tmem = x.tmem;
+  (void)tmem;
+  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
+  (void)kv;
+  // ======================= MMA warp: lane 0 issues
+  if (lane == 0) {
+    constexpr uint32_t ID_QK = idesc_f16(kRows, kTile, 0);
+    constexpr uint32_t ID_PV = idesc_f16(kRows, D, 1);
+    const uint32_t q_base = smem_u32(smem + C::Q_OFF), k_base = smem_u32(smem + C::K_OFF);
+    const uint32_t v_base = smem_u32(smem + C::V_OFF);
+    // Q and K regions share the [128 rows x 128 B] block shape (kRows == kTile)
+    static_assert(kRows == kTile, "Q and K block strides");
+    auto issue_qk = [&](int j) {
+      const uint32_t d = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = static_cast<uint32_t>(k >> 2) * (kRows * 128) + (k & 3) * 32;
+        mma_ss(d, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), ID_QK, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars[kBarSFull0 + (j & 1)]);
+      mma_commit(&bars[kBarKEmpty]);
+    };
+    bool ok = wait_phase(&bars[kBarQ], 0, abort_flag);
+    if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0);
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
+      if (j + 1 < ntiles) {
+        ok = wait_phase(&bars[kBarKFull], (j + 1) & 1, abort_flag);
+        // S buffer (j+1)&1 holds P_{j-1} until PV_{j-1} has run
+        if (ok && j >= 1) ok = wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(j + 1);
+      }
+      ok = wait_phase(&bars[kBarVFull], j & 1, abort_flag);
+      if (ok) ok = wait_phase(&bars[kBarPFull0 + (j & 1)], (j >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t p_tmem = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
+#pragma unroll
+      for (int k = 0; k < kTile / 16; ++k)  // 16 slots = 8 packed TMEM columns of P
+        mma_ts(tmem + C::O_COL, p_tmem + k * 8, sdesc(v_base + k * 2048, kTile * 128, 1024), ID_PV,
+               (j > 0 || k > 0) ? 1u : 0u);
+      mma_commit(&bars[kBarODone]);
+      mma_commit(&bars[kBarVEmpty]);
+      if (j + 1 == ntiles) mma_commit(&bars[kBarOFinal]);
+    }
+    if (!ok) {  // everything issued finishes before TMEM is released
+      mma_commit(&bars[kBarDrain]);
+      mbar_wait_bounded(&bars[kBarDrain], 0);
+    }
+  }
+  __syncwarp();
+}
+
+template <class C>
+__global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant__ PrefillArgs a) {
   constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (the 128-byte swizzle is a function of address bits 4-9)
@@ -299,6 +791,8 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const PrefillArgs a) 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
+  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
   float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
   float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
   float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
@@ -347,342 +841,13 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const PrefillArgs a) 
   const int loop_end = a.mask_is_causal ? min(kv, kv - a.Lq + last_pos + 1) : kv;
   const int ntiles = (loop_end + kTile - 1) / kTile;
 
-  if (warp < 4) {
-    // ======================= softmax warpgroup: query row t
-    const int t = tid;
-    const int g = t / RPH;
-    const int pos = xrow * RPH + (t - g * RPH);
-    const int hq = hk * a.G + hc * HPT + g;
-    const bool row_ok = pos < a.Lq;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    // last visible slot of this row (the loop bound and the causal rule), -1 if none
-    int vis_last = loop_end - 1;
-    if (a.is_causal) vis_last = min(vis_last, kv - a.Lq + pos);
-    if (!row_ok) vis_last = -1;
-
-    // Q row -> fp16 x 2^-sh, swizzled into shared memory
-    float qs = a.qscale;  // qscale * 2^sh
-    {
-      const uint4 *qp =
-          reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D);
-      uint32_t mx = 0;
-      if (row_ok) {
-#pragma unroll 4
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 w = __ldg(qp + c);
-          mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
-                                     __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
-        }
-      }
-      const uint32_t mb = max(mx & 0xFFFFu, mx >> 16);  // largest |q| as bf16 bits
-      int sh = 0;
-      if (mb != 0u) sh = max(-100, min(100, static_cast<int>((mb >> 7) & 0xFFu) - 127 - 14));
-      const float f = exp2i(-sh);
-      qs = a.qscale * exp2i(sh);
-#pragma unroll 2
-      for (int c = 0; c < D / 8; ++c) {
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (row_ok) w = __ldg(qp + c);
-        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __half2 h = __floats2half2_rn(bf16lo(in[i]) * f, bf16hi(in[i]) * f);
-          o[i] = *reinterpret_cast<const uint32_t *>(&h);
-        }
-        *reinterpret_cast<uint4 *>(smem + C::Q_OFF + (c >> 3) * (kRows * 128) + swz(t, c & 7)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-    proxy_fence();
-    mbar_arrive(&bars[kBarQ]);
-
-    float m = -INFINITY, l = 0.0f;
-    int E = 0;
-    bool have_e = false, ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int buf = j & 1;
-      const int t0 = j * kTile;
-      const int sb = j % kScaleBufs;
-      const uint32_t s_addr = tmem + (buf ? C::S_COL1 : C::S_COL0) + lane_base;
-      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      // pass 1, per 32 columns: scores (without qs unless masked), the tile max,
-      // and the scores written back over S
-      const float4 *ks4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
-      const bool full = t0 + kTile - 1 <= vis_last;
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32(s_addr + c * 32, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 kk = ks4[c * 8 + q4];
-          const float kf[4] = {kk.x, kk.y, kk.z, kk.w};
-          float mk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          if (C::MASK && row_ok && t0 + c * 32 + q4 * 4 < loop_end) {  // in bounds: loop_end <= S, S % 4 == 0
-            const float4 mv = *reinterpret_cast<const float4 *>(a.mask + static_cast<int64_t>(pos) * a.S + t0 +
-                                                                c * 32 + q4 * 4);
-            mk[0] = mv.x;
-            mk[1] = mv.y;
-            mk[2] = mv.z;
-            mk[3] = mv.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int jj = c * 32 + q4 * 4 + e;
-            float sc = __uint_as_float(u[q4 * 4 + e]) * kf[e];
-            if (C::MASK) sc = fmaf(sc, qs, mk[e] * 1.4426950408889634f);
-            if (!full && t0 + jj > vis_last) sc = -INFINITY;
-            u[q4 * 4 + e] = __float_as_uint(sc);
-            mt = fmaxf(mt, sc);
-          }
-        }
-        tmem_st32(s_addr + c * 32, u);
-      }
-      tmem_st_wait();
-      // running max (raised only by more than 8) and the P exponent E
-      const float mt_l = C::MASK ? mt : mt * qs;  // tile max in log2 units
-      const bool raise = mt_l > m + 8.0f;
-      const float mnew = raise ? mt_l : m;
-      const float am = (raise && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
-      const float4 vm4 = *reinterpret_cast<const float4 *>(vmx_s + sb * 4);
-      const float vmx = fmaxf(fmaxf(vm4.x, vm4.y), fmaxf(vm4.z, vm4.w));
-      int Enew = E;
-      if (vmx > 0.0f) {
-        const int et = ceil_log2(vmx);  // every v_scale of the tile is <= 2^et
-        if (!have_e || et > E - 2 || et < E - 10) Enew = max(-100, min(100, et + 2));
-      }
-      const float ae = have_e ? exp2i(E - Enew) : 1.0f;
-      have_e = have_e || vmx > 0.0f;
-      const float ao = am * ae;
-      if (j > 0 && __any_sync(0xffffffffu, ao != 1.0f)) {
-        // O must hold everything up to PV_{j-1} before it is rescaled
-        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * ao);
-          tmem_st32(tmem + C::O_COL + lane_base + c * 32, o);
-        }
-        tmem_st_wait();
-      }
-      l *= am;
-      m = mnew;
-      E = Enew;
-      const float fe = exp2i(-E);
-      const float mm = m == -INFINITY ? 0.0f : m;  // a row that has seen nothing yet: every p is 0
-      // P = p * v_scale * 2^-E as fp16 pairs, written over the first 64 columns of S
-      const float4 *vs4 = reinterpret_cast<const float4 *>(vs_s + sb * kTile);
-      // pass 2: P = p * v_scale * 2^-E as fp16 pairs; slots 32c..32c+31 become the
-      // packed columns 16c..16c+15, below every column not yet read back
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32(s_addr + c * 32, u);
-        tmem_ld_wait();
-        uint32_t pw[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 vv = vs4[c * 8 + q4];
-          const float vf[4] = {vv.x * fe, vv.y * fe, vv.z * fe, vv.w * fe};
-          float p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float sc = __uint_as_float(u[q4 * 4 + e]);
-            p[e] = ex2f(C::MASK ? sc - mm : fmaf(sc, qs, -mm));  // -inf -> 0
-            l += p[e];
-            p[e] *= vf[e];
-          }
-          const __half2 h0 = __floats2half2_rn(p[0], p[1]);
-          const __half2 h1 = __floats2half2_rn(p[2], p[3]);
-          pw[q4 * 2] = *reinterpret_cast<const uint32_t *>(&h0);
-          pw[q4 * 2 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
-        }
-        tmem_st16(s_addr + c * 16, pw);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[kBarPFull0 + buf]);
-    }
-    // ---- epilogue: O * 2^E / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
-    if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag));
-    if (ok) {
-      tc_fence_after();
-      uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
-      const float inv = l > 0.0f ? exp2i(E) / l : 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + C::O_COL + lane_base + c * 32, o);
-        tmem_ld_wait();
-        if (row_ok) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 v2 =
-                __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            w[i] = *reinterpret_cast<const uint32_t *>(&v2);
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
-      }
-    }
-  } else if (warp < 8) {
-    // ======================= converter warpgroup
-    const int c = tid - kSoftmaxThreads;  // 0..127
-    const int part = c % C::PPR;          // which 16 codes of a slot row
-    const int sg = c / C::PPR;            // this thread's slots: sg*NCH .. sg*NCH + NCH-1
-    // placement: 64-element block and 16-byte chunk of the two halves; lanes
-    // with bit 2 set store their halves in the other order, which puts the 8
-    // lanes of every quarter-warp on 8 different 16-byte bank groups
-    const int blk = part >> 2;
-    const int ch = (part & 3) * 2;
-    const bool swap = (c & 4) != 0;
-    const int8_t *kbase = a.k + bh * a.S * D + part * 16;
-    const int8_t *vbase = a.v + bh * a.S * D + part * 16;
-    const int8_t *kzb = a.kz + bh * a.S + sg * C::NCH;
-    const int8_t *vzb = a.vz + bh * a.S + sg * C::NCH;
-
-    uint4 w[C::NCH];
-    uint32_t zw[C::NCH / 4];  // the group's zero points, 4 per word
-    auto load_tile = [&](const int8_t *base, const int8_t *zb, int t0, int n) {
-      const bool any = sg * C::NCH < n;  // the group starts inside the tile (and inside the cache)
-#pragma unroll
-      for (int i = 0; i < C::NCH / 4; ++i) zw[i] = any ? ld_u32(zb + t0 + 4 * i) : 0u;
-#pragma unroll
-      for (int r = 0; r < C::NCH; ++r) {
-        const int s = sg * C::NCH + r;
-        w[r] = s < n ? ld_codes(base + static_cast<int64_t>(t0 + s) * D)
-                     : make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
-      }
-      // past the tile's end: code -128 with zero point -128 gives exactly 0
-#pragma unroll
-      for (int r = 0; r < C::NCH; ++r)
-        if (sg * C::NCH + r >= n) zw[r >> 2] = (zw[r >> 2] & ~(0xFFu << (8 * (r & 3)))) | (0x80u << (8 * (r & 3)));
-    };
-    auto store_tile = [&](int off) {
-#pragma unroll
-      for (int r = 0; r < C::NCH; ++r) {
-        const int s = sg * C::NCH + r;
-        const int zp = static_cast<int8_t>((zw[r >> 2] >> (8 * (r & 3))) & 0xFFu);
-        uint4 lo, hi;
-        codes16_to_f16(w[r], zp_const2(zp), lo, hi);
-        const uint32_t base = static_cast<uint32_t>(off + blk * (kTile * 128));
-        const uint32_t a_lo = base + swz(s, ch), a_hi = base + swz(s, ch + 1);
-        *reinterpret_cast<uint4 *>(smem + (swap ? a_hi : a_lo)) = swap ? hi : lo;
-        *reinterpret_cast<uint4 *>(smem + (swap ? a_lo : a_hi)) = swap ? lo : hi;
-      }
-    };
-    auto store_scales = [&](int sb, float ksv, float vsv) {
-      ks_s[sb * kTile + c] = ksv;
-      vs_s[sb * kTile + c] = vsv;
-      float vm = vsv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
-      if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
-    };
-    bool ok = true;
-    {  // K_0
-      const int n0 = min(kTile, loop_end);
-      load_tile(kbase, kzb, 0, n0);
-      const float ksv = c < n0 ? ld_f32(a.ks + bh * a.S + c) : 0.0f;
-      const float vsv = c < n0 ? ld_f32(a.vs + bh * a.S + c) : 0.0f;
-      store_tile(C::K_OFF);
-      store_scales(0, ksv, vsv);
-      proxy_fence();
-      mbar_arrive(&bars[kBarKFull]);
-    }
-    for (int j = 0; j < ntiles; ++j) {
-      if (j + 1 < ntiles) {  // K_{j+1}: the buffer is free once QK_j has run
-        const int t1 = (j + 1) * kTile;
-        const int n1 = min(kTile, loop_end - t1);
-        load_tile(kbase, kzb, t1, n1);
-        const float ksv = c < n1 ? ld_f32(a.ks + bh * a.S + t1 + c) : 0.0f;
-        const float vsv = c < n1 ? ld_f32(a.vs + bh * a.S + t1 + c) : 0.0f;
-        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarKEmpty], j & 1, abort_flag));
-        if (!ok) break;
-        store_tile(C::K_OFF);
-        store_scales((j + 1) % kScaleBufs, ksv, vsv);
-        proxy_fence();
-        mbar_arrive(&bars[kBarKFull]);
-      }
-      {  // V_j: the buffer is free once PV_{j-1} has run
-        const int t0 = j * kTile;
-        load_tile(vbase, vzb, t0, min(kTile, loop_end - t0));
-        if (j > 0) {
-          ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag));
-          if (!ok) break;
-        }
-        store_tile(C::V_OFF);
-        proxy_fence();
-        mbar_arrive(&bars[kBarVFull]);
-      }
-    }
-  } else {
-    // ======================= MMA warp: lane 0 issues
-    if (lane == 0) {
-      constexpr uint32_t ID_QK = idesc_f16(kRows, kTile, 0);
-      constexpr uint32_t ID_PV = idesc_f16(kRows, D, 1);
-      const uint32_t q_base = smem_u32(smem + C::Q_OFF), k_base = smem_u32(smem + C::K_OFF);
-      const uint32_t v_base = smem_u32(smem + C::V_OFF);
-      // Q and K regions share the [128 rows x 128 B] block shape (kRows == kTile)
-      static_assert(kRows == kTile, "Q and K block strides");
-      auto issue_qk = [&](int j) {
-        const uint32_t d = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = static_cast<uint32_t>(k >> 2) * (kRows * 128) + (k & 3) * 32;
-          mma_ss(d, sdesc(q_base + off, 16, 1024), sdesc(k_base + off, 16, 1024), ID_QK, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[kBarSFull0 + (j & 1)]);
-        mma_commit(&bars[kBarKEmpty]);
-      };
-      bool ok = wait_phase(&bars[kBarQ], 0, abort_flag);
-      if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
-      for (int j = 0; j < ntiles && ok; ++j) {
-        if (j + 1 < ntiles) {
-          ok = wait_phase(&bars[kBarKFull], (j + 1) & 1, abort_flag);
-          // S buffer (j+1)&1 holds P_{j-1} until PV_{j-1} has run
-          if (ok && j >= 1) ok = wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(j + 1);
-        }
-        ok = wait_phase(&bars[kBarVFull], j & 1, abort_flag);
-        if (ok) ok = wait_phase(&bars[kBarPFull0 + (j & 1)], (j >> 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
-#pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)  // 16 slots = 8 packed TMEM columns of P
-          mma_ts(tmem + C::O_COL, p_tmem + k * 8, sdesc(v_base + k * 2048, kTile * 128, 1024), ID_PV,
-                 (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&bars[kBarODone]);
-        mma_commit(&bars[kBarVEmpty]);
-        if (j + 1 == ntiles) mma_commit(&bars[kBarOFinal]);
-      }
-      if (!ok) {  // everything issued finishes before TMEM is released
-        mma_commit(&bars[kBarDrain]);
-        mbar_wait_bounded(&bars[kBarDrain], 0);
-      }
-    }
-    __syncwarp();
-  }
+  const Ctx x{smem, tmem, kv, loop_end, ntiles};
+  if (warp < 4)
+    role_softmax<C>(a, x);
+  else if (warp < 12)
+    role_convert<C>(a, x);
+  else
+    role_mma<C>(a, x);
 
   // ---- teardown
   tc_fence_before();
