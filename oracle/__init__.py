@@ -31,6 +31,10 @@ MODE_INT8_AFFINE = 0
 MODE_FP8_E4M3 = 1
 MODE_MXFP8 = 2
 MODE_MXFP4 = 3
+MODE_FP8_E5M2 = 4
+MODE_MXFP8_E5M2 = 5
+MODE_INT8_SYM = 6
+_F32_SCALE_MODES = (MODE_FP8_E4M3, MODE_FP8_E5M2, MODE_INT8_SYM)
 
 _CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
@@ -58,6 +62,12 @@ def _load():
         lib.kvqo_e4m3_value.restype = ctypes.c_double
         lib.kvqo_e4m3_encode.argtypes = [f32]
         lib.kvqo_e4m3_encode.restype = ctypes.c_uint8
+        lib.kvqo_e5m2_value.argtypes = [ctypes.c_uint8]
+        lib.kvqo_e5m2_value.restype = ctypes.c_double
+        lib.kvqo_e5m2_encode.argtypes = [f32]
+        lib.kvqo_e5m2_encode.restype = ctypes.c_uint8
+        lib.kvqo_e8m0_floor.argtypes = [f32]
+        lib.kvqo_e8m0_floor.restype = ctypes.c_uint8
         lib.kvqo_e2m1_value.argtypes = [ctypes.c_uint8]
         lib.kvqo_e2m1_value.restype = ctypes.c_double
         lib.kvqo_e2m1_encode.argtypes = [f32]
@@ -68,9 +78,9 @@ def _load():
         lib.kvqo_e8m0_ceil.restype = ctypes.c_uint8
         lib.kvqo_affine_int8_row.argtypes = [P, i32, P, P, P]
         lib.kvqo_affine_int8_row.restype = None
-        lib.kvqo_block_row.argtypes = [i32, P, i32, P, P, P]
+        lib.kvqo_block_row.argtypes = [i32, i32, P, i32, P, P, P]
         lib.kvqo_block_row.restype = None
-        lib.kvqo_write.argtypes = [i32, P, i32, i32, i32, i32, P, P, i64, P, P, P, P]
+        lib.kvqo_write.argtypes = [i32, i32, P, i32, i32, i32, i32, P, P, i64, P, P, P, P]
         lib.kvqo_write.restype = None
         lib.kvqo_sink_plan.argtypes = [i32, i32, i32, i32, i64, P, P, P]
         lib.kvqo_sink_plan.restype = None
@@ -98,7 +108,7 @@ def _u16(x: np.ndarray) -> np.ndarray:
     return x.view(np.uint16)
 
 
-# --- number formats (OCP FP8 E4M3 "fn", OCP MX E2M1 / E8M0) ----------------
+# --- number formats (OCP FP8 E4M3 "fn" and E5M2, OCP MX E2M1 / E8M0) ----------
 
 def e4m3_value(code: int) -> float:
     return _load().kvqo_e4m3_value(int(code))
@@ -106,6 +116,14 @@ def e4m3_value(code: int) -> float:
 
 def e4m3_encode(v: float) -> int:
     return int(_load().kvqo_e4m3_encode(float(v)))
+
+
+def e5m2_value(code: int) -> float:
+    return _load().kvqo_e5m2_value(int(code))
+
+
+def e5m2_encode(v: float) -> int:
+    return int(_load().kvqo_e5m2_encode(float(v)))
 
 
 def e2m1_value(code: int) -> float:
@@ -124,6 +142,10 @@ def e8m0_ceil(s: float) -> int:
     return int(_load().kvqo_e8m0_ceil(float(s)))
 
 
+def e8m0_floor(s: float) -> int:
+    return int(_load().kvqo_e8m0_floor(float(s)))
+
+
 # --- quantizers --------------------------------------------------------------
 
 def affine_int8_row(x_bits: np.ndarray):
@@ -139,7 +161,7 @@ def affine_int8_row(x_bits: np.ndarray):
     return q, scale[0], zp[0]
 
 
-def block_row(mode: int, x_bits: np.ndarray):
+def block_row(mode: int, x_bits: np.ndarray, round_scale: bool = True):
     """IndexerQuantCache, 计算公式: per-32 block quantization of one row.
 
     Returns (codes uint8 [d or d/2], scales float32 [d/32] or uint8 E8M0 [d/32])."""
@@ -148,12 +170,13 @@ def block_row(mode: int, x_bits: np.ndarray):
     codes = np.zeros(d // 2 if mode == MODE_MXFP4 else d, np.uint8)
     sf = np.zeros(d // 32, np.float32)
     se = np.zeros(d // 32, np.uint8)
-    _load().kvqo_block_row(mode, _ptr(x), d, _ptr(codes), _ptr(sf), _ptr(se))
-    return codes, (sf if mode == MODE_FP8_E4M3 else se)
+    _load().kvqo_block_row(mode, int(bool(round_scale)), _ptr(x), d, _ptr(codes), _ptr(sf), _ptr(se))
+    return codes, (sf if mode in _F32_SCALE_MODES else se)
 
 
 def write(mode: int, x_bits: np.ndarray, slot_mapping: np.ndarray, num_slots: int,
-          codes: np.ndarray, scales: np.ndarray, zero_points: np.ndarray | None = None) -> int:
+          codes: np.ndarray, scales: np.ndarray, zero_points: np.ndarray | None = None,
+          round_scale: bool = True) -> int:
     """The cache write (quantize + scatter by slot_mapping, -1 = skip), in place.
 
     x_bits: uint16 [B, H, T, D] (any strides are flattened to contiguous here).
@@ -164,8 +187,8 @@ def write(mode: int, x_bits: np.ndarray, slot_mapping: np.ndarray, num_slots: in
     sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
     assert sm.size == B * T
     err = np.zeros(1, np.int32)
-    _load().kvqo_write(mode, _ptr(x), B, H, T, D, _ptr(xs), _ptr(sm), int(num_slots), _ptr(codes),
-                       _ptr(scales), _ptr(zero_points), _ptr(err))
+    _load().kvqo_write(mode, int(bool(round_scale)), _ptr(x), B, H, T, D, _ptr(xs), _ptr(sm),
+                       int(num_slots), _ptr(codes), _ptr(scales), _ptr(zero_points), _ptr(err))
     return int(err[0])
 
 

@@ -51,6 +51,9 @@
 #define KVQO_MODE_FP8_E4M3 1
 #define KVQO_MODE_MXFP8 2
 #define KVQO_MODE_MXFP4 3
+#define KVQO_MODE_FP8_E5M2 4   /* Normal, FLOAT8_E5M2 cache, float32 scale */
+#define KVQO_MODE_MXFP8_E5M2 5 /* MX-FP8, FLOAT8_E5M2 cache, E8M0 scale */
+#define KVQO_MODE_INT8_SYM 6   /* Normal, UINT8 cache holding int8 codes, float32 scale */
 
 /* ------------------------------------------------------------------------- */
 /* bfloat16: the top 16 bits of a binary32.  Widening is exact.              */
@@ -95,6 +98,44 @@ uint8_t kvqo_e4m3_encode(float v)
         return sign | 0x7E;
     for (int c = 1; c <= 0x7E; ++c) {
         double diff = fabs(kvqo_e4m3_value((uint8_t)c) - a);
+        if (diff < bestdiff || (diff == bestdiff && (c & 1) == 0)) {
+            best = (uint8_t)c;
+            bestdiff = diff;
+        }
+    }
+    return sign | best;
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP8 E5M2 (OCP): 1 sign, 5 exponent bits (bias 15), 2 mantissa bits.       */
+/* Normal: (1 + m/4) * 2^(e-15); subnormal (e == 0): (m/4) * 2^-14;          */
+/* e == 31 is infinity (m == 0) or NaN; largest finite is 57344.             */
+/* ------------------------------------------------------------------------- */
+double kvqo_e5m2_value(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 2) & 31, m = c & 3;
+    double mag;
+    if (e == 31)
+        return m ? NAN : (s ? -INFINITY : INFINITY);
+    if (e == 0)
+        mag = ldexp((double)m, -16);          /* (m/4) * 2^-14 */
+    else
+        mag = ldexp((double)(4 + m), e - 17); /* (1 + m/4) * 2^(e-15) */
+    return s ? -mag : mag;
+}
+
+/* Same rule as the E4M3 encoder: nearest, ties to the even code, saturating
+ * to the largest finite magnitude (never infinity), sign kept. */
+uint8_t kvqo_e5m2_encode(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    uint8_t best = 0;
+    double bestdiff = a;
+    if (a >= 57344.0)
+        return sign | 0x7B;
+    for (int c = 1; c <= 0x7B; ++c) {
+        double diff = fabs(kvqo_e5m2_value((uint8_t)c) - a);
         if (diff < bestdiff || (diff == bestdiff && (c & 1) == 0)) {
             best = (uint8_t)c;
             bestdiff = diff;
@@ -161,6 +202,23 @@ uint8_t kvqo_e8m0_ceil(float s)
     return (uint8_t)e;
 }
 
+/* The largest power of two <= s, as an E8M0 byte clamped to [0, 254]
+ * (reading of round_scale=false: the scale is not rounded, so its exponent is
+ * taken as it stands; codes then saturate at Q_MAX).  s <= 0 gives 0. */
+uint8_t kvqo_e8m0_floor(float s)
+{
+    int k, e;
+    if (!(s > 0.0f))
+        return 0;
+    (void)frexp((double)s, &k); /* s = f * 2^k, 0.5 <= f < 1: floor(log2 s) = k - 1 */
+    e = (k - 1) + 127;
+    if (e < 0)
+        e = 0;
+    if (e > 254)
+        e = 254;
+    return (uint8_t)e;
+}
+
 /* ------------------------------------------------------------------------- */
 /* [P1] per-token-and-head affine asymmetric int8, one row of D values.      */
 /* fp32, each step rounded to nearest even, in exactly this order:           */
@@ -199,13 +257,21 @@ void kvqo_affine_int8_row(const uint16_t *x, int D, int8_t *q, float *scale_out,
 /* [P5] 计算公式: per-block dynamic quantization of one row of d values,      */
 /* groups of 32 along d.  scale_g = max|x_g| / Q_MAX, q_i = round(x_i/scale). */
 /*   mode 1 (Normal, FP8 E4M3): Q_MAX 448, scale stored as float32.          */
-/*   mode 2 (MX-FP8): Q_MAX 448, scale rounded up to 2^k, stored as E8M0.    */
+/*   mode 4 (Normal, FP8 E5M2): Q_MAX 57344, scale stored as float32.        */
+/*   mode 6 (Normal, INT8 in a UINT8 cache): Q_MAX 127, q = rne(x/scale)     */
+/*          clamped to [-127, 127], stored as its two's-complement byte;     */
+/*          scale stored as float32.                                         */
+/*   mode 2 (MX-FP8, E4M3) / mode 5 (MX-FP8, E5M2): Q_MAX 448 / 57344; the   */
+/*          scale becomes a power of two stored as E8M0 -- rounded up with   */
+/*          round_scale (the default), else its exponent taken as it stands.*/
 /*   mode 3 (MX-FP4): Q_MAX 6, E2M1 codes, two per byte (2i low nibble),     */
-/*                    scale rounded up to 2^k, stored as E8M0.               */
+/*          scale rounded up to 2^k, stored as E8M0 (round_scale is an       */
+/*          MX-FP8 option only).                                             */
 /* An all-zero group writes zero codes and a zero scale (E8M0 byte 0).       */
-/* codes: d bytes (mode 1, 2) or d/2 bytes (mode 3); scale: d/32 entries.    */
+/* codes: d bytes (modes 1, 2, 4, 5, 6) or d/2 bytes (mode 3);               */
+/* scale: d/32 entries.                                                      */
 /* ------------------------------------------------------------------------- */
-void kvqo_block_row(int mode, const uint16_t *x, int d, uint8_t *codes, float *scale_f32,
+void kvqo_block_row(int mode, int round_scale, const uint16_t *x, int d, uint8_t *codes, float *scale_f32,
                     uint8_t *scale_e8m0)
 {
     for (int g = 0; g < d / 32; ++g) {
@@ -216,17 +282,31 @@ void kvqo_block_row(int mode, const uint16_t *x, int d, uint8_t *codes, float *s
             if (a > amax)
                 amax = a;
         }
-        if (mode == KVQO_MODE_FP8_E4M3) {
-            float scale = amax / 448.0f;
+        if (mode == KVQO_MODE_FP8_E4M3 || mode == KVQO_MODE_FP8_E5M2) {
+            int e5 = (mode == KVQO_MODE_FP8_E5M2);
+            float scale = amax / (e5 ? 57344.0f : 448.0f);
             scale_f32[g] = scale;
-            for (int i = 0; i < 32; ++i)
-                codes[32 * g + i] = (amax == 0.0f) ? 0 : kvqo_e4m3_encode(bf16_to_float(xg[i]) / scale);
-        } else if (mode == KVQO_MODE_MXFP8) {
-            uint8_t e = kvqo_e8m0_ceil(amax / 448.0f);
+            for (int i = 0; i < 32; ++i) {
+                float y = bf16_to_float(xg[i]) / scale;
+                codes[32 * g + i] = (amax == 0.0f) ? 0 : (e5 ? kvqo_e5m2_encode(y) : kvqo_e4m3_encode(y));
+            }
+        } else if (mode == KVQO_MODE_INT8_SYM) {
+            float scale = amax / 127.0f;
+            scale_f32[g] = scale;
+            for (int i = 0; i < 32; ++i) {
+                long q = (amax == 0.0f) ? 0 : clampl(lrintf(bf16_to_float(xg[i]) / scale), -127, 127);
+                codes[32 * g + i] = (uint8_t)(int8_t)q;
+            }
+        } else if (mode == KVQO_MODE_MXFP8 || mode == KVQO_MODE_MXFP8_E5M2) {
+            int e5 = (mode == KVQO_MODE_MXFP8_E5M2);
+            float s = amax / (e5 ? 57344.0f : 448.0f);
+            uint8_t e = round_scale ? kvqo_e8m0_ceil(s) : kvqo_e8m0_floor(s);
             float scale = (float)ldexp(1.0, (int)e - 127); /* exact, possibly subnormal */
             scale_e8m0[g] = e;
-            for (int i = 0; i < 32; ++i)
-                codes[32 * g + i] = (amax == 0.0f) ? 0 : kvqo_e4m3_encode(bf16_to_float(xg[i]) / scale);
+            for (int i = 0; i < 32; ++i) {
+                float y = bf16_to_float(xg[i]) / scale;
+                codes[32 * g + i] = (amax == 0.0f) ? 0 : (e5 ? kvqo_e5m2_encode(y) : kvqo_e4m3_encode(y));
+            }
         } else { /* KVQO_MODE_MXFP4 */
             uint8_t e = kvqo_e8m0_ceil(amax / 6.0f);
             float scale = (float)ldexp(1.0, (int)e - 127);
@@ -251,9 +331,10 @@ void kvqo_block_row(int mode, const uint16_t *x, int d, uint8_t *codes, float *s
 /*   mode 1: codes u8 [B,H,S,D], scales f32 [B,H,S,D/32]                     */
 /*   mode 2: codes u8 [B,H,S,D], scales e8m0 [B,H,S,D/32]                    */
 /*   mode 3: codes u8 [B,H,S,D/2], scales e8m0 [B,H,S,D/32]                  */
+/*   modes 4, 6: as mode 1;  mode 5: as mode 2                               */
 /* With B = H = 1 this is the page's cache [num_slots, d] layout.            */
 /* ------------------------------------------------------------------------- */
-void kvqo_write(int mode, const uint16_t *x, int B, int H, int T, int D, const int64_t *xs,
+void kvqo_write(int mode, int round_scale, const uint16_t *x, int B, int H, int T, int D, const int64_t *xs,
                 const int32_t *slot_mapping, int64_t S, void *codes, void *scales, int8_t *zps,
                 int32_t *err)
 {
@@ -275,7 +356,7 @@ void kvqo_write(int mode, const uint16_t *x, int B, int H, int T, int D, const i
                     kvqo_affine_int8_row(row, D, (int8_t *)codes + r * code_row, (float *)scales + r,
                                          zps + r);
                 } else {
-                    kvqo_block_row(mode, row, D, (uint8_t *)codes + r * code_row,
+                    kvqo_block_row(mode, round_scale, row, D, (uint8_t *)codes + r * code_row,
                                    (float *)scales + r * scale_row, (uint8_t *)scales + r * scale_row);
                 }
             }

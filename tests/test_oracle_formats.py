@@ -120,3 +120,60 @@ def test_e8m0_ceil_is_smallest_power_of_two_not_below():
         val = oracle.e8m0_value(e)
         assert val >= float(x)
         assert val / 2 < float(x)
+
+
+def test_e5m2_decode_matches_torch_for_every_code():
+    # torch.float8_e5m2 is the OCP E5M2 type: an independent decoder.
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).double().numpy()
+    ours = np.array([oracle.e5m2_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(ours))
+    assert np.array_equal(ref[~nan], ours[~nan])
+    assert np.array_equal(np.signbit(ref[~nan]), np.signbit(ours[~nan]))
+    assert nan.sum() == 6 and np.isinf(ours).sum() == 2
+
+
+def test_e5m2_encode_matches_torch_cast_in_range():
+    # torch's float32 -> float8_e5m2 cast rounds to nearest-even; it maps
+    # overflow to infinity, so only |v| <= 57344 is compared.
+    g = torch.Generator().manual_seed(13)
+    parts = [
+        torch.randn(20000, generator=g) * 2000,
+        torch.randn(20000, generator=g) * 1e-4,   # subnormal range
+        torch.rand(20000, generator=g) * 57344,
+    ]
+    vals = torch.arange(0, 0x7C, dtype=torch.uint8).view(torch.float8_e5m2).float()
+    mids = (vals[:-1] + vals[1:]) / 2
+    parts += [vals, mids, -mids, -vals]
+    v = torch.cat(parts).clamp(-57344, 57344)
+    ref = v.to(torch.float8_e5m2).view(torch.uint8).numpy()
+    ours = np.array([oracle.e5m2_encode(float(x)) for x in v.numpy()], np.uint8)
+    assert np.array_equal(ref, ours)
+
+
+def test_e5m2_golden_points(golden_dir):
+    for kind, value, code in _points(os.path.join(golden_dir, "e5m2_points.txt")):
+        value, code = float(value), int(code, 16)
+        if kind == "dec":
+            got = oracle.e5m2_value(code)
+            assert got == value and math.copysign(1, got) == math.copysign(1, value), (code, got)
+        else:
+            assert oracle.e5m2_encode(value) == code, (value, hex(oracle.e5m2_encode(value)))
+
+
+def test_e8m0_floor_golden(golden_dir):
+    for s, e in _points(os.path.join(golden_dir, "e8m0_floor_points.txt")):
+        assert oracle.e8m0_floor(float(np.float32(s))) == int(e), (s, e)
+
+
+def test_e8m0_floor_is_largest_power_of_two_not_above():
+    rng = np.random.default_rng(9)
+    s = np.concatenate([
+        np.exp2(rng.uniform(-126, 126, 3000)),
+        np.exp2(np.arange(-126, 127, dtype=np.float64)),
+    ]).astype(np.float32)
+    for x in s:
+        e = oracle.e8m0_floor(float(x))
+        val = oracle.e8m0_value(e)
+        assert val <= float(x)
+        assert val * 2 > float(x)

@@ -1,5 +1,10 @@
 """Pins for the oracle's quantizers (CPU only).
 
+The remaining IndexerQuantCache cache types (参数说明: FLOAT8_E5M2 and UINT8
+caches, round_scale=false) follow the same formula with Q_MAX 57344 (E5M2) and
+127 (symmetric int8 stored as its two's-complement byte); they are pinned the
+same way.
+
 int8 affine per token and head: ExecuTorch PR 24473, Summary (affine
 asymmetric, float32 scale, int8 zero point) -- the formula is a reading, pinned
 by hand-derived rows and by the dequantization error bound.
@@ -103,12 +108,13 @@ def test_block_golden_groups(golden_dir):
         mode = int(b["mode"][0])
         xs = [float(v) for v in b["x"]]
         xs += [float(b["fill"][0])] * (32 - len(xs))
-        codes, scales = oracle.block_row(mode, _bits(xs))
+        rs = bool(int(b.get("round", ["1"])[0]))
+        codes, scales = oracle.block_row(mode, _bits(xs), round_scale=rs)
         want = [int(c, 16) for c in b["codes"]]
         nbytes = 16 if mode == 3 else 32
         want += [int(b["codefill"][0], 16)] * (nbytes - len(want))
         assert codes.tolist() == want, (mode, [hex(c) for c in codes], b)
-        if mode == 1:
+        if mode in (1, 4, 6):
             assert float(scales[0]) == float(np.float32(b["scale"][0]))
         else:
             assert int(scales[0]) == int(b["scale"][0])
@@ -185,3 +191,50 @@ def test_block_amax_element_hits_the_top_code():
                 continue
             j = np.argmax(np.abs(xv[gi]))
             assert codes[gi * 32 + j] & 0x7F == 0x7E    # |x| = amax -> 448
+
+
+def _decode_e5m2(codes):
+    table = np.array([oracle.e5m2_value(c) for c in range(256)])
+    return table[codes]
+
+
+@pytest.mark.parametrize("mode,round_scale", [(4, True), (5, True), (5, False), (6, True)])
+def test_block_more_modes_scale_and_error_bounds(mode, round_scale):
+    x = _block_input(64, 512, 91 + mode + 7 * round_scale)
+    for r in range(x.shape[0]):
+        row = x[r]
+        codes, scales = oracle.block_row(mode, wl.u16(row), round_scale=round_scale)
+        xv = row.double().numpy().reshape(-1, 32)
+        amax = np.abs(xv).max(axis=1)
+        nz = amax > 0
+        if mode in (4, 6):
+            qmax = 57344.0 if mode == 4 else 127.0
+            scale = scales.astype(np.float64)
+            assert np.all(np.abs(scale - amax / qmax) <= np.spacing(scales).astype(np.float64) / 2 + 1e-300)
+        else:
+            scale = np.exp2(scales.astype(np.float64) - 127)
+            r_ = amax[nz] / scale[nz]
+            if round_scale:   # smallest power of two with amax/scale <= Q_MAX
+                assert np.all(r_ <= 57344 * (1 + 2.0 ** -23)) and np.all(r_ > 57344 / 2 * (1 - 2.0 ** -23))
+            else:             # largest power of two <= amax / Q_MAX
+                assert np.all(r_ >= 57344 * (1 - 2.0 ** -23)) and np.all(r_ < 2 * 57344 * (1 + 2.0 ** -23))
+            assert np.all(scales[~nz] == 0)
+        if mode == 6:
+            q = codes.view(np.int8).astype(np.float64).reshape(-1, 32)
+            assert np.all(np.abs(q) <= 127)
+            deq = q * scale[:, None]
+            # half a step, plus the binary32 rounding of x / scale (<= 127 * 2^-24 of a step)
+            bound = scale[:, None] * (0.5 + 2.0 ** -16)
+            for gi in np.where(nz)[0]:   # the largest element lands on +-127
+                assert abs(q[gi, np.argmax(np.abs(xv[gi]))]) == 127
+        else:
+            deq = _decode_e5m2(codes).reshape(-1, 32) * scale[:, None]
+            # E5M2: half an ulp is 2^-3 relative for normals, 2^-17 absolute (units of
+            # scale) in the subnormal range; + binary32 rounding of x / scale
+            bound = 2.0 ** -3 * np.abs(xv) + 2.0 ** -17 * scale[:, None] + 1e-6 * np.abs(xv)
+            if mode == 5 and not round_scale:   # codes saturate at 57344 * scale
+                bound = np.maximum(bound, np.abs(xv) - 57344 * scale[:, None] + 1e-300)
+        err = np.abs(deq - xv)
+        assert np.all(err <= bound), (mode, round_scale, r, err.max())
+        for gi in np.where(~nz)[0]:
+            assert np.all(codes[gi * 32:(gi + 1) * 32] == 0)
