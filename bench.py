@@ -521,23 +521,26 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
         sm[torch.randperm(bw.tokens, generator=g, device=dev)[: int(bw.tokens * bw.skip_frac)]] = -1
         sets.append((x, sm))
     valid = bw.tokens - int(bw.tokens * bw.skip_frac)
-    for mode, name in ((1, "fp8_e4m3"), (2, "mxfp8"), (3, "mxfp4")):
+    for mode, name, rs in ((1, "fp8_e4m3", True), (2, "mxfp8", True), (3, "mxfp4", True),
+                           (4, "fp8_e5m2", True), (5, "mxfp8_e5m2", True), (6, "int8_sym", True),
+                           (2, "mxfp8_unrounded_scale", False)):
         code_row = bw.d // 2 if mode == 3 else bw.d
+        f32 = mode in (1, 4, 6)
         caches = []
         for i in range(NB):
             c = torch.zeros((1, 1, bw.num_slots, code_row), dtype=torch.uint8, device=dev)
-            s = torch.zeros((1, 1, bw.num_slots, bw.d // 32), dtype=torch.float32 if mode == 1 else torch.uint8,
+            s = torch.zeros((1, 1, bw.num_slots, bw.d // 32), dtype=torch.float32 if f32 else torch.uint8,
                             device=dev)
             caches.append((c, s))
 
         def blk():
             for (x, sm), (c, s) in zip(sets, caches):
-                kvq.write(mode, x, sm, c, s)
+                kvq.write(mode, x, sm, c, s, round_scale=rs)
         ms = _time_graph(stream, blk, 10) / NB
-        sbytes = (bw.d // 32) * (4 if mode == 1 else 1)
+        sbytes = (bw.d // 32) * (4 if f32 else 1)
         byts = valid * (bw.d * 2 + code_row + sbytes) + bw.tokens * 4
-        res[f"block_write_{name}"] = {"what": f"kvq_write mode {mode}, x [16384, 512], 10% skipped",
-                                      "us": ms * 1000, "GB/s": byts / (ms / 1000) / 1e9,
+        res[f"block_write_{name}"] = {"what": f"kvq_write mode {mode} (round_scale={int(rs)}), x [16384, 512], "
+                                              f"10% skipped", "us": ms * 1000, "GB/s": byts / (ms / 1000) / 1e9,
                                       "frac": byts / (ms / 1000) / 1e9 / peak, "bytes": byts}
         del caches
     del sets

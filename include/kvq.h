@@ -55,6 +55,9 @@ extern "C" {
 #define KVQ_MODE_FP8_E4M3 1    /* E4M3 codes, f32 scale per 32 elements ("Normal") */
 #define KVQ_MODE_MXFP8 2       /* E4M3 codes, E8M0 scale per 32 elements */
 #define KVQ_MODE_MXFP4 3       /* E2M1 codes two per byte, E8M0 scale per 32 elements */
+#define KVQ_MODE_FP8_E5M2 4    /* E5M2 codes, f32 scale per 32 elements ("Normal", FLOAT8_E5M2 cache) */
+#define KVQ_MODE_MXFP8_E5M2 5  /* E5M2 codes, E8M0 scale per 32 elements (MX-FP8, FLOAT8_E5M2 cache) */
+#define KVQ_MODE_INT8_SYM 6    /* int8 codes (two's complement in a uint8 cache), f32 scale per 32 ("Normal", UINT8) */
 
 /*
  * kvq_write -- quantize x and scatter it into the cache, in place.
@@ -78,12 +81,16 @@ extern "C" {
  * num_slots    S, slots per (b, h) in the cache.
  * Cache layouts (row-major, contiguous, 16-byte aligned):
  *   mode 0: codes int8 [B, H, S, D]; scales float [B, H, S]; zero_points int8 [B, H, S]
- *   mode 1: codes u8   [B, H, S, D]; scales float [B, H, S, D/32]; zero_points NULL
- *   mode 2: codes u8   [B, H, S, D]; scales u8 (E8M0) [B, H, S, D/32]
+ *   modes 1, 4, 6: codes u8 [B, H, S, D]; scales float [B, H, S, D/32]; zero_points NULL
+ *   modes 2, 5: codes u8 [B, H, S, D]; scales u8 (E8M0) [B, H, S, D/32]
  *   mode 3: codes u8   [B, H, S, D/2] (element 2i in the low nibble); scales u8 (E8M0)
  *   With B = H = 1 the block modes are the IndexerQuantCache [num_slots, d] layout.
- * round_scale  mode 2 only: must be 1 (scale rounded up to a power of two);
- *              0 returns KVQ_EUNSUPPORTED.  Ignored by the other modes.
+ *   Q_MAX: 448 (E4M3), 57344 (E5M2), 6 (E2M1), 127 (mode 6: q = rne(x / scale)
+ *   clamped to [-127, 127], stored as its two's-complement byte).
+ * round_scale  modes 2 and 5 (MX-FP8): 1 rounds the scale amax / Q_MAX up to a
+ *              power of two; 0 takes its exponent as it stands (the largest
+ *              power of two not above it), codes then saturate at Q_MAX.
+ *              Ignored by the other modes.
  * Sizes: mode 0 needs D in {64, 128, 256}; modes 1-3 need D % 32 == 0 and
  * D <= 8192 (KVQ_EUNSUPPORTED otherwise).  B, H, T >= 0 (0 enqueues nothing).
  * The arithmetic is binary32 with one round-to-nearest-even per operation, in

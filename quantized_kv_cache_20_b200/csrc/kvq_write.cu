@@ -51,6 +51,7 @@ struct WriteArgs {
   int8_t *zps;
   int32_t *err;
   uint32_t groups;  // total groups
+  int round_scale;  // MX-FP8 modes: 1 = scale rounded up to a power of two, 0 = its exponent as it stands
 };
 
 constexpr int kThreads = 256;
@@ -63,6 +64,16 @@ KVQ_DEVINL uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+KVQ_DEVINL uint32_t e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+template <bool E5>
+KVQ_DEVINL uint32_t fp8x2(float lo, float hi) {
+  return E5 ? e5m2x2(lo, hi) : e4m3x2(lo, hi);
 }
 
 KVQ_DEVINL uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6, float v7) {
@@ -92,6 +103,16 @@ KVQ_DEVINL int e8m0_ceil(float s) {
     l = -149 + (32 - __clz(static_cast<int>(M - 1)));  // subnormal: ceil(log2 M) - 149
   const int e = l + 127;
   return e < 0 ? 0 : (e > 254 ? 254 : e);
+}
+
+// floor(log2 s) + 127 for a finite s >= 0, clamped to [0, 254]; s == 0 gives 0.
+// (Largest power of two not above s, as E8M0.)
+KVQ_DEVINL int e8m0_floor(float s) {
+  const uint32_t u = __float_as_uint(s);
+  if (u == 0) return 0;
+  const int E = static_cast<int>(u >> 23);
+  if (E == 0) return 0;  // subnormal: below 2^-126, clamped
+  return E > 254 ? 254 : E;  // floor(log2 s) + 127 is the biased exponent field
 }
 
 // 2^(127 - e) as a binary32 (exact for e in [0, 254]; e = 254 is subnormal).
@@ -225,8 +246,9 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         v[2 * j + 1] = bf16hi(wx[j]);
       }
       const int64_t sidx = r * a.GPR + gi;  // scale index
-      if constexpr (MODE == KVQ_MODE_FP8_E4M3) {
-        const float scale = __fdiv_rn(amax, 448.0f);
+      if constexpr (MODE == KVQ_MODE_FP8_E4M3 || MODE == KVQ_MODE_FP8_E5M2) {
+        constexpr bool E5 = MODE == KVQ_MODE_FP8_E5M2;
+        const float scale = __fdiv_rn(amax, E5 ? 57344.0f : 448.0f);
         uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         if (amax != 0.0f) {
           const float rcp = __frcp_rn(scale);
@@ -241,26 +263,66 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
             const float2 h0 = __fmul2_rn(y0, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
             const float2 l1 = __fmul2_rn(y1, make_float2(1.0f - 0x1p-20f, 1.0f - 0x1p-20f));
             const float2 h1 = __fmul2_rn(y1, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
-            const uint32_t c = e4m3x2(y0.x, y0.y) | (e4m3x2(y1.x, y1.y) << 16);
-            const uint32_t cl = e4m3x2(l0.x, l0.y) | (e4m3x2(l1.x, l1.y) << 16);
-            const uint32_t ch = e4m3x2(h0.x, h0.y) | (e4m3x2(h1.x, h1.y) << 16);
+            const uint32_t c = fp8x2<E5>(y0.x, y0.y) | (fp8x2<E5>(y1.x, y1.y) << 16);
+            const uint32_t cl = fp8x2<E5>(l0.x, l0.y) | (fp8x2<E5>(l1.x, l1.y) << 16);
+            const uint32_t ch = fp8x2<E5>(h0.x, h0.y) | (fp8x2<E5>(h1.x, h1.y) << 16);
             diff |= (c ^ cl) | (c ^ ch);
             w[k] = c;
           }
           if (diff) {  // rare: exact division for the whole group
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              w[k] = e4m3x2(__fdiv_rn(v[4 * k], scale), __fdiv_rn(v[4 * k + 1], scale)) |
-                     (e4m3x2(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
+              w[k] = fp8x2<E5>(__fdiv_rn(v[4 * k], scale), __fdiv_rn(v[4 * k + 1], scale)) |
+                     (fp8x2<E5>(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
           }
         }
         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         static_cast<float *>(a.scales)[sidx] = scale;
+      } else if constexpr (MODE == KVQ_MODE_INT8_SYM) {
+        // q = clamp(rne(x / scale), -127, 127), scale = amax / 127.  As in mode
+        // 0, y = x * rcp(scale) lies within 1.5 * 2^-23 |y| of the correctly
+        // rounded quotient, so a distance to the nearest half-integer above
+        // 2^-22 |y| settles the code; otherwise the group is redone exactly.
+        const float scale = __fdiv_rn(amax, 127.0f);
+        float t2[32];
+        if (amax != 0.0f) {
+          const float rcp = __frcp_rn(scale);
+          float worst = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float y = fminf(fmaxf(__fmul_rn(v[i], rcp), -127.0f), 127.0f);
+            const float tt = __fadd_rn(y, kMagic);
+            const float dd = __fsub_rn(y, __fsub_rn(tt, kMagic));  // y - rne(y)
+            worst = fmaxf(worst, fmaf(fabsf(y), 0x1p-22f, fabsf(dd)));
+            t2[i] = tt;
+          }
+          if (worst >= 0.5f - 0x1p-17f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              int q = __float2int_rn(__fdiv_rn(v[i], scale));
+              q = q < -127 ? -127 : (q > 127 ? 127 : q);
+              t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t2[i] = kMagic;  // code 0
+        }
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        static_cast<float *>(a.scales)[sidx] = scale;
       } else {
-        constexpr float kQmax = (MODE == KVQ_MODE_MXFP8) ? 448.0f : 6.0f;
-        const int e = e8m0_ceil(__fdiv_rn(amax, kQmax));
+        constexpr bool MX8 = MODE == KVQ_MODE_MXFP8 || MODE == KVQ_MODE_MXFP8_E5M2;
+        constexpr bool E5 = MODE == KVQ_MODE_MXFP8_E5M2;
+        constexpr float kQmax = MX8 ? (E5 ? 57344.0f : 448.0f) : 6.0f;
+        const float s_ = __fdiv_rn(amax, kQmax);
+        const int e = (MX8 && !a.round_scale) ? e8m0_floor(s_) : e8m0_ceil(s_);
         const float inv = e8m0_inverse(e);  // x / 2^(e-127) == x * 2^(127-e), exactly rounded
         float y[32];
 #pragma unroll
@@ -269,11 +331,12 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
           y[i] = yy.x;
           y[i + 1] = yy.y;
         }
-        if constexpr (MODE == KVQ_MODE_MXFP8) {
+        if constexpr (MX8) {
           uint32_t w[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            w[k] = amax != 0.0f ? (e4m3x2(y[4 * k], y[4 * k + 1]) | (e4m3x2(y[4 * k + 2], y[4 * k + 3]) << 16)) : 0u;
+            w[k] = amax != 0.0f ? (fp8x2<E5>(y[4 * k], y[4 * k + 1]) | (fp8x2<E5>(y[4 * k + 2], y[4 * k + 3]) << 16))
+                                : 0u;
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -309,13 +372,12 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
                          const int64_t *x_strides, const int32_t *slot_mapping, int64_t num_slots, void *codes,
                          void *scales, int8_t *zero_points, int32_t *err_word, void *stream) {
   using namespace kvq;
-  if (mode < KVQ_MODE_INT8_AFFINE || mode > KVQ_MODE_MXFP4) return KVQ_EINVAL;
+  if (mode < KVQ_MODE_INT8_AFFINE || mode > KVQ_MODE_INT8_SYM) return KVQ_EINVAL;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || num_slots <= 0 || num_slots > INT32_MAX) return KVQ_EINVAL;
   if (mode == KVQ_MODE_INT8_AFFINE) {
     if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
   } else {
     if (D % 32 != 0 || D > 8192) return KVQ_EUNSUPPORTED;
-    if (mode == KVQ_MODE_MXFP8 && !round_scale) return KVQ_EUNSUPPORTED;
   }
   if (static_cast<int64_t>(B) * H * T == 0) return KVQ_OK;
   if (!x || !x_strides || !slot_mapping || !codes || !scales) return KVQ_EINVAL;
@@ -324,9 +386,10 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   if (!aligned16(x) || !aligned16(codes)) return KVQ_EINVAL;
   for (int i = 0; i < 3; ++i)
     if (x_strides[i] < 0 || (x_strides[i] & 7) != 0) return KVQ_EINVAL;
-  // float scales (modes 0 and 1) must be 4-byte aligned; E8M0 scales are bytes
-  if ((mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_FP8_E4M3) && (reinterpret_cast<uintptr_t>(scales) & 3u))
-    return KVQ_EINVAL;
+  // float scales (modes 0, 1, 4, 6) must be 4-byte aligned; E8M0 scales are bytes
+  const bool f32_scales = mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_FP8_E4M3 || mode == KVQ_MODE_FP8_E5M2 ||
+                          mode == KVQ_MODE_INT8_SYM;
+  if (f32_scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return KVQ_EINVAL;
   // group indices use 32-bit arithmetic
   const int64_t groups = static_cast<int64_t>(B) * H * T * (D / 32);
   if (groups >= (int64_t(1) << 31)) return KVQ_EUNSUPPORTED;
@@ -351,11 +414,15 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   a.zps = zero_points;
   a.err = err_word;
   a.groups = static_cast<uint32_t>(groups);
+  a.round_scale = round_scale ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (mode) {
     case KVQ_MODE_INT8_AFFINE: return launch_write<KVQ_MODE_INT8_AFFINE>(a, s);
     case KVQ_MODE_FP8_E4M3: return launch_write<KVQ_MODE_FP8_E4M3>(a, s);
     case KVQ_MODE_MXFP8: return launch_write<KVQ_MODE_MXFP8>(a, s);
-    default: return launch_write<KVQ_MODE_MXFP4>(a, s);
+    case KVQ_MODE_MXFP4: return launch_write<KVQ_MODE_MXFP4>(a, s);
+    case KVQ_MODE_FP8_E5M2: return launch_write<KVQ_MODE_FP8_E5M2>(a, s);
+    case KVQ_MODE_MXFP8_E5M2: return launch_write<KVQ_MODE_MXFP8_E5M2>(a, s);
+    default: return launch_write<KVQ_MODE_INT8_SYM>(a, s);
   }
 }

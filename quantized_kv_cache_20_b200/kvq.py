@@ -33,6 +33,9 @@ MODE_INT8_AFFINE = 0
 MODE_FP8_E4M3 = 1
 MODE_MXFP8 = 2
 MODE_MXFP4 = 3
+MODE_FP8_E5M2 = 4
+MODE_MXFP8_E5M2 = 5
+MODE_INT8_SYM = 6
 
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",

@@ -111,10 +111,10 @@ def int8_cache_like(B: int, H: int, S: int, D: int, gen: torch.Generator):
 
 def block_cache_random(B: int, H: int, S: int, d: int, mode: int, gen: torch.Generator):
     """Arbitrary pre-fill for a block-mode cache: random code bytes and either
-    float32 scales U(0.01, 0.1) (mode 1) or random E8M0 bytes in [100, 140]."""
+    float32 scales U(0.01, 0.1) (modes 1, 4, 6) or random E8M0 bytes in [100, 140]."""
     row = d // 2 if mode == 3 else d
     codes = torch.randint(0, 256, (B, H, S, row), generator=gen, dtype=torch.uint8)
-    if mode == 1:
+    if mode in (1, 4, 6):
         scales = torch.rand((B, H, S, d // 32), generator=gen) * 0.09 + 0.01
     else:
         scales = torch.randint(100, 141, (B, H, S, d // 32), generator=gen, dtype=torch.uint8)

@@ -61,8 +61,12 @@ def test_argument_checks_reject_before_any_launch(lib):
     # block modes need d % 32 == 0 and d <= 8192
     assert lib.kvq_write(1, 1, fake, 1, 1, 1, 48, strides, fake, 8, fake, fake, None, None, None) == -2
     assert lib.kvq_write(1, 1, fake, 1, 1, 1, 8224, strides, fake, 8, fake, fake, None, None, None) == -2
-    # MX-FP8 without round_scale is not built
-    assert lib.kvq_write(2, 0, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, None, None, None) == -2
+    # float-scale modes (1, 4, 6) need 4-byte aligned scales
+    for m in (1, 4, 6):
+        assert lib.kvq_write(m, 1, fake, 1, 1, 1, 64, strides, fake, 8, fake, P(17), None, None, None) == -1
+    # the new modes take the block-mode size rules
+    for m in (4, 5, 6):
+        assert lib.kvq_write(m, 1, fake, 1, 1, 1, 48, strides, fake, 8, fake, fake, None, None, None) == -2
     # null x
     assert lib.kvq_write(0, 1, None, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
     # misaligned x

@@ -20,15 +20,16 @@ def _prefill(mode, B, H, S, D, g):
     return [c, s, None]
 
 
-def _run_both(mode, x, sm, cache0, S):
+def _run_both(mode, x, sm, cache0, S, round_scale=True):
     """Write x on the GPU and in the oracle over identical pre-filled caches."""
     gpu = [None if c is None else c.to(DEV) for c in cache0]
     err = err_word()
-    kvq.write(mode, x.to(DEV) if not x.is_cuda else x, sm.to(DEV), gpu[0], gpu[1], gpu[2], err_word=err)
+    kvq.write(mode, x.to(DEV) if not x.is_cuda else x, sm.to(DEV), gpu[0], gpu[1], gpu[2], err_word=err,
+              round_scale=round_scale)
     torch.cuda.synchronize()
     ref = [None if c is None else c.numpy().copy() for c in cache0]
     xc = x.cpu()
-    oerr = oracle.write(mode, wl.u16(xc), sm.numpy(), S, ref[0], ref[1], ref[2])
+    oerr = oracle.write(mode, wl.u16(xc), sm.numpy(), S, ref[0], ref[1], ref[2], round_scale=round_scale)
     return [None if c is None else c.cpu().numpy() for c in gpu], ref, int(err.item()), oerr
 
 
@@ -87,35 +88,50 @@ def _special_rows(d, g):
                         5.5, 0.1, 0.3, 0.8, 2.2, 2.9, 4.9, -6.0, 7.0, 100.0, -100.0, 0.0, -0.0, 1.0, 3.0, 4.0,
                         -0.5])
     rows.append(fp4.repeat(d // 32))
+    # exact E5M2 midpoints at scale 1 (amax 57344)
+    e5 = torch.arange(0, 0x7C, dtype=torch.uint8).view(torch.float8_e5m2).float()
+    mids5 = (e5[:-1] + e5[1:]) / 2
+    r = torch.cat([torch.tensor([57344.0]), mids5, -mids5])[:d]
+    rows.append(torch.nn.functional.pad(r, (0, d - r.numel())))
+    # exact int8 half-integers at scale 1 (amax 127)
+    halves = torch.arange(-126, 127, dtype=torch.float32) + 0.5
+    r = torch.cat([torch.tensor([127.0, -127.0]), halves])[:d]
+    rows.append(torch.nn.functional.pad(r, (0, d - r.numel())))
     return torch.stack([r.to(torch.bfloat16) for r in rows])
 
 
-@pytest.mark.parametrize("mode", [1, 2, 3])
+# (mode, round_scale): the IndexerQuantCache quant modes and cache types built;
+# round_scale only matters for the MX-FP8 modes 2 and 5
+BLOCK_CASES = [(1, True), (2, True), (3, True), (4, True), (5, True), (6, True), (2, False), (5, False)]
+
+
+@pytest.mark.parametrize("mode,round_scale", BLOCK_CASES)
 @pytest.mark.parametrize("d", [32, 96, 512, 8192])
-def test_block_modes_small(mode, d):
-    g = wl.generator(2000 + mode * 10 + d)
+def test_block_modes_small(mode, round_scale, d):
+    g = wl.generator(2000 + mode * 10 + d + (0 if round_scale else 7))
     bs = 300 if d <= 512 else 24
     S = 2 * bs
     x = wl.bf16_normal((bs, d), g, outlier_p=0.01, outlier_scale=10.0)
-    x[: 8] = _special_rows(d, g)
+    sp = _special_rows(d, g)
+    x[: sp.shape[0]] = sp
     sm = wl.slot_mapping_random(bs, S, bs // 10, g)
     cache0 = _prefill(mode, 1, 1, S, d, g)
-    gpu, ref, err, oerr = _run_both(mode, x.view(1, 1, bs, d), sm, cache0, S)
+    gpu, ref, err, oerr = _run_both(mode, x.view(1, 1, bs, d), sm, cache0, S, round_scale)
     assert err == 0
-    _assert_equal(gpu, ref, f"mode {mode} d={d}")
+    _assert_equal(gpu, ref, f"mode {mode} round_scale={round_scale} d={d}")
 
 
-@pytest.mark.parametrize("mode", [1, 2, 3])
-def test_block_config_full_size(mode):
+@pytest.mark.parametrize("mode,round_scale", BLOCK_CASES)
+def test_block_config_full_size(mode, round_scale):
     """x [16384, 512] (1% x10 outliers) into 65536 slots, 10% skipped."""
     w = wl.BLOCK
     g = wl.generator(w.seed)
     x = wl.bf16_normal((w.tokens, w.d), g, outlier_p=w.outlier_p, outlier_scale=w.outlier_scale)
     sm = wl.slot_mapping_random(w.tokens, w.num_slots, int(w.tokens * w.skip_frac), g)
     cache0 = _prefill(mode, 1, 1, w.num_slots, w.d, g)
-    gpu, ref, err, oerr = _run_both(mode, x.view(1, 1, w.tokens, w.d), sm, cache0, w.num_slots)
+    gpu, ref, err, oerr = _run_both(mode, x.view(1, 1, w.tokens, w.d), sm, cache0, w.num_slots, round_scale)
     assert err == 0
-    _assert_equal(gpu, ref, f"block mode {mode}")
+    _assert_equal(gpu, ref, f"block mode {mode} round_scale={round_scale}")
 
 
 def test_decode_config_bulk_fill_full_size():
@@ -143,7 +159,7 @@ def test_long_config_chunk_write():
     _assert_equal(gpu, ref, "long chunk")
 
 
-@pytest.mark.parametrize("mode", [0, 1, 3])
+@pytest.mark.parametrize("mode", [0, 1, 3, 4, 6])
 def test_second_identical_write_is_a_no_op_on_gpu(mode):
     g = wl.generator(3000 + mode)
     B, H, T, D, S = 2, 4, 33, 128, 96
