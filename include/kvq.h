@@ -182,6 +182,26 @@ int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *
                     void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
 
 /*
+ * kvq_decode_attn_varlen -- kvq_decode_attn with one kv_len per batch row.
+ *
+ * Defines: as kvq_decode_attn; the device-side bound of ExecuTorch PR 20351
+ * (commit notes: kv_len read on the device, bounding the loop to the filled
+ * length) taken per batch row, so rows of a decode batch can hold different
+ * context lengths.
+ *
+ * kv_lens      int32 [B] device array: row b attends over slots [0, kv_lens[b]).
+ *              Values outside [0, S] are clamped and set KVQ_ERR_KV_LEN_RANGE;
+ *              a row with kv_lens[b] = 0 outputs zeros.
+ * mask         nullable float [S], shared by all rows (as for kvq_decode_attn).
+ * Other arguments, sizes and the workspace as for kvq_decode_attn.  The work
+ * is cut as for the longest row; tiles past a row's own length move no bytes.
+ */
+int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
+                           const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
+                           int64_t S, const int32_t *kv_lens, const float *mask, float sm_scale, void *out,
+                           void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
+
+/*
  * kvq_prefill_attn -- Lq-query (chunked prefill) attention over the int8 cache.
  *
  * Defines: as kvq_decode_attn, plus ExecuTorch PR 20351 commit notes (the
@@ -209,6 +229,21 @@ int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const
                      const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
                      int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
                      void *stream);
+
+/*
+ * kvq_prefill_attn_varlen -- kvq_prefill_attn with one kv_len per batch row.
+ *
+ * Defines: as kvq_prefill_attn, with the chunk of batch row b at positions
+ * kv_lens[b] - Lq + i (ExecuTorch PR 20351, commit notes, per row).
+ *
+ * kv_lens      int32 [B] device array, each clamped to [Lq, S]
+ *              (KVQ_ERR_KV_LEN_RANGE).  mask (nullable, [Lq, S]) is shared by
+ *              all rows.  Other arguments as for kvq_prefill_attn.
+ */
+int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
+                            const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
+                            const int8_t *v_zp, int64_t S, const int32_t *kv_lens, const float *mask, int is_causal,
+                            int mask_is_causal, float sm_scale, void *out, int32_t *err_word, void *stream);
 
 /*
  * kvq_decode_attn_static -- kvq_decode_attn without a caller-supplied workspace.

@@ -61,7 +61,8 @@ struct DecodeArgs {
   const float *vs;
   const int8_t *vz;
   const float *mask;
-  const int32_t *kv_len;
+  const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
+  int kv_per_batch;
   uint16_t *out;
   float *ws_ml;       // [C * smax][HC][2]
   float *ws_o;        // [C * smax][HC][D]
@@ -137,6 +138,41 @@ KVQ_DEVINL bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *
   }
 }
 
+// kv_len of batch row b, clamped to [0, S] (the out-of-range report is made once,
+// by max_kv_len).
+KVQ_DEVINL int row_kv(const DecodeArgs &a, int b) {
+  const int k = a.kv_per_batch ? a.kv_len[b] : *a.kv_len;
+  return k < 0 ? 0 : (k > a.S ? static_cast<int>(a.S) : k);
+}
+
+// The largest clamped kv_len over the batch, by the whole CTA; `report_bad`
+// makes this CTA flag an out-of-range value.  `red` is a shared int.
+KVQ_DEVINL int max_kv_len(const DecodeArgs &a, volatile int32_t *red, bool report_bad) {
+  if (!a.kv_per_batch) {
+    if (threadIdx.x == 0) {
+      const int k = *a.kv_len;
+      if (report_bad && (k < 0 || k > a.S)) report(a.err, KVQ_ERR_KV_LEN_RANGE);
+    }
+    return row_kv(a, 0);
+  }
+  if (threadIdx.x == 0) *red = 0;
+  __syncthreads();
+  int mx = 0;
+  bool bad = false;
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+    const int k = a.kv_len[b];
+    bad |= k < 0 || k > a.S;
+    mx = max(mx, k < 0 ? 0 : (k > a.S ? static_cast<int>(a.S) : k));
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if ((threadIdx.x & 31) == 0) atomicMax(const_cast<int32_t *>(red), mx);
+  if (report_bad && __any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(a.err, KVQ_ERR_KV_LEN_RANGE);
+  __syncthreads();
+  const int r = *red;
+  __syncthreads();
+  return r;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, HC = C::HC, NW = C::NW, NST = C::NST, L = C::L, NG = C::NG, TS = C::TS;
@@ -152,19 +188,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       mbar_init(&empty[i], NW);
     }
     fence_mbar_init();
-    int kv = *a.kv_len;
-    if (kv < 0 || kv > a.S) {
-      if (blockIdx.x == 0) report(a.err, KVQ_ERR_KV_LEN_RANGE);
-      kv = kv < 0 ? 0 : static_cast<int>(a.S);
-    }
-    sh[0] = kv;
     sh[1] = 0;
     sh[2] = 0;
   }
   __syncthreads();
+  // Every unit is cut into ceil(max kv_len / TS) tiles; with per-row lengths a
+  // row's tiles past its own kv_len carry no bytes and no work.
+  const int kv = max_kv_len(a, sh, blockIdx.x == 0);
   asm volatile("griddepcontrol.launch_dependents;");
-
-  const int kv = sh[0];
   const int ntiles = (kv + TS - 1) / TS;
   const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
   const int64_t CT = gridDim.x, cta = blockIdx.x;
@@ -193,6 +224,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       int t = static_cast<int>(t_begin - u * ntiles);
       int st = 0;
       uint32_t ephase = 0;  // parity of the empty-barrier phase to wait for at stage st
+      int64_t kv_u_of = -1;
+      int kv_u = kv;
       for (int64_t idx = t_begin; idx < t_end; ++idx) {
         const int64_t i = idx - t_begin;
         if (i >= NST && !wait_or_abort(&empty[st], ephase, sh + 1)) {
@@ -202,22 +235,28 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         }
         const int hc = static_cast<int>(u % a.nhc);
         const int64_t bhk = u / a.nhc;  // = b * Hkv + hk
+        if (u != kv_u_of) {
+          kv_u_of = u;
+          kv_u = a.kv_per_batch ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
+        }
         const int s0 = t * TS;
-        const int n = min(TS, kv - s0);
+        const int n = max(0, min(TS, kv_u - s0));
         const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
         const bool first = (t == 0) || (idx == t_begin);
         uint8_t *stage = smem + st * C::STAGE;
         const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * D + 10) + (a.mask ? 4u * n16 : 0u) +
                                (first ? 2u * HC * D : 0u);
-        mbar_arrive_expect_tx(&full[st], bytes);
+        mbar_arrive_expect_tx(&full[st], bytes);  // 0 bytes: a plain arrival
         const int64_t row = bhk * a.S + s0;
-        bulk_g2s_hint(stage + C::K_OFF, a.k + row * D, n16 * D, &full[st], pol);
-        bulk_g2s_hint(stage + C::V_OFF, a.v + row * D, n16 * D, &full[st], pol);
-        bulk_g2s(stage + C::KS_OFF, a.ks + row, n16 * 4, &full[st]);
-        bulk_g2s(stage + C::VS_OFF, a.vs + row, n16 * 4, &full[st]);
-        bulk_g2s(stage + C::KZ_OFF, a.kz + row, n16, &full[st]);
-        bulk_g2s(stage + C::VZ_OFF, a.vz + row, n16, &full[st]);
-        if (a.mask) bulk_g2s(stage + C::M_OFF, a.mask + s0, n16 * 4, &full[st]);
+        if (n16 > 0) {
+          bulk_g2s_hint(stage + C::K_OFF, a.k + row * D, n16 * D, &full[st], pol);
+          bulk_g2s_hint(stage + C::V_OFF, a.v + row * D, n16 * D, &full[st], pol);
+          bulk_g2s(stage + C::KS_OFF, a.ks + row, n16 * 4, &full[st]);
+          bulk_g2s(stage + C::VS_OFF, a.vs + row, n16 * 4, &full[st]);
+          bulk_g2s(stage + C::KZ_OFF, a.kz + row, n16, &full[st]);
+          bulk_g2s(stage + C::VZ_OFF, a.vz + row, n16, &full[st]);
+          if (a.mask) bulk_g2s(stage + C::M_OFF, a.mask + s0, n16 * 4, &full[st]);
+        }
         if (first) {
           const int64_t hk = bhk % a.Hkv, b = bhk / a.Hkv;
           const int64_t q0 = (b * a.Hq + hk * a.G + static_cast<int64_t>(hc) * HC) * D;
@@ -252,6 +291,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   float2 o2[HC][8];
   int64_t cur_u = -1;
   int seg = -1;
+  int kv_u = kv;  // kv_len of the current unit's batch row
 
   auto close_segment = [&](int64_t u, int sg) {
     // (1) denominators over the lane group, then merge the NG groups of the warp
@@ -346,6 +386,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       if (cur_u >= 0) close_segment(cur_u, seg);
       cur_u = u;
       ++seg;
+      kv_u = a.kv_per_batch ? row_kv(a, static_cast<int>(u / a.nhc / a.Hkv)) : kv;
       // new unit: q (from this stage) onto the fixed-point grid, fresh softmax state
       const uint16_t *qs = reinterpret_cast<const uint16_t *>(stage + C::Q_OFF);
 #pragma unroll
@@ -395,7 +436,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 
     const int s0 = t * TS;
     const int wbase = warp * 32;
-    if (ok && s0 + wbase < kv) {
+    if (ok && s0 + wbase < kv_u) {
       // ---- q . k on dp4a for the L slots of this lane group (slot = wbase + g + NG*jj)
       int part[L][HC];
 #pragma unroll
@@ -431,7 +472,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       }
       // ---- scores (log2 domain) for this lane's slot
       const int sl_own = wbase + own;
-      const bool valid = s0 + sl_own < kv;
+      const bool valid = s0 + sl_own < kv_u;
       const int kzp = static_cast<int8_t>(stage[C::KZ_OFF + sl_own]);
       const float ksc = reinterpret_cast<const float *>(stage + C::KS_OFF)[sl_own];
       const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[sl_own];
@@ -524,8 +565,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int deco
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int32_t recs[1024];
   __shared__ float mls[1024 * 2];
-  int kv = *a.kv_len;
-  kv = kv < 0 ? 0 : (kv > a.S ? static_cast<int>(a.S) : kv);
+  __shared__ int32_t red;
+  const int kv = max_kv_len(a, &red, false);
   const int64_t ntl = (kv + TS - 1) / TS;
   if (ntl == 0) return;
   const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
@@ -657,11 +698,12 @@ extern "C" size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int6
   return ws_layout(B, Hkv, D, G / hc, hc, sm_count()).total;
 }
 
-extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
-                               const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
-                               int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
-                               void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
-  using namespace kvq;
+namespace kvq {
+namespace {
+int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
+                const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp, int64_t S,
+                const int32_t *kv_len, int kv_per_batch, const float *mask, float sm_scale, void *out,
+                void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S > INT32_MAX) return KVQ_EINVAL;
   if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
   if (S % 16 != 0) return KVQ_EUNSUPPORTED;
@@ -689,6 +731,7 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
   a.vz = v_zp;
   a.mask = mask;
   a.kv_len = kv_len;
+  a.kv_per_batch = kv_per_batch;
   a.out = static_cast<uint16_t *>(out);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   a.ws_ml = reinterpret_cast<float *>(ws + w.ml);
@@ -712,6 +755,25 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
     case 128: return dispatch_hc<128>(a, hc, ctas, s);
     default: return dispatch_hc<256>(a, hc, ctas, s);
   }
+}
+}  // namespace
+}  // namespace kvq
+
+extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
+                               const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
+                               int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
+                               void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
+  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, mask, sm_scale, out,
+                          workspace, workspace_bytes, err_word, stream);
+}
+
+extern "C" int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
+                                      const float *k_scale, const int8_t *k_zp, const int8_t *v,
+                                      const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_lens,
+                                      const float *mask, float sm_scale, void *out, void *workspace,
+                                      size_t workspace_bytes, int32_t *err_word, void *stream) {
+  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_lens, 1, mask, sm_scale, out,
+                          workspace, workspace_bytes, err_word, stream);
 }
 
 // ----------------------------------------------------------------------------

@@ -2,11 +2,11 @@
 #include "kvq_common.cuh"
 #include "kvq_prefill_tc.cuh"
 
-extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
-                                const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
-                                const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
-                                int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
-                                void *stream) {
+namespace {
+int prefill_impl(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k, const float *k_scale,
+                 const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp, int64_t S,
+                 const int32_t *kv_len, int kv_per_batch, const float *mask, int is_causal, int mask_is_causal,
+                 float sm_scale, void *out, int32_t *err_word, void *stream) {
   using namespace kvq;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S > INT32_MAX || Lq <= 0 || Lq > S)
     return KVQ_EINVAL;
@@ -30,6 +30,7 @@ extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, i
   a.vz = v_zp;
   a.mask = mask;
   a.kv_len = kv_len;
+  a.kv_per_batch = kv_per_batch;
   a.out = static_cast<uint16_t *>(out);
   a.err = err_word;
   a.S = S;
@@ -48,4 +49,23 @@ extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, i
     case 128: return tc::dispatch_prefill_tc<128>(a, s);
     default: return tc::dispatch_prefill_tc<256>(a, s);
   }
+}
+}  // namespace
+
+extern "C" int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
+                                const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
+                                const int8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
+                                int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
+                                void *stream) {
+  return prefill_impl(q, B, Hq, Hkv, Lq, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, mask, is_causal,
+                      mask_is_causal, sm_scale, out, err_word, stream);
+}
+
+extern "C" int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
+                                       const float *k_scale, const int8_t *k_zp, const int8_t *v,
+                                       const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_lens,
+                                       const float *mask, int is_causal, int mask_is_causal, float sm_scale,
+                                       void *out, int32_t *err_word, void *stream) {
+  return prefill_impl(q, B, Hq, Hkv, Lq, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_lens, 1, mask, is_causal,
+                      mask_is_causal, sm_scale, out, err_word, stream);
 }

@@ -77,7 +77,8 @@ struct PrefillArgs {
   const float *vs;
   const int8_t *vz;
   const float *mask;
-  const int32_t *kv_len;
+  const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
+  int kv_per_batch;
   uint16_t *out;
   int32_t *err;
   int64_t S;
@@ -826,9 +827,9 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  int kv = *a.kv_len;
+  int kv = a.kv_per_batch ? a.kv_len[b] : *a.kv_len;
   if (kv < a.Lq || kv > a.S) {
-    if (tid == 0 && xrow == 0 && hkc == 0 && b == 0) report(a.err, KVQ_ERR_KV_LEN_RANGE);
+    if (tid == 0 && xrow == 0 && hkc == 0 && (a.kv_per_batch || b == 0)) report(a.err, KVQ_ERR_KV_LEN_RANGE);
     kv = kv < a.Lq ? a.Lq : static_cast<int>(a.S);
   }
   tc_fence_before();

@@ -39,7 +39,8 @@ MODE_INT8_SYM = 6
 
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
-    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_prefill_attn", "kvq_strerror", "kvq_version",
+    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_attn_varlen", "kvq_prefill_attn",
+    "kvq_prefill_attn_varlen", "kvq_strerror", "kvq_version",
 )
 
 _lib = None
@@ -73,10 +74,14 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_workspace_bytes.argtypes = [I, I, I, I, I64]
         lib.kvq_decode_workspace_bytes.restype = SZ
         lib.kvq_decode_attn.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
+        lib.kvq_decode_attn_varlen.argtypes = lib.kvq_decode_attn.argtypes
+        lib.kvq_decode_attn_varlen.restype = I
         lib.kvq_decode_attn.restype = I
         lib.kvq_decode_attn_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, P]
         lib.kvq_decode_attn_static.restype = I
         lib.kvq_prefill_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I, I, F, P, P, P]
+        lib.kvq_prefill_attn_varlen.argtypes = lib.kvq_prefill_attn.argtypes
+        lib.kvq_prefill_attn_varlen.restype = I
         lib.kvq_prefill_attn.restype = I
         lib.kvq_strerror.argtypes = [I]
         lib.kvq_strerror.restype = ctypes.c_char_p
@@ -187,7 +192,22 @@ def _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_w
 
 def decode_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,
                 workspace=None, err_word=None) -> torch.Tensor:
-    """kvq_decode_attn: q [B, Hq, 1, D] bf16 over the int8 cache [B, Hkv, S, D]."""
+    """kvq_decode_attn: q [B, Hq, 1, D] bf16 over the int8 cache [B, Hkv, S, D].
+    kv_len: int32 device scalar.  (decode_attn_varlen takes one per batch row.)"""
+    return _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, workspace, err_word,
+                   varlen=False)
+
+
+def decode_attn_varlen(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, *, out=None, mask=None, sm_scale=None,
+                       workspace=None, err_word=None) -> torch.Tensor:
+    """kvq_decode_attn_varlen: as decode_attn with kv_lens int32 [B] on the device."""
+    if kv_lens.numel() != q.shape[0]:
+        raise ValueError("kv_lens must hold one entry per batch row")
+    return _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, out, mask, sm_scale, workspace, err_word,
+                   varlen=True)
+
+
+def _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, workspace, err_word, varlen):
     if out is None:
         out = torch.empty_like(q)
     _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
@@ -199,11 +219,12 @@ def decode_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask
         sm_scale = 1.0 / math.sqrt(D)
     if workspace is None:
         workspace = decode_workspace(B, Hq, Hkv, D, S, q.device)
-    st = load().kvq_decode_attn(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
-                                _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
-                                _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
-                                _stream(q.device))
-    _check("kvq_decode_attn", st)
+    name = "kvq_decode_attn_varlen" if varlen else "kvq_decode_attn"
+    st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                               _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
+                               _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
+                               _stream(q.device))
+    _check(name, st)
     return out
 
 
@@ -230,6 +251,21 @@ def decode_attn_static(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=Non
 def prefill_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, is_causal=False,
                  mask_is_causal=False, sm_scale=None, err_word=None) -> torch.Tensor:
     """kvq_prefill_attn: q [B, Hq, Lq, D] bf16 (rows at positions kv_len - Lq + i)."""
+    return _prefill(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, is_causal, mask_is_causal,
+                    sm_scale, err_word, varlen=False)
+
+
+def prefill_attn_varlen(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, *, out=None, mask=None,
+                        is_causal=False, mask_is_causal=False, sm_scale=None, err_word=None) -> torch.Tensor:
+    """kvq_prefill_attn_varlen: as prefill_attn with kv_lens int32 [B] on the device."""
+    if kv_lens.numel() != q.shape[0]:
+        raise ValueError("kv_lens must hold one entry per batch row")
+    return _prefill(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, out, mask, is_causal, mask_is_causal,
+                    sm_scale, err_word, varlen=True)
+
+
+def _prefill(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, is_causal, mask_is_causal, sm_scale,
+             err_word, varlen):
     if out is None:
         out = torch.empty_like(q)
     _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
@@ -237,9 +273,10 @@ def prefill_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mas
     Hkv, S = k.shape[1], k.shape[2]
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(D)
-    st = load().kvq_prefill_attn(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
-                                 _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), int(bool(is_causal)),
-                                 int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
-                                 _stream(q.device))
-    _check("kvq_prefill_attn", st)
+    name = "kvq_prefill_attn_varlen" if varlen else "kvq_prefill_attn"
+    st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                               _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), int(bool(is_causal)),
+                               int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
+                               _stream(q.device))
+    _check(name, st)
     return out

@@ -288,3 +288,77 @@ def test_long_config_prefill_sampled_rows():
                            rows=rows, is_causal=True)
     got = bf16_to_f64(out)
     assert_attn_close(np.stack([got[b, h, i] for b, h, i in rows]), ref, "long prefill")
+
+
+# ---------------------------------------------------------------------------- per-row kv_len
+
+def _slice(c, b):
+    return [t[b:b + 1] for t in c]
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_decode_varlen_rows_match_the_oracle_per_row(D):
+    """Rows of one decode batch at different context lengths (0 .. 4000 of
+    4096 slots): each row equals the oracle run at its own kv_len."""
+    g = wl.generator(700 + D)
+    B, Hq, Hkv, S = 6, 8, 2, 4096
+    lens = [0, 1, 37, 352, 1000, 4000]
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    err = err_word()
+    out = kvq.decode_attn_varlen(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V],
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = bf16_to_f64(out)
+    for b in range(B):
+        ref = oracle.sdpa(wl.u16(q[b:b + 1]), *_np(_slice(K, b)), *_np(_slice(V, b)), kv_len=lens[b],
+                          sm_scale=1 / math.sqrt(D))
+        assert_attn_close(got[b:b + 1], ref, f"varlen decode D={D} row {b} kv={lens[b]}")
+    assert torch.all(out[0] == 0)
+
+
+def test_decode_varlen_equal_rows_is_the_scalar_path():
+    g = wl.generator(777)
+    B, Hq, Hkv, D, S = 4, 16, 4, 128, 2048
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    Kd = [t.to(DEV) for t in K]
+    Vd = [t.to(DEV) for t in V]
+    a = kvq.decode_attn(q.to(DEV), *Kd, *Vd, int32_scalar(1500))
+    b = kvq.decode_attn_varlen(q.to(DEV), *Kd, *Vd, torch.full((B,), 1500, dtype=torch.int32, device=DEV))
+    assert torch.equal(a, b)
+
+
+def test_decode_varlen_out_of_range_rows_are_clamped_and_flagged():
+    g = wl.generator(778)
+    B, Hq, Hkv, D, S = 3, 4, 2, 64, 512
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    Kd = [t.to(DEV) for t in K]
+    Vd = [t.to(DEV) for t in V]
+    err = err_word()
+    out = kvq.decode_attn_varlen(q.to(DEV), *Kd, *Vd, torch.tensor([-3, 9999, 100], dtype=torch.int32, device=DEV),
+                                 err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() & kvq.KVQ_ERR_KV_LEN_RANGE
+    ref = kvq.decode_attn_varlen(q.to(DEV), *Kd, *Vd, torch.tensor([0, S, 100], dtype=torch.int32, device=DEV))
+    assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_prefill_varlen_rows_match_the_oracle_per_row(D):
+    g = wl.generator(800 + D)
+    B, Hq, Hkv, S, Lq = 3, 4, 2, 320, 70
+    lens = [70, 171, 320]
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, Lq, D), g)
+    out = kvq.prefill_attn_varlen(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V],
+                                  torch.tensor(lens, dtype=torch.int32, device=DEV), is_causal=True,
+                                  mask_is_causal=True)
+    torch.cuda.synchronize()
+    got = bf16_to_f64(out)
+    for b in range(B):
+        ref = oracle.sdpa(wl.u16(q[b:b + 1]), *_np(_slice(K, b)), *_np(_slice(V, b)), kv_len=lens[b],
+                          sm_scale=1 / math.sqrt(D), is_causal=True)
+        assert_attn_close(got[b:b + 1], ref, f"varlen prefill D={D} row {b} kv={lens[b]}")
