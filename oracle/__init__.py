@@ -34,6 +34,7 @@ MODE_MXFP4 = 3
 MODE_FP8_E5M2 = 4
 MODE_MXFP8_E5M2 = 5
 MODE_INT8_SYM = 6
+MODE_INT4_AFFINE = 7
 _F32_SCALE_MODES = (MODE_FP8_E4M3, MODE_FP8_E5M2, MODE_INT8_SYM)
 
 _CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
@@ -78,6 +79,8 @@ def _load():
         lib.kvqo_e8m0_ceil.restype = ctypes.c_uint8
         lib.kvqo_affine_int8_row.argtypes = [P, i32, P, P, P]
         lib.kvqo_affine_int8_row.restype = None
+        lib.kvqo_affine_int4_row.argtypes = [P, i32, P, P, P]
+        lib.kvqo_affine_int4_row.restype = None
         lib.kvqo_block_row.argtypes = [i32, i32, P, i32, P, P, P]
         lib.kvqo_block_row.restype = None
         lib.kvqo_write.argtypes = [i32, i32, P, i32, i32, i32, i32, P, P, i64, P, P, P, P]
@@ -86,7 +89,7 @@ def _load():
         lib.kvqo_sink_plan.restype = None
         lib.kvqo_sink_mask.argtypes = [i32, i32, P, i64, P]
         lib.kvqo_sink_mask.restype = None
-        sdpa_args = [P, i32, i32, i32, i32, P, P, P, P, P, P, i32, i64, i32, P, i32, f32]
+        sdpa_args = [P, i32, i32, i32, i32, i32, P, P, P, P, P, P, i32, i64, i32, P, i32, f32]
         lib.kvqo_sdpa_row.argtypes = sdpa_args + [i32, i32, i32, P]
         lib.kvqo_sdpa_row.restype = None
         lib.kvqo_sdpa.argtypes = sdpa_args + [P]
@@ -161,6 +164,20 @@ def affine_int8_row(x_bits: np.ndarray):
     return q, scale[0], zp[0]
 
 
+def affine_int4_row(x_bits: np.ndarray):
+    """ExecuTorch PR 20351, commit notes (TQ4 cache: nibble-packed on the last
+    dim): the 4-bit affine per-token-and-head reading of one row.
+
+    Returns (packed uint8 [D/2], scale float32, zero_point uint8 in 0..15)."""
+    x = _u16(x_bits)
+    D = x.shape[-1]
+    q = np.zeros(D // 2, np.uint8)
+    scale = np.zeros(1, np.float32)
+    zp = np.zeros(1, np.uint8)
+    _load().kvqo_affine_int4_row(_ptr(x), D, _ptr(q), _ptr(scale), _ptr(zp))
+    return q, scale[0], zp[0]
+
+
 def block_row(mode: int, x_bits: np.ndarray, round_scale: bool = True):
     """IndexerQuantCache, 计算公式: per-32 block quantization of one row.
 
@@ -219,13 +236,18 @@ def sink_mask(input_pos: int, Lq: int, slot_pos: np.ndarray) -> np.ndarray:
 # --- attention -------------------------------------------------------------------
 
 def _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask):
+    """Codes are int8 [.., D] (kbits 8) or TQ4 nibbles uint8 [.., D/2] (kbits 4)."""
     q = _u16(q_bits)
     arrs = [np.ascontiguousarray(a) for a in (k, ks, kz, v, vs, vz)]
-    assert arrs[0].dtype == np.int8 and arrs[3].dtype == np.int8
+    for i in (0, 2, 3, 5):
+        assert arrs[i].dtype in (np.int8, np.uint8)
+        arrs[i] = arrs[i].view(np.int8)
     assert arrs[1].dtype == np.float32 and arrs[4].dtype == np.float32
-    assert arrs[2].dtype == np.int8 and arrs[5].dtype == np.int8
+    D = q.shape[-1]
+    kbits = 4 if arrs[0].shape[-1] * 2 == D else 8
+    assert arrs[0].shape[-1] * 8 == D * kbits and arrs[3].shape == arrs[0].shape
     m = None if mask is None else np.ascontiguousarray(mask, dtype=np.float32)
-    return q, arrs, m
+    return q, arrs, m, kbits
 
 
 def sdpa(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, mask=None,
@@ -233,13 +255,14 @@ def sdpa(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, mask=None,
     """fp64 attention over the dequantized int8 cache (abaddon KvCache::forward_attention
     shapes; ExecuTorch PR 20351 kv_len bound and causal rule; PR 24473 additive mask).
 
-    q_bits uint16 [B, Hq, Lq, D]; k/v int8 [B, Hkv, S, D]; ks/vs f32 and kz/vz int8
-    [B, Hkv, S].  Returns float64 [B, Hq, Lq, D]."""
-    q, (k, ks, kz, v, vs, vz), m = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
+    q_bits uint16 [B, Hq, Lq, D]; k/v int8 [B, Hkv, S, D] or, for the TQ4 packing,
+    uint8 nibbles [B, Hkv, S, D/2]; ks/vs f32 and kz/vz [B, Hkv, S].
+    Returns float64 [B, Hq, Lq, D]."""
+    q, (k, ks, kz, v, vs, vz), m, kbits = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
     B, Hq, Lq, D = q.shape
     Hkv, S = k.shape[1], k.shape[2]
     out = np.zeros((B, Hq, Lq, D), np.float64)
-    _load().kvqo_sdpa(_ptr(q), B, Hq, Lq, D, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs), _ptr(vz),
+    _load().kvqo_sdpa(_ptr(q), B, Hq, Lq, D, kbits, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs), _ptr(vz),
                       Hkv, S, int(kv_len), _ptr(m), int(bool(is_causal)), float(sm_scale), _ptr(out))
     return out
 
@@ -247,13 +270,13 @@ def sdpa(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, mask=None,
 def sdpa_rows(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, rows, mask=None,
               is_causal: bool = False) -> np.ndarray:
     """Same as ``sdpa`` for selected (b, h, i) rows only; returns float64 [len(rows), D]."""
-    q, (k, ks, kz, v, vs, vz), m = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
+    q, (k, ks, kz, v, vs, vz), m, kbits = _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask)
     B, Hq, Lq, D = q.shape
     Hkv, S = k.shape[1], k.shape[2]
     out = np.zeros((len(rows), D), np.float64)
     lib = _load()
     for n, (b, h, i) in enumerate(rows):
-        lib.kvqo_sdpa_row(_ptr(q), B, Hq, Lq, D, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs),
+        lib.kvqo_sdpa_row(_ptr(q), B, Hq, Lq, D, kbits, _ptr(k), _ptr(ks), _ptr(kz), _ptr(v), _ptr(vs),
                           _ptr(vz), Hkv, S, int(kv_len), _ptr(m), int(bool(is_causal)), float(sm_scale),
                           int(b), int(h), int(i), out[n].ctypes.data)
     return out

@@ -54,6 +54,7 @@
 #define KVQO_MODE_FP8_E5M2 4   /* Normal, FLOAT8_E5M2 cache, float32 scale */
 #define KVQO_MODE_MXFP8_E5M2 5 /* MX-FP8, FLOAT8_E5M2 cache, E8M0 scale */
 #define KVQO_MODE_INT8_SYM 6   /* Normal, UINT8 cache holding int8 codes, float32 scale */
+#define KVQO_MODE_INT4_AFFINE 7 /* TQ4 packing: 4-bit affine per token and head, two codes per byte */
 
 /* ------------------------------------------------------------------------- */
 /* bfloat16: the top 16 bits of a binary32.  Widening is exact.              */
@@ -254,6 +255,42 @@ void kvqo_affine_int8_row(const uint16_t *x, int D, int8_t *q, float *scale_out,
 }
 
 /* ------------------------------------------------------------------------- */
+/* [P4] TQ4 cache: nibble-packed along the last dim (D/2 bytes per slot),    */
+/* written along the position dim.  The pages give only the packing; the     */
+/* code is read here as the 4-bit form of the affine per-token-and-head      */
+/* quantizer above, onto [0, 15], same fp32 order and rounding:              */
+/*   mn = min(0, min x), mx = max(0, max x)                                  */
+/*   scale = (mx - mn) / 15, floored at FLT_EPSILON                          */
+/*   zp = clamp(-rne(mn / scale), 0, 15)                                     */
+/*   q_i = clamp(rne(x_i / scale) + zp, 0, 15)                               */
+/* packed[i] = q_{2i} | q_{2i+1} << 4 (element 2i in the low nibble).        */
+/* Dequantization is (q - zp) * scale.                                       */
+/* ------------------------------------------------------------------------- */
+void kvqo_affine_int4_row(const uint16_t *x, int D, uint8_t *packed, float *scale_out, uint8_t *zp_out)
+{
+    float mn = 0.0f, mx = 0.0f, scale;
+    long zp;
+    for (int i = 0; i < D; ++i) {
+        float v = bf16_to_float(x[i]);
+        if (v < mn)
+            mn = v;
+        if (v > mx)
+            mx = v;
+    }
+    scale = (mx - mn) / 15.0f;
+    if (scale < FLT_EPSILON)
+        scale = FLT_EPSILON;
+    zp = clampl(-lrintf(mn / scale), 0, 15);
+    for (int i = 0; i < D; i += 2) {
+        long q0 = clampl(lrintf(bf16_to_float(x[i]) / scale) + zp, 0, 15);
+        long q1 = clampl(lrintf(bf16_to_float(x[i + 1]) / scale) + zp, 0, 15);
+        packed[i / 2] = (uint8_t)(q0 | (q1 << 4));
+    }
+    *scale_out = scale;
+    *zp_out = (uint8_t)zp;
+}
+
+/* ------------------------------------------------------------------------- */
 /* [P5] 计算公式: per-block dynamic quantization of one row of d values,      */
 /* groups of 32 along d.  scale_g = max|x_g| / Q_MAX, q_i = round(x_i/scale). */
 /*   mode 1 (Normal, FP8 E4M3): Q_MAX 448, scale stored as float32.          */
@@ -332,14 +369,16 @@ void kvqo_block_row(int mode, int round_scale, const uint16_t *x, int d, uint8_t
 /*   mode 2: codes u8 [B,H,S,D], scales e8m0 [B,H,S,D/32]                    */
 /*   mode 3: codes u8 [B,H,S,D/2], scales e8m0 [B,H,S,D/32]                  */
 /*   modes 4, 6: as mode 1;  mode 5: as mode 2                               */
+/*   mode 7: codes u8 [B,H,S,D/2] (nibbles), scales f32 [B,H,S],             */
+/*           zps [B,H,S] holding 0..15                                       */
 /* With B = H = 1 this is the page's cache [num_slots, d] layout.            */
 /* ------------------------------------------------------------------------- */
 void kvqo_write(int mode, int round_scale, const uint16_t *x, int B, int H, int T, int D, const int64_t *xs,
                 const int32_t *slot_mapping, int64_t S, void *codes, void *scales, int8_t *zps,
                 int32_t *err)
 {
-    int64_t code_row = (mode == KVQO_MODE_MXFP4) ? D / 2 : D;
-    int64_t scale_row = (mode == KVQO_MODE_INT8_AFFINE) ? 1 : D / 32;
+    int64_t code_row = (mode == KVQO_MODE_MXFP4 || mode == KVQO_MODE_INT4_AFFINE) ? D / 2 : D;
+    int64_t scale_row = (mode == KVQO_MODE_INT8_AFFINE || mode == KVQO_MODE_INT4_AFFINE) ? 1 : D / 32;
     for (int b = 0; b < B; ++b) {
         for (int t = 0; t < T; ++t) {
             int32_t slot = slot_mapping[(int64_t)b * T + t];
@@ -355,6 +394,9 @@ void kvqo_write(int mode, int round_scale, const uint16_t *x, int B, int H, int 
                 if (mode == KVQO_MODE_INT8_AFFINE) {
                     kvqo_affine_int8_row(row, D, (int8_t *)codes + r * code_row, (float *)scales + r,
                                          zps + r);
+                } else if (mode == KVQO_MODE_INT4_AFFINE) {
+                    kvqo_affine_int4_row(row, D, (uint8_t *)codes + r * code_row, (float *)scales + r,
+                                         (uint8_t *)zps + r);
                 } else {
                     kvqo_block_row(mode, round_scale, row, D, (uint8_t *)codes + r * code_row,
                                    (float *)scales + r * scale_row, (uint8_t *)scales + r * scale_row);
@@ -407,10 +449,21 @@ void kvqo_sink_mask(int32_t input_pos, int Lq, const int32_t *slot_pos, int64_t 
 /* q head h reads kv head h / (Hq/Hkv).  [P4] only slots j < kv_len take     */
 /* part; with is_causal, row i (of Lq) sees j <= kv_len - Lq + i.  [P1] an   */
 /* additive mask [Lq, S] (row stride S) is added to the scaled scores.        */
-/* K and V are dequantized as (c - zp) * scale.  A row that sees nothing     */
-/* outputs zeros.                                                            */
+/* K and V are dequantized as (c - zp) * scale: c an int8 code (kbits 8), or */
+/* a 4-bit code 0..15 of the TQ4 packing (kbits 4: D/2 bytes per slot, code  */
+/* d in the low nibble of byte d/2 when d is even, else the high nibble).    */
+/* A row that sees nothing outputs zeros.                                    */
 /* ------------------------------------------------------------------------- */
-void kvqo_sdpa_row(const uint16_t *q, int B, int Hq, int Lq, int D, const int8_t *k, const float *ks,
+static double code_at(const int8_t *c, int64_t slot, int D, int d, int kbits)
+{
+    if (kbits == 4) {
+        uint8_t byte = (uint8_t)c[slot * (D / 2) + d / 2];
+        return (double)((d & 1) ? (byte >> 4) : (byte & 15));
+    }
+    return (double)c[slot * D + d];
+}
+
+void kvqo_sdpa_row(const uint16_t *q, int B, int Hq, int Lq, int D, int kbits, const int8_t *k, const float *ks,
                    const int8_t *kz, const int8_t *v, const float *vs, const int8_t *vz, int Hkv,
                    int64_t S, int32_t kv_len, const float *mask, int is_causal, float sm_scale, int b,
                    int h, int i, double *out)
@@ -427,7 +480,7 @@ void kvqo_sdpa_row(const uint16_t *q, int B, int Hq, int Lq, int D, const int8_t
         } else {
             double dot = 0.0;
             for (int d = 0; d < D; ++d) {
-                double kd = ((double)k[(base + j) * D + d] - (double)kz[base + j]) * (double)ks[base + j];
+                double kd = (code_at(k, base + j, D, d, kbits) - (double)kz[base + j]) * (double)ks[base + j];
                 dot += (double)bf16_to_float(qr[d]) * kd;
             }
             s[j] = dot * (double)sm_scale + (mask ? (double)mask[(int64_t)i * S + j] : 0.0);
@@ -447,7 +500,7 @@ void kvqo_sdpa_row(const uint16_t *q, int B, int Hq, int Lq, int D, const int8_t
         if (p == 0.0)
             continue;
         for (int d = 0; d < D; ++d)
-            out[d] += p * ((double)v[(base + j) * D + d] - (double)vz[base + j]) * (double)vs[base + j];
+            out[d] += p * (code_at(v, base + j, D, d, kbits) - (double)vz[base + j]) * (double)vs[base + j];
     }
     for (int d = 0; d < D; ++d)
         out[d] /= l;
@@ -455,13 +508,13 @@ void kvqo_sdpa_row(const uint16_t *q, int B, int Hq, int Lq, int D, const int8_t
 }
 
 /* Every row: out is [B, Hq, Lq, D]. */
-void kvqo_sdpa(const uint16_t *q, int B, int Hq, int Lq, int D, const int8_t *k, const float *ks,
+void kvqo_sdpa(const uint16_t *q, int B, int Hq, int Lq, int D, int kbits, const int8_t *k, const float *ks,
                const int8_t *kz, const int8_t *v, const float *vs, const int8_t *vz, int Hkv, int64_t S,
                int32_t kv_len, const float *mask, int is_causal, float sm_scale, double *out)
 {
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < Hq; ++h)
             for (int i = 0; i < Lq; ++i)
-                kvqo_sdpa_row(q, B, Hq, Lq, D, k, ks, kz, v, vs, vz, Hkv, S, kv_len, mask, is_causal,
+                kvqo_sdpa_row(q, B, Hq, Lq, D, kbits, k, ks, kz, v, vs, vz, Hkv, S, kv_len, mask, is_causal,
                               sm_scale, b, h, i, out + (((int64_t)b * Hq + h) * Lq + i) * D);
 }

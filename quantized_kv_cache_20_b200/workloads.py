@@ -121,6 +121,15 @@ def block_cache_random(B: int, H: int, S: int, d: int, mode: int, gen: torch.Gen
     return codes, scales
 
 
+def int4_cache_random(B: int, H: int, S: int, D: int, gen: torch.Generator):
+    """Arbitrary pre-fill / content for a TQ4 (4-bit, nibble-packed) cache: random
+    code bytes [B, H, S, D/2], scales U(0.3, 0.5), zero points in [5, 10]."""
+    codes = torch.randint(0, 256, (B, H, S, D // 2), generator=gen, dtype=torch.uint8)
+    scales = torch.rand((B, H, S), generator=gen) * 0.2 + 0.3
+    zps = torch.randint(5, 11, (B, H, S), generator=gen, dtype=torch.int8)
+    return codes, scales, zps
+
+
 def u16(t: torch.Tensor):
     """Raw bit patterns of a CPU bf16 tensor as a numpy uint16 array."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")

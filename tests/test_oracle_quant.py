@@ -238,3 +238,36 @@ def test_block_more_modes_scale_and_error_bounds(mode, round_scale):
         assert np.all(err <= bound), (mode, round_scale, r, err.max())
         for gi in np.where(~nz)[0]:
             assert np.all(codes[gi * 32:(gi + 1) * 32] == 0)
+
+
+def test_affine_int4_golden_rows(golden_dir):
+    blocks = _blocks(os.path.join(golden_dir, "affine_int4_rows.txt"))
+    assert len(blocks) == 5
+    for b in blocks:
+        packed, scale, zp = oracle.affine_int4_row(_bits(b["x"]))
+        q = [int(v) for v in b["q"]]
+        assert packed.tolist() == [int(c, 16) for c in b["packed"]], b
+        assert packed.tolist() == [q[2 * i] | (q[2 * i + 1] << 4) for i in range(len(q) // 2)]
+        assert float(scale) == float(np.float32(b["scale"][0]))
+        assert int(zp) == int(b["zp"][0])
+
+
+def _unpack4(packed):
+    return np.stack([packed & 15, packed >> 4], axis=-1).reshape(*packed.shape[:-1], -1)
+
+
+def test_affine_int4_dequant_error_bound_and_range():
+    # |(q - zp) * scale - x| <= scale * (1/2 + 2^-16): half a step plus the binary32
+    # rounding of x / scale (<= 15 * 2^-24 of a step) and of scale at the clamped top code
+    for row in _rows():
+        packed, scale, zp = oracle.affine_int4_row(wl.u16(row))
+        q = _unpack4(packed).astype(np.int64)
+        x = row.double().numpy()
+        deq = (q - int(zp)) * float(scale)
+        assert np.all(np.abs(deq - x) <= float(scale) * (0.5 + 2.0 ** -16)), row
+        assert 0 <= int(zp) <= 15 and q.min() >= 0 and q.max() <= 15
+        mn, mx = min(0.0, x.min()), max(0.0, x.max())
+        if mn < 0:
+            assert q[np.argmin(x)] == 0               # the minimum lands on the lowest code
+        if mx > 0 and float(scale) > FLT_EPS:
+            assert q[np.argmax(x)] >= 14              # the maximum lands at the top

@@ -127,3 +127,24 @@ def test_rows_helper_matches_full():
                             is_causal=True)
     for n, (b, h, i) in enumerate(rows):
         assert np.array_equal(part[n], full[b, h, i])
+
+
+def _unpack4(packed):
+    t = torch.from_numpy(packed.astype(np.int64))
+    return torch.stack([t & 15, t >> 4], dim=-1).reshape(*t.shape[:-1], -1)
+
+
+@pytest.mark.parametrize("is_causal", [False, True])
+def test_tq4_cache_matches_torch_sdpa_fp64(is_causal):
+    # the TQ4 (nibble-packed) cache: unpacked here independently of the oracle
+    g = wl.generator(61)
+    B, Hq, Hkv, Lq, D, S = 2, 4, 2, 3, 16, 24
+    q = wl.bf16_normal((B, Hq, Lq, D), g)
+    K = wl.int4_cache_random(B, Hkv, S, D, g)
+    V = wl.int4_cache_random(B, Hkv, S, D, g)
+    kv_len, sm = 19, 1 / math.sqrt(D)
+    ours = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=sm, is_causal=is_causal)
+    Ku = (_unpack4(K[0].numpy()), K[1], K[2])
+    Vu = (_unpack4(V[0].numpy()), V[1], V[2])
+    ref = _torch_ref(q, Ku, Vu, kv_len, sm, is_causal=is_causal)
+    np.testing.assert_allclose(ours, ref, rtol=1e-12, atol=1e-12)

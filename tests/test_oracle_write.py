@@ -22,6 +22,9 @@ def _setup(mode, seed, B=2, H=3, T=12, D=64, S=40):
     if mode == 0:
         codes, scales, zps = wl.int8_cache_random(B, H, S, D, g)
         cache = [codes.numpy().copy(), scales.numpy().copy(), zps.numpy().copy()]
+    elif mode == 7:
+        codes, scales, zps = wl.int4_cache_random(B, H, S, D, g)
+        cache = [codes.numpy().copy(), scales.numpy().copy(), zps.numpy().copy()]
     else:
         codes, scales = wl.block_cache_random(B, H, S, D, mode, g)
         cache = [codes.numpy().copy(), scales.numpy().copy(), None]
@@ -32,7 +35,7 @@ def _write(mode, x, sm, S, cache):
     return oracle.write(mode, wl.u16(x), sm, S, cache[0], cache[1], cache[2])
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5, 6, 7])
 def test_skipped_and_unwritten_slots_are_untouched(mode):
     S = 40
     x, sm, cache = _setup(mode, 100 + mode, S=S)
@@ -54,7 +57,7 @@ def test_skipped_and_unwritten_slots_are_untouched(mode):
                     assert np.array_equal(c[b, :, s], c0[b, :, s])
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5, 6, 7])
 def test_written_row_equals_the_row_quantized_alone(mode):
     # commuting: slot placement does not change the row's codes
     S = 40
@@ -68,8 +71,8 @@ def test_written_row_equals_the_row_quantized_alone(mode):
                 continue
             for h in range(H):
                 row = wl.u16(x[b, h, t])
-                if mode == 0:
-                    q, sc, zp = oracle.affine_int8_row(row)
+                if mode in (0, 7):
+                    q, sc, zp = (oracle.affine_int8_row if mode == 0 else oracle.affine_int4_row)(row)
                     assert np.array_equal(cache[0][b, h, s], q)
                     assert cache[1][b, h, s] == sc and cache[2][b, h, s] == zp
                 else:
@@ -78,7 +81,7 @@ def test_written_row_equals_the_row_quantized_alone(mode):
                     assert np.array_equal(cache[1][b, h, s], sc)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5, 6, 7])
 def test_second_identical_write_is_a_no_op(mode):
     S = 40
     x, sm, cache = _setup(mode, 300 + mode, S=S)
@@ -90,7 +93,7 @@ def test_second_identical_write_is_a_no_op(mode):
             assert np.array_equal(c, c1)
 
 
-@pytest.mark.parametrize("mode", [0, 3])
+@pytest.mark.parametrize("mode", [0, 3, 7])
 def test_permuting_tokens_with_their_slots(mode):
     S = 40
     x, sm, cache = _setup(mode, 400 + mode, B=1, S=S)
