@@ -545,6 +545,87 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
         del caches
     del sets
     torch.cuda.empty_cache()
+    # TQ4 cache (4-bit affine, two codes per byte) at the decode workload's shape: fill, then decode
+    tq = []
+    for _ in range(NL):
+        Kq = (torch.empty((w.B, w.Hkv, w.S, w.D // 2), dtype=torch.uint8, device=dev),
+              torch.empty((w.B, w.Hkv, w.S), dtype=torch.float32, device=dev),
+              torch.empty((w.B, w.Hkv, w.S), dtype=torch.int8, device=dev))
+        Vq = tuple(torch.empty_like(t) for t in Kq)
+        tq.append((Kq, Vq))
+
+    def tq4_fill():
+        for Kq, Vq in tq:
+            kvq.write(7, xk, sm_fill, *Kq)
+            kvq.write(7, xv, sm_fill, *Vq)
+    ms = _time_graph(stream, tq4_fill, 3) / (2 * NL)
+    qbytes = rows * w.D * 2 + rows * w.D // 2 + rows * 5 + w.B * Tf * 4
+    res["tq4_fill_write"] = {"what": "kvq_write mode 7 (TQ4), 8x8 heads x 4095 tokens, D=128", "us": ms * 1000,
+                             "GB/s": qbytes / (ms / 1000) / 1e9, "frac": qbytes / (ms / 1000) / 1e9 / peak,
+                             "bytes": qbytes}
+    kvl4 = torch.tensor([w.kv_len], dtype=torch.int32, device=dev)
+    qq = torch.randn((w.B, w.Hq, 1, w.D), device=dev).to(torch.bfloat16)
+    oq = torch.empty_like(qq)
+    wsq = kvq.decode_workspace(w.B, w.Hq, w.Hkv, w.D, w.S, dev)
+
+    def tq4_dec():
+        for Kq, Vq in tq:
+            kvq.decode_attn_tq4(qq, *Kq, *Vq, kvl4, out=oq, workspace=wsq)
+    ms = _time_graph(stream, tq4_dec, 20) / NL
+    dbytes = 2 * w.B * w.Hkv * w.kv_len * (w.D // 2 + 5) + 2 * w.B * w.Hq * w.D * 2
+    res["tq4_decode"] = {"what": "kvq_decode_attn_tq4, batch 8, 32 q / 8 kv heads, D=128, kv_len 4096 (TQ4 cache)",
+                         "us": ms * 1000, "tokens/s": w.B / (ms / 1000), "GB/s": dbytes / (ms / 1000) / 1e9,
+                         "frac": dbytes / (ms / 1000) / 1e9 / peak, "bytes": dbytes}
+    del tq, wsq
+    torch.cuda.empty_cache()
+    # the lines below read past position 4095: fill slots 4095..8191 of every layer first
+    Tr = w.S - Tf
+    xkr = torch.randn((w.B, w.Hkv, Tr, w.D), device=dev).to(torch.bfloat16)
+    smr_fill = (torch.arange(Tr, dtype=torch.int32, device=dev) + Tf).repeat(w.B)
+    for K, V in layers:
+        kvq.write(0, xkr, smr_fill, *K)
+        kvq.write(0, xkr, smr_fill, *V)
+    del xkr
+    # ragged decode batch: the 8 rows of the decode workload at 8 different context lengths
+    lens = [512, 1024, 2048, 3072, 4096, 5120, 6144, 8192]
+    kvs = torch.tensor(lens, dtype=torch.int32, device=dev)
+    qr = torch.randn((w.B, w.Hq, 1, w.D), device=dev).to(torch.bfloat16)
+    outr = torch.empty_like(qr)
+    wsr = kvq.decode_workspace(w.B, w.Hq, w.Hkv, w.D, w.S, dev)
+
+    def rdec():
+        for K, V in layers:
+            kvq.decode_attn_varlen(qr, *K, *V, kvs, out=outr, workspace=wsr)
+    ms = _time_graph(stream, rdec, 20) / NL
+    rbytes = sum(2 * w.Hkv * n * (w.D + 5) for n in lens) + 2 * w.B * w.Hq * w.D * 2
+    res["ragged_decode"] = {"what": "kvq_decode_attn_varlen, batch 8 at kv_len 512..8192 (mean 3776), 32 q / 8 kv "
+                                    "heads, D=128", "us": ms * 1000, "tokens/s": w.B / (ms / 1000),
+                            "GB/s": rbytes / (ms / 1000) / 1e9, "frac": rbytes / (ms / 1000) / 1e9 / peak,
+                            "bytes": rbytes}
+    # ring cache (sink 0) decode step at the decode workload's scale: the 8192-slot cache has wrapped
+    # (position 10000); plan the slot, write K and V, build the mask, attend over all 8192 slots
+    ring_pos = torch.tensor([10000], dtype=torch.int32, device=dev)
+    slot_pos = torch.arange(w.S, dtype=torch.int32, device=dev) + (10000 - w.S)  # positions 1808..9999 held
+    smr = torch.empty(w.B, dtype=torch.int32, device=dev)
+    kvr = torch.empty(1, dtype=torch.int32, device=dev)
+    maskr = torch.empty((1, w.S), dtype=torch.float32, device=dev)
+    knr = torch.randn((w.B, w.Hkv, 1, w.D), device=dev).to(torch.bfloat16)
+    vnr = torch.randn((w.B, w.Hkv, 1, w.D), device=dev).to(torch.bfloat16)
+
+    def ring():
+        for K, V in layers:
+            kvq.sink_plan(ring_pos, w.B, 1, 0, slot_pos, smr, kvr)
+            kvq.write(0, knr, smr, *K)
+            kvq.write(0, vnr, smr, *V)
+            kvq.sink_mask(ring_pos, 1, slot_pos, maskr)
+            kvq.decode_attn(qr, *K, *V, kvr, out=outr, mask=maskr, workspace=wsr)
+    ms = _time_graph(stream, ring, 20) / NL
+    gbytes = 2 * w.B * w.Hkv * w.S * (w.D + 5) + w.S * 4 * 2 + 2 * w.B * w.Hq * w.D * 2
+    res["ring_decode_step"] = {"what": "ring cache (sink 0, 8192 slots, wrapped): sink_plan + 2 x kvq_write + "
+                                       "sink_mask + kvq_decode_attn over 8192 slots, batch 8, 32 q / 8 kv heads",
+                               "us": ms * 1000, "tokens/s": w.B / (ms / 1000), "GB/s": gbytes / (ms / 1000) / 1e9,
+                               "frac": gbytes / (ms / 1000) / 1e9 / peak, "bytes": gbytes}
+    del wsr
     # long-context decode: batch 1, 32 q / 16 kv heads, D=256, kv_len 131072 (1 GiB of codes > L2)
     lw = wl.LONG
     K = (torch.randint(-128, 128, (1, lw.Hkv, lw.S, lw.D), dtype=torch.int8, device=dev),

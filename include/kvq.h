@@ -58,6 +58,7 @@ extern "C" {
 #define KVQ_MODE_FP8_E5M2 4    /* E5M2 codes, f32 scale per 32 elements ("Normal", FLOAT8_E5M2 cache) */
 #define KVQ_MODE_MXFP8_E5M2 5  /* E5M2 codes, E8M0 scale per 32 elements (MX-FP8, FLOAT8_E5M2 cache) */
 #define KVQ_MODE_INT8_SYM 6    /* int8 codes (two's complement in a uint8 cache), f32 scale per 32 ("Normal", UINT8) */
+#define KVQ_MODE_INT4_AFFINE 7 /* TQ4: 4-bit codes two per byte, f32 scale + zero point 0..15 per (token, head) */
 
 /*
  * kvq_write -- quantize x and scatter it into the cache, in place.
@@ -84,6 +85,11 @@ extern "C" {
  *   modes 1, 4, 6: codes u8 [B, H, S, D]; scales float [B, H, S, D/32]; zero_points NULL
  *   modes 2, 5: codes u8 [B, H, S, D]; scales u8 (E8M0) [B, H, S, D/32]
  *   mode 3: codes u8   [B, H, S, D/2] (element 2i in the low nibble); scales u8 (E8M0)
+ *   mode 7 (TQ4): codes u8 [B, H, S, D/2] (element 2i in the low nibble); scales float
+ *           [B, H, S]; zero_points [B, H, S] holding 0..15.  The 4-bit form of mode 0:
+ *           scale = max((mx - mn)/15, FLT_EPSILON), zp = clamp(-rne(mn/scale), 0, 15),
+ *           q = clamp(rne(x/scale) + zp, 0, 15) (ExecuTorch PR 20351, commit notes: the
+ *           TQ4 cache is nibble-packed on the last dim and written along positions).
  *   With B = H = 1 the block modes are the IndexerQuantCache [num_slots, d] layout.
  *   Q_MAX: 448 (E4M3), 57344 (E5M2), 6 (E2M1), 127 (mode 6: q = rne(x / scale)
  *   clamped to [-127, 127], stored as its two's-complement byte).
@@ -91,7 +97,7 @@ extern "C" {
  *              power of two; 0 takes its exponent as it stands (the largest
  *              power of two not above it), codes then saturate at Q_MAX.
  *              Ignored by the other modes.
- * Sizes: mode 0 needs D in {64, 128, 256}; modes 1-3 need D % 32 == 0 and
+ * Sizes: modes 0 and 7 need D in {64, 128, 256}; the other modes need D % 32 == 0 and
  * D <= 8192 (KVQ_EUNSUPPORTED otherwise).  B, H, T >= 0 (0 enqueues nothing).
  * The arithmetic is binary32 with one round-to-nearest-even per operation, in
  * a fixed order, so codes, scales and zero points are reproducible bit for bit.
@@ -200,6 +206,23 @@ int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const i
                            const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
                            int64_t S, const int32_t *kv_lens, const float *mask, float sm_scale, void *out,
                            void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
+
+/*
+ * kvq_decode_attn_tq4 -- kvq_decode_attn over a TQ4 cache (kvq_write mode 7).
+ *
+ * Defines: as kvq_decode_attn, over the cache ExecuTorch PR 20351 (commit
+ * notes) calls TQ4: nibble-packed on the last dim, D/2 bytes per slot, which
+ * halves the decode's bytes again.  K = (k - k_zp) * k_scale with k a 4-bit
+ * code 0..15 (element 2i in the low nibble of byte i), V likewise.
+ *
+ * k, v         u8 [B, Hkv, S, D/2];  k_scale, v_scale float [B, Hkv, S];
+ *              k_zp, v_zp u8 [B, Hkv, S] holding 0..15.
+ * Other arguments, sizes and the workspace as for kvq_decode_attn.
+ */
+int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k, const float *k_scale,
+                        const uint8_t *k_zp, const uint8_t *v, const float *v_scale, const uint8_t *v_zp,
+                        int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
+                        void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
 
 /*
  * kvq_prefill_attn -- Lq-query (chunked prefill) attention over the int8 cache.

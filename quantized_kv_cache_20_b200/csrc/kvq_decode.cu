@@ -73,16 +73,18 @@ struct DecodeArgs {
   float qscale;  // sm_scale * log2(e)
 };
 
-template <int D_, int HC_, int NW_, int NST_>
+template <int D_, int HC_, int NW_, int NST_, bool Q4_ = false>
 struct Cfg {
   static constexpr int D = D_, HC = HC_, NW = NW_, NST = NST_;
+  static constexpr bool Q4 = Q4_;          // TQ4 cache: 4-bit codes, two per byte
+  static constexpr int CB = Q4 ? D / 2 : D;  // code bytes per slot
   static constexpr int L = D / 16;     // lanes per slot group (16 dims per lane)
   static constexpr int NG = 32 / L;    // slot groups per warp
   static constexpr int TS = 32 * NW;   // slots per tile
   // one ring stage
   static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = TS * D;
-  static constexpr int KS_OFF = 2 * TS * D;
+  static constexpr int V_OFF = TS * CB;
+  static constexpr int KS_OFF = 2 * TS * CB;
   static constexpr int VS_OFF = KS_OFF + 4 * TS;
   static constexpr int M_OFF = VS_OFF + 4 * TS;
   static constexpr int KZ_OFF = M_OFF + 4 * TS;
@@ -110,6 +112,22 @@ KVQ_DEVINL int dp4a_us(uint32_t a, uint32_t b, int c) {
   int d;
   asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
+}
+KVQ_DEVINL int dp4a_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+KVQ_DEVINL int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// 8 packed 4-bit codes (element 2i in the low nibble of byte i) -> the even
+// elements (0, 2, 4, 6) and the odd elements (1, 3, 5, 7) as bytes 0..15.
+KVQ_DEVINL void unpack_nibbles(uint32_t w, uint32_t &even, uint32_t &odd) {
+  even = w & 0x0F0F0F0Fu;
+  odd = (w >> 4) & 0x0F0F0F0Fu;
 }
 KVQ_DEVINL float ex2(float x) {
   float y;
@@ -173,7 +191,9 @@ KVQ_DEVINL int max_kv_len(const DecodeArgs &a, volatile int32_t *red, bool repor
   return r;
 }
 
-template <class C>
+// VARLEN: kv_len is one value per batch row (a.kv_per_batch); the scalar form
+// is a separate instantiation so it carries no per-unit state.
+template <class C, bool VARLEN>
 __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, HC = C::HC, NW = C::NW, NST = C::NST, L = C::L, NG = C::NG, TS = C::TS;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -237,20 +257,20 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         const int64_t bhk = u / a.nhc;  // = b * Hkv + hk
         if (u != kv_u_of) {
           kv_u_of = u;
-          kv_u = a.kv_per_batch ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
+          kv_u = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
         }
         const int s0 = t * TS;
         const int n = max(0, min(TS, kv_u - s0));
         const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
         const bool first = (t == 0) || (idx == t_begin);
         uint8_t *stage = smem + st * C::STAGE;
-        const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * D + 10) + (a.mask ? 4u * n16 : 0u) +
+        const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * C::CB + 10) + (a.mask ? 4u * n16 : 0u) +
                                (first ? 2u * HC * D : 0u);
         mbar_arrive_expect_tx(&full[st], bytes);  // 0 bytes: a plain arrival
         const int64_t row = bhk * a.S + s0;
         if (n16 > 0) {
-          bulk_g2s_hint(stage + C::K_OFF, a.k + row * D, n16 * D, &full[st], pol);
-          bulk_g2s_hint(stage + C::V_OFF, a.v + row * D, n16 * D, &full[st], pol);
+          bulk_g2s_hint(stage + C::K_OFF, a.k + row * C::CB, n16 * C::CB, &full[st], pol);
+          bulk_g2s_hint(stage + C::V_OFF, a.v + row * C::CB, n16 * C::CB, &full[st], pol);
           bulk_g2s(stage + C::KS_OFF, a.ks + row, n16 * 4, &full[st]);
           bulk_g2s(stage + C::VS_OFF, a.vs + row, n16 * 4, &full[st]);
           bulk_g2s(stage + C::KZ_OFF, a.kz + row, n16, &full[st]);
@@ -291,7 +311,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   float2 o2[HC][8];
   int64_t cur_u = -1;
   int seg = -1;
-  int kv_u = kv;  // kv_len of the current unit's batch row
+  int kv_u = kv;  // kv_len of the current unit's batch row (VARLEN), else kv
 
   auto close_segment = [&](int64_t u, int sg) {
     // (1) denominators over the lane group, then merge the NG groups of the warp
@@ -386,7 +406,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       if (cur_u >= 0) close_segment(cur_u, seg);
       cur_u = u;
       ++seg;
-      kv_u = a.kv_per_batch ? row_kv(a, static_cast<int>(u / a.nhc / a.Hkv)) : kv;
+      if constexpr (VARLEN) kv_u = row_kv(a, static_cast<int>(u / a.nhc / a.Hkv));
       // new unit: q (from this stage) onto the fixed-point grid, fresh softmax state
       const uint16_t *qs = reinterpret_cast<const uint16_t *>(stage + C::Q_OFF);
 #pragma unroll
@@ -415,7 +435,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
           uint32_t hw = 0, lw = 0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            int n = __float2int_rn(x[4 * k + j] * inv);
+            // byte j of word k pairs with the code of dim 4k + j; unpacked TQ4
+            // nibbles come as (0,2,4,6), (1,3,5,7), (8,10,12,14), (9,11,13,15)
+            const int dim = C::Q4 ? (k >> 1) * 8 + (k & 1) + 2 * j : 4 * k + j;
+            int n = __float2int_rn(x[dim] * inv);
             n = n > 32767 ? 32767 : (n < -32767 ? -32767 : n);
             s += n;
             hw |= (static_cast<uint32_t>(n >> 8) & 0xFFu) << (8 * j);
@@ -442,19 +465,39 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 #pragma unroll
       for (int jj = 0; jj < L; ++jj) {
         const int sl = wbase + g + NG * jj;
-        const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
+        if constexpr (C::Q4) {
+          const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::K_OFF + sl * C::CB + sub * 8);
+          uint4 c;
+          unpack_nibbles(cw.x, c.x, c.y);
+          unpack_nibbles(cw.y, c.z, c.w);
 #pragma unroll
-        for (int h = 0; h < HC; ++h) {
-          int acc = dp4a_ss(qhi[h][0], c.x, 0);
-          acc = dp4a_ss(qhi[h][1], c.y, acc);
-          acc = dp4a_ss(qhi[h][2], c.z, acc);
-          acc = dp4a_ss(qhi[h][3], c.w, acc);
-          acc *= 256;
-          acc = dp4a_us(qlo[h][0], c.x, acc);
-          acc = dp4a_us(qlo[h][1], c.y, acc);
-          acc = dp4a_us(qlo[h][2], c.z, acc);
-          acc = dp4a_us(qlo[h][3], c.w, acc);
-          part[jj][h] = acc;
+          for (int h = 0; h < HC; ++h) {
+            int acc = dp4a_su(qhi[h][0], c.x, 0);
+            acc = dp4a_su(qhi[h][1], c.y, acc);
+            acc = dp4a_su(qhi[h][2], c.z, acc);
+            acc = dp4a_su(qhi[h][3], c.w, acc);
+            acc *= 256;
+            acc = dp4a_uu(qlo[h][0], c.x, acc);
+            acc = dp4a_uu(qlo[h][1], c.y, acc);
+            acc = dp4a_uu(qlo[h][2], c.z, acc);
+            acc = dp4a_uu(qlo[h][3], c.w, acc);
+            part[jj][h] = acc;
+          }
+        } else {
+          const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
+#pragma unroll
+          for (int h = 0; h < HC; ++h) {
+            int acc = dp4a_ss(qhi[h][0], c.x, 0);
+            acc = dp4a_ss(qhi[h][1], c.y, acc);
+            acc = dp4a_ss(qhi[h][2], c.z, acc);
+            acc = dp4a_ss(qhi[h][3], c.w, acc);
+            acc *= 256;
+            acc = dp4a_us(qlo[h][0], c.x, acc);
+            acc = dp4a_us(qlo[h][1], c.y, acc);
+            acc = dp4a_us(qlo[h][2], c.z, acc);
+            acc = dp4a_us(qlo[h][3], c.w, acc);
+            part[jj][h] = acc;
+          }
         }
       }
       // ---- butterfly reduce-scatter: lane `sub` ends with slot jj = sub
@@ -524,7 +567,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         const int zp = static_cast<int8_t>(stage[C::VZ_OFF + wbase + sl]);
         const float mz = neg_magic_zp(zp);
         const float2 mz2 = make_float2(mz, mz);
-        const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + (wbase + sl) * D + sub * 16);
+        uint4 c;
+        if constexpr (C::Q4) {  // nibbles back to element order: bytes (0,1,2,3), (4,5,6,7), ...
+          const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::V_OFF + (wbase + sl) * C::CB + sub * 8);
+          uint32_t e0, o0, e1, o1;
+          unpack_nibbles(cw.x, e0, o0);
+          unpack_nibbles(cw.y, e1, o1);
+          c = make_uint4(__byte_perm(e0, o0, 0x5140), __byte_perm(e0, o0, 0x7362), __byte_perm(e1, o1, 0x5140),
+                         __byte_perm(e1, o1, 0x7362));
+        } else {
+          c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + (wbase + sl) * D + sub * 16);
+        }
         float2 vv2[8];
         codes4_to_f2(c.x, mz2, vv2[0], vv2[1]);
         codes4_to_f2(c.y, mz2, vv2[2], vv2[3]);
@@ -657,11 +710,19 @@ WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
   return w;
 }
 
-template <int D, int HC>
+template <class C, bool VARLEN>
+struct KernelTag {};  // names one decode_kernel instantiation for ensure_smem
+
+template <int D, int HC, bool Q4>
 int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
-  using C = Cfg<D, HC, DTune<D>::NW, DTune<D>::NST>;
-  if (const int st = ensure_smem<C>(decode_kernel<C>, C::SMEM)) return st;
-  decode_kernel<C><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
+  using C = Cfg<D, HC, DTune<D>::NW, DTune<D>::NST, Q4>;
+  if (a.kv_per_batch) {
+    if (const int st = ensure_smem<KernelTag<C, true>>(decode_kernel<C, true>, C::SMEM)) return st;
+    decode_kernel<C, true><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
+  } else {
+    if (const int st = ensure_smem<KernelTag<C, false>>(decode_kernel<C, false>, C::SMEM)) return st;
+    decode_kernel<C, false><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
+  }
   if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.merge_ctas));
@@ -677,13 +738,13 @@ int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
   return launch_status();
 }
 
-template <int D>
+template <int D, bool Q4>
 int dispatch_hc(const DecodeArgs &a, int hc, int ctas, cudaStream_t s) {
   switch (hc) {
-    case 1: return launch_decode<D, 1>(a, ctas, s);
-    case 2: return launch_decode<D, 2>(a, ctas, s);
-    case 3: return launch_decode<D, 3>(a, ctas, s);
-    default: return launch_decode<D, 4>(a, ctas, s);
+    case 1: return launch_decode<D, 1, Q4>(a, ctas, s);
+    case 2: return launch_decode<D, 2, Q4>(a, ctas, s);
+    case 3: return launch_decode<D, 3, Q4>(a, ctas, s);
+    default: return launch_decode<D, 4, Q4>(a, ctas, s);
   }
 }
 
@@ -702,7 +763,7 @@ namespace kvq {
 namespace {
 int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
                 const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp, int64_t S,
-                const int32_t *kv_len, int kv_per_batch, const float *mask, float sm_scale, void *out,
+                const int32_t *kv_len, int kv_per_batch, bool q4, const float *mask, float sm_scale, void *out,
                 void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S > INT32_MAX) return KVQ_EINVAL;
   if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
@@ -750,10 +811,17 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   }
   a.qscale = sm_scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q4) {
+    switch (D) {
+      case 64: return dispatch_hc<64, true>(a, hc, ctas, s);
+      case 128: return dispatch_hc<128, true>(a, hc, ctas, s);
+      default: return dispatch_hc<256, true>(a, hc, ctas, s);
+    }
+  }
   switch (D) {
-    case 64: return dispatch_hc<64>(a, hc, ctas, s);
-    case 128: return dispatch_hc<128>(a, hc, ctas, s);
-    default: return dispatch_hc<256>(a, hc, ctas, s);
+    case 64: return dispatch_hc<64, false>(a, hc, ctas, s);
+    case 128: return dispatch_hc<128, false>(a, hc, ctas, s);
+    default: return dispatch_hc<256, false>(a, hc, ctas, s);
   }
 }
 }  // namespace
@@ -763,8 +831,19 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
                                const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
                                int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
                                void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
-  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, mask, sm_scale, out,
-                          workspace, workspace_bytes, err_word, stream);
+  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, false, mask, sm_scale,
+                          out, workspace, workspace_bytes, err_word, stream);
+}
+
+extern "C" int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k,
+                                   const float *k_scale, const uint8_t *k_zp, const uint8_t *v, const float *v_scale,
+                                   const uint8_t *v_zp, int64_t S, const int32_t *kv_len, const float *mask,
+                                   float sm_scale, void *out, void *workspace, size_t workspace_bytes,
+                                   int32_t *err_word, void *stream) {
+  return kvq::decode_impl(q, B, Hq, Hkv, D, reinterpret_cast<const int8_t *>(k), k_scale,
+                          reinterpret_cast<const int8_t *>(k_zp), reinterpret_cast<const int8_t *>(v), v_scale,
+                          reinterpret_cast<const int8_t *>(v_zp), S, kv_len, 0, true, mask, sm_scale, out, workspace,
+                          workspace_bytes, err_word, stream);
 }
 
 extern "C" int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
@@ -772,8 +851,8 @@ extern "C" int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int
                                       const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_lens,
                                       const float *mask, float sm_scale, void *out, void *workspace,
                                       size_t workspace_bytes, int32_t *err_word, void *stream) {
-  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_lens, 1, mask, sm_scale, out,
-                          workspace, workspace_bytes, err_word, stream);
+  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_lens, 1, false, mask,
+                          sm_scale, out, workspace, workspace_bytes, err_word, stream);
 }
 
 // ----------------------------------------------------------------------------

@@ -174,7 +174,10 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
     }
     const int64_t r = (static_cast<int64_t>(b) * a.H + h) * a.S + (slot < 0 ? 0 : slot);
 
-    if constexpr (MODE == KVQ_MODE_INT8_AFFINE) {
+    if constexpr (MODE == KVQ_MODE_INT8_AFFINE || MODE == KVQ_MODE_INT4_AFFINE) {
+      // int8 (mode 0): codes [-128, 127]; TQ4 (mode 7): codes [0, 15], two per byte
+      constexpr bool Q4 = MODE == KVQ_MODE_INT4_AFFINE;
+      constexpr float kLevels = Q4 ? 15.0f : 255.0f, kLo = Q4 ? 0.0f : -128.0f, kHi = Q4 ? 15.0f : 127.0f;
       // mn = min(0, min x), mx = max(0, max x) over the row: exact, order-free,
       // taken two bf16 at a time
       __nv_bfloat162 mn2 = __float2bfloat162_rn(0.0f), mx2 = mn2;
@@ -191,10 +194,10 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
       if (slot < 0) continue;
-      float scale = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+      float scale = __fdiv_rn(__fsub_rn(mx, mn), kLevels);
       if (scale < FLT_EPSILON) scale = FLT_EPSILON;
-      int zp = -128 - __float2int_rn(__fdiv_rn(mn, scale));
-      zp = zp < -128 ? -128 : (zp > 127 ? 127 : zp);
+      int zp = static_cast<int>(kLo) - __float2int_rn(__fdiv_rn(mn, scale));
+      zp = zp < static_cast<int>(kLo) ? static_cast<int>(kLo) : (zp > static_cast<int>(kHi) ? static_cast<int>(kHi) : zp);
       const float rcp = __frcp_rn(scale);
       const float zpf = static_cast<float>(zp);
       // q = clamp(rne(x/scale) + zp) = rne(clamp(y + zp)) for y = x*rcp, taken
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
       for (int i = 0; i < 32; ++i) {
         const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
         const float y = __fmul_rn(x, rcp);
-        const float yz = fminf(fmaxf(__fadd_rn(y, zpf), -128.0f), 127.0f);
+        const float yz = fminf(fmaxf(__fadd_rn(y, zpf), kLo), kHi);
         const float tt = __fadd_rn(yz, kMagic);
         const float dd = __fsub_rn(yz, __fsub_rn(tt, kMagic));  // yz - rne(yz)
         worst = fmaxf(worst, fmaf(fabsf(y), 0x1p-22f, fabsf(dd)));
@@ -219,16 +222,30 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         for (int i = 0; i < 32; ++i) {
           const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
           int q = __float2int_rn(__fdiv_rn(x, scale)) + zp;
-          q = q < -128 ? -128 : (q > 127 ? 127 : q);
+          q = q < static_cast<int>(kLo) ? static_cast<int>(kLo) : (q > static_cast<int>(kHi) ? static_cast<int>(kHi) : q);
           t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
         }
       }
-      uint32_t w[8];
+      if constexpr (Q4) {
+        // the code sits in the low mantissa bits of t2; element 2i goes to the low nibble of byte i
+        uint32_t w[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<int8_t *>(a.codes) + r * a.D + gi * 32);
-      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        for (int k = 0; k < 4; ++k) {
+          uint32_t acc = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc |= (__float_as_uint(t2[8 * k + j]) & 0xFu) << (4 * j);
+          w[k] = acc;
+        }
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * (a.D >> 1) + gi * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<int8_t *>(a.codes) + r * a.D + gi * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
       if (gi == 0) {
         static_cast<float *>(a.scales)[r] = scale;
         a.zps[r] = static_cast<int8_t>(zp);
@@ -372,23 +389,23 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
                          const int64_t *x_strides, const int32_t *slot_mapping, int64_t num_slots, void *codes,
                          void *scales, int8_t *zero_points, int32_t *err_word, void *stream) {
   using namespace kvq;
-  if (mode < KVQ_MODE_INT8_AFFINE || mode > KVQ_MODE_INT8_SYM) return KVQ_EINVAL;
+  if (mode < KVQ_MODE_INT8_AFFINE || mode > KVQ_MODE_INT4_AFFINE) return KVQ_EINVAL;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || num_slots <= 0 || num_slots > INT32_MAX) return KVQ_EINVAL;
-  if (mode == KVQ_MODE_INT8_AFFINE) {
+  if (mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_INT4_AFFINE) {
     if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
   } else {
     if (D % 32 != 0 || D > 8192) return KVQ_EUNSUPPORTED;
   }
   if (static_cast<int64_t>(B) * H * T == 0) return KVQ_OK;
   if (!x || !x_strides || !slot_mapping || !codes || !scales) return KVQ_EINVAL;
-  if (mode == KVQ_MODE_INT8_AFFINE && !zero_points) return KVQ_EINVAL;
+  if ((mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_INT4_AFFINE) && !zero_points) return KVQ_EINVAL;
   // every row start 16-byte aligned: base aligned and strides multiples of 8 elements
   if (!aligned16(x) || !aligned16(codes)) return KVQ_EINVAL;
   for (int i = 0; i < 3; ++i)
     if (x_strides[i] < 0 || (x_strides[i] & 7) != 0) return KVQ_EINVAL;
   // float scales (modes 0, 1, 4, 6) must be 4-byte aligned; E8M0 scales are bytes
   const bool f32_scales = mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_FP8_E4M3 || mode == KVQ_MODE_FP8_E5M2 ||
-                          mode == KVQ_MODE_INT8_SYM;
+                          mode == KVQ_MODE_INT8_SYM || mode == KVQ_MODE_INT4_AFFINE;
   if (f32_scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return KVQ_EINVAL;
   // group indices use 32-bit arithmetic
   const int64_t groups = static_cast<int64_t>(B) * H * T * (D / 32);
@@ -423,6 +440,7 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
     case KVQ_MODE_MXFP4: return launch_write<KVQ_MODE_MXFP4>(a, s);
     case KVQ_MODE_FP8_E5M2: return launch_write<KVQ_MODE_FP8_E5M2>(a, s);
     case KVQ_MODE_MXFP8_E5M2: return launch_write<KVQ_MODE_MXFP8_E5M2>(a, s);
-    default: return launch_write<KVQ_MODE_INT8_SYM>(a, s);
+    case KVQ_MODE_INT8_SYM: return launch_write<KVQ_MODE_INT8_SYM>(a, s);
+    default: return launch_write<KVQ_MODE_INT4_AFFINE>(a, s);
   }
 }

@@ -36,11 +36,12 @@ MODE_MXFP4 = 3
 MODE_FP8_E5M2 = 4
 MODE_MXFP8_E5M2 = 5
 MODE_INT8_SYM = 6
+MODE_INT4_AFFINE = 7
 
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
-    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_attn_varlen", "kvq_prefill_attn",
-    "kvq_prefill_attn_varlen", "kvq_strerror", "kvq_version",
+    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
+    "kvq_prefill_attn", "kvq_prefill_attn_varlen", "kvq_strerror", "kvq_version",
 )
 
 _lib = None
@@ -76,6 +77,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_attn.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
         lib.kvq_decode_attn_varlen.argtypes = lib.kvq_decode_attn.argtypes
         lib.kvq_decode_attn_varlen.restype = I
+        lib.kvq_decode_attn_tq4.argtypes = lib.kvq_decode_attn.argtypes
+        lib.kvq_decode_attn_tq4.restype = I
         lib.kvq_decode_attn.restype = I
         lib.kvq_decode_attn_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, P]
         lib.kvq_decode_attn_static.restype = I
@@ -207,7 +210,22 @@ def decode_attn_varlen(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, *, out=No
                    varlen=True)
 
 
-def _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, workspace, err_word, varlen):
+def decode_attn_tq4(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,
+                    workspace=None, err_word=None) -> torch.Tensor:
+    """kvq_decode_attn_tq4: q [B, Hq, 1, D] bf16 over the TQ4 cache: k/v uint8 nibbles
+    [B, Hkv, S, D/2], scales float32 and zero points (0..15, uint8 or int8) [B, Hkv, S]."""
+    for n, t in (("k", k), ("v", v)):
+        _cuda(n, t, torch.uint8)
+    if k.shape[-1] * 2 != q.shape[-1]:
+        raise ValueError("a TQ4 cache holds D/2 bytes per slot")
+    kz = k_zp.view(torch.int8) if k_zp.dtype == torch.uint8 else k_zp
+    vz = v_zp.view(torch.int8) if v_zp.dtype == torch.uint8 else v_zp
+    return _decode(q, k.view(torch.int8), k_scale, kz, v.view(torch.int8), v_scale, vz, kv_len, out, mask,
+                   sm_scale, workspace, err_word, varlen=False, tq4=True)
+
+
+def _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, workspace, err_word, varlen,
+            tq4=False):
     if out is None:
         out = torch.empty_like(q)
     _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word)
@@ -219,7 +237,7 @@ def _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, 
         sm_scale = 1.0 / math.sqrt(D)
     if workspace is None:
         workspace = decode_workspace(B, Hq, Hkv, D, S, q.device)
-    name = "kvq_decode_attn_varlen" if varlen else "kvq_decode_attn"
+    name = "kvq_decode_attn_varlen" if varlen else ("kvq_decode_attn_tq4" if tq4 else "kvq_decode_attn")
     st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
                                _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
                                _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),

@@ -362,3 +362,43 @@ def test_prefill_varlen_rows_match_the_oracle_per_row(D):
         ref = oracle.sdpa(wl.u16(q[b:b + 1]), *_np(_slice(K, b)), *_np(_slice(V, b)), kv_len=lens[b],
                           sm_scale=1 / math.sqrt(D), is_causal=True)
         assert_attn_close(got[b:b + 1], ref, f"varlen prefill D={D} row {b} kv={lens[b]}")
+
+
+# ---------------------------------------------------------------------------- TQ4 cache
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("Hq,Hkv,kv_len", [(4, 2, 40), (8, 2, 1000), (6, 3, 777), (32, 8, 4096)])
+def test_tq4_decode_matches_the_oracle(D, Hq, Hkv, kv_len):
+    g = wl.generator(900 + D + Hq + kv_len)
+    B, S = 2, 4096
+    K = wl.int4_cache_random(B, Hkv, S, D, g)
+    V = wl.int4_cache_random(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    err = err_word()
+    out = kvq.decode_attn_tq4(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V], int32_scalar(kv_len),
+                              err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=1 / math.sqrt(D))
+    assert_attn_close(bf16_to_f64(out), ref, f"tq4 decode D={D} Hq={Hq} Hkv={Hkv} kv={kv_len}")
+
+
+def test_tq4_decode_with_mask_and_written_cache():
+    """Write K/V through kvq_write mode 7, then attend with an additive mask."""
+    g = wl.generator(950)
+    B, Hq, Hkv, D, S, T = 1, 8, 2, 128, 512, 300
+    x_k = wl.bf16_normal((B, Hkv, T, D), g)
+    x_v = wl.bf16_normal((B, Hkv, T, D), g)
+    sm = torch.arange(T, dtype=torch.int32)
+    K = [t.to(DEV) for t in wl.int4_cache_random(B, Hkv, S, D, g)]
+    V = [t.to(DEV) for t in wl.int4_cache_random(B, Hkv, S, D, g)]
+    kvq.write(7, x_k.to(DEV), sm.to(DEV), *K)
+    kvq.write(7, x_v.to(DEV), sm.to(DEV), *V)
+    mask = torch.zeros(S, dtype=torch.float32)
+    mask[torch.randperm(T, generator=torch.Generator().manual_seed(3))[:90]] = -float("inf")
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    out = kvq.decode_attn_tq4(q.to(DEV), *K, *V, int32_scalar(T), mask=mask.to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.sdpa(wl.u16(q), *[t.cpu().numpy() for t in K], *[t.cpu().numpy() for t in V], kv_len=T,
+                      sm_scale=1 / math.sqrt(D), mask=mask.numpy()[None, :])
+    assert_attn_close(bf16_to_f64(out), ref, "tq4 decode, written cache, masked")

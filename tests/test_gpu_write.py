@@ -16,6 +16,9 @@ def _prefill(mode, B, H, S, D, g):
     if mode == 0:
         c, s, z = wl.int8_cache_random(B, H, S, D, g)
         return [c, s, z]
+    if mode == 7:
+        c, s, z = wl.int4_cache_random(B, H, S, D, g)
+        return [c, s, z]
     c, s = wl.block_cache_random(B, H, S, D, mode, g)
     return [c, s, None]
 
@@ -200,3 +203,22 @@ def test_empty_and_all_skipped():
     kvq.write(0, x0, torch.empty(0, dtype=torch.int32, device=DEV), *cache)
     for a, b in zip(cache, before):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 5, 37), (2, 8, 129)])
+def test_tq4_write_ragged_shapes(D, shape):
+    """Mode 7 (TQ4: 4-bit affine per token and head, two codes per byte):
+    codes, scales and zero points bit-exact, untouched slots byte-equal."""
+    B, H, T = shape
+    g = wl.generator(4000 + D + 7 * T)
+    S = 2 * T + 3
+    x = wl.bf16_normal((B, H, T, D), g, outlier_p=0.02, outlier_scale=8.0)
+    sp = _special_rows(D, g)
+    n = min(T, sp.shape[0])
+    x[0, 0, :n] = sp[:n]
+    sm = torch.stack([wl.slot_mapping_random(T, S, T // 5, g) for _ in range(B)]).reshape(-1)
+    cache0 = _prefill(7, B, H, S, D, g)
+    gpu, ref, err, oerr = _run_both(7, x, sm, cache0, S)
+    assert err == 0 and oerr == 0
+    _assert_equal(gpu, ref, f"tq4 D={D} shape={shape}")
