@@ -94,6 +94,11 @@ def _load():
         lib.kvqo_sdpa_row.restype = None
         lib.kvqo_sdpa.argtypes = sdpa_args + [P]
         lib.kvqo_sdpa.restype = None
+        lib.kvqo_dequant_block.argtypes = [i32, P, P, i64, i32, P]
+        lib.kvqo_dequant_block.restype = None
+        lib.kvqo_sdpa_dense_row.argtypes = [P, i32, i32, i32, i32, P, P, i32, i64, i32, P, i32, f32, i32, i32, i32,
+                                             P]
+        lib.kvqo_sdpa_dense_row.restype = None
         _lib = lib
         return lib
 
@@ -285,3 +290,44 @@ def sdpa_rows(q_bits, k, ks, kz, v, vs, vz, kv_len: int, sm_scale: float, rows, 
 def dequant_int8(codes: np.ndarray, scale: np.ndarray, zp: np.ndarray) -> np.ndarray:
     """(q - zp) * scale in fp64 (the dequantization of the affine int8 reading)."""
     return (codes.astype(np.float64) - zp.astype(np.float64)[..., None]) * scale.astype(np.float64)[..., None]
+
+
+# --- attention over the per-32 block caches ---------------------------------------
+
+def dequant_block(mode: int, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """IndexerQuantCache, 计算公式 (x ~ code * scale_g): the fp64 values of a block
+    cache, codes [.., d] (mode 3: [.., d/2]) and scales [.., d/32]."""
+    codes = np.ascontiguousarray(codes).view(np.uint8)
+    scales = np.ascontiguousarray(scales)
+    d = scales.shape[-1] * 32
+    rows = int(np.prod(codes.shape[:-1]))
+    out = np.zeros(codes.shape[:-1] + (d,), np.float64)
+    _load().kvqo_dequant_block(int(mode), _ptr(codes), _ptr(scales), rows, d, _ptr(out))
+    return out
+
+
+def sdpa_dense(q_bits, K: np.ndarray, V: np.ndarray, kv_len: int, sm_scale: float, mask=None,
+               is_causal: bool = False) -> np.ndarray:
+    """The same attention as ``sdpa`` over K, V given as fp64 values [B, Hkv, S, D]."""
+    q = _u16(q_bits)
+    K = np.ascontiguousarray(K, np.float64)
+    V = np.ascontiguousarray(V, np.float64)
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.float32)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = K.shape[1], K.shape[2]
+    out = np.zeros((B, Hq, Lq, D), np.float64)
+    lib = _load()
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(Lq):
+                lib.kvqo_sdpa_dense_row(_ptr(q), B, Hq, Lq, D, _ptr(K), _ptr(V), Hkv, S, int(kv_len), _ptr(m),
+                                        int(bool(is_causal)), float(sm_scale), b, h, i, out[b, h, i].ctypes.data)
+    return out
+
+
+def sdpa_block(mode: int, q_bits, k_codes, k_scales, v_codes, v_scales, kv_len: int, sm_scale: float,
+               mask=None, is_causal: bool = False) -> np.ndarray:
+    """fp64 attention over a per-32 block cache: dequantize, then ``sdpa_dense``."""
+    return sdpa_dense(q_bits, dequant_block(mode, k_codes, k_scales), dequant_block(mode, v_codes, v_scales),
+                      kv_len, sm_scale, mask=mask, is_causal=is_causal)
+

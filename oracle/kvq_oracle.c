@@ -518,3 +518,82 @@ void kvqo_sdpa(const uint16_t *q, int B, int Hq, int Lq, int D, int kbits, const
                 kvqo_sdpa_row(q, B, Hq, Lq, D, kbits, k, ks, kz, v, vs, vz, Hkv, S, kv_len, mask, is_causal,
                               sm_scale, b, h, i, out + (((int64_t)b * Hq + h) * Lq + i) * D);
 }
+
+/* ------------------------------------------------------------------------- */
+/* [P5] dequantization of the per-32 block caches (the inverse the page's    */
+/* formula implies: x ~ code_value * scale_g), for attention over them:      */
+/*   modes 1, 4, 6: code value (E4M3 / E5M2 / int8) * float32 scale          */
+/*   modes 2, 5, 3: code value (E4M3 / E5M2 / E2M1 nibble) * 2^(e - 127)     */
+/* codes: rows x d (mode 3: rows x d/2, element 2i in the low nibble);       */
+/* scales: rows x d/32 (float32 or E8M0 bytes).  out: rows x d, fp64.        */
+/* ------------------------------------------------------------------------- */
+void kvqo_dequant_block(int mode, const uint8_t *codes, const void *scales, int64_t rows, int d, double *out)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int i = 0; i < d; ++i) {
+            int64_t g = r * (d / 32) + i / 32;
+            double code, scale;
+            if (mode == KVQO_MODE_MXFP4) {
+                uint8_t byte = codes[r * (d / 2) + i / 2];
+                code = kvqo_e2m1_value((i & 1) ? (byte >> 4) : (byte & 15));
+            } else {
+                uint8_t c = codes[r * d + i];
+                if (mode == KVQO_MODE_FP8_E4M3 || mode == KVQO_MODE_MXFP8)
+                    code = kvqo_e4m3_value(c);
+                else if (mode == KVQO_MODE_FP8_E5M2 || mode == KVQO_MODE_MXFP8_E5M2)
+                    code = kvqo_e5m2_value(c);
+                else
+                    code = (double)(int8_t)c; /* KVQO_MODE_INT8_SYM */
+            }
+            if (mode == KVQO_MODE_FP8_E4M3 || mode == KVQO_MODE_FP8_E5M2 || mode == KVQO_MODE_INT8_SYM)
+                scale = (double)((const float *)scales)[g];
+            else
+                scale = kvqo_e8m0_value(((const uint8_t *)scales)[g]);
+            out[r * d + i] = code * scale;
+        }
+    }
+}
+
+/* fp64 attention for one row over dense fp64 K, V [B, Hkv, S, D] -- the same */
+/* definition as kvqo_sdpa_row ([P3] shapes and GQA, [P4] kv_len and causal  */
+/* rule, [P1] additive mask), with K and V given as values.                  */
+void kvqo_sdpa_dense_row(const uint16_t *q, int B, int Hq, int Lq, int D, const double *K, const double *V,
+                         int Hkv, int64_t S, int32_t kv_len, const float *mask, int is_causal, float sm_scale,
+                         int b, int h, int i, double *out)
+{
+    int G = Hq / Hkv, hk = h / G;
+    const uint16_t *qr = q + (((int64_t)b * Hq + h) * Lq + i) * D;
+    int64_t base = ((int64_t)b * Hkv + hk) * S;
+    double *s = (double *)malloc(sizeof(double) * (kv_len > 0 ? (size_t)kv_len : 1));
+    double m = -INFINITY, l = 0.0;
+    (void)B;
+    for (int64_t j = 0; j < kv_len; ++j) {
+        if (is_causal && j > (int64_t)kv_len - Lq + i) {
+            s[j] = -INFINITY;
+        } else {
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d)
+                dot += (double)bf16_to_float(qr[d]) * K[(base + j) * D + d];
+            s[j] = dot * (double)sm_scale + (mask ? (double)mask[(int64_t)i * S + j] : 0.0);
+        }
+        if (s[j] > m)
+            m = s[j];
+    }
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    if (m == -INFINITY) {
+        free(s);
+        return;
+    }
+    for (int64_t j = 0; j < kv_len; ++j) {
+        double p = exp(s[j] - m);
+        l += p;
+        if (p == 0.0)
+            continue;
+        for (int d = 0; d < D; ++d)
+            out[d] += p * V[(base + j) * D + d];
+    }
+    for (int d = 0; d < D; ++d)
+        out[d] /= l;
+    free(s);
+}

@@ -148,3 +148,72 @@ def test_tq4_cache_matches_torch_sdpa_fp64(is_causal):
     Vu = (_unpack4(V[0].numpy()), V[1], V[2])
     ref = _torch_ref(q, Ku, Vu, kv_len, sm, is_causal=is_causal)
     np.testing.assert_allclose(ours, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------- block caches
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # OCP MX FP4 E2M1 magnitudes
+
+
+def _dequant_independent(mode, codes, scales):
+    """Block-cache values computed here with torch's float8 decoders (modes 1, 2, 4, 5),
+    the OCP E2M1 magnitudes (mode 3), int8 (mode 6) and 2^(e-127) for E8M0."""
+    c = torch.from_numpy(np.ascontiguousarray(codes))
+    if mode == 3:
+        lo, hi = (c & 15).long(), (c >> 4).long()
+        nib = torch.stack([lo, hi], dim=-1).reshape(*c.shape[:-1], -1)
+        mag = torch.tensor(E2M1_VALUES, dtype=torch.float64)[nib & 7]
+        val = torch.where(nib >= 8, -mag, mag)
+    elif mode in (1, 2):
+        val = c.view(torch.float8_e4m3fn).double()
+    elif mode in (4, 5):
+        val = c.view(torch.float8_e5m2).double()
+    else:
+        val = c.view(torch.int8).double()
+    sc = torch.from_numpy(np.ascontiguousarray(scales))
+    sc = sc.double() if mode in (1, 4, 6) else torch.exp2(sc.double() - 127)
+    return (val.reshape(*val.shape[:-1], -1, 32) * sc[..., None]).reshape(val.shape).numpy()
+
+
+@pytest.mark.parametrize("mode", [1, 2, 3, 4, 5, 6])
+def test_block_dequant_matches_independent_decode(mode):
+    g = wl.generator(70 + mode)
+    codes, scales = wl.block_cache_random(2, 3, 5, 64, mode, g)
+    ours = oracle.dequant_block(mode, codes.numpy(), scales.numpy())
+    ref = _dequant_independent(mode, codes.numpy(), scales.numpy())
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(ours))          # NaN codes stay NaN
+    assert np.array_equal(ours[fin], ref[fin])
+
+
+@pytest.mark.parametrize("mode", [1, 2, 3, 4, 5, 6])
+def test_block_dequant_inverts_the_quantizer_within_its_bound(mode):
+    g = wl.generator(80 + mode)
+    x = wl.bf16_normal((16, 128), g, outlier_p=0.02, outlier_scale=10.0)
+    for r in range(x.shape[0]):
+        codes, scales = oracle.block_row(mode, wl.u16(x[r]))
+        deq = oracle.dequant_block(mode, codes[None], scales[None])[0]
+        xv = x[r].double().numpy()
+        amax = np.abs(xv.reshape(-1, 32)).max(axis=1).repeat(32)
+        # relative half-steps: E4M3 2^-4, E5M2 2^-3, E2M1 up to 1/6 of amax... bound by a step of the grid
+        step = {1: 2.0 ** -3, 2: 2.0 ** -3, 4: 2.0 ** -2, 5: 2.0 ** -2, 3: 1.0 / 3, 6: 1.0 / 127}[mode]
+        assert np.all(np.abs(deq - xv) <= step * amax + 1e-30), (mode, r)
+
+
+def test_dense_sdpa_matches_torch_fp64():
+    g = torch.Generator().manual_seed(91)
+    B, Hq, Hkv, Lq, D, S = 2, 6, 3, 3, 16, 24
+    q = wl.bf16_normal((B, Hq, Lq, D), wl.generator(92))
+    K = torch.randn((B, Hkv, S, D), generator=g, dtype=torch.float64)
+    V = torch.randn((B, Hkv, S, D), generator=g, dtype=torch.float64)
+    kv_len, sm = 21, 0.3
+    for is_causal in (False, True):
+        ours = oracle.sdpa_dense(wl.u16(q), K.numpy(), V.numpy(), kv_len, sm, is_causal=is_causal)
+        G = Hq // Hkv
+        kd, vd = K[:, :, :kv_len].repeat_interleave(G, 1), V[:, :, :kv_len].repeat_interleave(G, 1)
+        bias = torch.zeros(Lq, kv_len, dtype=torch.float64)
+        if is_causal:
+            i, j = torch.arange(Lq)[:, None], torch.arange(kv_len)[None, :]
+            bias = bias.masked_fill(j > kv_len - Lq + i, -math.inf)
+        ref = F.scaled_dot_product_attention(q.double(), kd, vd, attn_mask=bias, scale=float(np.float32(sm)))
+        np.testing.assert_allclose(ours, ref.numpy(), rtol=1e-12, atol=1e-12)
