@@ -578,6 +578,36 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
                          "frac": dbytes / (ms / 1000) / 1e9 / peak, "bytes": dbytes}
     del tq, wsq
     torch.cuda.empty_cache()
+    # decode over the per-32 block caches (E4M3 + f32 scale, MX-FP8, MX-FP4) at the decode workload's shape
+    for mode, name in ((1, "fp8_e4m3"), (2, "mxfp8"), (3, "mxfp4")):
+        row = w.D // 2 if mode == 3 else w.D
+        f32 = mode == 1
+        bl = []
+        for _ in range(NL):
+            kc = torch.empty((w.B, w.Hkv, w.S, row), dtype=torch.uint8, device=dev)
+            ksc = torch.empty((w.B, w.Hkv, w.S, w.D // 32), dtype=torch.float32 if f32 else torch.uint8, device=dev)
+            vc, vsc = torch.empty_like(kc), torch.empty_like(ksc)
+            kvq.write(mode, xk, sm_fill, kc, ksc)
+            kvq.write(mode, xv, sm_fill, vc, vsc)
+            bl.append((kc, ksc, vc, vsc))
+        qb = torch.randn((w.B, w.Hq, 1, w.D), device=dev).to(torch.bfloat16)
+        ob = torch.empty_like(qb)
+        kvb = torch.tensor([w.kv_len - 1], dtype=torch.int32, device=dev)
+        wsb = torch.empty(max(16, kvq.load().kvq_decode_block_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.S)),
+                          dtype=torch.uint8, device=dev)
+
+        def bdec():
+            for kc, ksc, vc, vsc in bl:
+                kvq.decode_attn_block(mode, qb, kc, ksc, vc, vsc, kvb, out=ob, workspace=wsb)
+        ms = _time_graph(stream, bdec, 20) / NL
+        sb = (w.D // 32) * (4 if f32 else 1)
+        bbytes = 2 * w.B * w.Hkv * (w.kv_len - 1) * (row + sb) + 2 * w.B * w.Hq * w.D * 2
+        res[f"block_decode_{name}"] = {"what": f"kvq_decode_attn_block mode {mode}, batch 8, 32 q / 8 kv heads, "
+                                               f"D=128, kv_len 4095", "us": ms * 1000, "tokens/s": w.B / (ms / 1000),
+                                       "GB/s": bbytes / (ms / 1000) / 1e9,
+                                       "frac": bbytes / (ms / 1000) / 1e9 / peak, "bytes": bbytes}
+        del bl, wsb
+    torch.cuda.empty_cache()
     # the lines below read past position 4095: fill slots 4095..8191 of every layer first
     Tr = w.S - Tf
     xkr = torch.randn((w.B, w.Hkv, Tr, w.D), device=dev).to(torch.bfloat16)

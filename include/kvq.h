@@ -225,6 +225,36 @@ int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint
                         void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
 
 /*
+ * kvq_decode_block_workspace_bytes -- size of the kvq_decode_attn_block workspace
+ * for (B, Hq, Hkv, D, S) on the current device; 0 for sizes it rejects.  The
+ * workspace holds per-split partials only and needs no initialisation.
+ */
+size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
+
+/*
+ * kvq_decode_attn_block -- one-query attention over a per-32 block cache
+ * (kvq_write modes 1-6).
+ *
+ * Defines: the attention of kvq_decode_attn, with K and V read from the
+ * IndexerQuantCache block format (计算公式: x ~ code * scale_g, one scale per 32
+ * elements along the head dim): E4M3 / E5M2 / int8 codes with float scales
+ * (modes 1, 4, 6), E4M3 / E5M2 codes with E8M0 scales (modes 2, 5), E2M1 codes
+ * two per byte with E8M0 scales (mode 3).
+ *
+ * mode         1..6, the kvq_write mode that wrote the cache.
+ * k_codes, v_codes  u8 [B, Hkv, S, D] (mode 3: [B, Hkv, S, D/2]).
+ * k_scales, v_scales  [B, Hkv, S, D/32]: float (modes 1, 4, 6) or E8M0 bytes.
+ * kv_len, mask, q, out, sm_scale, err_word as for kvq_decode_attn.
+ * workspace    device buffer of at least kvq_decode_block_workspace_bytes().
+ * Launches two kernels on `stream` (the split attention, the merge).
+ * Sizes: D in {64, 128, 256}; Hq % Hkv == 0 with Hq / Hkv <= 8; S % 16 == 0.
+ */
+int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k_codes,
+                          const void *k_scales, const uint8_t *v_codes, const void *v_scales, int64_t S,
+                          const int32_t *kv_len, const float *mask, float sm_scale, void *out, void *workspace,
+                          size_t workspace_bytes, int32_t *err_word, void *stream);
+
+/*
  * kvq_prefill_attn -- Lq-query (chunked prefill) attention over the int8 cache.
  *
  * Defines: as kvq_decode_attn, plus ExecuTorch PR 20351 commit notes (the

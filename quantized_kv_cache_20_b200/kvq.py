@@ -41,7 +41,8 @@ MODE_INT4_AFFINE = 7
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
     "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
-    "kvq_prefill_attn", "kvq_prefill_attn_varlen", "kvq_strerror", "kvq_version",
+    "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
+    "kvq_strerror", "kvq_version",
 )
 
 _lib = None
@@ -79,6 +80,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_attn_varlen.restype = I
         lib.kvq_decode_attn_tq4.argtypes = lib.kvq_decode_attn.argtypes
         lib.kvq_decode_attn_tq4.restype = I
+        lib.kvq_decode_block_workspace_bytes.argtypes = [I, I, I, I, I64]
+        lib.kvq_decode_block_workspace_bytes.restype = SZ
+        lib.kvq_decode_attn_block.argtypes = [I, P, I, I, I, I, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
+        lib.kvq_decode_attn_block.restype = I
         lib.kvq_decode_attn.restype = I
         lib.kvq_decode_attn_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, P]
         lib.kvq_decode_attn_static.restype = I
@@ -208,6 +213,41 @@ def decode_attn_varlen(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, *, out=No
         raise ValueError("kv_lens must hold one entry per batch row")
     return _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_lens, out, mask, sm_scale, workspace, err_word,
                    varlen=True)
+
+
+def decode_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len, *, out=None, mask=None,
+                      sm_scale=None, workspace=None, err_word=None) -> torch.Tensor:
+    """kvq_decode_attn_block: q [B, Hq, 1, D] bf16 over a per-32 block cache written by
+    kvq_write mode 1..6: codes uint8 [B, Hkv, S, D] (mode 3: D/2), scales [B, Hkv, S, D/32]
+    (float32 for modes 1, 4, 6, E8M0 uint8 otherwise)."""
+    _cuda("q", q, torch.bfloat16)
+    for n, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _cuda(n, t, torch.uint8)
+    f32 = mode in (MODE_FP8_E4M3, MODE_FP8_E5M2, MODE_INT8_SYM)
+    for n, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _cuda(n, t, torch.float32 if f32 else torch.uint8)
+    _cuda("kv_len", kv_len, torch.int32)
+    _cuda("mask", mask, torch.float32)
+    _cuda("err_word", err_word, torch.int32)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k_codes.shape[1], k_codes.shape[2]
+    if Lq != 1:
+        raise ValueError("decode takes one query row")
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda("out", out, torch.bfloat16)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        nbytes = int(load().kvq_decode_block_workspace_bytes(B, Hq, Hkv, D, S))
+        with torch.cuda.device(q.device):
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    st = load().kvq_decode_attn_block(int(mode), _ptr(q), B, Hq, Hkv, D, _ptr(k_codes), _ptr(k_scales),
+                                      _ptr(v_codes), _ptr(v_scales), S, _ptr(kv_len), _ptr(mask),
+                                      float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                      _ptr(err_word), _stream(q.device))
+    _check("kvq_decode_attn_block", st)
+    return out
 
 
 def decode_attn_tq4(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,

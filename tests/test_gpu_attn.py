@@ -402,3 +402,68 @@ def test_tq4_decode_with_mask_and_written_cache():
     ref = oracle.sdpa(wl.u16(q), *[t.cpu().numpy() for t in K], *[t.cpu().numpy() for t in V], kv_len=T,
                       sm_scale=1 / math.sqrt(D), mask=mask.numpy()[None, :])
     assert_attn_close(bf16_to_f64(out), ref, "tq4 decode, written cache, masked")
+
+
+# ---------------------------------------------------------------------------- block caches (modes 1-6)
+
+def _block_cache_from_writer(mode, B, Hkv, S, D, kv, g, round_scale=True):
+    """A block cache filled by kvq_write from bf16 N(0, 1) rows (1% x10 outliers):
+    slots [0, kv) written, the rest left at zero codes."""
+    x = wl.bf16_normal((B, Hkv, kv, D), g, outlier_p=0.01, outlier_scale=10.0)
+    row = D // 2 if mode == 3 else D
+    f32 = mode in (1, 4, 6)
+    codes = torch.zeros((B, Hkv, S, row), dtype=torch.uint8, device=DEV)
+    scales = torch.zeros((B, Hkv, S, D // 32), dtype=torch.float32 if f32 else torch.uint8, device=DEV)
+    sm = torch.arange(kv, dtype=torch.int32).repeat(B)
+    kvq.write(mode, x.to(DEV), sm.to(DEV), codes, scales, round_scale=round_scale)
+    return codes, scales
+
+
+@pytest.mark.parametrize("mode", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_block_cache_decode_matches_the_oracle(mode, D):
+    g = wl.generator(1100 + 10 * mode + D)
+    B, Hq, Hkv, S, kv = 2, 8, 2, 1024, 777
+    Kc, Ks = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    Vc, Vs = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    err = err_word()
+    out = kvq.decode_attn_block(mode, q.to(DEV), Kc, Ks, Vc, Vs, int32_scalar(kv), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle.sdpa_block(mode, wl.u16(q), Kc.cpu().numpy(), Ks.cpu().numpy(), Vc.cpu().numpy(),
+                            Vs.cpu().numpy(), kv_len=kv, sm_scale=1 / math.sqrt(D))
+    assert_attn_close(bf16_to_f64(out), ref, f"block-cache decode mode {mode} D={D}")
+
+
+@pytest.mark.parametrize("mode", [1, 3])
+@pytest.mark.parametrize("Hq,Hkv,kv", [(4, 4, 1), (8, 1, 300), (32, 8, 4096)])
+def test_block_cache_decode_shapes_and_mask(mode, Hq, Hkv, kv):
+    g = wl.generator(1200 + mode + Hq + kv)
+    B, D, S = 1, 128, 4096
+    Kc, Ks = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    Vc, Vs = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    mask = torch.zeros(S, dtype=torch.float32)
+    mask[torch.randperm(kv, generator=torch.Generator().manual_seed(kv))[: kv // 3]] = -float("inf")
+    mask[0] = 0.0
+    out = kvq.decode_attn_block(mode, q.to(DEV), Kc, Ks, Vc, Vs, int32_scalar(kv), mask=mask.to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.sdpa_block(mode, wl.u16(q), Kc.cpu().numpy(), Ks.cpu().numpy(), Vc.cpu().numpy(),
+                            Vs.cpu().numpy(), kv_len=kv, sm_scale=1 / math.sqrt(D), mask=mask.numpy()[None, :])
+    assert_attn_close(bf16_to_f64(out), ref, f"block-cache decode mode {mode} Hq={Hq} Hkv={Hkv} kv={kv}")
+
+
+def test_block_cache_decode_empty_and_out_of_range():
+    g = wl.generator(1300)
+    B, Hq, Hkv, D, S = 1, 4, 2, 64, 512
+    Kc, Ks = _block_cache_from_writer(1, B, Hkv, S, D, 100, g)
+    Vc, Vs = _block_cache_from_writer(1, B, Hkv, S, D, 100, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g).to(DEV)
+    z = kvq.decode_attn_block(1, q, Kc, Ks, Vc, Vs, int32_scalar(0))
+    assert torch.all(z == 0)
+    err = err_word()
+    a = kvq.decode_attn_block(1, q, Kc, Ks, Vc, Vs, int32_scalar(99999), err_word=err)
+    b = kvq.decode_attn_block(1, q, Kc, Ks, Vc, Vs, int32_scalar(S))
+    torch.cuda.synchronize()
+    assert err.item() & kvq.KVQ_ERR_KV_LEN_RANGE and torch.equal(a, b)
