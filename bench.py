@@ -38,6 +38,9 @@ METRIC = "KV-write GB/s + int8-KV decode attn tokens/s, % of B200 HBM roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# DRAM bytes of one decode_kernel launch on the decode workload, read + write, from one ncu
+# capture of the current kernel (69,871,616 + 775,168); algorithmic bytes are 69,861,376.
+DECODE_TRAFFIC_BYTES = 70646784
 
 
 def _args():
@@ -391,7 +394,9 @@ def run_kvq(args, dist: Dist):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
                 "kernel": "decode_kernel (split-K int8 decode attention)", "bytes_per_launch": dec_bytes,
-                "launch_us": dec_ms * 1000.0, "traffic": None}
+                "launch_us": dec_ms * 1000.0, "traffic": DECODE_TRAFFIC_BYTES,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_kernel on this "
+                                  "workload (profiles/decode_kernel__decode_b8_kv4096.md)"}
 
     # ---- end to end through the binding with host buffers
     e2e = _e2e(args, dist, kvq, layers, ws, kv_len, sm_step)
