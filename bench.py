@@ -39,8 +39,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM bytes of one decode_kernel launch on the decode workload, read + write, from one ncu
-# capture of the current kernel (69,871,616 + 775,168); algorithmic bytes are 69,861,376.
-DECODE_TRAFFIC_BYTES = 70646784
+# capture of the current kernel; None until the current kernel has been captured.
+DECODE_TRAFFIC_BYTES = None
 
 
 def _args():
@@ -409,7 +409,7 @@ def run_kvq(args, dist: Dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": 4 * nsteps, "clocks": clk, "detail": detail,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * nsteps, "clocks": clk, "detail": detail,
     }
     if dist.rank == 0 and dist.world == 1:
         steps_c, el_c, _ = _oracle_decode_steps(args.cpu_seconds)

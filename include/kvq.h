@@ -149,8 +149,11 @@ int kvq_sink_mask(const int32_t *input_pos, int Lq, const int32_t *slot_pos, int
  * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S) on the
  * current device (the size depends on its SM count), or 0 for arguments
  * kvq_decode_attn would reject.  The workspace holds per-CTA partial results
- * only: it needs no initialisation and can be reused by later calls in stream
- * order (not by two calls running at the same time).
+ * and one merge counter per (batch row, kv head, head chunk).  It must be
+ * zero-filled before its first use (cudaMemsetAsync); every call that
+ * completes leaves the counters at zero again, so the workspace can be reused
+ * by later calls in stream order without clearing (not by two calls running at
+ * the same time).  After a call that set KVQ_ERR_TIMEOUT, zero it again.
  */
 size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
 
@@ -176,9 +179,12 @@ size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
  * mask         nullable float [S] (row 0 of an [Lq, S] mask), added to the
  *              scaled scores; -INFINITY hides a slot.  A row that sees no slot
  *              outputs zeros.
- * workspace    device buffer of workspace_bytes >= kvq_decode_workspace_bytes().
- * Launches two kernels on `stream`: the split decode and, behind it, the merge
- * of split partials (programmatic dependent launch).
+ * workspace    device buffer of workspace_bytes >= kvq_decode_workspace_bytes(),
+ *              zero-filled before its first use (see above).
+ * Launches one kernel on `stream`, as a programmatic dependent launch: it may
+ * start while the kernel before it drains, and reads nothing before that kernel
+ * has completed.  The CTA that completes a split (b, kv head) merges its
+ * partials in CTA order, so results do not depend on timing.
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; every pointer
  * 16-byte aligned.
  */
@@ -316,10 +322,11 @@ int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D
  * above KVQ_STATIC_SCRATCH_BYTES) returns KVQ_ESCRATCH and enqueues nothing.
  * The first call on a device looks up the buffer's device address (with that
  * device current); make that first call before capturing a stream into a CUDA
- * graph.  All calls on a device share the one buffer, which keeps whatever the
- * last call left in it: nothing in it has to start at zero, but two calls
+ * graph.  All calls on a device share the one buffer: it starts zeroed and
+ * every call that completes leaves its merge counters at zero, but two calls
  * whose kernels overlap on the GPU (different streams without ordering) race
- * on it and produce wrong results.
+ * on it and produce wrong results.  After a call that set KVQ_ERR_TIMEOUT,
+ * kvq_decode_static_reset() clears the buffer.
  */
 #define KVQ_STATIC_SCRATCH_BYTES (8u << 20) /* 8 MiB per device */
 int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
@@ -327,6 +334,13 @@ int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const i
                            const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_len,
                            const float *mask, float sm_scale, void *out, int32_t *err_word,
                            void *stream);
+
+/*
+ * kvq_decode_static_reset -- zero the buffer of kvq_decode_attn_static on the
+ * current device (one memset on `stream`).  Needed only after a call that set
+ * KVQ_ERR_TIMEOUT, which can leave merge counters behind.
+ */
+int kvq_decode_static_reset(void *stream);
 
 /* A static, human-readable name for a host status code. */
 const char *kvq_strerror(int status);

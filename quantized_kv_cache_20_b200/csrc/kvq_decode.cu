@@ -7,19 +7,22 @@
 //   j in [0, kv_len), hk = h / G, K = (k - k_zp) * k_scale, V likewise.
 //
 // Design (B200, sm_100a).  Decode is HBM-bound in bytes but, with GQA, heavy in
-// CUDA-core instructions per byte, so the kernel is built to keep the issue
-// slots busy:
+// CUDA-core instructions per byte, so the kernel is built to keep both the
+// memory pipe and the issue slots busy:
 //  - Persistent grid: one CTA per SM.  The work -- units (b, kv head, head
-//    chunk) x tiles of TS slots, with the tile count derived on the device from
-//    *kv_len -- is flattened and cut into equal contiguous ranges, one per CTA,
-//    so every SM streams the same number of bytes whatever B, Hkv and kv_len
-//    are.  A CTA closes a segment whenever its range moves to the next unit.
-//  - One producer warp issues 1-D bulk async copies (TMA) of the K/V code
-//    tiles, scales, zero points, mask and (on a unit's first tile) the q rows
-//    into an NST-stage shared-memory ring (mbarrier tx counts; one arrival per
-//    consumer warp frees a stage).  Every wait is bounded.
-//  - NW consumer warps each take 32 slots of a tile.  A lane owns 16 dims of
-//    L = D/16 slots in turn.
+//    chunk) x chunks of 32 slots, with the chunk count derived on the device
+//    from *kv_len -- is flattened and cut into equal contiguous ranges, one per
+//    CTA, so every SM streams the same number of bytes (to one chunk) whatever
+//    B, Hkv and kv_len are.  A CTA closes a segment whenever its range moves to
+//    the next unit.
+//  - Inside a CTA, chunk i of the range belongs to warp i mod NW.  Every warp
+//    runs its own R-deep ring of chunk buffers: lane 0 issues the 1-D bulk
+//    async copies (TMA) of a chunk's K/V codes, scales, zero points and mask
+//    into a free buffer, completion is counted on that buffer's mbarrier, and
+//    the buffer is refilled with the warp's chunk R ahead as soon as the warp
+//    has consumed it.  No producer warp and no cross-warp hand-off: a slow warp
+//    never holds back another warp's loads.  Every wait is bounded.
+//  - A lane owns 16 dims of L = D/16 slots of its warp's chunk in turn.
 //      q.k: q is rounded once per segment onto a 16-bit fixed-point grid
 //      (n = rne(q * sm_scale * log2e / 2^E), |n| <= 32767, a power-of-two
 //      step per head), so the dot product with the int8 codes is exact integer
@@ -31,15 +34,23 @@
 //      softmax: online, per lane group, in the log2 domain, with the running
 //      maximum only raised when a new score exceeds it by more than 8 (the
 //      accumulators then hold values up to 2^8 times larger, harmless in fp32).
-//      p.v: the V codes become exact floats (c - zp) through a byte permute into
-//      the mantissa of 2^23 and one packed subtract; p*v_scale is broadcast per
-//      slot through shared memory and accumulated with packed fp32 FMA.
+//      p.v: one byte permute turns a V code into the exact subnormal float
+//      (c + 128) * 2^-149; the weights p * v_scale, scaled by 2^96, are
+//      broadcast per slot through shared memory and accumulated with packed
+//      fp32 FMA (the accumulators hold 2^-53 of the sums).  The zero point
+//      and the +128 bias leave as one per-head correction,
+//      sum_j p_j v_scale_j (128 + zp_j), subtracted when the warps merge; the
+//      cancellation costs at most a few bits of fp32 (the sums are < 2^16).
 //  - Segment close: groups merge by shuffles, warps through shared memory, in
 //    a fixed order.  A unit that a CTA covers alone is written directly; a
-//    unit split across CTAs leaves one partial per CTA in the workspace, and a
-//    small merge kernel, launched behind the decode kernel with programmatic
-//    dependent launch, combines them in CTA order.  No atomics, no counters:
-//    results are deterministic and the workspace needs no initialisation.
+//    unit split across CTAs leaves one partial per CTA in the workspace, and
+//    the owner that completes the unit (a per-unit counter in the workspace,
+//    reset to zero by that owner) merges the partials in owner order, so the
+//    result does not depend on which CTA finishes last.
+//  - The decode kernel itself is launched as a programmatic dependent of the
+//    kernel before it (typically the cache write of the new token): its launch
+//    and barrier set-up overlap that kernel's tail, and it reads nothing before
+//    griddepcontrol.wait has seen that kernel complete.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -51,6 +62,11 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p kept without rescaling
+// p.v runs on V codes held as subnormal floats b * 2^-149 (b = code + 128, exact)
+// and weights scaled by 2^96, so the accumulators hold 2^-53 of the true sums.
+constexpr float kWScale = 79228162514264337593543950336.0f;  // 2^96
+constexpr float kOScale = 9007199254740992.0f;                // 2^53
+constexpr int kMaxCtas = 256;  // grid size limit (owner records staged per unit)
 
 struct DecodeArgs {
   const uint16_t *q;
@@ -64,43 +80,45 @@ struct DecodeArgs {
   const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
   int kv_per_batch;
   uint16_t *out;
-  float *ws_ml;       // [C * smax][HC][2]
-  float *ws_o;        // [C * smax][HC][D]
-  int merge_ctas;     // grid of the merge kernel
+  float *ws_ml;       // [C][2][HC][2]: (m, l) of the CTA's first and last unit, when split
+  float *ws_o;        // [C][2][HC][D]
+  int32_t *ws_cnt;    // [U] owners of a split unit that have written their partial
   int32_t *err;
   int64_t S;
-  int B, Hq, Hkv, G, nhc, smax;
+  int B, Hq, Hkv, G, nhc;
   float qscale;  // sm_scale * log2(e)
 };
 
-template <int D_, int HC_, int NW_, int NST_, bool Q4_ = false>
+template <int D_, int HC_, int NW_, int R_, bool Q4_ = false>
 struct Cfg {
-  static constexpr int D = D_, HC = HC_, NW = NW_, NST = NST_;
-  static constexpr bool Q4 = Q4_;          // TQ4 cache: 4-bit codes, two per byte
+  static constexpr int D = D_, HC = HC_, NW = NW_, R = R_;
+  static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte
   static constexpr int CB = Q4 ? D / 2 : D;  // code bytes per slot
-  static constexpr int L = D / 16;     // lanes per slot group (16 dims per lane)
-  static constexpr int NG = 32 / L;    // slot groups per warp
-  static constexpr int TS = 32 * NW;   // slots per tile
-  // one ring stage
+  static constexpr int L = D / 16;           // lanes per slot group (16 dims per lane)
+  static constexpr int NG = 32 / L;          // slot groups per warp
+  static constexpr int CS = 32;              // slots per chunk (one warp step)
+  // one chunk buffer
   static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = TS * CB;
-  static constexpr int KS_OFF = 2 * TS * CB;
-  static constexpr int VS_OFF = KS_OFF + 4 * TS;
-  static constexpr int M_OFF = VS_OFF + 4 * TS;
-  static constexpr int KZ_OFF = M_OFF + 4 * TS;
-  static constexpr int VZ_OFF = KZ_OFF + TS;
-  static constexpr int Q_OFF = VZ_OFF + TS;
-  static constexpr int STAGE = Q_OFF + 2 * HC * D;
-  static_assert(STAGE % 16 == 0, "stage alignment");
-  // after the ring
-  static constexpr int WBUF_OFF = NST * STAGE;                 // [NW][32][4] float
+  static constexpr int V_OFF = CS * CB;
+  static constexpr int KS_OFF = 2 * CS * CB;
+  static constexpr int VS_OFF = KS_OFF + 4 * CS;
+  static constexpr int M_OFF = VS_OFF + 4 * CS;
+  static constexpr int KZ_OFF = M_OFF + 4 * CS;
+  static constexpr int VZ_OFF = KZ_OFF + CS;
+  static constexpr int CHUNK = VZ_OFF + CS;
+  static_assert(CHUNK % 16 == 0, "chunk alignment");
+  // NW rings of R chunk buffers, then the per-warp scratch
+  static constexpr int WBUF_OFF = NW * R * CHUNK;              // [NW][32][4] float
   static constexpr int OSCR_OFF = WBUF_OFF + NW * 32 * 16;     // [NW][HC][D] float
-  static constexpr int MLSCR_OFF = OSCR_OFF + NW * HC * D * 4; // [NW][HC][2] float
-  static constexpr int BAR_OFF = MLSCR_OFF + NW * HC * 8;
-  static constexpr int SH_OFF = BAR_OFF + 2 * NST * 8;
-  static constexpr int SMEM = SH_OFF + 16;
+  static constexpr int MLSCR_OFF = OSCR_OFF + NW * HC * D * 4; // [NW][HC][4] float: m, l, corr
+  static constexpr int BAR_OFF = MLSCR_OFF + NW * HC * 16;     // [NW][R] mbarrier
+  static constexpr int SH_OFF = BAR_OFF + NW * R * 8;           // 8 ints
+  static constexpr int Q_OFF = (SH_OFF + 32 + 15) / 16 * 16;     // [2][HC] q rows: D/4 high, D/4 low words
+  static constexpr int QMETA_OFF = Q_OFF + 2 * HC * 2 * D;       // [2][HC] (sum n, 2^E)
+  static constexpr int RECS_OFF = QMETA_OFF + 2 * HC * 8;        // [2][kMaxCtas] owner records
+  static constexpr int SMEM = RECS_OFF + 2 * kMaxCtas * 4;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static constexpr int THREADS = (NW + 1) * 32;
+  static constexpr int THREADS = NW * 32;
 };
 
 KVQ_DEVINL int dp4a_ss(uint32_t a, uint32_t b, int c) {
@@ -134,7 +152,13 @@ KVQ_DEVINL float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-KVQ_DEVINL void consumer_sync(int nthreads) { asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); }
+// Add 1 to a merge counter, releasing this CTA's partial (written before the
+// barrier that precedes the call) and acquiring the other owners'.
+KVQ_DEVINL int count_acq_rel(int32_t *p) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
 
 // Work split: CTA c owns flattened tiles [c*W/C, (c+1)*W/C).
 KVQ_DEVINL int64_t range_start(int64_t c, int64_t W, int64_t C) { return c * W / C; }
@@ -195,32 +219,30 @@ KVQ_DEVINL int max_kv_len(const DecodeArgs &a, volatile int32_t *red, bool repor
 // is a separate instantiation so it carries no per-unit state.
 template <class C, bool VARLEN>
 __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs a) {
-  constexpr int D = C::D, HC = C::HC, NW = C::NW, NST = C::NST, L = C::L, NG = C::NG, TS = C::TS;
+  constexpr int D = C::D, HC = C::HC, NW = C::NW, R = C::R, L = C::L, NG = C::NG, CS = C::CS, CB = C::CB;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-  uint64_t *empty = full + NST;
-  volatile int32_t *sh = reinterpret_cast<volatile int32_t *>(smem + C::SH_OFF);  // kv, abort, last
+  volatile int32_t *sh = reinterpret_cast<volatile int32_t *>(smem + C::SH_OFF);  // scratch int, abort
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NW);
-    }
+    for (int i = 0; i < NW * R; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
     sh[1] = 0;
-    sh[2] = 0;
+    sh[2] = 0;  // length of the merge list
   }
+  // everything read below may have been written by the kernel launched before this one
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
-  // Every unit is cut into ceil(max kv_len / TS) tiles; with per-row lengths a
-  // row's tiles past its own kv_len carry no bytes and no work.
+  // Every unit is cut into ceil(max kv_len / 32) chunks; with per-row lengths a
+  // row's chunks past its own kv_len carry no bytes and no work.
   const int kv = max_kv_len(a, sh, blockIdx.x == 0);
   asm volatile("griddepcontrol.launch_dependents;");
-  const int ntiles = (kv + TS - 1) / TS;
+  const int nch = (kv + CS - 1) / CS;
   const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
   const int64_t CT = gridDim.x, cta = blockIdx.x;
 
-  if (ntiles == 0) {  // nothing to attend to: every row is zero
+  if (nch == 0) {  // nothing to attend to: every row is zero
     for (int64_t u = cta; u < U; u += CT) {
       const int hc = static_cast<int>(u % a.nhc);
       const int64_t bhk = u / a.nhc;
@@ -232,97 +254,144 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     }
     return;
   }
-  const int64_t W = U * ntiles;
-  const int64_t t_begin = range_start(cta, W, CT), t_end = range_start(cta + 1, W, CT);
+  // chunk indices fit in 32 bits (the host checks U * ceil(S / 32) < 2^31)
+  const int W = static_cast<int>(U * nch);
+  const int c_begin = static_cast<int>(range_start(cta, W, CT)), c_end = static_cast<int>(range_start(cta + 1, W, CT));
+  if (c_begin >= c_end) return;  // more CTAs than chunks
 
-  // ------------------------------------------------------------------ producer
-  if (warp == NW) {
-    if (lane == 0) {
+  // ---- this warp's chunks: c_begin + warp + k * NW for k in [0, nk), chunk k in buffer k % R
+  const int nk = c_begin + warp < c_end ? (c_end - 1 - c_begin - warp) / NW + 1 : 0;
+  // lane 0 only: start the copies of the warp's chunk k (flattened index idx)
+  auto issue = [&](int idx, int k) {
+    const int uu = idx / nch;
+    const int s0 = (idx - uu * nch) * CS;
+    const int64_t bhk = uu / a.nhc;  // = b * Hkv + hk
+    const int kvu = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
+    const int n = max(0, min(CS, kvu - s0));
+    const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
+    uint8_t *buf = smem + (warp * R + k % R) * C::CHUNK;
+    uint64_t *bar = full + warp * R + k % R;
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n16) * (2 * CB + 10) + (a.mask ? 4u * n16 : 0u));
+    if (n16 > 0) {  // 0 bytes: the expect_tx above is a plain arrival
       const uint64_t pol = policy_evict_first();
-      int64_t issued = 0;
-      int64_t u = t_begin / ntiles;
-      int t = static_cast<int>(t_begin - u * ntiles);
-      int st = 0;
-      uint32_t ephase = 0;  // parity of the empty-barrier phase to wait for at stage st
-      int64_t kv_u_of = -1;
-      int kv_u = kv;
-      for (int64_t idx = t_begin; idx < t_end; ++idx) {
-        const int64_t i = idx - t_begin;
-        if (i >= NST && !wait_or_abort(&empty[st], ephase, sh + 1)) {
-          report(a.err, KVQ_ERR_TIMEOUT);
-          sh[1] = 1;
-          break;
-        }
-        const int hc = static_cast<int>(u % a.nhc);
-        const int64_t bhk = u / a.nhc;  // = b * Hkv + hk
-        if (u != kv_u_of) {
-          kv_u_of = u;
-          kv_u = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
-        }
-        const int s0 = t * TS;
-        const int n = max(0, min(TS, kv_u - s0));
-        const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
-        const bool first = (t == 0) || (idx == t_begin);
-        uint8_t *stage = smem + st * C::STAGE;
-        const uint32_t bytes = static_cast<uint32_t>(n16) * (2 * C::CB + 10) + (a.mask ? 4u * n16 : 0u) +
-                               (first ? 2u * HC * D : 0u);
-        mbar_arrive_expect_tx(&full[st], bytes);  // 0 bytes: a plain arrival
-        const int64_t row = bhk * a.S + s0;
-        if (n16 > 0) {
-          bulk_g2s_hint(stage + C::K_OFF, a.k + row * C::CB, n16 * C::CB, &full[st], pol);
-          bulk_g2s_hint(stage + C::V_OFF, a.v + row * C::CB, n16 * C::CB, &full[st], pol);
-          bulk_g2s(stage + C::KS_OFF, a.ks + row, n16 * 4, &full[st]);
-          bulk_g2s(stage + C::VS_OFF, a.vs + row, n16 * 4, &full[st]);
-          bulk_g2s(stage + C::KZ_OFF, a.kz + row, n16, &full[st]);
-          bulk_g2s(stage + C::VZ_OFF, a.vz + row, n16, &full[st]);
-          if (a.mask) bulk_g2s(stage + C::M_OFF, a.mask + s0, n16 * 4, &full[st]);
-        }
-        if (first) {
-          const int64_t hk = bhk % a.Hkv, b = bhk / a.Hkv;
-          const int64_t q0 = (b * a.Hq + hk * a.G + static_cast<int64_t>(hc) * HC) * D;
-          bulk_g2s(stage + C::Q_OFF, a.q + q0, 2 * HC * D, &full[st]);
-        }
-        issued = i + 1;
-        if (++t == ntiles) {
-          t = 0;
-          ++u;
-        }
-        if (++st == NST) {  // entering round r = (i+1)/NST waits for empty phase (r-1) & 1
-          st = 0;
-          if (i + 1 >= 2 * NST) ephase ^= 1u;
-        }
-      }
-      // the last copy issued into each stage must land before the CTA exits
-      for (int64_t i = issued > NST ? issued - NST : 0; i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % NST], static_cast<uint32_t>(i / NST) & 1u)) report(a.err, KVQ_ERR_TIMEOUT);
+      const int64_t row = bhk * a.S + s0;
+      bulk_g2s_hint(buf + C::K_OFF, a.k + row * CB, n16 * CB, bar, pol);
+      bulk_g2s_hint(buf + C::V_OFF, a.v + row * CB, n16 * CB, bar, pol);
+      bulk_g2s(buf + C::KS_OFF, a.ks + row, n16 * 4, bar);
+      bulk_g2s(buf + C::VS_OFF, a.vs + row, n16 * 4, bar);
+      bulk_g2s(buf + C::KZ_OFF, a.kz + row, n16, bar);
+      bulk_g2s(buf + C::VZ_OFF, a.vz + row, n16, bar);
+      if (a.mask) bulk_g2s(buf + C::M_OFF, a.mask + s0, n16 * 4, bar);
     }
-    return;
-  }
+  };
+  if (lane == 0)
+    for (int k = 0; k < min(R, nk); ++k) issue(c_begin + warp + k * NW, k);
 
-  // ------------------------------------------------------------------ consumers
+  const int u_first = c_begin / nch, u_last = (c_end - 1) / nch;  // the CTA's units
   const int g = lane / L, sub = lane % L;
-  const int own = g + NG * sub;  // this lane's slot within the warp's 32 after the reduce-scatter
+  const int own = g + NG * sub;  // this lane's slot within the chunk after the reduce-scatter
   float *wbuf = reinterpret_cast<float *>(smem + C::WBUF_OFF) + warp * 32 * 4;
 
   uint32_t qhi[HC][4], qlo[HC][4];
   int nsum[HC];
   float escale[HC];
-  float m[HC], lsum[HC];
+  float m[HC], lsum[HC], corr[HC];  // corr: sum of p * v_scale * (128 + v_zp), see kWScale
   float2 o2[HC][8];
-  int64_t cur_u = -1;
-  int seg = -1;
-  int kv_u = kv;  // kv_len of the current unit's batch row (VARLEN), else kv
 
-  auto close_segment = [&](int64_t u, int sg) {
-    // (1) denominators over the lane group, then merge the NG groups of the warp
+  // warps 0 .. HC-1: head `warp` of unit u onto the fixed-point grid, into q slot `slot`
+  //   n = rne(q * sm_scale * log2e / 2^E), |n| <= 32767, E per head; stored as the
+  //   high and low bytes of n, four dims per word in the order the dp4a lanes read
+  auto convert_q = [&](int u, int slot) {
+    if (warp >= HC) return;
+    const int h = warp;
+    const int hc = u % a.nhc;
+    const int64_t bhk = u / a.nhc;
+    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    const uint16_t *qg = a.q + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC + h) * D;
+    constexpr int NWD = D / 4;                 // words of one head
+    constexpr int PER = (NWD + 31) / 32;       // words per lane
+    float x[PER][4];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int wd = lane + 32 * i, sb = wd >> 2, kk = wd & 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // byte j of word kk of lane sb pairs with the code of dim 16 sb + (4 kk + j); unpacked
+        // TQ4 nibbles come as (0,2,4,6), (1,3,5,7), (8,10,12,14), (9,11,13,15)
+        const int dim = sb * 16 + (C::Q4 ? (kk >> 1) * 8 + (kk & 1) + 2 * j : 4 * kk + j);
+        x[i][j] = wd < NWD ? __uint_as_float(static_cast<uint32_t>(qg[dim]) << 16) * a.qscale : 0.0f;
+        amax = fmaxf(amax, fabsf(x[i][j]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // step 2^E with amax / 2^E < 2^15: E = floor(log2 amax) + 1 - 15
+    int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1 - 15;
+    E = E < -126 ? -126 : E;
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);  // 2^-E (E in [-126, 113])
+    uint32_t *qs = reinterpret_cast<uint32_t *>(smem + C::Q_OFF) + (slot * HC + h) * 2 * NWD;
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int wd = lane + 32 * i;
+      uint32_t hw = 0, lw = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int n = __float2int_rn(x[i][j] * inv);
+        n = n > 32767 ? 32767 : (n < -32767 ? -32767 : n);
+        s += n;
+        hw |= (static_cast<uint32_t>(n >> 8) & 0xFFu) << (8 * j);
+        lw |= (static_cast<uint32_t>(n) & 0xFFu) << (8 * j);
+      }
+      if (wd < NWD) {
+        qs[wd] = hw;
+        qs[NWD + wd] = lw;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) {
+      int32_t *meta = reinterpret_cast<int32_t *>(smem + C::QMETA_OFF) + (slot * HC + h) * 2;
+      meta[0] = s;
+      meta[1] = static_cast<int32_t>(static_cast<uint32_t>(127 + E) << 23);  // 2^E as float bits
+    }
+  };
+  // every lane: its slices of q slot `slot`, fresh softmax state
+  auto load_q = [&](int slot) {
+#pragma unroll
+    for (int h = 0; h < HC; ++h) {
+      const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::Q_OFF) + (slot * HC + h) * (D / 2);
+      const uint4 hw = *reinterpret_cast<const uint4 *>(qs + sub * 4);
+      const uint4 lw = *reinterpret_cast<const uint4 *>(qs + D / 4 + sub * 4);
+      qhi[h][0] = hw.x; qhi[h][1] = hw.y; qhi[h][2] = hw.z; qhi[h][3] = hw.w;
+      qlo[h][0] = lw.x; qlo[h][1] = lw.y; qlo[h][2] = lw.z; qlo[h][3] = lw.w;
+      const int2 meta = *reinterpret_cast<const int2 *>(smem + C::QMETA_OFF + (slot * HC + h) * 8);
+      nsum[h] = meta.x;
+      escale[h] = __int_as_float(meta.y);
+      m[h] = -INFINITY;
+      lsum[h] = 0.0f;
+      corr[h] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o2[h][j] = make_float2(0.0f, 0.0f);
+    }
+  };
+
+  // this warp's state: merge the NG lane groups (shuffles), then lane group 0
+  // writes (O, m, l, corr) for the warp: O at o_dst[h * D + d], the rest at ml_dst[h * 4]
+  auto publish = [&](float *o_dst, float *ml_dst) {
 #pragma unroll
     for (int h = 0; h < HC; ++h) {
 #pragma unroll
-      for (int o = L / 2; o >= 1; o >>= 1) lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
+      for (int o = L / 2; o >= 1; o >>= 1) {
+        lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
+        corr[h] += __shfl_xor_sync(0xffffffffu, corr[h], o);
+      }
 #pragma unroll
       for (int o = L; o < 32; o <<= 1) {
         const float mo = __shfl_xor_sync(0xffffffffu, m[h], o);
         const float lo = __shfl_xor_sync(0xffffffffu, lsum[h], o);
+        const float co = __shfl_xor_sync(0xffffffffu, corr[h], o);
         const float M = fmaxf(m[h], mo);
         const float fs = m[h] == -INFINITY ? 0.0f : ex2(m[h] - M);
         const float fo = mo == -INFINITY ? 0.0f : ex2(mo - M);
@@ -333,348 +402,343 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
           o2[h][k] = __ffma2_rn(o2[h][k], make_float2(fs, fs), __fmul2_rn(oo, make_float2(fo, fo)));
         }
         lsum[h] = lsum[h] * fs + lo * fo;
+        corr[h] = corr[h] * fs + co * fo;
         m[h] = M;
       }
     }
-    // (2) group 0 of each warp publishes the warp's state
-    float *oscr = reinterpret_cast<float *>(smem + C::OSCR_OFF);
-    float *mlscr = reinterpret_cast<float *>(smem + C::MLSCR_OFF);
     if (g == 0) {
 #pragma unroll
       for (int h = 0; h < HC; ++h) {
-        float4 *dst = reinterpret_cast<float4 *>(oscr + (warp * HC + h) * D + sub * 16);
+        float4 *dst = reinterpret_cast<float4 *>(o_dst + h * D + sub * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           dst[k] = make_float4(o2[h][2 * k].x, o2[h][2 * k].y, o2[h][2 * k + 1].x, o2[h][2 * k + 1].y);
-        if (sub == 0) {
-          mlscr[(warp * HC + h) * 2] = m[h];
-          mlscr[(warp * HC + h) * 2 + 1] = lsum[h];
-        }
+        if (sub == 0) *reinterpret_cast<float4 *>(ml_dst + h * 4) = make_float4(m[h], lsum[h], corr[h], 0.0f);
       }
     }
-    consumer_sync(NW * 32);
-    // (3) merge the warps in order; write the output or this CTA's partial
-    const int64_t ntl = ntiles;
-    const int64_t c_first = cta_of(u * ntl, W, CT), c_last = cta_of(u * ntl + ntl - 1, W, CT);
-    const bool alone = c_first == c_last;
-    const int hc = static_cast<int>(u % a.nhc);
+  };
+
+  // all threads: combine the NW warp states of unit u (warp w at o_base + w * stride, its
+  // (m, l, corr) at ml_base + w * stride) in warp order; write the rows, or this CTA's
+  // partial when other CTAs share the unit
+  auto combine = [&](int u, const float *o_base, int o_stride, const float *ml_base, int ml_stride) {
+    const int64_t CTn = gridDim.x;
+    const bool alone = cta_of(static_cast<int64_t>(u) * nch, W, CTn) ==
+                       cta_of(static_cast<int64_t>(u) * nch + nch - 1, W, CTn);
+    const int hc = u % a.nhc;
     const int64_t bhk = u / a.nhc;
     const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
-    const int64_t rec = cta * a.smax + sg;
-    for (int e = tid; e < HC * D; e += NW * 32) {
+    uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
+    const int64_t rec = 2 * static_cast<int64_t>(blockIdx.x) + (u == u_first ? 0 : 1);
+    for (int e = tid; e < HC * D; e += C::THREADS) {
       const int h = e / D, d = e - h * D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, mlscr[(w * HC + h) * 2]);
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, ml_base[w * ml_stride + h * 4]);
       float Lt = 0.0f, O = 0.0f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-          const float mw = mlscr[(w * HC + h) * 2];
-          const float f = mw == -INFINITY ? 0.0f : ex2(mw - M);
-          Lt = fmaf(f, mlscr[(w * HC + h) * 2 + 1], Lt);
-          O = fmaf(f, oscr[(w * HC + h) * D + d], O);
+          const float4 mlc = *reinterpret_cast<const float4 *>(ml_base + w * ml_stride + h * 4);
+          const float f = mlc.x == -INFINITY ? 0.0f : ex2(mlc.x - M);
+          Lt = fmaf(f, mlc.y, Lt);
+          O = fmaf(f, fmaf(o_base[w * o_stride + h * D + d], kOScale, -mlc.z), O);
         }
       }
       if (alone) {
-        const int hq = hk * a.G + hc * HC + h;
         const float r = Lt > 0.0f ? O / Lt : 0.0f;
-        a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+        orow[e] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
       } else {
         a.ws_o[(rec * HC + h) * D + d] = O;
-        if (d == 0) {
-          a.ws_ml[(rec * HC + h) * 2] = M;
-          a.ws_ml[(rec * HC + h) * 2 + 1] = Lt;
-        }
+        if (d == 0) *reinterpret_cast<float2 *>(a.ws_ml + (rec * HC + h) * 2) = make_float2(M, Lt);
       }
     }
-    consumer_sync(NW * 32);  // scratch free for the next segment
   };
 
-  int64_t u = t_begin / ntiles;
-  int t = static_cast<int>(t_begin - u * ntiles);
-  int st = 0;
-  uint32_t fphase = 0;
-  for (int64_t idx = t_begin; idx < t_end; ++idx) {
-    const bool ok = wait_or_abort(&full[st], fphase, sh + 1);
-    if (!ok && lane == 0) {
-      report(a.err, KVQ_ERR_TIMEOUT);
-      sh[1] = 1;
+  // owner records of the first (slot 0) and last (slot 1) unit when split:
+  // owner o's partial is record 2 c + (u is c's first unit ? 0 : 1), c = its CTA
+  int32_t *recs_s = reinterpret_cast<int32_t *>(smem + C::RECS_OFF);
+  auto owners_of = [&](int u, int64_t &cf) {
+    const int64_t CTn = gridDim.x;
+    cf = cta_of(static_cast<int64_t>(u) * nch, W, CTn);
+    const int64_t cl = cta_of(static_cast<int64_t>(u) * nch + nch - 1, W, CTn);
+    return cf == cl ? 1 : (W >= CTn ? static_cast<int>(cl - cf + 1) : nch);  // W < CTn: one chunk per CTA
+  };
+  auto stage_owners = [&](int u, int slot) {
+    int64_t cf;
+    const int owners = owners_of(u, cf);
+    const int64_t CTn = gridDim.x;
+    for (int o = tid; o < owners && owners > 1; o += C::THREADS) {
+      const int64_t c = W >= CTn ? cf + o : cta_of(static_cast<int64_t>(u) * nch + o, W, CTn);
+      recs_s[slot * kMaxCtas + o] = static_cast<int32_t>(2 * c + (u == range_start(c, W, CTn) / nch ? 0 : 1));
     }
-    const uint8_t *stage = smem + st * C::STAGE;
-    if (u != cur_u) {
-      if (cur_u >= 0) close_segment(cur_u, seg);
-      cur_u = u;
-      ++seg;
-      if constexpr (VARLEN) kv_u = row_kv(a, static_cast<int>(u / a.nhc / a.Hkv));
-      // new unit: q (from this stage) onto the fixed-point grid, fresh softmax state
-      const uint16_t *qs = reinterpret_cast<const uint16_t *>(stage + C::Q_OFF);
-#pragma unroll
-      for (int h = 0; h < HC; ++h) {
-        const uint4 c0 = *reinterpret_cast<const uint4 *>(qs + h * D + sub * 16);
-        const uint4 c1 = *reinterpret_cast<const uint4 *>(qs + h * D + sub * 16 + 8);
-        const uint32_t wq[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        float x[16];
-        float amax = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          x[2 * k] = bf16lo(wq[k]) * a.qscale;
-          x[2 * k + 1] = bf16hi(wq[k]) * a.qscale;
-          amax = fmaxf(amax, fmaxf(fabsf(x[2 * k]), fabsf(x[2 * k + 1])));
-        }
-#pragma unroll
-        for (int o = L / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        // step 2^E with amax / 2^E < 2^15: E = floor(log2 amax) + 1 - 15
-        int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1 - 15;
-        E = E < -126 ? -126 : E;
-        const float inv = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);  // 2^-E (E in [-126, 113])
-        escale[h] = __uint_as_float(static_cast<uint32_t>(127 + E) << 23);       // 2^E
-        int s = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t hw = 0, lw = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            // byte j of word k pairs with the code of dim 4k + j; unpacked TQ4
-            // nibbles come as (0,2,4,6), (1,3,5,7), (8,10,12,14), (9,11,13,15)
-            const int dim = C::Q4 ? (k >> 1) * 8 + (k & 1) + 2 * j : 4 * k + j;
-            int n = __float2int_rn(x[dim] * inv);
-            n = n > 32767 ? 32767 : (n < -32767 ? -32767 : n);
-            s += n;
-            hw |= (static_cast<uint32_t>(n >> 8) & 0xFFu) << (8 * j);
-            lw |= (static_cast<uint32_t>(n) & 0xFFu) << (8 * j);
-          }
-          qhi[h][k] = hw;
-          qlo[h][k] = lw;
-        }
-#pragma unroll
-        for (int o = L / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        nsum[h] = s;
-        m[h] = -INFINITY;
-        lsum[h] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) o2[h][k] = make_float2(0.0f, 0.0f);
-      }
-    }
+    return owners;
+  };
 
-    const int s0 = t * TS;
-    const int wbase = warp * 32;
-    if (ok && s0 + wbase < kv_u) {
-      // ---- q . k on dp4a for the L slots of this lane group (slot = wbase + g + NG*jj)
-      int part[L][HC];
-#pragma unroll
-      for (int jj = 0; jj < L; ++jj) {
-        const int sl = wbase + g + NG * jj;
-        if constexpr (C::Q4) {
-          const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::K_OFF + sl * C::CB + sub * 8);
-          uint4 c;
-          unpack_nibbles(cw.x, c.x, c.y);
-          unpack_nibbles(cw.y, c.z, c.w);
-#pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            int acc = dp4a_su(qhi[h][0], c.x, 0);
-            acc = dp4a_su(qhi[h][1], c.y, acc);
-            acc = dp4a_su(qhi[h][2], c.z, acc);
-            acc = dp4a_su(qhi[h][3], c.w, acc);
-            acc *= 256;
-            acc = dp4a_uu(qlo[h][0], c.x, acc);
-            acc = dp4a_uu(qlo[h][1], c.y, acc);
-            acc = dp4a_uu(qlo[h][2], c.z, acc);
-            acc = dp4a_uu(qlo[h][3], c.w, acc);
-            part[jj][h] = acc;
-          }
-        } else {
-          const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
-#pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            int acc = dp4a_ss(qhi[h][0], c.x, 0);
-            acc = dp4a_ss(qhi[h][1], c.y, acc);
-            acc = dp4a_ss(qhi[h][2], c.z, acc);
-            acc = dp4a_ss(qhi[h][3], c.w, acc);
-            acc *= 256;
-            acc = dp4a_us(qlo[h][0], c.x, acc);
-            acc = dp4a_us(qlo[h][1], c.y, acc);
-            acc = dp4a_us(qlo[h][2], c.z, acc);
-            acc = dp4a_us(qlo[h][3], c.w, acc);
-            part[jj][h] = acc;
-          }
-        }
-      }
-      // ---- butterfly reduce-scatter: lane `sub` ends with slot jj = sub
-#pragma unroll
-      for (int o = L / 2; o >= 1; o >>= 1) {
-        const bool upper = (sub & o) != 0;
-#pragma unroll
-        for (int j = 0; j < o; ++j)
-#pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            const int keep = upper ? part[j + o][h] : part[j][h];
-            const int send = upper ? part[j][h] : part[j + o][h];
-            part[j][h] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-          }
-      }
-      // ---- scores (log2 domain) for this lane's slot
-      const int sl_own = wbase + own;
-      const bool valid = s0 + sl_own < kv_u;
-      const int kzp = static_cast<int8_t>(stage[C::KZ_OFF + sl_own]);
-      const float ksc = reinterpret_cast<const float *>(stage + C::KS_OFF)[sl_own];
-      const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[sl_own];
-      const float madd = a.mask ? reinterpret_cast<const float *>(stage + C::M_OFF)[sl_own] * kLog2e : 0.0f;
-      float sc[HC], mt[HC];
-      bool need = false;
-#pragma unroll
-      for (int h = 0; h < HC; ++h) {
-        // exact: |sum n (c - zp)| < 2^31 for D <= 256 (computed modulo 2^32)
-        const int dz = static_cast<int>(static_cast<uint32_t>(part[0][h]) -
-                                        static_cast<uint32_t>(kzp) * static_cast<uint32_t>(nsum[h]));
-        sc[h] = valid ? fmaf(static_cast<float>(dz), escale[h] * ksc, madd) : -INFINITY;
-        mt[h] = sc[h];
-#pragma unroll
-        for (int o = L / 2; o >= 1; o >>= 1) mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
-        need |= mt[h] > m[h] + kRescaleThreshold;
-      }
-      if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int h = 0; h < HC; ++h) {
-          const float mnew = fmaxf(m[h], mt[h]);
-          if (mnew > m[h]) {
-            const float alpha = m[h] == -INFINITY ? 0.0f : ex2(m[h] - mnew);
-            lsum[h] *= alpha;
-            const float2 al2 = make_float2(alpha, alpha);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) o2[h][k] = __fmul2_rn(o2[h][k], al2);
-            m[h] = mnew;
-          }
-        }
-      }
-      float wv[4];
-#pragma unroll
-      for (int h = 0; h < HC; ++h) {
-        const float p = sc[h] == -INFINITY ? 0.0f : ex2(sc[h] - m[h]);
-        lsum[h] += p;
-        wv[h] = p > 0.0f ? p * vsc : 0.0f;
-      }
-#pragma unroll
-      for (int h = HC; h < 4; ++h) wv[h] = 0.0f;
-      *reinterpret_cast<float4 *>(wbuf + own * 4) = make_float4(wv[0], wv[1], wv[2], wv[3]);
-      __syncwarp();
-      // ---- p . v over the same L slots
-#pragma unroll
-      for (int jj = 0; jj < L; ++jj) {
-        const int sl = g + NG * jj;
-        const float4 w4 = *reinterpret_cast<const float4 *>(wbuf + sl * 4);
-        const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
-        const int zp = static_cast<int8_t>(stage[C::VZ_OFF + wbase + sl]);
-        const float mz = neg_magic_zp(zp);
-        const float2 mz2 = make_float2(mz, mz);
-        uint4 c;
-        if constexpr (C::Q4) {  // nibbles back to element order: bytes (0,1,2,3), (4,5,6,7), ...
-          const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::V_OFF + (wbase + sl) * C::CB + sub * 8);
-          uint32_t e0, o0, e1, o1;
-          unpack_nibbles(cw.x, e0, o0);
-          unpack_nibbles(cw.y, e1, o1);
-          c = make_uint4(__byte_perm(e0, o0, 0x5140), __byte_perm(e0, o0, 0x7362), __byte_perm(e1, o1, 0x5140),
-                         __byte_perm(e1, o1, 0x7362));
-        } else {
-          c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + (wbase + sl) * D + sub * 16);
-        }
-        float2 vv2[8];
-        codes4_to_f2(c.x, mz2, vv2[0], vv2[1]);
-        codes4_to_f2(c.y, mz2, vv2[2], vv2[3]);
-        codes4_to_f2(c.z, mz2, vv2[4], vv2[5]);
-        codes4_to_f2(c.w, mz2, vv2[6], vv2[7]);
-#pragma unroll
-        for (int h = 0; h < HC; ++h) {
-          const float2 w2 = make_float2(wj[h], wj[h]);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) o2[h][k] = __ffma2_rn(w2, vv2[k], o2[h][k]);
-        }
-      }
-      __syncwarp();
-    }
-    if (lane == 0) mbar_arrive(&empty[st]);
-    if (++t == ntiles) {
-      t = 0;
-      ++u;
-    }
-    if (++st == NST) {
-      st = 0;
-      fphase ^= 1u;
-    }
-  }
-  if (cur_u >= 0) close_segment(cur_u, seg);
-}
-
-// ----------------------------------------------------------------------------
-// Merge of split units: one CTA per unit.  Launched right after the decode
-// kernel (programmatic dependent launch: it may start while the decode grid
-// drains and waits for its completion, so all partials are visible); a unit
-// whose tiles one CTA owned alone was written by the decode kernel already.
-// Partials are combined in owner (CTA) order.
-// ----------------------------------------------------------------------------
-template <class C>
-__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int decode_ctas) {
-  constexpr int D = C::D, HC = C::HC, TS = C::TS;
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ int32_t recs[1024];
-  __shared__ float mls[1024 * 2];
-  __shared__ int32_t red;
-  const int kv = max_kv_len(a, &red, false);
-  const int64_t ntl = (kv + TS - 1) / TS;
-  if (ntl == 0) return;
-  const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
-  const int64_t W = U * ntl, CT = decode_ctas;
-  for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
-    const int64_t last_tile = u * ntl + ntl - 1;
-    const int64_t c_first = cta_of(u * ntl, W, CT);
-    const int64_t c_last = cta_of(last_tile, W, CT);
-    if (c_first == c_last) continue;
-    __syncthreads();  // recs / mls reuse across units
-    int owners;
-    if (W >= CT) {  // no CTA has an empty range: the owners are c_first..c_last
-      owners = static_cast<int>(c_last - c_first + 1);
-      for (int i = threadIdx.x; i < owners; i += blockDim.x) {
-        const int64_t c = c_first + i;
-        recs[i] = static_cast<int32_t>(c * a.smax + (u - range_start(c, W, CT) / ntl));
-      }
-    } else {
-      owners = 0;
-      for (int64_t c = c_first; c >= 0; c = next_owner(c, last_tile, W, CT)) {
-        if (threadIdx.x == 0) recs[owners] = static_cast<int32_t>(c * a.smax + (u - range_start(c, W, CT) / ntl));
-        ++owners;
-      }
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < owners * HC; i += blockDim.x) {
-      const int o = i / HC, h = i - o * HC;
-      const int64_t r = static_cast<int64_t>(recs[o]) * HC + h;
-      mls[i * 2] = a.ws_ml[r * 2];
-      mls[i * 2 + 1] = a.ws_ml[r * 2 + 1];
-    }
-    __syncthreads();
-    const int hc = static_cast<int>(u % a.nhc);
+  // all threads: merge the partials of split unit u (records in slot `slot`) in owner order
+  auto merge_unit = [&](int u, int slot, int owners) {
+    const int32_t *recs = recs_s + slot * kMaxCtas;
+    const int hc = u % a.nhc;
     const int64_t bhk = u / a.nhc;
     const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
-    for (int e = threadIdx.x; e < HC * D; e += blockDim.x) {
+    uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
+    for (int e = tid; e < HC * D; e += C::THREADS) {
       const int h = e / D, d = e - h * D;
-      float M = -INFINITY;
-      for (int o = 0; o < owners; ++o) M = fmaxf(M, mls[(o * HC + h) * 2]);
-      float Lt = 0.0f, O = 0.0f;
-      if (M != -INFINITY) {
-#pragma unroll 4
-        for (int o = 0; o < owners; ++o) {
-          const float oc = a.ws_o[(static_cast<int64_t>(recs[o]) * HC + h) * D + d];
-          const float mc = mls[(o * HC + h) * 2];
-          const float f = mc == -INFINITY ? 0.0f : ex2(mc - M);
-          Lt = fmaf(f, mls[(o * HC + h) * 2 + 1], Lt);
-          O = fmaf(f, oc, O);
+      float M = -INFINITY, Lt = 0.0f, O = 0.0f;
+      for (int o0 = 0; o0 < owners; o0 += 8) {  // eight owners' loads in flight at once
+        float2 ml[8];
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (o0 + t < owners) {
+            const int64_t r = static_cast<int64_t>(recs[o0 + t]) * HC + h;
+            ml[t] = __ldcg(reinterpret_cast<const float2 *>(a.ws_ml + r * 2));
+            v[t] = __ldcg(a.ws_o + r * D + d);
+          } else {
+            ml[t] = make_float2(-INFINITY, 0.0f);
+            v[t] = 0.0f;
+          }
+        }
+        float Mn = M;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) Mn = fmaxf(Mn, ml[t].x);
+        if (Mn == -INFINITY) continue;
+        const float fo = M == -INFINITY ? 0.0f : ex2(M - Mn);
+        Lt *= fo;
+        O *= fo;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float f = ml[t].x == -INFINITY ? 0.0f : ex2(ml[t].x - Mn);
+          Lt = fmaf(f, ml[t].y, Lt);
+          O = fmaf(f, v[t], O);
+        }
+        M = Mn;
+      }
+      const float r = Lt > 0.0f ? O / Lt : 0.0f;
+      orow[e] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    }
+  };
+
+  // ---- the CTA's units in order.  With at most two (a unit spans more chunks than
+  // a CTA range) no warp waits for another until the end: the first unit's warp
+  // states go to the scratch, the last unit's to each warp's own (then idle) ring.
+  // With more, every unit closes with two CTA barriers.
+  const bool deferred = u_last - u_first <= 1;
+  float *oscr = reinterpret_cast<float *>(smem + C::OSCR_OFF);
+  float *mlscr = reinterpret_cast<float *>(smem + C::MLSCR_OFF);
+  constexpr int kRingStride = R * C::CHUNK / 4;  // floats from one warp's ring to the next
+  const int own0 = stage_owners(u_first, 0);
+  const int own1 = u_last != u_first ? stage_owners(u_last, 1) : 1;
+  if (deferred) {
+    convert_q(u_first, 0);
+    if (u_last != u_first) convert_q(u_last, 1);
+  }
+  __syncthreads();  // q slots and owner records written
+  int k = 0;
+  for (int u = u_first; u <= u_last; ++u) {
+    if (!deferred) {
+      convert_q(u, 0);
+      __syncthreads();  // q slot written; the previous unit's combine has read the scratch
+    }
+    load_q(deferred && u != u_first ? 1 : 0);
+    const int kv_u = VARLEN ? row_kv(a, static_cast<int>(u / a.nhc / a.Hkv)) : kv;
+    const int seg_end = min(c_end, (u + 1) * nch);
+    for (; k < nk; ++k) {
+      const int idx = c_begin + warp + k * NW;
+      if (idx >= seg_end) break;
+      const uint8_t *stage = smem + (warp * R + k % R) * C::CHUNK;
+      const bool ok = wait_or_abort(full + warp * R + k % R, static_cast<uint32_t>(k / R) & 1u, sh + 1);
+      if (!ok && lane == 0) {
+        report(a.err, KVQ_ERR_TIMEOUT);
+        sh[1] = 1;
+      }
+      const int s0 = (idx - u * nch) * CS;
+      if (ok && s0 < kv_u) {
+        // ---- q . k on dp4a for the L slots of this lane group (slot = g + NG*jj)
+        int part[L][HC];
+#pragma unroll
+        for (int jj = 0; jj < L; ++jj) {
+          const int sl = g + NG * jj;
+          if constexpr (C::Q4) {
+            const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::K_OFF + sl * CB + sub * 8);
+            uint4 c;
+            unpack_nibbles(cw.x, c.x, c.y);
+            unpack_nibbles(cw.y, c.z, c.w);
+#pragma unroll
+            for (int h = 0; h < HC; ++h) {
+              int acc = dp4a_su(qhi[h][0], c.x, 0);
+              acc = dp4a_su(qhi[h][1], c.y, acc);
+              acc = dp4a_su(qhi[h][2], c.z, acc);
+              acc = dp4a_su(qhi[h][3], c.w, acc);
+              acc *= 256;
+              acc = dp4a_uu(qlo[h][0], c.x, acc);
+              acc = dp4a_uu(qlo[h][1], c.y, acc);
+              acc = dp4a_uu(qlo[h][2], c.z, acc);
+              acc = dp4a_uu(qlo[h][3], c.w, acc);
+              part[jj][h] = acc;
+            }
+          } else {
+            const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
+#pragma unroll
+            for (int h = 0; h < HC; ++h) {
+              int acc = dp4a_ss(qhi[h][0], c.x, 0);
+              acc = dp4a_ss(qhi[h][1], c.y, acc);
+              acc = dp4a_ss(qhi[h][2], c.z, acc);
+              acc = dp4a_ss(qhi[h][3], c.w, acc);
+              acc *= 256;
+              acc = dp4a_us(qlo[h][0], c.x, acc);
+              acc = dp4a_us(qlo[h][1], c.y, acc);
+              acc = dp4a_us(qlo[h][2], c.z, acc);
+              acc = dp4a_us(qlo[h][3], c.w, acc);
+              part[jj][h] = acc;
+            }
+          }
+        }
+        // ---- butterfly reduce-scatter: lane `sub` ends with slot jj = sub
+#pragma unroll
+        for (int o = L / 2; o >= 1; o >>= 1) {
+          const bool upper = (sub & o) != 0;
+#pragma unroll
+          for (int j = 0; j < o; ++j)
+#pragma unroll
+            for (int h = 0; h < HC; ++h) {
+              const int keep = upper ? part[j + o][h] : part[j][h];
+              const int send = upper ? part[j][h] : part[j + o][h];
+              part[j][h] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        // ---- scores (log2 domain) for this lane's slot
+        const bool valid = s0 + own < kv_u;
+        const int kzp = static_cast<int8_t>(stage[C::KZ_OFF + own]);
+        const float ksc = reinterpret_cast<const float *>(stage + C::KS_OFF)[own];
+        const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[own];
+        const float zc = static_cast<float>(128 + static_cast<int8_t>(stage[C::VZ_OFF + own]));
+        const float madd = a.mask ? reinterpret_cast<const float *>(stage + C::M_OFF)[own] * kLog2e : 0.0f;
+        float sc[HC];
+        bool need = false;
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          // exact: |sum n (c - zp)| < 2^31 for D <= 256 (computed modulo 2^32)
+          const int dz = static_cast<int>(static_cast<uint32_t>(part[0][h]) -
+                                          static_cast<uint32_t>(kzp) * static_cast<uint32_t>(nsum[h]));
+          sc[h] = valid ? fmaf(static_cast<float>(dz), escale[h] * ksc, madd) : -INFINITY;
+          need |= sc[h] > m[h] + kRescaleThreshold;
+        }
+        // the group maximum is only needed when some score would overflow the lazy bound
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int h = 0; h < HC; ++h) {
+            float mt = sc[h];
+#pragma unroll
+            for (int o = L / 2; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+            const float mnew = fmaxf(m[h], mt);
+            if (mnew > m[h] + kRescaleThreshold) {
+              const float alpha = m[h] == -INFINITY ? 0.0f : ex2(m[h] - mnew);
+              lsum[h] *= alpha;
+              corr[h] *= alpha;
+              const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) o2[h][j] = __fmul2_rn(o2[h][j], al2);
+              m[h] = mnew;
+            }
+          }
+        }
+        float wv[4];
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          const float p = sc[h] == -INFINITY ? 0.0f : ex2(sc[h] - m[h]);
+          lsum[h] += p;
+          const float wt = p > 0.0f ? p * vsc : 0.0f;
+          corr[h] = fmaf(wt, zc, corr[h]);
+          wv[h] = wt * kWScale;
+        }
+#pragma unroll
+        for (int h = HC; h < 4; ++h) wv[h] = 0.0f;
+        *reinterpret_cast<float4 *>(wbuf + own * 4) = make_float4(wv[0], wv[1], wv[2], wv[3]);
+        __syncwarp();
+        // ---- p . v over the same L slots: code + 128 as the subnormal float (code + 128) * 2^-149
+#pragma unroll
+        for (int jj = 0; jj < L; ++jj) {
+          const int sl = g + NG * jj;
+          const float4 w4 = *reinterpret_cast<const float4 *>(wbuf + sl * 4);
+          const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
+          uint32_t x[4], y[4];  // dims (4i .. 4i+3) of the lane's 16: bytes of x[i] (low dims) or x/y pairs
+          if constexpr (C::Q4) {  // element 2i in the low nibble of byte i
+            const uint2 cw = *reinterpret_cast<const uint2 *>(stage + C::V_OFF + sl * CB + sub * 8);
+            x[0] = (cw.x & 0x0F0F0F0Fu) | 0x80808080u;         // dims 0, 2, 4, 6
+            y[0] = ((cw.x >> 4) & 0x0F0F0F0Fu) | 0x80808080u;  // dims 1, 3, 5, 7
+            x[1] = (cw.y & 0x0F0F0F0Fu) | 0x80808080u;         // dims 8, 10, 12, 14
+            y[1] = ((cw.y >> 4) & 0x0F0F0F0Fu) | 0x80808080u;  // dims 9, 11, 13, 15
+          } else {
+            const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::V_OFF + sl * D + sub * 16);
+            x[0] = c.x ^ 0x80808080u;
+            x[1] = c.y ^ 0x80808080u;
+            x[2] = c.z ^ 0x80808080u;
+            x[3] = c.w ^ 0x80808080u;
+          }
+          float2 vv2[8];
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) {
+            uint32_t lo, hi;
+            if constexpr (C::Q4) {  // vv2[k2] = dims (2 k2, 2 k2 + 1): byte k2 % 4 of the even / odd word
+              const uint32_t ev = x[k2 >> 2], od = y[k2 >> 2];
+              lo = __byte_perm(ev, 0u, 0x4440u + (k2 & 3));
+              hi = __byte_perm(od, 0u, 0x4440u + (k2 & 3));
+            } else {  // vv2[k2] = bytes 2 (k2 % 2), 2 (k2 % 2) + 1 of word k2 / 2
+              const uint32_t wd = x[k2 >> 1];
+              lo = __byte_perm(wd, 0u, 0x4440u + 2 * (k2 & 1));
+              hi = __byte_perm(wd, 0u, 0x4441u + 2 * (k2 & 1));
+            }
+            vv2[k2] = make_float2(__uint_as_float(lo), __uint_as_float(hi));
+          }
+#pragma unroll
+          for (int h = 0; h < HC; ++h) {
+            const float2 w2 = make_float2(wj[h], wj[h]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o2[h][j] = __ffma2_rn(w2, vv2[j], o2[h][j]);
+          }
         }
       }
-      const int hq = hk * a.G + hc * HC + h;
-      const float r = Lt > 0.0f ? O / Lt : 0.0f;
-      a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+      __syncwarp();  // the buffer and wbuf are free again
+      if (lane == 0 && k + R < nk && !sh[1]) issue(idx + R * NW, k + R);
+    }
+    if (deferred) {
+      if (u == u_first) publish(oscr + warp * HC * D, mlscr + warp * HC * 4);
+      else publish(reinterpret_cast<float *>(smem) + warp * kRingStride,
+                   reinterpret_cast<float *>(smem) + warp * kRingStride + HC * D);
+    } else {
+      publish(oscr + warp * HC * D, mlscr + warp * HC * 4);
+      __syncthreads();
+      combine(u, oscr, HC * D, mlscr, HC * 4);
     }
   }
+  if (deferred) {
+    __syncthreads();
+    combine(u_first, oscr, HC * D, mlscr, HC * 4);
+    if (u_last != u_first)
+      combine(u_last, reinterpret_cast<const float *>(smem), kRingStride,
+              reinterpret_cast<const float *>(smem) + HC * D, kRingStride);
+  }
+  __syncthreads();  // every partial is written; the scratch is free for the merge
+
+  // Only the first and the last unit of a contiguous range can be shared with
+  // other CTAs.  Count this CTA's partials of those (threads 0 and 1); the owner
+  // whose count completes a unit merges it, in owner order.
+  if (tid < 2) {
+    const int u = tid == 0 ? u_first : u_last;
+    const int owners = tid == 0 ? own0 : own1;
+    bool mine = false;
+    if (owners > 1 && (tid == 0 || u_last != u_first)) {
+      if (count_acq_rel(a.ws_cnt + u) == owners - 1) {
+        a.ws_cnt[u] = 0;  // every owner has counted: ready for the next call
+        mine = true;
+      }
+    }
+    sh[2 + tid] = mine ? 1 : 0;
+  }
+  __syncthreads();
+  if (sh[2]) merge_unit(u_first, 0, own0);
+  if (sh[3]) merge_unit(u_last, 1, own1);
 }
 
 // ----------------------------------------------------------------------------
@@ -682,31 +746,33 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int deco
 // ----------------------------------------------------------------------------
 int head_chunk(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1)); }
 
-// Tile geometry per head dim: (consumer warps, ring stages).
-template <int D>
-struct DTune;
-template <>
-struct DTune<64> { static constexpr int NW = 11, NST = 3; };
-template <>
-struct DTune<128> { static constexpr int NW = 11, NST = 2; };
-template <>
-struct DTune<256> { static constexpr int NW = 4, NST = 3; };
-
-struct WsLayout {
-  size_t ml, o, total;
-  int smax;
+// Warps per CTA and ring depth per warp: D = 256 chunks are 16.5 KB, so fewer
+// warps; the ring takes what shared memory is left after the scratch (at most 4).
+template <int D, int HC, bool Q4>
+struct Tune {
+  static constexpr int NW = D == 256 ? (HC >= 3 ? 5 : 6) : 11;
+  static constexpr int CHUNK = 64 * (Q4 ? D / 2 : D) + 448;
+  static constexpr int FIXED =
+      NW * 512 + NW * HC * D * 4 + NW * HC * 16 + NW * 8 * 8 + 48 + 4 * HC * D + 16 * HC + 8 * kMaxCtas;
+  static constexpr int RMAX = (232448 - FIXED) / (NW * CHUNK);
+  static constexpr int R = RMAX > 4 ? 4 : RMAX;
+  static_assert(R >= 2, "ring depth");
 };
 
-// Partials of split units: one record per (CTA, segment) slot; a CTA touches
-// at most ceil(U / ctas) + 2 units.
+struct WsLayout {
+  size_t ml, o, cnt, total;
+};
+
+// Two partial records per CTA (its first and last unit, the only ones it can
+// share), then one merge counter per unit.
 WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
   WsLayout w;
   const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
-  w.smax = static_cast<int>((U + ctas - 1) / ctas + 2);
-  const size_t recs = static_cast<size_t>(ctas) * w.smax;
+  const size_t recs = 2 * static_cast<size_t>(ctas);
   w.ml = 0;
   w.o = (recs * HC * 2 * 4 + 255) / 256 * 256;
-  w.total = w.o + recs * HC * D * 4;
+  w.cnt = w.o + (recs * HC * D * 4 + 255) / 256 * 256;
+  w.total = w.cnt + (static_cast<size_t>(U) * 4 + 255) / 256 * 256;
   return w;
 }
 
@@ -715,26 +781,29 @@ struct KernelTag {};  // names one decode_kernel instantiation for ensure_smem
 
 template <int D, int HC, bool Q4>
 int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
-  using C = Cfg<D, HC, DTune<D>::NW, DTune<D>::NST, Q4>;
-  if (a.kv_per_batch) {
-    if (const int st = ensure_smem<KernelTag<C, true>>(decode_kernel<C, true>, C::SMEM)) return st;
-    decode_kernel<C, true><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
-  } else {
-    if (const int st = ensure_smem<KernelTag<C, false>>(decode_kernel<C, false>, C::SMEM)) return st;
-    decode_kernel<C, false><<<ctas, C::THREADS, C::SMEM, stream>>>(a);
-  }
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.merge_ctas));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
+  using T = Tune<D, HC, Q4>;
+  using C = Cfg<D, HC, T::NW, T::R, Q4>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, merge_kernel<C>, a, ctas) != cudaSuccess) return KVQ_ECUDA;
+  {
+    cudaLaunchConfig_t dc = {};
+    dc.gridDim = dim3(static_cast<unsigned>(ctas));
+    dc.blockDim = dim3(C::THREADS);
+    dc.dynamicSmemBytes = C::SMEM;
+    dc.stream = stream;
+    dc.attrs = attr;
+    dc.numAttrs = 1;
+    cudaError_t e;
+    if (a.kv_per_batch) {
+      if (const int st = ensure_smem<KernelTag<C, true>>(decode_kernel<C, true>, C::SMEM)) return st;
+      e = cudaLaunchKernelEx(&dc, decode_kernel<C, true>, a);
+    } else {
+      if (const int st = ensure_smem<KernelTag<C, false>>(decode_kernel<C, false>, C::SMEM)) return st;
+      e = cudaLaunchKernelEx(&dc, decode_kernel<C, false>, a);
+    }
+    if (e != cudaSuccess) return KVQ_ECUDA;
+  }
   return launch_status();
 }
 
@@ -778,9 +847,10 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   const int G = Hq / Hkv;
   const int hc = head_chunk(G);
   const int nhc = G / hc;
+  if (static_cast<int64_t>(B) * Hkv * nhc * ((S + 31) / 32) >= INT32_MAX) return KVQ_EUNSUPPORTED;
   const int ctas = sm_count();
   const WsLayout w = ws_layout(B, Hkv, D, nhc, hc, ctas);
-  if (ctas > 256) return KVQ_EUNSUPPORTED;  // merge staging holds 256 owners x 4 heads
+  if (ctas > kMaxCtas) return KVQ_EUNSUPPORTED;  // owner records staged per unit
   if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KVQ_EINVAL;
   DecodeArgs a;
   a.q = static_cast<const uint16_t *>(q);
@@ -797,6 +867,7 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   a.ws_ml = reinterpret_cast<float *>(ws + w.ml);
   a.ws_o = reinterpret_cast<float *>(ws + w.o);
+  a.ws_cnt = reinterpret_cast<int32_t *>(ws + w.cnt);
   a.err = err_word;
   a.S = S;
   a.B = B;
@@ -804,11 +875,6 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   a.Hkv = Hkv;
   a.G = G;
   a.nhc = nhc;
-  a.smax = w.smax;
-  {
-    const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
-    a.merge_ctas = static_cast<int>(U < 4 * ctas ? U : 4 * ctas);
-  }
   a.qscale = sm_scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q4) {
@@ -897,4 +963,13 @@ extern "C" int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int
   if (st != KVQ_OK) return st;
   return kvq_decode_attn(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, mask, sm_scale, out,
                          scratch, KVQ_STATIC_SCRATCH_BYTES, err_word, stream);
+}
+
+extern "C" int kvq_decode_static_reset(void *stream) {
+  void *scratch = nullptr;
+  const int st = kvq::static_scratch_address(&scratch);
+  if (st != KVQ_OK) return st;
+  if (cudaMemsetAsync(scratch, 0, KVQ_STATIC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KVQ_ECUDA;
+  return KVQ_OK;
 }

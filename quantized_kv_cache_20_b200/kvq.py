@@ -40,7 +40,7 @@ MODE_INT4_AFFINE = 7
 
 EXPORTS = (
     "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
-    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
+    "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_static_reset", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
     "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
     "kvq_strerror", "kvq_version",
 )
@@ -87,6 +87,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_attn.restype = I
         lib.kvq_decode_attn_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, P]
         lib.kvq_decode_attn_static.restype = I
+        lib.kvq_decode_static_reset.argtypes = [P]
+        lib.kvq_decode_static_reset.restype = I
         lib.kvq_prefill_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I, I, F, P, P, P]
         lib.kvq_prefill_attn_varlen.argtypes = lib.kvq_prefill_attn.argtypes
         lib.kvq_prefill_attn_varlen.restype = I
@@ -176,12 +178,13 @@ def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, S: int) -> int:
 
 
 def decode_workspace(B: int, Hq: int, Hkv: int, D: int, S: int, device) -> torch.Tensor:
-    """A workspace of the size kvq_decode_attn needs (no initialisation required)."""
+    """A zero-filled workspace of the size kvq_decode_attn needs (its merge counters
+    start at zero; each completed call leaves them at zero)."""
     with torch.cuda.device(device):
         n = decode_workspace_bytes(B, Hq, Hkv, D, S)
     if n == 0:
         raise ValueError("unsupported decode configuration")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_word):
@@ -304,6 +307,14 @@ def decode_attn_static(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=Non
                                        float(sm_scale), _ptr(out), _ptr(err_word), _stream(q.device))
     _check("kvq_decode_attn_static", st)
     return out
+
+
+def decode_static_reset(device=None):
+    """kvq_decode_static_reset: zero the static decode buffer on `device` (needed only
+    after a call that reported KVQ_ERR_TIMEOUT)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check("kvq_decode_static_reset", load().kvq_decode_static_reset(_stream(dev)))
 
 
 def prefill_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, is_causal=False,

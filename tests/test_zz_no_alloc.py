@@ -51,8 +51,9 @@ def test_static_scratch_decode_matches_workspace_decode(shape):
 
 
 def test_static_scratch_rejects_problems_that_do_not_fit():
-    # 4096 kv heads x 8 batch needs far more partial storage than 8 MiB
-    B, Hq, Hkv, D, S = 512, 512, 64, 256, 16
+    # the workspace holds one merge counter per (batch row, kv head, head chunk):
+    # 40000 x 64 x 2 of them take 20 MB, more than the 8 MiB buffer
+    B, Hq, Hkv, D, S = 40000, 512, 64, 256, 16
     assert kvq.decode_workspace_bytes(B, Hq, Hkv, D, S) > kvq.STATIC_SCRATCH_BYTES
     lib = kvq.load()
     fake = ctypes.c_void_p(256)
