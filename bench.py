@@ -322,8 +322,7 @@ def run_kvq(args, dist: Dist):
 
     def step(l):
         K, V = layers[l]
-        kvq.write(0, kn, sm_step, *K)
-        kvq.write(0, vn, sm_step, *V)
+        kvq.write_kv(0, kn, vn, sm_step, K, V)
         kvq.decode_attn(q, *K, *V, kv_len, out=out, workspace=ws)
 
     def decode_only(l):
@@ -409,7 +408,7 @@ def run_kvq(args, dist: Dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * nsteps, "clocks": clk, "detail": detail,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * nsteps, "clocks": clk, "detail": detail,
     }
     if dist.rank == 0 and dist.world == 1:
         steps_c, el_c, _ = _oracle_decode_steps(args.cpu_seconds)
@@ -446,8 +445,7 @@ def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        kvq.write(0, dk, sm_step, *K)
-        kvq.write(0, dv, sm_step, *V)
+        kvq.write_kv(0, dk, dv, sm_step, K, V)
         kvq.decode_attn(dq, *K, *V, kv_len, out=dout, workspace=ws)
         hout[i].copy_(dout, non_blocking=True)
 
@@ -465,7 +463,7 @@ def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
     h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
     return {"value": dist.world * B / (ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": dout.numel() * 2, "ms_per_step": ms, "steps": steps,
-            "path": "pinned host -> device copies, kvq.write x2 + kvq.decode_attn via the Python binding "
+            "path": "pinned host -> device copies, kvq.write_kv + kvq.decode_attn via the Python binding "
                     "(no graph), device -> pinned host copy of the output"}
 
 

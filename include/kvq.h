@@ -107,6 +107,28 @@ int kvq_write(int mode, int round_scale, const void *x, int B, int H, int T, int
               void *scales, int8_t *zero_points, int32_t *err_word, void *stream);
 
 /*
+ * kvq_write_kv -- kvq_write of a step's K and V in one launch.
+ *
+ * Defines: as kvq_write; the pages write the key and the value of each new
+ * token through the same slot_mapping (ExecuTorch PR 24473, Summary: K and V
+ * caches updated through update_cache_with_indices; IndexerQuantCache page,
+ * 功能说明: the cache update in place at slot_mapping).  The K rows are
+ * written exactly as kvq_write(mode, round_scale, k, ..., k_codes, k_scales,
+ * k_zero_points) and the V rows as the same call on v; bit for bit the same.
+ *
+ * k, v         bf16 inputs of one shape [B, H, T, D], each with its own strides
+ *              (k_strides, v_strides: host, 4 entries, as x_strides).
+ * k_*, v_*     the two caches, each in the layout of `mode` (see kvq_write).
+ * Other arguments, checks and errors as for kvq_write.  Both kvq_write and
+ * kvq_write_kv launch as programmatic dependents of the kernel before them:
+ * they may start while it drains and read nothing before it has completed.
+ */
+int kvq_write_kv(int mode, int round_scale, const void *k, const void *v, int B, int H, int T, int D,
+                 const int64_t *k_strides, const int64_t *v_strides, const int32_t *slot_mapping,
+                 int64_t num_slots, void *k_codes, void *k_scales, int8_t *k_zero_points, void *v_codes,
+                 void *v_scales, int8_t *v_zero_points, int32_t *err_word, void *stream);
+
+/*
  * kvq_sink_plan -- slots of an attention-sink / ring cache for T new tokens.
  *
  * Defines: ExecuTorch PR 24473, Summary (CachePositionsManagerWithSink: a

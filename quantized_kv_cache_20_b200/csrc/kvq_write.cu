@@ -39,18 +39,24 @@ struct FastDiv {
   KVQ_DEVINL uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
 };
 
-struct WriteArgs {
+// One tensor written: its input and its cache.
+struct WriteTensor {
   const uint16_t *x;
   int64_t xs0, xs1, xs2;  // element strides of b, h, t
+  void *codes;
+  void *scales;
+  int8_t *zps;
+};
+
+struct WriteArgs {
+  WriteTensor t[2];       // K and V for kvq_write_kv; t[0] alone for kvq_write
+  int ntens;
   int B, H, T, D, GPR;    // GPR: 32-element groups per row
   FastDiv div_T, div_H, div_G;
   const int32_t *slot_mapping;
   int64_t S;
-  void *codes;
-  void *scales;
-  int8_t *zps;
   int32_t *err;
-  uint32_t groups;  // total groups
+  uint32_t groups;  // groups of one tensor
   int round_scale;  // MX-FP8 modes: 1 = scale rounded up to a power of two, 0 = its exponent as it stands
 };
 
@@ -140,14 +146,22 @@ KVQ_DEVINL uint32_t pack_low_bytes(float a, float b, float c, float d) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
+__global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__ WriteArgs a) {
+  // launched as a programmatic dependent: read nothing before the kernel ahead has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t stride = gridDim.x * kThreads;
   // Every lane of a warp runs the loop the same number of times (the bound is
-  // rounded up to whole warps), so the int8 mode's row shuffles see the whole warp.
-  const uint32_t total = (a.groups + 31u) & ~31u;
-  for (uint32_t g = blockIdx.x * kThreads + threadIdx.x; g < total; g += stride) {
+  // rounded up to whole warps), so the int8 mode's row shuffles see the whole
+  // warp.  With two tensors the V groups follow the K groups; a row never
+  // straddles the two (groups is a multiple of the groups per row).
+  const uint32_t all = a.groups * static_cast<uint32_t>(a.ntens);
+  const uint32_t total = (all + 31u) & ~31u;
+  for (uint32_t gg = blockIdx.x * kThreads + threadIdx.x; gg < total; gg += stride) {
+    const int ti = gg >= a.groups ? 1 : 0;
+    const uint32_t g = gg - (ti ? a.groups : 0u);
+    const WriteTensor &wt = a.t[ti];
     int b = 0, h = 0, t = 0, gi = 0, slot = -1;
-    if (g < a.groups) {
+    if (gg < all) {
       group_coords(a, g, b, h, t, gi);
       const int s = __ldg(a.slot_mapping + static_cast<int64_t>(b) * a.T + t);
       if (s != -1 && (s < 0 || s >= a.S)) {
@@ -159,7 +173,7 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
     uint32_t wx[16];  // 32 bf16 values, element 2j in the low half of wx[j]
     if (slot >= 0) {
       const uint4 *p =
-          reinterpret_cast<const uint4 *>(a.x + b * a.xs0 + h * a.xs1 + static_cast<int64_t>(t) * a.xs2 + gi * 32);
+          reinterpret_cast<const uint4 *>(wt.x + b * wt.xs0 + h * wt.xs1 + static_cast<int64_t>(t) * wt.xs2 + gi * 32);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint4 c = __ldg(p + k);
@@ -236,19 +250,19 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
           for (int j = 0; j < 8; ++j) acc |= (__float_as_uint(t2[8 * k + j]) & 0xFu) << (4 * j);
           w[k] = acc;
         }
-        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * (a.D >> 1) + gi * 16) =
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * (a.D >> 1) + gi * 16) =
             make_uint4(w[0], w[1], w[2], w[3]);
       } else {
         uint32_t w[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<int8_t *>(a.codes) + r * a.D + gi * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<int8_t *>(wt.codes) + r * a.D + gi * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
       if (gi == 0) {
-        static_cast<float *>(a.scales)[r] = scale;
-        a.zps[r] = static_cast<int8_t>(zp);
+        static_cast<float *>(wt.scales)[r] = scale;
+        wt.zps[r] = static_cast<int8_t>(zp);
       }
     } else {
       if (slot < 0) continue;
@@ -293,10 +307,10 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
                      (fp8x2<E5>(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
           }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * a.D + gi * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        static_cast<float *>(a.scales)[sidx] = scale;
+        static_cast<float *>(wt.scales)[sidx] = scale;
       } else if constexpr (MODE == KVQ_MODE_INT8_SYM) {
         // q = clamp(rne(x / scale), -127, 127), scale = amax / 127.  As in mode
         // 0, y = x * rcp(scale) lies within 1.5 * 2^-23 |y| of the correctly
@@ -330,10 +344,10 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
         uint32_t w[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) w[k] = pack_low_bytes(t2[4 * k], t2[4 * k + 1], t2[4 * k + 2], t2[4 * k + 3]);
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * a.D + gi * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        static_cast<float *>(a.scales)[sidx] = scale;
+        static_cast<float *>(wt.scales)[sidx] = scale;
       } else {
         constexpr bool MX8 = MODE == KVQ_MODE_MXFP8 || MODE == KVQ_MODE_MXFP8_E5M2;
         constexpr bool E5 = MODE == KVQ_MODE_MXFP8_E5M2;
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
           for (int k = 0; k < 8; ++k)
             w[k] = amax != 0.0f ? (fp8x2<E5>(y[4 * k], y[4 * k + 1]) | (fp8x2<E5>(y[4 * k + 2], y[4 * k + 3]) << 16))
                                 : 0u;
-          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * a.D + gi * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * a.D + gi * 32);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         } else {
@@ -364,10 +378,10 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
             w[k] = amax != 0.0f ? e2m1x8(y[8 * k], y[8 * k + 1], y[8 * k + 2], y[8 * k + 3], y[8 * k + 4],
                                          y[8 * k + 5], y[8 * k + 6], y[8 * k + 7])
                                 : 0u;
-          *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.codes) + r * (a.D >> 1) + gi * 16) =
+          *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * (a.D >> 1) + gi * 16) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
-        static_cast<uint8_t *>(a.scales)[sidx] = static_cast<uint8_t>(e);
+        static_cast<uint8_t *>(wt.scales)[sidx] = static_cast<uint8_t>(e);
       }
     }
   }
@@ -375,20 +389,29 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const WriteArgs a) {
 
 template <int MODE>
 int launch_write(const WriteArgs &a, cudaStream_t stream) {
-  const int64_t blocks_needed = (static_cast<int64_t>(a.groups) + kThreads - 1) / kThreads;
+  const int64_t blocks_needed = (static_cast<int64_t>(a.groups) * a.ntens + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads = a full SM
   const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-  write_kernel<MODE><<<grid, kThreads, 0, stream>>>(a);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, write_kernel<MODE>, a) != cudaSuccess) return KVQ_ECUDA;
   return launch_status();
 }
 
 }  // namespace
 }  // namespace kvq
 
-extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H, int T, int D,
-                         const int64_t *x_strides, const int32_t *slot_mapping, int64_t num_slots, void *codes,
-                         void *scales, int8_t *zero_points, int32_t *err_word, void *stream) {
-  using namespace kvq;
+namespace kvq {
+namespace {
+// Checks shared by kvq_write and kvq_write_kv; returns KVQ_OK or the error.
+int check_common(int mode, int B, int H, int T, int D, int64_t num_slots) {
   if (mode < KVQ_MODE_INT8_AFFINE || mode > KVQ_MODE_INT4_AFFINE) return KVQ_EINVAL;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || num_slots <= 0 || num_slots > INT32_MAX) return KVQ_EINVAL;
   if (mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_INT4_AFFINE) {
@@ -396,26 +419,41 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   } else {
     if (D % 32 != 0 || D > 8192) return KVQ_EUNSUPPORTED;
   }
-  if (static_cast<int64_t>(B) * H * T == 0) return KVQ_OK;
-  if (!x || !x_strides || !slot_mapping || !codes || !scales) return KVQ_EINVAL;
+  return KVQ_OK;
+}
+
+// Checks of one tensor's input and cache; fills `t`.
+int check_tensor(int mode, const void *x, const int64_t *x_strides, void *codes, void *scales, int8_t *zero_points,
+                 WriteTensor &t) {
+  if (!x || !x_strides || !codes || !scales) return KVQ_EINVAL;
   if ((mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_INT4_AFFINE) && !zero_points) return KVQ_EINVAL;
   // every row start 16-byte aligned: base aligned and strides multiples of 8 elements
   if (!aligned16(x) || !aligned16(codes)) return KVQ_EINVAL;
   for (int i = 0; i < 3; ++i)
     if (x_strides[i] < 0 || (x_strides[i] & 7) != 0) return KVQ_EINVAL;
-  // float scales (modes 0, 1, 4, 6) must be 4-byte aligned; E8M0 scales are bytes
+  // float scales (modes 0, 1, 4, 6, 7) must be 4-byte aligned; E8M0 scales are bytes
   const bool f32_scales = mode == KVQ_MODE_INT8_AFFINE || mode == KVQ_MODE_FP8_E4M3 || mode == KVQ_MODE_FP8_E5M2 ||
                           mode == KVQ_MODE_INT8_SYM || mode == KVQ_MODE_INT4_AFFINE;
   if (f32_scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return KVQ_EINVAL;
+  t.x = static_cast<const uint16_t *>(x);
+  t.xs0 = x_strides[0];
+  t.xs1 = x_strides[1];
+  t.xs2 = x_strides[2];
+  t.codes = codes;
+  t.scales = scales;
+  t.zps = zero_points;
+  return KVQ_OK;
+}
+
+int write_impl(int mode, int round_scale, int B, int H, int T, int D, const int32_t *slot_mapping, int64_t num_slots,
+               const WriteTensor *tens, int ntens, int32_t *err_word, void *stream) {
   // group indices use 32-bit arithmetic
   const int64_t groups = static_cast<int64_t>(B) * H * T * (D / 32);
-  if (groups >= (int64_t(1) << 31)) return KVQ_EUNSUPPORTED;
-
+  if (groups * ntens >= (int64_t(1) << 31)) return KVQ_EUNSUPPORTED;
   WriteArgs a;
-  a.x = static_cast<const uint16_t *>(x);
-  a.xs0 = x_strides[0];
-  a.xs1 = x_strides[1];
-  a.xs2 = x_strides[2];
+  a.t[0] = tens[0];
+  a.t[1] = ntens > 1 ? tens[1] : tens[0];
+  a.ntens = ntens;
   a.B = B;
   a.H = H;
   a.T = T;
@@ -426,9 +464,6 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
   a.div_G = FastDiv(static_cast<uint32_t>(D / 32));
   a.slot_mapping = slot_mapping;
   a.S = num_slots;
-  a.codes = codes;
-  a.scales = scales;
-  a.zps = zero_points;
   a.err = err_word;
   a.groups = static_cast<uint32_t>(groups);
   a.round_scale = round_scale ? 1 : 0;
@@ -443,4 +478,32 @@ extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H,
     case KVQ_MODE_INT8_SYM: return launch_write<KVQ_MODE_INT8_SYM>(a, s);
     default: return launch_write<KVQ_MODE_INT4_AFFINE>(a, s);
   }
+}
+}  // namespace
+}  // namespace kvq
+
+extern "C" int kvq_write(int mode, int round_scale, const void *x, int B, int H, int T, int D,
+                         const int64_t *x_strides, const int32_t *slot_mapping, int64_t num_slots, void *codes,
+                         void *scales, int8_t *zero_points, int32_t *err_word, void *stream) {
+  using namespace kvq;
+  if (const int st = check_common(mode, B, H, T, D, num_slots)) return st;
+  if (static_cast<int64_t>(B) * H * T == 0) return KVQ_OK;
+  if (!slot_mapping) return KVQ_EINVAL;
+  WriteTensor t;
+  if (const int st = check_tensor(mode, x, x_strides, codes, scales, zero_points, t)) return st;
+  return write_impl(mode, round_scale, B, H, T, D, slot_mapping, num_slots, &t, 1, err_word, stream);
+}
+
+extern "C" int kvq_write_kv(int mode, int round_scale, const void *k, const void *v, int B, int H, int T, int D,
+                            const int64_t *k_strides, const int64_t *v_strides, const int32_t *slot_mapping,
+                            int64_t num_slots, void *k_codes, void *k_scales, int8_t *k_zero_points, void *v_codes,
+                            void *v_scales, int8_t *v_zero_points, int32_t *err_word, void *stream) {
+  using namespace kvq;
+  if (const int st = check_common(mode, B, H, T, D, num_slots)) return st;
+  if (static_cast<int64_t>(B) * H * T == 0) return KVQ_OK;
+  if (!slot_mapping) return KVQ_EINVAL;
+  WriteTensor t[2];
+  if (const int st = check_tensor(mode, k, k_strides, k_codes, k_scales, k_zero_points, t[0])) return st;
+  if (const int st = check_tensor(mode, v, v_strides, v_codes, v_scales, v_zero_points, t[1])) return st;
+  return write_impl(mode, round_scale, B, H, T, D, slot_mapping, num_slots, t, 2, err_word, stream);
 }

@@ -39,7 +39,7 @@ MODE_INT8_SYM = 6
 MODE_INT4_AFFINE = 7
 
 EXPORTS = (
-    "kvq_write", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
+    "kvq_write", "kvq_write_kv", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
     "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_static_reset", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
     "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
     "kvq_strerror", "kvq_version",
@@ -69,6 +69,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
         lib.kvq_write.argtypes = [I, I, P, I, I, I, I, P, P, I64, P, P, P, P, P]
         lib.kvq_write.restype = I
+        lib.kvq_write_kv.argtypes = [I, I, P, P, I, I, I, I, P, P, P, I64, P, P, P, P, P, P, P, P]
+        lib.kvq_write_kv.restype = I
         lib.kvq_sink_plan.argtypes = [P, I, I, I, I64, P, P, P, P, P]
         lib.kvq_sink_plan.restype = I
         lib.kvq_sink_mask.argtypes = [P, I, P, I64, P, P]
@@ -148,6 +150,34 @@ def write(mode: int, x: torch.Tensor, slot_mapping: torch.Tensor, codes: torch.T
                           _ptr(slot_mapping), int(codes.shape[2]), _ptr(codes), _ptr(scales),
                           _ptr(zero_points), _ptr(err_word), _stream(x.device))
     _check("kvq_write", st)
+
+
+def write_kv(mode: int, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_cache, v_cache, *,
+             round_scale: bool = True, err_word: torch.Tensor | None = None) -> None:
+    """kvq_write_kv: kvq_write of k and v (both bf16 [B, H, T, D], unit last stride)
+    in one launch.  k_cache / v_cache are (codes, scales, zero_points or None)."""
+    for n, t in (("k", k), ("v", v)):
+        _cuda(n, t, torch.bfloat16, contiguous=False)
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError(f"{n} must be [B, H, T, D] with a unit last stride")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    _cuda("slot_mapping", slot_mapping, torch.int32)
+    kc, ks, kz = (tuple(k_cache) + (None,))[:3]
+    vc, vs, vz = (tuple(v_cache) + (None,))[:3]
+    for n, t in (("k_codes", kc), ("k_scales", ks), ("k_zero_points", kz), ("v_codes", vc), ("v_scales", vs),
+                 ("v_zero_points", vz)):
+        _cuda(n, t)
+    if kc.shape[2] != vc.shape[2]:
+        raise ValueError("the K and V caches must have the same number of slots")
+    _cuda("err_word", err_word, torch.int32)
+    B, H, T, D = k.shape
+    ks_ = (ctypes.c_int64 * 4)(*k.stride())
+    vs_ = (ctypes.c_int64 * 4)(*v.stride())
+    st = load().kvq_write_kv(int(mode), int(bool(round_scale)), _ptr(k), _ptr(v), B, H, T, D, ks_, vs_,
+                             _ptr(slot_mapping), int(kc.shape[2]), _ptr(kc), _ptr(ks), _ptr(kz), _ptr(vc), _ptr(vs),
+                             _ptr(vz), _ptr(err_word), _stream(k.device))
+    _check("kvq_write_kv", st)
 
 
 def sink_plan(input_pos: torch.Tensor, B: int, T: int, sink_size: int, slot_pos: torch.Tensor,

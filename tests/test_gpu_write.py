@@ -222,3 +222,44 @@ def test_tq4_write_ragged_shapes(D, shape):
     gpu, ref, err, oerr = _run_both(7, x, sm, cache0, S)
     assert err == 0 and oerr == 0
     _assert_equal(gpu, ref, f"tq4 D={D} shape={shape}")
+
+
+@pytest.mark.parametrize("mode", [0, 1, 3, 7])
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 5, 37), (8, 8, 1)])
+def test_write_kv_matches_two_oracle_writes(mode, shape):
+    """kvq_write_kv: K and V written in one launch, each bit-exact against the
+    oracle's write of that tensor alone; k is a strided view (a slice of a
+    wider tensor), v contiguous; some slots are -1."""
+    B, H, T = shape
+    D = 128
+    g = wl.generator(7000 + mode + 3 * T)
+    S = 2 * T + 5
+    wide = wl.bf16_normal((B, H, T, 2 * D), g, outlier_p=0.01, outlier_scale=10.0)
+    k = wide[..., D:]  # row stride 2D elements: still 16-byte aligned rows
+    v = wl.bf16_normal((B, H, T, D), g)
+    sm = torch.stack([wl.slot_mapping_random(T, S, T // 4, g) for _ in range(B)]).reshape(-1)
+    k0, v0 = _prefill(mode, B, H, S, D, g), _prefill(mode, B, H, S, D, g)
+    kg = [None if c is None else c.to(DEV) for c in k0]
+    vg = [None if c is None else c.to(DEV) for c in v0]
+    err = err_word()
+    kvq.write_kv(mode, k.to(DEV), v.to(DEV), sm.to(DEV), kg, vg, err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for x, c0, cg, what in ((k, k0, kg, "K"), (v, v0, vg, "V")):
+        ref = [None if c is None else c.numpy().copy() for c in c0]
+        oerr = oracle.write(mode, wl.u16(x.contiguous()), sm.numpy(), S, ref[0], ref[1], ref[2])
+        assert oerr == 0
+        _assert_equal([None if c is None else c.cpu().numpy() for c in cg], ref, f"write_kv {what} mode={mode}")
+
+
+def test_write_kv_rejects_mismatched_arguments():
+    g = wl.generator(7100)
+    D, S = 64, 16
+    kc = [c.to(DEV) for c in _prefill(0, 1, 1, S, D, g)]
+    vc = [c.to(DEV) for c in _prefill(0, 1, 1, S, D, g)]
+    x = wl.bf16_normal((1, 1, 2, D), g).to(DEV)
+    sm = torch.tensor([0, 1], dtype=torch.int32, device=DEV)
+    with pytest.raises(ValueError):
+        kvq.write_kv(0, x, x[:, :, :1], sm, kc, vc)
+    with pytest.raises(RuntimeError):
+        kvq.write_kv(0, x, x, sm, kc, (vc[0], vc[1], None))  # mode 0 needs V zero points
