@@ -89,9 +89,13 @@ struct DecodeArgs {
   float qscale;  // sm_scale * log2(e)
 };
 
-template <int D_, int HC_, int NW_, int R_, bool Q4_ = false>
+// NP chunk pipelines of P warps each; a pipeline's warps share its chunk ring
+// and split the HC heads of the unit, HW each.
+template <int D_, int HC_, int NP_, int P_, int R_, bool Q4_ = false>
 struct Cfg {
-  static constexpr int D = D_, HC = HC_, NW = NW_, R = R_;
+  static constexpr int D = D_, HC = HC_, NP = NP_, P = P_, R = R_;
+  static constexpr int HW = HC / P, NW = NP * P;
+  static_assert(HW * P == HC, "heads split evenly over a pipeline's warps");
   static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte
   static constexpr int CB = Q4 ? D / 2 : D;  // code bytes per slot
   static constexpr int L = D / 16;           // lanes per slot group (16 dims per lane)
@@ -107,12 +111,15 @@ struct Cfg {
   static constexpr int VZ_OFF = KZ_OFF + CS;
   static constexpr int CHUNK = VZ_OFF + CS;
   static_assert(CHUNK % 16 == 0, "chunk alignment");
-  // NW rings of R chunk buffers, then the per-warp scratch
-  static constexpr int WBUF_OFF = NW * R * CHUNK;              // [NW][32][4] float
-  static constexpr int OSCR_OFF = WBUF_OFF + NW * 32 * 16;     // [NW][HC][D] float
-  static constexpr int MLSCR_OFF = OSCR_OFF + NW * HC * D * 4; // [NW][HC][4] float: m, l, corr
-  static constexpr int BAR_OFF = MLSCR_OFF + NW * HC * 16;     // [NW][R] mbarrier
-  static constexpr int SH_OFF = BAR_OFF + NW * R * 8;           // 8 ints
+  // NP rings of R chunk buffers, then the per-warp scratch
+  static constexpr int WBUF_OFF = NP * R * CHUNK;              // [NW][32][4] float
+  // a warp's published state: O [HW][D] float, then (m, l, corr, -) [HW][4] float
+  static constexpr int PUBW = HW * D * 4 + HW * 16;
+  static constexpr int OSCR_OFF = WBUF_OFF + NW * 32 * 16;     // [NW] published states (first unit)
+  static constexpr int BAR_OFF = OSCR_OFF + NW * PUBW;         // [NP][R] mbarrier
+  static constexpr int CNT_OFF = BAR_OFF + NP * R * 8;         // [NP][R] int: warps done with the buffer
+  static constexpr int SH_OFF = (CNT_OFF + NP * R * 4 + 15) / 16 * 16;  // 8 ints
+  static_assert(P * PUBW <= R * CHUNK, "the last unit's states fit a pipeline's (then idle) ring");
   static constexpr int Q_OFF = (SH_OFF + 32 + 15) / 16 * 16;     // [2][HC] q rows: D/4 high, D/4 low words
   static constexpr int QMETA_OFF = Q_OFF + 2 * HC * 2 * D;       // [2][HC] (sum n, 2^E)
   static constexpr int RECS_OFF = QMETA_OFF + 2 * HC * 8;        // [2][kMaxCtas] owner records
@@ -157,6 +164,14 @@ KVQ_DEVINL float ex2(float x) {
 KVQ_DEVINL int count_acq_rel(int32_t *p) {
   int old;
   asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
+// Count a warp as done with a ring buffer (the count orders its reads before
+// the refill that the last warp of the pipeline issues).
+KVQ_DEVINL int done_count(int32_t *p) {
+  int old;
+  asm volatile("atom.add.acq_rel.cta.shared::cta.s32 %0, [%1], 1;" : "=r"(old) : "r"(smem_u32(p)) : "memory");
   return old;
 }
 
@@ -220,13 +235,18 @@ KVQ_DEVINL int max_kv_len(const DecodeArgs &a, volatile int32_t *red, bool repor
 template <class C, bool VARLEN>
 __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, HC = C::HC, NW = C::NW, R = C::R, L = C::L, NG = C::NG, CS = C::CS, CB = C::CB;
+  constexpr int NP = C::NP, P = C::P, HW = C::HW;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   volatile int32_t *sh = reinterpret_cast<volatile int32_t *>(smem + C::SH_OFF);  // scratch int, abort
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int32_t *cnt = reinterpret_cast<int32_t *>(smem + C::CNT_OFF);
   if (tid == 0) {
-    for (int i = 0; i < NW * R; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < NP * R; ++i) {
+      mbar_init(&full[i], 1);
+      cnt[i] = 0;
+    }
     fence_mbar_init();
     sh[1] = 0;
     sh[2] = 0;  // length of the merge list
@@ -259,8 +279,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   const int c_begin = static_cast<int>(range_start(cta, W, CT)), c_end = static_cast<int>(range_start(cta + 1, W, CT));
   if (c_begin >= c_end) return;  // more CTAs than chunks
 
-  // ---- this warp's chunks: c_begin + warp + k * NW for k in [0, nk), chunk k in buffer k % R
-  const int nk = c_begin + warp < c_end ? (c_end - 1 - c_begin - warp) / NW + 1 : 0;
+  // ---- this warp's pipeline pi and its chunks: c_begin + pi + k * NP for k in [0, nk),
+  // chunk k in buffer k % R of the pipeline; member pm takes heads [pm * HW, pm * HW + HW)
+  const int pi = warp / P, pm = warp % P;
+  const int nk = c_begin + pi < c_end ? (c_end - 1 - c_begin - pi) / NP + 1 : 0;
   // lane 0 only: start the copies of the warp's chunk k (flattened index idx)
   auto issue = [&](int idx, int k) {
     const int uu = idx / nch;
@@ -269,8 +291,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     const int kvu = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
     const int n = max(0, min(CS, kvu - s0));
     const int n16 = (n + 15) & ~15;  // S % 16 == 0 keeps this inside the slab
-    uint8_t *buf = smem + (warp * R + k % R) * C::CHUNK;
-    uint64_t *bar = full + warp * R + k % R;
+    uint8_t *buf = smem + (pi * R + k % R) * C::CHUNK;
+    uint64_t *bar = full + pi * R + k % R;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n16) * (2 * CB + 10) + (a.mask ? 4u * n16 : 0u));
     if (n16 > 0) {  // 0 bytes: the expect_tx above is a plain arrival
       const uint64_t pol = policy_evict_first();
@@ -284,19 +306,19 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       if (a.mask) bulk_g2s(buf + C::M_OFF, a.mask + s0, n16 * 4, bar);
     }
   };
-  if (lane == 0)
-    for (int k = 0; k < min(R, nk); ++k) issue(c_begin + warp + k * NW, k);
+  if (lane == 0 && pm == 0)
+    for (int k = 0; k < min(R, nk); ++k) issue(c_begin + pi + k * NP, k);
 
   const int u_first = c_begin / nch, u_last = (c_end - 1) / nch;  // the CTA's units
   const int g = lane / L, sub = lane % L;
   const int own = g + NG * sub;  // this lane's slot within the chunk after the reduce-scatter
   float *wbuf = reinterpret_cast<float *>(smem + C::WBUF_OFF) + warp * 32 * 4;
 
-  uint32_t qhi[HC][4], qlo[HC][4];
-  int nsum[HC];
-  float escale[HC];
-  float m[HC], lsum[HC], corr[HC];  // corr: sum of p * v_scale * (128 + v_zp), see kWScale
-  float2 o2[HC][8];
+  uint32_t qhi[HW][4], qlo[HW][4];
+  int nsum[HW];
+  float escale[HW];
+  float m[HW], lsum[HW], corr[HW];  // corr: sum of p * v_scale * (128 + v_zp), see kWScale
+  float2 o2[HW][8];
 
   // warps 0 .. HC-1: head `warp` of unit u onto the fixed-point grid, into q slot `slot`
   //   n = rne(q * sm_scale * log2e / 2^E), |n| <= 32767, E per head; stored as the
@@ -360,13 +382,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   // every lane: its slices of q slot `slot`, fresh softmax state
   auto load_q = [&](int slot) {
 #pragma unroll
-    for (int h = 0; h < HC; ++h) {
-      const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::Q_OFF) + (slot * HC + h) * (D / 2);
+    for (int h = 0; h < HW; ++h) {
+      const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::Q_OFF) + (slot * HC + pm * HW + h) * (D / 2);
       const uint4 hw = *reinterpret_cast<const uint4 *>(qs + sub * 4);
       const uint4 lw = *reinterpret_cast<const uint4 *>(qs + D / 4 + sub * 4);
       qhi[h][0] = hw.x; qhi[h][1] = hw.y; qhi[h][2] = hw.z; qhi[h][3] = hw.w;
       qlo[h][0] = lw.x; qlo[h][1] = lw.y; qlo[h][2] = lw.z; qlo[h][3] = lw.w;
-      const int2 meta = *reinterpret_cast<const int2 *>(smem + C::QMETA_OFF + (slot * HC + h) * 8);
+      const int2 meta = *reinterpret_cast<const int2 *>(smem + C::QMETA_OFF + (slot * HC + pm * HW + h) * 8);
       nsum[h] = meta.x;
       escale[h] = __int_as_float(meta.y);
       m[h] = -INFINITY;
@@ -381,7 +403,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   // writes (O, m, l, corr) for the warp: O at o_dst[h * D + d], the rest at ml_dst[h * 4]
   auto publish = [&](float *o_dst, float *ml_dst) {
 #pragma unroll
-    for (int h = 0; h < HC; ++h) {
+    for (int h = 0; h < HW; ++h) {
 #pragma unroll
       for (int o = L / 2; o >= 1; o >>= 1) {
         lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
@@ -408,7 +430,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     }
     if (g == 0) {
 #pragma unroll
-      for (int h = 0; h < HC; ++h) {
+      for (int h = 0; h < HW; ++h) {
         float4 *dst = reinterpret_cast<float4 *>(o_dst + h * D + sub * 16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -418,10 +440,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     }
   };
 
-  // all threads: combine the NW warp states of unit u (warp w at o_base + w * stride, its
-  // (m, l, corr) at ml_base + w * stride) in warp order; write the rows, or this CTA's
-  // partial when other CTAs share the unit
-  auto combine = [&](int u, const float *o_base, int o_stride, const float *ml_base, int ml_stride) {
+  // all threads: combine the warp states of unit u in pipeline order; the state of
+  // head h is held by member h / HW of every pipeline: warp (pi, pm)'s O at
+  // o_base + pi * p_stride + pm * m_stride (+ hh * D + d), its (m, l, corr) at
+  // ml_base + the same offsets (+ hh * 4).  Write the rows, or this CTA's partial
+  // when other CTAs share the unit.
+  auto combine = [&](int u, const float *o_base, const float *ml_base, int p_stride, int m_stride) {
     const int64_t CTn = gridDim.x;
     const bool alone = cta_of(static_cast<int64_t>(u) * nch, W, CTn) ==
                        cta_of(static_cast<int64_t>(u) * nch + nch - 1, W, CTn);
@@ -432,17 +456,19 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     const int64_t rec = 2 * static_cast<int64_t>(blockIdx.x) + (u == u_first ? 0 : 1);
     for (int e = tid; e < HC * D; e += C::THREADS) {
       const int h = e / D, d = e - h * D;
+      const int off = (h / HW) * m_stride;
+      const int hh = h % HW;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, ml_base[w * ml_stride + h * 4]);
+      for (int q = 0; q < NP; ++q) M = fmaxf(M, ml_base[q * p_stride + off + hh * 4]);
       float Lt = 0.0f, O = 0.0f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float4 mlc = *reinterpret_cast<const float4 *>(ml_base + w * ml_stride + h * 4);
+        for (int q = 0; q < NP; ++q) {
+          const float4 mlc = *reinterpret_cast<const float4 *>(ml_base + q * p_stride + off + hh * 4);
           const float f = mlc.x == -INFINITY ? 0.0f : ex2(mlc.x - M);
           Lt = fmaf(f, mlc.y, Lt);
-          O = fmaf(f, fmaf(o_base[w * o_stride + h * D + d], kOScale, -mlc.z), O);
+          O = fmaf(f, fmaf(o_base[q * p_stride + off + hh * D + d], kOScale, -mlc.z), O);
         }
       }
       if (alone) {
@@ -525,8 +551,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   // With more, every unit closes with two CTA barriers.
   const bool deferred = u_last - u_first <= 1;
   float *oscr = reinterpret_cast<float *>(smem + C::OSCR_OFF);
-  float *mlscr = reinterpret_cast<float *>(smem + C::MLSCR_OFF);
-  constexpr int kRingStride = R * C::CHUNK / 4;  // floats from one warp's ring to the next
+  constexpr int kRingStride = R * C::CHUNK / 4;  // floats from one pipeline's ring to the next
   const int own0 = stage_owners(u_first, 0);
   const int own1 = u_last != u_first ? stage_owners(u_last, 1) : 1;
   if (deferred) {
@@ -544,10 +569,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     const int kv_u = VARLEN ? row_kv(a, static_cast<int>(u / a.nhc / a.Hkv)) : kv;
     const int seg_end = min(c_end, (u + 1) * nch);
     for (; k < nk; ++k) {
-      const int idx = c_begin + warp + k * NW;
+      const int idx = c_begin + pi + k * NP;
       if (idx >= seg_end) break;
-      const uint8_t *stage = smem + (warp * R + k % R) * C::CHUNK;
-      const bool ok = wait_or_abort(full + warp * R + k % R, static_cast<uint32_t>(k / R) & 1u, sh + 1);
+      const uint8_t *stage = smem + (pi * R + k % R) * C::CHUNK;
+      const bool ok = wait_or_abort(full + pi * R + k % R, static_cast<uint32_t>(k / R) & 1u, sh + 1);
       if (!ok && lane == 0) {
         report(a.err, KVQ_ERR_TIMEOUT);
         sh[1] = 1;
@@ -555,7 +580,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
       const int s0 = (idx - u * nch) * CS;
       if (ok && s0 < kv_u) {
         // ---- q . k on dp4a for the L slots of this lane group (slot = g + NG*jj)
-        int part[L][HC];
+        int part[L][HW];
 #pragma unroll
         for (int jj = 0; jj < L; ++jj) {
           const int sl = g + NG * jj;
@@ -565,7 +590,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
             unpack_nibbles(cw.x, c.x, c.y);
             unpack_nibbles(cw.y, c.z, c.w);
 #pragma unroll
-            for (int h = 0; h < HC; ++h) {
+            for (int h = 0; h < HW; ++h) {
               int acc = dp4a_su(qhi[h][0], c.x, 0);
               acc = dp4a_su(qhi[h][1], c.y, acc);
               acc = dp4a_su(qhi[h][2], c.z, acc);
@@ -580,7 +605,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
           } else {
             const uint4 c = *reinterpret_cast<const uint4 *>(stage + C::K_OFF + sl * D + sub * 16);
 #pragma unroll
-            for (int h = 0; h < HC; ++h) {
+            for (int h = 0; h < HW; ++h) {
               int acc = dp4a_ss(qhi[h][0], c.x, 0);
               acc = dp4a_ss(qhi[h][1], c.y, acc);
               acc = dp4a_ss(qhi[h][2], c.z, acc);
@@ -601,7 +626,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 #pragma unroll
           for (int j = 0; j < o; ++j)
 #pragma unroll
-            for (int h = 0; h < HC; ++h) {
+            for (int h = 0; h < HW; ++h) {
               const int keep = upper ? part[j + o][h] : part[j][h];
               const int send = upper ? part[j][h] : part[j + o][h];
               part[j][h] = keep + __shfl_xor_sync(0xffffffffu, send, o);
@@ -614,10 +639,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         const float vsc = reinterpret_cast<const float *>(stage + C::VS_OFF)[own];
         const float zc = static_cast<float>(128 + static_cast<int8_t>(stage[C::VZ_OFF + own]));
         const float madd = a.mask ? reinterpret_cast<const float *>(stage + C::M_OFF)[own] * kLog2e : 0.0f;
-        float sc[HC];
+        float sc[HW];
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < HC; ++h) {
+        for (int h = 0; h < HW; ++h) {
           // exact: |sum n (c - zp)| < 2^31 for D <= 256 (computed modulo 2^32)
           const int dz = static_cast<int>(static_cast<uint32_t>(part[0][h]) -
                                           static_cast<uint32_t>(kzp) * static_cast<uint32_t>(nsum[h]));
@@ -627,7 +652,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         // the group maximum is only needed when some score would overflow the lazy bound
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int h = 0; h < HC; ++h) {
+          for (int h = 0; h < HW; ++h) {
             float mt = sc[h];
 #pragma unroll
             for (int o = L / 2; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
@@ -645,7 +670,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         }
         float wv[4];
 #pragma unroll
-        for (int h = 0; h < HC; ++h) {
+        for (int h = 0; h < HW; ++h) {
           const float p = sc[h] == -INFINITY ? 0.0f : ex2(sc[h] - m[h]);
           lsum[h] += p;
           const float wt = p > 0.0f ? p * vsc : 0.0f;
@@ -653,7 +678,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
           wv[h] = wt * kWScale;
         }
 #pragma unroll
-        for (int h = HC; h < 4; ++h) wv[h] = 0.0f;
+        for (int h = HW; h < 4; ++h) wv[h] = 0.0f;
         *reinterpret_cast<float4 *>(wbuf + own * 4) = make_float4(wv[0], wv[1], wv[2], wv[3]);
         __syncwarp();
         // ---- p . v over the same L slots: code + 128 as the subnormal float (code + 128) * 2^-149
@@ -692,32 +717,39 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
             vv2[k2] = make_float2(__uint_as_float(lo), __uint_as_float(hi));
           }
 #pragma unroll
-          for (int h = 0; h < HC; ++h) {
+          for (int h = 0; h < HW; ++h) {
             const float2 w2 = make_float2(wj[h], wj[h]);
 #pragma unroll
             for (int j = 0; j < 8; ++j) o2[h][j] = __ffma2_rn(w2, vv2[j], o2[h][j]);
           }
         }
       }
-      __syncwarp();  // the buffer and wbuf are free again
-      if (lane == 0 && k + R < nk && !sh[1]) issue(idx + R * NW, k + R);
+      __syncwarp();  // the buffer and wbuf are free again (for this warp)
+      if (lane == 0 && (P == 1 || done_count(cnt + pi * R + k % R) == P - 1)) {
+        if (P > 1) cnt[pi * R + k % R] = 0;  // the pipeline's last warp refills the buffer
+        if (k + R < nk && !sh[1]) issue(idx + R * NP, k + R);
+      }
     }
-    if (deferred) {
-      if (u == u_first) publish(oscr + warp * HC * D, mlscr + warp * HC * 4);
-      else publish(reinterpret_cast<float *>(smem) + warp * kRingStride,
-                   reinterpret_cast<float *>(smem) + warp * kRingStride + HC * D);
-    } else {
-      publish(oscr + warp * HC * D, mlscr + warp * HC * 4);
+    if (deferred && u == u_last && u_last != u_first) {
+      // the rings hold the last unit's state once every warp is past its chunks
       __syncthreads();
-      combine(u, oscr, HC * D, mlscr, HC * 4);
+      float *rw = reinterpret_cast<float *>(smem + pi * R * C::CHUNK + pm * C::PUBW);
+      publish(rw, rw + HW * D);
+    } else {
+      float *ow = oscr + warp * (C::PUBW / 4);
+      publish(ow, ow + HW * D);
+      if (!deferred) {
+        __syncthreads();
+        combine(u, oscr, oscr + HW * D, P * C::PUBW / 4, C::PUBW / 4);
+      }
     }
   }
   if (deferred) {
     __syncthreads();
-    combine(u_first, oscr, HC * D, mlscr, HC * 4);
+    combine(u_first, oscr, oscr + HW * D, P * C::PUBW / 4, C::PUBW / 4);
     if (u_last != u_first)
-      combine(u_last, reinterpret_cast<const float *>(smem), kRingStride,
-              reinterpret_cast<const float *>(smem) + HC * D, kRingStride);
+      combine(u_last, reinterpret_cast<const float *>(smem), reinterpret_cast<const float *>(smem) + HW * D,
+              kRingStride, C::PUBW / 4);
   }
   __syncthreads();  // every partial is written; the scratch is free for the merge
 
@@ -746,15 +778,21 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 // ----------------------------------------------------------------------------
 int head_chunk(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1)); }
 
-// Warps per CTA and ring depth per warp: D = 256 chunks are 16.5 KB, so fewer
-// warps; the ring takes what shared memory is left after the scratch (at most 4).
+// Pipelines and warps per pipeline: with an even head chunk two warps share a
+// pipeline and take half the heads each (fewer registers per warp, so more
+// warps per SM to hide latency); D = 256 chunks are 16.5 KB, so fewer
+// pipelines.  The ring takes what shared memory is left (at most 4 deep).
 template <int D, int HC, bool Q4>
 struct Tune {
-  static constexpr int NW = D == 256 ? (HC >= 3 ? 5 : 6) : 11;
+  static constexpr int P = HC % 2 == 0 ? 2 : 1;
+  static constexpr int HW = HC / P;
+  static constexpr int NP = D == 256 ? (P == 2 ? (HC == 4 ? 5 : 6) : 5) : (P == 2 ? 8 : 11);
+  static constexpr int NW = NP * P;
   static constexpr int CHUNK = 64 * (Q4 ? D / 2 : D) + 448;
+  static constexpr int PUBW = HW * D * 4 + HW * 16;
   static constexpr int FIXED =
-      NW * 512 + NW * HC * D * 4 + NW * HC * 16 + NW * 8 * 8 + 48 + 4 * HC * D + 16 * HC + 8 * kMaxCtas;
-  static constexpr int RMAX = (232448 - FIXED) / (NW * CHUNK);
+      NW * 512 + NW * PUBW + NP * 8 * 12 + 64 + 4 * HC * D + 16 * HC + 8 * kMaxCtas;
+  static constexpr int RMAX = (232448 - FIXED) / (NP * CHUNK);
   static constexpr int R = RMAX > 4 ? 4 : RMAX;
   static_assert(R >= 2, "ring depth");
 };
@@ -782,7 +820,7 @@ struct KernelTag {};  // names one decode_kernel instantiation for ensure_smem
 template <int D, int HC, bool Q4>
 int launch_decode(DecodeArgs a, int ctas, cudaStream_t stream) {
   using T = Tune<D, HC, Q4>;
-  using C = Cfg<D, HC, T::NW, T::R, Q4>;
+  using C = Cfg<D, HC, T::NP, T::P, T::R, Q4>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
