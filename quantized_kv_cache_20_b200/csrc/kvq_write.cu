@@ -12,11 +12,13 @@
 //
 // The arithmetic is binary32, one round-to-nearest-even per operation, in the
 // order the definitions state, so codes, scales and zero points are
-// reproducible bit for bit.  A division by the per-row/per-group scale is done
-// as y = x * rcp(scale) (rcp correctly rounded): y lies within 3 ulp of the
-// correctly rounded quotient, so whenever y is provably clear of every rounding
-// boundary of the final code, the code is the same; a group with any element
-// next to a boundary is redone with exact IEEE division (__fdiv_rn).
+// reproducible bit for bit.  The affine modes (0, 7; scale >= FLT_EPSILON)
+// take the quotient x / scale from Markstein's correction of x * rcp(scale)
+// (rcp correctly rounded), which is the correctly rounded quotient wherever it
+// can move a code.  The block modes divide as y = x * rcp(scale): y lies within
+// 3 ulp of the correctly rounded quotient, so whenever y is provably clear of
+// every rounding boundary of the final code, the code is the same; a group with
+// any element next to a boundary is redone with exact IEEE division (__fdiv_rn).
 #include <cuda_bf16.h>
 #include <float.h>
 
@@ -212,33 +214,26 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
       if (scale < FLT_EPSILON) scale = FLT_EPSILON;
       int zp = static_cast<int>(kLo) - __float2int_rn(__fdiv_rn(mn, scale));
       zp = zp < static_cast<int>(kLo) ? static_cast<int>(kLo) : (zp > static_cast<int>(kHi) ? static_cast<int>(kHi) : zp);
+      // q = clamp(rne(x / scale) + zp): the quotient x / scale correctly rounded by
+      // Markstein's correction (IBM J. Res. Develop. 34(1), 1990) of q0 = x * rcp
+      // with rcp = RN(1 / scale): r = x - scale * q0 is exact (one FMA), and
+      // RN(q0 + r * rcp) is RN(x / scale) for every x of the row except subnormal
+      // ones, whose quotients lie far below 0.5 and give the code zp either way.
+      // Adding 1.5 * 2^23 then rounds it to an integer (rne), the zero point is an
+      // exact integer add, and the clamp is exact; the code is the low mantissa byte.
       const float rcp = __frcp_rn(scale);
-      const float zpf = static_cast<float>(zp);
-      // q = clamp(rne(x/scale) + zp) = rne(clamp(y + zp)) for y = x*rcp, taken
-      // with the kMagic add.  y is within 1.5 * 2^-23 |y| of the correctly
-      // rounded quotient and forming y + zp moves it by at most 2^-18 without
-      // crossing a half-integer, so a distance to the nearest half-integer
-      // above 2^-22 |y| + 2^-17 settles the code.
+      const float2 rcp2 = make_float2(rcp, rcp), nsc2 = make_float2(-scale, -scale);
+      const float2 mg2 = make_float2(kMagic, kMagic), zp2 = make_float2(static_cast<float>(zp), static_cast<float>(zp));
+      const float t_lo = kMagic + kLo, t_hi = kMagic + kHi;
       float t2[32];
-      float worst = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
-        const float y = __fmul_rn(x, rcp);
-        const float yz = fminf(fmaxf(__fadd_rn(y, zpf), kLo), kHi);
-        const float tt = __fadd_rn(yz, kMagic);
-        const float dd = __fsub_rn(yz, __fsub_rn(tt, kMagic));  // yz - rne(yz)
-        worst = fmaxf(worst, fmaf(fabsf(y), 0x1p-22f, fabsf(dd)));
-        t2[i] = tt;
-      }
-      if (worst >= 0.5f - 0x1p-17f) {  // rare: settle the group with exact division
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = (i & 1) ? bf16hi(wx[i >> 1]) : bf16lo(wx[i >> 1]);
-          int q = __float2int_rn(__fdiv_rn(x, scale)) + zp;
-          q = q < static_cast<int>(kLo) ? static_cast<int>(kLo) : (q > static_cast<int>(kHi) ? static_cast<int>(kHi) : q);
-          t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
-        }
+      for (int j = 0; j < 16; ++j) {
+        const float2 x = make_float2(bf16lo(wx[j]), bf16hi(wx[j]));
+        const float2 q0 = __fmul2_rn(x, rcp2);
+        const float2 q = __ffma2_rn(__ffma2_rn(q0, nsc2, x), rcp2, q0);
+        const float2 t = __fadd2_rn(__fadd2_rn(q, mg2), zp2);
+        t2[2 * j] = fminf(fmaxf(t.x, t_lo), t_hi);
+        t2[2 * j + 1] = fminf(fmaxf(t.y, t_lo), t_hi);
       }
       if constexpr (Q4) {
         // the code sits in the low mantissa bits of t2; element 2i goes to the low nibble of byte i
