@@ -12,13 +12,11 @@
 //
 // The arithmetic is binary32, one round-to-nearest-even per operation, in the
 // order the definitions state, so codes, scales and zero points are
-// reproducible bit for bit.  The affine modes (0, 7; scale >= FLT_EPSILON)
-// take the quotient x / scale from Markstein's correction of x * rcp(scale)
-// (rcp correctly rounded), which is the correctly rounded quotient wherever it
-// can move a code.  The block modes divide as y = x * rcp(scale): y lies within
-// 3 ulp of the correctly rounded quotient, so whenever y is provably clear of
-// every rounding boundary of the final code, the code is the same; a group with
-// any element next to a boundary is redone with exact IEEE division (__fdiv_rn).
+// reproducible bit for bit.  Division by a per-row/per-group scale takes the
+// quotient from Markstein's correction of x * rcp(scale) (rcp correctly
+// rounded), which is the correctly rounded quotient wherever it can move a code;
+// groups of tiny values (amax < 2^-60) divide exactly (__fdiv_rn).  MX scales are
+// powers of two, so their quotients are exact products.
 #include <cuda_bf16.h>
 #include <float.h>
 
@@ -140,6 +138,23 @@ KVQ_DEVINL void group_coords(const WriteArgs &a, uint32_t g, int &b, int &h, int
   b = static_cast<int>(bq);
 }
 
+// x / s correctly rounded, for two x, by Markstein's correction of x * rcp
+// (rcp = RN(1 / s); IBM J. Res. Develop. 34(1), 1990): the residual
+// s * q0 - x is exact in one FMA and RN(q0 - r * rcp) is the correctly rounded
+// quotient unless x or the quotient is subnormal (there both stay within an ulp
+// or two, with the same sign).  Taking the residual as s * q0 - x keeps the sign
+// of a zero x: q0 - (+0) * rcp = -0 for x = -0, as -0 / s is.
+KVQ_DEVINL float2 div2_markstein(float2 x, float s, float rcp) {
+  const float2 q0 = __fmul2_rn(x, make_float2(rcp, rcp));
+  const float2 r = __ffma2_rn(q0, make_float2(s, s), make_float2(-x.x, -x.y));
+  return __ffma2_rn(r, make_float2(-rcp, -rcp), q0);
+}
+// Groups with amax at least this use div2_markstein: the scale (amax / Q_MAX,
+// Q_MAX <= 57344) is then a normal float with a finite reciprocal, and a
+// subnormal x has a quotient below 2^-50, far under half the smallest FP8 or
+// integer step, so its code is 0 however it is rounded.
+constexpr float kMarksteinMin = 0x1p-60f;
+
 // Low bytes of four floats that hold integers in their low mantissa bits.
 KVQ_DEVINL uint32_t pack_low_bytes(float a, float b, float c, float d) {
   const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040u);
@@ -222,15 +237,12 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
       // Adding 1.5 * 2^23 then rounds it to an integer (rne), the zero point is an
       // exact integer add, and the clamp is exact; the code is the low mantissa byte.
       const float rcp = __frcp_rn(scale);
-      const float2 rcp2 = make_float2(rcp, rcp), nsc2 = make_float2(-scale, -scale);
       const float2 mg2 = make_float2(kMagic, kMagic), zp2 = make_float2(static_cast<float>(zp), static_cast<float>(zp));
       const float t_lo = kMagic + kLo, t_hi = kMagic + kHi;
       float t2[32];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float2 x = make_float2(bf16lo(wx[j]), bf16hi(wx[j]));
-        const float2 q0 = __fmul2_rn(x, rcp2);
-        const float2 q = __ffma2_rn(__ffma2_rn(q0, nsc2, x), rcp2, q0);
+        const float2 q = div2_markstein(make_float2(bf16lo(wx[j]), bf16hi(wx[j])), scale, rcp);
         const float2 t = __fadd2_rn(__fadd2_rn(q, mg2), zp2);
         t2[2 * j] = fminf(fmaxf(t.x, t_lo), t_hi);
         t2[2 * j + 1] = fminf(fmaxf(t.y, t_lo), t_hi);
@@ -276,65 +288,45 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
         constexpr bool E5 = MODE == KVQ_MODE_FP8_E5M2;
         const float scale = __fdiv_rn(amax, E5 ? 57344.0f : 448.0f);
         uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (amax != 0.0f) {
+        if (amax >= kMarksteinMin) {  // the correctly rounded quotient, then one cvt per pair
           const float rcp = __frcp_rn(scale);
-          // cvt is monotone: if y(1 - 2^-20) and y(1 + 2^-20) -- which bracket
-          // the correctly rounded quotient -- get the same code, so does it.
-          uint32_t diff = 0u;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float2 y0 = __fmul2_rn(make_float2(v[4 * k], v[4 * k + 1]), make_float2(rcp, rcp));
-            const float2 y1 = __fmul2_rn(make_float2(v[4 * k + 2], v[4 * k + 3]), make_float2(rcp, rcp));
-            const float2 l0 = __fmul2_rn(y0, make_float2(1.0f - 0x1p-20f, 1.0f - 0x1p-20f));
-            const float2 h0 = __fmul2_rn(y0, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
-            const float2 l1 = __fmul2_rn(y1, make_float2(1.0f - 0x1p-20f, 1.0f - 0x1p-20f));
-            const float2 h1 = __fmul2_rn(y1, make_float2(1.0f + 0x1p-20f, 1.0f + 0x1p-20f));
-            const uint32_t c = fp8x2<E5>(y0.x, y0.y) | (fp8x2<E5>(y1.x, y1.y) << 16);
-            const uint32_t cl = fp8x2<E5>(l0.x, l0.y) | (fp8x2<E5>(l1.x, l1.y) << 16);
-            const uint32_t ch = fp8x2<E5>(h0.x, h0.y) | (fp8x2<E5>(h1.x, h1.y) << 16);
-            diff |= (c ^ cl) | (c ^ ch);
-            w[k] = c;
+            const float2 y0 = div2_markstein(make_float2(v[4 * k], v[4 * k + 1]), scale, rcp);
+            const float2 y1 = div2_markstein(make_float2(v[4 * k + 2], v[4 * k + 3]), scale, rcp);
+            w[k] = fp8x2<E5>(y0.x, y0.y) | (fp8x2<E5>(y1.x, y1.y) << 16);
           }
-          if (diff) {  // rare: exact division for the whole group
+        } else if (amax != 0.0f) {  // a group of tiny values: exact division
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              w[k] = fp8x2<E5>(__fdiv_rn(v[4 * k], scale), __fdiv_rn(v[4 * k + 1], scale)) |
-                     (fp8x2<E5>(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
-          }
+          for (int k = 0; k < 8; ++k)
+            w[k] = fp8x2<E5>(__fdiv_rn(v[4 * k], scale), __fdiv_rn(v[4 * k + 1], scale)) |
+                   (fp8x2<E5>(__fdiv_rn(v[4 * k + 2], scale), __fdiv_rn(v[4 * k + 3], scale)) << 16);
         }
         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(wt.codes) + r * a.D + gi * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         static_cast<float *>(wt.scales)[sidx] = scale;
       } else if constexpr (MODE == KVQ_MODE_INT8_SYM) {
-        // q = clamp(rne(x / scale), -127, 127), scale = amax / 127.  As in mode
-        // 0, y = x * rcp(scale) lies within 1.5 * 2^-23 |y| of the correctly
-        // rounded quotient, so a distance to the nearest half-integer above
-        // 2^-22 |y| settles the code; otherwise the group is redone exactly.
+        // q = clamp(rne(x / scale), -127, 127), scale = amax / 127: the correctly
+        // rounded quotient, rounded to an integer by the 1.5 * 2^23 add, clamped
         const float scale = __fdiv_rn(amax, 127.0f);
         float t2[32];
-        if (amax != 0.0f) {
+        if (amax >= kMarksteinMin) {
           const float rcp = __frcp_rn(scale);
-          float worst = 0.0f;
+          const float2 mg2 = make_float2(kMagic, kMagic);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float2 t = __fadd2_rn(div2_markstein(make_float2(v[2 * j], v[2 * j + 1]), scale, rcp), mg2);
+            t2[2 * j] = fminf(fmaxf(t.x, kMagic - 127.0f), kMagic + 127.0f);
+            t2[2 * j + 1] = fminf(fmaxf(t.y, kMagic - 127.0f), kMagic + 127.0f);
+          }
+        } else {  // zero or a group of tiny values: exact division
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float y = fminf(fmaxf(__fmul_rn(v[i], rcp), -127.0f), 127.0f);
-            const float tt = __fadd_rn(y, kMagic);
-            const float dd = __fsub_rn(y, __fsub_rn(tt, kMagic));  // y - rne(y)
-            worst = fmaxf(worst, fmaf(fabsf(y), 0x1p-22f, fabsf(dd)));
-            t2[i] = tt;
+            int q = amax != 0.0f ? __float2int_rn(__fdiv_rn(v[i], scale)) : 0;
+            q = q < -127 ? -127 : (q > 127 ? 127 : q);
+            t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
           }
-          if (worst >= 0.5f - 0x1p-17f) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              int q = __float2int_rn(__fdiv_rn(v[i], scale));
-              q = q < -127 ? -127 : (q > 127 ? 127 : q);
-              t2[i] = __uint_as_float(0x4B400000u + static_cast<uint32_t>(q));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) t2[i] = kMagic;  // code 0
         }
         uint32_t w[8];
 #pragma unroll
