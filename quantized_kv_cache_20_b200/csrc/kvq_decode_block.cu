@@ -88,21 +88,41 @@ KVQ_DEVINL float group_scale(const void *scales, int64_t idx) {
   }
 }
 
+// 16-byte global -> shared copy that completes asynchronously (cp.async.cg).
+KVQ_DEVINL void cp_async16(void *dst_smem, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+KVQ_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+KVQ_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 KVQ_DEVINL float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
+// Bytes of one warp's staged V tile: 32 slots of codes, then their scales.
+template <int MODE, int D>
+struct VTile {
+  static constexpr int CB = Fmt<MODE>::FP4 ? D / 2 : D;
+  static constexpr int SB = Fmt<MODE>::F32_SCALE ? 32 * (D / 32) * 4 : 32 * (D / 32);
+  static constexpr int BYTES = 32 * CB + (SB + 15) / 16 * 16;
+};
+template <int MODE, int D>
+struct BlockTag {};  // names one decode_block_kernel instantiation for ensure_smem
+
 template <int MODE, int D>
 __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
   constexpr int CB = Fmt<MODE>::FP4 ? D / 2 : D;  // code bytes per slot
   constexpr int NGRP = D / 32;
   constexpr int DPL = D / 32;                     // head dims per lane in p.v
+  constexpr bool F32S = Fmt<MODE>::F32_SCALE;
   __shared__ __align__(16) float q_s[kMaxG * D];
   __shared__ __align__(16) float p_s[kWarps][32][kMaxG];
   __shared__ float mc_s[kMaxG], lc_s[kMaxG];  // the CTA's combined state, warp by warp
   __shared__ __align__(16) float oc_s[kMaxG][D];
+  // each warp's V tile (dynamic shared memory): codes of its 32 slots, then their scales
+  extern __shared__ __align__(16) uint8_t vt_s[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -132,54 +152,106 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
     for (int k = 0; k < DPL; ++k) acc[h][k] = 0.0f;
   }
 
+  uint8_t *vt = vt_s + warp * VTile<MODE, D>::BYTES;
   for (int base = s_begin + warp * 32; base < s_end; base += kWarps * 32) {
-    // ---- q.k, one lane per slot
-    const int slot = base + lane;
-    const bool valid = slot < s_end;
+    // ---- start the copy of this tile's V codes and scales (rows up to the slab
+    // end only: S % 16 == 0, so 16 or 32 rows), overlapped with q.k below
+    {
+      const int nrow = a.S - base < 32 ? static_cast<int>(a.S - base) : 32;
+      const int64_t row0 = bh * a.S + base;
+      const uint8_t *vsrc = a.vc + row0 * CB;
+      const int cbytes = nrow * CB;
+      for (int o = lane * 16; o < cbytes; o += 32 * 16) cp_async16(vt + o, vsrc + o);
+      const uint8_t *ssrc = static_cast<const uint8_t *>(a.vs) + row0 * NGRP * (F32S ? 4 : 1);
+      const int sbytes = nrow * NGRP * (F32S ? 4 : 1);
+      for (int o = lane * 16; o < sbytes; o += 32 * 16) cp_async16(vt + 32 * CB + o, ssrc + o);
+      cp_async_commit();
+    }
+    // ---- q.k, lanes over the head dim: lane (g, sub) takes dims [16 sub, 16 sub + 16)
+    // -- inside one 32-element scale group -- of slots g + NG jj, with q in
+    // registers (four heads per pass); a butterfly reduce-scatter across the L
+    // lanes of a slot group leaves lane (g, sub) with the scores of slot g + NG sub.
+    constexpr int L = D / 16, NG = 32 / L;
+    const int g = lane / L, sub = lane % L;
+    const int own = g + NG * sub;
     float sc[kMaxG];
 #pragma unroll
     for (int h = 0; h < kMaxG; ++h) sc[h] = 0.0f;
-    if (valid) {
-      const int64_t row = bh * a.S + slot;
-      const uint8_t *kp = a.kc + row * CB;
-#pragma unroll 1
-      for (int g = 0; g < NGRP; ++g) {
-        float part[kMaxG];
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) part[h] = 0.0f;
-        constexpr int GB = Fmt<MODE>::FP4 ? 16 : 32;  // code bytes per group of 32 elements
+    for (int h0 = 0; h0 < kMaxG; h0 += 4) {
+      if (h0 >= G) break;
+      float qr[4][16];
 #pragma unroll
-        for (int c16 = 0; c16 < GB / 16; ++c16) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4 *>(kp + g * GB) + c16);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      for (int hh = 0; hh < 4; ++hh) {
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            // elements of this word: FP4: 8 (bytes carry 2 each); else 4
-            constexpr int EPW = Fmt<MODE>::FP4 ? 8 : 4;
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const float4 q4 = h0 + hh < G ? *reinterpret_cast<const float4 *>(&q_s[(h0 + hh) * D + sub * 16 + 4 * k4])
+                                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          qr[hh][4 * k4] = q4.x;
+          qr[hh][4 * k4 + 1] = q4.y;
+          qr[hh][4 * k4 + 2] = q4.z;
+          qr[hh][4 * k4 + 3] = q4.w;
+        }
+      }
+      float part[L][4];
 #pragma unroll
-            for (int pi = 0; pi < EPW / 2; ++pi) {
-              const uint32_t two = Fmt<MODE>::FP4 ? (ww[wi] >> (8 * pi)) : (ww[wi] >> (16 * pi));
-              const float2 v = decode2<MODE>(two);
-              const int d = g * 32 + c16 * (Fmt<MODE>::FP4 ? 32 : 16) + wi * EPW + 2 * pi;
+      for (int jj = 0; jj < L; ++jj) {
+        const int slot = base + g + NG * jj;
+        float pj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (slot < s_end) {
+          const int64_t row = bh * a.S + slot;
+          float v[16];
+          if constexpr (Fmt<MODE>::FP4) {  // 8 bytes, element 2i in the low nibble of byte i
+            const uint2 w = __ldg(reinterpret_cast<const uint2 *>(a.kc + row * CB + sub * 8));
 #pragma unroll
-              for (int h = 0; h < kMaxG; ++h) {
-                if (h < G) {
-                  const float2 qq = *reinterpret_cast<const float2 *>(&q_s[h * D + d]);
-                  part[h] = fmaf(qq.x, v.x, fmaf(qq.y, v.y, part[h]));
-                }
-              }
+            for (int i = 0; i < 8; ++i) {
+              const float2 t = decode2<MODE>((i < 4 ? w.x : w.y) >> (8 * (i & 3)));
+              v[2 * i] = t.x;
+              v[2 * i + 1] = t.y;
+            }
+          } else {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.kc + row * CB + sub * 16));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 t = decode2<MODE>(ww[i >> 1] >> (16 * (i & 1)));
+              v[2 * i] = t.x;
+              v[2 * i + 1] = t.y;
             }
           }
+#pragma unroll
+          for (int d = 0; d < 16; ++d)
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) pj[hh] = fmaf(qr[hh][d], v[d], pj[hh]);
+          const float gs = group_scale<MODE>(a.ks, row * NGRP + sub / 2);
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) pj[hh] *= gs;
         }
-        const float gs = group_scale<MODE>(a.ks, row * NGRP + g);
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) sc[h] = fmaf(part[h], gs, sc[h]);
+        for (int hh = 0; hh < 4; ++hh) part[jj][hh] = pj[hh];
       }
-      if (a.mask) {
-        const float madd = __ldg(a.mask + slot) * kLog2e;
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) sc[h] += madd;
+      for (int o = L / 2; o >= 1; o >>= 1) {
+        const bool upper = (sub & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j)
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const float keep = upper ? part[j + o][hh] : part[j][hh];
+            const float send = upper ? part[j][hh] : part[j + o][hh];
+            part[j][hh] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
       }
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh)
+        if (h0 + hh < kMaxG) sc[h0 + hh] = part[0][hh];
+    }
+    const int slot = base + own;
+    const bool valid = slot < s_end;
+    if (valid && a.mask) {
+      const float madd = __ldg(a.mask + slot) * kLog2e;
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) sc[h] += madd;
     }
     // ---- online softmax over the warp's 32 slots
     bool need = false;
@@ -209,18 +281,25 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
     for (int h = 0; h < kMaxG; ++h) {
       const float p = sc[h] == -INFINITY ? 0.0f : ex2(sc[h] - m[h]);
       lsum[h] += p;
-      p_s[warp][lane][h] = p;
+      p_s[warp][own][h] = p;
     }
     __syncwarp();
-    // ---- p.v, lanes over the head dim
+    // ---- p.v, lanes over the head dim, V from the staged tile
+    cp_async_wait_all();
+    __syncwarp();
     const int nval = min(32, s_end - base);
     for (int j = 0; j < nval; ++j) {
-      const int64_t row = bh * a.S + base + j;
       const int d0 = lane * DPL;
-      const float vscale = group_scale<MODE>(a.vs, row * NGRP + d0 / 32);
+      float vscale;
+      if constexpr (F32S) {
+        vscale = reinterpret_cast<const float *>(vt + 32 * CB)[j * NGRP + d0 / 32];
+      } else {
+        const int e = vt[32 * CB + j * NGRP + d0 / 32];  // 2^(e - 127), e in [0, 254]
+        vscale = e >= 1 ? __uint_as_float(static_cast<uint32_t>(e) << 23) : __uint_as_float(1u << 22);
+      }
       float val[DPL];
       if constexpr (Fmt<MODE>::FP4) {  // DPL/2 bytes
-        const uint8_t *vp = a.vc + row * CB + d0 / 2;
+        const uint8_t *vp = vt + j * CB + d0 / 2;
         uint32_t bytes;
         if constexpr (DPL == 2) bytes = vp[0];
         else if constexpr (DPL == 4) bytes = *reinterpret_cast<const uint16_t *>(vp);
@@ -232,7 +311,7 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
           val[k + 1] = v.y * vscale;
         }
       } else {
-        const uint8_t *vp = a.vc + row * CB + d0;
+        const uint8_t *vp = vt + j * CB + d0;
         uint32_t w0 = 0, w1 = 0;
         if constexpr (DPL == 2) w0 = *reinterpret_cast<const uint16_t *>(vp);
         else if constexpr (DPL == 4) w0 = *reinterpret_cast<const uint32_t *>(vp);
@@ -344,7 +423,9 @@ inline Split split_for(int B, int Hkv, int64_t S, int ctas) {
 
 template <int MODE, int D>
 int launch(const Args &a, cudaStream_t s) {
-  decode_block_kernel<MODE, D><<<dim3(a.splits, a.Hkv, a.B), kThreads, 0, s>>>(a);
+  constexpr int dyn = kWarps * VTile<MODE, D>::BYTES;
+  if (const int st = ensure_smem<BlockTag<MODE, D>>(decode_block_kernel<MODE, D>, dyn)) return st;
+  decode_block_kernel<MODE, D><<<dim3(a.splits, a.Hkv, a.B), kThreads, dyn, s>>>(a);
   if (cudaGetLastError() != cudaSuccess) return KVQ_ECUDA;
   merge_block_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
   return launch_status();
@@ -384,7 +465,7 @@ extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int
   if (S % 16 != 0 || Hq / Hkv > blk::kMaxG) return KVQ_EUNSUPPORTED;
   if (B == 0) return KVQ_OK;
   if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !kv_len || !out) return KVQ_EINVAL;
-  const void *ptrs[] = {q, k_codes, v_codes, out};
+  const void *ptrs[] = {q, k_codes, v_codes, v_scales, out};  // V codes and scales are staged by 16-byte copies
   for (const void *p : ptrs)
     if (!aligned16(p)) return KVQ_EINVAL;
   const bool f32 = mode == KVQ_MODE_FP8_E4M3 || mode == KVQ_MODE_FP8_E5M2 || mode == KVQ_MODE_INT8_SYM;
