@@ -276,8 +276,8 @@ size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S
  * workspace    device buffer of at least kvq_decode_block_workspace_bytes().
  * Launches two kernels on `stream` (the split attention, the merge).
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0 with Hq / Hkv <= 8; S % 16 == 0.
- * q, the codes, v_scales and out 16-byte aligned (V tiles are staged into
- * shared memory by 16-byte asynchronous copies); float k_scales 4-byte aligned.
+ * q, the codes, the scales and out 16-byte aligned (K and V tiles are staged
+ * into shared memory by 16-byte asynchronous copies).
  */
 int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k_codes,
                           const void *k_scales, const uint8_t *v_codes, const void *v_scales, int64_t S,

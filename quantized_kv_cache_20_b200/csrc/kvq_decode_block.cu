@@ -94,6 +94,7 @@ KVQ_DEVINL void cp_async16(void *dst_smem, const void *src) {
 }
 KVQ_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 KVQ_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+KVQ_DEVINL void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 KVQ_DEVINL float ex2(float x) {
   float y;
@@ -101,13 +102,30 @@ KVQ_DEVINL float ex2(float x) {
   return y;
 }
 
-// Bytes of one warp's staged V tile: 32 slots of codes, then their scales.
+// One warp's staged tile of 32 slots: K codes, K scales, V codes, V scales
+// (each part 16-byte aligned); NBUF tiles per warp (two for D <= 128, so the
+// next tile's copies overlap this tile's work).
 template <int MODE, int D>
 struct VTile {
   static constexpr int CB = Fmt<MODE>::FP4 ? D / 2 : D;
   static constexpr int SB = Fmt<MODE>::F32_SCALE ? 32 * (D / 32) * 4 : 32 * (D / 32);
-  static constexpr int BYTES = 32 * CB + (SB + 15) / 16 * 16;
+  static constexpr int SBP = (SB + 15) / 16 * 16;
+  static constexpr int KS = 32 * CB, VC = KS + SBP, VS = VC + 32 * CB;  // part offsets
+  static constexpr int TB = VS + SBP;                                     // one tile
+  static constexpr int NBUF = D == 256 ? 1 : 2;
+  static constexpr int BYTES = NBUF * TB;                                 // one warp
 };
+
+// The scale of entry idx of a staged scale array (float, or E8M0 2^(e - 127)).
+template <int MODE>
+KVQ_DEVINL float staged_scale(const uint8_t *p, int idx) {
+  if constexpr (Fmt<MODE>::F32_SCALE) {
+    return reinterpret_cast<const float *>(p)[idx];
+  } else {
+    const int e = p[idx];
+    return e >= 1 ? __uint_as_float(static_cast<uint32_t>(e) << 23) : __uint_as_float(1u << 22);
+  }
+}
 template <int MODE, int D>
 struct BlockTag {};  // names one decode_block_kernel instantiation for ensure_smem
 
@@ -152,21 +170,37 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
     for (int k = 0; k < DPL; ++k) acc[h][k] = 0.0f;
   }
 
-  uint8_t *vt = vt_s + warp * VTile<MODE, D>::BYTES;
-  for (int base = s_begin + warp * 32; base < s_end; base += kWarps * 32) {
-    // ---- start the copy of this tile's V codes and scales (rows up to the slab
-    // end only: S % 16 == 0, so 16 or 32 rows), overlapped with q.k below
-    {
-      const int nrow = a.S - base < 32 ? static_cast<int>(a.S - base) : 32;
-      const int64_t row0 = bh * a.S + base;
-      const uint8_t *vsrc = a.vc + row0 * CB;
-      const int cbytes = nrow * CB;
-      for (int o = lane * 16; o < cbytes; o += 32 * 16) cp_async16(vt + o, vsrc + o);
-      const uint8_t *ssrc = static_cast<const uint8_t *>(a.vs) + row0 * NGRP * (F32S ? 4 : 1);
-      const int sbytes = nrow * NGRP * (F32S ? 4 : 1);
-      for (int o = lane * 16; o < sbytes; o += 32 * 16) cp_async16(vt + 32 * CB + o, ssrc + o);
-      cp_async_commit();
+  using TL = VTile<MODE, D>;
+  uint8_t *wt = vt_s + warp * TL::BYTES;
+  // issue the copies of the tile at slot bs into dst (rows up to the slab end
+  // only: S % 16 == 0, so 16 or 32 rows)
+  auto stage = [&](int bs, uint8_t *dst) {
+    const int nrow = a.S - bs < 32 ? static_cast<int>(a.S - bs) : 32;
+    const int64_t row0 = bh * a.S + bs;
+    const int cbytes = nrow * CB, sbytes = nrow * NGRP * (F32S ? 4 : 1);
+    const int64_t soff = row0 * NGRP * (F32S ? 4 : 1);
+    for (int o = lane * 16; o < cbytes; o += 32 * 16) {
+      cp_async16(dst + o, a.kc + row0 * CB + o);
+      cp_async16(dst + TL::VC + o, a.vc + row0 * CB + o);
     }
+    for (int o = lane * 16; o < sbytes; o += 32 * 16) {
+      cp_async16(dst + TL::KS + o, static_cast<const uint8_t *>(a.ks) + soff + o);
+      cp_async16(dst + TL::VS + o, static_cast<const uint8_t *>(a.vs) + soff + o);
+    }
+    cp_async_commit();
+  };
+  int it = 0;
+  if (s_begin + warp * 32 < s_end) stage(s_begin + warp * 32, wt);
+  for (int base = s_begin + warp * 32; base < s_end; base += kWarps * 32, ++it) {
+    const uint8_t *cur = wt + (TL::NBUF == 2 ? (it & 1) * TL::TB : 0);
+    const int nb = base + kWarps * 32;
+    if (TL::NBUF == 2 && nb < s_end) {
+      stage(nb, wt + ((it + 1) & 1) * TL::TB);  // the next tile, while this one is worked on
+      cp_async_wait_one();
+    } else {
+      cp_async_wait_all();
+    }
+    __syncwarp();
     // ---- q.k, lanes over the head dim: lane (g, sub) takes dims [16 sub, 16 sub + 16)
     // -- inside one 32-element scale group -- of slots g + NG jj, with q in
     // registers (four heads per pass); a butterfly reduce-scatter across the L
@@ -199,10 +233,10 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
         const int slot = base + g + NG * jj;
         float pj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (slot < s_end) {
-          const int64_t row = bh * a.S + slot;
+          const int sl = g + NG * jj;  // slot within the tile
           float v[16];
           if constexpr (Fmt<MODE>::FP4) {  // 8 bytes, element 2i in the low nibble of byte i
-            const uint2 w = __ldg(reinterpret_cast<const uint2 *>(a.kc + row * CB + sub * 8));
+            const uint2 w = *reinterpret_cast<const uint2 *>(cur + sl * CB + sub * 8);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float2 t = decode2<MODE>((i < 4 ? w.x : w.y) >> (8 * (i & 3)));
@@ -210,7 +244,7 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
               v[2 * i + 1] = t.y;
             }
           } else {
-            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.kc + row * CB + sub * 16));
+            const uint4 w = *reinterpret_cast<const uint4 *>(cur + sl * CB + sub * 16);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -223,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
           for (int d = 0; d < 16; ++d)
 #pragma unroll
             for (int hh = 0; hh < 4; ++hh) pj[hh] = fmaf(qr[hh][d], v[d], pj[hh]);
-          const float gs = group_scale<MODE>(a.ks, row * NGRP + sub / 2);
+          const float gs = staged_scale<MODE>(cur + TL::KS, sl * NGRP + sub / 2);
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) pj[hh] *= gs;
         }
@@ -285,21 +319,13 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
     }
     __syncwarp();
     // ---- p.v, lanes over the head dim, V from the staged tile
-    cp_async_wait_all();
-    __syncwarp();
     const int nval = min(32, s_end - base);
     for (int j = 0; j < nval; ++j) {
       const int d0 = lane * DPL;
-      float vscale;
-      if constexpr (F32S) {
-        vscale = reinterpret_cast<const float *>(vt + 32 * CB)[j * NGRP + d0 / 32];
-      } else {
-        const int e = vt[32 * CB + j * NGRP + d0 / 32];  // 2^(e - 127), e in [0, 254]
-        vscale = e >= 1 ? __uint_as_float(static_cast<uint32_t>(e) << 23) : __uint_as_float(1u << 22);
-      }
+      const float vscale = staged_scale<MODE>(cur + TL::VS, j * NGRP + d0 / 32);
       float val[DPL];
       if constexpr (Fmt<MODE>::FP4) {  // DPL/2 bytes
-        const uint8_t *vp = vt + j * CB + d0 / 2;
+        const uint8_t *vp = cur + TL::VC + j * CB + d0 / 2;
         uint32_t bytes;
         if constexpr (DPL == 2) bytes = vp[0];
         else if constexpr (DPL == 4) bytes = *reinterpret_cast<const uint16_t *>(vp);
@@ -311,7 +337,7 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
           val[k + 1] = v.y * vscale;
         }
       } else {
-        const uint8_t *vp = vt + j * CB + d0;
+        const uint8_t *vp = cur + TL::VC + j * CB + d0;
         uint32_t w0 = 0, w1 = 0;
         if constexpr (DPL == 2) w0 = *reinterpret_cast<const uint16_t *>(vp);
         else if constexpr (DPL == 4) w0 = *reinterpret_cast<const uint32_t *>(vp);
@@ -337,7 +363,8 @@ __global__ void __launch_bounds__(kThreads) decode_block_kernel(const Args a) {
 #pragma unroll
           for (int k = 0; k < DPL; ++k) acc[h][k] = fmaf(pv[h], val[k], acc[h][k]);
     }
-    __syncwarp();
+    __syncwarp();  // this tile's buffer is free
+    if (TL::NBUF == 1 && base + kWarps * 32 < s_end) stage(base + kWarps * 32, wt);
   }
 
   // ---- combine the warps in order (shared running state), write this split's partial
@@ -465,7 +492,7 @@ extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int
   if (S % 16 != 0 || Hq / Hkv > blk::kMaxG) return KVQ_EUNSUPPORTED;
   if (B == 0) return KVQ_OK;
   if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !kv_len || !out) return KVQ_EINVAL;
-  const void *ptrs[] = {q, k_codes, v_codes, v_scales, out};  // V codes and scales are staged by 16-byte copies
+  const void *ptrs[] = {q, k_codes, k_scales, v_codes, v_scales, out};  // tiles are staged by 16-byte copies
   for (const void *p : ptrs)
     if (!aligned16(p)) return KVQ_EINVAL;
   const bool f32 = mode == KVQ_MODE_FP8_E4M3 || mode == KVQ_MODE_FP8_E5M2 || mode == KVQ_MODE_INT8_SYM;

@@ -467,3 +467,21 @@ def test_block_cache_decode_empty_and_out_of_range():
     b = kvq.decode_attn_block(1, q, Kc, Ks, Vc, Vs, int32_scalar(S))
     torch.cuda.synchronize()
     assert err.item() & kvq.KVQ_ERR_KV_LEN_RANGE and torch.equal(a, b)
+
+
+@pytest.mark.parametrize("mode", [1, 3])
+@pytest.mark.parametrize("D", [64, 256])
+def test_block_cache_decode_several_tiles_per_warp(mode, D):
+    """64 (b, kv head) units split about 5 ways give every warp two or three
+    32-slot tiles: the staged-tile ring (two buffers at D 64, one at D 256) is
+    reused within a split."""
+    g = wl.generator(1400 + mode + D)
+    B, Hq, Hkv, S, kv = 8, 32, 8, 4096, 3000
+    Kc, Ks = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    Vc, Vs = _block_cache_from_writer(mode, B, Hkv, S, D, kv, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    out = kvq.decode_attn_block(mode, q.to(DEV), Kc, Ks, Vc, Vs, int32_scalar(kv))
+    torch.cuda.synchronize()
+    ref = oracle.sdpa_block(mode, wl.u16(q), Kc.cpu().numpy(), Ks.cpu().numpy(), Vc.cpu().numpy(),
+                            Vs.cpu().numpy(), kv_len=kv, sm_scale=1 / math.sqrt(D))
+    assert_attn_close(bf16_to_f64(out), ref, f"block-cache decode mode {mode} D={D}, several tiles per warp")
