@@ -67,6 +67,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p kept without
 constexpr float kWScale = 79228162514264337593543950336.0f;  // 2^96
 constexpr float kOScale = 9007199254740992.0f;                // 2^53
 constexpr int kMaxCtas = 256;  // grid size limit (owner records staged per unit)
+constexpr int kMaxRows = 1024;  // per-row kv_len: batches up to this many rows are flattened by their own lengths
 
 struct DecodeArgs {
   const uint16_t *q;
@@ -123,7 +124,8 @@ struct Cfg {
   static constexpr int Q_OFF = (SH_OFF + 32 + 15) / 16 * 16;     // [2][HC] q rows: D/4 high, D/4 low words
   static constexpr int QMETA_OFF = Q_OFF + 2 * HC * 2 * D;       // [2][HC] (sum n, 2^E)
   static constexpr int RECS_OFF = QMETA_OFF + 2 * HC * 8;        // [2][kMaxCtas] owner records
-  static constexpr int SMEM = RECS_OFF + 2 * kMaxCtas * 4;
+  static constexpr int PFX_OFF = RECS_OFF + 2 * kMaxCtas * 4;    // [kMaxRows + 1] chunk prefix, [32] scratch
+  static constexpr int SMEM = PFX_OFF + (kMaxRows + 1 + 32) * 4;
   static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr int THREADS = NW * 32;
 };
@@ -254,8 +256,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   // everything read below may have been written by the kernel launched before this one
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
-  // Every unit is cut into ceil(max kv_len / 32) chunks; with per-row lengths a
-  // row's chunks past its own kv_len carry no bytes and no work.
+  // Every unit is cut into ceil(kv_len / 32) chunks.  With one kv_len per batch
+  // row (up to kMaxRows rows) the chunks are flattened by each row's own length
+  // through a prefix over the rows; above that every unit takes ceil(max
+  // kv_len / 32) chunks and a row's chunks past its own kv_len move no bytes.
   const int kv = max_kv_len(a, sh, blockIdx.x == 0);
   asm volatile("griddepcontrol.launch_dependents;");
   const int nch = (kv + CS - 1) / CS;
@@ -275,7 +279,67 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     return;
   }
   // chunk indices fit in 32 bits (the host checks U * ceil(S / 32) < 2^31)
-  const int W = static_cast<int>(U * nch);
+  const bool ragged = VARLEN && a.B <= kMaxRows;
+  const int UH = a.Hkv * a.nhc;  // units per batch row
+  int32_t *pfx = reinterpret_cast<int32_t *>(smem + C::PFX_OFF);  // pfx[b]: first chunk of row b
+  if (ragged) {  // block scan of the rows' chunk counts, rows [b0, b1) per thread
+    const int per = (a.B + C::THREADS - 1) / C::THREADS;
+    const int b0 = min(a.B, tid * per), b1 = min(a.B, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += UH * ((row_kv(a, b) + CS - 1) / CS);
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    int32_t *wsum = pfx + kMaxRows + 1;
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int off = 0;
+    for (int w = 0; w < warp; ++w) off += wsum[w];
+    int run = off + x - sum;
+    for (int b = b0; b < b1; ++b) {
+      pfx[b] = run;
+      run += UH * ((row_kv(a, b) + CS - 1) / CS);
+    }
+    if (tid == C::THREADS - 1) pfx[a.B] = off + x;
+    __syncthreads();
+  }
+  // unit u's chunks: [ustart(u), ustart(u) + ulen(u)); unit_of(chunk)
+  auto ulen = [&](int u) -> int {
+    if (!ragged) return nch;
+    const int b = u / UH;
+    return (pfx[b + 1] - pfx[b]) / UH;
+  };
+  auto ustart = [&](int u) -> int {
+    if (!ragged) return u * nch;
+    const int b = u / UH;
+    return pfx[b] + (u - b * UH) * ((pfx[b + 1] - pfx[b]) / UH);
+  };
+  auto unit_of = [&](int idx) -> int {
+    if (!ragged) return idx / nch;
+    int lo = 0, hi = a.B - 1;  // the last row b with pfx[b] <= idx has chunks
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pfx[mid] <= idx) lo = mid;
+      else hi = mid - 1;
+    }
+    return lo * UH + (idx - pfx[lo]) / ((pfx[lo + 1] - pfx[lo]) / UH);
+  };
+  if (ragged) {  // units of empty rows own no chunks: their rows are zero
+    for (int64_t u = cta; u < U; u += CT) {
+      if (ulen(static_cast<int>(u)) != 0) continue;
+      const int hc = static_cast<int>(u % a.nhc);
+      const int64_t bhk = u / a.nhc;
+      const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+      for (int e = tid; e < HC * D; e += C::THREADS) {
+        const int hq = hk * a.G + hc * HC + e / D;
+        a.out[(static_cast<int64_t>(b) * a.Hq + hq) * D + e % D] = 0;
+      }
+    }
+  }
+  const int W = ragged ? pfx[a.B] : static_cast<int>(U * nch);
   const int c_begin = static_cast<int>(range_start(cta, W, CT)), c_end = static_cast<int>(range_start(cta + 1, W, CT));
   if (c_begin >= c_end) return;  // more CTAs than chunks
 
@@ -285,8 +349,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   const int nk = c_begin + pi < c_end ? (c_end - 1 - c_begin - pi) / NP + 1 : 0;
   // lane 0 only: start the copies of the warp's chunk k (flattened index idx)
   auto issue = [&](int idx, int k) {
-    const int uu = idx / nch;
-    const int s0 = (idx - uu * nch) * CS;
+    const int uu = unit_of(idx);
+    const int s0 = (idx - ustart(uu)) * CS;
     const int64_t bhk = uu / a.nhc;  // = b * Hkv + hk
     const int kvu = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
     const int n = max(0, min(CS, kvu - s0));
@@ -309,7 +373,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   if (lane == 0 && pm == 0)
     for (int k = 0; k < min(R, nk); ++k) issue(c_begin + pi + k * NP, k);
 
-  const int u_first = c_begin / nch, u_last = (c_end - 1) / nch;  // the CTA's units
+  const int u_first = unit_of(c_begin), u_last = unit_of(c_end - 1);  // the CTA's units
   const int g = lane / L, sub = lane % L;
   const int own = g + NG * sub;  // this lane's slot within the chunk after the reduce-scatter
   float *wbuf = reinterpret_cast<float *>(smem + C::WBUF_OFF) + warp * 32 * 4;
@@ -447,8 +511,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   // when other CTAs share the unit.
   auto combine = [&](int u, const float *o_base, const float *ml_base, int p_stride, int m_stride) {
     const int64_t CTn = gridDim.x;
-    const bool alone = cta_of(static_cast<int64_t>(u) * nch, W, CTn) ==
-                       cta_of(static_cast<int64_t>(u) * nch + nch - 1, W, CTn);
+    const bool alone = cta_of(ustart(u), W, CTn) == cta_of(ustart(u) + ulen(u) - 1, W, CTn);
     const int hc = u % a.nhc;
     const int64_t bhk = u / a.nhc;
     const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
@@ -486,17 +549,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   int32_t *recs_s = reinterpret_cast<int32_t *>(smem + C::RECS_OFF);
   auto owners_of = [&](int u, int64_t &cf) {
     const int64_t CTn = gridDim.x;
-    cf = cta_of(static_cast<int64_t>(u) * nch, W, CTn);
-    const int64_t cl = cta_of(static_cast<int64_t>(u) * nch + nch - 1, W, CTn);
-    return cf == cl ? 1 : (W >= CTn ? static_cast<int>(cl - cf + 1) : nch);  // W < CTn: one chunk per CTA
+    cf = cta_of(ustart(u), W, CTn);
+    const int64_t cl = cta_of(ustart(u) + ulen(u) - 1, W, CTn);
+    return cf == cl ? 1 : (W >= CTn ? static_cast<int>(cl - cf + 1) : ulen(u));  // W < CTn: one chunk per CTA
   };
   auto stage_owners = [&](int u, int slot) {
     int64_t cf;
     const int owners = owners_of(u, cf);
     const int64_t CTn = gridDim.x;
     for (int o = tid; o < owners && owners > 1; o += C::THREADS) {
-      const int64_t c = W >= CTn ? cf + o : cta_of(static_cast<int64_t>(u) * nch + o, W, CTn);
-      recs_s[slot * kMaxCtas + o] = static_cast<int32_t>(2 * c + (u == range_start(c, W, CTn) / nch ? 0 : 1));
+      const int64_t c = W >= CTn ? cf + o : cta_of(ustart(u) + o, W, CTn);
+      recs_s[slot * kMaxCtas + o] =
+          static_cast<int32_t>(2 * c + (u == unit_of(static_cast<int>(range_start(c, W, CTn))) ? 0 : 1));
     }
     return owners;
   };
@@ -561,13 +625,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   __syncthreads();  // q slots and owner records written
   int k = 0;
   for (int u = u_first; u <= u_last; ++u) {
+    if (ragged && ulen(u) == 0) continue;  // an empty row between the CTA's first and last unit
     if (!deferred) {
       convert_q(u, 0);
       __syncthreads();  // q slot written; the previous unit's combine has read the scratch
     }
     load_q(deferred && u != u_first ? 1 : 0);
     const int kv_u = VARLEN ? row_kv(a, static_cast<int>(u / a.nhc / a.Hkv)) : kv;
-    const int seg_end = min(c_end, (u + 1) * nch);
+    const int seg_end = min(c_end, ustart(u) + ulen(u));
     for (; k < nk; ++k) {
       const int idx = c_begin + pi + k * NP;
       if (idx >= seg_end) break;
@@ -577,7 +642,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
         report(a.err, KVQ_ERR_TIMEOUT);
         sh[1] = 1;
       }
-      const int s0 = (idx - u * nch) * CS;
+      const int s0 = (idx - ustart(u)) * CS;
       if (ok && s0 < kv_u) {
         // ---- q . k on dp4a for the L slots of this lane group (slot = g + NG*jj)
         int part[L][HW];
@@ -791,7 +856,7 @@ struct Tune {
   static constexpr int CHUNK = 64 * (Q4 ? D / 2 : D) + 448;
   static constexpr int PUBW = HW * D * 4 + HW * 16;
   static constexpr int FIXED =
-      NW * 512 + NW * PUBW + NP * 8 * 12 + 64 + 4 * HC * D + 16 * HC + 8 * kMaxCtas;
+      NW * 512 + NW * PUBW + NP * 8 * 12 + 64 + 4 * HC * D + 16 * HC + 8 * kMaxCtas + 4 * (kMaxRows + 33);
   static constexpr int RMAX = (232448 - FIXED) / (NP * CHUNK);
   static constexpr int R = RMAX > 4 ? 4 : RMAX;
   static_assert(R >= 2, "ring depth");

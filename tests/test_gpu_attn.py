@@ -318,6 +318,34 @@ def test_decode_varlen_rows_match_the_oracle_per_row(D):
     assert torch.all(out[0] == 0)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_varlen_many_short_rows_with_empty_ones(D):
+    """64 rows of 0..200 slots, a fifth of them empty: CTA ranges, flattened by
+    each row's own length, span up to several rows (empty rows in between own
+    no chunks and must still come out zero)."""
+    g = wl.generator(760 + D)
+    B, Hq, Hkv, S = 64, 8, 2, 256
+    rng = torch.Generator().manual_seed(761 + D)
+    lens = torch.randint(1, 201, (B,), generator=rng)
+    lens[torch.randperm(B, generator=rng)[: B // 5]] = 0
+    lens = lens.tolist()
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hq, 1, D), g)
+    err = err_word()
+    out = kvq.decode_attn_varlen(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V],
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = bf16_to_f64(out)
+    for b in range(B):
+        if lens[b] == 0:
+            assert torch.all(out[b] == 0), f"row {b} (kv 0) is not zero"
+            continue
+        ref = oracle.sdpa(wl.u16(q[b:b + 1]), *_np(_slice(K, b)), *_np(_slice(V, b)), kv_len=lens[b],
+                          sm_scale=1 / math.sqrt(D))
+        assert_attn_close(got[b:b + 1], ref, f"varlen decode D={D} row {b} kv={lens[b]}")
+
+
 def test_decode_varlen_equal_rows_is_the_scalar_path():
     g = wl.generator(777)
     B, Hq, Hkv, D, S = 4, 16, 4, 128, 2048
