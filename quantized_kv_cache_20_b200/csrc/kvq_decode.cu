@@ -13,16 +13,19 @@
 //    chunk) x chunks of 32 slots, with the chunk count derived on the device
 //    from *kv_len -- is flattened and cut into equal contiguous ranges, one per
 //    CTA, so every SM streams the same number of bytes (to one chunk) whatever
-//    B, Hkv and kv_len are.  A CTA closes a segment whenever its range moves to
-//    the next unit.
-//  - Inside a CTA, chunk i of the range belongs to warp i mod NW.  Every warp
-//    runs its own R-deep ring of chunk buffers: lane 0 issues the 1-D bulk
-//    async copies (TMA) of a chunk's K/V codes, scales, zero points and mask
-//    into a free buffer, completion is counted on that buffer's mbarrier, and
-//    the buffer is refilled with the warp's chunk R ahead as soon as the warp
-//    has consumed it.  No producer warp and no cross-warp hand-off: a slow warp
-//    never holds back another warp's loads.  Every wait is bounded.
-//  - A lane owns 16 dims of L = D/16 slots of its warp's chunk in turn.
+//    B, Hkv and kv_len are.  With one kv_len per batch row the flattening uses
+//    each row's own length (a prefix of the rows' chunk counts in shared
+//    memory), so long rows do not pile onto a few CTAs.  A CTA closes a segment
+//    whenever its range moves to the next unit.
+//  - Inside a CTA, chunk i of the range belongs to pipeline i mod NP.  A
+//    pipeline is P warps (two when the head chunk is even: each takes half the
+//    heads, which halves its registers and lets 16 warps share an SM) around an
+//    R-deep ring of chunk buffers: the 1-D bulk async copies (TMA) of a chunk's
+//    K/V codes, scales, zero points and mask land in a free buffer, completion
+//    is counted on that buffer's mbarrier, and the warp of the pipeline that
+//    finishes a buffer last refills it with the pipeline's chunk R ahead.  No
+//    producer warp and no cross-pipeline hand-off.  Every wait is bounded.
+//  - A lane owns 16 dims of L = D/16 slots of its pipeline's chunk in turn.
 //      q.k: q is rounded once per segment onto a 16-bit fixed-point grid
 //      (n = rne(q * sm_scale * log2e / 2^E), |n| <= 32767, a power-of-two
 //      step per head), so the dot product with the int8 codes is exact integer

@@ -13,13 +13,19 @@
 // q.k, so they are applied per 32-element group in fp32):
 //  - Split-K: grid (splits, Hkv, B); a CTA takes a contiguous slot range of
 //    one (b, kv head) for all G q heads (G <= 8), 8 warps x 32 slots at a time.
-//  - q.k: one lane per slot.  Codes are decoded two at a time by the sm_100
-//    cvt.rn.f16x2.{e4m3x2, e5m2x2, e2m1x2} conversions (exact), multiplied by
-//    q read from shared memory (broadcast) in fp32, one partial per group,
-//    scaled by the group's scale.
-//  - p.v: lanes over the head dim (a coalesced V row per slot), p broadcast
-//    through shared memory; online softmax per warp in the log2 domain (the
-//    running max is raised only when a score exceeds it by more than 8).
+//  - Each warp stages its 32-slot tile (K and V codes and scales) into shared
+//    memory with 16-byte asynchronous copies (cp.async), the next tile while it
+//    works on the current one (two buffers for D <= 128, one for D = 256).
+//  - q.k: lanes over the head dim.  Lane (g, sub) takes dims [16 sub, 16 sub +
+//    16) -- inside one 32-element scale group -- of L = D/16 slots, with q in
+//    registers (four heads per pass, fp32).  Codes are decoded two at a time
+//    by the sm_100 cvt.rn.f16x2.{e4m3x2, e5m2x2, e2m1x2} conversions (exact),
+//    the lane's partial is scaled by its group's scale, and a butterfly
+//    reduce-scatter across the L lanes leaves each lane one slot's scores.
+//  - p.v: lanes over the head dim (a V row per slot from the staged tile), p
+//    broadcast through shared memory; online softmax per warp in the log2
+//    domain (the running max is raised only when a score exceeds it by more
+//    than 8).
 //  - Warps combine through shared memory; each CTA writes its (m, l, O)
 //    partial, and a merge kernel combines the splits in order.
 #include <cuda_bf16.h>
