@@ -431,20 +431,19 @@ def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
     NL = len(layers)
     steps = max(NL, min(args.steps, 2000))
     g = torch.Generator().manual_seed(7)
-    hq = torch.randn((B, Hq, 1, D), generator=g).to(torch.bfloat16).pin_memory()
-    hk = torch.randn((B, Hkv, 1, D), generator=g).to(torch.bfloat16).pin_memory()
-    hv = torch.randn((B, Hkv, 1, D), generator=g).to(torch.bfloat16).pin_memory()
+    # the step's inputs q, k, v in one pinned host buffer, copied in with one transfer
+    nq, nk = B * Hq * D, B * Hkv * D
+    hin = torch.randn((nq + 2 * nk,), generator=g).to(torch.bfloat16).pin_memory()
     hout = torch.empty((steps, B, Hq, 1, D), dtype=torch.bfloat16).pin_memory()
-    dq = torch.empty_like(hq, device=dev)
-    dk = torch.empty_like(hk, device=dev)
-    dv = torch.empty_like(hv, device=dev)
+    din = torch.empty_like(hin, device=dev)
+    dq = din[:nq].view(B, Hq, 1, D)
+    dk = din[nq:nq + nk].view(B, Hkv, 1, D)
+    dv = din[nq + nk:].view(B, Hkv, 1, D)
     dout = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=dev)
 
     def one(i):
         K, V = layers[i % NL]
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
+        din.copy_(hin, non_blocking=True)
         kvq.write_kv(0, dk, dv, sm_step, K, V)
         kvq.decode_attn(dq, *K, *V, kv_len, out=dout, workspace=ws)
         hout[i].copy_(dout, non_blocking=True)
@@ -460,10 +459,10 @@ def _e2e(args, dist, kvq, layers, ws, kv_len, sm_step):
     e1.record()
     torch.cuda.synchronize()
     ms = dist.max(e0.elapsed_time(e1) / steps)
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    h2d = hin.numel() * 2
     return {"value": dist.world * B / (ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": dout.numel() * 2, "ms_per_step": ms, "steps": steps,
-            "path": "pinned host -> device copies, kvq.write_kv + kvq.decode_attn via the Python binding "
+            "path": "pinned host -> device copy of q, k, v (one buffer), kvq.write_kv + kvq.decode_attn via the Python binding "
                     "(no graph), device -> pinned host copy of the output"}
 
 

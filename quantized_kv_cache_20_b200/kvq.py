@@ -58,6 +58,8 @@ class KvqError(RuntimeError):
 def load(path: str | None = None) -> ctypes.CDLL:
     """Load libkvq.so (once) and declare its signatures."""
     global _lib
+    if _lib is not None:  # loaded: no lock on the call path
+        return _lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -113,11 +115,19 @@ def _check(fn: str, status: int):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """A tensor's device address as a plain int (ctypes passes it as void*), or None."""
+    return None if t is None else t.data_ptr()
 
 
-def _stream(device) -> ctypes.c_void_p:
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+# The current stream's raw handle without building a Stream object (the
+# binding sits on every decode step's host path); the public call otherwise.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(device) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(device.index if device.index is not None else torch.cuda.current_device())
+    return torch.cuda.current_stream(device).cuda_stream
 
 
 def _cuda(name, t, dtype=None, contiguous=True):
