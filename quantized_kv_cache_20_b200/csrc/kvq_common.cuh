@@ -45,25 +45,8 @@ inline int sm_count() {
 }
 
 // ---------------------------------------------------------------------------
-// Global memory access
+// Error word, bf16 unpacking, device clock
 // ---------------------------------------------------------------------------
-// 16-byte streaming load that bypasses L1 (data read exactly once).
-KVQ_DEVINL uint4 ld_stream_v4(const void *p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-KVQ_DEVINL void st_v2(void *p, uint32_t a, uint32_t b) {
-  asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(a), "r"(b) : "memory");
-}
-
-KVQ_DEVINL void st_u32(void *p, uint32_t a) {
-  asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
-}
-
 KVQ_DEVINL void report(int32_t *err_word, int32_t bits) {
   if (err_word) atomicOr(err_word, bits);
 }
@@ -151,27 +134,6 @@ KVQ_DEVINL uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-
-// ---------------------------------------------------------------------------
-// int8 -> float, exact, without I2F: the byte (biased by 128) is placed in the
-// low mantissa bits of 2^23, giving 2^23 + (c + 128); subtracting the per-row
-// constant 2^23 + 128 + zp leaves exactly c - zp.
-// ---------------------------------------------------------------------------
-KVQ_DEVINL float magic_byte(uint32_t w_biased, uint32_t sel) {
-  return __uint_as_float(__byte_perm(w_biased, 0x4B000000u, sel));
-}
-// The float -(2^23 + 128 + zp) for a zero point zp in [-128, 127].
-KVQ_DEVINL float neg_magic_zp(int zp) { return __uint_as_float(0xCB000080u + static_cast<uint32_t>(zp)); }
-
-// Four int8 codes in w -> two float2 holding (c - zp) exactly; mzp2 holds
-// neg_magic_zp(zp) in both lanes.
-KVQ_DEVINL void codes4_to_f2(uint32_t w, float2 mzp2, float2 &a, float2 &b) {
-  const uint32_t wb = w ^ 0x80808080u;
-  float2 t0 = make_float2(magic_byte(wb, 0x7540u), magic_byte(wb, 0x7541u));
-  float2 t1 = make_float2(magic_byte(wb, 0x7542u), magic_byte(wb, 0x7543u));
-  a = __fadd2_rn(t0, mzp2);
-  b = __fadd2_rn(t1, mzp2);
 }
 
 }  // namespace kvq

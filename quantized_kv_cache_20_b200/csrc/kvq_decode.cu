@@ -180,15 +180,9 @@ KVQ_DEVINL int done_count(int32_t *p) {
   return old;
 }
 
-// Work split: CTA c owns flattened tiles [c*W/C, (c+1)*W/C).
+// Work split: CTA c owns flattened chunks [c*W/C, (c+1)*W/C); cta_of is its inverse.
 KVQ_DEVINL int64_t range_start(int64_t c, int64_t W, int64_t C) { return c * W / C; }
 KVQ_DEVINL int64_t cta_of(int64_t idx, int64_t W, int64_t C) { return ((idx + 1) * C - 1) / W; }
-// The CTA after c that owns a tile of [.., last], or -1: CTAs with empty ranges
-// (more CTAs than tiles) are skipped.
-KVQ_DEVINL int64_t next_owner(int64_t c, int64_t last, int64_t W, int64_t C) {
-  const int64_t e = range_start(c + 1, W, C);
-  return e > last ? -1 : cta_of(e, W, C);
-}
 
 KVQ_DEVINL bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;

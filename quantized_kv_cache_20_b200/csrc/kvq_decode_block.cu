@@ -84,15 +84,6 @@ KVQ_DEVINL float2 decode2(uint32_t two) {
   }
 }
 
-template <int MODE>
-KVQ_DEVINL float group_scale(const void *scales, int64_t idx) {
-  if constexpr (Fmt<MODE>::F32_SCALE) {
-    return __ldg(static_cast<const float *>(scales) + idx);
-  } else {
-    const int e = __ldg(static_cast<const uint8_t *>(scales) + idx);  // 2^(e - 127), e in [0, 254]
-    return e >= 1 ? __uint_as_float(static_cast<uint32_t>(e) << 23) : __uint_as_float(1u << 22);
-  }
-}
 
 // 16-byte global -> shared copy that completes asynchronously (cp.async.cg).
 KVQ_DEVINL void cp_async16(void *dst_smem, const void *src) {
