@@ -73,3 +73,24 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.kvq_write(0, 1, P(18), 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
     # empty work is a no-op
     assert lib.kvq_write(0, 1, fake, 0, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == 0
+
+
+def test_write_kv_argument_checks_reject_before_any_launch(lib):
+    """kvq_write_kv checks both tensors and the shared arguments on the host."""
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.kvq_write_kv.argtypes = [I, I, P, P, I, I, I, I, P, P, P, I64, P, P, P, P, P, P, P, P]
+    st = (ctypes.c_int64 * 4)(8, 8, 8, 1)
+    f = P(16)
+
+    def call(mode=0, k=f, v=f, D=64, B=1, ks=st, vs=st, sm=f, kc=f, ksc=f, kz=f, vc=f, vsc=f, vz=f):
+        return lib.kvq_write_kv(mode, 1, k, v, B, 1, 1, D, ks, vs, sm, 8, kc, ksc, kz, vc, vsc, vz, None, None)
+
+    assert call(mode=9) == -1                      # unknown mode
+    assert call(D=96) == -2                        # int8 affine needs D in {64, 128, 256}
+    assert call(v=None) == -1                      # null v
+    assert call(v=P(24)) == -1                     # misaligned v
+    assert call(vs=(ctypes.c_int64 * 4)(8, 8, 4, 1)) == -1   # V row stride not a multiple of 8 elements
+    assert call(vz=None) == -1                     # int8 affine needs the V zero points
+    assert call(sm=None) == -1                     # null slot_mapping
+    assert call(mode=1, ksc=P(17), kz=None, vz=None) == -1  # float scales 4-byte aligned
+    assert call(B=0) == 0                          # empty work is a no-op
