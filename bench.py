@@ -647,13 +647,12 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
     def ring():
         for K, V in layers:
             kvq.sink_plan(ring_pos, w.B, 1, 0, slot_pos, smr, kvr)
-            kvq.write(0, knr, smr, *K)
-            kvq.write(0, vnr, smr, *V)
+            kvq.write_kv(0, knr, vnr, smr, K, V)
             kvq.sink_mask(ring_pos, 1, slot_pos, maskr)
             kvq.decode_attn(qr, *K, *V, kvr, out=outr, mask=maskr, workspace=wsr)
     ms = _time_graph(stream, ring, 20) / NL
     gbytes = 2 * w.B * w.Hkv * w.S * (w.D + 5) + w.S * 4 * 2 + 2 * w.B * w.Hq * w.D * 2
-    res["ring_decode_step"] = {"what": "ring cache (sink 0, 8192 slots, wrapped): sink_plan + 2 x kvq_write + "
+    res["ring_decode_step"] = {"what": "ring cache (sink 0, 8192 slots, wrapped): sink_plan + kvq_write_kv + "
                                        "sink_mask + kvq_decode_attn over 8192 slots, batch 8, 32 q / 8 kv heads",
                                "us": ms * 1000, "tokens/s": w.B / (ms / 1000), "GB/s": gbytes / (ms / 1000) / 1e9,
                                "frac": gbytes / (ms / 1000) / 1e9 / peak, "bytes": gbytes}
