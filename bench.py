@@ -39,8 +39,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM bytes of one decode_kernel launch on the decode workload, read + write, from one ncu
-# capture of the current kernel (69,885,696 + 822,272); algorithmic bytes are 69,861,376.
-DECODE_TRAFFIC_BYTES = 70707968
+# capture of the current kernel (69,882,112 + 702,208); algorithmic bytes are 69,861,376.
+DECODE_TRAFFIC_BYTES = 70584320
 
 
 def _args():
