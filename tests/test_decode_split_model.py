@@ -1,0 +1,98 @@
+"""Host model of the decode kernel's work split, swept over many shapes.
+
+The kernel flattens (unit, 32-slot chunk) pairs, where a unit is (batch row, kv
+head, head chunk), and gives CTA c the contiguous chunks [c W / C, (c + 1) W / C).
+Two chunk layouts exist:
+  - uniform: every unit has ceil(max kv_len / 32) chunks;
+  - per-row: a unit has ceil(kv_len[b] / 32) chunks, placed through a prefix over
+    the rows.
+A split unit is merged in the kernel from one partial record per owner CTA:
+record 2 c for c's first unit and 2 c + 1 for its last.  This model restates the
+kernel's integer rules and checks the invariants the merge relies on:
+  - every chunk has exactly one owner;
+  - the owner count the kernel computes equals the number of CTAs whose range
+    meets the unit;
+  - a CTA shares at most its first and its last unit;
+  - record slots are unique per (CTA, slot).
+"""
+import random
+
+
+def range_start(c, W, C):
+    return c * W // C
+
+
+def cta_of(idx, W, C):
+    return ((idx + 1) * C - 1) // W
+
+
+def check_split(lens_per_unit, C):
+    starts, W = [], 0
+    for n in lens_per_unit:
+        starts.append(W)
+        W += n
+    if W == 0:
+        return
+
+    def unit_of(idx):  # the unit whose chunk range holds idx (units with no chunks are skipped)
+        lo, hi = 0, len(starts) - 1
+        while lo < hi:
+            mid = (lo + hi + 1) // 2
+            if starts[mid] <= idx:
+                lo = mid
+            else:
+                hi = mid - 1
+        while lens_per_unit[lo] == 0:  # several units may share a start; the one with chunks comes last
+            lo += 1
+        return lo
+
+    # every chunk is owned by the CTA whose range holds it
+    for idx in range(W):
+        c = cta_of(idx, W, C)
+        assert range_start(c, W, C) <= idx < range_start(c + 1, W, C)
+    used = set()
+    for u, n in enumerate(lens_per_unit):
+        if n == 0:
+            continue
+        s, e = starts[u], starts[u] + n - 1
+        cf, cl = cta_of(s, W, C), cta_of(e, W, C)
+        true_owners = sorted({cta_of(i, W, C) for i in range(s, e + 1)})
+        if cf == cl:
+            assert true_owners == [cf]
+            continue
+        owners = cl - cf + 1 if W >= C else n  # the kernel's count
+        assert owners == len(true_owners), (lens_per_unit, C, u)
+        listed = [cf + o if W >= C else cta_of(s + o, W, C) for o in range(owners)]
+        assert listed == true_owners
+        for c in listed:
+            first = unit_of(range_start(c, W, C))
+            last = unit_of(range_start(c + 1, W, C) - 1)
+            slot = 0 if u == first else 1
+            assert u in (first, last), "a CTA shares only its first and last unit"
+            assert (c, slot) not in used
+            used.add((c, slot))
+
+
+def test_uniform_split_invariants():
+    rng = random.Random(1)
+    for _ in range(400):
+        U = rng.randint(1, 80)
+        nch = rng.randint(1, 300)
+        C = rng.choice([1, 2, 7, 148, 256])
+        check_split([nch] * U, C)
+
+
+def test_per_row_split_invariants():
+    rng = random.Random(2)
+    for _ in range(400):
+        B = rng.randint(1, 40)
+        UH = rng.choice([1, 2, 8, 16])  # units per row (kv heads x head chunks)
+        rows = [0 if rng.random() < 0.2 else rng.randint(1, 300) for _ in range(B)]
+        C = rng.choice([1, 3, 148, 256])
+        check_split([n for n in rows for _ in range(UH)], C)
+
+
+def test_fewer_chunks_than_ctas():
+    # one chunk per CTA at most: every split unit has one owner per chunk
+    check_split([3, 1, 0, 2], 148)
+    check_split([1] * 100, 148)
