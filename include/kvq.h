@@ -169,13 +169,17 @@ int kvq_sink_mask(const int32_t *input_pos, int Lq, const int32_t *slot_pos, int
  * kvq_decode_workspace_bytes -- size of the kvq_decode_attn workspace.
  *
  * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S) on the
- * current device (the size depends on its SM count), or 0 for arguments
- * kvq_decode_attn would reject.  The workspace holds per-CTA partial results
- * and one merge counter per (batch row, kv head, head chunk).  It must be
- * zero-filled before its first use (cudaMemsetAsync); every call that
- * completes leaves the counters at zero again, so the workspace can be reused
- * by later calls in stream order without clearing (not by two calls running at
- * the same time).  After a call that set KVQ_ERR_TIMEOUT, zero it again.
+ * current device, or 0 for arguments kvq_decode_attn would reject.  The size
+ * depends only on D, the q heads per kv head and the device's SM count (not
+ * on B, Hkv or S).  Layout: the first 1 KiB holds 256 int32 merge counters,
+ * at that offset for every shape; the per-CTA partial records follow.
+ * Reuse rule: zero-fill the workspace once before its first use
+ * (cudaMemsetAsync).  Every call that completes leaves the counters at zero,
+ * and no call writes anything else into the first 1 KiB, so one workspace of
+ * at least the size each call needs serves any sequence of calls, of any
+ * shapes, ordered on streams, without clearing.  Two calls whose kernels run
+ * at the same time must not share it.  After a call that set
+ * KVQ_ERR_TIMEOUT, zero it again.
  */
 size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
 
@@ -346,13 +350,17 @@ int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D
  * above KVQ_STATIC_SCRATCH_BYTES) returns KVQ_ESCRATCH and enqueues nothing.
  * The first call on a device looks up the buffer's device address (with that
  * device current); make that first call before capturing a stream into a CUDA
- * graph.  All calls on a device share the one buffer: it starts zeroed and
- * every call that completes leaves its merge counters at zero, but two calls
- * whose kernels overlap on the GPU (different streams without ordering) race
- * on it and produce wrong results.  After a call that set KVQ_ERR_TIMEOUT,
- * kvq_decode_static_reset() clears the buffer.
+ * graph.  All calls on a device share the one buffer: it starts zeroed, every
+ * call that completes leaves its merge counters at zero, and the counters sit
+ * at the same offset for every shape, so calls of different shapes can follow
+ * one another in stream order.  Two calls whose kernels overlap on the GPU
+ * (different streams without ordering) race on it and produce wrong results.
+ * After a call that set KVQ_ERR_TIMEOUT, kvq_decode_static_reset() clears the
+ * buffer.  On a 148-SM B200 every problem with D <= 128 fits, and so does
+ * D = 256 unless the q heads per kv head are a multiple of 4: those need
+ * 1.2 MB and return KVQ_ESCRATCH.
  */
-#define KVQ_STATIC_SCRATCH_BYTES (8u << 20) /* 8 MiB per device */
+#define KVQ_STATIC_SCRATCH_BYTES (1u << 20) /* 1 MiB per device */
 int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
                            const float *k_scale, const int8_t *k_zp, const int8_t *v,
                            const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_len,

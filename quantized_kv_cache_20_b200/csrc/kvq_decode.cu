@@ -84,9 +84,9 @@ struct DecodeArgs {
   const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
   int kv_per_batch;
   uint16_t *out;
+  int32_t *ws_cnt;    // [kMaxCtas] merge counters, one per CTA: the split unit whose first owner it is
   float *ws_ml;       // [C][2][HC][2]: (m, l) of the CTA's first and last unit, when split
   float *ws_o;        // [C][2][HC][D]
-  int32_t *ws_cnt;    // [U] owners of a split unit that have written their partial
   int32_t *err;
   int64_t S;
   int B, Hq, Hkv, G, nhc;
@@ -550,9 +550,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
     const int64_t cl = cta_of(ustart(u) + ulen(u) - 1, W, CTn);
     return cf == cl ? 1 : (W >= CTn ? static_cast<int>(cl - cf + 1) : ulen(u));  // W < CTn: one chunk per CTA
   };
-  auto stage_owners = [&](int u, int slot) {
+  // returns the owner count; `first` gets the unit's first owner CTA, which names its merge counter
+  auto stage_owners = [&](int u, int slot, int &first) {
     int64_t cf;
     const int owners = owners_of(u, cf);
+    first = static_cast<int>(cf);
     const int64_t CTn = gridDim.x;
     for (int o = tid; o < owners && owners > 1; o += C::THREADS) {
       const int64_t c = W >= CTn ? cf + o : cta_of(ustart(u) + o, W, CTn);
@@ -613,8 +615,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
   const bool deferred = u_last - u_first <= 1;
   float *oscr = reinterpret_cast<float *>(smem + C::OSCR_OFF);
   constexpr int kRingStride = R * C::CHUNK / 4;  // floats from one pipeline's ring to the next
-  const int own0 = stage_owners(u_first, 0);
-  const int own1 = u_last != u_first ? stage_owners(u_last, 1) : 1;
+  int cf0 = 0, cf1 = 0;
+  const int own0 = stage_owners(u_first, 0, cf0);
+  const int own1 = u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
   if (deferred) {
     convert_q(u_first, 0);
     if (u_last != u_first) convert_q(u_last, 1);
@@ -817,14 +820,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) decode_kernel(const DecodeArgs 
 
   // Only the first and the last unit of a contiguous range can be shared with
   // other CTAs.  Count this CTA's partials of those (threads 0 and 1); the owner
-  // whose count completes a unit merges it, in owner order.
+  // whose count completes a unit merges it, in owner order.  A split unit's
+  // counter is the one of its first owner CTA: only the last unit of a CTA's
+  // range can run past it, so no two split units share a first owner, and the
+  // counters sit at the same place for every problem shape.
   if (tid < 2) {
-    const int u = tid == 0 ? u_first : u_last;
     const int owners = tid == 0 ? own0 : own1;
+    const int cf = tid == 0 ? cf0 : cf1;
     bool mine = false;
     if (owners > 1 && (tid == 0 || u_last != u_first)) {
-      if (count_acq_rel(a.ws_cnt + u) == owners - 1) {
-        a.ws_cnt[u] = 0;  // every owner has counted: ready for the next call
+      if (count_acq_rel(a.ws_cnt + cf) == owners - 1) {
+        a.ws_cnt[cf] = 0;  // every owner has counted: ready for the next call
         mine = true;
       }
     }
@@ -860,19 +866,20 @@ struct Tune {
 };
 
 struct WsLayout {
-  size_t ml, o, cnt, total;
+  size_t cnt, ml, o, total;
 };
 
-// Two partial records per CTA (its first and last unit, the only ones it can
-// share), then one merge counter per unit.
-WsLayout ws_layout(int B, int Hkv, int D, int nhc, int HC, int ctas) {
+// The merge counters first, at offset 0 for every shape (one per CTA, kMaxCtas
+// of them), then two partial records per CTA (its first and last unit, the only
+// ones it can share).  Records of any shape never land on the counters, so a
+// workspace can serve calls of different shapes one after another.
+WsLayout ws_layout(int D, int HC, int ctas) {
   WsLayout w;
-  const int64_t U = static_cast<int64_t>(B) * Hkv * nhc;
   const size_t recs = 2 * static_cast<size_t>(ctas);
-  w.ml = 0;
-  w.o = (recs * HC * 2 * 4 + 255) / 256 * 256;
-  w.cnt = w.o + (recs * HC * D * 4 + 255) / 256 * 256;
-  w.total = w.cnt + (static_cast<size_t>(U) * 4 + 255) / 256 * 256;
+  w.cnt = 0;
+  w.ml = kMaxCtas * 4;
+  w.o = w.ml + (recs * HC * 2 * 4 + 255) / 256 * 256;
+  w.total = w.o + (recs * HC * D * 4 + 255) / 256 * 256;
   return w;
 }
 
@@ -925,7 +932,7 @@ extern "C" size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int6
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S % 16 != 0) return 0;
   if (D != 64 && D != 128 && D != 256) return 0;
   const int G = Hq / Hkv, hc = head_chunk(G);
-  return ws_layout(B, Hkv, D, G / hc, hc, sm_count()).total;
+  return ws_layout(D, hc, sm_count()).total;
 }
 
 namespace kvq {
@@ -949,7 +956,7 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   const int nhc = G / hc;
   if (static_cast<int64_t>(B) * Hkv * nhc * ((S + 31) / 32) >= INT32_MAX) return KVQ_EUNSUPPORTED;
   const int ctas = sm_count();
-  const WsLayout w = ws_layout(B, Hkv, D, nhc, hc, ctas);
+  const WsLayout w = ws_layout(D, hc, ctas);
   if (ctas > kMaxCtas) return KVQ_EUNSUPPORTED;  // owner records staged per unit
   if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KVQ_EINVAL;
   DecodeArgs a;

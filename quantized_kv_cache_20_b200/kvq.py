@@ -22,7 +22,7 @@ KVQ_EINVAL = -1
 KVQ_EUNSUPPORTED = -2
 KVQ_ECUDA = -3
 KVQ_ESCRATCH = -4
-STATIC_SCRATCH_BYTES = 8 << 20
+STATIC_SCRATCH_BYTES = 1 << 20
 
 KVQ_ERR_SLOT_RANGE = 1
 KVQ_ERR_KV_LEN_RANGE = 2
@@ -130,6 +130,15 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _on_current_device(t):
+    """The library launches on the current device (its SM count, its per-device
+    state); a tensor on another device would be read from the wrong context."""
+    idx = t.device.index
+    if idx is not None and idx != torch.cuda.current_device():
+        raise ValueError(f"tensors are on cuda:{idx} but the current device is cuda:{torch.cuda.current_device()}; "
+                         "call under torch.cuda.device(...)")
+
+
 def _cuda(name, t, dtype=None, contiguous=True):
     if t is None:
         return
@@ -154,6 +163,7 @@ def write(mode: int, x: torch.Tensor, slot_mapping: torch.Tensor, codes: torch.T
     _cuda("scales", scales)
     _cuda("zero_points", zero_points)
     _cuda("err_word", err_word, torch.int32)
+    _on_current_device(x)
     B, H, T, D = x.shape
     strides = (ctypes.c_int64 * 4)(*x.stride())
     st = load().kvq_write(int(mode), int(bool(round_scale)), _ptr(x), B, H, T, D, strides,
@@ -181,6 +191,7 @@ def write_kv(mode: int, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Te
     if kc.shape[2] != vc.shape[2]:
         raise ValueError("the K and V caches must have the same number of slots")
     _cuda("err_word", err_word, torch.int32)
+    _on_current_device(k)
     B, H, T, D = k.shape
     ks_ = (ctypes.c_int64 * 4)(*k.stride())
     vs_ = (ctypes.c_int64 * 4)(*v.stride())
@@ -198,6 +209,7 @@ def sink_plan(input_pos: torch.Tensor, B: int, T: int, sink_size: int, slot_pos:
     for n, t in (("input_pos", input_pos), ("slot_pos", slot_pos), ("slot_mapping", slot_mapping),
                  ("kv_len", kv_len), ("err_word", err_word)):
         _cuda(n, t, torch.int32)
+    _on_current_device(slot_pos)
     st = load().kvq_sink_plan(_ptr(input_pos), B, T, sink_size, slot_pos.numel(), _ptr(slot_mapping),
                               _ptr(slot_pos), _ptr(kv_len), _ptr(err_word), _stream(slot_pos.device))
     _check("kvq_sink_plan", st)
@@ -208,6 +220,7 @@ def sink_mask(input_pos: torch.Tensor, Lq: int, slot_pos: torch.Tensor, mask: to
     _cuda("input_pos", input_pos, torch.int32)
     _cuda("slot_pos", slot_pos, torch.int32)
     _cuda("mask", mask, torch.float32)
+    _on_current_device(mask)
     st = load().kvq_sink_mask(_ptr(input_pos), Lq, _ptr(slot_pos), slot_pos.numel(), _ptr(mask),
                               _stream(mask.device))
     _check("kvq_sink_mask", st)
@@ -218,8 +231,9 @@ def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, S: int) -> int:
 
 
 def decode_workspace(B: int, Hq: int, Hkv: int, D: int, S: int, device) -> torch.Tensor:
-    """A zero-filled workspace of the size kvq_decode_attn needs (its merge counters
-    start at zero; each completed call leaves them at zero)."""
+    """A zero-filled workspace of the size kvq_decode_attn needs (its merge counters,
+    the first 1 KiB, start at zero; each completed call leaves them at zero, so it
+    can be reused by later calls of any shape that fit it)."""
     with torch.cuda.device(device):
         n = decode_workspace_bytes(B, Hq, Hkv, D, S)
     if n == 0:
@@ -239,6 +253,7 @@ def _attn_common(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, mask, out, err_w
     _cuda("err_word", err_word, torch.int32)
     if k.dim() != 4 or q.dim() != 4:
         raise ValueError("q must be [B, Hq, Lq, D] and k/v [B, Hkv, S, D]")
+    _on_current_device(q)
 
 
 def decode_attn(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, *, out=None, mask=None, sm_scale=None,
@@ -272,6 +287,7 @@ def decode_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len
     _cuda("kv_len", kv_len, torch.int32)
     _cuda("mask", mask, torch.float32)
     _cuda("err_word", err_word, torch.int32)
+    _on_current_device(q)
     B, Hq, Lq, D = q.shape
     Hkv, S = k_codes.shape[1], k_codes.shape[2]
     if Lq != 1:

@@ -13,7 +13,9 @@ kernel's integer rules and checks the invariants the merge relies on:
   - the owner count the kernel computes equals the number of CTAs whose range
     meets the unit;
   - a CTA shares at most its first and its last unit;
-  - record slots are unique per (CTA, slot).
+  - record slots are unique per (CTA, slot);
+  - no two split units have the same first owner CTA (the merge counter of a
+    split unit is the one of its first owner, at a shape-independent offset).
 """
 import random
 
@@ -51,6 +53,7 @@ def check_split(lens_per_unit, C):
         c = cta_of(idx, W, C)
         assert range_start(c, W, C) <= idx < range_start(c + 1, W, C)
     used = set()
+    counters = set()
     for u, n in enumerate(lens_per_unit):
         if n == 0:
             continue
@@ -62,6 +65,9 @@ def check_split(lens_per_unit, C):
             continue
         owners = cl - cf + 1 if W >= C else n  # the kernel's count
         assert owners == len(true_owners), (lens_per_unit, C, u)
+        assert cf not in counters, "two split units would share a merge counter"
+        assert 0 <= cf < C
+        counters.add(cf)
         listed = [cf + o if W >= C else cta_of(s + o, W, C) for o in range(owners)]
         assert listed == true_owners
         for c in listed:

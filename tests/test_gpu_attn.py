@@ -193,6 +193,26 @@ def test_decode_is_deterministic():
     assert torch.equal(a, b)
 
 
+def test_decode_workspace_reused_across_shapes_keeps_counters_at_zero():
+    """One caller workspace, zero-filled once, serves calls of changing D, q heads
+    per kv head and batch in stream order.  Each call is checked against the
+    oracle, and after each the merge counters (the first 1 KiB) are zero again."""
+    seq = [(2, 4, 2, 256, 2048, 2048), (3, 8, 2, 64, 2048, 1999), (2, 16, 4, 128, 1024, 1024),
+           (2, 12, 4, 128, 2048, 1537), (5, 4, 2, 64, 1024, 1000), (1, 8, 2, 256, 4096, 3000)]
+    size = max(kvq.decode_workspace_bytes(B, Hq, Hkv, D, S) for B, Hq, Hkv, D, S, _ in seq)
+    ws = torch.zeros(size, dtype=torch.uint8, device=DEV)
+    for i, (B, Hq, Hkv, D, S, n) in enumerate(seq):
+        g = wl.generator(5150 + i)
+        K, V = _cache(B, Hkv, S, D, g)
+        q = wl.bf16_normal((B, Hq, 1, D), g)
+        out = kvq.decode_attn(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V], int32_scalar(n),
+                              workspace=ws)
+        torch.cuda.synchronize()
+        ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=n, sm_scale=1 / math.sqrt(D))
+        assert_attn_close(bf16_to_f64(out), ref, f"reused workspace call {i}")
+        assert torch.count_nonzero(ws[:1024]).item() == 0, f"merge counters left set after call {i}"
+
+
 # ---------------------------------------------------------------------------- prefill
 
 def _prefill_gpu(q, K, V, kv_len, **kw):
