@@ -356,9 +356,10 @@ int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D
  * one another in stream order.  Two calls whose kernels overlap on the GPU
  * (different streams without ordering) race on it and produce wrong results.
  * After a call that set KVQ_ERR_TIMEOUT, kvq_decode_static_reset() clears the
- * buffer.  On a 148-SM B200 every problem with D <= 128 fits, and so does
- * D = 256 unless the q heads per kv head are a multiple of 4: those need
- * 1.2 MB and return KVQ_ESCRATCH.
+ * buffer.  A problem needs 1 KiB + 2 x SMs x HC x (D + 2) x 4 bytes, HC being
+ * the largest divisor of Hq / Hkv not above 8: on a 148-SM B200 every D = 64
+ * problem fits, D = 128 fits up to HC = 6 and D = 256 up to HC = 3; larger
+ * ones return KVQ_ESCRATCH.
  */
 #define KVQ_STATIC_SCRATCH_BYTES (1u << 20) /* 1 MiB per device */
 int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
@@ -373,6 +374,22 @@ int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const i
  * KVQ_ERR_TIMEOUT, which can leave merge counters behind.
  */
 int kvq_decode_static_reset(void *stream);
+
+/*
+ * kvq_set_wait_limit_ns -- bound on each main-loop wait of the decode kernels.
+ *
+ * Every wait inside the library's kernels is bounded; a wait that runs out
+ * sets KVQ_ERR_TIMEOUT in *err_word, the kernel stops issuing copies, waits
+ * (with the full 1 s bound, whatever this setting) for the copies it already
+ * issued, completes its merge bookkeeping and returns (its output is invalid;
+ * the merge counters end at zero all the same).  The default bound is 1 s;
+ * `ns` = 0 restores it.  The setting is process-wide and applies to decode
+ * kernels launched after the call (a CUDA graph keeps the value it captured).
+ * A bound below 1000 ns gives up every main-loop wait at once, without
+ * looking at the copy it waits for: that is how tests run the timeout path
+ * deterministically, without withholding any copy.  Returns KVQ_OK.
+ */
+int kvq_set_wait_limit_ns(uint64_t ns);
 
 /* A static, human-readable name for a host status code. */
 const char *kvq_strerror(int status);

@@ -72,6 +72,10 @@ KVQ_DEVINL void mbar_init(uint64_t *bar, uint32_t count) {
 
 KVQ_DEVINL void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
+// Order this thread's generic-proxy shared-memory accesses before later
+// async-proxy (bulk copy) accesses to the same bytes.
+KVQ_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 KVQ_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");

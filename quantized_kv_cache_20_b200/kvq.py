@@ -42,7 +42,7 @@ EXPORTS = (
     "kvq_write", "kvq_write_kv", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
     "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_static_reset", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
     "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
-    "kvq_strerror", "kvq_version",
+    "kvq_set_wait_limit_ns", "kvq_strerror", "kvq_version",
 )
 
 _lib = None
@@ -97,6 +97,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_prefill_attn_varlen.argtypes = lib.kvq_prefill_attn.argtypes
         lib.kvq_prefill_attn_varlen.restype = I
         lib.kvq_prefill_attn.restype = I
+        lib.kvq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.kvq_set_wait_limit_ns.restype = I
         lib.kvq_strerror.argtypes = [I]
         lib.kvq_strerror.restype = ctypes.c_char_p
         lib.kvq_version.argtypes = []

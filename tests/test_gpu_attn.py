@@ -111,8 +111,9 @@ def test_long_config_decode_full_size():
 
 
 def test_sink_config_decode_steps():
-    """4 sink + 2044 ring slots: plan -> write K/V -> mask -> decode, checked at
-    positions around the wrap; the oracle keeps its own cache and plan."""
+    """4 sink + 2044 ring slots: plan -> write K/V -> mask -> decode for positions
+    0 .. 10000, checked around the first wrap (2048), the second (4096), the
+    third (6143) and at the end (10000); the oracle keeps its own cache and plan."""
     w = wl.SINK
     g = wl.generator(w.seed)
     S, D = w.S, w.D
@@ -129,7 +130,7 @@ def test_sink_config_decode_steps():
     kv_d = torch.empty(1, dtype=torch.int32, device=DEV)
     mask_d = torch.empty((1, S), dtype=torch.float32, device=DEV)
     ws = kvq.decode_workspace(1, w.Hq, w.Hkv, D, S, DEV)
-    checks = {0, 3, 4, 5, 2047, 2048, 2049, 2300, 4095, 4096}
+    checks = {0, 3, 4, 5, 2047, 2048, 2049, 2300, 4095, 4096, 6143, 10000}
     last = max(checks)
     gen = wl.generator(w.seed + 1)
     for p in range(last + 1):
@@ -255,8 +256,9 @@ def test_prefill_tile_skip_is_bit_identical(D):
 
 
 def test_sink_config_prefill_chunks():
-    """128-token chunks through the 4 + 2044 ring, checked on chunks that span
-    positions 2048 and 4096 (masked attention, no causal flag)."""
+    """128-token chunks through the 4 + 2044 ring over positions 0 .. 10111 (79
+    chunks), checked on the chunks that span positions 2048, 4096, 6144 and 8192,
+    on an early one and on the last (masked attention, no causal flag)."""
     w = wl.SINK
     g = wl.generator(w.seed + 7)
     S, D, Lq = w.S, w.D, w.Lq
@@ -272,7 +274,7 @@ def test_sink_config_prefill_chunks():
     sm_d = torch.empty(Lq, dtype=torch.int32, device=DEV)
     kv_d = torch.empty(1, dtype=torch.int32, device=DEV)
     mask_d = torch.empty((Lq, S), dtype=torch.float32, device=DEV)
-    for c in range(33):
+    for c in range(79):
         p = c * Lq
         k = wl.bf16_normal((1, w.Hkv, Lq, D), g)
         v = wl.bf16_normal((1, w.Hkv, Lq, D), g)
@@ -283,7 +285,7 @@ def test_sink_config_prefill_chunks():
         sm_o, kv_o = oracle.sink_plan(p, 1, Lq, w.sink, S, sp_o)
         oracle.write(0, wl.u16(k), sm_o, S, *Ko)
         oracle.write(0, wl.u16(v), sm_o, S, *Vo)
-        if p <= 2048 < p + Lq or p <= 4096 < p + Lq or c == 3:
+        if any(p <= x < p + Lq for x in (2048, 4096, 6144, 8192)) or c in (3, 78):
             q = wl.bf16_normal((1, w.Hq, Lq, D), g)
             kvq.sink_mask(ip, Lq, sp_d, mask_d)
             out = kvq.prefill_attn(q.to(DEV), *Kd, *Vd, kv_d, mask=mask_d)
@@ -297,13 +299,15 @@ def test_sink_config_prefill_chunks():
 
 def test_long_config_prefill_sampled_rows():
     """Lq = 2048 causal chunk at kv_len 131072 (32 q / 16 kv heads, D=256),
-    checked on sampled rows: the first and last row of several 128-row tiles."""
+    checked on the first and the last row of every 64-row block (a CTA takes 128
+    rows = 2 q heads x 64 positions here, and the per-tile causal bound moves at
+    each block edge; the 128-row tile edges are among them), across heads."""
     w = wl.LONG
     g = wl.generator(w.seed + 200)
     K, V = _cache(w.B, w.Hkv, w.S, w.D, g)
     q = wl.bf16_normal((w.B, w.Hq, w.Lq, w.D), g)
     out = _prefill_gpu(q, K, V, w.kv_len, is_causal=True, mask_is_causal=True)
-    rows = [(0, 0, 0), (0, 1, 127), (0, 7, 128), (0, 16, 1023), (0, 30, 1920), (0, 31, 2047)]
+    rows = [(0, (5 * t + e) % w.Hq, 64 * t + 63 * e) for t in range(w.Lq // 64) for e in (0, 1)]
     ref = oracle.sdpa_rows(wl.u16(q), *_np(K), *_np(V), kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D),
                            rows=rows, is_causal=True)
     got = bf16_to_f64(out)
