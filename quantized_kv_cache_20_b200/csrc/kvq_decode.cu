@@ -732,7 +732,7 @@ struct MmaCore {
     }
     // the chunk's largest v scale (the same in every lane)
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    for (int sft = 16; sft >= 1; sft >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, sft));
     // ---- q.K: n-tile nt = slots 8 nt .. 8 nt + 7; ldmatrix x4 gives the B
     // fragments of two k-steps (64 dims) for one n-tile
     int sacc[NT][4];
