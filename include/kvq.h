@@ -306,10 +306,12 @@ int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D
  *               which enables the per-tile bound.
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; 1 <= Lq <= S.
  * Launches one kernel on `stream`: 128 query rows per CTA on the tcgen05
- * tensor cores, S = Q K^T and O += P V in bf16 with fp32 accumulation in
- * tensor memory.  K/V codes enter as the exact bf16 values (c - zp); the scales
- * are applied in fp32 (k_scale to the scores, v_scale folded into P, which
- * enters as the sum of two bf16 terms so that it keeps ~16 significant bits).
+ * tensor cores, S = Q K^T and O += P V with fp16 operands and fp32
+ * accumulation in tensor memory.  K/V codes enter as the exact fp16 values
+ * (c - zp); q enters as fp16 after one power-of-two rescale per CTA (exact for
+ * every element at least 2^-32 times the CTA's largest |q|); k_scale multiplies the fp32
+ * scores, and v_scale is folded into P = p * v_scale * 2^-E, rounded to fp16
+ * once (relative error <= 2^-11).
  */
 int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
                      const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
@@ -331,6 +333,37 @@ int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D
                             const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
                             const int8_t *v_zp, int64_t S, const int32_t *kv_lens, const float *mask, int is_causal,
                             int mask_is_causal, float sm_scale, void *out, int32_t *err_word, void *stream);
+
+/*
+ * kvq_prefill_attn_block -- Lq-query (chunked prefill) attention over a per-32
+ * block cache (kvq_write modes 1-6).
+ *
+ * Defines: the attention of kvq_prefill_attn (positions, causal rule, per-tile
+ * bound, additive mask), with K and V read from the IndexerQuantCache block
+ * format (计算公式: x ~ code * scale_g, one scale per 32 elements along the
+ * head dim), as for kvq_decode_attn_block.
+ *
+ * mode         1..6, the kvq_write mode that wrote the cache.
+ * k_codes, v_codes  u8 [B, Hkv, S, D] (mode 3: [B, Hkv, S, D/2]).
+ * k_scales, v_scales  [B, Hkv, S, D/32]: float (modes 1, 4, 6) or E8M0 bytes
+ *              (modes 2, 3, 5; 0xFF, which kvq_write never stores, gives
+ *              undefined results).
+ * q, out, kv_len, mask, is_causal, mask_is_causal, sm_scale, err_word as for
+ * kvq_prefill_attn.  No workspace.
+ * Launches one kernel on `stream`, the tcgen05 kernel of kvq_prefill_attn.  Its
+ * converters apply the scales per element: each slot's K (and V) is divided by
+ * the power of two 2^E at or above its largest group scale and rounded to fp16,
+ * and 2^E multiplies the fp32 scores (for V: folds into P).  E8M0 modes are
+ * exact except for elements below 2^-24 of their slot's largest group factor;
+ * float-scale modes round each element once (relative error <= 2^-11).
+ * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; 1 <= Lq <= S; every
+ * pointer 16-byte aligned.
+ */
+int kvq_prefill_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int Lq, int D,
+                           const uint8_t *k_codes, const void *k_scales, const uint8_t *v_codes,
+                           const void *v_scales, int64_t S, const int32_t *kv_len, const float *mask,
+                           int is_causal, int mask_is_causal, float sm_scale, void *out, int32_t *err_word,
+                           void *stream);
 
 /*
  * kvq_decode_attn_static -- kvq_decode_attn without a caller-supplied workspace.
@@ -376,15 +409,18 @@ int kvq_decode_attn_static(const void *q, int B, int Hq, int Hkv, int D, const i
 int kvq_decode_static_reset(void *stream);
 
 /*
- * kvq_set_wait_limit_ns -- bound on each main-loop wait of the decode kernels.
+ * kvq_set_wait_limit_ns -- bound on each main-loop wait of the decode kernels
+ * (kvq_decode_attn, _varlen, _tq4, _static) and the prefill kernels
+ * (kvq_prefill_attn, _varlen, _block).
  *
  * Every wait inside the library's kernels is bounded; a wait that runs out
- * sets KVQ_ERR_TIMEOUT in *err_word, the kernel stops issuing copies, waits
- * (with the full 1 s bound, whatever this setting) for the copies it already
- * issued, completes its merge bookkeeping and returns (its output is invalid;
- * the merge counters end at zero all the same).  The default bound is 1 s;
- * `ns` = 0 restores it.  The setting is process-wide and applies to decode
- * kernels launched after the call (a CUDA graph keeps the value it captured).
+ * sets KVQ_ERR_TIMEOUT in *err_word, the kernel stops issuing copies and
+ * tensor-core work, waits (with the full 1 s bound, whatever this setting) for
+ * what it already issued, completes its merge bookkeeping and returns (its
+ * output is invalid; decode merge counters end at zero all the same).  The
+ * default bound is 1 s; `ns` = 0 restores it.  The setting is process-wide and
+ * applies to kernels launched after the call (a CUDA graph keeps the value it
+ * captured).
  * A bound below 1000 ns gives up every main-loop wait at once, without
  * looking at the copy it waits for: that is how tests run the timeout path
  * deterministically, without withholding any copy.  Returns KVQ_OK.

@@ -325,6 +325,23 @@ def sdpa_dense(q_bits, K: np.ndarray, V: np.ndarray, kv_len: int, sm_scale: floa
     return out
 
 
+def sdpa_dense_rows(q_bits, K: np.ndarray, V: np.ndarray, kv_len: int, sm_scale: float, rows, mask=None,
+                    is_causal: bool = False) -> np.ndarray:
+    """``sdpa_dense`` for selected (b, h, i) rows only; returns float64 [len(rows), D]."""
+    q = _u16(q_bits)
+    K = np.ascontiguousarray(K, np.float64)
+    V = np.ascontiguousarray(V, np.float64)
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.float32)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = K.shape[1], K.shape[2]
+    out = np.zeros((len(rows), D), np.float64)
+    lib = _load()
+    for n, (b, h, i) in enumerate(rows):
+        lib.kvqo_sdpa_dense_row(_ptr(q), B, Hq, Lq, D, _ptr(K), _ptr(V), Hkv, S, int(kv_len), _ptr(m),
+                                int(bool(is_causal)), float(sm_scale), int(b), int(h), int(i), out[n].ctypes.data)
+    return out
+
+
 def sdpa_block(mode: int, q_bits, k_codes, k_scales, v_codes, v_scales, kv_len: int, sm_scale: float,
                mask=None, is_causal: bool = False) -> np.ndarray:
     """fp64 attention over a per-32 block cache: dequantize, then ``sdpa_dense``."""

@@ -106,6 +106,15 @@ KVQ_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // phase completing the wait gives up and the caller reports KVQ_ERR_TIMEOUT.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
+// Bounds below this give up every main-loop wait at once, without probing the
+// barrier: the deterministic way to run the timeout path (nothing is withheld;
+// what was issued still lands and is drained with the full bound).
+constexpr uint64_t kNoProbeBelowNs = 1000;
+
+// The bound on main-loop waits for kernels launched from now on (process-wide,
+// set by kvq_set_wait_limit_ns; kWaitLimitNs by default).
+uint64_t wait_limit_ns();
+
 KVQ_DEVINL bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();

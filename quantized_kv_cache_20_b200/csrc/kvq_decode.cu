@@ -84,10 +84,6 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p kept without
 constexpr int kMaxCtas = 256;   // grid size limit (owner records staged per unit; merge counters)
 constexpr int kMaxRows = 1024;  // per-row kv_len: batches up to this many rows are flattened by their own lengths
 
-// Bound on the main-loop waits of the decode kernels, in ns (process-wide;
-// kvq_set_wait_limit_ns changes it for kernels launched afterwards).
-std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
-
 struct DecodeArgs {
   const uint16_t *q;
   const int8_t *k;
@@ -206,11 +202,6 @@ KVQ_DEVINL bool mbar_try_wait_ns(uint64_t *bar, uint32_t parity, uint32_t hint_n
       : "memory");
   return ok != 0;
 }
-
-// Bounds below this give up every main-loop wait at once, without probing the
-// barrier: the deterministic way to run the timeout path (nothing is withheld;
-// the copies still land and are drained).
-constexpr uint64_t kNoProbeBelowNs = 1000;
 
 // Wait for a ring buffer, giving up after `limit_ns` or once another warp of
 // the CTA has given up (abort_flag).
@@ -1480,11 +1471,6 @@ extern "C" size_t kvq_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int6
   return ws_bytes(Hq / Hkv, D, sm_count());
 }
 
-extern "C" int kvq_set_wait_limit_ns(uint64_t ns) {
-  kvq::g_wait_limit_ns.store(ns == 0 ? kvq::kWaitLimitNs : ns, std::memory_order_relaxed);
-  return KVQ_OK;
-}
-
 namespace kvq {
 namespace {
 int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
@@ -1535,7 +1521,7 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   a.G = G;
   a.nhc = nhc;
   a.qscale = sm_scale * kLog2e;
-  a.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  a.wait_ns = wait_limit_ns();
   KvMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

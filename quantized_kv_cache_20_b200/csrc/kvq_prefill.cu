@@ -1,4 +1,4 @@
-// kvq_prefill.cu -- chunked-prefill attention entry point.
+// kvq_prefill.cu -- chunked-prefill attention entry points over the int8 cache.
 #include "kvq_common.cuh"
 #include "kvq_prefill_tc.cuh"
 
@@ -43,12 +43,10 @@ int prefill_impl(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int
   a.is_causal = is_causal ? 1 : 0;
   a.mask_is_causal = mask_is_causal ? 1 : 0;
   a.qscale = sm_scale * 1.4426950408889634f;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch (D) {
-    case 64: return tc::dispatch_prefill_tc<64>(a, s);
-    case 128: return tc::dispatch_prefill_tc<128>(a, s);
-    default: return tc::dispatch_prefill_tc<256>(a, s);
-  }
+  a.wait_ns = wait_limit_ns();
+  a.ks8 = nullptr;
+  a.vs8 = nullptr;
+  return tc::dispatch_prefill_mode<0>(a, D, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 

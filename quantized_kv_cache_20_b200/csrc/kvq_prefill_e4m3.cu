@@ -1,0 +1,11 @@
+// kvq_prefill_e4m3.cu -- the tcgen05 prefill kernel variants over block caches of
+// modes 1 (E4M3, float scales) and 2 (MX-FP8, E8M0 scales); one file per mode pair so the variants compile in parallel.
+#include "kvq_common.cuh"
+#include "kvq_prefill_tc.cuh"
+
+namespace kvq {
+namespace tc {
+template int dispatch_prefill_mode<KVQ_MODE_FP8_E4M3>(const PrefillArgs &, int, cudaStream_t);
+template int dispatch_prefill_mode<KVQ_MODE_MXFP8>(const PrefillArgs &, int, cudaStream_t);
+}  // namespace tc
+}  // namespace kvq

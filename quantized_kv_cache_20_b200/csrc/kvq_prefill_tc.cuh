@@ -84,7 +84,11 @@ struct PrefillArgs {
   int64_t S;
   int B, Hq, Hkv, G, Lq, nhc;  // nhc: head chunks of HPT heads per kv head
   int is_causal, mask_is_causal;
-  float qscale;  // sm_scale * log2(e)
+  float qscale;      // sm_scale * log2(e)
+  uint64_t wait_ns;  // bound on each main-loop wait
+  // block caches (kvq_write modes 1-6): codes in k / v, per-32 scales as float
+  // (ks / vs) or E8M0 bytes (ks8 / vs8); kz / vz unused
+  const uint8_t *ks8, *vs8;
 };
 
 // mbarriers.  A parity wait is only meaningful when the barrier has already
@@ -107,10 +111,14 @@ enum : int {
   kNumBars
 };
 
-template <int D_, int HPT_, bool MASK_>
+// MODE: the kvq_write mode of the cache (0: int8 affine; 1-6: per-32 block
+// formats, whose converters use the factor region FAC_OFF).
+template <int D_, int HPT_, bool MASK_, int MODE_ = 0>
 struct Cfg {
   static constexpr int D = D_, HPT = HPT_, RPH = kRows / HPT;
   static constexpr bool MASK = MASK_;
+  static constexpr int MODE = MODE_;
+  static constexpr int NG = D / 32;  // per-32 scale groups of a slot row (block modes)
   static constexpr int PPR = D / 16;                    // 16-code parts per slot row
   static constexpr int NSG = kConvThreads / PPR;        // groups of consecutive slots
   static constexpr int NCH = kTile / NSG;               // slots per group = chunks per converter thread
@@ -120,7 +128,10 @@ struct Cfg {
   static constexpr int KS_OFF = V_OFF + kTile * 2 * D;  // float [kScaleBufs][128]
   static constexpr int VS_OFF = KS_OFF + kScaleBufs * kTile * 4;
   static constexpr int VMX_OFF = VS_OFF + kScaleBufs * kTile * 4;  // float [kScaleBufs][4]
-  static constexpr int BAR_OFF = VMX_OFF + kScaleBufs * 16;
+  // block modes: float [K, V][2 tiles][kTile slots][NG] group factors scale_g * 2^-E_slot
+  static constexpr int FAC_OFF = VMX_OFF + kScaleBufs * 16;
+  static constexpr int FAC_BYTES = MODE == 0 ? 0 : 2 * 2 * kTile * NG * 4;
+  static constexpr int BAR_OFF = FAC_OFF + FAC_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag, qs, 4 x max|q|
   static constexpr int SMEM = MISC_OFF + 32 + 1024;        // + slack to align the base to 1024
   static constexpr int S_COL0 = 0, S_COL1 = kTile, O_COL = 2 * kTile;
@@ -216,14 +227,20 @@ KVQ_DEVINL bool try_wait_short(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait that also gives up once another role has raised the abort flag.
-KVQ_DEVINL bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// Bounded wait (limit_ns, the launch's main-loop bound) that also gives up once
+// another role has raised the abort flag.  A bound below kNoProbeBelowNs gives
+// up at once without probing.
+KVQ_DEVINL bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint64_t limit_ns) {
+  if (limit_ns < kNoProbeBelowNs) {
+    *abort_flag = 1;
+    return false;
+  }
   if (try_wait_short(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (try_wait_short(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       return false;
     }
@@ -305,33 +322,19 @@ struct Ctx {
 template <class C>
 __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
   constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
-  (void)HPT;
-  (void)RPH;
   uint8_t *smem = x.smem;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
   float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
   uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
-  float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
-  float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
-  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
-  (void)qs_s;
-  (void)qmax_s;
-  (void)ks_s;
-  (void)vs_s;
-  (void)vmx_s;
+  const float *ks_s = reinterpret_cast<const float *>(smem + C::KS_OFF);
+  const float *vs_s = reinterpret_cast<const float *>(smem + C::VS_OFF);
+  const float *vmx_s = reinterpret_cast<const float *>(smem + C::VMX_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)lane;
   const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
   const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
-  (void)xrow;
-  (void)hc;
-  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
-  (void)bh;
   const uint32_t tmem = x.tmem;
-  (void)tmem;
   const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
-  (void)kv;
   // ======================= softmax warpgroup: query row t
   const int t = tid;
   const int g = t / RPH;
@@ -402,7 +405,7 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     const float4 *kq4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
     const float4 *vs4 = reinterpret_cast<const float4 *>(vs_s + sb * kTile);
     const bool full = t0 + kTile - 1 <= vis_last;  // every slot of the tile visible to this row
-    ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag));
+    ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag, a.wait_ns));
     if (!ok) break;
     tc_fence_after();
     // pass 1, per 32 columns: the tile max (masked scores are written back over S)
@@ -470,7 +473,7 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     const float ao = am * ae;
     if (j > 0 && __any_sync(0xffffffffu, ao != 1.0f)) {
       // O must hold everything up to PV_{j-1} before it is rescaled
-      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag, a.wait_ns));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
@@ -527,7 +530,7 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     mbar_arrive(&bars[kBarPFull0 + buf]);
   }
   // ---- epilogue: O / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
-  if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag));
+  if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag, a.wait_ns));
   if (ok) {
     tc_fence_after();
     uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
@@ -556,34 +559,17 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
 // converter warpgroups: K (warps 4-7), V (warps 8-11)
 template <class C>
 __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
-  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
-  (void)HPT;
-  (void)RPH;
+  constexpr int D = C::D;
   uint8_t *smem = x.smem;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
-  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
-  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
+  const float *qs_s = reinterpret_cast<const float *>(smem + C::MISC_OFF + 8);  // sm_scale * log2e * 2^sh
   float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
   float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
   float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
-  (void)qs_s;
-  (void)qmax_s;
-  (void)ks_s;
-  (void)vs_s;
-  (void)vmx_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)lane;
-  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
-  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
-  (void)xrow;
-  (void)hc;
-  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
-  (void)bh;
-  const uint32_t tmem = x.tmem;
-  (void)tmem;
-  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
-  (void)kv;
+  const int64_t bh = static_cast<int64_t>(blockIdx.z) * a.Hkv + blockIdx.y / a.nhc;
+  const int loop_end = x.loop_end, ntiles = x.ntiles;
   // ======================= converter warpgroups: K (warps 4-7), V (warps 8-11)
   const bool is_k = warp < 8;
   const int c = tid - kSoftmaxThreads - (is_k ? 0 : kConvThreads);  // 0..127
@@ -667,8 +653,8 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
         vsn = c < n1 ? ld_f32(a.vs + bh * a.S + t1 + c) : 0.0f;
       }
       // the buffer is free once QK_{j-1} has run; qs is published with Q
-      ok = __all_sync(0xffffffffu, j == 0 ? wait_phase(&bars[kBarQ], 0, abort_flag)
-                                          : wait_phase(&bars[kBarKEmpty], (j - 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, j == 0 ? wait_phase(&bars[kBarQ], 0, abort_flag, a.wait_ns)
+                                          : wait_phase(&bars[kBarKEmpty], (j - 1) & 1, abort_flag, a.wait_ns));
       if (!ok) break;
       if (j == 0) qs = *qs_s;
       convert_tile(j);
@@ -688,7 +674,7 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
     for (int j = 0; j < ntiles; ++j) {
       if (j + 1 < ntiles) load_zp(zn, (j + 1) * kTile, tile_n(j + 1));
       if (j > 0) {  // the buffer is free once PV_{j-1} has run
-        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag, a.wait_ns));
         if (!ok) break;
       }
       convert_tile(j);
@@ -698,37 +684,318 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
   }
 }
 
-// MMA warp: lane 0 issues
+// ---- block caches (kvq_write modes 1-6) ---------------------------------------
+// IndexerQuantCache, 计算公式: x ~ code * scale_g with one scale per 32
+// elements along the head dim.  The scales vary along the contraction of
+// Q K^T (and along the output dim of P V), so they cannot be applied to the
+// fp32 scores as the int8 k_scale is; the converters apply them instead, per
+// element, after factoring out one power of two per slot:
+//   K'[s][d] = code * scale_g(d) * 2^-E_s  (fp16),  k factor of slot s = 2^E_s,
+// with 2^E_s the smallest power of two >= the slot's largest group scale, so
+// |K'| <= |code| (at most 57344 for E5M2, inside fp16).  V likewise with its
+// own exponent F_s, and 2^F_s takes the place of v_scale in P.  With E8M0
+// scales the group factor is a power of two and K', V' are exact unless they
+// fall below fp16's smallest subnormal (2^-24 of the slot's largest group
+// factor); with float scales (modes 1, 4, 6) each element is rounded to fp16
+// once (relative error <= 2^-11).
+template <int MODE>
+struct BlockFmt {
+  static constexpr bool FP4 = MODE == KVQ_MODE_MXFP4;
+  static constexpr bool E5 = MODE == KVQ_MODE_FP8_E5M2 || MODE == KVQ_MODE_MXFP8_E5M2;
+  static constexpr bool I8 = MODE == KVQ_MODE_INT8_SYM;
+  static constexpr bool F32S = MODE == KVQ_MODE_FP8_E4M3 || MODE == KVQ_MODE_FP8_E5M2 || I8;
+  static constexpr int PART_BYTES = FP4 ? 8 : 16;  // bytes holding 16 codes
+};
+
+// Four byte codes of a word -> two f16x2 words (code 0 in the low half), exact.
+template <int MODE>
+KVQ_DEVINL void codes4_to_f16(uint32_t w, uint32_t &h01, uint32_t &h23) {
+  using F = BlockFmt<MODE>;
+  if constexpr (F::E5) {  // an E5M2 code is the high byte of the equal fp16
+    h01 = __byte_perm(w, 0u, 0x1404);
+    h23 = __byte_perm(w, 0u, 0x3424);
+  } else if constexpr (F::I8) {  // (c + 128) in the mantissa of 1024, minus 1152
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t a = __byte_perm(u, 0x64646464u, 0x4140), b = __byte_perm(u, 0x64646464u, 0x4342);
+    const __half2 k1152 = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    const __half2 ra = __hsub2(*reinterpret_cast<const __half2 *>(&a), k1152);
+    const __half2 rb = __hsub2(*reinterpret_cast<const __half2 *>(&b), k1152);
+    h01 = *reinterpret_cast<const uint32_t *>(&ra);
+    h23 = *reinterpret_cast<const uint32_t *>(&rb);
+  } else {  // E4M3
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(static_cast<uint16_t>(w >> 16)));
+  }
+}
+
+// 16 codes of one part (16 bytes; E2M1: 8 bytes, element 2i in the low nibble
+// of byte i) -> 16 fp16 values code * f, in element order.
+template <int MODE>
+KVQ_DEVINL void block16_to_f16(const uint4 &w, float f, uint4 &lo, uint4 &hi) {
+  using F = BlockFmt<MODE>;
+  uint32_t h[8];
+  if constexpr (F::FP4) {
+    const uint32_t in[2] = {w.x, w.y};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
+          : "=r"(h[i])
+          : "r"((in[i >> 2] >> (8 * (i & 3))) & 0xFFu));
+  } else {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) codes4_to_f16<MODE>(in[i], h[2 * i], h[2 * i + 1]);
+  }
+  if constexpr (F::F32S) {  // one rounding: code * f in fp32, then to fp16
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
+      const __half2 r = __floats2half2_rn(v.x * f, v.y * f);
+      h[i] = *reinterpret_cast<const uint32_t *>(&r);
+    }
+  } else {  // f is a power of two (or 0): exact unless the result is below 2^-24
+    const __half2 ff = __float2half2_rn(f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&h[i]), ff);
+      h[i] = *reinterpret_cast<const uint32_t *>(&r);
+    }
+  }
+  lo = make_uint4(h[0], h[1], h[2], h[3]);
+  hi = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
+KVQ_DEVINL uint2 ld_codes8(const void *p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+// The NG per-32 scales of one slot as raw 32-bit words (floats, or E8M0 bytes
+// packed four per word).
+template <int MODE, int NG>
+struct ScaleRow {
+  static constexpr int W = BlockFmt<MODE>::F32S ? NG : (NG + 3) / 4;
+  uint32_t w[W];
+  KVQ_DEVINL void clear() {
+#pragma unroll
+    for (int i = 0; i < W; ++i) w[i] = 0u;
+  }
+  KVQ_DEVINL void load(const void *row) {
+    if constexpr (BlockFmt<MODE>::F32S) {
+#pragma unroll
+      for (int i = 0; i < NG; i += 2) {
+        const uint2 v = ld_codes8(static_cast<const uint32_t *>(row) + i);
+        w[i] = v.x;
+        w[i + 1] = v.y;
+      }
+    } else if constexpr (NG == 2) {
+      uint16_t h;
+      asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(row));
+      w[0] = h;
+    } else if constexpr (NG == 4) {
+      w[0] = ld_u32(row);
+    } else {
+      const uint2 v = ld_codes8(row);
+      w[0] = v.x;
+      w[1] = v.y;
+    }
+  }
+  // The slot's exponent E (2^E >= every group scale, E in [-126, 126]) and the
+  // group factors scale_g * 2^-E.
+  KVQ_DEVINL int factors(float (&f)[NG]) const {
+    if constexpr (BlockFmt<MODE>::F32S) {
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) mx = max(mx, w[g] & 0x7FFFFFFFu);
+      const int E = mx == 0u ? 0 : max(-126, min(126, ceil_log2(__uint_as_float(mx))));
+      const float inv = exp2i(-E);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) f[g] = __uint_as_float(w[g]) * inv;
+      return E;
+    } else {
+      int e[NG], mx = 0;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        e[g] = static_cast<int>((w[g >> 2] >> (8 * (g & 3))) & 0xFFu);
+        mx = max(mx, e[g]);
+      }
+      const int E = max(-126, mx - 127);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const int k = e[g] - 127 - E;  // <= 0
+        f[g] = k >= -126 ? exp2i(k) : 0.0f;
+      }
+      return E;
+    }
+  }
+};
+
+// AND of `v` over the 128 threads of one converter warpgroup (named barrier
+// `id`); also orders their shared-memory accesses like a barrier.
+KVQ_DEVINL bool group_and(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+// converter warpgroups over a block cache: K (warps 4-7), V (warps 8-11).
+// Thread c first turns the scale row of slot c into the slot's exponent and
+// group factors (shared memory, double-buffered by tile), then converts its
+// 16-code parts as the int8 converters do.
 template <class C>
-__device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
-  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
-  (void)HPT;
-  (void)RPH;
+__device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx x) {
+  constexpr int D = C::D, MODE = C::MODE, NG = C::NG;
+  using F = BlockFmt<MODE>;
+  using Row = ScaleRow<MODE, NG>;
+  constexpr int CBS = F::FP4 ? D / 2 : D;  // code bytes per slot
+  constexpr int SRB = F::F32S ? NG * 4 : NG;  // scale bytes per slot
   uint8_t *smem = x.smem;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
-  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
-  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
+  const float *qs_s = reinterpret_cast<const float *>(smem + C::MISC_OFF + 8);
   float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
   float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
   float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
-  (void)qs_s;
-  (void)qmax_s;
-  (void)ks_s;
-  (void)vs_s;
-  (void)vmx_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)lane;
-  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
-  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
-  (void)xrow;
-  (void)hc;
-  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
-  (void)bh;
+  const int64_t bh = static_cast<int64_t>(blockIdx.z) * a.Hkv + blockIdx.y / a.nhc;
+  const int loop_end = x.loop_end, ntiles = x.ntiles;
+  const bool is_k = warp < 8;
+  const int c = tid - kSoftmaxThreads - (is_k ? 0 : kConvThreads);  // 0..127
+  const int part = c % C::PPR, sg = c / C::PPR, grp = part >> 1;
+  const int blk = part >> 2, ch = (part & 3) * 2;
+  const bool swap = (c & 4) != 0;  // bank spreading of the stores, as in role_convert
+  const uint8_t *base = reinterpret_cast<const uint8_t *>(is_k ? a.k : a.v) + bh * a.S * CBS + part * F::PART_BYTES;
+  const uint8_t *own_sc =
+      F::F32S ? reinterpret_cast<const uint8_t *>(is_k ? a.ks : a.vs) : (is_k ? a.ks8 : a.vs8);
+  const uint8_t *v_sc = F::F32S ? reinterpret_cast<const uint8_t *>(a.vs) : a.vs8;
+  own_sc += bh * a.S * SRB;
+  v_sc += bh * a.S * SRB;
+  float *fac = reinterpret_cast<float *>(smem + C::FAC_OFF) + (is_k ? 0 : 2 * kTile * NG);
+  const int off = is_k ? C::K_OFF : C::V_OFF;
+  const int bar_id = is_k ? 2 : 3;
+
+  constexpr int W = C::NCH < 8 ? C::NCH : 8;
+  static_assert(C::NCH % W == 0, "window");
+  uint4 w[W];
+  auto load_chunk = [&](int r, int t0, int n) {
+    const int s = sg * C::NCH + r;
+    if (s < n) {
+      const uint8_t *p = base + static_cast<int64_t>(t0 + s) * CBS;
+      if constexpr (F::FP4) {
+        const uint2 v = ld_codes8(p);
+        w[r % W] = make_uint4(v.x, v.y, 0u, 0u);
+      } else {
+        w[r % W] = ld_codes(p);
+      }
+    } else {
+      w[r % W] = make_uint4(0u, 0u, 0u, 0u);  // code 0 is +0 in every format
+    }
+  };
+  auto tile_n = [&](int j) { return min(kTile, loop_end - j * kTile); };
+  auto convert_tile = [&](int j) {
+    const bool next = j + 1 < ntiles;
+    const int t0 = j * kTile, n0 = tile_n(j);
+    const int t1 = (j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
+    const float *fb = fac + (j & 1) * kTile * NG;
+#pragma unroll
+    for (int r = 0; r < C::NCH; ++r) {
+      const int s = sg * C::NCH + r;
+      uint4 lo, hi;
+      block16_to_f16<MODE>(w[r % W], fb[s * NG + grp], lo, hi);
+      const uint32_t o = static_cast<uint32_t>(off + blk * (kTile * 128));
+      const uint32_t a_lo = o + swz(s, ch), a_hi = o + swz(s, ch + 1);
+      *reinterpret_cast<uint4 *>(smem + (swap ? a_hi : a_lo)) = swap ? hi : lo;
+      *reinterpret_cast<uint4 *>(smem + (swap ? a_lo : a_hi)) = swap ? lo : hi;
+      if (r + W < C::NCH)
+        load_chunk(r + W, t0, n0);
+      else if (next)
+        load_chunk(r + W - C::NCH, t1, n1);
+    }
+  };
+
+  // scale rows of slot c: this tile's (cur) and the next tile's (nxt); the K
+  // converters also read the V rows, for the per-slot V factor 2^F
+  Row cur, nxt, vcur, vnxt;
+  {
+    const int n0 = tile_n(0);
+#pragma unroll
+    for (int r = 0; r < W; ++r) load_chunk(r, 0, n0);
+    cur.clear();
+    vcur.clear();
+    if (c < n0) {
+      cur.load(own_sc + static_cast<int64_t>(c) * SRB);
+      if (is_k) vcur.load(v_sc + static_cast<int64_t>(c) * SRB);
+    }
+  }
+  float qs = 0.0f;
+  bool ok = true;
+  for (int j = 0; j < ntiles; ++j) {
+    const int n = tile_n(j);
+    nxt.clear();
+    vnxt.clear();
+    if (j + 1 < ntiles && c < tile_n(j + 1)) {
+      const int64_t t = static_cast<int64_t>(j + 1) * kTile + c;
+      nxt.load(own_sc + t * SRB);
+      if (is_k) vnxt.load(v_sc + t * SRB);
+    }
+    // K: the buffer is free once QK_{j-1} has run (qs is published with Q);
+    // V: once PV_{j-1} has run
+    if (is_k)
+      ok = __all_sync(0xffffffffu, j == 0 ? wait_phase(&bars[kBarQ], 0, abort_flag, a.wait_ns)
+                                          : wait_phase(&bars[kBarKEmpty], (j - 1) & 1, abort_flag, a.wait_ns));
+    else if (j > 0)
+      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag, a.wait_ns));
+    if (ok) {
+      float f[NG];
+      const int E = cur.factors(f);
+      const bool valid = c < n;
+      float *fr = fac + ((j & 1) * kTile + c) * NG;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) fr[g] = valid ? f[g] : 0.0f;
+      if (is_k) {
+        if (j == 0) qs = *qs_s;
+        float fv[NG];
+        const int Ev = vcur.factors(fv);
+        const int sb = j % kScaleBufs;
+        const float vsv = valid ? exp2i(Ev) : 0.0f;
+        ks_s[sb * kTile + c] = valid ? exp2i(E) * qs : 0.0f;
+        vs_s[sb * kTile + c] = vsv;
+        float vm = vsv;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+        if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
+      }
+    }
+    // one decision for the warpgroup (a warp that gave up must not leave the
+    // others at the barrier), which also publishes the factors
+    ok = group_and(bar_id, ok);
+    if (!ok) break;
+    convert_tile(j);
+    proxy_fence();
+    mbar_arrive(&bars[is_k ? kBarKFull : kBarVFull]);
+    cur = nxt;
+    vcur = vnxt;
+  }
+}
+
+// MMA warp: lane 0 issues
+template <class C>
+__device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
+  constexpr int D = C::D;
+  uint8_t *smem = x.smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  const int lane = threadIdx.x & 31;
   const uint32_t tmem = x.tmem;
-  (void)tmem;
-  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
-  (void)kv;
+  const int ntiles = x.ntiles;
   // ======================= MMA warp: lane 0 issues
   if (lane == 0) {
     constexpr uint32_t ID_QK = idesc_f16(kRows, kTile, 0);
@@ -747,23 +1014,23 @@ __device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
       mma_commit(&bars[kBarSFull0 + (j & 1)]);
       mma_commit(&bars[kBarKEmpty]);
     };
-    bool ok = wait_phase(&bars[kBarQ], 0, abort_flag);
-    if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag);
+    bool ok = wait_phase(&bars[kBarQ], 0, abort_flag, a.wait_ns);
+    if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag, a.wait_ns);
     if (ok) {
       tc_fence_after();
       issue_qk(0);
     }
     for (int j = 0; j < ntiles && ok; ++j) {
       if (j + 1 < ntiles) {
-        ok = wait_phase(&bars[kBarKFull], (j + 1) & 1, abort_flag);
+        ok = wait_phase(&bars[kBarKFull], (j + 1) & 1, abort_flag, a.wait_ns);
         // S buffer (j+1)&1 holds P_{j-1} until PV_{j-1} has run
-        if (ok && j >= 1) ok = wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag);
+        if (ok && j >= 1) ok = wait_phase(&bars[kBarODone], (j - 1) & 1, abort_flag, a.wait_ns);
         if (!ok) break;
         tc_fence_after();
         issue_qk(j + 1);
       }
-      ok = wait_phase(&bars[kBarVFull], j & 1, abort_flag);
-      if (ok) ok = wait_phase(&bars[kBarPFull0 + (j & 1)], (j >> 1) & 1, abort_flag);
+      ok = wait_phase(&bars[kBarVFull], j & 1, abort_flag, a.wait_ns);
+      if (ok) ok = wait_phase(&bars[kBarPFull0 + (j & 1)], (j >> 1) & 1, abort_flag, a.wait_ns);
       if (!ok) break;
       tc_fence_after();
       const uint32_t p_tmem = tmem + ((j & 1) ? C::S_COL1 : C::S_COL0);
@@ -775,33 +1042,25 @@ __device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
       mma_commit(&bars[kBarVEmpty]);
       if (j + 1 == ntiles) mma_commit(&bars[kBarOFinal]);
     }
-    if (!ok) {  // everything issued finishes before TMEM is released
-      mma_commit(&bars[kBarDrain]);
-      mbar_wait_bounded(&bars[kBarDrain], 0);
-    }
+    // everything issued finishes before TMEM is released, on every path (after
+    // an abort the softmax may have stopped waiting for the last PV)
+    mma_commit(&bars[kBarDrain]);
+    mbar_wait_bounded(&bars[kBarDrain], 0);
   }
   __syncwarp();
 }
 
 template <class C>
 __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant__ PrefillArgs a) {
-  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
+  constexpr int RPH = C::RPH;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (the 128-byte swizzle is a function of address bits 4-9)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
-  float *qs_s = reinterpret_cast<float *>(smem + C::MISC_OFF + 8);          // sm_scale * log2e * 2^sh
-  uint32_t *qmax_s = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 12);  // per softmax warp
-  float *ks_s = reinterpret_cast<float *>(smem + C::KS_OFF);
-  float *vs_s = reinterpret_cast<float *>(smem + C::VS_OFF);
-  float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
-  const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
-  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
 
   // ---- set-up
   if (tid == 0) {
@@ -846,7 +1105,10 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
   if (warp < 4)
     role_softmax<C>(a, x);
   else if (warp < 12)
-    role_convert<C>(a, x);
+    if constexpr (C::MODE == 0)
+      role_convert<C>(a, x);
+    else
+      role_convert_block<C>(a, x);
   else
     role_mma<C>(a, x);
 
@@ -863,9 +1125,9 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
 
 inline int hpt_for(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
 
-template <int D, int HPT, bool MASK>
+template <int D, int HPT, bool MASK, int MODE>
 int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
-  using C = Cfg<D, HPT, MASK>;
+  using C = Cfg<D, HPT, MASK, MODE>;
   if (const int st = ensure_smem<C>(prefill_tc_kernel<C>, C::SMEM)) return st;
   a.nhc = a.G / HPT;
   dim3 grid((a.Lq + C::RPH - 1) / C::RPH, a.Hkv * a.nhc, a.B);
@@ -873,18 +1135,23 @@ int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   return launch_status();
 }
 
-template <int D, bool MASK>
+template <int D, bool MASK, int MODE>
 int dispatch_hpt(const PrefillArgs &a, cudaStream_t s) {
   switch (hpt_for(a.G)) {
-    case 4: return launch_prefill_tc<D, 4, MASK>(a, s);
-    case 2: return launch_prefill_tc<D, 2, MASK>(a, s);
-    default: return launch_prefill_tc<D, 1, MASK>(a, s);
+    case 4: return launch_prefill_tc<D, 4, MASK, MODE>(a, s);
+    case 2: return launch_prefill_tc<D, 2, MASK, MODE>(a, s);
+    default: return launch_prefill_tc<D, 1, MASK, MODE>(a, s);
   }
 }
 
-template <int D>
-int dispatch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
-  return a.mask ? dispatch_hpt<D, true>(a, s) : dispatch_hpt<D, false>(a, s);
+// Every (D, mask, GQA head chunk) variant of one cache mode; D is 64, 128 or 256.
+template <int MODE>
+int dispatch_prefill_mode(const PrefillArgs &a, int D, cudaStream_t s) {
+  switch (D) {
+    case 64: return a.mask ? dispatch_hpt<64, true, MODE>(a, s) : dispatch_hpt<64, false, MODE>(a, s);
+    case 128: return a.mask ? dispatch_hpt<128, true, MODE>(a, s) : dispatch_hpt<128, false, MODE>(a, s);
+    default: return a.mask ? dispatch_hpt<256, true, MODE>(a, s) : dispatch_hpt<256, false, MODE>(a, s);
+  }
 }
 
 }  // namespace tc

@@ -42,6 +42,7 @@ EXPORTS = (
     "kvq_write", "kvq_write_kv", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
     "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_static_reset", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
     "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
+    "kvq_prefill_attn_block",
     "kvq_set_wait_limit_ns", "kvq_strerror", "kvq_version",
 )
 
@@ -97,6 +98,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_prefill_attn_varlen.argtypes = lib.kvq_prefill_attn.argtypes
         lib.kvq_prefill_attn_varlen.restype = I
         lib.kvq_prefill_attn.restype = I
+        lib.kvq_prefill_attn_block.argtypes = [I, P, I, I, I, I, I, P, P, P, P, I64, P, P, I, I, F, P, P, P]
+        lib.kvq_prefill_attn_block.restype = I
         lib.kvq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.kvq_set_wait_limit_ns.restype = I
         lib.kvq_strerror.argtypes = [I]
@@ -281,11 +284,7 @@ def decode_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len
     kvq_write mode 1..6: codes uint8 [B, Hkv, S, D] (mode 3: D/2), scales [B, Hkv, S, D/32]
     (float32 for modes 1, 4, 6, E8M0 uint8 otherwise)."""
     _cuda("q", q, torch.bfloat16)
-    for n, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        _cuda(n, t, torch.uint8)
-    f32 = mode in (MODE_FP8_E4M3, MODE_FP8_E5M2, MODE_INT8_SYM)
-    for n, t in (("k_scales", k_scales), ("v_scales", v_scales)):
-        _cuda(n, t, torch.float32 if f32 else torch.uint8)
+    _block_cache_args(mode, k_codes, k_scales, v_codes, v_scales)
     _cuda("kv_len", kv_len, torch.int32)
     _cuda("mask", mask, torch.float32)
     _cuda("err_word", err_word, torch.int32)
@@ -308,6 +307,39 @@ def decode_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len
                                       float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                       _ptr(err_word), _stream(q.device))
     _check("kvq_decode_attn_block", st)
+    return out
+
+
+def _block_cache_args(mode, k_codes, k_scales, v_codes, v_scales):
+    for n, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _cuda(n, t, torch.uint8)
+    f32 = mode in (MODE_FP8_E4M3, MODE_FP8_E5M2, MODE_INT8_SYM)
+    for n, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _cuda(n, t, torch.float32 if f32 else torch.uint8)
+
+
+def prefill_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len, *, out=None, mask=None,
+                       is_causal=False, mask_is_causal=False, sm_scale=None, err_word=None) -> torch.Tensor:
+    """kvq_prefill_attn_block: q [B, Hq, Lq, D] bf16 (rows at positions kv_len - Lq + i) over a
+    per-32 block cache written by kvq_write mode 1..6 (layouts as for decode_attn_block)."""
+    _cuda("q", q, torch.bfloat16)
+    _block_cache_args(mode, k_codes, k_scales, v_codes, v_scales)
+    _cuda("kv_len", kv_len, torch.int32)
+    _cuda("mask", mask, torch.float32)
+    _cuda("err_word", err_word, torch.int32)
+    _on_current_device(q)
+    B, Hq, Lq, D = q.shape
+    Hkv, S = k_codes.shape[1], k_codes.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda("out", out, torch.bfloat16)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    st = load().kvq_prefill_attn_block(int(mode), _ptr(q), B, Hq, Hkv, Lq, D, _ptr(k_codes), _ptr(k_scales),
+                                       _ptr(v_codes), _ptr(v_scales), S, _ptr(kv_len), _ptr(mask),
+                                       int(bool(is_causal)), int(bool(mask_is_causal)), float(sm_scale), _ptr(out),
+                                       _ptr(err_word), _stream(q.device))
+    _check("kvq_prefill_attn_block", st)
     return out
 
 
