@@ -77,6 +77,8 @@ def _load():
         lib.kvqo_e8m0_value.restype = ctypes.c_double
         lib.kvqo_e8m0_ceil.argtypes = [f32]
         lib.kvqo_e8m0_ceil.restype = ctypes.c_uint8
+        lib.kvqo_e8m0_ocp.argtypes = [f32, i32]
+        lib.kvqo_e8m0_ocp.restype = ctypes.c_uint8
         lib.kvqo_affine_int8_row.argtypes = [P, i32, P, P, P]
         lib.kvqo_affine_int8_row.restype = None
         lib.kvqo_affine_int4_row.argtypes = [P, i32, P, P, P]
@@ -154,6 +156,11 @@ def e8m0_floor(s: float) -> int:
     return int(_load().kvqo_e8m0_floor(float(s)))
 
 
+def e8m0_ocp(amax: float, emax_elem: int) -> int:
+    """OCP MX v1.0 shared exponent floor(log2 amax) - emax_elem, as E8M0."""
+    return int(_load().kvqo_e8m0_ocp(float(amax), int(emax_elem)))
+
+
 # --- quantizers --------------------------------------------------------------
 
 def affine_int8_row(x_bits: np.ndarray):
@@ -183,8 +190,9 @@ def affine_int4_row(x_bits: np.ndarray):
     return q, scale[0], zp[0]
 
 
-def block_row(mode: int, x_bits: np.ndarray, round_scale: bool = True):
+def block_row(mode: int, x_bits: np.ndarray, round_scale: int = 1):
     """IndexerQuantCache, 计算公式: per-32 block quantization of one row.
+    round_scale (modes 2, 3, 5): 1 scale rounded up, 0 floor, 2 the OCP MX rule.
 
     Returns (codes uint8 [d or d/2], scales float32 [d/32] or uint8 E8M0 [d/32])."""
     x = _u16(x_bits)
@@ -192,13 +200,13 @@ def block_row(mode: int, x_bits: np.ndarray, round_scale: bool = True):
     codes = np.zeros(d // 2 if mode == MODE_MXFP4 else d, np.uint8)
     sf = np.zeros(d // 32, np.float32)
     se = np.zeros(d // 32, np.uint8)
-    _load().kvqo_block_row(mode, int(bool(round_scale)), _ptr(x), d, _ptr(codes), _ptr(sf), _ptr(se))
+    _load().kvqo_block_row(mode, int(round_scale), _ptr(x), d, _ptr(codes), _ptr(sf), _ptr(se))
     return codes, (sf if mode in _F32_SCALE_MODES else se)
 
 
 def write(mode: int, x_bits: np.ndarray, slot_mapping: np.ndarray, num_slots: int,
           codes: np.ndarray, scales: np.ndarray, zero_points: np.ndarray | None = None,
-          round_scale: bool = True) -> int:
+          round_scale: int = 1) -> int:
     """The cache write (quantize + scatter by slot_mapping, -1 = skip), in place.
 
     x_bits: uint16 [B, H, T, D] (any strides are flattened to contiguous here).
@@ -209,7 +217,7 @@ def write(mode: int, x_bits: np.ndarray, slot_mapping: np.ndarray, num_slots: in
     sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
     assert sm.size == B * T
     err = np.zeros(1, np.int32)
-    _load().kvqo_write(mode, int(bool(round_scale)), _ptr(x), B, H, T, D, _ptr(xs), _ptr(sm),
+    _load().kvqo_write(mode, int(round_scale), _ptr(x), B, H, T, D, _ptr(xs), _ptr(sm),
                        int(num_slots), _ptr(codes), _ptr(scales), _ptr(zero_points), _ptr(err))
     return int(err[0])
 

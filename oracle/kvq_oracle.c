@@ -220,6 +220,24 @@ uint8_t kvqo_e8m0_floor(float s)
     return (uint8_t)e;
 }
 
+/* The OCP MX rule (OCP Microscaling Formats v1.0, section 6.3: the shared   */
+/* exponent is floor(log2 amax) minus the element format's largest exponent, */
+/* emax 8 for E4M3, 15 for E5M2, 2 for E2M1), as an E8M0 byte clamped to     */
+/* [0, 254]; amax <= 0 gives 0.  Codes may then exceed Q_MAX and saturate.   */
+uint8_t kvqo_e8m0_ocp(float amax, int emax_elem)
+{
+    int k, e;
+    if (!(amax > 0.0f))
+        return 0;
+    (void)frexp((double)amax, &k); /* amax = f * 2^k, 0.5 <= f < 1: floor(log2 amax) = k - 1 */
+    e = (k - 1) - emax_elem + 127;
+    if (e < 0)
+        e = 0;
+    if (e > 254)
+        e = 254;
+    return (uint8_t)e;
+}
+
 /* ------------------------------------------------------------------------- */
 /* [P1] per-token-and-head affine asymmetric int8, one row of D values.      */
 /* fp32, each step rounded to nearest even, in exactly this order:           */
@@ -299,11 +317,12 @@ void kvqo_affine_int4_row(const uint16_t *x, int D, uint8_t *packed, float *scal
 /*          clamped to [-127, 127], stored as its two's-complement byte;     */
 /*          scale stored as float32.                                         */
 /*   mode 2 (MX-FP8, E4M3) / mode 5 (MX-FP8, E5M2): Q_MAX 448 / 57344; the   */
-/*          scale becomes a power of two stored as E8M0 -- rounded up with   */
-/*          round_scale (the default), else its exponent taken as it stands.*/
+/*          scale becomes a power of two stored as E8M0.                     */
 /*   mode 3 (MX-FP4): Q_MAX 6, E2M1 codes, two per byte (2i low nibble),     */
-/*          scale rounded up to 2^k, stored as E8M0 (round_scale is an       */
-/*          MX-FP8 option only).                                             */
+/*          scale a power of two stored as E8M0.                             */
+/*   The power of two for modes 2, 3, 5 follows round_scale: 1 (the default) */
+/*   rounds amax / Q_MAX up, 0 takes its exponent as it stands (floor), 2    */
+/*   takes the OCP MX rule floor(log2 amax) - emax (kvqo_e8m0_ocp).          */
 /* An all-zero group writes zero codes and a zero scale (E8M0 byte 0).       */
 /* codes: d bytes (modes 1, 2, 4, 5, 6) or d/2 bytes (mode 3);               */
 /* scale: d/32 entries.                                                      */
@@ -337,7 +356,9 @@ void kvqo_block_row(int mode, int round_scale, const uint16_t *x, int d, uint8_t
         } else if (mode == KVQO_MODE_MXFP8 || mode == KVQO_MODE_MXFP8_E5M2) {
             int e5 = (mode == KVQO_MODE_MXFP8_E5M2);
             float s = amax / (e5 ? 57344.0f : 448.0f);
-            uint8_t e = round_scale ? kvqo_e8m0_ceil(s) : kvqo_e8m0_floor(s);
+            uint8_t e = round_scale == 2 ? kvqo_e8m0_ocp(amax, e5 ? 15 : 8)
+                        : round_scale   ? kvqo_e8m0_ceil(s)
+                                        : kvqo_e8m0_floor(s);
             float scale = (float)ldexp(1.0, (int)e - 127); /* exact, possibly subnormal */
             scale_e8m0[g] = e;
             for (int i = 0; i < 32; ++i) {
@@ -345,7 +366,10 @@ void kvqo_block_row(int mode, int round_scale, const uint16_t *x, int d, uint8_t
                 codes[32 * g + i] = (amax == 0.0f) ? 0 : (e5 ? kvqo_e5m2_encode(y) : kvqo_e4m3_encode(y));
             }
         } else { /* KVQO_MODE_MXFP4 */
-            uint8_t e = kvqo_e8m0_ceil(amax / 6.0f);
+            float s = amax / 6.0f;
+            uint8_t e = round_scale == 2 ? kvqo_e8m0_ocp(amax, 2)
+                        : round_scale   ? kvqo_e8m0_ceil(s)
+                                        : kvqo_e8m0_floor(s);
             float scale = (float)ldexp(1.0, (int)e - 127);
             scale_e8m0[g] = e;
             for (int i = 0; i < 32; i += 2) {
