@@ -60,6 +60,11 @@ extern "C" {
 #define KVQ_MODE_INT8_SYM 6    /* int8 codes (two's complement in a uint8 cache), f32 scale per 32 ("Normal", UINT8) */
 #define KVQ_MODE_INT4_AFFINE 7 /* TQ4: 4-bit codes two per byte, f32 scale + zero point 0..15 per (token, head) */
 
+/* round_scale values of kvq_write (E8M0-scaled modes 2, 3, 5) */
+#define KVQ_SCALE_FLOOR 0 /* the exponent of amax / Q_MAX as it stands */
+#define KVQ_SCALE_CEIL 1  /* amax / Q_MAX rounded up to a power of two */
+#define KVQ_SCALE_OCP 2   /* OCP MX v1.0: 2^(floor(log2 amax) - emax of the element format) */
+
 /*
  * kvq_write -- quantize x and scatter it into the cache, in place.
  *
@@ -93,10 +98,14 @@ extern "C" {
  *   With B = H = 1 the block modes are the IndexerQuantCache [num_slots, d] layout.
  *   Q_MAX: 448 (E4M3), 57344 (E5M2), 6 (E2M1), 127 (mode 6: q = rne(x / scale)
  *   clamped to [-127, 127], stored as its two's-complement byte).
- * round_scale  modes 2 and 5 (MX-FP8): 1 rounds the scale amax / Q_MAX up to a
- *              power of two; 0 takes its exponent as it stands (the largest
- *              power of two not above it), codes then saturate at Q_MAX.
- *              Ignored by the other modes.
+ * round_scale  modes 2, 3 and 5 (the E8M0-scaled modes; IndexerQuantCache,
+ *              参数说明, round_scale): how the scale becomes a power of two.
+ *              KVQ_SCALE_CEIL (1, the default reading) rounds amax / Q_MAX up;
+ *              KVQ_SCALE_FLOOR (0) takes its exponent as it stands (the largest
+ *              power of two not above it); KVQ_SCALE_OCP (2) takes the OCP
+ *              Microscaling v1.0 rule 2^(floor(log2 amax) - emax), emax 8
+ *              (E4M3), 15 (E5M2), 2 (E2M1).  With FLOOR and OCP codes saturate
+ *              at Q_MAX.  Other values: KVQ_EINVAL.  Ignored by the other modes.
  * Sizes: modes 0 and 7 need D in {64, 128, 256}; the other modes need D % 32 == 0 and
  * D <= 8192 (KVQ_EUNSUPPORTED otherwise).  B, H, T >= 0 (0 enqueues nothing).
  * The arithmetic is binary32 with one round-to-nearest-even per operation, in
@@ -166,6 +175,42 @@ int kvq_sink_mask(const int32_t *input_pos, int Lq, const int32_t *slot_pos, int
                   void *stream);
 
 /*
+ * kvq_sink_plan_rows -- kvq_sink_plan for a batch whose rows sit at their own
+ * positions (a ragged sink / ring batch).
+ *
+ * Defines: ExecuTorch PR 24473, Summary (CachePositionsManagerWithSink), read
+ * per batch row: each row is its own sequence with its own position and its
+ * own cache rows, so each keeps its own slot table.  Row b's token t at
+ * position p = input_pos[b] + t goes to slot p if p < sink_size, else to
+ * sink_size + (p - sink_size) mod (S - sink_size), of row b's cache.
+ *
+ * input_pos    int32 [B] device array, the first position of each row's T tokens.
+ * slot_mapping int32 [B*T] out: the slot (within row b) of token (b, t), as
+ *              kvq_write expects for a cache [B, H, S, ...].
+ * slot_pos     int32 [B, S] in/out: per row, the position each slot holds,
+ *              -1 = empty; initialise a row to -1 when its sequence starts.
+ * kv_lens      int32 [B] out: min(input_pos[b] + T, S), for the _varlen
+ *              attention entry points.
+ * A row with input_pos[b] < 0 gets -1 slots and kv_lens[b] = 0 and sets
+ * KVQ_ERR_INPUT_POS.  Sizes and checks as for kvq_sink_plan, and B <= 65535.
+ */
+int kvq_sink_plan_rows(const int32_t *input_pos, int B, int T, int sink_size, int64_t S, int32_t *slot_mapping,
+                       int32_t *slot_pos, int32_t *kv_lens, int32_t *err_word, void *stream);
+
+/*
+ * kvq_sink_mask_rows -- kvq_sink_mask per batch row.
+ *
+ * Defines: as kvq_sink_mask (ExecuTorch PR 24473, Summary), per row: query row
+ * r of batch row b sits at input_pos[b] + r and sees slot s iff
+ * 0 <= slot_pos[b, s] <= input_pos[b] + r; mask[(b * Lq + r) * S + s] = 0.0f
+ * if visible, -INFINITY otherwise.  input_pos int32 [B], slot_pos int32 [B, S],
+ * mask float [B, Lq, S] (pass mask_batch_stride = Lq * S to the _varlen
+ * attention).  S % 4 == 0; slot_pos and mask 16-byte aligned.
+ */
+int kvq_sink_mask_rows(const int32_t *input_pos, int B, int Lq, const int32_t *slot_pos, int64_t S, float *mask,
+                       void *stream);
+
+/*
  * kvq_decode_workspace_bytes -- size of the kvq_decode_attn workspace.
  *
  * Returns the bytes the split-K decode needs for (B, Hq, Hkv, D, S) on the
@@ -230,14 +275,22 @@ int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *
  * kv_lens      int32 [B] device array: row b attends over slots [0, kv_lens[b]).
  *              Values outside [0, S] are clamped and set KVQ_ERR_KV_LEN_RANGE;
  *              a row with kv_lens[b] = 0 outputs zeros.
- * mask         nullable float [S], shared by all rows (as for kvq_decode_attn).
- * Other arguments, sizes and the workspace as for kvq_decode_attn.  The work
- * is cut as for the longest row; tiles past a row's own length move no bytes.
+ * mask         nullable float: row b adds mask[b * mask_batch_stride + s] to the
+ *              score of slot s (a ragged sink / ring batch: kvq_sink_mask_rows
+ *              with Lq = 1 writes it with stride S).
+ * mask_batch_stride  floats between two rows' masks; 0 shares one mask [S]
+ *              among all rows.  A multiple of 4 (KVQ_EINVAL otherwise); the
+ *              mask holds (B - 1) * mask_batch_stride + S floats.
+ * Other arguments, sizes and the workspace as for kvq_decode_attn.  Batches of
+ * up to 1024 rows are cut into split units by each row's own length (rows of
+ * kv_lens 0 own no work); larger batches are cut as for the longest row, and
+ * tiles past a row's own length move no bytes.
  */
 int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
                            const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
-                           int64_t S, const int32_t *kv_lens, const float *mask, float sm_scale, void *out,
-                           void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream);
+                           int64_t S, const int32_t *kv_lens, const float *mask, int64_t mask_batch_stride,
+                           float sm_scale, void *out, void *workspace, size_t workspace_bytes,
+                           int32_t *err_word, void *stream);
 
 /*
  * kvq_decode_attn_tq4 -- kvq_decode_attn over a TQ4 cache (kvq_write mode 7).
@@ -326,13 +379,19 @@ int kvq_prefill_attn(const void *q, int B, int Hq, int Hkv, int Lq, int D, const
  * kv_lens[b] - Lq + i (ExecuTorch PR 20351, commit notes, per row).
  *
  * kv_lens      int32 [B] device array, each clamped to [Lq, S]
- *              (KVQ_ERR_KV_LEN_RANGE).  mask (nullable, [Lq, S]) is shared by
- *              all rows.  Other arguments as for kvq_prefill_attn.
+ *              (KVQ_ERR_KV_LEN_RANGE).
+ * mask         nullable float: query row i of batch row b adds
+ *              mask[b * mask_batch_stride + i * S + s] to the score of slot s
+ *              (kvq_sink_mask_rows writes it with stride Lq * S).
+ * mask_batch_stride  floats between two batch rows' masks; 0 shares one mask
+ *              [Lq, S] among all rows.  A multiple of 4 (KVQ_EINVAL otherwise).
+ * Other arguments as for kvq_prefill_attn.
  */
 int kvq_prefill_attn_varlen(const void *q, int B, int Hq, int Hkv, int Lq, int D, const int8_t *k,
                             const float *k_scale, const int8_t *k_zp, const int8_t *v, const float *v_scale,
-                            const int8_t *v_zp, int64_t S, const int32_t *kv_lens, const float *mask, int is_causal,
-                            int mask_is_causal, float sm_scale, void *out, int32_t *err_word, void *stream);
+                            const int8_t *v_zp, int64_t S, const int32_t *kv_lens, const float *mask,
+                            int64_t mask_batch_stride, int is_causal, int mask_is_causal, float sm_scale, void *out,
+                            int32_t *err_word, void *stream);
 
 /*
  * kvq_prefill_attn_block -- Lq-query (chunked prefill) attention over a per-32

@@ -246,6 +246,30 @@ def sink_mask(input_pos: int, Lq: int, slot_pos: np.ndarray) -> np.ndarray:
     return mask
 
 
+def sink_plan_rows(input_pos, T: int, sink: int, S: int, slot_pos: np.ndarray):
+    """The sink plan per batch row (each row its own sequence, with its own position
+    input_pos[b] and its own slot table slot_pos[b]); updates slot_pos [B, S] in place.
+
+    Returns (slot_mapping int32 [B*T], kv_lens int32 [B])."""
+    assert slot_pos.dtype == np.int32 and slot_pos.ndim == 2 and slot_pos.shape[1] == S
+    B = slot_pos.shape[0]
+    sm = np.zeros(B * T, np.int32)
+    kv = np.zeros(B, np.int32)
+    for b in range(B):
+        if int(input_pos[b]) < 0:  # no position: nothing is written, nothing is visible
+            sm[b * T:(b + 1) * T] = -1
+            continue
+        row = np.ascontiguousarray(slot_pos[b])
+        sm[b * T:(b + 1) * T], kv[b] = sink_plan(int(input_pos[b]), 1, T, sink, S, row)
+        slot_pos[b] = row
+    return sm, kv
+
+
+def sink_mask_rows(input_pos, Lq: int, slot_pos: np.ndarray) -> np.ndarray:
+    """The sink mask per batch row: [B, Lq, S], row b from input_pos[b] and slot_pos[b]."""
+    return np.stack([sink_mask(int(input_pos[b]), Lq, slot_pos[b]) for b in range(slot_pos.shape[0])])
+
+
 # --- attention -------------------------------------------------------------------
 
 def _sdpa_common(q_bits, k, ks, kz, v, vs, vz, mask):

@@ -93,6 +93,7 @@ struct DecodeArgs {
   const float *vs;
   const int8_t *vz;
   const float *mask;
+  int64_t mask_bstride;   // floats between batch rows' masks (0: one mask for every row)
   const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
   int kv_per_batch;
   uint16_t *out;
@@ -992,6 +993,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // unit's chunk range, first code row (b * Hkv + hk) * S and kv_len.
   int ik = 0, iu = u_first - 1, iustart = 0, iuend = 0, ikv = kv;
   int64_t ibase = 0;
+  const float *imask = a.mask;  // the unit's batch row of the mask
   const uint64_t pol = policy_evict_first();
   uint32_t outstanding = 0, outpar = 0;  // ring buffers with copies in flight, and their phases (lane 0)
   auto issue = [&](int kk) {
@@ -1005,6 +1007,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int64_t bhk = iu / a.nhc;  // = b * Hkv + hk
       ibase = bhk * a.S;
       ikv = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
+      if (a.mask) imask = a.mask + (bhk / a.Hkv) * a.mask_bstride;
     }
     const int s0 = (idx - iustart) * CS;
     const int kvu = ikv;
@@ -1032,7 +1035,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       bulk_g2s(small + C::VS_OFF, a.vs + row, n16 * 4, bar);
       bulk_g2s(small + C::KZ_OFF, a.kz + row, n16, bar);
       bulk_g2s(small + C::VZ_OFF, a.vz + row, n16, bar);
-      if (a.mask) bulk_g2s(small + C::M_OFF, a.mask + s0, n16 * 4, bar);
+      if (a.mask) bulk_g2s(small + C::M_OFF, imask + s0, n16 * 4, bar);
     }
     outstanding |= 1u << rb;
     outpar = (outpar & ~(1u << rb)) | ((static_cast<uint32_t>(kk / R) & 1u) << rb);
@@ -1475,8 +1478,9 @@ namespace kvq {
 namespace {
 int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
                 const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp, int64_t S,
-                const int32_t *kv_len, int kv_per_batch, bool q4, const float *mask, float sm_scale, void *out,
-                void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
+                const int32_t *kv_len, int kv_per_batch, bool q4, const float *mask, int64_t mask_bstride,
+                float sm_scale, void *out, void *workspace, size_t workspace_bytes, int32_t *err_word,
+                void *stream) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S > INT32_MAX) return KVQ_EINVAL;
   if (D != 64 && D != 128 && D != 256) return KVQ_EUNSUPPORTED;
   if (S % 16 != 0) return KVQ_EUNSUPPORTED;
@@ -1486,6 +1490,7 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   for (const void *p : ptrs)
     if (!aligned16(p)) return KVQ_EINVAL;
   if (mask && !aligned16(mask)) return KVQ_EINVAL;
+  if (mask_bstride < 0 || mask_bstride % 4 != 0) return KVQ_EINVAL;  // keeps every row's mask 16-byte aligned
   if (!(sm_scale == sm_scale)) return KVQ_EINVAL;
   const int G = Hq / Hkv;
   const int hc = q4 ? head_chunk_simt(G) : head_chunk_mma(G);
@@ -1506,6 +1511,7 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   a.vs = v_scale;
   a.vz = v_zp;
   a.mask = mask;
+  a.mask_bstride = mask_bstride;
   a.kv_len = kv_len;
   a.kv_per_batch = kv_per_batch;
   a.out = static_cast<uint16_t *>(out);
@@ -1549,8 +1555,8 @@ extern "C" int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, con
                                const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
                                int64_t S, const int32_t *kv_len, const float *mask, float sm_scale, void *out,
                                void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
-  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, false, mask, sm_scale,
-                          out, workspace, workspace_bytes, err_word, stream);
+  return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_len, 0, false, mask, 0,
+                          sm_scale, out, workspace, workspace_bytes, err_word, stream);
 }
 
 extern "C" int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k,
@@ -1560,17 +1566,17 @@ extern "C" int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D,
                                    int32_t *err_word, void *stream) {
   return kvq::decode_impl(q, B, Hq, Hkv, D, reinterpret_cast<const int8_t *>(k), k_scale,
                           reinterpret_cast<const int8_t *>(k_zp), reinterpret_cast<const int8_t *>(v), v_scale,
-                          reinterpret_cast<const int8_t *>(v_zp), S, kv_len, 0, true, mask, sm_scale, out, workspace,
-                          workspace_bytes, err_word, stream);
+                          reinterpret_cast<const int8_t *>(v_zp), S, kv_len, 0, true, mask, 0, sm_scale, out,
+                          workspace, workspace_bytes, err_word, stream);
 }
 
 extern "C" int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k,
                                       const float *k_scale, const int8_t *k_zp, const int8_t *v,
                                       const float *v_scale, const int8_t *v_zp, int64_t S, const int32_t *kv_lens,
-                                      const float *mask, float sm_scale, void *out, void *workspace,
-                                      size_t workspace_bytes, int32_t *err_word, void *stream) {
+                                      const float *mask, int64_t mask_batch_stride, float sm_scale, void *out,
+                                      void *workspace, size_t workspace_bytes, int32_t *err_word, void *stream) {
   return kvq::decode_impl(q, B, Hq, Hkv, D, k, k_scale, k_zp, v, v_scale, v_zp, S, kv_lens, 1, false, mask,
-                          sm_scale, out, workspace, workspace_bytes, err_word, stream);
+                          mask_batch_stride, sm_scale, out, workspace, workspace_bytes, err_word, stream);
 }
 
 // ----------------------------------------------------------------------------

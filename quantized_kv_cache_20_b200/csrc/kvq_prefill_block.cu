@@ -48,6 +48,7 @@ extern "C" int kvq_prefill_attn_block(int mode, const void *q, int B, int Hq, in
   a.kz = nullptr;
   a.vz = nullptr;
   a.mask = mask;
+  a.mask_bstride = 0;
   a.kv_len = kv_len;
   a.kv_per_batch = 0;
   a.out = static_cast<uint16_t *>(out);

@@ -77,6 +77,7 @@ struct PrefillArgs {
   const float *vs;
   const int8_t *vz;
   const float *mask;
+  int64_t mask_bstride;   // floats between batch rows' masks (0: one mask for every row)
   const int32_t *kv_len;  // one device scalar, or [B] with kv_per_batch
   int kv_per_batch;
   uint16_t *out;
@@ -422,7 +423,7 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
           const float4 kk = kq4[c * 8 + q4];
           float4 mv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
           if (row_ok && j0 < loop_end)  // in bounds: loop_end <= S, S % 4 == 0
-            mv = *reinterpret_cast<const float4 *>(a.mask + static_cast<int64_t>(pos) * a.S + j0);
+            mv = *reinterpret_cast<const float4 *>(a.mask + b * a.mask_bstride + static_cast<int64_t>(pos) * a.S + j0);
           const float kf[4] = {kk.x, kk.y, kk.z, kk.w}, mf[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {

@@ -57,7 +57,7 @@ struct WriteArgs {
   int64_t S;
   int32_t *err;
   uint32_t groups;  // groups of one tensor
-  int round_scale;  // MX-FP8 modes: 1 = scale rounded up to a power of two, 0 = its exponent as it stands
+  int round_scale;  // MX modes: KVQ_SCALE_CEIL, KVQ_SCALE_FLOOR or KVQ_SCALE_OCP
 };
 
 constexpr int kThreads = 256;
@@ -119,6 +119,17 @@ KVQ_DEVINL int e8m0_floor(float s) {
   const int E = static_cast<int>(u >> 23);
   if (E == 0) return 0;  // subnormal: below 2^-126, clamped
   return E > 254 ? 254 : E;  // floor(log2 s) + 127 is the biased exponent field
+}
+
+// The OCP MX v1.0 shared exponent floor(log2 amax) - emax + 127 for a finite
+// amax >= 0, clamped to [0, 254]; amax == 0 gives 0.
+KVQ_DEVINL int e8m0_ocp(float amax, int emax) {
+  const uint32_t u = __float_as_uint(amax);
+  if (u == 0) return 0;
+  const int E = static_cast<int>(u >> 23);
+  const int l = E > 0 ? E - 127 : (31 - __clz(static_cast<int>(u & 0x7FFFFFu))) - 149;  // floor(log2 amax)
+  const int e = l - emax + 127;
+  return e < 0 ? 0 : (e > 254 ? 254 : e);
 }
 
 // 2^(127 - e) as a binary32 (exact for e in [0, 254]; e = 254 is subnormal).
@@ -339,8 +350,11 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
         constexpr bool MX8 = MODE == KVQ_MODE_MXFP8 || MODE == KVQ_MODE_MXFP8_E5M2;
         constexpr bool E5 = MODE == KVQ_MODE_MXFP8_E5M2;
         constexpr float kQmax = MX8 ? (E5 ? 57344.0f : 448.0f) : 6.0f;
+        constexpr int kEmax = MX8 ? (E5 ? 15 : 8) : 2;  // the element format's largest exponent
         const float s_ = __fdiv_rn(amax, kQmax);
-        const int e = (MX8 && !a.round_scale) ? e8m0_floor(s_) : e8m0_ceil(s_);
+        const int e = a.round_scale == KVQ_SCALE_OCP    ? e8m0_ocp(amax, kEmax)
+                      : a.round_scale == KVQ_SCALE_CEIL ? e8m0_ceil(s_)
+                                                        : e8m0_floor(s_);
         const float inv = e8m0_inverse(e);  // x / 2^(e-127) == x * 2^(127-e), exactly rounded
         float y[32];
 #pragma unroll
@@ -453,7 +467,8 @@ int write_impl(int mode, int round_scale, int B, int H, int T, int D, const int3
   a.S = num_slots;
   a.err = err_word;
   a.groups = static_cast<uint32_t>(groups);
-  a.round_scale = round_scale ? 1 : 0;
+  if (round_scale < KVQ_SCALE_FLOOR || round_scale > KVQ_SCALE_OCP) return KVQ_EINVAL;
+  a.round_scale = round_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (mode) {
     case KVQ_MODE_INT8_AFFINE: return launch_write<KVQ_MODE_INT8_AFFINE>(a, s);

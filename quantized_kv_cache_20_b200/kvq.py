@@ -38,8 +38,13 @@ MODE_MXFP8_E5M2 = 5
 MODE_INT8_SYM = 6
 MODE_INT4_AFFINE = 7
 
+SCALE_FLOOR = 0  # round_scale values for the E8M0-scaled modes 2, 3, 5
+SCALE_CEIL = 1
+SCALE_OCP = 2
+
 EXPORTS = (
-    "kvq_write", "kvq_write_kv", "kvq_sink_plan", "kvq_sink_mask", "kvq_decode_workspace_bytes",
+    "kvq_write", "kvq_write_kv", "kvq_sink_plan", "kvq_sink_mask", "kvq_sink_plan_rows", "kvq_sink_mask_rows",
+    "kvq_decode_workspace_bytes",
     "kvq_decode_attn", "kvq_decode_attn_static", "kvq_decode_static_reset", "kvq_decode_attn_varlen", "kvq_decode_attn_tq4",
     "kvq_decode_block_workspace_bytes", "kvq_decode_attn_block", "kvq_prefill_attn", "kvq_prefill_attn_varlen",
     "kvq_prefill_attn_block",
@@ -78,10 +83,14 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_sink_plan.restype = I
         lib.kvq_sink_mask.argtypes = [P, I, P, I64, P, P]
         lib.kvq_sink_mask.restype = I
+        lib.kvq_sink_plan_rows.argtypes = [P, I, I, I, I64, P, P, P, P, P]
+        lib.kvq_sink_plan_rows.restype = I
+        lib.kvq_sink_mask_rows.argtypes = [P, I, I, P, I64, P, P]
+        lib.kvq_sink_mask_rows.restype = I
         lib.kvq_decode_workspace_bytes.argtypes = [I, I, I, I, I64]
         lib.kvq_decode_workspace_bytes.restype = SZ
         lib.kvq_decode_attn.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, F, P, P, SZ, P, P]
-        lib.kvq_decode_attn_varlen.argtypes = lib.kvq_decode_attn.argtypes
+        lib.kvq_decode_attn_varlen.argtypes = [P, I, I, I, I, P, P, P, P, P, P, I64, P, P, I64, F, P, P, SZ, P, P]
         lib.kvq_decode_attn_varlen.restype = I
         lib.kvq_decode_attn_tq4.argtypes = lib.kvq_decode_attn.argtypes
         lib.kvq_decode_attn_tq4.restype = I
@@ -95,7 +104,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.kvq_decode_static_reset.argtypes = [P]
         lib.kvq_decode_static_reset.restype = I
         lib.kvq_prefill_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I, I, F, P, P, P]
-        lib.kvq_prefill_attn_varlen.argtypes = lib.kvq_prefill_attn.argtypes
+        lib.kvq_prefill_attn_varlen.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P, P, I64, I, I, F, P, P,
+                                                P]
         lib.kvq_prefill_attn_varlen.restype = I
         lib.kvq_prefill_attn.restype = I
         lib.kvq_prefill_attn_block.argtypes = [I, P, I, I, I, I, I, P, P, P, P, I64, P, P, I, I, F, P, P, P]
@@ -156,10 +166,11 @@ def _cuda(name, t, dtype=None, contiguous=True):
 
 
 def write(mode: int, x: torch.Tensor, slot_mapping: torch.Tensor, codes: torch.Tensor,
-          scales: torch.Tensor, zero_points: torch.Tensor | None = None, *, round_scale: bool = True,
+          scales: torch.Tensor, zero_points: torch.Tensor | None = None, *, round_scale: int = SCALE_CEIL,
           err_word: torch.Tensor | None = None) -> None:
     """kvq_write: quantize x [B, H, T, D] (bf16, any strides with unit last stride)
-    and scatter into the cache in place.  num_slots is codes.shape[2]."""
+    and scatter into the cache in place.  num_slots is codes.shape[2].  round_scale
+    (modes 2, 3, 5): SCALE_CEIL (1 / True), SCALE_FLOOR (0 / False) or SCALE_OCP (2)."""
     _cuda("x", x, torch.bfloat16, contiguous=False)
     if x.dim() != 4 or x.stride(3) != 1:
         raise ValueError("x must be [B, H, T, D] with a unit last stride")
@@ -171,14 +182,14 @@ def write(mode: int, x: torch.Tensor, slot_mapping: torch.Tensor, codes: torch.T
     _on_current_device(x)
     B, H, T, D = x.shape
     strides = (ctypes.c_int64 * 4)(*x.stride())
-    st = load().kvq_write(int(mode), int(bool(round_scale)), _ptr(x), B, H, T, D, strides,
+    st = load().kvq_write(int(mode), int(round_scale), _ptr(x), B, H, T, D, strides,
                           _ptr(slot_mapping), int(codes.shape[2]), _ptr(codes), _ptr(scales),
                           _ptr(zero_points), _ptr(err_word), _stream(x.device))
     _check("kvq_write", st)
 
 
 def write_kv(mode: int, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_cache, v_cache, *,
-             round_scale: bool = True, err_word: torch.Tensor | None = None) -> None:
+             round_scale: int = SCALE_CEIL, err_word: torch.Tensor | None = None) -> None:
     """kvq_write_kv: kvq_write of k and v (both bf16 [B, H, T, D], unit last stride)
     in one launch.  k_cache / v_cache are (codes, scales, zero_points or None)."""
     for n, t in (("k", k), ("v", v)):
@@ -200,7 +211,7 @@ def write_kv(mode: int, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Te
     B, H, T, D = k.shape
     ks_ = (ctypes.c_int64 * 4)(*k.stride())
     vs_ = (ctypes.c_int64 * 4)(*v.stride())
-    st = load().kvq_write_kv(int(mode), int(bool(round_scale)), _ptr(k), _ptr(v), B, H, T, D, ks_, vs_,
+    st = load().kvq_write_kv(int(mode), int(round_scale), _ptr(k), _ptr(v), B, H, T, D, ks_, vs_,
                              _ptr(slot_mapping), int(kc.shape[2]), _ptr(kc), _ptr(ks), _ptr(kz), _ptr(vc), _ptr(vs),
                              _ptr(vz), _ptr(err_word), _stream(k.device))
     _check("kvq_write_kv", st)
@@ -229,6 +240,46 @@ def sink_mask(input_pos: torch.Tensor, Lq: int, slot_pos: torch.Tensor, mask: to
     st = load().kvq_sink_mask(_ptr(input_pos), Lq, _ptr(slot_pos), slot_pos.numel(), _ptr(mask),
                               _stream(mask.device))
     _check("kvq_sink_mask", st)
+
+
+def sink_plan_rows(input_pos: torch.Tensor, T: int, sink_size: int, slot_pos: torch.Tensor,
+                   slot_mapping: torch.Tensor, kv_lens: torch.Tensor,
+                   err_word: torch.Tensor | None = None) -> None:
+    """kvq_sink_plan_rows: per batch row b, T tokens from input_pos[b] (int32 [B]);
+    slot_pos int32 [B, S] in/out, slot_mapping int32 [B*T] and kv_lens int32 [B] out."""
+    for n, t in (("input_pos", input_pos), ("slot_pos", slot_pos), ("slot_mapping", slot_mapping),
+                 ("kv_lens", kv_lens), ("err_word", err_word)):
+        _cuda(n, t, torch.int32)
+    if slot_pos.dim() != 2 or slot_pos.shape[0] != input_pos.numel():
+        raise ValueError("slot_pos must be [B, S] with B = input_pos.numel()")
+    _on_current_device(slot_pos)
+    B, S = slot_pos.shape
+    st = load().kvq_sink_plan_rows(_ptr(input_pos), B, T, sink_size, S, _ptr(slot_mapping), _ptr(slot_pos),
+                                   _ptr(kv_lens), _ptr(err_word), _stream(slot_pos.device))
+    _check("kvq_sink_plan_rows", st)
+
+
+def sink_mask_rows(input_pos: torch.Tensor, Lq: int, slot_pos: torch.Tensor, mask: torch.Tensor) -> None:
+    """kvq_sink_mask_rows: additive mask [B, Lq, S] (float32) from slot_pos [B, S]."""
+    _cuda("input_pos", input_pos, torch.int32)
+    _cuda("slot_pos", slot_pos, torch.int32)
+    _cuda("mask", mask, torch.float32)
+    if slot_pos.dim() != 2 or mask.shape != (slot_pos.shape[0], Lq, slot_pos.shape[1]):
+        raise ValueError("slot_pos must be [B, S] and mask [B, Lq, S]")
+    _on_current_device(mask)
+    B, S = slot_pos.shape
+    st = load().kvq_sink_mask_rows(_ptr(input_pos), B, Lq, _ptr(slot_pos), S, _ptr(mask), _stream(mask.device))
+    _check("kvq_sink_mask_rows", st)
+
+
+def _mask_batch_stride(mask, B, Lq, S):
+    """0 for one mask shared by every batch row ([S] / [Lq, S]); Lq * S for a
+    per-row mask [B, Lq, S] (decode: [B, 1, S] or [B, S])."""
+    if mask is None or mask.numel() == Lq * S:
+        return 0
+    if mask.numel() == B * Lq * S:
+        return Lq * S
+    raise ValueError(f"mask must hold Lq*S or B*Lq*S floats, got shape {tuple(mask.shape)}")
 
 
 def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, S: int) -> int:
@@ -370,11 +421,20 @@ def _decode(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, sm_scale, 
         sm_scale = 1.0 / math.sqrt(D)
     if workspace is None:
         workspace = decode_workspace(B, Hq, Hkv, D, S, q.device)
-    name = "kvq_decode_attn_varlen" if varlen else ("kvq_decode_attn_tq4" if tq4 else "kvq_decode_attn")
-    st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
-                               _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
-                               _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
-                               _stream(q.device))
+    if varlen:
+        name = "kvq_decode_attn_varlen"
+        st = load().kvq_decode_attn_varlen(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                           _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask),
+                                           _mask_batch_stride(mask, B, 1, S), float(sm_scale), _ptr(out),
+                                           _ptr(workspace), workspace.numel(), _ptr(err_word), _stream(q.device))
+    else:
+        if mask is not None and mask.numel() != S:
+            raise ValueError("decode_attn takes one mask row [S] (per-row masks: decode_attn_varlen)")
+        name = "kvq_decode_attn_tq4" if tq4 else "kvq_decode_attn"
+        st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                   _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), float(sm_scale),
+                                   _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err_word),
+                                   _stream(q.device))
     _check(name, st)
     return out
 
@@ -432,10 +492,20 @@ def _prefill(q, k, k_scale, k_zp, v, v_scale, v_zp, kv_len, out, mask, is_causal
     Hkv, S = k.shape[1], k.shape[2]
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(D)
-    name = "kvq_prefill_attn_varlen" if varlen else "kvq_prefill_attn"
-    st = getattr(load(), name)(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
-                               _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), int(bool(is_causal)),
-                               int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
-                               _stream(q.device))
+    if varlen:
+        name = "kvq_prefill_attn_varlen"
+        st = load().kvq_prefill_attn_varlen(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp),
+                                            _ptr(v), _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask),
+                                            _mask_batch_stride(mask, B, Lq, S), int(bool(is_causal)),
+                                            int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
+                                            _stream(q.device))
+    else:
+        if mask is not None and mask.numel() != Lq * S:
+            raise ValueError("prefill_attn takes one mask [Lq, S] (per-row masks: prefill_attn_varlen)")
+        name = "kvq_prefill_attn"
+        st = load().kvq_prefill_attn(_ptr(q), B, Hq, Hkv, Lq, D, _ptr(k), _ptr(k_scale), _ptr(k_zp), _ptr(v),
+                                     _ptr(v_scale), _ptr(v_zp), S, _ptr(kv_len), _ptr(mask), int(bool(is_causal)),
+                                     int(bool(mask_is_causal)), float(sm_scale), _ptr(out), _ptr(err_word),
+                                     _stream(q.device))
     _check(name, st)
     return out

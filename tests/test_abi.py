@@ -56,6 +56,9 @@ def test_argument_checks_reject_before_any_launch(lib):
     fake = P(16)
     # unknown mode
     assert lib.kvq_write(9, 1, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
+    # round_scale is one of the three scale rules
+    assert lib.kvq_write(2, 3, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
+    assert lib.kvq_write(3, -1, fake, 1, 1, 1, 64, strides, fake, 8, fake, fake, fake, None, None) == -1
     # int8 mode needs D in {64, 128, 256}
     assert lib.kvq_write(0, 1, fake, 1, 1, 1, 96, strides, fake, 8, fake, fake, fake, None, None) == -2
     # block modes need d % 32 == 0 and d <= 8192

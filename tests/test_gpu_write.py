@@ -23,7 +23,7 @@ def _prefill(mode, B, H, S, D, g):
     return [c, s, None]
 
 
-def _run_both(mode, x, sm, cache0, S, round_scale=True):
+def _run_both(mode, x, sm, cache0, S, round_scale=1):
     """Write x on the GPU and in the oracle over identical pre-filled caches."""
     gpu = [None if c is None else c.to(DEV) for c in cache0]
     err = err_word()
@@ -104,14 +104,14 @@ def _special_rows(d, g):
 
 
 # (mode, round_scale): the IndexerQuantCache quant modes and cache types built;
-# round_scale only matters for the MX-FP8 modes 2 and 5
-BLOCK_CASES = [(1, True), (2, True), (3, True), (4, True), (5, True), (6, True), (2, False), (5, False)]
+# round_scale (1 ceil, 0 floor, 2 the OCP MX rule) matters for the E8M0 modes 2, 3, 5
+BLOCK_CASES = [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (6, 1), (2, 0), (5, 0), (3, 0), (2, 2), (3, 2), (5, 2)]
 
 
 @pytest.mark.parametrize("mode,round_scale", BLOCK_CASES)
 @pytest.mark.parametrize("d", [32, 96, 512, 8192])
 def test_block_modes_small(mode, round_scale, d):
-    g = wl.generator(2000 + mode * 10 + d + (0 if round_scale else 7))
+    g = wl.generator(2000 + mode * 10 + d + (0 if round_scale == 1 else 7 + round_scale))
     bs = 300 if d <= 512 else 24
     S = 2 * bs
     x = wl.bf16_normal((bs, d), g, outlier_p=0.01, outlier_scale=10.0)

@@ -86,3 +86,28 @@ def test_filled_count_sinks_visible_and_window():
             # visible count never exceeds what a one-token-at-a-time decode sees
             assert vis.sum() <= min(qpos + 1, S)
         p += T
+
+
+def test_rows_plan_is_the_single_sequence_plan_per_row():
+    """Per-row positions (a ragged batch): each row's slots, slot table, kv_len and
+    mask are those of the single-sequence plan run on that row alone; rows with
+    the same position agree; a negative position writes nothing."""
+    S, sink, T = 64, 4, 3
+    pos = np.array([0, 5, 61, 130, 5, -1], np.int32)
+    sp = np.full((len(pos), S), -1, np.int32)
+    sm, kv = oracle.sink_plan_rows(pos, T, sink, S, sp)
+    for b, p in enumerate(pos):
+        if p < 0:
+            assert np.all(sm[b * T:(b + 1) * T] == -1) and kv[b] == 0 and np.all(sp[b] == -1)
+            continue
+        alone = np.full(S, -1, np.int32)
+        sm1, kv1 = oracle.sink_plan(int(p), 1, T, sink, S, alone)
+        assert np.array_equal(sm[b * T:(b + 1) * T], sm1) and kv[b] == kv1 and np.array_equal(sp[b], alone)
+        # the ring formula, by hand
+        for t in range(T):
+            q = int(p) + t
+            assert sm[b * T + t] == (q if q < sink else sink + (q - sink) % (S - sink))
+    assert np.array_equal(sm[T:2 * T], sm[4 * T:5 * T]) and np.array_equal(sp[1], sp[4])
+    m = oracle.sink_mask_rows(np.maximum(pos, 0), T, sp)
+    for b in range(len(pos)):
+        assert np.array_equal(m[b], oracle.sink_mask(int(max(pos[b], 0)), T, sp[b]))
