@@ -289,6 +289,17 @@ KVQ_DEVINL void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// A load of the word at p whose value is never read: it only brings the page's
+// address translation (and the line, into L2) close.  Nothing waits for it.
+KVQ_DEVINL void touch_translation(const void *p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<uintptr_t>(p) & ~uintptr_t(3)));
+  asm volatile("" ::"r"(v));
+}
+// Bring a TMA descriptor (a __grid_constant__ kernel parameter) into the descriptor cache.
+KVQ_DEVINL void prefetch_tensormap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 // One 2-D TMA box of the map at element (x, y), completion counted on bar.
 KVQ_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar, uint64_t policy) {
   asm volatile(
@@ -327,13 +338,21 @@ struct SimtCore {
   float2 o2[HC][VPL];
   float sm_[HC], sl_[HC], sc_[HC], so_[HC][VPL];  // the first unit's state (deferred close)
 
+  // q of one head as the converter gets it: here the row pointer (the loads
+  // happen inside convert_q).
+  struct QRaw {
+    const uint16_t *qg;
+  };
+  static __device__ __forceinline__ QRaw load_q_raw(const uint16_t *qg, int) { return QRaw{qg}; }
+
   // warp `h` (< HC): head h of q onto the fixed-point grid, into q slot `slot`.
   //   n = rne(q * qscale / 2^E), |n| <= 32767.  Word w of lane sub pairs (low half,
   //   high half) with bytes {0,1} (w even) or {2,3} (w odd) of the lane's code word
   //   w / 2, which holds the unpacked nibbles of dims (0,2,4,6), (1,3,5,7),
   //   (8,10,12,14), (9,11,13,15) of the lane's 16.
-  static __device__ __forceinline__ void convert_q(uint8_t *smem, const uint16_t *qg, float qscale, int slot, int h,
+  static __device__ __forceinline__ void convert_q(uint8_t *smem, const QRaw &raw, float qscale, int slot, int h,
                                                    int lane) {
+    const uint16_t *qg = raw.qg;
     constexpr int NWD = D / 2;            // words of one head
     constexpr int PER = (NWD + 31) / 32;  // words per lane
     float x[PER][2];
@@ -591,16 +610,41 @@ struct MmaCore {
     return tile + st * SUBT + row * ROWB + ((unit ^ x) << 4);
   }
 
+  // q of one head as the converter gets it: the lane's D/32 bf16 values (dims
+  // [lane * D/32, lane * D/32 + D/32)), loaded with one access so that the load can
+  // be issued well before the conversion.
+  struct QRaw {
+    uint32_t w[D / 64];
+  };
+  static __device__ __forceinline__ QRaw load_q_raw(const uint16_t *qg, int lane) {
+    QRaw r;
+    if constexpr (D == 64) {
+      r.w[0] = reinterpret_cast<const uint32_t *>(qg)[lane];
+    } else if constexpr (D == 128) {
+      const uint2 v = reinterpret_cast<const uint2 *>(qg)[lane];
+      r.w[0] = v.x;
+      r.w[1] = v.y;
+    } else {
+      const uint4 v = reinterpret_cast<const uint4 *>(qg)[lane];
+      r.w[0] = v.x;
+      r.w[1] = v.y;
+      r.w[2] = v.z;
+      r.w[3] = v.w;
+    }
+    return r;
+  }
+
   // warp `h` (< HC): head h of q onto the fixed-point grid, split into the two
   // signed byte planes n = 256 hi + lo, into q slot `slot` ([plane][HC][D] bytes)
-  static __device__ __forceinline__ void convert_q(uint8_t *smem, const uint16_t *qg, float qscale, int slot, int h,
+  static __device__ __forceinline__ void convert_q(uint8_t *smem, const QRaw &raw, float qscale, int slot, int h,
                                                    int lane) {
     constexpr int PER = D / 32;  // dims per lane: [lane * PER, lane * PER + PER)
     float x[PER];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      x[i] = __uint_as_float(static_cast<uint32_t>(qg[lane * PER + i]) << 16) * qscale;
+      const uint32_t w = raw.w[i / 2];
+      x[i] = ((i & 1) ? bf16hi(w) : bf16lo(w)) * qscale;
       amax = fmaxf(amax, fabsf(x[i]));
     }
 #pragma unroll
@@ -891,6 +935,43 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     sh[1] = 0;
     sh[2] = 0;
   }
+  // the TMA descriptors are launch parameters, not data of the kernel before this one:
+  // fetch them while that kernel drains
+  if constexpr (C::MMA) {
+    if (tid == 32) {
+      prefetch_tensormap(&maps.k);
+      prefetch_tensormap(&maps.v);
+    }
+  }
+  // Warm the address translations of every buffer this CTA touches (a first touch
+  // of a page costs more than a cache miss to DRAM): one relaxed gpu-scope load per
+  // buffer, at the rows this CTA is likely to reach, issued before the wait so that
+  // the misses overlap the kernel before this one.  The values are never used (and
+  // a gpu-scope load is served by L2, never by a stale L1 line).
+  if (tid < 16) {
+    const int64_t U0 = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
+    const int64_t u = U0 * blockIdx.x / gridDim.x;  // a unit near this CTA's first one
+    const int64_t bhk = u / a.nhc, row = bhk * a.S;
+    const int64_t b = bhk / a.Hkv;
+    const void *p = nullptr;
+    switch (tid) {
+      case 0: p = a.kv_len; break;
+      case 1: p = a.q + (b * a.Hq + (bhk - b * a.Hkv) * a.G) * D; break;
+      case 2: p = a.out + (b * a.Hq + (bhk - b * a.Hkv) * a.G) * D; break;
+      case 3: p = a.ws_cnt; break;
+      case 4: p = a.ws_o + 2 * static_cast<int64_t>(blockIdx.x) * HC * D; break;
+      case 5: p = a.ws_ml + 4 * static_cast<int64_t>(blockIdx.x) * HC; break;
+      case 6: p = a.k + row * CB; break;
+      case 7: p = a.v + row * CB; break;
+      case 8: p = a.ks + row; break;
+      case 9: p = a.vs + row; break;
+      case 10: p = a.kz + row; break;
+      case 11: p = a.vz + row; break;
+      case 12: p = a.mask; break;
+      default: break;
+    }
+    if (p) touch_translation(p);
+  }
   // everything read below may have been written by the kernel launched before this one
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
@@ -1060,15 +1141,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   };
 
-  // warp w: heads w, w + NW, .. of unit u onto the core's q layout, into q slot `slot`
-  auto convert_q = [&](int u, int slot) {
+  // the q row of head h of unit u
+  auto q_row = [&](int u, int h) {
     const int hc = u % a.nhc;
     const int64_t bhk = u / a.nhc;
     const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
-    for (int h = warp; h < HC; h += NW) {
-      const uint16_t *qg = a.q + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC + h) * D;
-      Core::convert_q(smem, qg, a.qscale, slot, h, lane);
-    }
+    return a.q + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC + h) * D;
+  };
+  // warp w: heads w, w + NW, .. of unit u onto the core's q layout, into q slot `slot`
+  auto convert_q = [&](int u, int slot) {
+    for (int h = warp; h < HC; h += NW)
+      Core::convert_q(smem, Core::load_q_raw(q_row(u, h), lane), a.qscale, slot, h, lane);
   };
 
   // all threads: combine the warp records of unit u, found at tiles + rec (floats)
@@ -1222,16 +1305,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   };
 
-  // ---- start the copies, stage q and the owner records
-  if (lane == 0) top_up(0, deferred ? c_end : min(c_end, ustart(u_first) + ulen(u_first)));
-  int cf0 = 0, cf1 = 0;
-  const int own0 = stage_owners(u_first, 0, cf0);
-  const int own1 = u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
-  if (deferred) {
-    convert_q(u_first, 0);
-    if (u_last != u_first) convert_q(u_last, 1);
+  // ---- stage q and start the copies.  The heads of the first and the last unit
+  // are spread over all warps (at most kQItems per warp); their loads are issued
+  // before the warp's burst of bulk copies (loads issued behind it wait for the
+  // copy engine), and converted after it.
+  constexpr int kQItems = (2 * HC + NW - 1) / NW;
+  const int q_items = deferred ? (u_last != u_first ? 2 : 1) * HC : 0;
+  typename Core::QRaw qraw[kQItems];
+#pragma unroll
+  for (int j = 0; j < kQItems; ++j) {
+    const int i = warp + j * NW;
+    if (i < q_items) qraw[j] = Core::load_q_raw(q_row(i < HC ? u_first : u_last, i % HC), lane);
   }
-  __syncthreads();  // q slots and owner records written
+  if (lane == 0) top_up(0, deferred ? c_end : min(c_end, ustart(u_first) + ulen(u_first)));
+#pragma unroll
+  for (int j = 0; j < kQItems; ++j) {
+    const int i = warp + j * NW;
+    if (i < q_items) Core::convert_q(smem, qraw[j], a.qscale, i < HC ? 0 : 1, i % HC, lane);
+  }
+  __syncthreads();  // q slots written
 
   // ---- the CTA's units in order
   Core core;
@@ -1283,6 +1375,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       core.reset();
     }
   }
+  // owner records of the split units (needed by the merge only), staged while
+  // the slower warps of the CTA still finish their chunks
+  int cf0 = 0, cf1 = 0;
+  const int own0 = stage_owners(u_first, 0, cf0);
+  const int own1 = u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
   if (deferred) {
     drain();
     // every warp is past its chunks and its ring is idle: records of the first unit at 0, the last at PUB
@@ -1297,7 +1394,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     combine(u_first, 0, 0);
     if (u_last != u_first) combine(u_last, C::PUB / 4, 1);
   }
-  __syncthreads();  // every partial is written; the scratch is free for the merge
+  __syncthreads();  // every partial and owner record is written; the scratch is free for the merge
 
   // Only the first and the last unit of a contiguous range can be shared with
   // other CTAs.  Count this CTA's partials of those (threads 0 and 1); the owner
@@ -1335,6 +1432,9 @@ int head_chunk_simt(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 ==
 
 // Warps per CTA and ring depth.  Tensor-core path: registers hold q fragments
 // (D/8 per lane), O^T accumulators (D/4) and the first unit's saved O^T (D/4).
+// A warp's chunk is a chain of dependent steps, so what sets the pace is warps
+// per SM sub-partition: eight warps (two per sub-partition) with one buffer each
+// beat six with two (two sub-partitions then run one warp alone) at D <= 128.
 // CUDA-core path: q (8 words per head), accumulators (2 x D/32 per head) and
 // q.k partials (D/16 per head).  The ring takes what shared memory is left.
 template <int D, int HC, bool MMA, bool Q4>
@@ -1342,7 +1442,7 @@ struct Tune {
   // tensor-core path: 64-slot chunks up to D = 128 (two chunks' worth of independent
   // MMAs and scores per warp step, fixed costs per chunk halved), 32 for D = 256
   static constexpr int CS = MMA && D <= 128 ? 64 : 32;
-  static constexpr int NW = MMA ? (D == 256 ? 6 : (D == 128 ? 6 : 8))
+  static constexpr int NW = MMA ? (D == 256 ? 6 : 8)
                                 : (D == 256 ? 8 : (D == 128 ? (HC <= 2 ? 16 : 12) : 16));
   static constexpr int CB = Q4 ? D / 2 : D;
   static constexpr int PER_BUF = 2 * CS * CB + 14 * CS;
