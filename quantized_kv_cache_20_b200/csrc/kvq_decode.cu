@@ -289,8 +289,8 @@ KVQ_DEVINL void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// A load of the word at p whose value is never read: it only brings the page's
-// address translation (and the line, into L2) close.  Nothing waits for it.
+// A load of the word at p whose value is never read: it only starts the first
+// access to p's page (translation, line into L2).  Nothing waits for it.
 KVQ_DEVINL void touch_translation(const void *p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<uintptr_t>(p) & ~uintptr_t(3)));
@@ -943,11 +943,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       prefetch_tensormap(&maps.v);
     }
   }
-  // Warm the address translations of every buffer this CTA touches (a first touch
-  // of a page costs more than a cache miss to DRAM): one relaxed gpu-scope load per
-  // buffer, at the rows this CTA is likely to reach, issued before the wait so that
-  // the misses overlap the kernel before this one.  The values are never used (and
-  // a gpu-scope load is served by L2, never by a stale L1 line).
+  // One relaxed gpu-scope load per buffer, at the rows this CTA is likely to reach,
+  // issued before the wait so that the first access to each buffer (its address
+  // translation, its line into L2) can overlap the kernel before this one.  The
+  // values are never used (and a gpu-scope load is served by L2, never by a stale
+  // L1 line).
   if (tid < 16) {
     const int64_t U0 = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
     const int64_t u = U0 * blockIdx.x / gridDim.x;  // a unit near this CTA's first one
