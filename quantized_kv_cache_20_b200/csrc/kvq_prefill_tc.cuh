@@ -87,6 +87,7 @@ struct PrefillArgs {
   int is_causal, mask_is_causal;
   float qscale;      // sm_scale * log2(e)
   uint64_t wait_ns;  // bound on each main-loop wait
+  int ns;            // KV splits: a cluster of ns CTAs shares one row block, each a share of its KV tiles
   // block caches (kvq_write modes 1-6): codes in k / v, per-32 scales as float
   // (ks / vs) or E8M0 bytes (ks8 / vs8); kz / vz unused
   const uint8_t *ks8, *vs8;
@@ -133,8 +134,12 @@ struct Cfg {
   static constexpr int FAC_OFF = VMX_OFF + kScaleBufs * 16;
   static constexpr int FAC_BYTES = MODE == 0 ? 0 : 2 * 2 * kTile * NG * 4;
   static constexpr int BAR_OFF = FAC_OFF + FAC_BYTES;
-  static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag, qs, 4 x max|q|
-  static constexpr int SMEM = MISC_OFF + 32 + 1024;        // + slack to align the base to 1024
+  static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag, qs, 4 x max|q|, O valid
+  static constexpr int STAT_OFF = MISC_OFF + 32;             // KV split: float4 [kRows] (m, E, l, -) per row
+  static constexpr int SMEM = STAT_OFF + kRows * 16 + 1024;  // + slack to align the base to 1024
+  // KV split: the rows' pre-scaled fp32 partial O, [kRows][D], over the Q/K/V tiles
+  static constexpr int CONTRIB_OFF = Q_OFF;
+  static_assert(kRows * D * 4 <= BAR_OFF, "the partial O fits over the tiles");
   static constexpr int S_COL0 = 0, S_COL1 = kTile, O_COL = 2 * kTile;
   static constexpr int TMEM_COLS = 512;
   static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
@@ -316,7 +321,9 @@ KVQ_DEVINL uint32_t zp_const2(int zp) {
 struct Ctx {
   uint8_t *smem;  // 1024-byte aligned dynamic shared memory
   uint32_t tmem;  // TMEM base address
-  int kv, loop_end, ntiles;
+  int kv, loop_end;
+  int jb, ntiles;  // this CTA's KV tiles: jb .. jb + ntiles - 1 (loops count j from 0)
+  int vis_end;     // with is_causal, no row of the CTA sees a slot at or past this
 };
 
 // softmax warpgroup: query row t = threadIdx.x, TMEM lane t
@@ -332,10 +339,10 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
   const float *vs_s = reinterpret_cast<const float *>(smem + C::VS_OFF);
   const float *vmx_s = reinterpret_cast<const float *>(smem + C::VMX_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
+  const int xrow = blockIdx.x / a.ns, hkc = blockIdx.y, b = blockIdx.z;  // a.ns CTAs share a row block
   const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
   const uint32_t tmem = x.tmem;
-  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles;
+  const int kv = x.kv, loop_end = x.loop_end, ntiles = x.ntiles, jb = x.jb;
   // ======================= softmax warpgroup: query row t
   const int t = tid;
   const int g = t / RPH;
@@ -400,7 +407,7 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
   bool have_e = false, ok = true;
   for (int j = 0; j < ntiles; ++j) {
     const int buf = j & 1;
-    const int t0 = j * kTile;
+    const int t0 = (jb + j) * kTile;
     const int sb = j % kScaleBufs;
     const uint32_t s_addr = tmem + (buf ? C::S_COL1 : C::S_COL0) + lane_base;
     const float4 *kq4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
@@ -531,7 +538,15 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     mbar_arrive(&bars[kBarPFull0 + buf]);
   }
   // ---- epilogue: O / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
-  if (ok) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag, a.wait_ns));
+  if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag, a.wait_ns));
+  if (a.ns > 1) {
+    // KV split: publish this row's running max, P exponent and sum; the cluster
+    // merge reads O from TMEM
+    const bool have = ok && ntiles > 0 && m != -INFINITY;
+    reinterpret_cast<float4 *>(smem + C::STAT_OFF)[t] =
+        make_float4(have ? m : -INFINITY, static_cast<float>(E), have ? l : 0.0f, 0.0f);
+    return;
+  }
   if (ok) {
     tc_fence_after();
     uint16_t *op = a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D;
@@ -570,7 +585,7 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
   float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = static_cast<int64_t>(blockIdx.z) * a.Hkv + blockIdx.y / a.nhc;
-  const int loop_end = x.loop_end, ntiles = x.ntiles;
+  const int loop_end = x.loop_end, ntiles = x.ntiles, jb = x.jb;
   // ======================= converter warpgroups: K (warps 4-7), V (warps 8-11)
   const bool is_k = warp < 8;
   const int c = tid - kSoftmaxThreads - (is_k ? 0 : kConvThreads);  // 0..127
@@ -609,12 +624,12 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
     for (int r = 0; r < C::NCH; ++r)
       if (sg * C::NCH + r >= n) z[r >> 2] = (z[r >> 2] & ~(0xFFu << (8 * (r & 3)))) | (0x80u << (8 * (r & 3)));
   };
-  auto tile_n = [&](int j) { return min(kTile, loop_end - j * kTile); };
+  auto tile_n = [&](int j) { return min(kTile, loop_end - (jb + j) * kTile); };
   // convert + store this tile's chunks, loading W chunks ahead behind them
   auto convert_tile = [&](int j) {
     const bool next = j + 1 < ntiles;
-    const int t0 = j * kTile, n0 = tile_n(j);
-    const int t1 = (j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
+    const int t0 = (jb + j) * kTile, n0 = tile_n(j);
+    const int t1 = (jb + j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
 #pragma unroll
     for (int r = 0; r < C::NCH; ++r) {
       const int s = sg * C::NCH + r;
@@ -637,18 +652,18 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
   {
     const int n0 = tile_n(0);
 #pragma unroll
-    for (int r = 0; r < W; ++r) load_chunk(r, 0, n0);
-    load_zp(zw, 0, n0);
+    for (int r = 0; r < W; ++r) load_chunk(r, jb * kTile, n0);
+    load_zp(zw, jb * kTile, n0);
   }
   if (is_k) {
     // K tiles, and with each the per-slot k_scale * qs, v_scale and max v_scale
     float qs = 0.0f;
-    float ksv = c < tile_n(0) ? ld_f32(a.ks + bh * a.S + c) : 0.0f;
-    float vsv = c < tile_n(0) ? ld_f32(a.vs + bh * a.S + c) : 0.0f;
+    float ksv = c < tile_n(0) ? ld_f32(a.ks + bh * a.S + jb * kTile + c) : 0.0f;
+    float vsv = c < tile_n(0) ? ld_f32(a.vs + bh * a.S + jb * kTile + c) : 0.0f;
     for (int j = 0; j < ntiles; ++j) {
       float ksn = 0.0f, vsn = 0.0f;
       if (j + 1 < ntiles) {
-        const int t1 = (j + 1) * kTile, n1 = tile_n(j + 1);
+        const int t1 = (jb + j + 1) * kTile, n1 = tile_n(j + 1);
         load_zp(zn, t1, n1);
         ksn = c < n1 ? ld_f32(a.ks + bh * a.S + t1 + c) : 0.0f;
         vsn = c < n1 ? ld_f32(a.vs + bh * a.S + t1 + c) : 0.0f;
@@ -662,7 +677,7 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
       const int sb = j % kScaleBufs;
       ks_s[sb * kTile + c] = ksv * qs;
       vs_s[sb * kTile + c] = vsv;
-      float vm = vsv;
+      float vm = (jb + j) * kTile + c < x.vis_end ? vsv : 0.0f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
       if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
@@ -673,7 +688,7 @@ __device__ __noinline__ void role_convert(const PrefillArgs &a, const Ctx x) {
     }
   } else {
     for (int j = 0; j < ntiles; ++j) {
-      if (j + 1 < ntiles) load_zp(zn, (j + 1) * kTile, tile_n(j + 1));
+      if (j + 1 < ntiles) load_zp(zn, (jb + j + 1) * kTile, tile_n(j + 1));
       if (j > 0) {  // the buffer is free once PV_{j-1} has run
         ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarVEmpty], (j - 1) & 1, abort_flag, a.wait_ns));
         if (!ok) break;
@@ -867,7 +882,7 @@ __device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx 
   float *vmx_s = reinterpret_cast<float *>(smem + C::VMX_OFF);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = static_cast<int64_t>(blockIdx.z) * a.Hkv + blockIdx.y / a.nhc;
-  const int loop_end = x.loop_end, ntiles = x.ntiles;
+  const int loop_end = x.loop_end, ntiles = x.ntiles, jb = x.jb;
   const bool is_k = warp < 8;
   const int c = tid - kSoftmaxThreads - (is_k ? 0 : kConvThreads);  // 0..127
   const int part = c % C::PPR, sg = c / C::PPR, grp = part >> 1;
@@ -900,11 +915,11 @@ __device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx 
       w[r % W] = make_uint4(0u, 0u, 0u, 0u);  // code 0 is +0 in every format
     }
   };
-  auto tile_n = [&](int j) { return min(kTile, loop_end - j * kTile); };
+  auto tile_n = [&](int j) { return min(kTile, loop_end - (jb + j) * kTile); };
   auto convert_tile = [&](int j) {
     const bool next = j + 1 < ntiles;
-    const int t0 = j * kTile, n0 = tile_n(j);
-    const int t1 = (j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
+    const int t0 = (jb + j) * kTile, n0 = tile_n(j);
+    const int t1 = (jb + j + 1) * kTile, n1 = next ? tile_n(j + 1) : 0;
     const float *fb = fac + (j & 1) * kTile * NG;
 #pragma unroll
     for (int r = 0; r < C::NCH; ++r) {
@@ -928,12 +943,12 @@ __device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx 
   {
     const int n0 = tile_n(0);
 #pragma unroll
-    for (int r = 0; r < W; ++r) load_chunk(r, 0, n0);
+    for (int r = 0; r < W; ++r) load_chunk(r, jb * kTile, n0);
     cur.clear();
     vcur.clear();
     if (c < n0) {
-      cur.load(own_sc + static_cast<int64_t>(c) * SRB);
-      if (is_k) vcur.load(v_sc + static_cast<int64_t>(c) * SRB);
+      cur.load(own_sc + static_cast<int64_t>(jb * kTile + c) * SRB);
+      if (is_k) vcur.load(v_sc + static_cast<int64_t>(jb * kTile + c) * SRB);
     }
   }
   float qs = 0.0f;
@@ -943,7 +958,7 @@ __device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx 
     nxt.clear();
     vnxt.clear();
     if (j + 1 < ntiles && c < tile_n(j + 1)) {
-      const int64_t t = static_cast<int64_t>(j + 1) * kTile + c;
+      const int64_t t = static_cast<int64_t>(jb + j + 1) * kTile + c;
       nxt.load(own_sc + t * SRB);
       if (is_k) vnxt.load(v_sc + t * SRB);
     }
@@ -969,7 +984,7 @@ __device__ __noinline__ void role_convert_block(const PrefillArgs &a, const Ctx 
         const float vsv = valid ? exp2i(Ev) : 0.0f;
         ks_s[sb * kTile + c] = valid ? exp2i(E) * qs : 0.0f;
         vs_s[sb * kTile + c] = vsv;
-        float vm = vsv;
+        float vm = (jb + j) * kTile + c < x.vis_end ? vsv : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
         if (lane == 0) vmx_s[sb * 4 + (warp - 4)] = vm;
@@ -1015,7 +1030,8 @@ __device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
       mma_commit(&bars[kBarSFull0 + (j & 1)]);
       mma_commit(&bars[kBarKEmpty]);
     };
-    bool ok = wait_phase(&bars[kBarQ], 0, abort_flag, a.wait_ns);
+    bool ok = ntiles > 0;  // a KV split can be left without tiles
+    if (ok) ok = wait_phase(&bars[kBarQ], 0, abort_flag, a.wait_ns);
     if (ok) ok = wait_phase(&bars[kBarKFull], 0, abort_flag, a.wait_ns);
     if (ok) {
       tc_fence_after();
@@ -1051,6 +1067,127 @@ __device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
   __syncwarp();
 }
 
+// ---- KV split across a thread-block cluster --------------------------------
+KVQ_DEVINL uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; orders shared-memory accesses across it.
+KVQ_DEVINL void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of this CTA's shared-memory byte `local` in cluster CTA `rank`.
+KVQ_DEVINL uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+KVQ_DEVINL float4 ld_peer_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// The cluster's CTAs each hold (m, E, l, O) of one share of the KV tiles for
+// the same 128 query rows (O and l in units of 2^-(m+E)).  Against the share r
+// with the largest m (the first such), share c weighs f_c = 2^(m_c - m_r) 2^(E_c - E_r),
+// the power of two applied exactly, and contributes O_c f_c / L with
+// L = sum_c l_c f_c.  A share whose E moved by k over tiles that no row sees
+// has O and l scaled by exactly 2^-k and f_c by 2^k, so the output does not
+// depend on whether such tiles were visited.  Each CTA writes its contribution
+// to its own shared memory, then sums one slice of the rows over the cluster
+// (distributed shared memory) and stores it.  All threads take part.
+template <class C>
+__device__ __noinline__ void cluster_merge(const PrefillArgs &a, const Ctx x, bool o_valid) {
+  constexpr int D = C::D, HPT = C::HPT, RPH = C::RPH;
+  uint8_t *smem = x.smem;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int ns = a.ns;
+  const uint32_t rank = cluster_rank();
+  const uint32_t stat_l = smem_u32(smem + C::STAT_OFF), contrib_l = smem_u32(smem + C::CONTRIB_OFF);
+  // 16-byte chunk k of row r sits at chunk k ^ (r & 7) (rows are D * 4 bytes apart)
+  auto cidx = [](int r, int k) { return r * (D / 4) + (k ^ (r & 7)); };
+  cluster_sync();  // every share's row statistics are published
+  if (tid < kRows) {  // the softmax warps own TMEM lanes 0..127: row t
+    const int t = tid;
+    float4 st[8];  // (m, E, l, -) of every share (ns <= 8)
+    float mr = -INFINITY, er = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (c < ns) {
+        st[c] = ld_peer_f4(peer_addr(stat_l + 16 * t, c));
+        if (st[c].x > mr) {
+          mr = st[c].x;
+          er = st[c].y;
+        }
+      }
+    }
+    auto weight = [&](const float4 &sc) {
+      return sc.x == -INFINITY ? 0.0f : ldexpf(ex2f(sc.x - mr), static_cast<int>(sc.y - er));
+    };
+    float L = 0.0f, w_self = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (c < ns) {
+        const float w = weight(st[c]);
+        L = fmaf(st[c].z, w, L);
+        if (c == static_cast<int>(rank)) w_self = w;
+      }
+    }
+    const float f = L > 0.0f ? w_self / L : 0.0f;
+    float4 *dst = reinterpret_cast<float4 *>(smem + C::CONTRIB_OFF);
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    if (o_valid) tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (o_valid) {  // warp-uniform
+        tmem_ld32(x.tmem + C::O_COL + lane_base + cc * 32, o);
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = o_valid && f != 0.0f
+                             ? make_float4(__uint_as_float(o[4 * i]) * f, __uint_as_float(o[4 * i + 1]) * f,
+                                           __uint_as_float(o[4 * i + 2]) * f, __uint_as_float(o[4 * i + 3]) * f)
+                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        dst[cidx(t, cc * 8 + i)] = v;
+      }
+    }
+  }
+  cluster_sync();  // every contribution is written
+  {
+    const int xrow = blockIdx.x / ns, hkc = blockIdx.y, b = blockIdx.z;
+    const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
+    const int r0 = static_cast<int>(rank) * kRows / ns, r1 = (static_cast<int>(rank) + 1) * kRows / ns;
+    for (int i = tid; i < (r1 - r0) * (D / 4); i += kThreads) {
+      const int r = r0 + i / (D / 4), k = i % (D / 4);
+      const int g = r / RPH, pos = xrow * RPH + (r - g * RPH);
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int c = 0; c < ns; ++c) {
+        const float4 v = ld_peer_f4(peer_addr(contrib_l + 16 * cidx(r, k), c));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if (pos < a.Lq) {
+        const int hq = hk * a.G + hc * HPT + g;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + pos) * D + 4 * k) = pk;
+      }
+    }
+  }
+  cluster_sync();  // no CTA leaves while others still read its shared memory
+}
+
 template <class C>
 __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant__ PrefillArgs a) {
   constexpr int RPH = C::RPH;
@@ -1061,7 +1198,7 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int xrow = blockIdx.x, hkc = blockIdx.y, b = blockIdx.z;
+  const int xrow = blockIdx.x / a.ns, hkc = blockIdx.y, b = blockIdx.z;
 
   // ---- set-up
   if (tid == 0) {
@@ -1100,9 +1237,21 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
   // per-tile causal bound (the same in every role)
   const int last_pos = min(xrow * RPH + RPH, a.Lq) - 1;
   const int loop_end = a.mask_is_causal ? min(kv, kv - a.Lq + last_pos + 1) : kv;
-  const int ntiles = (loop_end + kTile - 1) / kTile;
+  // With a KV split, share r of the cluster takes tiles [r T / ns, (r + 1) T / ns) of
+  // the T tiles of the whole kv_len, clipped to the causal bound: the shares do not
+  // depend on the bound, so the output is the same bit for bit with or without it.
+  int jb = 0, ntiles = (loop_end + kTile - 1) / kTile;
+  if (a.ns > 1) {
+    const int T = (kv + kTile - 1) / kTile, r = static_cast<int>(cluster_rank());
+    jb = r * T / a.ns;
+    ntiles = max(0, min((r + 1) * T / a.ns, ntiles) - jb);
+  }
 
-  const Ctx x{smem, tmem, kv, loop_end, ntiles};
+  // The P exponent follows the largest v_scale of the slots some row of the CTA
+  // can see; slots past the causal bound are left out, so visiting them (no
+  // per-tile bound) changes nothing
+  const int vis_end = a.is_causal ? min(kv, kv - a.Lq + last_pos + 1) : kv;
+  const Ctx x{smem, tmem, kv, loop_end, jb, ntiles, vis_end};
   if (warp < 4)
     role_softmax<C>(a, x);
   else if (warp < 12)
@@ -1116,6 +1265,7 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  if (a.ns > 1) cluster_merge<C>(a, x, ntiles > 0 && !*abort_flag);
   if (tid == 0 && *abort_flag) report(a.err, KVQ_ERR_TIMEOUT);
   if (warp == kMmaWarp) {
     tc_fence_after();
@@ -1131,8 +1281,27 @@ int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   using C = Cfg<D, HPT, MASK, MODE>;
   if (const int st = ensure_smem<C>(prefill_tc_kernel<C>, C::SMEM)) return st;
   a.nhc = a.G / HPT;
-  dim3 grid((a.Lq + C::RPH - 1) / C::RPH, a.Hkv * a.nhc, a.B);
-  prefill_tc_kernel<C><<<grid, kThreads, C::SMEM, stream>>>(a);
+  const int rowblocks = (a.Lq + C::RPH - 1) / C::RPH;
+  // KV split: when the row blocks leave most SMs idle, a cluster of ns CTAs
+  // shares each one (up to 4, while the grid still fits one wave and every
+  // share can hold a tile of the cache)
+  const int64_t base = static_cast<int64_t>(rowblocks) * a.Hkv * a.nhc * a.B;
+  const int64_t tiles = (a.S + kTile - 1) / kTile;
+  a.ns = 1;
+  while (a.ns < 4 && base * a.ns * 2 <= sm_count() && a.ns * 2 <= tiles) a.ns *= 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rowblocks * a.ns, a.Hkv * a.nhc, a.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.ns;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.ns > 1 ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, prefill_tc_kernel<C>, a) != cudaSuccess) return KVQ_ECUDA;
   return launch_status();
 }
 
