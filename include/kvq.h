@@ -348,7 +348,9 @@ int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D
  * chunk's rows sit at positions kv_len - Lq + i; with a causal mask row i sees
  * j <= kv_len - Lq + i; mask_is_causal enables the per-tile causal upper bound
  * loop_end = min(kv_len, (kv_len - Lq) + max(seq_pos in tile) + 1), which skips
- * KV tiles that are fully masked, so the output is bit-identical either way).
+ * KV tiles that are fully masked).  With is_causal the output is bit-identical
+ * with or without the bound; with a causal additive mask alone it can differ in
+ * a rare last bit (the fp16 P exponent then also sees the slots the mask hides).
  *
  * q, out        bf16 [B, Hq, Lq, D] contiguous.  Cache arguments as for decode.
  * kv_len        int32 device scalar, clamped to [Lq, S] (KVQ_ERR_KV_LEN_RANGE).
@@ -360,7 +362,10 @@ int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0; S % 16 == 0; 1 <= Lq <= S.
  * Launches one kernel on `stream`: 128 query rows per CTA on the tcgen05
  * tensor cores, S = Q K^T and O += P V with fp16 operands and fp32
- * accumulation in tensor memory.  K/V codes enter as the exact fp16 values
+ * accumulation in tensor memory.  When the row blocks would leave most SMs
+ * idle, a thread-block cluster of up to 4 CTAs shares each row block, each CTA
+ * taking a share of its KV tiles; the shares merge through distributed shared
+ * memory (no workspace).  K/V codes enter as the exact fp16 values
  * (c - zp); q enters as fp16 after one power-of-two rescale per CTA (exact for
  * every element at least 2^-32 times the CTA's largest |q|); k_scale multiplies the fp32
  * scores, and v_scale is folded into P = p * v_scale * 2^-E, rounded to fp16
