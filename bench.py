@@ -13,10 +13,12 @@ the time is the max over ranks.
 
 Printed (rank 0): one JSON line with the headline metric (tokens/s), the
 roofline of the dominant kernel (decode attention, HBM-bound), the end-to-end
-number through the Python binding with host buffers, the CPU oracle baseline,
-clocks sampled during the timed region, and per-kernel detail lines for the
-bulk fill write, the block-quantized writes, the long-context decode, and the
-two chunked prefills (long causal chunk, sink/ring chunk) on the tensor cores.
+number through the Python binding with host buffers, the CPU oracle baseline
+(all host cores, and one core), the GPU clocks (sampled from the warm-up to the
+end of the detail workloads, and read just before and after the timed region),
+and per-kernel detail lines for the bulk fill write, the block-quantized writes,
+the long-context decode, and the chunked prefills on the tensor cores, with
+bounded oracle timings beside some of them.
 """
 from __future__ import annotations
 
@@ -38,9 +40,28 @@ METRIC = "KV-write GB/s + int8-KV decode attn tokens/s, % of B200 HBM roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# DRAM bytes of one decode_kernel launch on the decode workload, read + write, from one ncu
-# capture of the current kernel (69,882,112 + 702,208); algorithmic bytes are 69,861,376.
-DECODE_TRAFFIC_BYTES = 70584320
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode_kernel launch on
+# the decode workload, from one ncu capture, and the SHA-256 of the decode source it was
+# taken on: the line reports the figure only while the source is unchanged (else null).
+DECODE_TRAFFIC_BYTES = 70780160  # 69,880,320 read + 899,840 written; algorithmic 69,861,376
+DECODE_TRAFFIC_SRC_SHA256 = "b75dca97a135dfec007a6997c0e450f578e1a5b9e0302017ea6052dd2d3fecf1"
+DECODE_SRC = ("quantized_kv_cache_20_b200/csrc/kvq_decode.cu", "quantized_kv_cache_20_b200/csrc/kvq_common.cuh")
+
+
+def decode_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in DECODE_SRC:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 def _args():
@@ -98,6 +119,17 @@ class ClockSampler:
         self.index = index
         self.proc = None
 
+    def once(self):
+        """One reading: {sm_mhz, sm_max_mhz, reasons} (None fields when nvidia-smi is missing)."""
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                  "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                 timeout=10).stdout
+        except Exception:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        r = self._parse(out)
+        return {"sm_mhz": r["sm_mhz"], "sm_max_mhz": r["sm_max_mhz"], "reasons": r["reasons"]}
+
     def start(self):
         try:
             self.proc = subprocess.Popen(
@@ -115,6 +147,10 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        return self._parse(out)
+
+    @staticmethod
+    def _parse(out):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
@@ -228,6 +264,116 @@ def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | No
             break
     full = (t_write + t_attn * len(rows) / r) / steps
     return steps, el, full
+
+
+def _oracle_decode_steps_threads(seconds: float, cores: int):
+    """The decode workload's full steps on the CPU oracle, called unchanged from
+    `cores` threads (ctypes releases the GIL inside each call): the write of the
+    step's 64 K and 64 V rows split by token, the 256 attention rows by row.
+    Returns (steps, seconds)."""
+    import concurrent.futures as cf
+    import numpy as np
+    import oracle
+    from quantized_kv_cache_20_b200 import workloads as wl
+
+    w = wl.DECODE
+    g = wl.generator(w.seed)
+    S = w.kv_len
+    K = [t.numpy().copy() for t in wl.int8_cache_like(w.B, w.Hkv, S, w.D, g)]
+    V = [t.numpy().copy() for t in wl.int8_cache_like(w.B, w.Hkv, S, w.D, g)]
+    k = wl.u16(wl.bf16_normal((w.B, w.Hkv, 1, w.D), g))
+    v = wl.u16(wl.bf16_normal((w.B, w.Hkv, 1, w.D), g))
+    q = wl.u16(wl.bf16_normal((w.B, w.Hq, 1, w.D), g))
+    sm = np.full(1, S - 1, np.int32)
+    rows = [(b, h, 0) for b in range(w.B) for h in range(w.Hq)]
+    parts = [rows[i::cores] for i in range(cores)]
+    oracle.build()
+
+    def write_row(b):  # batch row b's token, into batch row b of the caches
+        oracle.write(0, k[b:b + 1], sm, S, *[t[b:b + 1] for t in K])
+        oracle.write(0, v[b:b + 1], sm, S, *[t[b:b + 1] for t in V])
+
+    def attend(part):
+        if part:
+            oracle.sdpa_rows(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D), rows=part)
+
+    steps = 0
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        t0 = time.perf_counter()
+        while True:
+            list(ex.map(write_row, range(w.B)))
+            list(ex.map(attend, parts))
+            steps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return steps, el
+
+
+def _cpu_detail(detail, cores):
+    """Bounded oracle timings beside the detail lines, on all host cores (the
+    unchanged C oracle from `cores` threads over independent tokens / rows)."""
+    import concurrent.futures as cf
+    import numpy as np
+    import oracle
+    from quantized_kv_cache_20_b200 import workloads as wl
+
+    def timed(fn, units, scale, label):
+        t0 = time.perf_counter()
+        with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+            list(ex.map(fn, units))
+        el = time.perf_counter() - t0
+        return {"kind": "oracle", "cores": cores, "sample": label, "sample_s": el, "us_full": 1e6 * el * scale}
+
+    # int8 fill write: 8 x 8 heads x 4095 tokens; sample: batch row 0 (1/8), split by head
+    w = wl.DECODE
+    g = wl.generator(11)
+    x = wl.u16(wl.bf16_normal((1, w.Hkv, w.kv_len - 1, w.D), g))
+    Kc = [np.zeros((1, w.Hkv, w.kv_len, w.D), np.int8), np.zeros((1, w.Hkv, w.kv_len), np.float32),
+          np.zeros((1, w.Hkv, w.kv_len), np.int8)]
+    sm = np.arange(w.kv_len - 1, dtype=np.int32)
+
+    def fill_head(h):
+        oracle.write(0, x[:, h:h + 1], sm, w.kv_len, *[t[:, h:h + 1] for t in Kc])
+    if "int8_fill_write" in detail:
+        c = timed(fill_head, range(w.Hkv), 8 * 2, "K of batch row 0 (1/16 of the fill: 8 heads x 4095 tokens)")
+        c["GB/s"] = detail["int8_fill_write"]["bytes"] / (c["us_full"] / 1e6) / 1e9
+        detail["int8_fill_write"]["cpu"] = c
+    # block writes: x [16384, 512]; sample 2048 tokens, split in chunks of 128
+    bw = wl.BLOCK
+    xb = wl.u16(wl.bf16_normal((1, 1, 2048, bw.d), g, outlier_p=bw.outlier_p, outlier_scale=bw.outlier_scale))
+    for mode, name in ((1, "fp8_e4m3"), (2, "mxfp8"), (3, "mxfp4")):
+        key = f"block_write_{name}"
+        if key not in detail:
+            continue
+        row = bw.d // 2 if mode == 3 else bw.d
+        codes = np.zeros((1, 1, 2048, row), np.uint8)
+        scales = np.zeros((1, 1, 2048, bw.d // 32), np.float32 if mode == 1 else np.uint8)
+
+        def blk(i, mode=mode, codes=codes, scales=scales):
+            sl = slice(128 * i, 128 * i + 128)
+            oracle.write(mode, xb[:, :, sl], np.arange(128, dtype=np.int32), 128, codes[:, :, sl], scales[:, :, sl])
+        c = timed(blk, range(16), bw.tokens / 2048, "2048 of the 16384 tokens (no skipped rows), scaled")
+        c["GB/s"] = detail[key]["bytes"] / (c["us_full"] / 1e6) / 1e9
+        detail[key]["cpu"] = c
+    # long prefill: 64 rows of the 2048-row causal chunk (the first and the last row of every
+    # 128-row tile, over the heads), fp64 over a 131072-slot cache, scaled to 2048 x 32 rows
+    if "long_prefill" in detail:
+        lw = wl.LONG
+        Hk = 1  # one kv head's cache holds the sample's rows (the cost per row does not depend on the head)
+        Kl = [t.numpy() for t in wl.int8_cache_like(1, Hk, lw.kv_len, lw.D, g)]
+        Vl = [t.numpy() for t in wl.int8_cache_like(1, Hk, lw.kv_len, lw.D, g)]
+        ql = wl.u16(wl.bf16_normal((1, 2, lw.Lq, lw.D), g))
+        rows = [(0, e % 2, 128 * t + 127 * e) for t in range(lw.Lq // 128) for e in (0, 1)]
+        rows += [(0, 1, 64 * t + 63) for t in range(32)]  # 64 rows in all
+        rows = rows[:64]
+
+        def att(r):
+            oracle.sdpa_rows(ql, *Kl, *Vl, kv_len=lw.kv_len, sm_scale=1 / math.sqrt(lw.D), rows=[r], is_causal=True)
+        c = timed(att, rows, lw.Lq * lw.Hq / len(rows), "64 rows of the causal chunk (first and last row of every "
+                                                         "128-row tile), scaled to the 2048 x 32 rows")
+        c["TFLOP/s"] = detail["long_prefill"]["flops"] / (c["us_full"] / 1e6) / 1e12
+        detail["long_prefill"]["cpu"] = c
 
 
 REFERENCE_BUDGET_S = 120.0  # the timed part of --impl reference stays near this
@@ -351,7 +497,11 @@ def run_kvq(args, dist: Dist):
         step_graphs.append(gph)
     torch.cuda.synchronize()
 
-    # ---- headline: exactly K steps (whole rotations, then single steps)
+    # ---- headline: exactly K steps (whole rotations, then single steps).  nvidia-smi
+    # samples every 200 ms from here to the end of the detail workloads (a timed region
+    # of a few ms would see no sample), plus one reading right before and after it.
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
     reps, rem = divmod(args.steps, NL)
     nsteps = args.steps
     with torch.cuda.stream(stream):
@@ -360,8 +510,7 @@ def run_kvq(args, dist: Dist):
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    clocks.start()
+    clk_before = clocks.once()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -371,8 +520,8 @@ def run_kvq(args, dist: Dist):
             step_graphs[l].replay()
         e1.record(stream)
     torch.cuda.synchronize()
+    clk_after = clocks.once()
     dist.barrier()
-    clk = clocks.stop()
     ms_local = e0.elapsed_time(e1) / nsteps
     ms = dist.max(ms_local)
     value = dist.world * B / (ms / 1000.0)
@@ -393,9 +542,12 @@ def run_kvq(args, dist: Dist):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
                 "kernel": "decode_kernel (split-K int8 decode attention)", "bytes_per_launch": dec_bytes,
-                "launch_us": dec_ms * 1000.0, "traffic": DECODE_TRAFFIC_BYTES,
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_kernel on this "
-                                  "workload (profiles/decode_kernel__decode_b8_kv4096.md)"}
+                "launch_us": dec_ms * 1000.0}
+    same_src = DECODE_TRAFFIC_BYTES is not None and decode_source_sha256() == DECODE_TRAFFIC_SRC_SHA256
+    roofline["traffic"] = DECODE_TRAFFIC_BYTES if same_src else None
+    roofline["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch "
+                                  "on this workload, captured on the current decode source" if same_src else
+                                  "null: the decode source changed since the last ncu capture")
 
     # ---- end to end through the binding with host buffers
     e2e = _e2e(args, dist, kvq, layers, ws, kv_len, sm_step)
@@ -403,19 +555,33 @@ def run_kvq(args, dist: Dist):
     detail = {}
     if not args.no_detail:
         detail = _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak)
+    clk = clocks.stop()
+    clk["window"] = ("200 ms samples from the warm-up of the timed steps to the end of the detail workloads "
+                     "(continuous GPU load); at_timed_start / at_timed_end bracket the timed region")
+    clk["at_timed_start"] = clk_before
+    clk["at_timed_end"] = clk_after
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(args),
+        "vs_baseline": None, "dtype": "s8 x s8 -> s32 (q.K), f16 x f16 -> f32 (P.V), f32 softmax",
+        "data": "synthetic", "config": _config(args),
         "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * nsteps, "clocks": clk, "detail": detail,
     }
     if dist.rank == 0 and dist.world == 1:
-        steps_c, el_c, _ = _oracle_decode_steps(args.cpu_seconds)
+        cores = _cpu_cores()
+        steps_n, el_n = _oracle_decode_steps_threads(args.cpu_seconds, cores)
         line["cpu_baseline"] = {
+            "value": B * steps_n / el_n, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps_n} full decode steps of the same workload (write 1 token K/V for 8x8 rows + 256 "
+                      f"attention rows at kv_len 4096), the unchanged C oracle called from {cores} threads "
+                      f"(writes split by token, attention by row), {el_n:.1f} s"}
+        steps_c, el_c, _ = _oracle_decode_steps(args.cpu_seconds / 2)
+        line["cpu_baseline_1core"] = {
             "value": B * steps_c / el_c, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps_c} full decode steps of the same workload (write 1 token K/V for 8x8 rows + "
-                      f"256 attention rows at kv_len 4096), single-threaded C oracle, {el_c:.1f} s"}
+            "sample": f"{steps_c} full decode steps, single-threaded C oracle, {el_c:.1f} s"}
+        if detail:
+            _cpu_detail(detail, cores)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     del rot_graph, dec_graph, step_graphs
@@ -726,6 +892,32 @@ def _detail(args, dist, kvq, wl, layers, xk, xv, sm_fill, stream, peak):
                                          "32 q / 8 kv heads, D=128, additive mask", "us": ms * 1000,
                                  "tokens/s": sw.Lq / (ms / 1000), "TFLOP/s": fl / (ms / 1000) / 1e12,
                                  "frac": fl / (ms / 1000) / 1e12 / tpeak, "flops": fl}
+    del rings, mask
+    torch.cuda.empty_cache()
+    # chunked prefill over a per-32 block cache (MX-FP8): causal 2048-row chunk at kv_len 16384
+    Hq_b, Hkv_b, D_b, S_b, Lq_b = 32, 8, 128, 16384, 2048
+    cb = []
+    for _ in range(2):
+        xb = torch.randn((1, Hkv_b, S_b, D_b), device=dev).to(torch.bfloat16)
+        c = torch.empty((1, Hkv_b, S_b, D_b), dtype=torch.uint8, device=dev)
+        sc = torch.empty((1, Hkv_b, S_b, D_b // 32), dtype=torch.uint8, device=dev)
+        kvq.write(2, xb, torch.arange(S_b, dtype=torch.int32, device=dev), c, sc)
+        cb.append((c, sc))
+        del xb
+    qb = torch.randn((1, Hq_b, Lq_b, D_b), device=dev).to(torch.bfloat16)
+    ob = torch.empty_like(qb)
+    kvb = torch.tensor([S_b], dtype=torch.int32, device=dev)
+
+    def bpre():
+        kvq.prefill_attn_block(2, qb, *cb[0], *cb[1], kvb, out=ob, is_causal=True, mask_is_causal=True)
+    ms = _time_graph(stream, bpre, 5)
+    fl = causal_prefill_flops(Hq_b, D_b, Lq_b, S_b)
+    res["block_prefill_mxfp8"] = {"what": "kvq_prefill_attn_block mode 2 (MX-FP8 K/V, E8M0 per 32), causal chunk "
+                                          "Lq 2048 at kv_len 16384, 32 q / 8 kv heads, D=128", "us": ms * 1000,
+                                  "tokens/s": Lq_b / (ms / 1000), "TFLOP/s": fl / (ms / 1000) / 1e12,
+                                  "frac": fl / (ms / 1000) / 1e12 / tpeak, "flops": fl}
+    del cb, qb, ob
+    torch.cuda.empty_cache()
     return res
 
 
