@@ -266,11 +266,14 @@ def _oracle_decode_steps(seconds: float, min_steps: int = 1, max_steps: int | No
     return steps, el, full
 
 
-def _oracle_decode_steps_threads(seconds: float, cores: int):
-    """The decode workload's full steps on the CPU oracle, called unchanged from
-    `cores` threads (ctypes releases the GIL inside each call): the write of the
-    step's 64 K and 64 V rows split by token, the 256 attention rows by row.
-    Returns (steps, seconds)."""
+def _oracle_decode_steps_threads(seconds: float, cores: int, min_steps: int = 1, max_steps: int | None = None,
+                                 rows_per_step: int | None = None):
+    """The decode workload's steps on the CPU oracle, called unchanged from `cores`
+    threads (ctypes releases the GIL inside each call): the write of the step's 64 K
+    and 64 V rows split by batch row, the attention rows by row.  A step computes
+    `rows_per_step` of the 256 (b, h) rows (all by default; a sample cycles through
+    them).  Returns (steps, seconds, full_step_seconds), the last estimated from the
+    sample as for _oracle_decode_steps."""
     import concurrent.futures as cf
     import numpy as np
     import oracle
@@ -286,7 +289,7 @@ def _oracle_decode_steps_threads(seconds: float, cores: int):
     q = wl.u16(wl.bf16_normal((w.B, w.Hq, 1, w.D), g))
     sm = np.full(1, S - 1, np.int32)
     rows = [(b, h, 0) for b in range(w.B) for h in range(w.Hq)]
-    parts = [rows[i::cores] for i in range(cores)]
+    r = len(rows) if rows_per_step is None else max(1, min(len(rows), rows_per_step))
     oracle.build()
 
     def write_row(b):  # batch row b's token, into batch row b of the caches
@@ -297,17 +300,24 @@ def _oracle_decode_steps_threads(seconds: float, cores: int):
         if part:
             oracle.sdpa_rows(q, *K, *V, kv_len=w.kv_len, sm_scale=1 / math.sqrt(w.D), rows=part)
 
-    steps = 0
+    steps, t_write, t_attn = 0, 0.0, 0.0
     with cf.ThreadPoolExecutor(max_workers=cores) as ex:
         t0 = time.perf_counter()
         while True:
+            ta = time.perf_counter()
             list(ex.map(write_row, range(w.B)))
-            list(ex.map(attend, parts))
+            tb = time.perf_counter()
+            sel = rows if r == len(rows) else [rows[(steps * r + j) % len(rows)] for j in range(r)]
+            list(ex.map(attend, [sel[i::cores] for i in range(cores)]))
+            tc = time.perf_counter()
+            t_write += tb - ta
+            t_attn += tc - tb
             steps += 1
-            el = time.perf_counter() - t0
-            if el >= seconds:
+            el = tc - t0
+            if (steps >= min_steps and el >= seconds) or (max_steps is not None and steps >= max_steps):
                 break
-    return steps, el
+    full = (t_write + t_attn * len(rows) / r) / steps
+    return steps, el, full
 
 
 def _cpu_detail(detail, cores):
@@ -388,22 +398,24 @@ def run_reference(args, dist: Dist):
         return
     from quantized_kv_cache_20_b200 import workloads as wl
     w = wl.DECODE
-    _, _, full = _oracle_decode_steps(0.0, min_steps=1, max_steps=1)  # calibration (and build)
+    cores = _cpu_cores()
+    _, _, full = _oracle_decode_steps_threads(0.0, cores, min_steps=1, max_steps=1)  # calibration (and build)
     rows_total = w.B * w.Hq
     per_row = full / rows_total
     r = int(max(1, min(rows_total, REFERENCE_BUDGET_S / max(1, args.steps) / per_row)))
-    _oracle_decode_steps(0.0, min_steps=args.warmup, max_steps=args.warmup, rows_per_step=r)
-    steps, el, full = _oracle_decode_steps(0.0, min_steps=args.steps, max_steps=args.steps, rows_per_step=r)
+    _oracle_decode_steps_threads(0.0, cores, min_steps=args.warmup, max_steps=args.warmup, rows_per_step=r)
+    steps, el, full = _oracle_decode_steps_threads(0.0, cores, min_steps=args.steps, max_steps=args.steps,
+                                                   rows_per_step=r)
     value = w.B / full
     sample = (f"{steps} decode steps, each writing 1 token K/V for 8x8 rows and computing {r} of the 256 "
-              f"attention rows at kv_len 4096 (rows cycle); tokens/s scaled to full 256-row steps; "
-              f"single-threaded C oracle, {el:.1f} s")
+              f"attention rows at kv_len 4096 (rows cycle); tokens/s scaled to full 256-row steps; the unchanged "
+              f"C oracle called from {cores} threads, {el:.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * full,
         "measured_ms_per_sampled_step": 1000 * el / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(args),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -570,7 +582,7 @@ def run_kvq(args, dist: Dist):
     }
     if dist.rank == 0 and dist.world == 1:
         cores = _cpu_cores()
-        steps_n, el_n = _oracle_decode_steps_threads(args.cpu_seconds, cores)
+        steps_n, el_n, _ = _oracle_decode_steps_threads(args.cpu_seconds, cores)
         line["cpu_baseline"] = {
             "value": B * steps_n / el_n, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{steps_n} full decode steps of the same workload (write 1 token K/V for 8x8 rows + 256 "
