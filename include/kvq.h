@@ -51,6 +51,13 @@ extern "C" {
 #define KVQ_ERR_TIMEOUT 8      /* a bounded wait inside a kernel gave up; its output is invalid */
 
 /* Cache-write modes. */
+/* kvq_write modes.  They number cache formats, not the IndexerQuantCache page's
+ * quant_mode (参数说明: 0 MX-FP8, 1 Normal, 2 HiFloat8, 3 MX-FP4, with the cache
+ * type a separate attribute).  The page's (quant_mode, cache type) maps to:
+ *   (0, FLOAT8_E4M3FN) -> 2   (0, FLOAT8_E5M2) -> 5   (3, -) -> 3
+ *   (1, FLOAT8_E4M3FN) -> 1   (1, FLOAT8_E5M2) -> 4   (1, INT8 as uint8) -> 6
+ *   (2, HiFloat8): not built (the page names the format but does not define it).
+ * Modes 0 and 7 are the int8 and 4-bit affine caches of the other pages. */
 #define KVQ_MODE_INT8_AFFINE 0 /* int8 codes, f32 scale + int8 zero point per (token, head) */
 #define KVQ_MODE_FP8_E4M3 1    /* E4M3 codes, f32 scale per 32 elements ("Normal") */
 #define KVQ_MODE_MXFP8 2       /* E4M3 codes, E8M0 scale per 32 elements */
