@@ -177,6 +177,9 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__ WriteArgs a) {
   // launched as a programmatic dependent: read nothing before the kernel ahead has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the grid fits one wave, so every CTA is resident by now: let the next kernel's launch
+  // (a programmatic dependent, which in turn waits for this grid to complete) start
+  asm volatile("griddepcontrol.launch_dependents;");
   const uint32_t stride = gridDim.x * kThreads;
   // Every lane of a warp runs the loop the same number of times (the bound is
   // rounded up to whole warps), so the int8 mode's row shuffles see the whole
@@ -189,17 +192,14 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
     const uint32_t g = gg - (ti ? a.groups : 0u);
     const WriteTensor &wt = a.t[ti];
     int b = 0, h = 0, t = 0, gi = 0, slot = -1;
+    // The group's x is loaded together with its slot, not after it: the two loads'
+    // latencies overlap, at the price of reading the x of skipped tokens too.
+    uint32_t wx[16];  // 32 bf16 values, element 2j in the low half of wx[j]
+#pragma unroll
+    for (int j = 0; j < 16; ++j) wx[j] = 0u;
     if (gg < all) {
       group_coords(a, g, b, h, t, gi);
       const int s = __ldg(a.slot_mapping + static_cast<int64_t>(b) * a.T + t);
-      if (s != -1 && (s < 0 || s >= a.S)) {
-        if (gi == 0) report(a.err, KVQ_ERR_SLOT_RANGE);
-      } else {
-        slot = s;
-      }
-    }
-    uint32_t wx[16];  // 32 bf16 values, element 2j in the low half of wx[j]
-    if (slot >= 0) {
       const uint4 *p =
           reinterpret_cast<const uint4 *>(wt.x + b * wt.xs0 + h * wt.xs1 + static_cast<int64_t>(t) * wt.xs2 + gi * 32);
 #pragma unroll
@@ -210,7 +210,13 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const __grid_constant__
         wx[4 * k + 2] = c.z;
         wx[4 * k + 3] = c.w;
       }
-    } else {
+      if (s != -1 && (s < 0 || s >= a.S)) {
+        if (gi == 0) report(a.err, KVQ_ERR_SLOT_RANGE);
+      } else {
+        slot = s;
+      }
+    }
+    if (slot < 0) {  // skipped: the int8 mode still shuffles row statistics, over zeros
 #pragma unroll
       for (int j = 0; j < 16; ++j) wx[j] = 0u;
     }
