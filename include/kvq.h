@@ -319,7 +319,9 @@ int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint
 /*
  * kvq_decode_block_workspace_bytes -- size of the kvq_decode_attn_block workspace
  * for (B, Hq, Hkv, D, S) on the current device; 0 for sizes it rejects.  The
- * workspace holds per-split partials only and needs no initialisation.
+ * workspace must be zero-filled before its first use (its first 1 KiB holds
+ * merge counters, which every completed call leaves at zero, as for
+ * kvq_decode_attn); it can then serve later calls of any shape that fit it.
  */
 size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S);
 
@@ -337,11 +339,16 @@ size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S
  * k_codes, v_codes  u8 [B, Hkv, S, D] (mode 3: [B, Hkv, S, D/2]).
  * k_scales, v_scales  [B, Hkv, S, D/32]: float (modes 1, 4, 6) or E8M0 bytes.
  * kv_len, mask, q, out, sm_scale, err_word as for kvq_decode_attn.
- * workspace    device buffer of at least kvq_decode_block_workspace_bytes().
- * Launches two kernels on `stream` (the split attention, the merge).
+ * workspace    device buffer of at least kvq_decode_block_workspace_bytes(),
+ *              zero-filled before its first use.
+ * Modes 1, 2, 4, 5, 6 (byte codes) launch one kernel on `stream`: the split
+ * decode of kvq_decode_attn on the tensor cores (TMA tiles, in-kernel merge),
+ * with the codes converted to fp16 and multiplied by their group scale over one
+ * power of two per slot (exact for E8M0 scales; one fp16 rounding per element
+ * for float scales), that power of two applied to the fp32 score (K) or to P
+ * (V).  Mode 3 launches two kernels (a CUDA-core split attention, a merge).
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0 with Hq / Hkv <= 8; S % 16 == 0.
- * q, the codes, the scales and out 16-byte aligned (K and V tiles are staged
- * into shared memory by 16-byte asynchronous copies).
+ * q, the codes, the scales, out and the mask 16-byte aligned.
  */
 int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k_codes,
                           const void *k_scales, const uint8_t *v_codes, const void *v_scales, int64_t S,

@@ -32,6 +32,7 @@
 #include <cuda_fp16.h>
 
 #include "kvq_common.cuh"
+#include "kvq_decode_blk.h"
 
 namespace kvq {
 namespace blk {
@@ -470,12 +471,17 @@ int dispatch_mode(int mode, const Args &a, cudaStream_t s) {
 }  // namespace blk
 }  // namespace kvq
 
+// The larger of the two paths' needs: the tensor-core path (modes 1, 2, 4, 5, 6:
+// merge counters + two partial records per CTA) and the CUDA-core path (mode 3:
+// per-split partials).
 extern "C" size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S) {
   using namespace kvq;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || S % 16 != 0) return 0;
   if (D != 64 && D != 128 && D != 256) return 0;
   const blk::Split sp = blk::split_for(B, Hkv, S, sm_count());
-  return static_cast<size_t>(B) * Hkv * sp.splits * (Hq / Hkv) * (D + 2) * sizeof(float);
+  const size_t simt = static_cast<size_t>(B) * Hkv * sp.splits * (Hq / Hkv) * (D + 2) * sizeof(float);
+  const size_t mma = decode_blk_ws_bytes(Hq / Hkv, D);
+  return simt > mma ? simt : mma;
 }
 
 extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k_codes,
@@ -501,6 +507,19 @@ extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u)) return KVQ_EINVAL;
   if (static_cast<int64_t>(B) * Hkv > 65535 || B > 65535 || static_cast<int64_t>(B) * Hq > INT32_MAX)
     return KVQ_EUNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mode != KVQ_MODE_MXFP4) {  // byte codes: the tensor-core decode
+    if (mask && !aligned16(mask)) return KVQ_EINVAL;  // the mask arrives by bulk copies
+    BlkCall c{q, B, Hq, Hkv, D, k_codes, v_codes, k_scales, v_scales, S, kv_len, mask, sm_scale, out,
+              workspace, workspace_bytes, err_word, s};
+    switch (mode) {
+      case KVQ_MODE_FP8_E4M3: return decode_blk_run<KVQ_MODE_FP8_E4M3>(c);
+      case KVQ_MODE_MXFP8: return decode_blk_run<KVQ_MODE_MXFP8>(c);
+      case KVQ_MODE_FP8_E5M2: return decode_blk_run<KVQ_MODE_FP8_E5M2>(c);
+      case KVQ_MODE_MXFP8_E5M2: return decode_blk_run<KVQ_MODE_MXFP8_E5M2>(c);
+      default: return decode_blk_run<KVQ_MODE_INT8_SYM>(c);
+    }
+  }
   const blk::Split sp = blk::split_for(B, Hkv, S, sm_count());
   blk::Args a;
   a.q = static_cast<const uint16_t *>(q);
@@ -521,7 +540,6 @@ extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int
   a.splits = sp.splits;
   a.span = sp.span;
   a.qscale = sm_scale * blk::kLog2e;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
     case 64: return blk::dispatch_mode<64>(mode, a, s);
     case 128: return blk::dispatch_mode<128>(mode, a, s);

@@ -109,6 +109,9 @@ struct DecodeArgs {
   int B, Hq, Hkv, G, nhc;
   float qscale;       // sm_scale * log2(e)
   uint64_t wait_ns;   // bound on each main-loop wait
+  // block caches (kvq_write modes 1, 2, 4, 5, 6): per-32 scales [rows][D / 32], float
+  // or E8M0 bytes (k / v hold the codes; ks, vs, kz, vz unused)
+  const void *kscl, *vscl;
 };
 
 // 2-D TMA descriptors of the K and V code slabs [B * Hkv * S rows, D bytes]
@@ -122,12 +125,19 @@ struct __align__(64) KvMaps {
 // then V codes of 32 slots) and a small part (k scales, v scales, mask, k zero
 // points, v zero points); tiles are 1024-byte aligned for the TMA swizzle.
 // ---------------------------------------------------------------------------
-template <int D_, int HC_, int NW_, int R_, bool MMA_, bool Q4_, int CS_ = 32>
+template <int D_, int HC_, int NW_, int R_, bool MMA_, bool Q4_, int CS_ = 32, int MODE_ = 0>
 struct Cfg {
   static constexpr int D = D_, HC = HC_, NW = NW_, R = R_;
-  static constexpr bool MMA = MMA_;          // int8 cache on the tensor cores
+  static constexpr bool MMA = MMA_;          // int8 or block cache on the tensor cores
   static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte (CUDA cores)
   static_assert(!(MMA && Q4), "the TQ4 cache runs on the CUDA cores");
+  static constexpr int MODE = MODE_;         // kvq_write mode of the cache: 0 int8 affine, else a block mode
+  static constexpr bool BLK = MODE_ != 0;
+  static_assert(!BLK || (MMA && MODE_ != KVQ_MODE_MXFP4 && MODE_ <= KVQ_MODE_INT8_SYM),
+                "byte-coded block caches on the tensor cores");
+  static constexpr bool F32S = MODE_ == KVQ_MODE_FP8_E4M3 || MODE_ == KVQ_MODE_FP8_E5M2 || MODE_ == KVQ_MODE_INT8_SYM;
+  static constexpr int NGS = D / 32;         // scale groups of a slot (block caches)
+  static constexpr int SB = F32S ? 4 : 1;    // bytes of one group scale
   static constexpr int CB = Q4 ? D / 2 : D;  // code bytes per slot
   static constexpr int CS = CS_;             // slots per chunk
   static_assert(CS == 32 || (MMA && CS == 64), "the CUDA-core path maps 32 lanes onto 32 slots");
@@ -135,9 +145,13 @@ struct Cfg {
   static constexpr int TILE = 2 * KT;        // K tile, V tile
   static constexpr int ROWB = D < 128 ? D : 128;  // bytes of a swizzled tile row (tensor-core path)
   static constexpr int SUBT = CS_ * ROWB;         // bytes of one swizzled sub-tile
-  // small part of a buffer
-  static constexpr int KS_OFF = 0, VS_OFF = 4 * CS, M_OFF = 8 * CS, KZ_OFF = 12 * CS, VZ_OFF = 13 * CS;
-  static constexpr int SMALL = 14 * CS;
+  // small part of a buffer: int8 cache, k / v scales, mask, k / v zero points;
+  // block cache, the k / v scale rows [CS][NG] and the mask
+  static constexpr int KS_OFF = 0, VS_OFF = BLK ? CS * NGS * SB : 4 * CS;
+  static constexpr int M_OFF = BLK ? 2 * CS * NGS * SB : 8 * CS;
+  static constexpr int KZ_OFF = 12 * CS, VZ_OFF = 13 * CS;
+  static constexpr int SMALL = BLK ? M_OFF + 4 * CS : 14 * CS;
+  static_assert(VS_OFF % 16 == 0 && M_OFF % 16 == 0 && SMALL % 16 == 0, "bulk copy alignment");
   // CUDA-core path geometry
   static constexpr int L = D / 16;           // q.k: lanes per slot (16 dims per lane)
   static constexpr int NG = 32 / L;          // q.k: slot groups per warp
@@ -149,7 +163,9 @@ struct Cfg {
   // per-warp scratch: CUDA-core path, weights [HC][CS]; tensor-core path, per-slot values
   // [CS] float4 + [CS] float
   static constexpr int WBUF_OFF = SMALL_OFF + NW * R * SMALL;
-  static constexpr int WBUF_W = MMA ? CS * 20 : HC * CS * 4;  // bytes per warp
+  // block caches: (k factor, -, mask, v factor) [CS] float4, then the group factors
+  // of K and V, [NG][CS] float each
+  static constexpr int WBUF_W = BLK ? CS * 16 + 2 * NGS * CS * 4 : (MMA ? CS * 20 : HC * CS * 4);  // bytes per warp
   static constexpr int BAR_OFF = WBUF_OFF + NW * WBUF_W;     // [NW][R] mbarrier
   static constexpr int SH_OFF = (BAR_OFF + NW * R * 8 + 15) / 16 * 16;     // 8 ints
   static constexpr int Q_OFF = SH_OFF + 32;                  // [2] q slots of 2 HC D bytes
@@ -917,6 +933,397 @@ struct MmaCore {
 };
 
 // ---------------------------------------------------------------------------
+// Per-warp math of one unit over a per-32 block cache (kvq_write modes 1, 2, 4,
+// 5, 6; IndexerQuantCache, 计算公式: x ~ code * scale_g), on the tensor cores.
+//  - Codes become fp16 on the way into the MMAs, exactly (cvt for E4M3, a byte
+//    move for E5M2, the 1024-mantissa form for int8), and are multiplied by
+//    their group's factor scale_g * 2^-E_s, with 2^E_s one power of two per
+//    slot at or above the slot's largest group scale: exact for E8M0 scales
+//    (down to 2^-24 of the slot's largest factor), one rounding for float
+//    scales.  2^E_s of K multiplies the fp32 score; 2^F_s of V takes v_scale's
+//    place in P.  There is no zero point.
+//  - q.K: f16 m16n8k16 with q in rows 0..7 as exact fp16 (a power-of-two step
+//    per head; the score scale is applied in fp32).  An ldmatrix row of the K
+//    tile gives a lane four consecutive codes of one slot, so the MMA's k order
+//    is permuted to match: lane c's k pairs (2c, 2c + 1) and (2c + 8, 2c + 9)
+//    are dims 4c, 4c + 1 and 4c + 2, 4c + 3 of a 16-dim step, in q's fragments
+//    as in K's, which leaves every dot product unchanged.
+//  - Softmax and P.V as in MmaCore, the V codes converted and scaled per group.
+// ---------------------------------------------------------------------------
+template <class C>
+struct BlkCore {
+  static constexpr int D = C::D, HC = C::HC, CS = C::CS, ROWB = C::ROWB, SUBT = C::SUBT, MODE = C::MODE;
+  static constexpr int NG = C::NGS;
+  static constexpr int KT16 = D / 16;  // q.K k-steps of 16 dims
+  static constexpr int MT = D / 16;    // P.V m-tiles
+  static constexpr bool F32S = C::F32S;
+  static constexpr bool E5 = MODE == KVQ_MODE_FP8_E5M2 || MODE == KVQ_MODE_MXFP8_E5M2;
+  static constexpr bool I8 = MODE == KVQ_MODE_INT8_SYM;
+  static_assert(HC <= 8, "q heads of a unit fit the 8 MMA rows");
+  static constexpr float OSCALE = 1.0f;  // records hold O itself
+
+  uint32_t qa[KT16][2];  // q A fragment words a0, a2 (rows 8..15 carry no head)
+  int qslot;
+  float es;              // head r: qscale * the q step 2^E
+  float m, lsum, corr;   // corr stays 0 (no zero point)
+  int vexp;
+  float o[MT][4];
+  float sm_, sl_, sc_;
+  int sv_;
+  float so_[MT][4];
+
+  static __device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int db) {
+    const int st = db / ROWB, unit = (db % ROWB) >> 4;
+    const int x = ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
+    return tile + st * SUBT + row * ROWB + ((unit ^ x) << 4);
+  }
+
+  struct QRaw {
+    uint32_t w[D / 64];
+  };
+  static __device__ __forceinline__ QRaw load_q_raw(const uint16_t *qg, int lane) {
+    QRaw r;
+    if constexpr (D == 64) {
+      r.w[0] = reinterpret_cast<const uint32_t *>(qg)[lane];
+    } else if constexpr (D == 128) {
+      const uint2 v = reinterpret_cast<const uint2 *>(qg)[lane];
+      r.w[0] = v.x;
+      r.w[1] = v.y;
+    } else {
+      const uint4 v = reinterpret_cast<const uint4 *>(qg)[lane];
+      r.w[0] = v.x;
+      r.w[1] = v.y;
+      r.w[2] = v.z;
+      r.w[3] = v.w;
+    }
+    return r;
+  }
+
+  // warp `h`: head h of q as fp16 times 2^-E, max |q| 2^-E in [2^14, 2^15) (exact for
+  // every bf16 element at least 2^-24 of the step), into q slot `slot` ([HC][D] fp16);
+  // meta (0, qscale * 2^E)
+  static __device__ __forceinline__ void convert_q(uint8_t *smem, const QRaw &raw, float qscale, int slot, int h,
+                                                   int lane) {
+    constexpr int PER = D / 32;
+    float x[PER];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const uint32_t w = raw.w[i / 2];
+      x[i] = (i & 1) ? bf16hi(w) : bf16lo(w);
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int E = amax > 0.0f ? static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1 - 15 : 0;
+    E = E < -126 ? -126 : E;
+    const float inv = pow2i(-E);
+    uint32_t hw[PER / 2];
+#pragma unroll
+    for (int i = 0; i < PER / 2; ++i) hw[i] = pack_f16x2(x[2 * i] * inv, x[2 * i + 1] * inv);
+    uint8_t *hp = smem + C::Q_OFF + ((slot * HC + h) * D + lane * PER) * 2;
+    if constexpr (PER == 2) {
+      *reinterpret_cast<uint32_t *>(hp) = hw[0];
+    } else if constexpr (PER == 4) {
+      *reinterpret_cast<uint2 *>(hp) = make_uint2(hw[0], hw[1]);
+    } else {
+      *reinterpret_cast<uint4 *>(hp) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+    if (lane == 0) {
+      int32_t *meta = reinterpret_cast<int32_t *>(smem + C::QMETA_OFF) + (slot * HC + h) * 2;
+      meta[0] = 0;
+      meta[1] = static_cast<int32_t>(__float_as_uint(qscale * pow2i(E)));
+    }
+  }
+
+  __device__ __forceinline__ void load_q(const uint8_t *smem, int slot, int lane) {
+    const int r = lane >> 2, c = lane & 3;
+    const bool on = r < HC;
+    const uint8_t *qp = smem + C::Q_OFF + (slot * HC + (on ? r : 0)) * D * 2;
+#pragma unroll
+    for (int t = 0; t < KT16; ++t) {
+      const uint2 v = *reinterpret_cast<const uint2 *>(qp + (16 * t + 4 * c) * 2);
+      qa[t][0] = on ? v.x : 0u;
+      qa[t][1] = on ? v.y : 0u;
+    }
+    qslot = slot;
+    es = __int_as_float(reinterpret_cast<const int2 *>(smem + C::QMETA_OFF)[slot * HC + (on ? r : 0)].y);
+  }
+
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY;
+    lsum = 0.0f;
+    corr = 0.0f;
+    vexp = -127;
+#pragma unroll
+    for (int g = 0; g < MT; ++g)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[g][i] = 0.0f;
+  }
+
+  __device__ __forceinline__ void save() {
+    sm_ = m;
+    sl_ = lsum;
+    sc_ = corr;
+    sv_ = vexp;
+#pragma unroll
+    for (int g = 0; g < MT; ++g)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) so_[g][i] = o[g][i];
+  }
+
+  // four codes (byte i = code i) -> fp16 pairs (codes 0, 1) and (2, 3), exact
+  static __device__ __forceinline__ void codes4(uint32_t w, uint32_t &h01, uint32_t &h23) {
+    if constexpr (E5) {
+      h01 = __byte_perm(w, 0u, 0x1404);
+      h23 = __byte_perm(w, 0u, 0x3424);
+    } else if constexpr (I8) {
+      const uint32_t u = w ^ 0x80808080u;
+      h01 = sub1152(__byte_perm(u, 0x64646464u, 0x4140));
+      h23 = sub1152(__byte_perm(u, 0x64646464u, 0x4342));
+    } else {
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(static_cast<uint16_t>(w >> 16)));
+    }
+  }
+  // codes in bytes 0 and 2 (ev) or 1 and 3 (od) of w -> one fp16 pair, exact
+  template <bool ODD>
+  static __device__ __forceinline__ uint32_t codes2(uint32_t w) {
+    if constexpr (E5) {
+      return __byte_perm(w, 0u, ODD ? 0x3414 : 0x2404);
+    } else if constexpr (I8) {
+      return sub1152(__byte_perm(w ^ 0x80808080u, 0x64646464u, ODD ? 0x4341 : 0x4240));
+    } else {
+      uint32_t h;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(__byte_perm(w, 0u, ODD ? 0x0031 : 0x0020))));
+      return h;
+    }
+  }
+  static __device__ __forceinline__ uint32_t sub1152(uint32_t h) {
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2 *>(&h),
+                              __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+    return *reinterpret_cast<const uint32_t *>(&r);
+  }
+  // an fp16 pair times (f0, f1): E8M0 factors are powers of two (exact product);
+  // float factors take the pair through fp32 and round once
+  static __device__ __forceinline__ uint32_t scale2(uint32_t h, float f0, float f1) {
+    if constexpr (F32S) {
+      const float2 v = unpack_f16x2(h);
+      return pack_f16x2(v.x * f0, v.y * f1);
+    } else {
+      const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&h), __floats2half2_rn(f0, f1));
+      return *reinterpret_cast<const uint32_t *>(&r);
+    }
+  }
+  // the exponent of a slot and its group factors scale_g * 2^-E, from the slot's
+  // scale row (NG floats, or NG E8M0 bytes)
+  static __device__ __forceinline__ int slot_factors(const uint8_t *row, float (&f)[NG]) {
+    if constexpr (F32S) {
+      uint32_t mx = 0u;
+      float sg[NG];
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        sg[g] = reinterpret_cast<const float *>(row)[g];
+        mx = max(mx, __float_as_uint(sg[g]) & 0x7FFFFFFFu);
+      }
+      int E = 0;
+      if (mx != 0u) {  // ceil(log2) of the largest scale, from its bits
+        const int ex = static_cast<int>(mx >> 23);
+        E = ex == 0 ? -126 : ex - 127 + ((mx & 0x7FFFFFu) != 0u ? 1 : 0);
+        E = E < -126 ? -126 : (E > 126 ? 126 : E);
+      }
+      const float inv = pow2i(-E);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) f[g] = sg[g] * inv;
+      return E;
+    } else {
+      int e[NG], mx = 0;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        e[g] = row[g];
+        mx = max(mx, e[g]);
+      }
+      const int E = max(-126, mx - 127);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const int k = e[g] - 127 - E;  // <= 0
+        f[g] = k >= -126 ? pow2i(k) : 0.0f;
+      }
+      return E;
+    }
+  }
+
+  __device__ __forceinline__ void chunk(const uint8_t *smem, const uint8_t *tile, const uint8_t *small, float *scr,
+                                        int s0, int kv_u, bool has_mask, int lane) {
+    constexpr int NT = CS / 8;   // q.K n-tiles (8 slots each)
+    constexpr int PK = CS / 16;  // P.V k-steps (16 slots each)
+    constexpr int RB = NG * C::SB;
+    const int r = lane >> 2, c = lane & 3;
+    const uint32_t kt = smem_u32(tile), vt = kt + C::KT;
+    float4 *s4 = reinterpret_cast<float4 *>(scr);  // [CS] (k factor, -, mask, v factor)
+    float *kf = scr + 4 * CS;                      // [NG][CS] K group factors
+    float *vf = kf + NG * CS;                      // [NG][CS] V group factors
+    // ---- per-slot factors, one lane per slot (0 past kv_len, where the mask is -inf)
+    float vmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < CS / 32; ++i) {
+      const int j = lane + 32 * i;
+      const bool valid = s0 + j < kv_u;
+      float fk[NG], fv[NG];
+      const int ek = slot_factors(small + C::KS_OFF + j * RB, fk);
+      const int ev = slot_factors(small + C::VS_OFF + j * RB, fv);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        kf[g * CS + j] = valid ? fk[g] : 0.0f;
+        vf[g * CS + j] = valid ? fv[g] : 0.0f;
+      }
+      const float mk = has_mask ? reinterpret_cast<const float *>(small + C::M_OFF)[j] * kLog2e : 0.0f;
+      float4 f;
+      f.x = valid ? pow2i(ek) : 0.0f;
+      f.y = 0.0f;
+      f.z = valid ? mk : -INFINITY;
+      f.w = valid ? pow2i(ev) : 0.0f;
+      s4[j] = f;
+      vmax = fmaxf(vmax, f.w);
+    }
+#pragma unroll
+    for (int sft = 16; sft >= 1; sft >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, sft));
+    __syncwarp();  // the factors are written
+    // ---- q.K: n-tile nt = slots 8 nt .. 8 nt + 7; ldmatrix x4 gives four 16-dim
+    // steps (64 dims) of one n-tile, lane (r, c) holding dims 4c .. 4c + 3 of slot r
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.0f;
+#pragma unroll
+      for (int kp = 0; kp < D / 64; ++kp) {
+        uint32_t b[4];
+        ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = 4 * kp + i;
+          const float f = kf[(t >> 1) * CS + nt * 8 + r];
+          uint32_t b0, b1;
+          codes4(b[i], b0, b1);
+          b0 = scale2(b0, f, f);
+          b1 = scale2(b1, f, f);
+          const uint32_t a[4] = {qa[t][0], 0u, qa[t][1], 0u};
+          mma_f16(sacc[nt], a, b0, b1);
+        }
+      }
+    }
+    // ---- scores of head r at slots j = 8 nt + 2c + e (log2 domain)
+    float sc[NT][2], vv[NT][2];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int j = nt * 8 + 2 * c;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4 f = s4[j + e];
+        sc[nt][e] = fmaf(sacc[nt][e], es * f.x, f.z);  // -inf past kv_len (k factor 0 there)
+        vv[nt][e] = f.w;
+        mt = fmaxf(mt, sc[nt][e]);
+      }
+    }
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+    const bool need = r < HC && mt > m + kRescaleThreshold;
+    if (__any_sync(0xffffffffu, need)) {
+      const float alpha = need ? (m == -INFINITY ? 0.0f : ex2(m - mt)) : 1.0f;
+      if (need) {
+        lsum *= alpha;
+        m = mt;
+      }
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c + 4);
+#pragma unroll
+      for (int g = 0; g < MT; ++g) {
+        o[g][0] *= a0;
+        o[g][1] *= a1;
+        o[g][2] *= a0;
+        o[g][3] *= a1;
+      }
+    }
+    // weights w = p * 2^F * 2^-E_v below 2^15 (p <= 2^8); E_v only grows
+    if (vmax > 0.0f) {
+      int evx = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xFF) - 127 - 6;
+      evx = evx < -120 ? -120 : (evx > 120 ? 120 : evx);
+      if (evx > vexp) {
+        const float f = vexp - evx < -126 ? 0.0f : pow2i(vexp - evx);
+#pragma unroll
+        for (int g = 0; g < MT; ++g)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[g][i] *= f;
+        vexp = evx;
+      }
+    }
+    const float vsc = r < HC ? pow2i(-vexp) : 0.0f;
+    const float mm = r < HC ? (m == -INFINITY ? 0.0f : m) : INFINITY;
+    uint32_t ph[NT], pl[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float w[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float p = ex2(sc[nt][e] - mm);
+        lsum += p;
+        w[e] = p * (vv[nt][e] * vsc);
+      }
+      ph[nt] = pack_f16x2(w[0], w[1]);
+      const float2 back = unpack_f16x2(ph[nt]);
+      pl[nt] = pack_f16x2(w[0] - back.x, w[1] - back.y);
+    }
+    // ---- P.V: k-step ks = slots 16 ks .. 16 ks + 15, m-tile pair gp = dims 32 gp ..
+    // 32 gp + 31 (one scale group)
+#pragma unroll
+    for (int ks = 0; ks < PK; ++ks) {
+#pragma unroll
+      for (int gp = 0; gp < MT / 2; ++gp) {
+        uint32_t mr[4];
+        const int mi = lane >> 3;
+        ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
+        // factors of slots 16 ks + 2c, + 1 (matrices 0, 2) and 16 ks + 8 + 2c, + 1 (1, 3)
+        const float2 fa = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 2 * c);
+        const float2 fb = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 8 + 2 * c);
+        uint32_t af[2][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 ff = (i & 1) ? fb : fa;
+          af[i >> 1][(i & 1) * 2 + 0] = scale2(codes2<false>(mr[i]), ff.x, ff.y);  // dim 2r of the two slots
+          af[i >> 1][(i & 1) * 2 + 1] = scale2(codes2<true>(mr[i]), ff.x, ff.y);   // dim 2r + 1
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t a[4] = {af[t][0], af[t][1], af[t][2], af[t][3]};
+          mma_f16(o[2 * gp + t], a, ph[2 * ks], ph[2 * ks + 1]);
+          mma_f16(o[2 * gp + t], a, pl[2 * ks], pl[2 * ks + 1]);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void publish(float *dst, bool first, int lane) {
+    const int r = lane >> 2, c = lane & 3;
+    float ll = first ? sl_ : lsum;
+    ll += __shfl_xor_sync(0xffffffffu, ll, 1);
+    ll += __shfl_xor_sync(0xffffffffu, ll, 2);
+    const float sv = pow2i(first ? sv_ : vexp);
+#pragma unroll
+    for (int g = 0; g < MT; ++g) {
+      const float *og = first ? so_[g] : o[g];
+      const int d = 16 * g + 2 * r;
+      if (2 * c < HC) *reinterpret_cast<float2 *>(dst + (2 * c) * D + d) = make_float2(og[0] * sv, og[2] * sv);
+      if (2 * c + 1 < HC)
+        *reinterpret_cast<float2 *>(dst + (2 * c + 1) * D + d) = make_float2(og[1] * sv, og[3] * sv);
+    }
+    if (r < HC && c == 0)
+      *reinterpret_cast<float4 *>(dst + HC * D + r * 4) = make_float4(first ? sm_ : m, ll, 0.0f, 0.0f);
+  }
+};
+
+// ---------------------------------------------------------------------------
 // The kernel: work split, chunk rings, unit close and split merge.
 // VARLEN: kv_len is one value per batch row (a.kv_per_batch); the scalar form
 // is a separate instantiation so it carries no per-unit state.
@@ -924,7 +1331,8 @@ struct MmaCore {
 template <class C, bool VARLEN>
 __global__ void __launch_bounds__(C::THREADS, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ KvMaps maps) {
-  using Core = typename std::conditional<C::MMA, MmaCore<C>, SimtCore<C>>::type;
+  using Core = typename std::conditional<C::BLK, BlkCore<C>,
+                                         typename std::conditional<C::MMA, MmaCore<C>, SimtCore<C>>::type>::type;
   constexpr int D = C::D, HC = C::HC, NW = C::NW, R = C::R, CS = C::CS, CB = C::CB;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   // the tiles start at the first 1024-byte boundary (TMA swizzle atoms)
@@ -967,10 +1375,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       case 5: p = a.ws_ml + 4 * static_cast<int64_t>(blockIdx.x) * HC; break;
       case 6: p = a.k + row * CB; break;
       case 7: p = a.v + row * CB; break;
-      case 8: p = a.ks + row; break;
-      case 9: p = a.vs + row; break;
-      case 10: p = a.kz + row; break;
-      case 11: p = a.vz + row; break;
+      case 8: p = C::BLK ? static_cast<const uint8_t *>(a.kscl) + row * C::NGS * C::SB : (const void *)(a.ks + row); break;
+      case 9: p = C::BLK ? static_cast<const uint8_t *>(a.vscl) + row * C::NGS * C::SB : (const void *)(a.vs + row); break;
+      case 10: p = C::BLK ? nullptr : a.kz + row; break;
+      case 11: p = C::BLK ? nullptr : a.vz + row; break;
       case 12: p = a.mask; break;
       default: break;
     }
@@ -1103,7 +1511,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint8_t *small = smalls + rb * C::SMALL;
     uint64_t *bar = bars + rb;
     const uint32_t code_bytes = n16 == 0 ? 0u : (C::MMA ? 2u * C::KT : static_cast<uint32_t>(n16) * 2 * CB);
-    mbar_arrive_expect_tx(bar, code_bytes + static_cast<uint32_t>(n16) * 10 + (a.mask ? 4u * n16 : 0u));
+    const uint32_t small_bytes = static_cast<uint32_t>(n16) * (C::BLK ? 2 * C::NGS * C::SB : 10);
+    mbar_arrive_expect_tx(bar, code_bytes + small_bytes + (a.mask ? 4u * n16 : 0u));
     if (n16 > 0) {  // 0 bytes: the expect_tx above is a plain arrival
       const int64_t row = ibase + s0;
       if constexpr (C::MMA) {  // full CS-row boxes (rows past the slab read as zeros, past kv_len are masked)
@@ -1116,10 +1525,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         bulk_g2s_hint(tile, a.k + row * CB, n16 * CB, bar, pol);
         bulk_g2s_hint(tile + C::KT, a.v + row * CB, n16 * CB, bar, pol);
       }
-      bulk_g2s(small + C::KS_OFF, a.ks + row, n16 * 4, bar);
-      bulk_g2s(small + C::VS_OFF, a.vs + row, n16 * 4, bar);
-      bulk_g2s(small + C::KZ_OFF, a.kz + row, n16, bar);
-      bulk_g2s(small + C::VZ_OFF, a.vz + row, n16, bar);
+      if constexpr (C::BLK) {
+        constexpr int RB = C::NGS * C::SB;  // scale bytes of a slot
+        bulk_g2s(small + C::KS_OFF, static_cast<const uint8_t *>(a.kscl) + row * RB, n16 * RB, bar);
+        bulk_g2s(small + C::VS_OFF, static_cast<const uint8_t *>(a.vscl) + row * RB, n16 * RB, bar);
+      } else {
+        bulk_g2s(small + C::KS_OFF, a.ks + row, n16 * 4, bar);
+        bulk_g2s(small + C::VS_OFF, a.vs + row, n16 * 4, bar);
+        bulk_g2s(small + C::KZ_OFF, a.kz + row, n16, bar);
+        bulk_g2s(small + C::VZ_OFF, a.vz + row, n16, bar);
+      }
       if (a.mask) bulk_g2s(small + C::M_OFF, imask + s0, n16 * 4, bar);
     }
     outstanding |= 1u << rb;
@@ -1441,16 +1856,18 @@ int head_chunk_simt(int G) { return G % 4 == 0 ? 4 : (G % 3 == 0 ? 3 : (G % 2 ==
 // beat six with two (two sub-partitions then run one warp alone) at D <= 128.
 // CUDA-core path: q (8 words per head), accumulators (2 x D/32 per head) and
 // q.k partials (D/16 per head).  The ring takes what shared memory is left.
-template <int D, int HC, bool MMA, bool Q4>
+template <int D, int HC, bool MMA, bool Q4, int MODE = 0>
 struct Tune {
   // tensor-core path: 64-slot chunks up to D = 128 (two chunks' worth of independent
   // MMAs and scores per warp step, fixed costs per chunk halved), 32 for D = 256
   static constexpr int CS = MMA && D <= 128 ? 64 : 32;
-  static constexpr int NW = MMA ? (D == 256 ? 6 : 8)
+  static constexpr int NW = MMA ? (D == 256 ? (MODE ? 4 : 6) : 8)  // block caches at D = 256: two buffers a warp
                                 : (D == 256 ? 8 : (D == 128 ? (HC <= 2 ? 16 : 12) : 16));
   static constexpr int CB = Q4 ? D / 2 : D;
-  static constexpr int PER_BUF = 2 * CS * CB + 14 * CS;
-  static constexpr int FIXED = (MMA ? 1024 + NW * CS * 20 : NW * HC * 128) + NW * 4 * 8 + 64 + 4 * HC * D +
+  static constexpr int SBB = MODE == KVQ_MODE_FP8_E4M3 || MODE == KVQ_MODE_FP8_E5M2 || MODE == KVQ_MODE_INT8_SYM ? 4 : 1;
+  static constexpr int PER_BUF = 2 * CS * CB + (MODE ? 2 * CS * (D / 32) * SBB + 4 * CS : 14 * CS);
+  static constexpr int WB = MODE ? CS * 16 + 2 * (D / 32) * CS * 4 : CS * 20;
+  static constexpr int FIXED = (MMA ? 1024 + NW * WB : NW * HC * 128) + NW * 4 * 8 + 64 + 4 * HC * D +
                                16 * HC + 8 * kMaxCtas + 4 * (kMaxRows + 33) + 8 * (NW + 3) * HC;
   static constexpr int RMAX = (232448 - FIXED) / (NW * PER_BUF);
   static constexpr int R = RMAX > 4 ? 4 : RMAX;
@@ -1511,10 +1928,10 @@ int make_code_map(CUtensorMap *map, const void *base, int D, int64_t rows, int b
 template <class C, bool VARLEN>
 struct KernelTag {};  // names one decode_kernel instantiation for ensure_smem
 
-template <int D, int HC, bool MMA, bool Q4>
+template <int D, int HC, bool MMA, bool Q4, int MODE = 0>
 int launch_decode(const DecodeArgs &a, const KvMaps &maps, int ctas, cudaStream_t stream) {
-  using T = Tune<D, HC, MMA, Q4>;
-  using C = Cfg<D, HC, T::NW, T::R, MMA, Q4, T::CS>;
+  using T = Tune<D, HC, MMA, Q4, MODE>;
+  using C = Cfg<D, HC, T::NW, T::R, MMA, Q4, T::CS, MODE>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1548,6 +1965,29 @@ int dispatch_mma(const DecodeArgs &a, const KvMaps &maps, int hc, int ctas, cuda
     case 6: return launch_decode<D, 6, true, false>(a, maps, ctas, s);
     case 7: return launch_decode<D, 7, true, false>(a, maps, ctas, s);
     default: return launch_decode<D, 8, true, false>(a, maps, ctas, s);
+  }
+}
+
+// block caches of byte codes (kvq_write modes 1, 2, 4, 5, 6)
+template <int D, int MODE>
+int dispatch_blk(const DecodeArgs &a, const KvMaps &maps, int hc, int ctas, cudaStream_t s) {
+  switch (hc) {
+    case 1: return launch_decode<D, 1, true, false, MODE>(a, maps, ctas, s);
+    case 2: return launch_decode<D, 2, true, false, MODE>(a, maps, ctas, s);
+    case 3: return launch_decode<D, 3, true, false, MODE>(a, maps, ctas, s);
+    case 4: return launch_decode<D, 4, true, false, MODE>(a, maps, ctas, s);
+    case 5: return launch_decode<D, 5, true, false, MODE>(a, maps, ctas, s);
+    case 6: return launch_decode<D, 6, true, false, MODE>(a, maps, ctas, s);
+    case 7: return launch_decode<D, 7, true, false, MODE>(a, maps, ctas, s);
+    default: return launch_decode<D, 8, true, false, MODE>(a, maps, ctas, s);
+  }
+}
+template <int MODE>
+int dispatch_blk_mode(const DecodeArgs &a, const KvMaps &maps, int D, int hc, int ctas, cudaStream_t s) {
+  switch (D) {
+    case 64: return dispatch_blk<64, MODE>(a, maps, hc, ctas, s);
+    case 128: return dispatch_blk<128, MODE>(a, maps, hc, ctas, s);
+    default: return dispatch_blk<256, MODE>(a, maps, hc, ctas, s);
   }
 }
 

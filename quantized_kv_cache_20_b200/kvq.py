@@ -352,7 +352,7 @@ def decode_attn_block(mode: int, q, k_codes, k_scales, v_codes, v_scales, kv_len
     if workspace is None:
         nbytes = int(load().kvq_decode_block_workspace_bytes(B, Hq, Hkv, D, S))
         with torch.cuda.device(q.device):
-            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+            workspace = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     st = load().kvq_decode_attn_block(int(mode), _ptr(q), B, Hq, Hkv, D, _ptr(k_codes), _ptr(k_scales),
                                       _ptr(v_codes), _ptr(v_scales), S, _ptr(kv_len), _ptr(mask),
                                       float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
