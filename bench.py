@@ -45,7 +45,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # taken on: the line reports the figure only while the source is unchanged (else null).
 DECODE_TRAFFIC_BYTES = 70780160  # 69,880,320 read + 899,840 written; algorithmic 69,861,376
 DECODE_TRAFFIC_SRC_SHA256 = "b75dca97a135dfec007a6997c0e450f578e1a5b9e0302017ea6052dd2d3fecf1"
-DECODE_SRC = ("quantized_kv_cache_20_b200/csrc/kvq_decode.cu", "quantized_kv_cache_20_b200/csrc/kvq_common.cuh")
+DECODE_SRC = ("quantized_kv_cache_20_b200/csrc/kvq_decode.cu", "quantized_kv_cache_20_b200/csrc/kvq_decode_kernel.cuh",
+              "quantized_kv_cache_20_b200/csrc/kvq_common.cuh")
 
 
 def decode_source_sha256() -> str:

@@ -341,12 +341,13 @@ size_t kvq_decode_block_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t S
  * kv_len, mask, q, out, sm_scale, err_word as for kvq_decode_attn.
  * workspace    device buffer of at least kvq_decode_block_workspace_bytes(),
  *              zero-filled before its first use.
- * Modes 1, 2, 4, 5, 6 (byte codes) launch one kernel on `stream`: the split
- * decode of kvq_decode_attn on the tensor cores (TMA tiles, in-kernel merge),
- * with the codes converted to fp16 and multiplied by their group scale over one
- * power of two per slot (exact for E8M0 scales; one fp16 rounding per element
- * for float scales), that power of two applied to the fp32 score (K) or to P
- * (V).  Mode 3 launches two kernels (a CUDA-core split attention, a merge).
+ * Modes 1, 2, 4, 5, 6, and mode 3 at D >= 128, launch one kernel on `stream`:
+ * the split decode of kvq_decode_attn on the tensor cores (TMA tiles, in-kernel
+ * merge), with the codes converted to fp16 and multiplied by their group scale
+ * over one power of two per slot (exact for E8M0 scales; one fp16 rounding per
+ * element for float scales), that power of two applied to the fp32 score (K) or
+ * to P (V).  Mode 3 at D = 64 launches two kernels (a CUDA-core split
+ * attention, a merge).
  * Sizes: D in {64, 128, 256}; Hq % Hkv == 0 with Hq / Hkv <= 8; S % 16 == 0.
  * q, the codes, the scales, out and the mask 16-byte aligned.
  */

@@ -1,5 +1,5 @@
-// kvq_decode_blk.cuh -- the launch of the tensor-core decode over a byte-coded block
-// cache, shared by the per-mode translation units.
+// kvq_decode_blk.cuh -- the launch of the tensor-core decode over a block cache,
+// shared by the per-mode translation units.
 #pragma once
 
 #include <cstring>
@@ -50,8 +50,9 @@ int decode_blk_run_impl(const BlkCall &c) {
   std::memset(&maps, 0, sizeof(maps));
   const int64_t rows = static_cast<int64_t>(c.B) * c.Hkv * c.S;
   const int box_rows = c.D <= 128 ? 64 : 32;  // the tensor-core path's chunk (Tune::CS)
-  if (const int st = make_code_map(&maps.k, c.k_codes, c.D, rows, box_rows)) return st;
-  if (const int st = make_code_map(&maps.v, c.v_codes, c.D, rows, box_rows)) return st;
+  const int row_bytes = MODE == KVQ_MODE_MXFP4 ? c.D / 2 : c.D;  // E2M1: two codes a byte
+  if (const int st = make_code_map(&maps.k, c.k_codes, row_bytes, rows, box_rows)) return st;
+  if (const int st = make_code_map(&maps.v, c.v_codes, row_bytes, rows, box_rows)) return st;
   return dispatch_blk_mode<MODE>(a, maps, c.D, hc, ctas, c.stream);
 }
 

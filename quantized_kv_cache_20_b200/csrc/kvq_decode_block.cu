@@ -508,13 +508,14 @@ extern "C" int kvq_decode_attn_block(int mode, const void *q, int B, int Hq, int
   if (static_cast<int64_t>(B) * Hkv > 65535 || B > 65535 || static_cast<int64_t>(B) * Hq > INT32_MAX)
     return KVQ_EUNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (mode != KVQ_MODE_MXFP4) {  // byte codes: the tensor-core decode
+  if (mode != KVQ_MODE_MXFP4 || D >= 128) {  // the tensor-core decode (E2M1 codes from D = 128)
     if (mask && !aligned16(mask)) return KVQ_EINVAL;  // the mask arrives by bulk copies
     BlkCall c{q, B, Hq, Hkv, D, k_codes, v_codes, k_scales, v_scales, S, kv_len, mask, sm_scale, out,
               workspace, workspace_bytes, err_word, s};
     switch (mode) {
       case KVQ_MODE_FP8_E4M3: return decode_blk_run<KVQ_MODE_FP8_E4M3>(c);
       case KVQ_MODE_MXFP8: return decode_blk_run<KVQ_MODE_MXFP8>(c);
+      case KVQ_MODE_MXFP4: return decode_blk_run<KVQ_MODE_MXFP4>(c);
       case KVQ_MODE_FP8_E5M2: return decode_blk_run<KVQ_MODE_FP8_E5M2>(c);
       case KVQ_MODE_MXFP8_E5M2: return decode_blk_run<KVQ_MODE_MXFP8_E5M2>(c);
       default: return decode_blk_run<KVQ_MODE_INT8_SYM>(c);

@@ -18,12 +18,16 @@
 // too small for tcgen05's 64/128-row tiles), leaving the CUDA cores the
 // softmax bookkeeping:
 //  - Persistent grid: one CTA per SM.  The work -- units (b, kv head, head
-//    chunk of HC q heads) x chunks of 32 slots, with the chunk count derived
+//    chunk of HC q heads) x chunks of CS slots, with the chunk count derived
 //    on the device from *kv_len -- is flattened and cut into equal contiguous
 //    ranges, one per CTA, so every SM streams the same bytes (to one chunk)
 //    whatever B, Hkv and kv_len are.  With one kv_len per batch row the
 //    flattening uses each row's own length (a prefix of the rows' chunk counts
-//    in shared memory).
+//    in shared memory).  With one kv_len, when the units divide the grid into
+//    k >= 1 CTAs each at no cost in rounds of chunks per warp, only those U k
+//    CTAs stream, each a k-th of one unit: a warp's time is set by its rounds
+//    of chunks (copy latency, then compute), and a CTA confined to one unit
+//    skips the second combine and the three-owner merges of the flattened cut.
 //  - Every warp is its own pipeline: chunk i of the CTA's range belongs to
 //    warp i mod NW, whose R-deep ring of chunk buffers is filled by async
 //    copies -- K and V tiles by 2-D TMA with the 128-byte (64-byte for D = 64)
@@ -133,17 +137,17 @@ struct Cfg {
   static_assert(!(MMA && Q4), "the TQ4 cache runs on the CUDA cores");
   static constexpr int MODE = MODE_;         // kvq_write mode of the cache: 0 int8 affine, else a block mode
   static constexpr bool BLK = MODE_ != 0;
-  static_assert(!BLK || (MMA && MODE_ != KVQ_MODE_MXFP4 && MODE_ <= KVQ_MODE_INT8_SYM),
-                "byte-coded block caches on the tensor cores");
+  static_assert(!BLK || (MMA && MODE_ <= KVQ_MODE_INT8_SYM && (MODE_ != KVQ_MODE_MXFP4 || D_ >= 128)),
+                "block caches on the tensor cores (MX-FP4 from D = 128)");
   static constexpr bool F32S = MODE_ == KVQ_MODE_FP8_E4M3 || MODE_ == KVQ_MODE_FP8_E5M2 || MODE_ == KVQ_MODE_INT8_SYM;
   static constexpr int NGS = D / 32;         // scale groups of a slot (block caches)
   static constexpr int SB = F32S ? 4 : 1;    // bytes of one group scale
-  static constexpr int CB = Q4 ? D / 2 : D;  // code bytes per slot
+  static constexpr int CB = Q4 || MODE_ == KVQ_MODE_MXFP4 ? D / 2 : D;  // code bytes per slot
   static constexpr int CS = CS_;             // slots per chunk
   static_assert(CS == 32 || (MMA && CS == 64), "the CUDA-core path maps 32 lanes onto 32 slots");
   static constexpr int KT = CS * CB;         // one tile of codes
   static constexpr int TILE = 2 * KT;        // K tile, V tile
-  static constexpr int ROWB = D < 128 ? D : 128;  // bytes of a swizzled tile row (tensor-core path)
+  static constexpr int ROWB = CB < 128 ? CB : 128;  // bytes of a swizzled tile row (tensor-core path)
   static constexpr int SUBT = CS_ * ROWB;         // bytes of one swizzled sub-tile
   // small part of a buffer: int8 cache, k / v scales, mask, k / v zero points;
   // block cache, the k / v scale rows [CS][NG] and the mask
@@ -210,6 +214,18 @@ KVQ_DEVINL int count_acq_rel(int32_t *p) {
 // Work split: CTA c owns flattened chunks [c*W/C, (c+1)*W/C); cta_of is its inverse.
 KVQ_DEVINL int64_t range_start(int64_t c, int64_t W, int64_t C) { return c * W / C; }
 KVQ_DEVINL int64_t cta_of(int64_t idx, int64_t W, int64_t C) { return ((idx + 1) * C - 1) / W; }
+// CTAs that take part when every one of the U units has nch chunks: all CT0 of the
+// grid (the flattened split), or U * k of them, k = floor(CT0 / U), when that costs a
+// warp no more rounds of chunks (a warp takes every NW-th chunk of its CTA).  With
+// U * k CTAs the range of CTA c lies inside unit floor(c / k), so a CTA never combines
+// two units and a unit has exactly k owners (none to merge when k = 1).
+KVQ_DEVINL int64_t active_ctas(int64_t U, int64_t nch, int64_t CT0, int NW) {
+  const int64_t k = CT0 / U;
+  if (k < 1) return CT0;
+  const int64_t rounds_all = ((U * nch + CT0 - 1) / CT0 + NW - 1) / NW;
+  const int64_t rounds_units = ((nch + k - 1) / k + NW - 1) / NW;
+  return rounds_units <= rounds_all ? U * k : CT0;
+}
 
 // One probe of the phase, suspending the thread for at most `hint_ns`.
 KVQ_DEVINL bool mbar_try_wait_ns(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
@@ -959,6 +975,9 @@ struct BlkCore {
   static constexpr bool F32S = C::F32S;
   static constexpr bool E5 = MODE == KVQ_MODE_FP8_E5M2 || MODE == KVQ_MODE_MXFP8_E5M2;
   static constexpr bool I8 = MODE == KVQ_MODE_INT8_SYM;
+  // MX-FP4: two E2M1 codes a byte (element 2i in the low nibble of byte i), so a
+  // 16-byte ldmatrix row holds 32 dims, one scale group
+  static constexpr bool FP4 = MODE == KVQ_MODE_MXFP4;
   static_assert(HC <= 8, "q heads of a unit fit the 8 MMA rows");
   static constexpr float OSCALE = 1.0f;  // records hold O itself
 
@@ -1040,11 +1059,22 @@ struct BlkCore {
     const int r = lane >> 2, c = lane & 3;
     const bool on = r < HC;
     const uint8_t *qp = smem + C::Q_OFF + (slot * HC + (on ? r : 0)) * D * 2;
+    if constexpr (FP4) {  // k-steps 2u, 2u + 1 of group u: lane c takes dims 32 u + 8 c .. + 7
 #pragma unroll
-    for (int t = 0; t < KT16; ++t) {
-      const uint2 v = *reinterpret_cast<const uint2 *>(qp + (16 * t + 4 * c) * 2);
-      qa[t][0] = on ? v.x : 0u;
-      qa[t][1] = on ? v.y : 0u;
+      for (int u = 0; u < D / 32; ++u) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(qp + (32 * u + 8 * c) * 2);
+        qa[2 * u][0] = on ? v.x : 0u;
+        qa[2 * u][1] = on ? v.y : 0u;
+        qa[2 * u + 1][0] = on ? v.z : 0u;
+        qa[2 * u + 1][1] = on ? v.w : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < KT16; ++t) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(qp + (16 * t + 4 * c) * 2);
+        qa[t][0] = on ? v.x : 0u;
+        qa[t][1] = on ? v.y : 0u;
+      }
     }
     qslot = slot;
     es = __int_as_float(reinterpret_cast<const int2 *>(smem + C::QMETA_OFF)[slot * HC + (on ? r : 0)].y);
@@ -1098,6 +1128,20 @@ struct BlkCore {
       asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(__byte_perm(w, 0u, ODD ? 0x0031 : 0x0020))));
       return h;
     }
+  }
+  // the E2M1 codes in the low byte of w -> fp16 pair (low nibble first), exact
+  static __device__ __forceinline__ uint32_t e2m1x2(uint32_t w) {
+    uint32_t h;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h) : "r"(w));
+    return h;
+  }
+  // ldmatrix.trans word of E2M1 codes: dims 4i .. 4i + 3 of slot s (bytes 0, 1) and
+  // of slot s + 1 (bytes 2, 3) -> byte j holds dim 4i + j of slot s (low nibble) and
+  // of slot s + 1 (high nibble)
+  static __device__ __forceinline__ uint32_t fp4_slot_pairs(uint32_t w) {
+    const uint32_t x = __byte_perm(w, 0u, 0x3120);    // bytes: s lo, s+1 lo, s hi, s+1 hi
+    const uint32_t t = ((x >> 4) ^ x) & 0x00F000F0u;  // swap the middle nibbles of each half
+    return x ^ t ^ (t << 4);
   }
   static __device__ __forceinline__ uint32_t sub1152(uint32_t h) {
     const __half2 r = __hsub2(*reinterpret_cast<const __half2 *>(&h),
@@ -1196,20 +1240,40 @@ struct BlkCore {
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.0f;
+      if constexpr (FP4) {  // matrix i of an ldmatrix x4: scale group u = 4 kp + i, lane c: dims 8 c .. 8 c + 7
 #pragma unroll
-      for (int kp = 0; kp < D / 64; ++kp) {
-        uint32_t b[4];
-        ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
+        for (int kp = 0; kp < D / 128; ++kp) {
+          uint32_t b[4];
+          ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = 4 * kp + i;
-          const float f = kf[(t >> 1) * CS + nt * 8 + r];
-          uint32_t b0, b1;
-          codes4(b[i], b0, b1);
-          b0 = scale2(b0, f, f);
-          b1 = scale2(b1, f, f);
-          const uint32_t a[4] = {qa[t][0], 0u, qa[t][1], 0u};
-          mma_f16(sacc[nt], a, b0, b1);
+          for (int i = 0; i < 4; ++i) {
+            const int u = 4 * kp + i;
+            const float f = kf[u * CS + nt * 8 + r];
+            uint32_t h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = scale2(e2m1x2(b[i] >> (8 * j)), f, f);
+            const uint32_t a0[4] = {qa[2 * u][0], 0u, qa[2 * u][1], 0u};
+            mma_f16(sacc[nt], a0, h[0], h[1]);
+            const uint32_t a1[4] = {qa[2 * u + 1][0], 0u, qa[2 * u + 1][1], 0u};
+            mma_f16(sacc[nt], a1, h[2], h[3]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int kp = 0; kp < D / 64; ++kp) {
+          uint32_t b[4];
+          ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 4 * kp + i;
+            const float f = kf[(t >> 1) * CS + nt * 8 + r];
+            uint32_t b0, b1;
+            codes4(b[i], b0, b1);
+            b0 = scale2(b0, f, f);
+            b1 = scale2(b1, f, f);
+            const uint32_t a[4] = {qa[t][0], 0u, qa[t][1], 0u};
+            mma_f16(sacc[nt], a, b0, b1);
+          }
         }
       }
     }
@@ -1277,28 +1341,59 @@ struct BlkCore {
     }
     // ---- P.V: k-step ks = slots 16 ks .. 16 ks + 15, m-tile pair gp = dims 32 gp ..
     // 32 gp + 31 (one scale group)
+    if constexpr (FP4) {
+      // group pair gp (dims 64 gp .. + 63, two scale groups) of slots 16 ks .. + 15: four
+      // MMAs j, m-tile 4 gp + j, whose row i is dim 64 gp + 4 i + j and row i + 8 is
+      // dim 64 gp + 32 + 4 i + j
 #pragma unroll
-    for (int ks = 0; ks < PK; ++ks) {
+      for (int ks = 0; ks < PK; ++ks) {
 #pragma unroll
-      for (int gp = 0; gp < MT / 2; ++gp) {
-        uint32_t mr[4];
-        const int mi = lane >> 3;
-        ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
-        // factors of slots 16 ks + 2c, + 1 (matrices 0, 2) and 16 ks + 8 + 2c, + 1 (1, 3)
-        const float2 fa = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 2 * c);
-        const float2 fb = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 8 + 2 * c);
-        uint32_t af[2][4];
+        for (int gp = 0; gp < D / 64; ++gp) {
+          uint32_t mr[4];
+          const int mi = lane >> 3;
+          ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
+          const float2 f00 = *reinterpret_cast<const float2 *>(vf + (2 * gp) * CS + 16 * ks + 2 * c);
+          const float2 f01 = *reinterpret_cast<const float2 *>(vf + (2 * gp) * CS + 16 * ks + 8 + 2 * c);
+          const float2 f10 = *reinterpret_cast<const float2 *>(vf + (2 * gp + 1) * CS + 16 * ks + 2 * c);
+          const float2 f11 = *reinterpret_cast<const float2 *>(vf + (2 * gp + 1) * CS + 16 * ks + 8 + 2 * c);
+          uint32_t y[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 ff = (i & 1) ? fb : fa;
-          af[i >> 1][(i & 1) * 2 + 0] = scale2(codes2<false>(mr[i]), ff.x, ff.y);  // dim 2r of the two slots
-          af[i >> 1][(i & 1) * 2 + 1] = scale2(codes2<true>(mr[i]), ff.x, ff.y);   // dim 2r + 1
+          for (int i = 0; i < 4; ++i) y[i] = fp4_slot_pairs(mr[i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t a[4] = {scale2(e2m1x2(y[0] >> (8 * j)), f00.x, f00.y),
+                                   scale2(e2m1x2(y[2] >> (8 * j)), f10.x, f10.y),
+                                   scale2(e2m1x2(y[1] >> (8 * j)), f01.x, f01.y),
+                                   scale2(e2m1x2(y[3] >> (8 * j)), f11.x, f11.y)};
+            mma_f16(o[4 * gp + j], a, ph[2 * ks], ph[2 * ks + 1]);
+            mma_f16(o[4 * gp + j], a, pl[2 * ks], pl[2 * ks + 1]);
+          }
         }
+      }
+    } else {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const uint32_t a[4] = {af[t][0], af[t][1], af[t][2], af[t][3]};
-          mma_f16(o[2 * gp + t], a, ph[2 * ks], ph[2 * ks + 1]);
-          mma_f16(o[2 * gp + t], a, pl[2 * ks], pl[2 * ks + 1]);
+      for (int ks = 0; ks < PK; ++ks) {
+#pragma unroll
+        for (int gp = 0; gp < MT / 2; ++gp) {
+          uint32_t mr[4];
+          const int mi = lane >> 3;
+          ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
+          // factors of slots 16 ks + 2c, + 1 (matrices 0, 2) and 16 ks + 8 + 2c, + 1 (1, 3)
+          const float2 fa = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 2 * c);
+          const float2 fb = *reinterpret_cast<const float2 *>(vf + gp * CS + 16 * ks + 8 + 2 * c);
+          uint32_t af[2][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 ff = (i & 1) ? fb : fa;
+            af[i >> 1][(i & 1) * 2 + 0] = scale2(codes2<false>(mr[i]), ff.x, ff.y);  // dim 2r of the two slots
+            af[i >> 1][(i & 1) * 2 + 1] = scale2(codes2<true>(mr[i]), ff.x, ff.y);   // dim 2r + 1
+          }
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t a[4] = {af[t][0], af[t][1], af[t][2], af[t][3]};
+            mma_f16(o[2 * gp + t], a, ph[2 * ks], ph[2 * ks + 1]);
+            mma_f16(o[2 * gp + t], a, pl[2 * ks], pl[2 * ks + 1]);
+          }
         }
       }
     }
@@ -1313,10 +1408,22 @@ struct BlkCore {
 #pragma unroll
     for (int g = 0; g < MT; ++g) {
       const float *og = first ? so_[g] : o[g];
-      const int d = 16 * g + 2 * r;
-      if (2 * c < HC) *reinterpret_cast<float2 *>(dst + (2 * c) * D + d) = make_float2(og[0] * sv, og[2] * sv);
-      if (2 * c + 1 < HC)
-        *reinterpret_cast<float2 *>(dst + (2 * c + 1) * D + d) = make_float2(og[1] * sv, og[3] * sv);
+      if constexpr (FP4) {  // rows r, r + 8 of m-tile g: dims 64 (g / 4) + 4 r + g % 4, and + 32
+        const int d = 64 * (g >> 2) + 4 * r + (g & 3);
+        if (2 * c < HC) {
+          dst[(2 * c) * D + d] = og[0] * sv;
+          dst[(2 * c) * D + d + 32] = og[2] * sv;
+        }
+        if (2 * c + 1 < HC) {
+          dst[(2 * c + 1) * D + d] = og[1] * sv;
+          dst[(2 * c + 1) * D + d + 32] = og[3] * sv;
+        }
+      } else {
+        const int d = 16 * g + 2 * r;
+        if (2 * c < HC) *reinterpret_cast<float2 *>(dst + (2 * c) * D + d) = make_float2(og[0] * sv, og[2] * sv);
+        if (2 * c + 1 < HC)
+          *reinterpret_cast<float2 *>(dst + (2 * c + 1) * D + d) = make_float2(og[1] * sv, og[3] * sv);
+      }
     }
     if (r < HC && c == 0)
       *reinterpret_cast<float4 *>(dst + HC * D + r * 4) = make_float4(first ? sm_ : m, ll, 0.0f, 0.0f);
@@ -1395,10 +1502,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   asm volatile("griddepcontrol.launch_dependents;");
   const int nch = (kv + CS - 1) / CS;
   const int64_t U = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
-  const int64_t CT = gridDim.x, cta = blockIdx.x;
+  const int64_t CT0 = gridDim.x, pcta = blockIdx.x;
 
   if (nch == 0) {  // nothing to attend to: every row is zero
-    for (int64_t u = cta; u < U; u += CT) {
+    for (int64_t u = pcta; u < U; u += CT0) {
       const int hc = static_cast<int>(u % a.nhc);
       const int64_t bhk = u / a.nhc;
       const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
@@ -1413,11 +1520,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const bool ragged = VARLEN && a.B <= kMaxRows;
   const int UH = a.Hkv * a.nhc;  // units per batch row
   int32_t *pfx = reinterpret_cast<int32_t *>(smem + C::PFX_OFF);  // pfx[b]: first chunk of row b
+  const int nch0 = ragged ? (row_kv(a, 0) + CS - 1) / CS : nch;    // row 0's chunks
+  bool equal_rows = !ragged;  // every unit has nch0 chunks
   if (ragged) {  // block scan of the rows' chunk counts, rows [b0, b1) per thread
     const int per = (a.B + C::THREADS - 1) / C::THREADS;
     const int b0 = min(a.B, tid * per), b1 = min(a.B, b0 + per);
     int sum = 0;
-    for (int b = b0; b < b1; ++b) sum += UH * ((row_kv(a, b) + CS - 1) / CS);
+    bool same = true;
+    for (int b = b0; b < b1; ++b) {
+      const int n = (row_kv(a, b) + CS - 1) / CS;
+      same = same && n == nch0;
+      sum += UH * n;
+    }
     int x = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1426,7 +1540,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     int32_t *wsum = pfx + kMaxRows + 1;
     if (lane == 31) wsum[warp] = x;
-    __syncthreads();
+    equal_rows = __syncthreads_and(same) != 0;
     int off = 0;
     for (int w = 0; w < warp; ++w) off += wsum[w];
     int run = off + x - sum;
@@ -1459,7 +1573,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     return lo * UH + (idx - pfx[lo]) / ((pfx[lo + 1] - pfx[lo]) / UH);
   };
   if (ragged) {  // units of empty rows own no chunks: their rows are zero
-    for (int64_t u = cta; u < U; u += CT) {
+    for (int64_t u = pcta; u < U; u += CT0) {
       if (ulen(static_cast<int>(u)) != 0) continue;
       const int hc = static_cast<int>(u % a.nhc);
       const int64_t bhk = u / a.nhc;
@@ -1471,6 +1585,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
   const int W = ragged ? pfx[a.B] : static_cast<int>(U * nch);
+  // CTAs with chunks to stream: the first CT of the grid (the same split for equal rows
+  // whether kv_len is one scalar or one per row)
+  const int64_t CT = equal_rows ? active_ctas(U, nch0, CT0, NW) : CT0;
+  const int64_t cta = pcta;
+  if (cta >= CT) return;
+  // Two CTAs a unit, launched as clusters of two: the pair merges its two partials
+  // through distributed shared memory.  Uniform over the grid, and then no CTA of a
+  // pair returns before the cluster barriers (both halves of a unit hold chunks).
+  const bool pair_merge = CT == 2 * U && nch0 >= 2 && cluster_size() == 2;
   const int c_begin = static_cast<int>(range_start(cta, W, CT)), c_end = static_cast<int>(range_start(cta + 1, W, CT));
   if (c_begin >= c_end) return;  // more CTAs than chunks
 
@@ -1517,7 +1640,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int64_t row = ibase + s0;
       if constexpr (C::MMA) {  // full CS-row boxes (rows past the slab read as zeros, past kv_len are masked)
 #pragma unroll
-        for (int st = 0; st < D / C::ROWB; ++st) {
+        for (int st = 0; st < CB / C::ROWB; ++st) {
           tma_load_2d(tile + st * C::SUBT, &maps.k, st * C::ROWB, static_cast<int>(row), bar, pol);
           tma_load_2d(tile + C::KT + st * C::SUBT, &maps.v, st * C::ROWB, static_cast<int>(row), bar, pol);
         }
@@ -1577,14 +1700,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // in every warp's ring, in warp order.  Write the rows, or this CTA's partial
   // when other CTAs share the unit.  The factors 2^(m_w - M) and the sums of l
   // and corr are per head: HC threads compute them once (scratch `fs`, 0 or 1).
-  auto combine = [&](int u, int rec, int fs) {
-    const int64_t CTn = gridDim.x;
-    const bool alone = cta_of(ustart(u), W, CTn) == cta_of(ustart(u) + ulen(u) - 1, W, CTn);
+  auto combine = [&](int u, int rec, int fs, float *prec) {
+    const bool alone = cta_of(ustart(u), W, CT) == cta_of(ustart(u) + ulen(u) - 1, W, CT);
     const int hc = u % a.nhc;
     const int64_t bhk = u / a.nhc;
     const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
     uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
-    const int64_t wrec = 2 * static_cast<int64_t>(blockIdx.x) + (u == u_first ? 0 : 1);
+    const int64_t wrec = 2 * cta + (u == u_first ? 0 : 1);
     constexpr int RS = R * C::TILE / 4;  // floats from one warp's ring of tiles to the next
     const float *base = reinterpret_cast<const float *>(smem) + rec;
     float *fac = reinterpret_cast<float *>(smem + C::FAC_OFF) + fs * (NW + 3) * HC;  // [NW][HC], then M, L, C
@@ -1630,6 +1752,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         pk.y = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(O.z * inv))) |
                (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(O.w * inv))) << 16);
         *reinterpret_cast<uint2 *>(orow + e) = pk;
+      } else if (prec) {  // the pair's record in shared memory: O [HC][D], then (M, L) [HC]
+        const int d = e - h * D;
+        *reinterpret_cast<float4 *>(prec + h * D + d) = O;
+        if (d == 0) *reinterpret_cast<float2 *>(prec + HC * D + h * 2) = make_float2(fac[NW * HC + h], Lt);
       } else {
         const int d = e - h * D;
         *reinterpret_cast<float4 *>(a.ws_o + (wrec * HC + h) * D + d) = O;
@@ -1642,21 +1768,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // owner o's partial is record 2 c + (u is c's first unit ? 0 : 1), c = its CTA
   int32_t *recs_s = reinterpret_cast<int32_t *>(smem + C::RECS_OFF);
   auto owners_of = [&](int u, int64_t &cf) {
-    const int64_t CTn = gridDim.x;
-    cf = cta_of(ustart(u), W, CTn);
-    const int64_t cl = cta_of(ustart(u) + ulen(u) - 1, W, CTn);
-    return cf == cl ? 1 : (W >= CTn ? static_cast<int>(cl - cf + 1) : ulen(u));  // W < CTn: one chunk per CTA
+    cf = cta_of(ustart(u), W, CT);
+    const int64_t cl = cta_of(ustart(u) + ulen(u) - 1, W, CT);
+    return cf == cl ? 1 : (W >= CT ? static_cast<int>(cl - cf + 1) : ulen(u));  // W < CT: one chunk per CTA
   };
   // returns the owner count; `first` gets the unit's first owner CTA, which names its merge counter
   auto stage_owners = [&](int u, int slot, int &first) {
     int64_t cf;
     const int owners = owners_of(u, cf);
     first = static_cast<int>(cf);
-    const int64_t CTn = gridDim.x;
     for (int o = tid; o < owners && owners > 1; o += C::THREADS) {
-      const int64_t c = W >= CTn ? cf + o : cta_of(ustart(u) + o, W, CTn);
+      const int64_t c = W >= CT ? cf + o : cta_of(ustart(u) + o, W, CT);
       recs_s[slot * kMaxCtas + o] =
-          static_cast<int32_t>(2 * c + (u == unit_of(static_cast<int>(range_start(c, W, CTn))) ? 0 : 1));
+          static_cast<int32_t>(2 * c + (u == unit_of(static_cast<int>(range_start(c, W, CT))) ? 0 : 1));
     }
     return owners;
   };
@@ -1788,7 +1912,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       drain();
       core.publish(reinterpret_cast<float *>(tiles), false, lane);
       __syncthreads();
-      combine(u, 0, 0);
+      combine(u, 0, 0, nullptr);
       fence_proxy_async_smem();  // the rings' generic stores and loads before the next async copies into them
       __syncthreads();           // the rings are free for the next unit's copies
       core.reset();
@@ -1797,8 +1921,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // owner records of the split units (needed by the merge only), staged while
   // the slower warps of the CTA still finish their chunks
   int cf0 = 0, cf1 = 0;
-  const int own0 = stage_owners(u_first, 0, cf0);
-  const int own1 = u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
+  const int own0 = pair_merge ? 2 : stage_owners(u_first, 0, cf0);
+  const int own1 = !pair_merge && u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
+  // the pair's record of its one unit: in warp 1's (idle) ring, past that warp's record
+  float *prec = pair_merge ? reinterpret_cast<float *>(smem + R * C::TILE + C::PUB) : nullptr;
   if (deferred) {
     drain();
     // every warp is past its chunks and its ring is idle: records of the first unit at 0, the last at PUB
@@ -1810,8 +1936,40 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       core.publish(rw, false, lane);
     }
     __syncthreads();
-    combine(u_first, 0, 0);
-    if (u_last != u_first) combine(u_last, C::PUB / 4, 1);
+    combine(u_first, 0, 0, prec);
+    if (u_last != u_first) combine(u_last, C::PUB / 4, 1, nullptr);
+  }
+  if (pair_merge) {
+    // Both records written (cluster-wide release / acquire).  Rank r merges half of
+    // the unit's dims from the two records in rank (= owner) order, as the owner
+    // merge below would, and writes those rows.
+    cluster_sync();
+    constexpr int Q = HC * D / 4;  // float4 items of the unit
+    const uint32_t rank = cluster_rank();
+    const uint32_t r0 = peer_addr(smem_u32(prec), 0), r1 = peer_addr(smem_u32(prec), 1);
+    const int hc = u_first % a.nhc;
+    const int64_t bhk = u_first / a.nhc;
+    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
+    for (int i = static_cast<int>(rank) * (Q / 2) + tid; i < static_cast<int>(rank + 1) * (Q / 2); i += C::THREADS) {
+      const int e = 4 * i, h = e / D;
+      const float2 ml0 = ld_peer_f2(r0 + (HC * D + h * 2) * 4), ml1 = ld_peer_f2(r1 + (HC * D + h * 2) * 4);
+      const float4 v0 = ld_peer_f4(r0 + e * 4), v1 = ld_peer_f4(r1 + e * 4);
+      const float M = fmaxf(ml0.x, ml1.x);
+      const float f0 = ml0.x == -INFINITY ? 0.0f : ex2(ml0.x - M), f1 = ml1.x == -INFINITY ? 0.0f : ex2(ml1.x - M);
+      const float Lt = fmaf(f1, ml1.y, fmaf(f0, ml0.y, 0.0f));
+      const float inv = Lt > 0.0f ? 1.0f / Lt : 0.0f;
+      const float o0 = fmaf(f1, v1.x, fmaf(f0, v0.x, 0.0f)), o1 = fmaf(f1, v1.y, fmaf(f0, v0.y, 0.0f));
+      const float o2 = fmaf(f1, v1.z, fmaf(f0, v0.z, 0.0f)), o3 = fmaf(f1, v1.w, fmaf(f0, v0.w, 0.0f));
+      uint2 pk;
+      pk.x = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o0 * inv))) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o1 * inv))) << 16);
+      pk.y = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o2 * inv))) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o3 * inv))) << 16);
+      *reinterpret_cast<uint2 *>(orow + e) = pk;
+    }
+    cluster_sync();  // the other CTA has read this one's record
+    return;
   }
   __syncthreads();  // every partial and owner record is written; the scratch is free for the merge
 
@@ -1863,7 +2021,7 @@ struct Tune {
   static constexpr int CS = MMA && D <= 128 ? 64 : 32;
   static constexpr int NW = MMA ? (D == 256 ? (MODE ? 4 : 6) : 8)  // block caches at D = 256: two buffers a warp
                                 : (D == 256 ? 8 : (D == 128 ? (HC <= 2 ? 16 : 12) : 16));
-  static constexpr int CB = Q4 ? D / 2 : D;
+  static constexpr int CB = Q4 || MODE == KVQ_MODE_MXFP4 ? D / 2 : D;
   static constexpr int SBB = MODE == KVQ_MODE_FP8_E4M3 || MODE == KVQ_MODE_FP8_E5M2 || MODE == KVQ_MODE_INT8_SYM ? 4 : 1;
   static constexpr int PER_BUF = 2 * CS * CB + (MODE ? 2 * CS * (D / 32) * SBB + 4 * CS : 14 * CS);
   static constexpr int WB = MODE ? CS * 16 + 2 * (D / 32) * CS * 4 : CS * 20;
@@ -1928,13 +2086,46 @@ int make_code_map(CUtensorMap *map, const void *base, int D, int64_t rows, int b
 template <class C, bool VARLEN>
 struct KernelTag {};  // names one decode_kernel instantiation for ensure_smem
 
+// Whether a grid of `ctas` CTAs of `kernel` (one per SM) runs in one wave as
+// clusters of two: the SMs of a cluster come from one GPC, so an odd GPC could
+// leave a pair unplaced.  Queried once per kernel and device.
+template <class Tag, class Kernel>
+bool pairs_fit(Kernel kernel, int threads, int smem, int ctas) {
+  static std::atomic<uint64_t> known{0}, fit{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (known.load(std::memory_order_acquire) & bit) return (fit.load(std::memory_order_acquire) & bit) != 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const bool ok = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && 2 * n >= ctas;
+  if (!ok) (void)cudaGetLastError();
+  if (ok) fit.fetch_or(bit, std::memory_order_acq_rel);
+  known.fetch_or(bit, std::memory_order_acq_rel);
+  return ok;
+}
+
 template <int D, int HC, bool MMA, bool Q4, int MODE = 0>
 int launch_decode(const DecodeArgs &a, const KvMaps &maps, int ctas, cudaStream_t stream) {
   using T = Tune<D, HC, MMA, Q4, MODE>;
   using C = Cfg<D, HC, T::NW, T::R, MMA, Q4, T::CS, MODE>;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t dc = {};
   dc.gridDim = dim3(static_cast<unsigned>(ctas));
   dc.blockDim = dim3(C::THREADS);
@@ -1942,12 +2133,18 @@ int launch_decode(const DecodeArgs &a, const KvMaps &maps, int ctas, cudaStream_
   dc.stream = stream;
   dc.attrs = attr;
   dc.numAttrs = 1;
+  // two CTAs a unit (floor(ctas / units) = 2) may stream as cluster pairs that merge
+  // through distributed shared memory
+  const int64_t units = static_cast<int64_t>(a.B) * a.Hkv * a.nhc;
+  const bool pairs = ctas % 2 == 0 && units > 0 && ctas / units == 2;
   cudaError_t e;
   if (a.kv_per_batch) {
     if (const int st = ensure_smem<KernelTag<C, true>>(decode_kernel<C, true>, C::SMEM)) return st;
+    if (pairs && pairs_fit<KernelTag<C, true>>(decode_kernel<C, true>, C::THREADS, C::SMEM, ctas)) dc.numAttrs = 2;
     e = cudaLaunchKernelEx(&dc, decode_kernel<C, true>, a, maps);
   } else {
     if (const int st = ensure_smem<KernelTag<C, false>>(decode_kernel<C, false>, C::SMEM)) return st;
+    if (pairs && pairs_fit<KernelTag<C, false>>(decode_kernel<C, false>, C::THREADS, C::SMEM, ctas)) dc.numAttrs = 2;
     e = cudaLaunchKernelEx(&dc, decode_kernel<C, false>, a, maps);
   }
   if (e != cudaSuccess) return KVQ_ECUDA;
@@ -1985,7 +2182,9 @@ int dispatch_blk(const DecodeArgs &a, const KvMaps &maps, int hc, int ctas, cuda
 template <int MODE>
 int dispatch_blk_mode(const DecodeArgs &a, const KvMaps &maps, int D, int hc, int ctas, cudaStream_t s) {
   switch (D) {
-    case 64: return dispatch_blk<64, MODE>(a, maps, hc, ctas, s);
+    case 64:
+      if constexpr (MODE == KVQ_MODE_MXFP4) return KVQ_EUNSUPPORTED;  // E2M1 codes from D = 128
+      else return dispatch_blk<64, MODE>(a, maps, hc, ctas, s);
     case 128: return dispatch_blk<128, MODE>(a, maps, hc, ctas, s);
     default: return dispatch_blk<256, MODE>(a, maps, hc, ctas, s);
   }

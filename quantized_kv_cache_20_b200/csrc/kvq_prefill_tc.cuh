@@ -1068,30 +1068,6 @@ __device__ __noinline__ void role_mma(const PrefillArgs &a, const Ctx x) {
 }
 
 // ---- KV split across a thread-block cluster --------------------------------
-KVQ_DEVINL uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Every thread of every CTA of the cluster; orders shared-memory accesses across it.
-KVQ_DEVINL void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The address of this CTA's shared-memory byte `local` in cluster CTA `rank`.
-KVQ_DEVINL uint32_t peer_addr(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-KVQ_DEVINL float4 ld_peer_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
 // The cluster's CTAs each hold (m, E, l, O) of one share of the KV tiles for
 // the same 128 query rows (O and l in units of 2^-(m+E)).  Against the share r
 // with the largest m (the first such), share c weighs f_c = 2^(m_c - m_r) 2^(E_c - E_r),

@@ -16,6 +16,9 @@ kernel's integer rules and checks the invariants the merge relies on:
   - record slots are unique per (CTA, slot);
   - no two split units have the same first owner CTA (the merge counter of a
     split unit is the one of its first owner, at a shape-independent offset).
+With one kv_len for every row the kernel may stream with U k of its CT0 CTAs
+(k = floor(CT0 / U)) instead of all of them, when that costs a warp no more
+rounds of chunks; each CTA's range then lies inside one unit.
 """
 import random
 
@@ -26,6 +29,15 @@ def range_start(c, W, C):
 
 def cta_of(idx, W, C):
     return ((idx + 1) * C - 1) // W
+
+
+def active_ctas(U, nch, CT0, NW):
+    k = CT0 // U
+    if k < 1:
+        return CT0
+    rounds_all = (-(-U * nch // CT0) + NW - 1) // NW
+    rounds_units = (-(-nch // k) + NW - 1) // NW
+    return U * k if rounds_units <= rounds_all else CT0
 
 
 def check_split(lens_per_unit, C):
@@ -102,3 +114,33 @@ def test_fewer_chunks_than_ctas():
     # one chunk per CTA at most: every split unit has one owner per chunk
     check_split([3, 1, 0, 2], 148)
     check_split([1] * 100, 148)
+
+
+def test_unit_aligned_grid():
+    rng = random.Random(3)
+    for _ in range(600):
+        U = rng.randint(1, 160)
+        nch = rng.randint(1, 400)
+        CT0 = rng.choice([132, 148, 256])
+        NW = rng.choice([4, 6, 8])
+        C = active_ctas(U, nch, CT0, NW)
+        assert 1 <= C <= CT0
+        check_split([nch] * U, C)
+        if C != CT0:
+            k = C // U
+            assert C == U * k and k == CT0 // U
+            W = U * nch
+            for c in range(C):  # every CTA's range lies inside unit c // k
+                b, e = range_start(c, W, C), range_start(c + 1, W, C)
+                if b < e:
+                    assert (c // k) * nch <= b and e <= (c // k + 1) * nch
+    # the CTAs that stream are spread over the grid: CTA b takes place floor(b CT / CT0)
+    # when the next CTA's is larger, and the places are 0 .. CT - 1, once each
+    for CT0 in (132, 148):
+        for CT in range(1, CT0 + 1):
+            places = [b * CT // CT0 for b in range(CT0) if (b + 1) * CT // CT0 > b * CT // CT0]
+            assert places == list(range(CT))
+    # the decode workload (8 x 8 units, 64 chunks of 64 slots, 8 warps): two CTAs a unit
+    assert active_ctas(64, 64, 148, 8) == 128
+    # a long single-row decode keeps the flattened split (fewer rounds per warp)
+    assert active_ctas(16, 4096, 148, 6) == 148
