@@ -176,10 +176,12 @@ struct Cfg {
   static constexpr int QMETA_OFF = Q_OFF + 4 * HC * D;       // [2][HC] (sum n, 2^E)
   static constexpr int RECS_OFF = QMETA_OFF + 2 * HC * 8;    // [2][kMaxCtas] owner records
   static constexpr int PFX_OFF = RECS_OFF + 2 * kMaxCtas * 4;  // [kMaxRows + 1] chunk prefix, [32] scratch
-  // combine factors of the two unit records: [2][NW][HC] f, then [2][3][HC] (M, L, C)
-  static constexpr int FAC_OFF = PFX_OFF + (kMaxRows + 1 + 32) * 4;
+  // cluster pair merge: the half of the unit's O this CTA merges, from either CTA
+  // ([2 sources][HC D / 2] float), then every head's (M, L) from either ([2][HC] float2)
+  static constexpr int PAIR_OFF = (PFX_OFF + (kMaxRows + 1 + 32) * 4 + 15) / 16 * 16;
+  static constexpr int PAIR_BYTES = HC * D * 4 + HC * 16;
   static constexpr int ALIGN = MMA ? 1024 : 0;                 // slack to align the tiles
-  static constexpr int SMEM = FAC_OFF + 2 * (NW + 3) * HC * 4 + ALIGN;
+  static constexpr int SMEM = PAIR_OFF + PAIR_BYTES + ALIGN;
   static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr int THREADS = NW * 32;
 };
@@ -219,13 +221,17 @@ KVQ_DEVINL int64_t cta_of(int64_t idx, int64_t W, int64_t C) { return ((idx + 1)
 // warp no more rounds of chunks (a warp takes every NW-th chunk of its CTA).  With
 // U * k CTAs the range of CTA c lies inside unit floor(c / k), so a CTA never combines
 // two units and a unit has exactly k owners (none to merge when k = 1).
-KVQ_DEVINL int64_t active_ctas(int64_t U, int64_t nch, int64_t CT0, int NW) {
-  const int64_t k = CT0 / U;
-  if (k < 1) return CT0;
-  const int64_t rounds_all = ((U * nch + CT0 - 1) / CT0 + NW - 1) / NW;
-  const int64_t rounds_units = ((nch + k - 1) / k + NW - 1) / NW;
-  return rounds_units <= rounds_all ? U * k : CT0;
+// Index math in 32 bits (U * nch < 2^31, CT0 <= kMaxCtas): a 64-bit division by a
+// run-time value is a long dependent chain, and these sit before the first copy.
+KVQ_DEVINL int active_ctas(uint32_t U, uint32_t nch, uint32_t CT0, uint32_t NW) {
+  const uint32_t k = CT0 / U;
+  if (k < 1) return static_cast<int>(CT0);
+  const uint32_t rounds_all = ((U * nch + CT0 - 1) / CT0 + NW - 1) / NW;
+  const uint32_t rounds_units = ((nch + k - 1) / k + NW - 1) / NW;
+  return static_cast<int>(rounds_units <= rounds_all ? U * k : CT0);
 }
+// range_start(c, W, C) for 0 <= c <= C <= kMaxCtas, given q = W / C and r = W % C
+KVQ_DEVINL int range_start_qr(uint32_t c, uint32_t q, uint32_t r, uint32_t C) { return static_cast<int>(c * q + c * r / C); }
 
 // One probe of the phase, suspending the thread for at most `hint_ns`.
 KVQ_DEVINL bool mbar_try_wait_ns(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
@@ -1587,14 +1593,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int W = ragged ? pfx[a.B] : static_cast<int>(U * nch);
   // CTAs with chunks to stream: the first CT of the grid (the same split for equal rows
   // whether kv_len is one scalar or one per row)
-  const int64_t CT = equal_rows ? active_ctas(U, nch0, CT0, NW) : CT0;
-  const int64_t cta = pcta;
+  const int CT = equal_rows ? active_ctas(static_cast<uint32_t>(U), nch0, static_cast<uint32_t>(CT0), NW)
+                            : static_cast<int>(CT0);
+  const int cta = static_cast<int>(pcta);
   if (cta >= CT) return;
   // Two CTAs a unit, launched as clusters of two: the pair merges its two partials
   // through distributed shared memory.  Uniform over the grid, and then no CTA of a
   // pair returns before the cluster barriers (both halves of a unit hold chunks).
   const bool pair_merge = CT == 2 * U && nch0 >= 2 && cluster_size() == 2;
-  const int c_begin = static_cast<int>(range_start(cta, W, CT)), c_end = static_cast<int>(range_start(cta + 1, W, CT));
+  const uint32_t wq = static_cast<uint32_t>(W) / CT, wr = static_cast<uint32_t>(W) % CT;
+  const int c_begin = range_start_qr(cta, wq, wr, CT), c_end = range_start_qr(cta + 1, wq, wr, CT);
   if (c_begin >= c_end) return;  // more CTAs than chunks
 
   // ---- this warp's chunks: c_begin + warp + k * NW for k in [0, nk), chunk k in buffer k % R
@@ -1620,10 +1628,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         iustart = ustart(iu);
         iuend = iustart + ulen(iu);
       } while (idx >= iuend);
-      const int64_t bhk = iu / a.nhc;  // = b * Hkv + hk
-      ibase = bhk * a.S;
-      ikv = VARLEN ? row_kv(a, static_cast<int>(bhk / a.Hkv)) : kv;
-      if (a.mask) imask = a.mask + (bhk / a.Hkv) * a.mask_bstride;
+      const int bhk = iu / a.nhc;  // = b * Hkv + hk
+      ibase = static_cast<int64_t>(bhk) * a.S;
+      const int brow = bhk / a.Hkv;
+      ikv = VARLEN ? row_kv(a, brow) : kv;
+      if (a.mask) imask = a.mask + brow * a.mask_bstride;
     }
     const int s0 = (idx - iustart) * CS;
     const int kvu = ikv;
@@ -1685,9 +1694,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   // the q row of head h of unit u
   auto q_row = [&](int u, int h) {
-    const int hc = u % a.nhc;
-    const int64_t bhk = u / a.nhc;
-    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    const int bhk = u / a.nhc, hc = u - bhk * a.nhc;
+    const int b = bhk / a.Hkv, hk = bhk - b * a.Hkv;
     return a.q + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC + h) * D;
   };
   // warp w: heads w, w + NW, .. of unit u onto the core's q layout, into q slot `slot`
@@ -1698,48 +1706,40 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   // all threads: combine the warp records of unit u, found at tiles + rec (floats)
   // in every warp's ring, in warp order.  Write the rows, or this CTA's partial
-  // when other CTAs share the unit.  The factors 2^(m_w - M) and the sums of l
-  // and corr are per head: HC threads compute them once (scratch `fs`, 0 or 1).
-  auto combine = [&](int u, int rec, int fs, float *prec) {
-    const bool alone = cta_of(ustart(u), W, CT) == cta_of(ustart(u) + ulen(u) - 1, W, CT);
-    const int hc = u % a.nhc;
-    const int64_t bhk = u / a.nhc;
-    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+  // when other CTAs share the unit: for the pair merge into the pair buffer of the
+  // CTA that merges each half (its own, or the other CTA's through distributed
+  // shared memory), else into the workspace.  A thread takes four dims of one head
+  // and forms that head's factors 2^(m_w - M) and sums of l and corr itself.
+  auto combine = [&](int u, int rec, bool pair) {
+    const bool alone = ustart(u) >= c_begin && ustart(u) + ulen(u) <= c_end;  // no other CTA has chunks of u
+    const int bhk = u / a.nhc, hc = u - bhk * a.nhc;
+    const int b = bhk / a.Hkv, hk = bhk - b * a.Hkv;
     uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
-    const int64_t wrec = 2 * cta + (u == u_first ? 0 : 1);
+    const int64_t wrec = 2 * static_cast<int64_t>(cta) + (u == u_first ? 0 : 1);
     constexpr int RS = R * C::TILE / 4;  // floats from one warp's ring of tiles to the next
     const float *base = reinterpret_cast<const float *>(smem) + rec;
-    float *fac = reinterpret_cast<float *>(smem + C::FAC_OFF) + fs * (NW + 3) * HC;  // [NW][HC], then M, L, C
-    if (tid < HC) {
-      const int h = tid;
-      float M = -INFINITY;
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * RS + HC * D + h * 4]);
-      float Lt = 0.0f, Ct = 0.0f;
-      for (int w = 0; w < NW; ++w) {
-        const float4 mlc = *reinterpret_cast<const float4 *>(base + w * RS + HC * D + h * 4);
-        const float f = mlc.x == -INFINITY ? 0.0f : ex2(mlc.x - M);
-        fac[w * HC + h] = f;
-        Lt = fmaf(f, mlc.y, Lt);
-        Ct = fmaf(f, mlc.z, Ct);
-      }
-      fac[NW * HC + h] = M;
-      fac[(NW + 1) * HC + h] = Lt;
-      fac[(NW + 2) * HC + h] = Ct;
-    }
-    __syncthreads();
     for (int e = 4 * tid; e < HC * D; e += 4 * C::THREADS) {  // four dims of one head per step
       const int h = e / D;
-      float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
+      float4 mlc[NW];
+      float M = -INFINITY;
+#pragma unroll
       for (int w = 0; w < NW; ++w) {
-        const float f = fac[w * HC + h];
+        mlc[w] = *reinterpret_cast<const float4 *>(base + w * RS + HC * D + h * 4);
+        M = fmaxf(M, mlc[w].x);
+      }
+      float Lt = 0.0f, Ct = 0.0f;
+      float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float f = mlc[w].x == -INFINITY ? 0.0f : ex2(mlc[w].x - M);
+        Lt = fmaf(f, mlc[w].y, Lt);
+        Ct = fmaf(f, mlc[w].z, Ct);
         const float4 x = *reinterpret_cast<const float4 *>(base + w * RS + e);
         O.x = fmaf(f, x.x, O.x);
         O.y = fmaf(f, x.y, O.y);
         O.z = fmaf(f, x.z, O.z);
         O.w = fmaf(f, x.w, O.w);
       }
-      const float Ct = fac[(NW + 2) * HC + h], Lt = fac[(NW + 1) * HC + h];
       O.x = fmaf(O.x, Core::OSCALE, -Ct);
       O.y = fmaf(O.y, Core::OSCALE, -Ct);
       O.z = fmaf(O.z, Core::OSCALE, -Ct);
@@ -1752,14 +1752,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         pk.y = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(O.z * inv))) |
                (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(O.w * inv))) << 16);
         *reinterpret_cast<uint2 *>(orow + e) = pk;
-      } else if (prec) {  // the pair's record in shared memory: O [HC][D], then (M, L) [HC]
-        const int d = e - h * D;
-        *reinterpret_cast<float4 *>(prec + h * D + d) = O;
-        if (d == 0) *reinterpret_cast<float2 *>(prec + HC * D + h * 2) = make_float2(fac[NW * HC + h], Lt);
+      } else if (pair) {
+        constexpr int Q2 = HC * D / 8;  // float4 items of one half
+        const uint32_t me = cluster_rank(), i = static_cast<uint32_t>(e >> 2), owner = i < Q2 ? 0u : 1u;
+        const uint32_t buf = smem_u32(smem) + C::PAIR_OFF;
+        const uint32_t at = buf + me * (Q2 * 16) + (i - owner * Q2) * 16;
+        if (owner == me) st_shared_f4(at, O);
+        else st_peer_f4(peer_addr(at, owner), O);
+        if (e - h * D == 0) {  // (M, L) of head h to both CTAs
+          const uint32_t ml = buf + HC * D * 4 + (me * HC + h) * 8;
+          st_shared_f2(ml, make_float2(M, Lt));
+          st_peer_f2(peer_addr(ml, me ^ 1u), make_float2(M, Lt));
+        }
       } else {
         const int d = e - h * D;
         *reinterpret_cast<float4 *>(a.ws_o + (wrec * HC + h) * D + d) = O;
-        if (d == 0) *reinterpret_cast<float2 *>(a.ws_ml + (wrec * HC + h) * 2) = make_float2(fac[NW * HC + h], Lt);
+        if (d == 0) *reinterpret_cast<float2 *>(a.ws_ml + (wrec * HC + h) * 2) = make_float2(M, Lt);
       }
     }
   };
@@ -1912,7 +1920,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       drain();
       core.publish(reinterpret_cast<float *>(tiles), false, lane);
       __syncthreads();
-      combine(u, 0, 0, nullptr);
+      combine(u, 0, false);
       fence_proxy_async_smem();  // the rings' generic stores and loads before the next async copies into them
       __syncthreads();           // the rings are free for the next unit's copies
       core.reset();
@@ -1923,8 +1931,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   int cf0 = 0, cf1 = 0;
   const int own0 = pair_merge ? 2 : stage_owners(u_first, 0, cf0);
   const int own1 = !pair_merge && u_last != u_first ? stage_owners(u_last, 1, cf1) : 1;
-  // the pair's record of its one unit: in warp 1's (idle) ring, past that warp's record
-  float *prec = pair_merge ? reinterpret_cast<float *>(smem + R * C::TILE + C::PUB) : nullptr;
   if (deferred) {
     drain();
     // every warp is past its chunks and its ring is idle: records of the first unit at 0, the last at PUB
@@ -1936,25 +1942,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       core.publish(rw, false, lane);
     }
     __syncthreads();
-    combine(u_first, 0, 0, prec);
-    if (u_last != u_first) combine(u_last, C::PUB / 4, 1, nullptr);
+    combine(u_first, 0, pair_merge);
+    if (u_last != u_first) combine(u_last, C::PUB / 4, false);
   }
   if (pair_merge) {
-    // Both records written (cluster-wide release / acquire).  Rank r merges half of
-    // the unit's dims from the two records in rank (= owner) order, as the owner
-    // merge below would, and writes those rows.
+    // Both CTAs' partials of this CTA's half are in its pair buffer once the cluster
+    // barrier (release / acquire) is passed; nothing touches this CTA's shared memory
+    // after it.  Merge them in rank (= owner) order, as the owner merge below would.
     cluster_sync();
-    constexpr int Q = HC * D / 4;  // float4 items of the unit
-    const uint32_t rank = cluster_rank();
-    const uint32_t r0 = peer_addr(smem_u32(prec), 0), r1 = peer_addr(smem_u32(prec), 1);
-    const int hc = u_first % a.nhc;
-    const int64_t bhk = u_first / a.nhc;
-    const int hk = static_cast<int>(bhk % a.Hkv), b = static_cast<int>(bhk / a.Hkv);
+    constexpr int Q2 = HC * D / 8;  // float4 items of one half
+    const int me = static_cast<int>(cluster_rank());
+    const float *pb = reinterpret_cast<const float *>(smem + C::PAIR_OFF);
+    const float2 *pml = reinterpret_cast<const float2 *>(smem + C::PAIR_OFF + HC * D * 4);
+    const int bhk = u_first / a.nhc, hc = u_first - bhk * a.nhc;
+    const int b = bhk / a.Hkv, hk = bhk - b * a.Hkv;
     uint16_t *orow = a.out + (static_cast<int64_t>(b) * a.Hq + hk * a.G + hc * HC) * D;
-    for (int i = static_cast<int>(rank) * (Q / 2) + tid; i < static_cast<int>(rank + 1) * (Q / 2); i += C::THREADS) {
-      const int e = 4 * i, h = e / D;
-      const float2 ml0 = ld_peer_f2(r0 + (HC * D + h * 2) * 4), ml1 = ld_peer_f2(r1 + (HC * D + h * 2) * 4);
-      const float4 v0 = ld_peer_f4(r0 + e * 4), v1 = ld_peer_f4(r1 + e * 4);
+    for (int j = tid; j < Q2; j += C::THREADS) {
+      const int e = 4 * (me * Q2 + j), h = e / D;
+      const float2 ml0 = pml[h], ml1 = pml[HC + h];
+      const float4 v0 = *reinterpret_cast<const float4 *>(pb + 4 * j);
+      const float4 v1 = *reinterpret_cast<const float4 *>(pb + 4 * (Q2 + j));
       const float M = fmaxf(ml0.x, ml1.x);
       const float f0 = ml0.x == -INFINITY ? 0.0f : ex2(ml0.x - M), f1 = ml1.x == -INFINITY ? 0.0f : ex2(ml1.x - M);
       const float Lt = fmaf(f1, ml1.y, fmaf(f0, ml0.y, 0.0f));
@@ -1968,7 +1975,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o3 * inv))) << 16);
       *reinterpret_cast<uint2 *>(orow + e) = pk;
     }
-    cluster_sync();  // the other CTA has read this one's record
     return;
   }
   __syncthreads();  // every partial and owner record is written; the scratch is free for the merge
@@ -2026,7 +2032,7 @@ struct Tune {
   static constexpr int PER_BUF = 2 * CS * CB + (MODE ? 2 * CS * (D / 32) * SBB + 4 * CS : 14 * CS);
   static constexpr int WB = MODE ? CS * 16 + 2 * (D / 32) * CS * 4 : CS * 20;
   static constexpr int FIXED = (MMA ? 1024 + NW * WB : NW * HC * 128) + NW * 4 * 8 + 64 + 4 * HC * D +
-                               16 * HC + 8 * kMaxCtas + 4 * (kMaxRows + 33) + 8 * (NW + 3) * HC;
+                               16 * HC + 8 * kMaxCtas + 4 * (kMaxRows + 33) + 16 + 4 * HC * D + 16 * HC;
   static constexpr int RMAX = (232448 - FIXED) / (NW * PER_BUF);
   static constexpr int R = RMAX > 4 ? 4 : RMAX;
   static_assert(R >= 1, "ring depth");
