@@ -65,6 +65,7 @@ constexpr int kConvThreads = 128;  // per converter warpgroup (one for K, one fo
 constexpr int kThreads = kSoftmaxThreads + 2 * kConvThreads + 32;
 constexpr int kMmaWarp = 12;
 constexpr int kScaleBufs = 3;  // k_scale / v_scale tile buffers
+constexpr int kMaxSplit = 4;  // CTAs of a KV-split cluster
 // registers per thread: 13 warps, one SM sub-partition holds four of them
 constexpr int kRegsLaunch = 128;
 
@@ -110,6 +111,9 @@ enum : int {
   kBarODone,   // a PV finished (commit)
   kBarOFinal,  // the last PV finished (commit, once)
   kBarDrain,   // abort path: everything issued has finished (commit)
+  kBarMask0,   // mask rows of a tile staged in buffer 0 / 1 / 2 (bulk copies, RPH arrivals)
+  kBarMask1,
+  kBarMask2,
   kNumBars
 };
 
@@ -135,8 +139,17 @@ struct Cfg {
   static constexpr int FAC_BYTES = MODE == 0 ? 0 : 2 * 2 * kTile * NG * 4;
   static constexpr int BAR_OFF = FAC_OFF + FAC_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + kNumBars * 8;  // TMEM base, abort flag, qs, 4 x max|q|, O valid
-  static constexpr int STAT_OFF = MISC_OFF + 32;             // KV split: float4 [kRows] (m, E, l, -) per row
-  static constexpr int SMEM = STAT_OFF + kRows * 16 + 1024;  // + slack to align the base to 1024
+  static constexpr int STAT_OFF = (MISC_OFF + 32 + 15) / 16 * 16;  // KV split: float4 [kRows] (m, E, l, -) per row
+  // additive mask: with one position per 32 rows of the CTA (4 heads a row block) the
+  // mask rows of a tile are staged by bulk copies into a ring of three buffers of
+  // [RPH][kTile] floats (rows 16 bytes apart more than their length, which spreads a
+  // warp's float4 reads over all banks); else read from global memory
+  static constexpr int MROW = kTile * 4 + 16;
+  static constexpr int MSK_OFF = STAT_OFF + kRows * 16;
+  static constexpr int SMEM_BASE = MSK_OFF + 1024;  // + slack to align the base to 1024
+  static constexpr bool MSTAGE = MASK && RPH <= 32 && SMEM_BASE + 3 * RPH * MROW <= 232448;
+  static constexpr int SMEM = SMEM_BASE + (MSTAGE ? 3 * RPH * MROW : 0);
+  static_assert(STAT_OFF % 16 == 0 && MSK_OFF % 16 == 0 && MROW % 16 == 0, "float4 stores and bulk copies");
   // KV split: the rows' pre-scaled fp32 partial O, [kRows][D], over the Q/K/V tiles
   static constexpr int CONTRIB_OFF = Q_OFF;
   static_assert(kRows * D * 4 <= BAR_OFF, "the partial O fits over the tiles");
@@ -359,14 +372,62 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
   // the CTA, chosen so that the largest |q| lands in [2^14, 2^15)
   const uint4 *qp =
       reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + (row_ok ? pos : 0)) * D);
+  // Staged mask (C::MSTAGE): thread t < RPH (the first head of each position) copies
+  // its position's mask row of tile j into buffer j % 3.  Tile j + 1's copy is issued
+  // once S_j is computed: QK_j needed PV_{j-2}, so every row is past tile j - 2, the
+  // last user of that buffer.
+  uint8_t *msk = smem + C::MSK_OFF;
+  const bool missue = C::MSTAGE && t < RPH;
+  uint32_t mpend = 0, mpar = 0;  // buffers with a copy in flight and their phases (issuing threads)
+  auto issue_mask = [&](int j) {
+    const int mb = j % 3;
+    const int t0 = (jb + j) * kTile;
+    const int n = row_ok ? max(0, min(kTile, loop_end - t0)) : 0;
+    const uint32_t bytes = static_cast<uint32_t>((n + 3) & ~3) * 4;  // loop_end <= S, S % 4 == 0
+    mbar_arrive_expect_tx(&bars[kBarMask0 + mb], bytes);
+    if (bytes)
+      bulk_g2s(msk + (mb * RPH + t) * C::MROW, a.mask + b * a.mask_bstride + static_cast<int64_t>(pos) * a.S + t0,
+               bytes, &bars[kBarMask0 + mb]);
+    mpend |= 1u << mb;
+    mpar = (mpar & ~(1u << mb)) | (static_cast<uint32_t>((j / 3) & 1) << mb);
+  };
+  if (missue && ntiles > 0) issue_mask(0);
+  // Unstaged mask: the row's mask for the first tile into L1 while Q is staged (each
+  // tile's is fetched one tile ahead below), so the score pass reads it at L1 latency.
+  auto prefetch_mask = [&](int j) {
+    if constexpr (C::MASK && !C::MSTAGE) {
+      const int t0 = (jb + j) * kTile;
+      if (row_ok)
+#pragma unroll
+        for (int i = 0; i < kTile / 32; ++i)
+          if (t0 + 32 * i < loop_end)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(a.mask + b * a.mask_bstride +
+                                                          static_cast<int64_t>(pos) * a.S + t0 + 32 * i));
+    }
+  };
+  if (ntiles > 0) prefetch_mask(0);
+  // Q row up to D = 128: all its loads in flight at once (one round trip) and kept in
+  // registers for the conversion; at D = 256 in groups of four, read twice
+  constexpr int QC = D / 8;
+  constexpr bool QREG = QC <= 16;
+  uint4 qw[QREG ? QC : 1];
   {
     uint32_t mx = 0;
     if (row_ok) {
+      if constexpr (QREG) {
+#pragma unroll
+        for (int i = 0; i < QC; ++i) qw[i] = __ldg(qp + i);
+#pragma unroll
+        for (int i = 0; i < QC; ++i)
+          mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(qw[i].x & 0x7FFF7FFFu, qw[i].y & 0x7FFF7FFFu),
+                                     __vmaxu2(qw[i].z & 0x7FFF7FFFu, qw[i].w & 0x7FFF7FFFu)));
+      } else {
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 w = __ldg(qp + c);
-        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
-                                   __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+        for (int c = 0; c < QC; ++c) {
+          const uint4 w = __ldg(qp + c);
+          mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                     __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+        }
       }
     }
     const uint32_t mw = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
@@ -379,10 +440,14 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
   const float qs = a.qscale * exp2i(sh);
   {
     const float f = exp2i(-sh);
-#pragma unroll 2
+#pragma unroll QREG ? 16 : 2
     for (int c = 0; c < D / 8; ++c) {
       uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (row_ok) w = __ldg(qp + c);
+      if constexpr (QREG) {
+        if (row_ok) w = qw[c];
+      } else {
+        if (row_ok) w = __ldg(qp + c);
+      }
       const uint32_t in[4] = {w.x, w.y, w.z, w.w};
       uint32_t o[4];
 #pragma unroll
@@ -410,12 +475,20 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     const int t0 = (jb + j) * kTile;
     const int sb = j % kScaleBufs;
     const uint32_t s_addr = tmem + (buf ? C::S_COL1 : C::S_COL0) + lane_base;
+    if (j + 1 < ntiles) prefetch_mask(j + 1);
     const float4 *kq4 = reinterpret_cast<const float4 *>(ks_s + sb * kTile);
     const float4 *vs4 = reinterpret_cast<const float4 *>(vs_s + sb * kTile);
     const bool full = t0 + kTile - 1 <= vis_last;  // every slot of the tile visible to this row
     ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarSFull0 + buf], (j >> 1) & 1, abort_flag, a.wait_ns));
     if (!ok) break;
     tc_fence_after();
+    if constexpr (C::MSTAGE) {
+      if (missue && j + 1 < ntiles) issue_mask(j + 1);
+      ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarMask0 + j % 3], (j / 3) & 1, abort_flag, a.wait_ns));
+      if (!ok) break;
+      mpend &= ~(1u << (j % 3));
+    }
+    const float *mrow = reinterpret_cast<const float *>(msk + ((j % 3) * RPH + (t - g * RPH)) * C::MROW);
     // pass 1, per 32 columns: the tile max (masked scores are written back over S)
     float mt = -INFINITY;
 #pragma unroll 1
@@ -429,8 +502,12 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
           const int j0 = t0 + c * 32 + q4 * 4;
           const float4 kk = kq4[c * 8 + q4];
           float4 mv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (row_ok && j0 < loop_end)  // in bounds: loop_end <= S, S % 4 == 0
-            mv = *reinterpret_cast<const float4 *>(a.mask + b * a.mask_bstride + static_cast<int64_t>(pos) * a.S + j0);
+          if (row_ok && j0 < loop_end) {  // in bounds: loop_end <= S, S % 4 == 0
+            if constexpr (C::MSTAGE)
+              mv = *reinterpret_cast<const float4 *>(mrow + c * 32 + q4 * 4);
+            else
+              mv = *reinterpret_cast<const float4 *>(a.mask + b * a.mask_bstride + static_cast<int64_t>(pos) * a.S + j0);
+          }
           const float kf[4] = {kk.x, kk.y, kk.z, kk.w}, mf[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -537,6 +614,10 @@ __device__ __noinline__ void role_softmax(const PrefillArgs &a, const Ctx x) {
     tc_fence_before();
     mbar_arrive(&bars[kBarPFull0 + buf]);
   }
+  // after an abort: this thread's mask copies still in flight land before the CTA exits
+  if (missue && mpend)
+    for (int mb = 0; mb < 3; ++mb)
+      if (mpend & (1u << mb)) mbar_wait_bounded(&bars[kBarMask0 + mb], (mpar >> mb) & 1u);
   // ---- epilogue: O / l -> bf16 (the TMEM loads are warp-collective: every lane runs them)
   if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, wait_phase(&bars[kBarOFinal], 0, abort_flag, a.wait_ns));
   if (a.ns > 1) {
@@ -1090,16 +1171,16 @@ __device__ __noinline__ void cluster_merge(const PrefillArgs &a, const Ctx x, bo
   cluster_sync();  // every share's row statistics are published
   if (tid < kRows) {  // the softmax warps own TMEM lanes 0..127: row t
     const int t = tid;
-    float4 st[8];  // (m, E, l, -) of every share (ns <= 8)
+    float4 st[kMaxSplit];  // (m, E, l, -) of every share, all loads in flight at once
+#pragma unroll
+    for (int c = 0; c < kMaxSplit; ++c)
+      st[c] = c < ns ? ld_peer_f4(peer_addr(stat_l + 16 * t, c)) : make_float4(-INFINITY, 0.0f, 0.0f, 0.0f);
     float mr = -INFINITY, er = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      if (c < ns) {
-        st[c] = ld_peer_f4(peer_addr(stat_l + 16 * t, c));
-        if (st[c].x > mr) {
-          mr = st[c].x;
-          er = st[c].y;
-        }
+    for (int c = 0; c < kMaxSplit; ++c) {
+      if (c < ns && st[c].x > mr) {
+        mr = st[c].x;
+        er = st[c].y;
       }
     }
     auto weight = [&](const float4 &sc) {
@@ -1107,7 +1188,7 @@ __device__ __noinline__ void cluster_merge(const PrefillArgs &a, const Ctx x, bo
     };
     float L = 0.0f, w_self = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kMaxSplit; ++c) {
       if (c < ns) {
         const float w = weight(st[c]);
         L = fmaf(st[c].z, w, L);
@@ -1140,24 +1221,45 @@ __device__ __noinline__ void cluster_merge(const PrefillArgs &a, const Ctx x, bo
     const int xrow = blockIdx.x / ns, hkc = blockIdx.y, b = blockIdx.z;
     const int hk = hkc / a.nhc, hc = hkc - hk * a.nhc;
     const int r0 = static_cast<int>(rank) * kRows / ns, r1 = (static_cast<int>(rank) + 1) * kRows / ns;
-    for (int i = tid; i < (r1 - r0) * (D / 4); i += kThreads) {
-      const int r = r0 + i / (D / 4), k = i % (D / 4);
-      const int g = r / RPH, pos = xrow * RPH + (r - g * RPH);
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int c = 0; c < ns; ++c) {
-        const float4 v = ld_peer_f4(peer_addr(contrib_l + 16 * cidx(r, k), c));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    // kBatch items a thread at a time, every share's loads of all of them in flight
+    // before the first add (a load from another CTA's shared memory is a long trip)
+    constexpr int kBatch = 4;
+    const int items = (r1 - r0) * (D / 4);
+    for (int i0 = tid; i0 < items; i0 += kBatch * kThreads) {
+      float4 v[kBatch][kMaxSplit];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kThreads;
+        const int r = r0 + i / (D / 4), k = i % (D / 4);
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c)
+          v[u][c] = i < items && c < ns ? ld_peer_f4(peer_addr(contrib_l + 16 * cidx(r, k), c))
+                                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
-      if (pos < a.Lq) {
-        const int hq = hk * a.G + hc * HPT + g;
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t *>(&lo);
-        pk.y = *reinterpret_cast<const uint32_t *>(&hi);
-        *reinterpret_cast<uint2 *>(a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + pos) * D + 4 * k) = pk;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i >= items) break;
+        const int r = r0 + i / (D / 4), k = i % (D / 4);
+        const int g = r / RPH, pos = xrow * RPH + (r - g * RPH);
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int c = 0; c < kMaxSplit; ++c) {
+          if (c < ns) {
+            acc.x += v[u][c].x;
+            acc.y += v[u][c].y;
+            acc.z += v[u][c].z;
+            acc.w += v[u][c].w;
+          }
+        }
+        if (pos < a.Lq) {
+          const int hq = hk * a.G + hc * HPT + g;
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+          *reinterpret_cast<uint2 *>(a.out + ((static_cast<int64_t>(b) * a.Hq + hq) * a.Lq + pos) * D + 4 * k) = pk;
+        }
       }
     }
   }
@@ -1190,6 +1292,7 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
     mbar_init(&bars[kBarODone], 1);
     mbar_init(&bars[kBarOFinal], 1);
     mbar_init(&bars[kBarDrain], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[kBarMask0 + i], RPH);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1264,7 +1367,7 @@ int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   const int64_t base = static_cast<int64_t>(rowblocks) * a.Hkv * a.nhc * a.B;
   const int64_t tiles = (a.S + kTile - 1) / kTile;
   a.ns = 1;
-  while (a.ns < 4 && base * a.ns * 2 <= sm_count() && a.ns * 2 <= tiles) a.ns *= 2;
+  while (a.ns < kMaxSplit && base * a.ns * 2 <= sm_count() && a.ns * 2 <= tiles) a.ns *= 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rowblocks * a.ns, a.Hkv * a.nhc, a.B);
   cfg.blockDim = dim3(kThreads);
