@@ -98,6 +98,28 @@ def test_decode_config_full_size():
     assert_attn_close(bf16_to_f64(out), ref, "decode config")
 
 
+@pytest.mark.parametrize("B,Hkv,G,D,kv_len", [
+    (12, 8, 4, 128, 1000),   # 96 units: one CTA a unit (k = 1), no merge
+    (5, 8, 4, 128, 1500),    # 40 units: three CTAs a unit (k = 3), counter merge
+    (8, 8, 4, 128, 50),      # 64 units of one chunk: the second CTA of every pair has none
+    (8, 8, 4, 128, 8000),    # 64 units of 125 chunks: the flattened split takes fewer rounds
+    (37, 2, 4, 128, 700),    # 74 units: every CTA streams, as cluster pairs
+    (4, 8, 8, 64, 3000),     # 32 units (one head chunk of 8): four CTAs a unit
+    (16, 4, 2, 256, 760),    # D = 256 (two buffers a warp), 64 units of 24 chunks in pairs
+])
+def test_decode_split_choices(B, Hkv, G, D, kv_len):
+    """The kernel picks its split from the shape and the kv_len it reads: the
+    flattened cut over every CTA, or U k CTAs that each take a k-th of one unit
+    (merged in pairs through distributed shared memory when k = 2)."""
+    g = wl.generator(B * 7 + Hkv * 13 + G + D + kv_len)
+    S = (kv_len + 63) // 64 * 64 + 64
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hkv * G, 1, D), g)
+    out = _decode_gpu(q, K, V, kv_len)
+    ref = oracle.sdpa(wl.u16(q), *_np(K), *_np(V), kv_len=kv_len, sm_scale=1 / math.sqrt(D))
+    assert_attn_close(bf16_to_f64(out), ref, f"decode split B={B} Hkv={Hkv} G={G} D={D} kv={kv_len}")
+
+
 def test_long_config_decode_full_size():
     """batch 1, 32 q / 16 kv heads, D=256, kv_len = 131072 (the whole cache)."""
     w = wl.LONG
