@@ -309,7 +309,10 @@ int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const i
  *
  * k, v         u8 [B, Hkv, S, D/2];  k_scale, v_scale float [B, Hkv, S];
  *              k_zp, v_zp u8 [B, Hkv, S] holding 0..15.
- * Other arguments, sizes and the workspace as for kvq_decode_attn.
+ * Other arguments, sizes and the workspace as for kvq_decode_attn.  At D = 128
+ * and 256 the kernel is kvq_decode_attn's on the tensor cores (codes unpacked to
+ * bytes for q.K, to the fp16 values 1024 + c for P.V; exact); at D = 64 a
+ * CUDA-core form of it (dp2a for q.k, packed fp32 FMA for p.v).
  */
 int kvq_decode_attn_tq4(const void *q, int B, int Hq, int Hkv, int D, const uint8_t *k, const float *k_scale,
                         const uint8_t *k_zp, const uint8_t *v, const float *v_scale, const uint8_t *v_zp,

@@ -34,11 +34,12 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   if (mask_bstride < 0 || mask_bstride % 4 != 0) return KVQ_EINVAL;  // keeps every row's mask 16-byte aligned
   if (!(sm_scale == sm_scale)) return KVQ_EINVAL;
   const int G = Hq / Hkv;
-  const int hc = q4 ? head_chunk_simt(G) : head_chunk_mma(G);
+  const bool q4_mma = q4 && D >= 128;  // TQ4 on the tensor cores; at D = 64 on the CUDA cores
+  const int hc = q4 && !q4_mma ? head_chunk_simt(G) : head_chunk_mma(G);
   const int nhc = G / hc;
   if (static_cast<int64_t>(B) * Hkv * nhc * ((S + 31) / 32) >= INT32_MAX) return KVQ_EUNSUPPORTED;
   // TMA row coordinates are 32-bit
-  if (!q4 && static_cast<int64_t>(B) * Hkv * S >= INT32_MAX) return KVQ_EUNSUPPORTED;
+  if ((!q4 || q4_mma) && static_cast<int64_t>(B) * Hkv * S >= INT32_MAX) return KVQ_EUNSUPPORTED;
   const int ctas = sm_count();
   const WsLayout w = ws_layout(D, hc, ctas);
   if (ctas > kMaxCtas) return KVQ_EUNSUPPORTED;  // owner records staged per unit
@@ -72,17 +73,13 @@ int decode_impl(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, c
   KvMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (q4) {
-    switch (D) {
-      case 64: return dispatch_q4<64>(a, maps, hc, ctas, s);
-      case 128: return dispatch_q4<128>(a, maps, hc, ctas, s);
-      default: return dispatch_q4<256>(a, maps, hc, ctas, s);
-    }
-  }
+  if (q4 && !q4_mma) return dispatch_q4<64>(a, maps, hc, ctas, s);
   const int64_t rows = static_cast<int64_t>(B) * Hkv * S;
   const int box_rows = D <= 128 ? 64 : 32;  // the tensor-core path's chunk (Tune::CS)
-  if (const int st = make_code_map(&maps.k, k, D, rows, box_rows)) return st;
-  if (const int st = make_code_map(&maps.v, v, D, rows, box_rows)) return st;
+  const int row_bytes = q4 ? D / 2 : D;     // TQ4: two codes a byte
+  if (const int st = make_code_map(&maps.k, k, row_bytes, rows, box_rows)) return st;
+  if (const int st = make_code_map(&maps.v, v, row_bytes, rows, box_rows)) return st;
+  if (q4) return D == 128 ? dispatch_q4mma<128>(a, maps, hc, ctas, s) : dispatch_q4mma<256>(a, maps, hc, ctas, s);
   switch (D) {
     case 64: return dispatch_mma<64>(a, maps, hc, ctas, s);
     case 128: return dispatch_mma<128>(a, maps, hc, ctas, s);

@@ -134,7 +134,7 @@ struct Cfg {
   static constexpr int D = D_, HC = HC_, NW = NW_, R = R_;
   static constexpr bool MMA = MMA_;          // int8 or block cache on the tensor cores
   static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte (CUDA cores)
-  static_assert(!(MMA && Q4), "the TQ4 cache runs on the CUDA cores");
+  static_assert(!(MMA && Q4) || D_ >= 128, "the TQ4 cache on the tensor cores from D = 128");
   static constexpr int MODE = MODE_;         // kvq_write mode of the cache: 0 int8 affine, else a block mode
   static constexpr bool BLK = MODE_ != 0;
   static_assert(!BLK || (MMA && MODE_ <= KVQ_MODE_INT8_SYM && (MODE_ != KVQ_MODE_MXFP4 || D_ >= 128)),
@@ -630,7 +630,10 @@ struct MmaCore {
   static constexpr int MT = D / 16;  // P.V m-tiles
   static_assert(HC <= 8, "q heads of a unit fit the 8 MMA rows");
   static constexpr float OSCALE = 1.0f;    // records hold O itself
-  static constexpr float kVOff = 1152.0f;  // a V code c enters as the fp16 value 1152 + c
+  // TQ4 cache: 4-bit codes 0..15, two a byte (element 2i in the low nibble of byte i)
+  static constexpr bool Q4 = C::Q4;
+  // a V code c enters as the fp16 value 1152 + c (int8), 1024 + c (TQ4)
+  static constexpr float kVOff = Q4 ? 1024.0f : 1152.0f;
 
   uint32_t qa[KS][4];  // q A fragments
   int qslot;
@@ -744,12 +747,15 @@ struct MmaCore {
     const bool on = r < HC;
     const uint8_t *hp = smem + C::Q_OFF + slot * 2 * HC * D + (on ? r : 0) * D;
     const uint8_t *lp = hp + HC * D;
+    // k-step k: lane c's K bytes are dims 32 k + 4 c .. + 3 and 32 k + 16 + 4 c .. + 3 (int8);
+    // TQ4: its 8 codes of one ldmatrix row are dims 32 k + 8 c .. + 7, unpacked in that order
+    const int o0 = Q4 ? 8 * c : 4 * c, o1 = Q4 ? 8 * c + 4 : 16 + 4 * c;
 #pragma unroll
     for (int k = 0; k < KS; ++k) {
-      qa[k][0] = on ? *reinterpret_cast<const uint32_t *>(hp + 32 * k + 4 * c) : 0u;
-      qa[k][1] = on ? *reinterpret_cast<const uint32_t *>(lp + 32 * k + 4 * c) : 0u;
-      qa[k][2] = on ? *reinterpret_cast<const uint32_t *>(hp + 32 * k + 16 + 4 * c) : 0u;
-      qa[k][3] = on ? *reinterpret_cast<const uint32_t *>(lp + 32 * k + 16 + 4 * c) : 0u;
+      qa[k][0] = on ? *reinterpret_cast<const uint32_t *>(hp + 32 * k + o0) : 0u;
+      qa[k][1] = on ? *reinterpret_cast<const uint32_t *>(lp + 32 * k + o0) : 0u;
+      qa[k][2] = on ? *reinterpret_cast<const uint32_t *>(hp + 32 * k + o1) : 0u;
+      qa[k][3] = on ? *reinterpret_cast<const uint32_t *>(lp + 32 * k + o1) : 0u;
     }
     qslot = slot;
     const int2 meta = reinterpret_cast<const int2 *>(smem + C::QMETA_OFF)[slot * HC + (on ? r : 0)];
@@ -818,12 +824,25 @@ struct MmaCore {
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) sacc[nt][i] = 0;
+      if constexpr (Q4) {  // 64 bytes of codes = four k-steps; nibbles unpacked to bytes 0..15
 #pragma unroll
-      for (int kp = 0; kp < KS / 2; ++kp) {
-        uint32_t b[4];
-        ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
-        mma_s8(sacc[nt], qa[2 * kp], b[0], b[1]);
-        mma_s8(sacc[nt], qa[2 * kp + 1], b[2], b[3]);
+        for (int kp = 0; kp < KS / 4; ++kp) {
+          uint32_t b[4];
+          ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = b[i] & 0x0F0F0F0Fu, hi = (b[i] >> 4) & 0x0F0F0F0Fu;
+            mma_s8(sacc[nt], qa[4 * kp + i], __byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int kp = 0; kp < KS / 2; ++kp) {
+          uint32_t b[4];
+          ldsm_x4(b, swz(kt, nt * 8 + (lane & 7), 64 * kp + 16 * (lane >> 3)));
+          mma_s8(sacc[nt], qa[2 * kp], b[0], b[1]);
+          mma_s8(sacc[nt], qa[2 * kp + 1], b[2], b[3]);
+        }
       }
     }
     __syncwarp();  // the per-slot values are written
@@ -902,30 +921,65 @@ struct MmaCore {
     }
     // ---- P.V: k-step ks = slots 16 ks .. 16 ks + 15; ldmatrix.trans x4 gives the
     // V^T fragments of two m-tiles (32 dims)
+    if constexpr (Q4) {
+      // 32 bytes of V codes = 64 dims (gp): a 16-bit element of ldmatrix.trans is four
+      // dims of one slot; a byte permute and a nibble swap give, per byte j, dim 4 i + j
+      // of slots 2c and 2c + 1, made the fp16 pair (1024 + c0, 1024 + c1).  Four MMAs j,
+      // m-tile 4 gp + j: row i is dim 64 gp + 4 i + j, row i + 8 is dim 64 gp + 32 + 4 i + j.
 #pragma unroll
-    for (int ks = 0; ks < PK; ++ks) {
+      for (int ks = 0; ks < PK; ++ks) {
 #pragma unroll
-      for (int gp = 0; gp < MT / 2; ++gp) {
-        uint32_t mr[4];
-        const int mi = lane >> 3;  // matrix: rows 16 ks + 8 (mi & 1) .., dim bytes 32 gp + 16 (mi >> 1)
-        ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
-        uint32_t af[2][4];
+        for (int gp = 0; gp < D / 64; ++gp) {
+          uint32_t mr[4];
+          const int mi = lane >> 3;
+          ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
+          uint32_t y[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // bytes: (slot 2c, dim 2n), (2c, 2n + 1), (2c + 1, 2n), (2c + 1, 2n + 1); +128 then fp16 0x64xx
-          const uint32_t x = mr[i] ^ 0x80808080u;
-          const uint32_t ev = __byte_perm(x, 0x64646464u, 0x4240u);  // dim 2n of slots 2c, 2c + 1
-          const uint32_t od = __byte_perm(x, 0x64646464u, 0x4341u);  // dim 2n + 1
-          // matrices 0, 1: m-tile 2gp (slots +0, +8); 2, 3: m-tile 2gp + 1
-          af[i >> 1][(i & 1) * 2 + 0] = ev;
-          af[i >> 1][(i & 1) * 2 + 1] = od;
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t x = __byte_perm(mr[i], 0u, 0x3120);  // bytes: s lo, s+1 lo, s hi, s+1 hi
+            const uint32_t t = ((x >> 4) ^ x) & 0x00F000F0u;     // swap the middle nibbles of each half
+            y[i] = x ^ t ^ (t << 4);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t a[4];
+            const int src[4] = {0, 2, 1, 3};  // a0: unit 2gp slots 2c..; a1: unit 2gp+1; a2, a3: slots + 8
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t bj = (y[src[e]] >> (8 * j)) & 0xFFu;
+              a[e] = (bj & 0x0Fu) | ((bj & 0xF0u) << 12) | 0x64006400u;
+            }
+            mma_f16(o[4 * gp + j], a, ph[2 * ks], ph[2 * ks + 1]);
+            mma_f16(o[4 * gp + j], a, pl[2 * ks], pl[2 * ks + 1]);
+          }
         }
-        // A fragment order: a0 = rows 0..7 (even dims) k 0..7, a1 = rows 8..15 (odd) k 0..7, a2/a3 k 8..15
+      }
+    } else {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const uint32_t a[4] = {af[t][0], af[t][1], af[t][2], af[t][3]};
-          mma_f16(o[2 * gp + t], a, ph[2 * ks], ph[2 * ks + 1]);
-          mma_f16(o[2 * gp + t], a, pl[2 * ks], pl[2 * ks + 1]);
+      for (int ks = 0; ks < PK; ++ks) {
+#pragma unroll
+        for (int gp = 0; gp < MT / 2; ++gp) {
+          uint32_t mr[4];
+          const int mi = lane >> 3;  // matrix: rows 16 ks + 8 (mi & 1) .., dim bytes 32 gp + 16 (mi >> 1)
+          ldsm_x4_trans(mr, swz(vt, 16 * ks + 8 * (mi & 1) + (lane & 7), 32 * gp + 16 * (mi >> 1)));
+          uint32_t af[2][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // bytes: (slot 2c, dim 2n), (2c, 2n + 1), (2c + 1, 2n), (2c + 1, 2n + 1); +128 then fp16 0x64xx
+            const uint32_t x = mr[i] ^ 0x80808080u;
+            const uint32_t ev = __byte_perm(x, 0x64646464u, 0x4240u);  // dim 2n of slots 2c, 2c + 1
+            const uint32_t od = __byte_perm(x, 0x64646464u, 0x4341u);  // dim 2n + 1
+            // matrices 0, 1: m-tile 2gp (slots +0, +8); 2, 3: m-tile 2gp + 1
+            af[i >> 1][(i & 1) * 2 + 0] = ev;
+            af[i >> 1][(i & 1) * 2 + 1] = od;
+          }
+          // A fragment order: a0 = rows 0..7 (even dims) k 0..7, a1 = rows 8..15 (odd) k 0..7, a2/a3 k 8..15
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t a[4] = {af[t][0], af[t][1], af[t][2], af[t][3]};
+            mma_f16(o[2 * gp + t], a, ph[2 * ks], ph[2 * ks + 1]);
+            mma_f16(o[2 * gp + t], a, pl[2 * ks], pl[2 * ks + 1]);
+          }
         }
       }
     }
@@ -944,10 +998,22 @@ struct MmaCore {
 #pragma unroll
     for (int g = 0; g < MT; ++g) {
       const float *og = first ? so_[g] : o[g];
-      const int d = 16 * g + 2 * r;
-      if (2 * c < HC) *reinterpret_cast<float2 *>(dst + (2 * c) * D + d) = make_float2(og[0] * sv, og[2] * sv);
-      if (2 * c + 1 < HC)
-        *reinterpret_cast<float2 *>(dst + (2 * c + 1) * D + d) = make_float2(og[1] * sv, og[3] * sv);
+      if constexpr (Q4) {  // rows r, r + 8 of m-tile g: dims 64 (g / 4) + 4 r + g % 4, and + 32
+        const int d = 64 * (g >> 2) + 4 * r + (g & 3);
+        if (2 * c < HC) {
+          dst[(2 * c) * D + d] = og[0] * sv;
+          dst[(2 * c) * D + d + 32] = og[2] * sv;
+        }
+        if (2 * c + 1 < HC) {
+          dst[(2 * c + 1) * D + d] = og[1] * sv;
+          dst[(2 * c + 1) * D + d + 32] = og[3] * sv;
+        }
+      } else {
+        const int d = 16 * g + 2 * r;
+        if (2 * c < HC) *reinterpret_cast<float2 *>(dst + (2 * c) * D + d) = make_float2(og[0] * sv, og[2] * sv);
+        if (2 * c + 1 < HC)
+          *reinterpret_cast<float2 *>(dst + (2 * c + 1) * D + d) = make_float2(og[1] * sv, og[3] * sv);
+      }
     }
     if (r < HC && c == 0)
       *reinterpret_cast<float4 *>(dst + HC * D + r * 4) = make_float4(first ? sm_ : m, ll, cc * sv, 0.0f);
@@ -2210,6 +2276,21 @@ int dispatch_blk_mode(const DecodeArgs &a, const KvMaps &maps, int D, int hc, in
       else return dispatch_blk<64, MODE>(a, maps, hc, ctas, s);
     case 128: return dispatch_blk<128, MODE>(a, maps, hc, ctas, s);
     default: return dispatch_blk<256, MODE>(a, maps, hc, ctas, s);
+  }
+}
+
+// TQ4 cache on the tensor cores (D = 128, 256)
+template <int D>
+int dispatch_q4mma(const DecodeArgs &a, const KvMaps &maps, int hc, int ctas, cudaStream_t s) {
+  switch (hc) {
+    case 1: return launch_decode<D, 1, true, true>(a, maps, ctas, s);
+    case 2: return launch_decode<D, 2, true, true>(a, maps, ctas, s);
+    case 3: return launch_decode<D, 3, true, true>(a, maps, ctas, s);
+    case 4: return launch_decode<D, 4, true, true>(a, maps, ctas, s);
+    case 5: return launch_decode<D, 5, true, true>(a, maps, ctas, s);
+    case 6: return launch_decode<D, 6, true, true>(a, maps, ctas, s);
+    case 7: return launch_decode<D, 7, true, true>(a, maps, ctas, s);
+    default: return launch_decode<D, 8, true, true>(a, maps, ctas, s);
   }
 }
 
