@@ -1657,18 +1657,81 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
   const int W = ragged ? pfx[a.B] : static_cast<int>(U * nch);
+  // Rows of different lengths, at most 32 of them and one CTA a unit at least: each
+  // row b gets k_b CTAs a unit (one each, then one more at a time to the row with the
+  // most chunks a CTA, while the grid lasts), and CTA (b, unit, j) takes the j-th of
+  // k_b equal parts of its unit; used when no warp takes more rounds of chunks than
+  // with the flattened cut.  A CTA then never spans two units (see active_ctas).
+  // kb[b], and Kb[b] the first CTA of row b, sit in the prefix area past pfx[B].
+  int32_t *kb = pfx + a.B + 1, *Kb = kb + a.B;
+  bool row_aligned = false;
+  if (ragged && !equal_rows && a.B <= 32 && static_cast<int64_t>(a.B) * UH <= CT0) {
+    if (warp == 0) {
+      const int b = lane;
+      const int nb = b < a.B ? (pfx[b + 1] - pfx[b]) / UH : 0;
+      int k = nb > 0 ? 1 : 0;
+      int used = k;  // rows with chunks: one CTA a unit each
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) used += __shfl_xor_sync(0xffffffffu, used, o);
+      int rem = static_cast<int>(CT0) / UH - used;  // a row's extra CTA a unit costs UH CTAs
+      while (rem > 0) {  // one more CTA a unit to the row with the most chunks a CTA
+        int best = k > 0 ? (nb + k - 1) / k : 0, who = b;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          const int ob = __shfl_xor_sync(0xffffffffu, best, o), ow = __shfl_xor_sync(0xffffffffu, who, o);
+          if (ob > best || (ob == best && ow < who)) {
+            best = ob;
+            who = ow;
+          }
+        }
+        if (best <= 1) break;
+        if (b == who) ++k;
+        --rem;
+      }
+      const int per = k > 0 ? (nb + k - 1) / k : 0;  // chunks of this row's CTAs, at most
+      int mx = (per + NW - 1) / NW;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const int rounds_all = ((W + static_cast<int>(CT0) - 1) / static_cast<int>(CT0) + NW - 1) / NW;
+      int run = k * UH;  // exclusive prefix of the rows' CTAs
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, run, o);
+        if (lane >= o) run += y;
+      }
+      if (b < a.B) {
+        kb[b] = k;
+        Kb[b] = run - k * UH;
+      }
+      if (lane == 31) sh[4] = mx <= rounds_all ? run : 0;  // CTAs in use, 0: not used
+    }
+    __syncthreads();
+    row_aligned = sh[4] > 0;
+  }
   // CTAs with chunks to stream: the first CT of the grid (the same split for equal rows
   // whether kv_len is one scalar or one per row)
-  const int CT = equal_rows ? active_ctas(static_cast<uint32_t>(U), nch0, static_cast<uint32_t>(CT0), NW)
-                            : static_cast<int>(CT0);
+  const int CT = row_aligned ? sh[4]
+                 : equal_rows ? active_ctas(static_cast<uint32_t>(U), nch0, static_cast<uint32_t>(CT0), NW)
+                              : static_cast<int>(CT0);
   const int cta = static_cast<int>(pcta);
   if (cta >= CT) return;
   // Two CTAs a unit, launched as clusters of two: the pair merges its two partials
   // through distributed shared memory.  Uniform over the grid, and then no CTA of a
   // pair returns before the cluster barriers (both halves of a unit hold chunks).
-  const bool pair_merge = CT == 2 * U && nch0 >= 2 && cluster_size() == 2;
-  const uint32_t wq = static_cast<uint32_t>(W) / CT, wr = static_cast<uint32_t>(W) % CT;
-  const int c_begin = range_start_qr(cta, wq, wr, CT), c_end = range_start_qr(cta + 1, wq, wr, CT);
+  const bool pair_merge = !row_aligned && CT == 2 * U && nch0 >= 2 && cluster_size() == 2;
+  int c_begin, c_end;
+  if (row_aligned) {  // CTA cta: row b, unit uu of the row, part j of k_b
+    int b = 0;
+    while (b + 1 < a.B && Kb[b + 1] <= cta) ++b;
+    const int k = kb[b], off = cta - Kb[b], uu = off / k, j = off - uu * k;
+    const int n = (pfx[b + 1] - pfx[b]) / UH, us = pfx[b] + uu * n;
+    c_begin = us + j * n / k;
+    c_end = us + (j + 1) * n / k;
+  } else {
+    const uint32_t wq = static_cast<uint32_t>(W) / CT, wr = static_cast<uint32_t>(W) % CT;
+    c_begin = range_start_qr(cta, wq, wr, CT);
+    c_end = range_start_qr(cta + 1, wq, wr, CT);
+  }
   if (c_begin >= c_end) return;  // more CTAs than chunks
 
   // ---- this warp's chunks: c_begin + warp + k * NW for k in [0, nk), chunk k in buffer k % R
@@ -1859,6 +1922,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // owner o's partial is record 2 c + (u is c's first unit ? 0 : 1), c = its CTA
   int32_t *recs_s = reinterpret_cast<int32_t *>(smem + C::RECS_OFF);
   auto owners_of = [&](int u, int64_t &cf) {
+    if (row_aligned) {  // the k_b CTAs of unit u, in order
+      const int b = u / UH, k = kb[b];
+      cf = Kb[b] + (u - b * UH) * k;
+      return k;
+    }
     cf = cta_of(ustart(u), W, CT);
     const int64_t cl = cta_of(ustart(u) + ulen(u) - 1, W, CT);
     return cf == cl ? 1 : (W >= CT ? static_cast<int>(cl - cf + 1) : ulen(u));  // W < CT: one chunk per CTA
@@ -1869,6 +1937,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int owners = owners_of(u, cf);
     first = static_cast<int>(cf);
     for (int o = tid; o < owners && owners > 1; o += C::THREADS) {
+      if (row_aligned) {  // every owner's only unit: record 2 c
+        recs_s[slot * kMaxCtas + o] = static_cast<int32_t>(2 * (cf + o));
+        continue;
+      }
       const int64_t c = W >= CT ? cf + o : cta_of(ustart(u) + o, W, CT);
       recs_s[slot * kMaxCtas + o] =
           static_cast<int32_t>(2 * c + (u == unit_of(static_cast<int>(range_start(c, W, CT))) ? 0 : 1));

@@ -144,3 +144,61 @@ def test_unit_aligned_grid():
     assert active_ctas(64, 64, 148, 8) == 128
     # a long single-row decode keeps the flattened split (fewer rounds per warp)
     assert active_ctas(16, 4096, 148, 6) == 148
+
+
+def row_aligned_split(row_chunks, UH, CT0, NW):
+    """The kernel's split for rows of different lengths (at most 32 rows): k_b CTAs a
+    unit for row b, one each, then one more at a time to the row with the most chunks
+    a CTA (ties: the lower row) while UH * sum(k_b) stays within the grid; used when no
+    warp then takes more rounds than with the flattened cut.  Returns the CTAs' chunk
+    ranges, or None when the flattened cut is kept."""
+    B = len(row_chunks)
+    if B > 32 or B * UH > CT0:
+        return None
+    k = [1 if n > 0 else 0 for n in row_chunks]
+    rem = CT0 // UH - sum(k)
+    while rem > 0:
+        best, who = max(((-(-n // kk) if kk else 0), -b) for b, (n, kk) in enumerate(zip(row_chunks, k)))
+        if best <= 1:
+            break
+        k[-who] += 1
+        rem -= 1
+    W = UH * sum(row_chunks)
+    rounds_all = (-(-W // CT0) + NW - 1) // NW
+    mx = max(((-(-n // kk) if kk else 0) + NW - 1) // NW for n, kk in zip(row_chunks, k))
+    if mx > rounds_all:
+        return None
+    ranges, start = [], 0
+    for n, kk in zip(row_chunks, k):
+        for uu in range(UH):
+            us = start + uu * n
+            for j in range(kk):
+                ranges.append((us + j * n // kk, us + (j + 1) * n // kk))
+        start += UH * n
+    return ranges
+
+
+def test_row_aligned_split():
+    rng = random.Random(4)
+    for _ in range(500):
+        B = rng.randint(1, 32)
+        UH = rng.choice([1, 2, 4, 8])
+        rows = [0 if rng.random() < 0.15 else rng.randint(1, 300) for _ in range(B)]
+        NW = rng.choice([6, 8])
+        r = row_aligned_split(rows, UH, 148, NW)
+        if r is None:
+            continue
+        assert len(r) <= 148
+        covered = sorted(i for b, e in r for i in range(b, e))
+        assert covered == list(range(UH * sum(rows)))  # every chunk once
+        starts = [0]
+        for n in rows:
+            for _ in range(UH):
+                starts.append(starts[-1] + n)
+        for b, e in r:  # a CTA's range lies inside one unit
+            if b < e:
+                u = max(i for i, s0 in enumerate(starts[:-1]) if s0 <= b and starts[i + 1] > b)
+                assert e <= starts[u + 1]
+    # the ragged bench batch (8 rows of 512..8192 slots, 64-slot chunks, 8 kv heads)
+    r = row_aligned_split([8, 16, 32, 48, 64, 80, 96, 128], 8, 148, 8)
+    assert r is not None and len(r) == 144 and max(e - b for b, e in r) == 32

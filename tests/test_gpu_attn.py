@@ -392,6 +392,33 @@ def test_decode_varlen_many_short_rows_with_empty_ones(D):
         assert_attn_close(got[b:b + 1], ref, f"varlen decode D={D} row {b} kv={lens[b]}")
 
 
+@pytest.mark.parametrize("D,lens", [
+    (128, [512, 1024, 2048, 3072, 4096, 5120, 6144, 8192]),  # the ragged bench batch: 144 CTAs, 1-4 a unit
+    (256, [100, 3000, 0, 7000, 64, 2500]),                     # D = 256, an empty row, a one-chunk row
+])
+def test_decode_varlen_row_aligned_split(D, lens):
+    """A few rows of different lengths: each row's units get their own CTAs (more for
+    longer rows), so no CTA spans two units; every row equals the oracle at its length."""
+    g = wl.generator(790 + D + len(lens))
+    B, Hkv, G = len(lens), 8 if D == 128 else 4, 4 if D == 128 else 2
+    S = 8192
+    K, V = _cache(B, Hkv, S, D, g)
+    q = wl.bf16_normal((B, Hkv * G, 1, D), g)
+    err = err_word()
+    out = kvq.decode_attn_varlen(q.to(DEV), *[t.to(DEV) for t in K], *[t.to(DEV) for t in V],
+                                 torch.tensor(lens, dtype=torch.int32, device=DEV), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = bf16_to_f64(out)
+    for b in range(B):
+        if lens[b] == 0:
+            assert torch.all(out[b] == 0)
+            continue
+        ref = oracle.sdpa(wl.u16(q[b:b + 1]), *_np(_slice(K, b)), *_np(_slice(V, b)), kv_len=lens[b],
+                          sm_scale=1 / math.sqrt(D))
+        assert_attn_close(got[b:b + 1], ref, f"row-aligned varlen decode D={D} row {b} kv={lens[b]}")
+
+
 def test_decode_varlen_equal_rows_is_the_scalar_path():
     g = wl.generator(777)
     B, Hq, Hkv, D, S = 4, 16, 4, 128, 2048
