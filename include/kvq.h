@@ -291,7 +291,10 @@ int kvq_decode_attn(const void *q, int B, int Hq, int Hkv, int D, const int8_t *
  * Other arguments, sizes and the workspace as for kvq_decode_attn.  Batches of
  * up to 1024 rows are cut into split units by each row's own length (rows of
  * kv_lens 0 own no work); larger batches are cut as for the longest row, and
- * tiles past a row's own length move no bytes.
+ * tiles past a row's own length move no bytes.  With at most 32 rows of
+ * different lengths each row's (kv head, head chunk) units may instead get CTAs
+ * of their own, more for longer rows, when that costs no rounds of tiles; rows
+ * of equal length are cut exactly as kvq_decode_attn cuts them (equal results).
  */
 int kvq_decode_attn_varlen(const void *q, int B, int Hq, int Hkv, int D, const int8_t *k, const float *k_scale,
                            const int8_t *k_zp, const int8_t *v, const float *v_scale, const int8_t *v_zp,
