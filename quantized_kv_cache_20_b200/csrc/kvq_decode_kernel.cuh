@@ -54,9 +54,12 @@
 //    permute makes a pair of codes the exact fp16 values 1152 + c, and the
 //    offset and zero point leave as one per-head correction,
 //    sum_j w_j (1152 + zp_j).
-//  - The TQ4 cache (4-bit codes) runs the same skeleton on the CUDA cores: q.k
-//    on dp2a with an exact 16-bit q, p.v on packed fp32 FMA over codes turned
-//    into exact subnormal floats.
+//  - The TQ4 cache (4-bit codes, two a byte) runs the same core at D = 128 and
+//    256: a lane's codes of an ldmatrix row are unpacked to bytes for the int8
+//    q.K MMA (q loaded in the matching order), and made the fp16 values 1024 + c
+//    for P.V.  At D = 64 (32-byte code rows) it runs the skeleton on the CUDA
+//    cores: q.k on dp2a with an exact 16-bit q, p.v on packed fp32 FMA over
+//    codes turned into exact subnormal floats.
 //  - Unit close: when a CTA spans at most two units, a warp keeps its first
 //    unit's state in registers and starts the second; at the end the (idle)
 //    rings hold every warp's records and the CTA merges them in warp order.
@@ -133,7 +136,7 @@ template <int D_, int HC_, int NW_, int R_, bool MMA_, bool Q4_, int CS_ = 32, i
 struct Cfg {
   static constexpr int D = D_, HC = HC_, NW = NW_, R = R_;
   static constexpr bool MMA = MMA_;          // int8 or block cache on the tensor cores
-  static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte (CUDA cores)
+  static constexpr bool Q4 = Q4_;            // TQ4 cache: 4-bit codes, two per byte
   static_assert(!(MMA && Q4) || D_ >= 128, "the TQ4 cache on the tensor cores from D = 128");
   static constexpr int MODE = MODE_;         // kvq_write mode of the cache: 0 int8 affine, else a block mode
   static constexpr bool BLK = MODE_ != 0;
@@ -358,7 +361,7 @@ KVQ_DEVINL uint32_t pack_f16x2(float x, float y) {
 KVQ_DEVINL float2 unpack_f16x2(uint32_t u) { return __half22float2(*reinterpret_cast<const __half2 *>(&u)); }
 
 // ---------------------------------------------------------------------------
-// Per-warp math of one unit on the CUDA cores (TQ4 cache).
+// Per-warp math of one unit on the CUDA cores (TQ4 cache at D = 64).
 //   q.k: a lane takes 16 dims of L = D/16 slots; lane `sub` visits slot
 //   g + NG*(t ^ sub) at step t, which makes the reduce-scatter over the L lanes
 //   a plain butterfly that leaves each lane the full dot products of one slot.
