@@ -50,6 +50,7 @@
 // for what it issued, TMEM is freed and KVQ_ERR_TIMEOUT is reported.
 #pragma once
 
+#include <atomic>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -1355,6 +1356,33 @@ __global__ void __maxnreg__(kRegsLaunch) prefill_tc_kernel(const __grid_constant
 
 inline int hpt_for(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
 
+// Clusters of ns CTAs of kernel C that can be resident at once (0 if the query
+// fails), queried once per kernel and cluster size.
+template <class C>
+int clusters_fit(int ns, dim3 grid) {
+  static std::atomic<int> known[kMaxSplit + 1];
+  const int k = known[ns].load(std::memory_order_relaxed);
+  if (k != 0) return k > 0 ? k : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(ns);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, prefill_tc_kernel<C>, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = -1;
+  }
+  known[ns].store(n, std::memory_order_relaxed);
+  return n > 0 ? n : 0;
+}
+
 template <int D, int HPT, bool MASK, int MODE>
 int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   using C = Cfg<D, HPT, MASK, MODE>;
@@ -1366,8 +1394,26 @@ int launch_prefill_tc(PrefillArgs a, cudaStream_t stream) {
   // share can hold a tile of the cache)
   const int64_t base = static_cast<int64_t>(rowblocks) * a.Hkv * a.nhc * a.B;
   const int64_t tiles = (a.S + kTile - 1) / kTile;
+  const int sms = sm_count();
   a.ns = 1;
-  while (a.ns < kMaxSplit && base * a.ns * 2 <= sm_count() && a.ns * 2 <= tiles) a.ns *= 2;
+  if (base * 2 <= sms) {
+    while (a.ns < kMaxSplit && base * a.ns * 2 <= sms && a.ns * 2 <= tiles) a.ns *= 2;
+  } else {
+    // Several waves of one CTA an SM: a launch takes about ceil(row blocks / clusters
+    // resident at once) waves of 1/ns of a row block's tiles each; split when that is
+    // shorter by more than the merge costs (a few percent), e.g. 512 row blocks on 148
+    // SMs: 4 waves unsplit, 7 half-waves in pairs.
+    double best = static_cast<double>((base + sms - 1) / sms);
+    for (int ns = 2; ns <= kMaxSplit && ns * 2 <= tiles; ns *= 2) {
+      const int fit = clusters_fit<C>(ns, dim3(rowblocks * ns, a.Hkv * a.nhc, a.B));
+      if (fit <= 0) continue;
+      const double t = static_cast<double>((base + fit - 1) / fit) / ns;
+      if (t < 0.97 * best) {
+        best = t;
+        a.ns = ns;
+      }
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rowblocks * a.ns, a.Hkv * a.nhc, a.B);
   cfg.blockDim = dim3(kThreads);
