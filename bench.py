@@ -44,7 +44,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the decode workload, from one ncu capture, and the SHA-256 of the decode source it was
 # taken on: the line reports the figure only while the source is unchanged (else null).
 DECODE_TRAFFIC_BYTES = 70691328  # 69,872,384 read + 818,944 written; algorithmic 69,861,376
-DECODE_TRAFFIC_SRC_SHA256 = "b6c2d97851c1d0d335c6f5ddfc1ae24edbc378d4f979dd65c2fa805887c45f36"
+DECODE_TRAFFIC_SRC_SHA256 = "07319a2aab83d131daf76006a29d6c7d5a2d2a9e02764c2c769c529e1ed9ae82"
 DECODE_SRC = ("quantized_kv_cache_20_b200/csrc/kvq_decode.cu", "quantized_kv_cache_20_b200/csrc/kvq_decode_kernel.cuh",
               "quantized_kv_cache_20_b200/csrc/kvq_common.cuh")
 

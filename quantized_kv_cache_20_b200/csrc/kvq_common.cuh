@@ -38,10 +38,20 @@ inline int ensure_smem(Kernel kernel, int bytes) {
   return KVQ_OK;
 }
 
+// SMs of the current device, queried once per device
 inline int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  static std::atomic<int> known[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int k = known[dev].load(std::memory_order_relaxed);
+    if (k > 0) return k;
+  }
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 0 ? n : 148;
+  if (dev >= 0 && dev < 64) known[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // ---------------------------------------------------------------------------

@@ -145,11 +145,16 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+# The current device index without the lazy-init check of torch.cuda.current_device
+# (CUDA is initialised once a CUDA tensor exists); the public call otherwise.
+_get_device = getattr(torch._C, "_cuda_getDevice", None) or torch.cuda.current_device
+
+
 def _on_current_device(t):
     """The library launches on the current device (its SM count, its per-device
     state); a tensor on another device would be read from the wrong context."""
     idx = t.device.index
-    if idx is not None and idx != torch.cuda.current_device():
+    if idx is not None and idx != _get_device():
         raise ValueError(f"tensors are on cuda:{idx} but the current device is cuda:{torch.cuda.current_device()}; "
                          "call under torch.cuda.device(...)")
 
